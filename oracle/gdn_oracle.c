@@ -1,0 +1,199 @@
+/*
+ * fp64 CPU oracle for the gated delta rule -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Plain, slow, token-by-token evaluation of the recurrences whose chunked
+ * form the CUDA library computes.  No chunking, no blocking, no reordering:
+ * each token is one rank-1 state update followed by one read-out.  Only the
+ * tests, the package's smoke check and the benchmark's CPU-baseline leg may
+ * load this file's library.  It shares no code with the CUDA path.
+ *
+ * State convention: the state S_t is d_v x d_k (it maps keys to values, so
+ * o_t = S_t q_t).  Initial and final states are exchanged in the transposed
+ * layout h = S^T, shape [B, H, d_k, d_v], row-major with d_v innermost.
+ *
+ * Sources (page title, then section):
+ *   - Gated delta rule.  The pages name Gated DeltaNet and its chunkwise
+ *     form ("Quando o 'Bom o Suficiente' e Otimo: Aproximacao de Inversao de
+ *     Matriz Baseada Apenas em Multiplicacao para Gated DeltaNet Quantizado",
+ *     section "Declaracao do Problema") and read the delta rule as an online
+ *     SGD step on the least-squares loss 1/2 ||S k_t - v_t||^2 ("Resumo
+ *     Tecnico: Preconditioned DeltaNet", section 1; the Arabic summary of
+ *     the same paper, section 1), with alpha the decay axis and beta the gain
+ *     axis of the DGPS taxonomy (Arabic summary, section 2c).  The update
+ *     itself is not printed on the pages; the form used here is the standard
+ *     one: S_t = S_{t-1} alpha_t (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *     o_t = S_t q_t.
+ *   - Preconditioned two-gate variant.  Diagonal curvature accumulator of the
+ *     squared keys with the preconditioned write key ("Preconditioned
+ *     DeltaNet: Curvature-aware Sequence Modeling for Linear Recurrences",
+ *     Arabic summary, section 2b "the diagonal approximation"); separate read
+ *     and write keys ("Resumo Tecnico: Preconditioned DeltaNet", section 2,
+ *     "Estabilidade e Parametrizacao"); channel-wise erase gate b_t on the
+ *     key axis and write gate w_t on the value axis ("NVIDIA Apresenta Gated
+ *     DeltaNet-2", section "Como DeltaNet-2 Redesenhou a Arquitetura").  The
+ *     accumulator used is the moving average rho_t = c rho_{t-1} + k_t (.) k_t
+ *     with write key k_t / sqrt(rho_t + eps); c = 1 gives the pages' plain
+ *     running sum.
+ *
+ * Build: gcc -O2 -fopenmp -shared -fPIC gdn_oracle.c -o libgdn_oracle.so -lm
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static size_t tok(int b, int t, int h, int T, int H) {
+    return ((size_t)b * T + t) * H + h;
+}
+
+/*
+ * Gated delta rule, one (batch, head) sequence per outer iteration.
+ *   q, k  [B,T,H,dk]; v [B,T,H,dv]; alpha, beta [B,T,H] (alpha NULL => 1,
+ *   beta NULL => 1); h0 [B,H,dk,dv] or NULL (=> 0);
+ *   o [B,T,H,dv]; hT [B,H,dk,dv] or NULL.
+ * Per token:  p = S k_t  (prediction of the undecayed state)
+ *             S = alpha_t S - alpha_t beta_t p k_t^T + beta_t v_t k_t^T
+ *             o_t = S q_t
+ * which is S_{t-1} alpha_t (I - beta_t k_t k_t^T) + beta_t v_t k_t^T.
+ */
+void oracle_gated_delta_fwd(int B, int T, int H, int dk, int dv,
+                            const double *q, const double *k, const double *v,
+                            const double *alpha, const double *beta,
+                            const double *h0, double *o, double *hT,
+                            int nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int bh = 0; bh < B * H; ++bh) {
+        const int b = bh / H, h = bh % H;
+        double *S = (double *)calloc((size_t)dv * dk, sizeof(double));
+        double *p = (double *)malloc((size_t)dv * sizeof(double));
+        if (h0) {
+            const double *src = h0 + (size_t)bh * dk * dv;
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j)
+                    S[(size_t)j * dk + i] = src[(size_t)i * dv + j];
+        }
+        for (int t = 0; t < T; ++t) {
+            const size_t r = tok(b, t, h, T, H);
+            const double *kt = k + r * dk, *qt = q + r * dk, *vt = v + r * dv;
+            const double a = alpha ? alpha[r] : 1.0;
+            const double be = beta ? beta[r] : 1.0;
+            for (int j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < dk; ++i) acc += S[(size_t)j * dk + i] * kt[i];
+                p[j] = acc;
+            }
+            for (int j = 0; j < dv; ++j) {
+                const double cp = a * be * p[j], cv = be * vt[j];
+                double *row = S + (size_t)j * dk;
+                for (int i = 0; i < dk; ++i)
+                    row[i] = a * row[i] - cp * kt[i] + cv * kt[i];
+            }
+            double *ot = o + r * dv;
+            for (int j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < dk; ++i) acc += S[(size_t)j * dk + i] * qt[i];
+                ot[j] = acc;
+            }
+        }
+        if (hT) {
+            double *dst = hT + (size_t)bh * dk * dv;
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j)
+                    dst[(size_t)i * dv + j] = S[(size_t)j * dk + i];
+        }
+        free(S);
+        free(p);
+    }
+}
+
+/*
+ * Preconditioned two-gate delta rule.
+ *   q (read key), k (raw key) [B,T,H,dk]; v [B,T,H,dv];
+ *   alpha [B,T,H,dk] per key channel, or NULL (=> 1);
+ *   erase b_t [B,T,H,dk] or NULL (=> 1); write w_t [B,T,H,dv] or NULL (=> 1);
+ *   precond != 0 enables the curvature accumulator, otherwise the write key
+ *   is k_t itself.
+ * Per token:  rho   = rho_decay * rho + k_t (.) k_t          (rho_0 = 0)
+ *             kw    = k_t / sqrt(rho + rho_eps)               (write key)
+ *             e     = b_t (.) kw                              (erase key)
+ *             p     = S e
+ *             S     = S diag(alpha_t) - p kw^T + (w_t (.) v_t) kw^T
+ *             o_t   = S q_t
+ */
+void oracle_precond_two_gate_fwd(int B, int T, int H, int dk, int dv,
+                                 const double *q, const double *k, const double *v,
+                                 const double *alpha, const double *erase,
+                                 const double *write, int precond,
+                                 double rho_decay, double rho_eps,
+                                 const double *h0, double *o, double *hT,
+                                 int nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int bh = 0; bh < B * H; ++bh) {
+        const int b = bh / H, h = bh % H;
+        double *S = (double *)calloc((size_t)dv * dk, sizeof(double));
+        double *rho = (double *)calloc((size_t)dk, sizeof(double));
+        double *kw = (double *)malloc((size_t)dk * sizeof(double));
+        double *e = (double *)malloc((size_t)dk * sizeof(double));
+        double *p = (double *)malloc((size_t)dv * sizeof(double));
+        if (h0) {
+            const double *src = h0 + (size_t)bh * dk * dv;
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j)
+                    S[(size_t)j * dk + i] = src[(size_t)i * dv + j];
+        }
+        for (int t = 0; t < T; ++t) {
+            const size_t r = tok(b, t, h, T, H);
+            const double *kt = k + r * dk, *qt = q + r * dk, *vt = v + r * dv;
+            for (int i = 0; i < dk; ++i) {
+                if (precond) {
+                    rho[i] = rho_decay * rho[i] + kt[i] * kt[i];
+                    kw[i] = kt[i] / sqrt(rho[i] + rho_eps);
+                } else {
+                    kw[i] = kt[i];
+                }
+                e[i] = (erase ? erase[r * dk + i] : 1.0) * kw[i];
+            }
+            for (int j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < dk; ++i) acc += S[(size_t)j * dk + i] * e[i];
+                p[j] = acc;
+            }
+            for (int j = 0; j < dv; ++j) {
+                const double u = (write ? write[r * dv + j] : 1.0) * vt[j];
+                double *row = S + (size_t)j * dk;
+                for (int i = 0; i < dk; ++i) {
+                    const double a = alpha ? alpha[r * dk + i] : 1.0;
+                    row[i] = row[i] * a - p[j] * kw[i] + u * kw[i];
+                }
+            }
+            double *ot = o + r * dv;
+            for (int j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < dk; ++i) acc += S[(size_t)j * dk + i] * qt[i];
+                ot[j] = acc;
+            }
+        }
+        if (hT) {
+            double *dst = hT + (size_t)bh * dk * dv;
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j)
+                    dst[(size_t)i * dv + j] = S[(size_t)j * dk + i];
+        }
+        free(S);
+        free(rho);
+        free(kw);
+        free(e);
+        free(p);
+    }
+}

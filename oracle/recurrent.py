@@ -1,0 +1,117 @@
+"""ctypes wrapper of the fp64 token-by-token oracle (``gdn_oracle.c``).
+
+Test infrastructure only.  Inputs may be numpy arrays or CPU torch tensors of
+any float dtype; they are widened to float64 exactly as the CUDA path receives
+them (bf16 values widen losslessly).  Returns ``(o, h_T)`` as float64 numpy
+arrays with ``o`` shaped [B, T, H, d_v] and ``h_T`` shaped [B, H, d_k, d_v]
+(the transposed state h = S^T).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdn_oracle.c")
+_LIB = os.path.join(_HERE, "libgdn_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle in place with gcc (OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", _SRC,
+                               "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            dp = ctypes.POINTER(ctypes.c_double)
+            i = ctypes.c_int
+            lib.oracle_gated_delta_fwd.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, dp,
+                                                   dp, dp, i]
+            lib.oracle_gated_delta_fwd.restype = None
+            lib.oracle_precond_two_gate_fwd.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp,
+                                                        dp, i, ctypes.c_double,
+                                                        ctypes.c_double, dp, dp, dp, i]
+            lib.oracle_precond_two_gate_fwd.restype = None
+            _lib = lib
+    return _lib
+
+
+def _f64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _threads(nthreads):
+    if nthreads is not None:
+        return int(nthreads)
+    return len(os.sched_getaffinity(0))
+
+
+def gated_delta_fwd(q, k, v, alpha=None, beta=None, h0=None, nthreads=None):
+    """S_t = S_{t-1} alpha_t (I - beta_t k_t k_t^T) + beta_t v_t k_t^T, o_t = S_t q_t.
+
+    alpha, beta: [B, T, H] or None (meaning 1).  h0: [B, H, d_k, d_v] or None.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    alpha, beta, h0 = _f64(alpha), _f64(beta), _f64(h0)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == q.shape and v.shape[:3] == q.shape[:3]
+    for a in (alpha, beta):
+        assert a is None or a.shape == (B, T, H)
+    assert h0 is None or h0.shape == (B, H, dk, dv)
+    o = np.zeros((B, T, H, dv))
+    hT = np.zeros((B, H, dk, dv))
+    _load().oracle_gated_delta_fwd(B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                   _ptr(beta), _ptr(h0), _ptr(o), _ptr(hT),
+                                   _threads(nthreads))
+    return o, hT
+
+
+def precond_two_gate_fwd(q, k, v, alpha=None, erase=None, write=None, precond=True,
+                         rho_decay=0.99, rho_eps=1e-6, h0=None, nthreads=None):
+    """Preconditioned write key, per-channel decay, erase/write channel gates.
+
+    rho_t = rho_decay rho_{t-1} + k_t (.) k_t; kw = k_t / sqrt(rho_t + rho_eps);
+    S_t = S_{t-1}(diag(alpha_t) - (b_t (.) kw) kw^T) + (w_t (.) v_t) kw^T;
+    o_t = S_t q_t.  alpha, erase: [B, T, H, d_k]; write: [B, T, H, d_v];
+    each may be None (meaning all ones).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    alpha, erase, write, h0 = _f64(alpha), _f64(erase), _f64(write), _f64(h0)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert alpha is None or alpha.shape == (B, T, H, dk)
+    assert erase is None or erase.shape == (B, T, H, dk)
+    assert write is None or write.shape == (B, T, H, dv)
+    assert h0 is None or h0.shape == (B, H, dk, dv)
+    o = np.zeros((B, T, H, dv))
+    hT = np.zeros((B, H, dk, dv))
+    _load().oracle_precond_two_gate_fwd(B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v),
+                                        _ptr(alpha), _ptr(erase), _ptr(write),
+                                        int(bool(precond)), float(rho_decay), float(rho_eps),
+                                        _ptr(h0), _ptr(o), _ptr(hT), _threads(nthreads))
+    return o, hT
