@@ -1,0 +1,408 @@
+"""Benchmark of the chunkwise gated delta-rule forward on B200.
+
+Default workload: the Gated DeltaNet layer with 1.3B-class head geometry,
+B=4, H=16, T=4096, d_k=d_v=128, chunk 64, bf16 q/k/v, fp32 alpha/beta, fp32 o
+and S_T, exact blocked inversion.  One step = one gdn_chunk_fwd call over the
+whole batch (every step of the hot path: staging, gate scans, Gram, inverse,
+WY products, state passing, output).  Inputs are synthetic (seeded), resident
+in HBM when the timed region starts.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Under torchrun each rank runs its own independent batch (weak scaling, no
+collective on the data path); the time is the max over ranks.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "gdn_bf16"
+METRIC = "tokens/s (fwd, bf16, H=16, d=128, T=4096) and % of roofline on 1 B200"
+UNIT = "tokens/s"
+PROFILE = os.path.join(ROOT, "profiles", "gdn_fwd_gdn_bf16_ncu.md")
+
+
+# --------------------------------------------------------------------- utils
+
+def env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                source="fallback")
+
+
+def algorithmic_bytes(w, o_bytes):
+    """Bytes the method must move once: q, k, v, alpha, beta, o per token-head,
+    S0 (if given) and S_T per (batch, head)."""
+    in_b = 2 if w.io == "bf16" else 4
+    per_th = 2 * w.dk * in_b + w.dv * in_b + w.dv * o_bytes
+    per_th += 4 if w.decay == "scalar" else (4 * w.dk if w.decay == "channel" else 0)
+    per_th += 4 if w.beta else 0
+    per_th += (w.dk + w.dv) * in_b if w.gates else 0
+    state = w.dk * w.dv * 4 * (2 if w.s0_std > 0 else 1)
+    return w.token_heads * per_th + w.B * w.H * state
+
+
+def algorithmic_flops(w):
+    """Per chunk-head (C tokens, triangular structure exploited): K K^T strict
+    lower C(C-1)dk, Q K^T incl. diagonal C(C+1)dk, triangular inverse C^3/3,
+    U and W 2C(C-1)d, W h, Q h, K^T Delta 3*2*C*dk*dv, P Delta C(C+1)dv."""
+    C, dk, dv = w.chunk, w.dk, w.dv
+    f = C * (C - 1) * dk + C * (C + 1) * dk + C ** 3 / 3 + C * (C - 1) * (dk + dv) \
+        + 6 * C * dk * dv + C * (C + 1) * dv
+    chunks = -(-w.T // C)
+    return f * chunks * w.B * w.H
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "chunked_gated_delta_14_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, fn), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(kernel_name):
+    """dram read+write bytes per launch from the committed ncu summary, if it was
+    taken on the current kernel sources."""
+    if not os.path.exists(PROFILE):
+        return None
+    txt = open(PROFILE).read()
+    m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
+    m_k = re.search(rf"traffic_bytes_per_launch\[{re.escape(kernel_name)}\]:\s*([0-9.e+]+)", txt)
+    if not (m_sha and m_k) or m_sha.group(1) != kernel_source_sha():
+        return None
+    return float(m_k.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.marks = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def mark(self, t0, t1):
+        self.marks = (t0, t1)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = self.samples
+        if self.marks:
+            inside = [r for r in rows if self.marks[0] <= r[0] <= self.marks[1]]
+            rows = inside or rows
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for _, line in rows:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=[], samples=0)
+        return dict(sm_mhz=float(np.median(sm)), sm_max_mhz=float(max(smax)),
+                    reasons=sorted(reasons), samples=len(sm))
+
+
+# ------------------------------------------------------------ our arm (GPU)
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import chunked_gated_delta_14_b200 as gdn
+    from chunked_gated_delta_14_b200.inputs import make_inputs, workload
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workload(WORKLOAD)
+    x = make_inputs(w, seed=rank)   # each rank its own batch
+    d = {k: (None if v is None else v.to(dev)) for k, v in x.items()}
+    o = torch.empty((w.B, w.T, w.H, w.dv), device=dev, dtype=torch.float32)
+    S_T = torch.empty((w.B, w.H, w.dk, w.dv), device=dev, dtype=torch.float32)
+    stream = torch.cuda.current_stream(dev)
+    ptr = lambda t: None if t is None else t.data_ptr()
+    a = gdn.make_args(B=w.B, T=w.T, H=w.H, dk=w.dk, dv=w.dv, chunk=w.chunk, io_dtype=1,
+                      o_dtype=0, q=ptr(d["q"]), k=ptr(d["k"]), v=ptr(d["v"]),
+                      alpha=ptr(d["alpha"]), beta=ptr(d["beta"]), S0=None, o=o.data_ptr(),
+                      S_T=S_T.data_ptr(), mode=0, kernel=0)
+    kernel_id = gdn.select_kernel(a)
+    kernel_name = {1: "simt_chunk_kernel", 2: "tc_chunk_kernel"}.get(kernel_id, "?")
+    sh = stream.cuda_stream
+
+    def step():
+        gdn.call(a, sh)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local_rank)
+    if rank == 0:
+        clocks.start()
+        time.sleep(1.0)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    clocks.mark(t_wall0, t_wall1)
+    time.sleep(0.3)
+    clocks.stop()
+
+    ms_step = ms / args.steps
+    tokens_step = w.B * w.T
+    value = tokens_step * world * args.steps / (ms / 1e3)
+
+    # end to end through the public API: pinned host inputs -> device -> kernel -> host o
+    e2e = None
+    if args.e2e_steps > 0:
+        host = {k: (None if v is None else v.pin_memory()) for k, v in x.items()}
+        dev_in = {k: (None if v is None else torch.empty_like(v, device=dev)) for k, v in x.items()}
+        o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+        d2h = o_host.numel() * o_host.element_size()
+
+        def e2e_step():
+            for k, v in host.items():
+                if v is not None:
+                    dev_in[k].copy_(v, non_blocking=True)
+            gdn.chunk_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"],
+                          dev_in["beta"], chunk=w.chunk, o_dtype=torch.float32, out=o,
+                          S_T=S_T)
+            o_host.copy_(o, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        ems = f0.elapsed_time(f1)
+        if world > 1:
+            t = torch.tensor([ems], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = dict(value=tokens_step * world * args.e2e_steps / (ems / 1e3), unit=UNIT,
+                   h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h),
+                   ms_per_step=ems / args.e2e_steps)
+
+    pk = peaks()
+    bytes_launch = algorithmic_bytes(w, o_bytes=4)
+    achieved = bytes_launch / (ms_step / 1e3) / 1e9
+    flops = algorithmic_flops(w)
+    roof = dict(bound="hbm", achieved=achieved, peak=pk["hbm_gbs"], unit="GB/s",
+                frac=achieved / pk["hbm_gbs"], traffic=profile_traffic(kernel_name),
+                peak_source=pk["source"] + " (burst copy bandwidth)",
+                algorithmic_bytes_per_launch=bytes_launch,
+                tensor_tflops=flops / (ms_step / 1e3) / 1e12,
+                tensor_frac_of_bf16_peak=flops / (ms_step / 1e3) / 1e12 / pk["bf16_tflops"],
+                roofline_ms=max(bytes_launch / (pk["hbm_gbs"] * 1e9),
+                                flops / (pk["bf16_tflops"] * 1e12)) * 1e3)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, x, budget_s=args.cpu_budget)
+
+    if rank == 0:
+        line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps,
+                    warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True,
+                    scaling="weak", vs_baseline=None, dtype="bf16",
+                    compute="bf16 q/k/v in HBM; fp16 tensor-core operands, fp32 accumulate and state",
+                    data="synthetic (seeded; Gated DeltaNet layer shapes)",
+                    config=dict(workload=f"{WORKLOAD}: B={w.B} H={w.H} T={w.T} dk={w.dk} "
+                                f"dv={w.dv} chunk={w.chunk} exact inverse, o fp32",
+                                global_batch=w.B * world, seq_len=w.T,
+                                parallelism=f"independent batch per GPU x{world}",
+                                l2="no flush: inputs+outputs 341 MB per step > 126 MB L2",
+                                kernel=kernel_name),
+                    clocks=clocks.summary() if rank == 0 else None,
+                    e2e=e2e, gpu_launches=args.steps, roofline=roof, cpu_baseline=cpu)
+        print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(w, x, budget_s=12.0):
+    """The fp64 oracle as it stands, timed on this host's cores, on whole
+    (batch, head) sequences of the same workload until ~budget_s seconds."""
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    H = w.H
+    done_th = 0
+    t0 = time.time()
+    b = 0
+    while True:
+        sl = lambda t: None if t is None else t[b:b + 1]
+        oracle.gated_delta_fwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["alpha"]),
+                               sl(x["beta"]), sl(x["S0"]), nthreads=cores)
+        done_th += w.T * H
+        b = (b + 1) % w.B
+        if time.time() - t0 >= budget_s:
+            break
+    el = time.time() - t0
+    return dict(value=done_th / H / el, unit=UNIT, cores=cores, kind="oracle",
+                sample=f"{done_th // (w.T * H)} x (batch row of {H} heads x {w.T} tokens) "
+                       f"of {WORKLOAD}, fp64 C oracle, {el:.1f} s")
+
+
+# ------------------------------------------------- reference arm (the oracle)
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    from chunked_gated_delta_14_b200.inputs import make_inputs, workload
+    w = workload(WORKLOAD)
+    x = make_inputs(w)
+    cores = len(os.sched_getaffinity(0))
+    # per-step sample: a prefix of one (batch, head) row group sized so that
+    # warmup + steps fit in about args.ref_budget seconds
+    total_steps = max(1, args.steps + args.warmup)
+    per_step_s = args.ref_budget / total_steps
+    probe_T = 256
+    t0 = time.time()
+    sl = lambda t, b, n: None if t is None else t[b:b + 1, :n].contiguous()
+    oracle.gated_delta_fwd(sl(x["q"], 0, probe_T), sl(x["k"], 0, probe_T), sl(x["v"], 0, probe_T),
+                           sl(x["alpha"], 0, probe_T), sl(x["beta"], 0, probe_T), nthreads=cores)
+    rate = probe_T / max(time.time() - t0, 1e-6)           # tokens (all heads) per second
+    Ts = int(min(w.T, max(16, rate * per_step_s)))
+    def step(i):
+        b = i % w.B
+        oracle.gated_delta_fwd(sl(x["q"], b, Ts), sl(x["k"], b, Ts), sl(x["v"], b, Ts),
+                               sl(x["alpha"], b, Ts), sl(x["beta"], b, Ts), nthreads=cores)
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    el = time.perf_counter() - t0
+    value = Ts * args.steps / el
+    sample = f"tokens [0,{Ts}) of one batch row (all {w.H} heads) of {WORKLOAD} per step"
+    line = dict(impl="reference", metric=METRIC, value=value, unit=UNIT, n_gpus=world,
+                steps=args.steps, warmup=args.warmup, ms_per_step=el / args.steps * 1e3,
+                higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
+                data="synthetic (seeded; Gated DeltaNet layer shapes)",
+                config=dict(workload=f"{WORKLOAD}: B={w.B} H={w.H} T={w.T} dk={w.dk} "
+                            f"dv={w.dv} chunk={w.chunk}", global_batch=w.B, seq_len=w.T,
+                            parallelism="CPU oracle, rank 0 only"),
+                cpu_baseline=dict(value=value, unit=UNIT, cores=cores, kind="oracle",
+                                  sample=sample),
+                e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--ref-budget", type=float, default=60.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = env_int("WORLD_SIZE", 1)
+    rank = env_int("RANK", 0)
+    local_rank = env_int("LOCAL_RANK", 0)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_gpu(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,166 @@
+// Host side of libgdn.so: argument validation, kernel selection, launch.
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+
+#include "gdn_internal.cuh"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+gdn_status fail(gdn_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+    if (getenv("GDN_LOG")) fprintf(stderr, "[gdn] %s: %s\n", gdn_status_string(s), g_msg);
+    return s;
+}
+
+bool pow2_in(int x, int lo, int hi) { return x >= lo && x <= hi && (x & (x - 1)) == 0; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validate and resolve; on success fills *out.  Never touches the GPU.
+gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
+    if (!a) return fail(GDN_ERR_INVALID_ARG, "args is NULL");
+    if (a->B < 1 || a->H < 1 || a->T < 1)
+        return fail(GDN_ERR_INVALID_ARG, "B, T, H must be >= 1 (got %d, %d, %d)", a->B, a->T, a->H);
+    if ((long long)a->B * a->T * a->H > (1ll << 40))
+        return fail(GDN_ERR_INVALID_ARG, "B*T*H too large");
+    if (!pow2_in(a->dk, 16, 128) || !pow2_in(a->dv, 16, 128))
+        return fail(GDN_ERR_INVALID_ARG, "dk, dv must be 16, 32, 64 or 128 (got %d, %d)", a->dk, a->dv);
+    if (!pow2_in(a->chunk, 16, 128))
+        return fail(GDN_ERR_INVALID_ARG, "chunk must be 16, 32, 64 or 128 (got %d)", a->chunk);
+    if (a->io_dtype != GDN_F32 && a->io_dtype != GDN_BF16)
+        return fail(GDN_ERR_INVALID_ARG, "io_dtype %d unknown", a->io_dtype);
+    if (a->o_dtype != GDN_F32 && a->o_dtype != GDN_BF16)
+        return fail(GDN_ERR_INVALID_ARG, "o_dtype %d unknown", a->o_dtype);
+    if (!a->q || !a->k || !a->v || !a->o)
+        return fail(GDN_ERR_INVALID_ARG, "q, k, v and o are required");
+    if (a->mode != GDN_INV_EXACT && a->mode != GDN_INV_NEUMANN)
+        return fail(GDN_ERR_INVALID_ARG, "mode %d unknown", a->mode);
+    if (a->mode == GDN_INV_NEUMANN && (a->neumann_N < 0 || a->neumann_N > a->chunk - 1))
+        return fail(GDN_ERR_INVALID_ARG, "neumann_N must be in [0, chunk-1] (got %d)", a->neumann_N);
+    if (a->alpha_per_channel && !a->alpha)
+        return fail(GDN_ERR_INVALID_ARG, "alpha_per_channel needs alpha");
+    if (a->alpha_per_channel != 0 && a->alpha_per_channel != 1)
+        return fail(GDN_ERR_INVALID_ARG, "alpha_per_channel must be 0 or 1");
+    if (a->precond != 0 && a->precond != 1)
+        return fail(GDN_ERR_INVALID_ARG, "precond must be 0 or 1");
+    const int general = a->alpha_per_channel || a->precond || a->erase || a->write;
+    if (general && a->beta)
+        return fail(GDN_ERR_INVALID_ARG,
+                    "beta must be NULL with the two-gate rule (erase/write/precond/per-channel alpha)");
+    if (a->precond && !(a->rho_eps > 0.f && a->rho_decay >= 0.f))
+        return fail(GDN_ERR_INVALID_ARG, "precond needs rho_eps > 0 and rho_decay >= 0");
+    const void *ins[] = {a->q, a->k, a->v, a->alpha, a->beta, a->erase, a->write, a->S0};
+    for (const void *x : ins)
+        if (x && x == a->o) return fail(GDN_ERR_INVALID_ARG, "o aliases an input");
+    if (a->S_T && (const void *)a->S_T == a->o) return fail(GDN_ERR_INVALID_ARG, "o aliases S_T");
+    const void *al[] = {a->q, a->k, a->v, a->o, a->erase, a->write, a->S0, a->S_T, a->alpha, a->beta};
+    for (const void *x : al)
+        if (x && !aligned16(x)) return fail(GDN_ERR_ALIGNMENT, "pointers must be 16-byte aligned");
+    if (a->kernel < GDN_KERNEL_AUTO || a->kernel > GDN_KERNEL_TC)
+        return fail(GDN_ERR_INVALID_ARG, "kernel %d unknown", a->kernel);
+    if (a->dv_split < 0 || (a->dv_split > 0 && (a->dv % a->dv_split != 0 || a->dv / a->dv_split < 16)))
+        return fail(GDN_ERR_INVALID_ARG, "dv_split must divide dv into slices of >= 16 columns");
+
+    gdn::FwdParams p{};
+    p.B = a->B; p.T = a->T; p.H = a->H; p.dk = a->dk; p.dv = a->dv; p.C = a->chunk;
+    p.io_bf16 = a->io_dtype == GDN_BF16;
+    p.o_bf16 = a->o_dtype == GDN_BF16;
+    p.q = a->q; p.k = a->k; p.v = a->v;
+    p.alpha = a->alpha; p.alpha_pc = a->alpha_per_channel; p.beta = a->beta;
+    p.precond = a->precond; p.rho_decay = a->rho_decay; p.rho_eps = a->rho_eps;
+    p.erase = a->erase; p.write = a->write; p.S0 = a->S0; p.o = a->o; p.S_T = a->S_T;
+    p.mode = a->mode; p.N = a->mode == GDN_INV_NEUMANN ? a->neumann_N : 0;
+    p.general = general;
+
+    const char *why = "";
+    int kern = a->kernel;
+    if (kern == GDN_KERNEL_AUTO) kern = gdn::tc_supports(p, &why) ? GDN_KERNEL_TC : GDN_KERNEL_SIMT;
+    if (kern == GDN_KERNEL_TC) {
+        if (!gdn::tc_supports(p, &why))
+            return fail(GDN_ERR_UNSUPPORTED, "tensor-core kernel: %s", why);
+        p.slices = a->dv_split ? a->dv_split : gdn::tc_default_slices(p);
+        if (p.dv % p.slices) return fail(GDN_ERR_UNSUPPORTED, "dv_split does not divide dv");
+        p.dvs = p.dv / p.slices;
+        if (!gdn::tc_supports(p, &why))
+            return fail(GDN_ERR_UNSUPPORTED, "tensor-core kernel: %s", why);
+    } else {
+        // SIMT: widest value slice that fits shared memory, at least
+        // ~one block per SM where the problem allows it.
+        int slices = a->dv_split;
+        if (!slices) {
+            slices = 1;
+            while (p.dv / (slices * 2) >= 16 && (long long)p.B * p.H * slices < 148) slices *= 2;
+        }
+        for (;;) {
+            p.slices = slices;
+            p.dvs = p.dv / slices;
+            if (gdn::simt_smem_bytes(p) <= 227 * 1024) break;
+            if (a->dv_split || p.dvs <= 16)
+                return fail(GDN_ERR_UNSUPPORTED,
+                            "SIMT kernel: chunk %d, dk %d, value slice %d needs %zu B of shared memory",
+                            p.C, p.dk, p.dvs, gdn::simt_smem_bytes(p));
+            slices *= 2;
+        }
+    }
+    *out = p;
+    *kernel = kern;
+    return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *gdn_status_string(gdn_status s) {
+    switch (s) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+        case GDN_ERR_ALIGNMENT: return "GDN_ERR_ALIGNMENT";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+        case GDN_ERR_DEVICE_CHECK: return "GDN_ERR_DEVICE_CHECK";
+        case GDN_ERR_FAULT_INJECTED: return "GDN_ERR_FAULT_INJECTED";
+    }
+    return "GDN_UNKNOWN_STATUS";
+}
+
+const char *gdn_last_error(void) { return g_msg; }
+
+int32_t gdn_abi_version(void) { return GDN_ABI_VERSION; }
+
+int32_t gdn_select_kernel(const gdn_fwd_args *args) {
+    gdn::FwdParams p;
+    int kern = 0;
+    gdn_status s = resolve(args, &p, &kern);
+    if (s != GDN_OK) return -(int32_t)s;
+    g_msg[0] = 0;
+    return kern;
+}
+
+gdn_status gdn_chunk_fwd(const gdn_fwd_args *args, void *stream) {
+    const char *inj = getenv("GDN_FAULT_INJECT");
+    if (inj && inj[0] == '1') return fail(GDN_ERR_FAULT_INJECTED, "GDN_FAULT_INJECT=1");
+    gdn::FwdParams p;
+    int kern = 0;
+    gdn_status s = resolve(args, &p, &kern);
+    if (s != GDN_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    const char *why = "";
+    if (kern == GDN_KERNEL_TC) e = gdn::launch_tc(p, st, &why);
+    else e = gdn::launch_simt(p, st);
+    if (e != cudaSuccess)
+        return fail(GDN_ERR_CUDA, "%s launch: %s %s", kern == GDN_KERNEL_TC ? "tc" : "simt",
+                    cudaGetErrorString(e), why);
+    g_msg[0] = 0;
+    return GDN_OK;
+}
+
+}  // extern "C"

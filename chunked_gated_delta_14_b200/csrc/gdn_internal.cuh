@@ -1,0 +1,40 @@
+// Internal declarations shared by the launchers of libgdn.so.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdn.h"
+
+namespace gdn {
+
+// Everything a kernel needs, resolved from gdn_fwd_args by the host layer.
+struct FwdParams {
+    int B, T, H, dk, dv, C;
+    int dvs;            // value columns per block (dv / slices)
+    int slices;
+    int io_bf16, o_bf16;
+    const void *q, *k, *v;
+    const float *alpha;
+    int alpha_pc;
+    const float *beta;
+    int precond;
+    float rho_decay, rho_eps;
+    const void *erase, *write;
+    const float *S0;
+    void *o;
+    float *S_T;
+    int mode, N;
+    int general;        // two-gate rule (per-channel decay / gates / preconditioner)
+};
+
+// SIMT fp32 chunk kernel: shared-memory bytes for p, or 0 if p does not fit.
+size_t simt_smem_bytes(const FwdParams &p);
+cudaError_t launch_simt(const FwdParams &p, cudaStream_t stream);
+
+// Tensor-core kernel (tcgen05 / TMEM / TMA).
+bool tc_supports(const FwdParams &p, const char **why);
+int tc_default_slices(const FwdParams &p);
+cudaError_t launch_tc(const FwdParams &p, cudaStream_t stream, const char **why);
+
+}  // namespace gdn

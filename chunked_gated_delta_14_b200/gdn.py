@@ -1,0 +1,203 @@
+"""Thin ctypes binding of libgdn.so (the C ABI declared in include/gdn.h).
+
+Argument marshalling only: every step of the forward pass runs in the CUDA
+kernels of libgdn.so.  PyTorch provides device memory and the current stream.
+There is no fallback: if the library is missing or the device is not a CUDA
+device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn.so")
+
+GDN_OK = 0
+GDN_ERR_INVALID_ARG = 1
+GDN_ERR_UNSUPPORTED = 2
+GDN_ERR_ALIGNMENT = 3
+GDN_ERR_CUDA = 4
+GDN_ERR_DEVICE_CHECK = 5
+GDN_ERR_FAULT_INJECTED = 6
+
+GDN_F32, GDN_BF16 = 0, 1
+GDN_INV_EXACT, GDN_INV_NEUMANN = 0, 1
+KERNELS = {"auto": 0, "simt": 1, "tc": 2}
+KERNEL_NAMES = {v: k for k, v in KERNELS.items()}
+MODES = {"exact": GDN_INV_EXACT, "neumann": GDN_INV_NEUMANN}
+
+EXPORTS = ("gdn_chunk_fwd", "gdn_select_kernel", "gdn_status_string", "gdn_last_error",
+           "gdn_abi_version")
+
+
+class GDNError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{status_string(status)}: {message}")
+        self.status = status
+
+
+class FwdArgs(ctypes.Structure):
+    """Mirror of ``gdn_fwd_args``."""
+    _fields_ = [
+        ("B", ctypes.c_int32), ("T", ctypes.c_int32), ("H", ctypes.c_int32),
+        ("dk", ctypes.c_int32), ("dv", ctypes.c_int32), ("chunk", ctypes.c_int32),
+        ("io_dtype", ctypes.c_int32), ("o_dtype", ctypes.c_int32),
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("alpha", ctypes.c_void_p), ("alpha_per_channel", ctypes.c_int32),
+        ("beta", ctypes.c_void_p), ("precond", ctypes.c_int32),
+        ("rho_decay", ctypes.c_float), ("rho_eps", ctypes.c_float),
+        ("erase", ctypes.c_void_p), ("write", ctypes.c_void_p),
+        ("S0", ctypes.c_void_p), ("o", ctypes.c_void_p), ("S_T", ctypes.c_void_p),
+        ("mode", ctypes.c_int32), ("neumann_N", ctypes.c_int32),
+        ("kernel", ctypes.c_int32), ("dv_split", ctypes.c_int32),
+    ]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgdn.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m chunked_gated_delta_14_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            L.gdn_chunk_fwd.argtypes = [ctypes.POINTER(FwdArgs), ctypes.c_void_p]
+            L.gdn_chunk_fwd.restype = ctypes.c_int
+            L.gdn_select_kernel.argtypes = [ctypes.POINTER(FwdArgs)]
+            L.gdn_select_kernel.restype = ctypes.c_int32
+            L.gdn_status_string.argtypes = [ctypes.c_int]
+            L.gdn_status_string.restype = ctypes.c_char_p
+            L.gdn_last_error.argtypes = []
+            L.gdn_last_error.restype = ctypes.c_char_p
+            L.gdn_abi_version.argtypes = []
+            L.gdn_abi_version.restype = ctypes.c_int32
+            _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    try:
+        return lib().gdn_status_string(int(s)).decode()
+    except Exception:  # pragma: no cover - message formatting only
+        return f"status {s}"
+
+
+def last_error() -> str:
+    return lib().gdn_last_error().decode()
+
+
+def abi_version() -> int:
+    return int(lib().gdn_abi_version())
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return GDN_BF16
+    if dt == torch.float32:
+        return GDN_F32
+    raise TypeError(f"unsupported dtype {dt}; use torch.bfloat16 or torch.float32")
+
+
+def _check(t: Optional[torch.Tensor], name: str, shape, dtype=None):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (got {t.device})")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def make_args(**kw) -> FwdArgs:
+    a = FwdArgs()
+    a.rho_decay = 0.99
+    a.rho_eps = 1e-6
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def select_kernel(args: FwdArgs) -> int:
+    """Kernel gdn_chunk_fwd would launch (1 simt, 2 tc) or -status. Host only."""
+    return int(lib().gdn_select_kernel(ctypes.byref(args)))
+
+
+def call(args: FwdArgs, stream: Optional[int] = None) -> None:
+    """Raw gdn_chunk_fwd call; raises GDNError on a non-OK status."""
+    s = lib().gdn_chunk_fwd(ctypes.byref(args), ctypes.c_void_p(stream or 0))
+    if s != GDN_OK:
+        raise GDNError(s, last_error())
+
+
+def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+              alpha: Optional[torch.Tensor] = None, beta: Optional[torch.Tensor] = None, *,
+              erase: Optional[torch.Tensor] = None, write: Optional[torch.Tensor] = None,
+              precond: bool = False, rho_decay: float = 0.99, rho_eps: float = 1e-6,
+              S0: Optional[torch.Tensor] = None, chunk: int = 64, mode: str = "exact",
+              N: int = 3, o_dtype: Optional[torch.dtype] = None, kernel: str = "auto",
+              dv_split: int = 0, out: Optional[torch.Tensor] = None,
+              final_state: bool = True, S_T: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None
+              ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunkwise gated delta-rule forward; returns ``(o, S_T)``.
+
+    q, k: [B, T, H, dk]; v: [B, T, H, dv] (bf16 or fp32, same dtype).
+    alpha: [B, T, H] or [B, T, H, dk] fp32 decay (None = 1); beta: [B, T, H]
+    fp32 (None = 1).  erase [B, T, H, dk], write [B, T, H, dv] gates and
+    ``precond`` select the preconditioned two-gate rule.  S0 / S_T:
+    [B, H, dk, dv] fp32 (h = S^T).  ``o_dtype`` defaults to q's dtype.
+    """
+    if q.dim() != 4:
+        raise ValueError("q must be [B, T, H, dk]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    io = q.dtype
+    _check(q, "q", (B, T, H, dk), io)
+    _check(k, "k", (B, T, H, dk), io)
+    _check(v, "v", (B, T, H, dv), io)
+    per_channel = alpha is not None and alpha.dim() == 4
+    _check(alpha, "alpha", (B, T, H, dk) if per_channel else (B, T, H), torch.float32)
+    _check(beta, "beta", (B, T, H), torch.float32)
+    _check(erase, "erase", (B, T, H, dk), io)
+    _check(write, "write", (B, T, H, dv), io)
+    _check(S0, "S0", (B, H, dk, dv), torch.float32)
+    od = o_dtype or io
+    if out is None:
+        out = torch.empty((B, T, H, dv), device=q.device, dtype=od)
+    _check(out, "out", (B, T, H, dv), od)
+    if final_state and S_T is None:
+        S_T = torch.empty((B, H, dk, dv), device=q.device, dtype=torch.float32)
+    if not final_state:
+        S_T = None
+    _check(S_T, "S_T", (B, H, dk, dv), torch.float32)
+    args = make_args(
+        B=B, T=T, H=H, dk=dk, dv=dv, chunk=int(chunk), io_dtype=_dtype_code(io),
+        o_dtype=_dtype_code(od), q=_ptr(q), k=_ptr(k), v=_ptr(v), alpha=_ptr(alpha),
+        alpha_per_channel=int(per_channel), beta=_ptr(beta), precond=int(bool(precond)),
+        rho_decay=float(rho_decay), rho_eps=float(rho_eps), erase=_ptr(erase),
+        write=_ptr(write), S0=_ptr(S0), o=_ptr(out), S_T=_ptr(S_T), mode=MODES[mode],
+        neumann_N=int(N), kernel=KERNELS[kernel], dv_split=int(dv_split))
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        call(args, stream.cuda_stream)
+    return out, S_T

@@ -1,0 +1,144 @@
+/*
+ * gdn.h -- C ABI of libgdn.so, the B200 (sm_100a) chunkwise gated delta-rule
+ * forward pass.
+ *
+ * What it computes.  For every (batch b, head h) sequence, with the state S_t
+ * a d_v x d_k matrix (keys to values):
+ *
+ *   gated delta rule (default):
+ *     S_t = S_{t-1} alpha_t (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *     o_t = S_t q_t.
+ *   The pages read the delta rule as an online SGD step on the least-squares
+ *   loss 1/2||S k_t - v_t||^2 ("Resumo Tecnico: Preconditioned DeltaNet",
+ *   section 1), alpha is the decay axis and beta the gain axis ("Preconditioned
+ *   DeltaNet: Curvature-aware Sequence Modeling for Linear Recurrences",
+ *   Arabic summary, section 2c).
+ *
+ *   preconditioned two-gate rule (precond / erase / write / per-channel alpha):
+ *     rho_t = rho_decay rho_{t-1} + k_t (.) k_t,  kw_t = k_t / sqrt(rho_t + rho_eps),
+ *     S_t = S_{t-1}(diag(alpha_t) - (b_t (.) kw_t) kw_t^T) + (w_t (.) v_t) kw_t^T,
+ *     o_t = S_t q_t  (q is the read key, kw the write key).
+ *   Diagonal curvature preconditioner: same Arabic summary, section 2b; read
+ *   and write keys: "Resumo Tecnico: Preconditioned DeltaNet", section 2;
+ *   channel-wise erase gate b_t (key axis) and write gate w_t (value axis):
+ *   "NVIDIA Apresenta Gated DeltaNet-2", section "Como DeltaNet-2 Redesenhou
+ *   a Arquitetura".
+ *
+ * How.  Chunkwise-parallel (WY/UT) form over chunks of C tokens: per chunk the
+ * strictly lower triangular A is built from the key Gram matrix, and
+ * T = (I - A)^-1 ("Quando o 'Bom o Suficiente' e Otimo: Aproximacao de
+ * Inversao de Matriz Baseada Apenas em Multiplicacao para Gated DeltaNet
+ * Quantizado", section "Declaracao do Problema") is formed either exactly
+ * (GDN_INV_EXACT) or as the truncated Neumann series sum_{n<=N} A^n with the
+ * structural diagonal mask M_ij = [i - j <= N] (GDN_INV_NEUMANN; same page,
+ * section "Metodologia", items 1 and 2).  The fp32 state is carried from
+ * chunk to chunk inside one kernel.
+ *
+ * Layouts (all row-major, innermost last, no padding):
+ *   q, k     [B, T, H, dk]   io_dtype          (q is the read key)
+ *   v        [B, T, H, dv]   io_dtype
+ *   alpha    [B, T, H] fp32, or [B, T, H, dk] fp32 when alpha_per_channel
+ *   beta     [B, T, H] fp32
+ *   erase    [B, T, H, dk]   io_dtype          (gate b_t)
+ *   write    [B, T, H, dv]   io_dtype          (gate w_t)
+ *   S0, S_T  [B, H, dk, dv]  fp32              (h = S^T: row = key channel)
+ *   o        [B, T, H, dv]   o_dtype
+ *
+ * Ownership.  Every pointer is a DEVICE pointer owned by the caller, who
+ * allocates inputs and outputs.  The library allocates no device memory and
+ * keeps no state between calls.
+ *
+ * Execution and errors.  gdn_chunk_fwd validates its arguments on the host
+ * and returns an error before launching anything (nothing is written) when
+ * they are invalid.  Otherwise it enqueues the work on `stream` (a
+ * cudaStream_t passed as void*, NULL = legacy default stream) and returns
+ * without synchronising; launch failures map to GDN_ERR_CUDA.  o must not
+ * alias any input; S_T may alias S0 (each block reads its slice of S0 before
+ * it writes the same slice of S_T).  gdn_last_error() returns a message for
+ * the calling thread's most recent failure.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDN_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,    /* NULL pointer, bad size, bad enum value */
+    GDN_ERR_UNSUPPORTED = 2,    /* valid request this build cannot run */
+    GDN_ERR_ALIGNMENT = 3,      /* a pointer or row stride is not 16-byte aligned */
+    GDN_ERR_CUDA = 4,           /* the CUDA runtime reported an error */
+    GDN_ERR_DEVICE_CHECK = 5,   /* a kernel's own bounds check recorded a failure */
+    GDN_ERR_FAULT_INJECTED = 6  /* GDN_FAULT_INJECT=1 in the environment (tests) */
+} gdn_status;
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+typedef enum {
+    GDN_INV_EXACT = 0,          /* T = (I - A)^-1 exactly (blocked inversion) */
+    GDN_INV_NEUMANN = 1         /* T = M^(N) (.) sum_{n=0}^{N} A^n */
+} gdn_inv_mode;
+
+typedef enum {
+    GDN_KERNEL_AUTO = 0,        /* tensor-core kernel when it supports the call, else SIMT */
+    GDN_KERNEL_SIMT = 1,        /* fp32 CUDA-core chunk kernel (all variants) */
+    GDN_KERNEL_TC = 2           /* tcgen05/TMEM/TMA kernel (bf16 io, scalar decay, C = 64) */
+} gdn_kernel;
+
+typedef struct {
+    int32_t B, T, H;            /* batch, tokens (>= 1), heads */
+    int32_t dk, dv;             /* key / value head dims: 16, 32, 64 or 128 */
+    int32_t chunk;              /* C: 16, 32, 64 or 128 */
+    int32_t io_dtype;           /* gdn_dtype of q, k, v, erase, write */
+    int32_t o_dtype;            /* gdn_dtype of o */
+    const void *q, *k, *v;
+    const float *alpha;         /* decay in (0, 1]; NULL => 1 */
+    int32_t alpha_per_channel;  /* 0: [B,T,H]; 1: [B,T,H,dk] */
+    const float *beta;          /* write strength; NULL => 1 */
+    int32_t precond;            /* 1: diagonal curvature preconditioned write key */
+    float rho_decay, rho_eps;   /* preconditioner EMA constant and epsilon */
+    const void *erase;          /* erase gate b_t or NULL (=> 1); needs beta == NULL */
+    const void *write;          /* write gate w_t or NULL (=> 1); needs beta == NULL */
+    const float *S0;            /* initial state or NULL (=> 0) */
+    void *o;                    /* output, caller-allocated */
+    float *S_T;                 /* final state, caller-allocated, or NULL */
+    int32_t mode;               /* gdn_inv_mode */
+    int32_t neumann_N;          /* N for GDN_INV_NEUMANN: 0 <= N <= chunk - 1 */
+    int32_t kernel;             /* gdn_kernel selection */
+    int32_t dv_split;           /* value-axis slices per head (0 = choose) */
+} gdn_fwd_args;
+
+/* Chunkwise forward: o and S_T from q, k, v, gates and S0 (see above). */
+GDN_API gdn_status gdn_chunk_fwd(const gdn_fwd_args *args, void *stream);
+
+/* Which kernel gdn_chunk_fwd would launch for these arguments (gdn_kernel
+ * value, never AUTO), or a negative gdn_status if they are invalid.  Host
+ * only; launches nothing. */
+GDN_API int32_t gdn_select_kernel(const gdn_fwd_args *args);
+
+/* Static string for a status code. */
+GDN_API const char *gdn_status_string(gdn_status s);
+
+/* Message for the calling thread's most recent non-OK return ("" if none). */
+GDN_API const char *gdn_last_error(void);
+
+/* GDN_ABI_VERSION of the loaded library. */
+GDN_API int32_t gdn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

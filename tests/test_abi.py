@@ -1,0 +1,111 @@
+"""Host-only checks of libgdn.so: it loads, exports every declared symbol and
+rejects bad arguments before launching anything.  No GPU needed."""
+import os
+import re
+import subprocess
+
+import pytest
+
+import chunked_gated_delta_14_b200 as gdn
+from chunked_gated_delta_14_b200 import build as gbuild
+from chunked_gated_delta_14_b200.gdn import (GDN_ERR_ALIGNMENT, GDN_ERR_FAULT_INJECTED,
+                                             GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED)
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"GDN_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+    return names
+
+
+def test_library_builds_and_loads():
+    gbuild.build()
+    assert gdn.abi_version() == 1
+
+
+def test_exports_every_declared_symbol():
+    names = declared_functions()
+    assert "gdn_chunk_fwd" in names and len(names) >= 5
+    out = subprocess.check_output(["nm", "-D", "--defined-only", gbuild.LIB]).decode()
+    exported = set(line.split()[-1] for line in out.splitlines() if " T " in line)
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    lib = gdn.lib()
+    for n in names:
+        getattr(lib, n)
+
+
+def _args(**kw):
+    base = dict(B=2, T=100, H=3, dk=128, dv=128, chunk=64, io_dtype=1, o_dtype=0,
+                q=0x10000, k=0x20000, v=0x30000, o=0x40000)
+    base.update(kw)
+    return gdn.make_args(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=0), GDN_ERR_INVALID_ARG),
+    (dict(T=0), GDN_ERR_INVALID_ARG),
+    (dict(dk=48), GDN_ERR_INVALID_ARG),
+    (dict(dv=256), GDN_ERR_INVALID_ARG),
+    (dict(chunk=8), GDN_ERR_INVALID_ARG),
+    (dict(chunk=96), GDN_ERR_INVALID_ARG),
+    (dict(io_dtype=7), GDN_ERR_INVALID_ARG),
+    (dict(q=None), GDN_ERR_INVALID_ARG),
+    (dict(o=None), GDN_ERR_INVALID_ARG),
+    (dict(o=0x10000), GDN_ERR_INVALID_ARG),             # o aliases q
+    (dict(mode=1, neumann_N=64), GDN_ERR_INVALID_ARG),  # N > C - 1
+    (dict(mode=5), GDN_ERR_INVALID_ARG),
+    (dict(alpha_per_channel=1), GDN_ERR_INVALID_ARG),   # no alpha given
+    (dict(erase=0x50000, beta=0x60000), GDN_ERR_INVALID_ARG),
+    (dict(precond=1, rho_eps=0.0), GDN_ERR_INVALID_ARG),
+    (dict(q=0x10008), GDN_ERR_ALIGNMENT),
+    (dict(kernel=9), GDN_ERR_INVALID_ARG),
+    (dict(dv_split=3), GDN_ERR_INVALID_ARG),
+    (dict(kernel=2, io_dtype=0), GDN_ERR_UNSUPPORTED),  # tensor cores need bf16 io
+    (dict(alpha=0x70000, alpha_per_channel=1, chunk=128, kernel=1, dv_split=8),
+     GDN_ERR_UNSUPPORTED),                              # two-gate SIMT at C=128 too big
+])
+def test_invalid_arguments_rejected_on_host(kw, status):
+    a = _args(**kw)
+    assert gdn.select_kernel(a) == -status, gdn.last_error()
+    assert gdn.last_error()
+    with pytest.raises(gdn.GDNError) as ei:
+        gdn.call(a)  # returns before any CUDA call
+    assert ei.value.status == status
+
+
+def test_null_args_pointer():
+    import ctypes
+    assert gdn.lib().gdn_chunk_fwd(None, None) == GDN_ERR_INVALID_ARG
+
+
+def test_valid_arguments_select_a_kernel():
+    assert gdn.select_kernel(_args(kernel=1)) == 1
+    assert gdn.select_kernel(_args(io_dtype=0, dk=64, dv=64)) == 1   # fp32 io -> SIMT
+    assert gdn.select_kernel(_args(alpha=0x70000, precond=1, erase=0x50000,
+                                   write=0x58000, alpha_per_channel=1)) in (1, 2)
+    assert gdn.select_kernel(_args(S0=0x80000, S_T=0x80000)) in (1, 2)  # S_T may alias S0
+
+
+def test_fault_injection_env(monkeypatch):
+    monkeypatch.setenv("GDN_FAULT_INJECT", "1")
+    with pytest.raises(gdn.GDNError) as ei:
+        gdn.call(_args())
+    assert ei.value.status == GDN_ERR_FAULT_INJECTED
+
+
+def test_status_strings():
+    for s in range(7):
+        assert gdn.status_string(s).startswith("GDN_")
+
+
+def test_python_wrapper_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 4, 1, 16, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        gdn.chunk_fwd(q, q, q)

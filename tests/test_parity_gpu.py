@@ -1,0 +1,194 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Every workload is drawn by the shared seeded generator, so both sides see the
+same bits.  The full-size cases run in the launch configuration the benchmark
+times (kernel selection "auto", default value-axis split).
+"""
+import numpy as np
+import pytest
+import torch
+
+from chunked_gated_delta_14_b200.inputs import make_inputs, workload
+from oracle import chunk_forms as cf
+
+from gpu_util import (TOL_BF16_REL_RMS, TOL_F32_ABS, bf16_allowance_ok, report, run_gpu,
+                      run_oracle, stats)
+
+pytestmark = pytest.mark.gpu
+
+needs_cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+
+
+def _check_bf16(name, w, x, o_ref, s_ref, **kw):
+    o, s = run_gpu(x, w, o_dtype=torch.float32, **kw)
+    so, ss = stats(o, o_ref), stats(s, s_ref)
+    report(name, o=so, S_T=ss, **{k: str(v) for k, v in kw.items()})
+    assert so["max_rel_rms"] <= TOL_BF16_REL_RMS, so
+    assert ss["max_rel_rms"] <= TOL_BF16_REL_RMS, ss
+    return o, s
+
+
+# ------------------------------------------------------------ configuration 1
+
+@needs_cuda
+def test_plain_delta_rule_fp32():
+    w = workload("plain_fp32")
+    x = make_inputs(w)
+    o_ref, s_ref = run_oracle(x, w)
+    o, s = run_gpu(x, w)
+    report("plain_fp32", o=stats(o, o_ref), S_T=stats(s, s_ref))
+    assert np.abs(o - o_ref).max() <= TOL_F32_ABS
+    assert np.abs(s - s_ref).max() <= TOL_F32_ABS
+
+
+# ------------------------------------------------------------ configuration 2
+
+@needs_cuda
+@pytest.mark.parametrize("kernel", ["auto", "simt"])
+def test_gdn_bf16_small_ragged(kernel):
+    w = workload("gdn_bf16", B=2, H=3, T=1000)
+    x = make_inputs(w, seed=3)
+    o_ref, s_ref = run_oracle(x, w)
+    _check_bf16(f"gdn_small_{kernel}", w, x, o_ref, s_ref, kernel=kernel)
+
+
+@needs_cuda
+def test_gdn_bf16_full_size():
+    w = workload("gdn_bf16")
+    x = make_inputs(w)
+    o_ref, s_ref = run_oracle(x, w)
+    _check_bf16("gdn_full_auto", w, x, o_ref, s_ref)
+    # bf16 output: the bar plus one bf16 ulp of the reference
+    o16, _ = run_gpu(x, w, o_dtype=torch.bfloat16)
+    report("gdn_full_auto_o_bf16", o=stats(o16, o_ref))
+    assert bf16_allowance_ok(o16, o_ref)
+
+
+# ------------------------------------------------------------ configuration 3
+
+@needs_cuda
+def test_long_context_state_carry():
+    w = workload("long_context")
+    x = make_inputs(w)
+    o_ref, s_ref = run_oracle(x, w)
+    _check_bf16("long_context_full_auto", w, x, o_ref, s_ref)
+
+
+# ------------------------------------------------------------ configuration 4
+
+@needs_cuda
+@pytest.mark.parametrize("chunk", [64, 128])
+@pytest.mark.parametrize("N", [2, 3, 4])
+def test_neumann_sweep(chunk, N):
+    w = workload("neumann", B=1, H=4, chunk=chunk, neumann_N=N)
+    x = make_inputs(w)
+    o_ref, s_ref = run_oracle(x, w)               # chunk model with the masked series
+    o, s = _check_bf16(f"neumann_C{chunk}_N{N}", w, x, o_ref, s_ref)
+    ex = w.replace(mode="exact")
+    o_ex, s_ex = run_oracle(x, ex)
+    report(f"neumann_C{chunk}_N{N}_vs_exact_oracle", o=stats(o, o_ex), S_T=stats(s, s_ex))
+
+
+# ------------------------------------------------------------ configuration 5
+
+@needs_cuda
+def test_precond_two_gate_small():
+    w = workload("precond_two_gate", B=1, H=2, T=300)
+    x = make_inputs(w, seed=5)
+    o_ref, s_ref = run_oracle(x, w)
+    _check_bf16("precond_small", w, x, o_ref, s_ref)
+
+
+@needs_cuda
+def test_precond_two_gate_full_size():
+    w = workload("precond_two_gate")
+    x = make_inputs(w)
+    o_ref, s_ref = run_oracle(x, w)
+    _check_bf16("precond_full_auto", w, x, o_ref, s_ref)
+
+
+# ------------------------------------------------------------------ edges
+
+@needs_cuda
+@pytest.mark.parametrize("T", [1, 15, 63, 64, 65, 130])
+@pytest.mark.parametrize("chunk", [16, 32, 64, 128])
+def test_ragged_lengths_and_chunk_sizes_fp32(T, chunk):
+    w = workload("plain_fp32", T=T, chunk=chunk, decay="scalar", s0_std=0.02, H=2)
+    x = make_inputs(w, seed=11)
+    o_ref, s_ref = run_oracle(x, w)
+    o, s = run_gpu(x, w)
+    assert np.abs(o - o_ref).max() <= TOL_F32_ABS
+    assert np.abs(s - s_ref).max() <= TOL_F32_ABS
+
+
+@needs_cuda
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 64), (64, 128), (32, 16)])
+def test_head_dims(dk, dv):
+    w = workload("gdn_bf16", B=1, H=2, T=200, dk=dk, dv=dv, s0_std=0.02)
+    x = make_inputs(w, seed=12)
+    o_ref, s_ref = run_oracle(x, w)
+    _check_bf16(f"dims_{dk}_{dv}", w, x, o_ref, s_ref)
+
+
+@needs_cuda
+@pytest.mark.parametrize("kernel", ["auto", "simt"])
+def test_state_chaining_and_in_place_state(kernel):
+    """S_T of the first half fed as S0 of the second equals one call; S_T may alias S0."""
+    w = workload("gdn_bf16", B=1, H=4, T=640, s0_std=0.02)
+    x = make_inputs(w, seed=13)
+    d = {k: (None if v is None else v.cuda()) for k, v in x.items()}
+    import chunked_gated_delta_14_b200 as gdn
+    o_full, s_full = gdn.chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S0=d["S0"],
+                                   o_dtype=torch.float32, kernel=kernel)
+    half = 320
+    sl = lambda t: t[:, :half].contiguous()
+    sr = lambda t: t[:, half:].contiguous()
+    state = d["S0"].clone()
+    o1, _ = gdn.chunk_fwd(sl(d["q"]), sl(d["k"]), sl(d["v"]), sl(d["alpha"]), sl(d["beta"]),
+                          S0=state, S_T=state, o_dtype=torch.float32, kernel=kernel)
+    o2, _ = gdn.chunk_fwd(sr(d["q"]), sr(d["k"]), sr(d["v"]), sr(d["alpha"]), sr(d["beta"]),
+                          S0=state, S_T=state, o_dtype=torch.float32, kernel=kernel)
+    torch.cuda.synchronize()
+    o_cat = torch.cat([o1, o2], dim=1)
+    rms = o_full.double().pow(2).mean().sqrt().item()
+    assert (o_cat - o_full).abs().max().item() <= 1e-2 * rms
+    srms = s_full.double().pow(2).mean().sqrt().item()
+    assert (state - s_full).abs().max().item() <= 1e-2 * srms
+
+
+@needs_cuda
+def test_two_gate_engine_reduces_to_gated_delta():
+    """Per-channel alpha_t 1, erase alpha_t beta_t, write beta_t, no preconditioner
+    on the two-gate path equals the gated delta rule (fp32 io)."""
+    w = workload("plain_fp32", B=1, H=2, T=150, decay="scalar", s0_std=0.02)
+    x = make_inputs(w, seed=14)
+    dk, dv = w.dk, w.dv
+    o_ref, s_ref = run_oracle(x, w)
+    a = x["alpha"]
+    y = dict(x)
+    y["alpha"] = a[..., None].expand(*a.shape, dk).contiguous()
+    y["erase"] = (a * x["beta"])[..., None].expand(*a.shape, dk).contiguous()
+    y["write"] = x["beta"][..., None].expand(*a.shape, dv).contiguous()
+    y["beta"] = None
+    o, s = run_gpu(y, None, precond=False)
+    assert np.abs(o - o_ref).max() <= TOL_F32_ABS
+    assert np.abs(s - s_ref).max() <= TOL_F32_ABS
+
+
+@needs_cuda
+def test_neumann_full_series_equals_exact():
+    """Neumann mode with N = C - 1 is the exact inverse (Lemma 3.1)."""
+    w = workload("gdn_bf16", B=1, H=2, T=256, chunk=32)
+    x = make_inputs(w, seed=15)
+    o_ref, s_ref = run_oracle(x, w)
+    _check_bf16("neumann_N_eq_C_minus_1", w.replace(mode="neumann", neumann_N=31), x,
+                o_ref, s_ref)
+
+
+@needs_cuda
+@pytest.mark.parametrize("split", [1, 2, 4, 8])
+def test_value_split_invariance(split):
+    w = workload("gdn_bf16", B=1, H=2, T=300, s0_std=0.02)
+    x = make_inputs(w, seed=16)
+    o_ref, s_ref = run_oracle(x, w)
+    _check_bf16(f"split_{split}", w, x, o_ref, s_ref, dv_split=split)
