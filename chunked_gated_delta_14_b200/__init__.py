@@ -5,8 +5,8 @@ its Python binding plus the seeded synthetic workloads used by the tests and
 the benchmark.  Build the library with
 ``python -m chunked_gated_delta_14_b200.build``.
 """
-from .gdn import (GDNError, FwdArgs, abi_version, call, chunk_fwd, last_error,  # noqa: F401
-                  lib, make_args, select_kernel, status_string)
+from .gdn import (GDNError, FwdArgs, abi_version, call, chunk_fwd, device_check,  # noqa: F401
+                  last_error, lib, make_args, select_kernel, status_string)
 
-__all__ = ["chunk_fwd", "GDNError", "FwdArgs", "make_args", "call", "select_kernel",
+__all__ = ["chunk_fwd", "device_check", "GDNError", "FwdArgs", "make_args", "call", "select_kernel",
            "abi_version", "last_error", "status_string", "lib"]

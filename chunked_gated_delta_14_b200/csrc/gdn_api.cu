@@ -144,6 +144,15 @@ int32_t gdn_select_kernel(const gdn_fwd_args *args) {
     return kern;
 }
 
+gdn_status gdn_device_check(void *stream) {
+    cudaError_t e = cudaSuccess;
+    const unsigned int code = gdn::tc_read_and_clear_error(reinterpret_cast<cudaStream_t>(stream), &e);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "device check: %s", cudaGetErrorString(e));
+    if (code) return fail(GDN_ERR_DEVICE_CHECK, "tensor-core kernel wait %u gave up", code);
+    g_msg[0] = 0;
+    return GDN_OK;
+}
+
 gdn_status gdn_chunk_fwd(const gdn_fwd_args *args, void *stream) {
     const char *inj = getenv("GDN_FAULT_INJECT");
     if (inj && inj[0] == '1') return fail(GDN_ERR_FAULT_INJECTED, "GDN_FAULT_INJECT=1");

@@ -31,8 +31,8 @@ KERNELS = {"auto": 0, "simt": 1, "tc": 2}
 KERNEL_NAMES = {v: k for k, v in KERNELS.items()}
 MODES = {"exact": GDN_INV_EXACT, "neumann": GDN_INV_NEUMANN}
 
-EXPORTS = ("gdn_chunk_fwd", "gdn_select_kernel", "gdn_status_string", "gdn_last_error",
-           "gdn_abi_version")
+EXPORTS = ("gdn_chunk_fwd", "gdn_select_kernel", "gdn_device_check", "gdn_status_string",
+           "gdn_last_error", "gdn_abi_version")
 
 
 class GDNError(RuntimeError):
@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
             L.gdn_chunk_fwd.restype = ctypes.c_int
             L.gdn_select_kernel.argtypes = [ctypes.POINTER(FwdArgs)]
             L.gdn_select_kernel.restype = ctypes.c_int32
+            L.gdn_device_check.argtypes = [ctypes.c_void_p]
+            L.gdn_device_check.restype = ctypes.c_int
             L.gdn_status_string.argtypes = [ctypes.c_int]
             L.gdn_status_string.restype = ctypes.c_char_p
             L.gdn_last_error.argtypes = []
@@ -144,6 +146,13 @@ def select_kernel(args: FwdArgs) -> int:
 def call(args: FwdArgs, stream: Optional[int] = None) -> None:
     """Raw gdn_chunk_fwd call; raises GDNError on a non-OK status."""
     s = lib().gdn_chunk_fwd(ctypes.byref(args), ctypes.c_void_p(stream or 0))
+    if s != GDN_OK:
+        raise GDNError(s, last_error())
+
+
+def device_check(stream: Optional[int] = None) -> None:
+    """Synchronise and raise GDNError if a kernel recorded a device-side failure."""
+    s = lib().gdn_device_check(ctypes.c_void_p(stream or 0))
     if s != GDN_OK:
         raise GDNError(s, last_error())
 

@@ -128,6 +128,14 @@ GDN_API gdn_status gdn_chunk_fwd(const gdn_fwd_args *args, void *stream);
  * only; launches nothing. */
 GDN_API int32_t gdn_select_kernel(const gdn_fwd_args *args);
 
+/* Synchronises `stream` (void* cudaStream_t), then reports and clears a
+ * failure recorded on the device by the kernels' own checks: a bounded wait
+ * inside the tensor-core kernel that gave up (after about two seconds) makes
+ * the block skip its remaining work and record an error code; this call then
+ * returns GDN_ERR_DEVICE_CHECK.  GDN_ERR_CUDA if synchronising failed, else
+ * GDN_OK. */
+GDN_API gdn_status gdn_device_check(void *stream);
+
 /* Static string for a status code. */
 GDN_API const char *gdn_status_string(gdn_status s);
 
