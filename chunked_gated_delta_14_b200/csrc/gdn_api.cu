@@ -81,7 +81,16 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
 
     const char *why = "";
     int kern = a->kernel;
-    if (kern == GDN_KERNEL_AUTO) kern = gdn::tc_supports(p, &why) ? GDN_KERNEL_TC : GDN_KERNEL_SIMT;
+    if (kern == GDN_KERNEL_AUTO) {
+        // tensor-core kernel when it supports the call, including the requested value split
+        gdn::FwdParams t = p;
+        kern = GDN_KERNEL_SIMT;
+        if (gdn::tc_supports(t, &why)) {
+            t.slices = a->dv_split ? a->dv_split : gdn::tc_default_slices(t);
+            t.dvs = t.dv / t.slices;
+            if (t.dv % t.slices == 0 && gdn::tc_supports(t, &why)) kern = GDN_KERNEL_TC;
+        }
+    }
     if (kern == GDN_KERNEL_TC) {
         if (!gdn::tc_supports(p, &why))
             return fail(GDN_ERR_UNSUPPORTED, "tensor-core kernel: %s", why);

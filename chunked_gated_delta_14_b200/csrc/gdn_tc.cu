@@ -54,7 +54,8 @@ using namespace sm100;
 constexpr int C = 64;          // chunk
 constexpr int DK = 128;        // key dim
 constexpr int DVS = 64;        // value columns per CTA
-constexpr int kThreads = 320;  // 10 warps
+constexpr int kThreads = 448;  // 14 warps
+constexpr int kKsThreads = 256, kChThreads = 128;
 constexpr int kNeumannMaxN = 15;
 
 // shared memory map (bytes from a 1024-aligned base)
@@ -77,6 +78,8 @@ constexpr uint32_t OFF_PAR = OFF_YB + YB_FLOATS * 4;
 
 struct ChunkParams {
     float g2[C];    // cumulative log2 decay at each row
+    float al[C];    // alpha_r (1 on padded rows)
+    float dblk[C];  // e^{g_(end of r's 16-row block) - g_r}
     float eg[C];    // e^{g_r}
     float bet[C];   // beta_r (0 on padded rows)
     float egc[C];   // e^{g_C - g_r}
@@ -85,15 +88,16 @@ struct ChunkParams {
     float pad[2];
 };
 constexpr uint32_t PAR_BYTES = (sizeof(ChunkParams) + 15) & ~15u;
-constexpr uint32_t OFF_BAR = OFF_PAR + 2 * PAR_BYTES;
-enum { B_FULL = 0, B_EMPTY = 2, B_KSREADY = 4, B_KSFREE = 6, B_G = 8, B_X = 9, B_D = 10, B_H = 11,
-       N_BARS = 12 };
+constexpr uint32_t OFF_BAR = OFF_PAR + 3 * PAR_BYTES;   // params ring of 3
+enum { B_FULL = 0, B_EMPTY = 2, B_KSREADY = 4, B_KSFREE = 6, B_G = 8, B_X = 10, B_D = 11, B_H = 12,
+       N_BARS = 13 };
 constexpr uint32_t OFF_MISC = OFF_BAR + N_BARS * 8;    // tmem slot, abort flag, group slots
-constexpr uint32_t SMEM_USED = OFF_MISC + 32;
+constexpr uint32_t SMEM_USED = OFF_MISC + 32;   // tmem slot, abort flag, 3 x 2 group slots
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;      // slack to align the base
+static_assert(SMEM_ALLOC <= 232448, "shared memory budget of one sm_100 block");
 
 // TMEM columns
-constexpr uint32_t TM_G = 0, TM_X0 = 64, TM_X1 = 128, TM_D = 192, TM_H = 256;
+constexpr uint32_t TM_G0 = 0, TM_G1 = 64, TM_X0 = 128, TM_X1 = 192, TM_D = 256, TM_H = 320;
 constexpr uint32_t TM_COLS = 512;
 
 // error codes recorded in g_tc_error (first one wins)
@@ -109,17 +113,12 @@ struct TcParams {
     void *o;
     float *S_T;
     int o_bf16, neumann, N;
-    unsigned long long limit_ns;
+    unsigned long long limit_cycles;
 };
 
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
     __half2 h = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t *>(&h);
-}
-
-__device__ __forceinline__ float2 unpack_h2(uint32_t u) {
-    __half2 h = *reinterpret_cast<__half2 *>(&u);
-    return __half22float2(h);
 }
 
 __device__ __forceinline__ float2 unpack_bf2(uint32_t u) {
@@ -166,9 +165,11 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const float *x) {
 __global__ void __launch_bounds__(kThreads, 1)
 tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const TcParams p) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~static_cast<uintptr_t>(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned base for the 128-byte swizzled tiles.  The offset is
+    // applied to the __shared__ array itself so that every access below stays
+    // a shared-memory access (an integer round trip would turn them generic).
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int T = p.T, H = p.H, dv = p.dv;
@@ -181,11 +182,23 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // Named barrier that also broadcasts the abort state, so that every thread
     // of a role leaves its loop at the same barrier (a failed wait can never
     // strand the others at a bar.sync).  Two alternating slots per role.
-    auto sync_ok = [&](int id, bool leader, int &cnt) -> bool {
+    const unsigned long long lim = p.limit_cycles;
+    // One thread of a role waits for the phase (sleeping), the others wait at
+    // the role's named barrier and then take the acquire with one test.
+    auto group_wait = [&](uint64_t *bar, uint32_t parity, int code, int id, int nthreads, bool leader,
+                          bool sleep = true) {
+        if (leader) {
+            if (sleep) mbar_wait(bar, parity, abort_flag, code, lim);
+            else mbar_wait_spin(bar, parity, abort_flag, code, lim);
+        }
+        named_bar(id, nthreads);
+        if (!leader) mbar_try_wait(bar, parity);
+    };
+    auto sync_ok = [&](int id, int nthreads, bool leader, int &cnt) -> bool {
         volatile int *slots = reinterpret_cast<volatile int *>(sm + OFF_MISC + 8 + 8 * (id - 1));
         const int k = cnt++ & 1;
         if (leader) slots[k] = *abort_flag;
-        named_bar(id, 128);
+        named_bar(id, nthreads);
         return slots[k] == 0;
     };
     ChunkParams *params = reinterpret_cast<ChunkParams *>(sm + OFF_PAR);
@@ -193,7 +206,6 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float *Tb = reinterpret_cast<float *>(sm + OFF_TB);
     float *Yb = reinterpret_cast<float *>(sm + OFF_YB);
     const uint32_t sbase = smem_u32(sm);
-    const unsigned long long lim = p.limit_ns;
 
     // ------------------------------------------------------------- setup
     if (tid == 0) {
@@ -204,6 +216,7 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&bars[B_KSFREE + i], 1);
         }
         mbar_init(&bars[B_G], 1);
+        mbar_init(&bars[B_G + 1], 1);
         mbar_init(&bars[B_X], 1);
         mbar_init(&bars[B_D], 1);
         mbar_init(&bars[B_H], 1);
@@ -252,13 +265,16 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int m = issued - 2 < 0 ? 0 : issued - 2; m < issued; ++m)
                 mbar_wait_drain(&bars[B_FULL + (m & 1)], (m >> 1) & 1, lim);
         }
-    } else if (warp >= 2 && warp < 6) {
+    } else if (warp >= 2 && warp < 10) {
         // ========================================================= key side
-        const int kt = tid - 64;          // 0..127
-        const int sp = warp & 3;          // TMEM sub-partition
-        const bool scan_warp = (sp == 0);
-        // alpha / beta for the next chunk, prefetched by the scan warp
-        float a_nx0 = 0.f, a_nx1 = 0.f, b_nx0 = 0.f, b_nx1 = 0.f;
+        // 8 warps: two per TMEM sub-partition; warp half hf takes columns
+        // [32 hf, 32 hf + 32) of the Gram rows its sub-partition holds.
+        const int kt = tid - 64;                 // 0..255
+        const int sp = warp & 3;
+        const int hf = (warp - 2) >> 2;
+        const bool leader = (kt == 0);
+        const bool scan_warp = (kt >> 5) == 2;    // not used by the diagonal-block solve
+        float a_nx0 = 1.f, a_nx1 = 1.f, b_nx0 = 0.f, b_nx1 = 0.f;
         auto fetch_gates = [&](int m) {
             const int t0 = m * C;
             const int r0 = lane, r1 = lane + 32;
@@ -270,226 +286,296 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             b_nx0 = ok0 ? (p.beta ? __ldg(p.beta + i0) : 1.f) : 0.f;
             b_nx1 = ok1 ? (p.beta ? __ldg(p.beta + i1) : 1.f) : 0.f;
         };
-        if (scan_warp) fetch_gates(0);
-        uint32_t pk[32];  // this thread's row of P, fp16 pairs (sub-partitions 0, 1)
+        // per-chunk gate scan into params[m % 3] (one warp, from prefetched gates)
+        auto scan_chunk = [&](int m) {
+            ChunkParams *par = &params[m % 3];
+            const float x0i = lg2_approx(a_nx0), x1i = lg2_approx(a_nx1);
+            float x0 = x0i, x1 = x1i;
+            const float be0 = b_nx0, be1 = b_nx1, al0 = a_nx0, al1 = a_nx1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y0 = __shfl_up_sync(0xffffffffu, x0, o);
+                const float y1 = __shfl_up_sync(0xffffffffu, x1, o);
+                if (lane >= o) { x0 += y0; x1 += y1; }
+            }
+            x1 += __shfl_sync(0xffffffffu, x0, 31);
+            const float gC = __shfl_sync(0xffffffffu, x1, 31);
+            // cumulative decay at the last row of each row's 16-row block
+            const float e0 = __shfl_sync(0xffffffffu, x0, lane | 15);
+            const float e1 = __shfl_sync(0xffffffffu, x1, lane | 15);
+            par->g2[lane] = x0;
+            par->g2[lane + 32] = x1;
+            par->al[lane] = al0;
+            par->al[lane + 32] = al1;
+            par->dblk[lane] = ex2_approx(e0 - x0);
+            par->dblk[lane + 32] = ex2_approx(e1 - x1);
+            par->eg[lane] = ex2_approx(x0);
+            par->eg[lane + 32] = ex2_approx(x1);
+            par->egc[lane] = ex2_approx(gC - x0);
+            par->egc[lane + 32] = ex2_approx(gC - x1);
+            par->bet[lane] = be0;
+            par->bet[lane + 32] = be1;
+            if (lane == 0) {
+                par->egC = ex2_approx(gC);
+                par->Cv = min(C, T - m * C);
+            }
+            fetch_gates(m + 1);
+        };
+        if (scan_warp) {
+            fetch_gates(0);
+            scan_chunk(0);
+        }
+        uint32_t pk[16];        // this thread's half row of P, fp16 pairs (sub-partitions 0, 1)
         int kcnt = 0;
-        int gram_pending = -1;  // parity of an issued Gram not yet known complete (leader)
+        int gram_next = 0;      // leader: first chunk whose Gram is not issued yet
+        int gram_pend = -1;     // leader: chunk of the last issued Gram (for the error-path drain)
+        auto issue_gram = [&](int m) {
+            uint8_t *stg = sm + (m & 1) * STAGE_BYTES;
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(stg);
+            const uint32_t dst = tmem + ((m & 1) ? TM_G1 : TM_G0);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                umma_f16_ss(dst, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(a0 + off + 8192, 16, 1024),
+                            IDESC_GRAM, kk > 0);
+            }
+            umma_commit(&bars[B_G + (m & 1)]);
+            gram_pend = m;
+            gram_next = m + 1;
+        };
+        // leader: issue the next chunk's Gram early if its tiles have landed
+        auto try_prefetch_gram = [&](int m) {
+            if (leader && gram_next == m + 1 && m + 1 < NC &&
+                mbar_try_wait(&bars[B_FULL + ((m + 1) & 1)], ((m + 1) >> 1) & 1))
+                issue_gram(m + 1);
+        };
         for (int m = 0; m < NC; ++m) {
             const int s = m & 1;
-            ChunkParams *par = &params[s];
+            ChunkParams *par = &params[m % 3];
             uint8_t *st = sm + s * STAGE_BYTES;
             uint8_t *pzt = sm + OFF_PZT + s * PZT_BYTES;
-            // chain finished chunk m-2: params[s] and [P|Z|T][s] are free
-            if (m >= 2) mbar_wait(&bars[B_KSFREE + s], ((m - 2) >> 1) & 1, abort_flag, E_KSFREE, lim);
-            if (scan_warp) {
-                // cumulative log2 decay over the chunk (warp-shuffle scan, 2 rows per lane)
-                float x0 = log2f(a_nx0), x1 = log2f(a_nx1);
-                const float be0 = b_nx0, be1 = b_nx1;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float y0 = __shfl_up_sync(0xffffffffu, x0, o);
-                    const float y1 = __shfl_up_sync(0xffffffffu, x1, o);
-                    if (lane >= o) { x0 += y0; x1 += y1; }
-                }
-                x1 += __shfl_sync(0xffffffffu, x0, 31);
-                const float gC = __shfl_sync(0xffffffffu, x1, 31);
-                par->g2[lane] = x0;
-                par->g2[lane + 32] = x1;
-                par->eg[lane] = exp2f(x0);
-                par->eg[lane + 32] = exp2f(x1);
-                par->egc[lane] = exp2f(gC - x0);
-                par->egc[lane + 32] = exp2f(gC - x1);
-                par->bet[lane] = be0;
-                par->bet[lane + 32] = be1;
-                if (lane == 0) {
-                    par->egC = exp2f(gC);
-                    par->Cv = min(C, T - m * C);
-                }
-                fetch_gates(m + 1);
-            }
-            mbar_wait(&bars[B_FULL + s], (m >> 1) & 1, abort_flag, E_FULL, lim);
+            // chain finished chunk m-2: params[(m+1) % 3] and [P|Z|T][s] are free
+            if (m >= 2) group_wait(&bars[B_KSFREE + s], ((m - 2) >> 1) & 1, E_KSFREE, 1, kKsThreads, leader);
+            group_wait(&bars[B_FULL + s], (m >> 1) & 1, E_FULL, 1, kKsThreads, leader);
             // params written; previous reads of the Gram TMEM done
-            if (!sync_ok(1, kt == 0, kcnt)) break;
-            if (kt == 0) {
-                tc_fence_after();
-                const uint32_t a0 = smem_u32(st);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    umma_f16_ss(tmem + TM_G, sdesc_sw128(a0 + off, 16, 1024),
-                                sdesc_sw128(a0 + off + 8192, 16, 1024), IDESC_GRAM, kk > 0);
-                }
-                umma_commit(&bars[B_G]);
-                gram_pending = m & 1;
-            }
-            mbar_wait(&bars[B_G], m & 1, abort_flag, E_GRAM, lim);
-            if (!sync_ok(1, kt == 0, kcnt)) break;
-            gram_pending = -1;
+            if (!sync_ok(1, kKsThreads, leader, kcnt)) break;
+            if (leader && gram_next == m) issue_gram(m);
+            group_wait(&bars[B_G + s], (m >> 1) & 1, E_GRAM, 1, kKsThreads, leader);
+            if (!sync_ok(1, kKsThreads, leader, kcnt)) break;
             tc_fence_after();
-            // in-place fp16 conversion: Q -> e^{g_r} Q, K, V
-            for (int u = kt; u < 2560; u += 128) {
-                uint8_t *addr;
-                float sc = 1.f;
-                if (u < 1024) {
-                    const int kb = u >> 9, row = (u >> 3) & 63;
-                    addr = st + (kb ? ST_Q1 : ST_Q0) + ((u & 511) << 4);
-                    sc = par->eg[row];
-                } else if (u < 2048) {
-                    const int v = u - 1024;
-                    addr = st + ((v >> 9) ? ST_K1 : ST_K0) + ((v & 511) << 4);
-                } else {
-                    addr = st + ST_V + ((u - 2048) << 4);
-                }
+            // in-place fp16 conversion of the MMA operands: Q -> e^{g_r} Q, K -> K
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+                const int u = kt + 256 * (it & 1);             // chunk within one 8 KB tile
+                const int tile = it >> 1;                      // Q0, Q1, K0, K1
+                uint8_t *addr = st + (tile == 0 ? ST_Q0 : tile == 1 ? ST_Q1 : tile == 2 ? ST_K0 : ST_K1) + (u << 4);
+                const float sc = tile < 2 ? par->eg[u >> 3] : 1.f;
                 uint4 w = *reinterpret_cast<uint4 *>(addr);
-                float2 f0 = unpack_bf2(w.x), f1 = unpack_bf2(w.y), f2 = unpack_bf2(w.z), f3 = unpack_bf2(w.w);
+                const float2 f0 = unpack_bf2(w.x), f1 = unpack_bf2(w.y), f2 = unpack_bf2(w.z), f3 = unpack_bf2(w.w);
                 w.x = pack_h2(f0.x * sc, f0.y * sc);
                 w.y = pack_h2(f1.x * sc, f1.y * sc);
                 w.z = pack_h2(f2.x * sc, f2.y * sc);
                 w.w = pack_h2(f3.x * sc, f3.y * sc);
                 *reinterpret_cast<uint4 *>(addr) = w;
             }
-            // Gram rows: sub-partitions 0,1 hold Q K^T (-> P), 2,3 hold K K^T (-> L)
+            // Gram rows: sub-partitions 0,1 hold Q K^T (-> P), 2,3 hold K K^T (-> L).
+            // This warp's 32 x 32 tile: rows 32 (sp & 1) .., columns 32 hf ..
+            // Decay factors exp(g_r - g_i) without per-element exponentials:
+            // 16-blocks left of r's block as e^{g_r - g_blockend} * dblk[i],
+            // r's own block as a running product of alpha.
             {
-                float x[64];
-                tmem_ld64(tmem + ((uint32_t)(32 * sp) << 16) + TM_G, x);
-                if (sp < 2) {
-                    const int r = 32 * sp + lane;
-                    const float gr = par->g2[r];
+                const int rh = sp & 1;                       // row half (warp-uniform)
+                const int r = 32 * rh + lane;
+                const bool is_p = sp < 2;
+                if (hf > rh) {
+                    // strictly above the diagonal: zero
+                    if (is_p) {
 #pragma unroll
-                    for (int i = 0; i < 64; i += 2) {
-                        const float p0 = (i <= r) ? exp2f(gr - par->g2[i]) * x[i] : 0.f;
-                        const float p1 = (i + 1 <= r) ? exp2f(gr - par->g2[i + 1]) * x[i + 1] : 0.f;
-                        pk[i >> 1] = pack_h2(p0, p1);
+                        for (int j = 0; j < 16; ++j) pk[j] = 0u;
+                    } else {
+                        float *Lr = Lb + r * LSTR + 32 * hf;
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4 *>(Lr + j) = make_float4(0.f, 0.f, 0.f, 0.f);
                     }
                 } else {
-                    const int r = 32 * (sp - 2) + lane;
-                    const float gr = par->g2[r], br = par->bet[r];
-                    float *Lr = Lb + r * LSTR;
+                    uint32_t xr[32];
+                    tmem_ld32(tmem + ((uint32_t)(32 * sp) << 16) + (s ? TM_G1 : TM_G0) + 32 * hf, xr);
+                    const float gr = par->g2[r];
+                    float gam[32];
+                    if (hf < rh) {
+                        const float E0 = ex2_approx(gr - par->g2[32 * hf + 15]);
+                        const float E1 = ex2_approx(gr - par->g2[32 * hf + 31]);
 #pragma unroll
-                    for (int i = 0; i < 64; i += 4) {
-                        float4 v;
-                        v.x = (i + 0 < r) ? br * exp2f(gr - par->g2[i + 0]) * x[i + 0] : 0.f;
-                        v.y = (i + 1 < r) ? br * exp2f(gr - par->g2[i + 1]) * x[i + 1] : 0.f;
-                        v.z = (i + 2 < r) ? br * exp2f(gr - par->g2[i + 2]) * x[i + 2] : 0.f;
-                        v.w = (i + 3 < r) ? br * exp2f(gr - par->g2[i + 3]) * x[i + 3] : 0.f;
-                        *reinterpret_cast<float4 *>(Lr + i) = v;
+                        for (int j = 0; j < 32; ++j) gam[j] = (j < 16 ? E0 : E1) * par->dblk[32 * hf + j];
+                    } else {
+                        const int br = r >> 4;
+#pragma unroll
+                        for (int bb = 0; bb < 2; ++bb) {
+                            const int blk = 2 * hf + bb;
+                            const float E = ex2_approx(gr - par->g2[16 * blk + 15]);
+                            float c = 1.f;
+#pragma unroll
+                            for (int ii = 15; ii >= 0; --ii) {
+                                const int i = 16 * blk + ii;
+                                const float chain = (i <= r) ? c : 0.f;
+                                c = (i <= r) ? c * par->al[i] : c;
+                                gam[16 * bb + ii] = (blk < br) ? E * par->dblk[i] : ((blk == br) ? chain : 0.f);
+                            }
+                        }
+                    }
+                    tmem_wait_ld();
+                    if (is_p) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 2)
+                            pk[j >> 1] = pack_h2(gam[j] * __uint_as_float(xr[j]), gam[j + 1] * __uint_as_float(xr[j + 1]));
+                    } else {
+                        const float br_ = par->bet[r];
+                        float *Lr = Lb + r * LSTR + 32 * hf;
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            const int i = 32 * hf + j;
+                            float4 v;
+                            v.x = (i + 0 < r) ? br_ * gam[j + 0] * __uint_as_float(xr[j + 0]) : 0.f;
+                            v.y = (i + 1 < r) ? br_ * gam[j + 1] * __uint_as_float(xr[j + 1]) : 0.f;
+                            v.z = (i + 2 < r) ? br_ * gam[j + 2] * __uint_as_float(xr[j + 2]) : 0.f;
+                            v.w = (i + 3 < r) ? br_ * gam[j + 3] * __uint_as_float(xr[j + 3]) : 0.f;
+                            *reinterpret_cast<float4 *>(Lr + j) = v;
+                        }
                     }
                 }
             }
             tc_fence_before();
-            named_bar(1, 128);  // L complete
+            named_bar(1, kKsThreads);  // L complete, Gram buffer s read
+            try_prefetch_gram(m);
+            // gates of the next chunk, overlapping the diagonal-block solve
+            if (scan_warp && m + 1 < NC) scan_chunk(m + 1);
             // ------------------------------------------------ T = (I + L)^-1
             if (!p.neumann) {
                 if (kt < 64) {
-                    // 16 x 16 diagonal blocks by forward substitution, one column per thread
+                    // 16 x 16 diagonal blocks by forward substitution, one column per
+                    // thread; each solved entry updates the rows below it at once
                     const int c = kt, base = c & ~15, jc = c & 15;
-                    float xs[16];
+                    float acc[16];
 #pragma unroll
-                    for (int r = 0; r < 16; ++r) {
-                        float acc = (r == jc) ? 1.f : 0.f;
-                        const float *Lr = Lb + (base + r) * LSTR + base;
+                    for (int r = 0; r < 16; ++r) acc[r] = (r == jc) ? 1.f : 0.f;
 #pragma unroll
-                        for (int i = 0; i < r; ++i) acc -= Lr[i] * xs[i];
-                        xs[r] = acc;
+                    for (int i = 0; i < 16; ++i) {
+                        const float xi = acc[i];
+#pragma unroll
+                        for (int r = i + 1; r < 16; ++r) acc[r] -= Lb[(base + r) * LSTR + base + i] * xi;
                     }
 #pragma unroll
-                    for (int r = 0; r < 16; ++r) Tb[(base + r) * LSTR + c] = xs[r];
+                    for (int r = 0; r < 16; ++r) Tb[(base + r) * LSTR + c] = acc[r];
                 }
-                named_bar(1, 128);
-                // 16 -> 32: T_{b1 b0} = -T_{b1 b1} (L_{b1 b0} T_{b0 b0}), for both 32-blocks
+                named_bar(1, kKsThreads);
+                // 16 -> 32: T_{b1 b0} = -T_{b1 b1} (L_{b1 b0} T_{b0 b0}) for both 32-blocks;
+                // two adjacent columns per thread
                 {
-                    const int pr = kt >> 6, rr = (kt >> 2) & 15, c0 = (kt & 3) * 4;
+                    const int pr = kt >> 7, rr = (kt >> 3) & 15, c0 = (kt & 7) * 2;
                     const int b0 = 32 * pr, b1 = b0 + 16;
-                    float y[4] = {0.f, 0.f, 0.f, 0.f};
+                    float y0 = 0.f, y1 = 0.f;
                     const float *Lr = Lb + (b1 + rr) * LSTR + b0;
 #pragma unroll
                     for (int k = 0; k < 16; ++k) {
                         const float l = Lr[k];
-                        const float4 t = *reinterpret_cast<const float4 *>(Tb + (b0 + k) * LSTR + b0 + c0);
-                        y[0] += l * t.x; y[1] += l * t.y; y[2] += l * t.z; y[3] += l * t.w;
+                        const float2 t = *reinterpret_cast<const float2 *>(Tb + (b0 + k) * LSTR + b0 + c0);
+                        y0 += l * t.x; y1 += l * t.y;
                     }
-                    *reinterpret_cast<float4 *>(Yb + pr * 256 + rr * 16 + c0) = make_float4(y[0], y[1], y[2], y[3]);
-                    named_bar(1, 128);
-                    float z[4] = {0.f, 0.f, 0.f, 0.f};
+                    *reinterpret_cast<float2 *>(Yb + pr * 256 + rr * 16 + c0) = make_float2(y0, y1);
+                    named_bar(1, kKsThreads);
+                    float z0 = 0.f, z1 = 0.f;
                     const float *Tr = Tb + (b1 + rr) * LSTR + b1;
 #pragma unroll
                     for (int k = 0; k < 16; ++k) {
-                        const float t = (k <= rr) ? Tr[k] : 0.f;
-                        const float4 yy = *reinterpret_cast<const float4 *>(Yb + pr * 256 + k * 16 + c0);
-                        z[0] += t * yy.x; z[1] += t * yy.y; z[2] += t * yy.z; z[3] += t * yy.w;
+                        const float t = Tr[k];   // T_{b1 b1} is lower triangular, zeros above
+                        const float2 yy = *reinterpret_cast<const float2 *>(Yb + pr * 256 + k * 16 + c0);
+                        z0 += t * yy.x; z1 += t * yy.y;
                     }
-                    *reinterpret_cast<float4 *>(Tb + (b1 + rr) * LSTR + b0 + c0) =
-                        make_float4(-z[0], -z[1], -z[2], -z[3]);
+                    *reinterpret_cast<float2 *>(Tb + (b1 + rr) * LSTR + b0 + c0) = make_float2(-z0, -z1);
                 }
-                named_bar(1, 128);
-                // 32 -> 64: T_{10} = -T_{11} (L_{10} T_{00}) with 32 x 32 blocks
+                named_bar(1, kKsThreads);
+                // 32 -> 64: T_{10} = -T_{11} (L_{10} T_{00}) with 32 x 32 blocks.  The
+                // triangular factors make the work per output uneven; each thread
+                // takes two output pairs whose work sums to about the same.
                 {
-                    const int rr = kt >> 2, c0 = (kt & 3) * 8;
-                    float y[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) y[j] = 0.f;
+                    const int rr = kt >> 3, q = kt & 7;          // row of L_10, column pair group
+                    const int ca = 2 * q, cb = 30 - 2 * q;       // column pairs (ca, ca+1), (cb, cb+1)
+                    float ya0 = 0.f, ya1 = 0.f, yb0 = 0.f, yb1 = 0.f;
                     const float *Lr = Lb + (32 + rr) * LSTR;
-#pragma unroll 8
-                    for (int k = 0; k < 32; ++k) {
+                    for (int k = ca; k < 32; ++k) {
                         const float l = Lr[k];
-                        const float4 t0 = *reinterpret_cast<const float4 *>(Tb + k * LSTR + c0);
-                        const float4 t1 = *reinterpret_cast<const float4 *>(Tb + k * LSTR + c0 + 4);
-                        y[0] += l * t0.x; y[1] += l * t0.y; y[2] += l * t0.z; y[3] += l * t0.w;
-                        y[4] += l * t1.x; y[5] += l * t1.y; y[6] += l * t1.z; y[7] += l * t1.w;
+                        const float2 t = *reinterpret_cast<const float2 *>(Tb + k * LSTR + ca);
+                        ya0 += l * t.x; ya1 += l * t.y;
                     }
-                    *reinterpret_cast<float4 *>(Yb + rr * 32 + c0) = make_float4(y[0], y[1], y[2], y[3]);
-                    *reinterpret_cast<float4 *>(Yb + rr * 32 + c0 + 4) = make_float4(y[4], y[5], y[6], y[7]);
-                    named_bar(1, 128);
-                    float z[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) z[j] = 0.f;
-                    const float *Tr = Tb + (32 + rr) * LSTR + 32;
-#pragma unroll 8
-                    for (int k = 0; k < 32; ++k) {
-                        const float t = (k <= rr) ? Tr[k] : 0.f;
-                        const float4 a0 = *reinterpret_cast<const float4 *>(Yb + k * 32 + c0);
-                        const float4 a1 = *reinterpret_cast<const float4 *>(Yb + k * 32 + c0 + 4);
-                        z[0] += t * a0.x; z[1] += t * a0.y; z[2] += t * a0.z; z[3] += t * a0.w;
-                        z[4] += t * a1.x; z[5] += t * a1.y; z[6] += t * a1.z; z[7] += t * a1.w;
+                    for (int k = cb; k < 32; ++k) {
+                        const float l = Lr[k];
+                        const float2 t = *reinterpret_cast<const float2 *>(Tb + k * LSTR + cb);
+                        yb0 += l * t.x; yb1 += l * t.y;
                     }
-                    float *dst = Tb + (32 + rr) * LSTR + c0;
-                    *reinterpret_cast<float4 *>(dst) = make_float4(-z[0], -z[1], -z[2], -z[3]);
-                    *reinterpret_cast<float4 *>(dst + 4) = make_float4(-z[4], -z[5], -z[6], -z[7]);
+                    *reinterpret_cast<float2 *>(Yb + rr * 32 + ca) = make_float2(ya0, ya1);
+                    *reinterpret_cast<float2 *>(Yb + rr * 32 + cb) = make_float2(yb0, yb1);
+                    named_bar(1, kKsThreads);
+                    // rows (ra, rb) = (p, 31 - p) pair up the triangular sums k <= row
+                    const int pp = kt >> 4, cq = (kt & 15) * 2;
+                    const int ra = pp, rb = 31 - pp;
+                    float za0 = 0.f, za1 = 0.f, zb0 = 0.f, zb1 = 0.f;
+                    const float *Ta = Tb + (32 + ra) * LSTR + 32;
+                    const float *Tbr = Tb + (32 + rb) * LSTR + 32;
+                    for (int k = 0; k <= ra; ++k) {
+                        const float t = Ta[k];
+                        const float2 yy = *reinterpret_cast<const float2 *>(Yb + k * 32 + cq);
+                        za0 += t * yy.x; za1 += t * yy.y;
+                    }
+                    for (int k = 0; k <= rb; ++k) {
+                        const float t = Tbr[k];
+                        const float2 yy = *reinterpret_cast<const float2 *>(Yb + k * 32 + cq);
+                        zb0 += t * yy.x; zb1 += t * yy.y;
+                    }
+                    *reinterpret_cast<float2 *>(Tb + (32 + ra) * LSTR + cq) = make_float2(-za0, -za1);
+                    *reinterpret_cast<float2 *>(Tb + (32 + rb) * LSTR + cq) = make_float2(-zb0, -zb1);
                 }
             } else {
                 // masked Neumann series by Horner's rule on the band (A = -L):
-                // T^(0) = I, T^(s)_ij = [i-j <= N] (delta_ij - sum_k L_ik T^(s-1)_kj)
-                const int N = p.N, W = N + 1;
-                float *cur = Yb, *nxt = Yb + 64 * W;
-                for (int e = kt; e < 64 * W; e += 128) cur[e] = (e % W == 0) ? 1.f : 0.f;
-                named_bar(1, 128);
+                // T^(0) = I, T^(s)_ij = [i-j <= N] (delta_ij - sum_k L_ik T^(s-1)_kj).
+                // band rows are 16 wide: band[i*16 + d] = T_{i, i-d}, d <= N <= 15;
+                // thread (i, dq) owns diagonals dq, dq+4, dq+8, dq+12 of row i
+                const int N = p.N;
+                const int i = kt >> 2, dq = kt & 3;
+                float *cur = Yb, *nxt = Yb + 1024;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) cur[i * 16 + dq + 4 * u] = (dq + 4 * u == 0) ? 1.f : 0.f;
+                named_bar(1, kKsThreads);
                 for (int step = 0; step < N; ++step) {
-                    for (int e = kt; e < 64 * W; e += 128) {
-                        const int i = e / W, d = e % W, j = i - d;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int d = dq + 4 * u, j = i - d;
                         float val = 0.f;
-                        if (j >= 0) {
+                        if (j >= 0 && d <= N) {
                             val = (d == 0) ? 1.f : 0.f;
-                            const int kmax = min(i - 1, j + N);
-                            for (int k = j; k <= kmax; ++k) val -= Lb[i * LSTR + k] * cur[k * W + (k - j)];
+                            // k from j to i-1; T_kj is in the band while k - j <= N
+                            for (int k = j; k < i; ++k) val -= Lb[i * LSTR + k] * cur[k * 16 + (k - j)];
                         }
-                        nxt[e] = val;
+                        nxt[i * 16 + d] = val;
                     }
-                    named_bar(1, 128);
+                    named_bar(1, kKsThreads);
                     float *sw = cur; cur = nxt; nxt = sw;
                 }
-                for (int e = kt; e < 64 * 64; e += 128) {
-                    const int i = e >> 6, j = e & 63, d = i - j;
-                    Tb[i * LSTR + j] = (d >= 0 && d <= N) ? cur[i * W + d] : 0.f;
+#pragma unroll 4
+                for (int qq = 0; qq < 16; ++qq) {
+                    const int e = kt + 256 * qq, ii = e >> 6, j = e & 63, d = ii - j;
+                    Tb[ii * LSTR + j] = (d >= 0 && d <= N) ? cur[ii * 16 + d] : 0.f;
                 }
             }
-            named_bar(1, 128);  // T complete
+            named_bar(1, kKsThreads);  // T complete
+            try_prefetch_gram(m);
             // ------------------------------------------ T and P to fp16 operands
             {
-                const int r = kt >> 1, hf = kt & 1;
+                const int r = kt >> 2, j0 = (kt & 3) * 2;
                 const float *Tr = Tb + r * LSTR;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int j = hf * 4 + q;
+                for (int q = 0; q < 2; ++q) {
+                    const int j = j0 + q;
                     const float4 a = *reinterpret_cast<const float4 *>(Tr + 8 * j);
                     const float4 c = *reinterpret_cast<const float4 *>(Tr + 8 * j + 4);
                     uint4 u;
@@ -500,19 +586,20 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (sp < 2) {
                     const int rp = 32 * sp + lane;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<uint4 *>(pzt + sw128_off(rp, j)) =
-                            make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                    for (int jj = 0; jj < 4; ++jj)
+                        *reinterpret_cast<uint4 *>(pzt + sw128_off(rp, 4 * hf + jj)) =
+                            make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
                 }
             }
             fence_proxy_async_smem();
-            named_bar(1, 128);
-            if (kt == 0) mbar_arrive(&bars[B_KSREADY + s]);
+            named_bar(1, kKsThreads);
+            if (leader) mbar_arrive(&bars[B_KSREADY + s]);
         }
-        if (kt == 0 && gram_pending >= 0) mbar_wait_drain(&bars[B_G], gram_pending, lim);
-    } else if (warp >= 6) {
+        if (leader && gram_pend >= 0 && *abort_flag)
+            mbar_wait_drain(&bars[B_G + (gram_pend & 1)], (gram_pend >> 1) & 1, lim);
+    } else if (warp >= 10) {
         // ========================================================= state chain
-        const int ct = tid - 192;          // 0..127
+        const int ct = tid - 320;          // 0..127
         const int sp = warp & 3;
         const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
         const int hrow = 32 * sp + lane;   // dk row of h held by this thread
@@ -563,34 +650,40 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
         };
-        int ccnt = 0;
-        // leader only: barrier index and parity of the last commit not yet known complete
+        int ccnt = 0, dcnt = 0;
+        // issuer only: barrier index and parity of the last commit not yet known complete
         int pend_bar = -1, pend_par = 0;
+        const bool issuer = (ct == 0);        // warp 10, sub-partition 2
+        const bool rowpart = (sp >= 2);       // R and Delta rows live in TMEM lanes 64..127
         bool done = true;
         for (int n = 0; n < NC; ++n) {
             const int s = n & 1;
-            const ChunkParams *par = &params[s];
+            const ChunkParams *par = &params[n % 3];
             uint8_t *st = sm + s * STAGE_BYTES;
             uint8_t *pzt = sm + OFF_PZT + s * PZT_BYTES;
             const uint32_t tx = tmem + (s ? TM_X1 : TM_X0);
-            mbar_wait(&bars[B_KSREADY + s], (n >> 1) & 1, abort_flag, E_KSREADY, lim);
-            if (n > 0) mbar_wait(&bars[B_H], (n - 1) & 1, abort_flag, E_H, lim);
+            group_wait(&bars[B_KSREADY + s], (n >> 1) & 1, E_KSREADY, 2, kChThreads, issuer, true);
+            if (n > 0) group_wait(&bars[B_H], (n - 1) & 1, E_H, 2, kChThreads, issuer, false);
             tc_fence_after();
-            // ---- h -> fp16 operand; h <- e^{g_C} h
+            // ---- h <- e^{g_C} h in TMEM (issued first), h -> fp16 operand
             {
                 float x[64];
                 tmem_ld64(tmem + lane_base + TM_H, x);
-                st_row_f16(hs, hrow, x);
                 const float egC = par->egC;
 #pragma unroll
-                for (int j = 0; j < 64; ++j) x[j] *= egC;
-                tmem_st64(tmem + lane_base + TM_H, x);
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t y[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) y[j] = __float_as_uint(x[32 * hh + j] * egC);
+                    tmem_st32(tmem + lane_base + TM_H + 32 * hh, y);
+                }
+                st_row_f16(hs, hrow, x);
                 tmem_wait_st();
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            if (!sync_ok(2, ct == 0, ccnt)) { done = false; break; }
-            if (ct == 0) {
+            if (!sync_ok(2, kChThreads, issuer, ccnt)) { done = false; break; }
+            if (issuer) {
                 tc_fence_after();
                 const uint32_t a0 = smem_u32(st), b0 = smem_u32(hs);
 #pragma unroll
@@ -602,11 +695,15 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 umma_commit(&bars[B_X]);
                 pend_bar = B_X; pend_par = n & 1;
             }
-            if (n > 0 && sp < 2) store_o(n - 1);
-            mbar_wait(&bars[B_X], n & 1, abort_flag, E_X, lim);
+            if (!rowpart) {
+                // sub-partitions 0, 1: output rows of the previous chunk, off the chain
+                if (n > 0) store_o(n - 1);
+                continue;
+            }
+            group_wait(&bars[B_X], n & 1, E_X, 3, 64, issuer, false);
             tc_fence_after();
             // ---- R = beta (v - e^g K h), rows in lanes 64..127
-            if (sp >= 2) {
+            {
                 const int r = 32 * (sp - 2) + lane;
                 float x[64];
                 tmem_ld64(tmem + lane_base + (s ? TM_X1 : TM_X0), x);
@@ -615,7 +712,7 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const uint4 w = *reinterpret_cast<const uint4 *>(vrow + sw128_off(r, j));
-                    const float2 f0 = unpack_h2(w.x), f1 = unpack_h2(w.y), f2 = unpack_h2(w.z), f3 = unpack_h2(w.w);
+                    const float2 f0 = unpack_bf2(w.x), f1 = unpack_bf2(w.y), f2 = unpack_bf2(w.z), f3 = unpack_bf2(w.w);
                     x[8 * j + 0] = br * (f0.x - er * x[8 * j + 0]);
                     x[8 * j + 1] = br * (f0.y - er * x[8 * j + 1]);
                     x[8 * j + 2] = br * (f1.x - er * x[8 * j + 2]);
@@ -629,8 +726,9 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            if (!sync_ok(2, ct == 0, ccnt)) { done = false; break; }
-            if (ct == 0) {
+            // 64-thread barrier of sub-partitions 2, 3; an abort here only stops the
+            // MMAs, the loop exits at the next 128-thread barrier
+            if (sync_ok(3, 64, issuer, dcnt) && issuer) {
                 tc_fence_after();
                 const uint32_t a0 = smem_u32(pzt + PZT_Z), b0 = smem_u32(rs);
 #pragma unroll
@@ -640,10 +738,10 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 umma_commit(&bars[B_D]);
                 pend_bar = B_D; pend_par = n & 1;
             }
-            mbar_wait(&bars[B_D], n & 1, abort_flag, E_D, lim);
+            group_wait(&bars[B_D], n & 1, E_D, 3, 64, issuer, false);
             tc_fence_after();
             // ---- Delta (rows in lanes 64..127) -> fp16 operands
-            if (sp >= 2) {
+            {
                 const int r = 32 * (sp - 2) + lane;
                 float x[64];
                 tmem_ld64(tmem + lane_base + TM_D, x);
@@ -655,8 +753,7 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            if (!sync_ok(2, ct == 0, ccnt)) { done = false; break; }
-            if (ct == 0) {
+            if (sync_ok(3, 64, issuer, dcnt) && issuer) {
                 tc_fence_after();
                 const uint32_t ap = smem_u32(pzt), bd = smem_u32(ds);
                 const uint32_t ak = smem_u32(st + ST_K0), bdp = smem_u32(dps);
@@ -675,11 +772,11 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
         if (done && NC > 0) {
-            mbar_wait(&bars[B_H], (NC - 1) & 1, abort_flag, E_H, lim);
-            if (sync_ok(2, ct == 0, ccnt)) {
-                if (ct == 0) pend_bar = -1;
+            group_wait(&bars[B_H], (NC - 1) & 1, E_H, 2, kChThreads, issuer, false);
+            if (sync_ok(2, kChThreads, issuer, ccnt)) {
+                if (issuer) pend_bar = -1;
                 tc_fence_after();
-                if (sp < 2) store_o(NC - 1);
+                if (!rowpart) store_o(NC - 1);
                 if (p.S_T) {
                     float x[64];
                     tmem_ld64(tmem + lane_base + TM_H, x);
@@ -691,7 +788,7 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
         // error path: no MMA of this role may still be running when TMEM is released
-        if (ct == 0 && pend_bar >= 0 && *abort_flag) mbar_wait_drain(&bars[pend_bar], pend_par, lim);
+        if (issuer && pend_bar >= 0 && *abort_flag) mbar_wait_drain(&bars[pend_bar], pend_par, lim);
     }
     // ---------------------------------------------------------- teardown
     tc_fence_before();
@@ -762,7 +859,7 @@ cudaError_t launch_tc(const FwdParams &p, cudaStream_t stream, const char **why)
     tp.B = p.B; tp.T = p.T; tp.H = p.H; tp.dv = p.dv;
     tp.alpha = p.alpha; tp.beta = p.beta; tp.S0 = p.S0; tp.o = p.o; tp.S_T = p.S_T;
     tp.o_bf16 = p.o_bf16; tp.neumann = p.mode == GDN_INV_NEUMANN; tp.N = p.N;
-    tp.limit_ns = 2000000000ull;
+    tp.limit_cycles = 4000000000ull;  // ~2 s at the B200 boost clock
     dim3 grid(p.slices, p.H, p.B);
     tc_chunk_kernel<<<grid, kThreads, SMEM_ALLOC, stream>>>(mq, mk, mv, tp);
     return cudaGetLastError();

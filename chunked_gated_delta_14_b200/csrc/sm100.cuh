@@ -14,12 +14,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
@@ -54,17 +48,53 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but lets the hardware suspend the thread until the phase
+// completes or about `hint_ns` elapse, so that a waiting warp does not keep
+// polling shared memory.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for phase `parity` of `bar`.  Gives up (returns false) when
-// *abort is set by another role or after `limit_ns`, recording `code` in
-// *abort in the latter case.
+// *abort is set by another role or after about `limit_cycles` SM clock
+// cycles, recording `code` in *abort in the latter case.  The clock and the
+// abort flag are only consulted every 8 (sleeping) polls so that a waiting warp costs
+// its SM sub-partition as few issue slots as possible.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          int code, uint64_t limit_ns) {
+                                          int code, uint64_t limit_cycles) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const uint64_t t0 = clock64();
     for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i)
+            if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
         if (*abort) return false;
-        if (globaltimer_ns() - t0 > limit_ns) {
+        if (static_cast<uint64_t>(clock64()) - t0 > limit_cycles) {
+            atomicCAS(const_cast<int *>(abort), 0, code);
+            return false;
+        }
+    }
+}
+
+// As mbar_wait but polling without sleeping: for short waits on the critical
+// path (an MMA commit) where the wake-up latency of a suspended thread shows.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                               int code, uint64_t limit_cycles) {
+    const uint64_t t0 = clock64();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (static_cast<uint64_t>(clock64()) - t0 > limit_cycles) {
             atomicCAS(const_cast<int *>(abort), 0, code);
             return false;
         }
@@ -73,11 +103,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 
 // Bounded wait that ignores the abort flag (drains copies or MMAs still in
 // flight before a block releases its resources on an error path).
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
-    const uint64_t t0 = globaltimer_ns();
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, uint64_t limit_cycles) {
+    const uint64_t t0 = clock64();
     while (!mbar_try_wait(bar, parity))
-        if (globaltimer_ns() - t0 > limit_ns) return false;
+        if (static_cast<uint64_t>(clock64()) - t0 > limit_cycles) return false;
     return true;
+}
+
+// log2(x) on the special-function unit (PTX lg2.approx.ftz.f32).
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// 2^x on the special-function unit (PTX ex2.approx.ftz.f32; relative error
+// about 2^-22 over the range used here, x <= 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // ----------------------------------------------------------------------- TMA
