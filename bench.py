@@ -186,8 +186,12 @@ def run_gpu(args, rank, world, local_rank):
                       o_dtype=0, q=ptr(d["q"]), k=ptr(d["k"]), v=ptr(d["v"]),
                       alpha=ptr(d["alpha"]), beta=ptr(d["beta"]), S0=None, o=o.data_ptr(),
                       S_T=S_T.data_ptr(), mode=0, kernel=0)
+    ws = gdn.workspace_for(a, dev)
+    if ws is not None:
+        a.workspace = ws.data_ptr()
+        a.workspace_bytes = ws.numel()
     kernel_id = gdn.select_kernel(a)
-    kernel_name = {1: "simt_chunk_kernel", 2: "tc_chunk_kernel"}.get(kernel_id, "?")
+    kernel_name = {1: "simt_chunk_kernel", 2: "keyside_kernel+chain_kernel"}.get(kernel_id, "?")
     sh = stream.cuda_stream
 
     def step():

@@ -60,7 +60,8 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
     for (const void *x : ins)
         if (x && x == a->o) return fail(GDN_ERR_INVALID_ARG, "o aliases an input");
     if (a->S_T && (const void *)a->S_T == a->o) return fail(GDN_ERR_INVALID_ARG, "o aliases S_T");
-    const void *al[] = {a->q, a->k, a->v, a->o, a->erase, a->write, a->S0, a->S_T, a->alpha, a->beta};
+    const void *al[] = {a->q, a->k, a->v, a->o, a->erase, a->write, a->S0, a->S_T, a->alpha, a->beta,
+                        a->workspace};
     for (const void *x : al)
         if (x && !aligned16(x)) return fail(GDN_ERR_ALIGNMENT, "pointers must be 16-byte aligned");
     if (a->kernel < GDN_KERNEL_AUTO || a->kernel > GDN_KERNEL_TC)
@@ -144,6 +145,14 @@ const char *gdn_last_error(void) { return g_msg; }
 
 int32_t gdn_abi_version(void) { return GDN_ABI_VERSION; }
 
+uint64_t gdn_workspace_bytes(const gdn_fwd_args *args) {
+    gdn::FwdParams p;
+    int kern = 0;
+    if (resolve(args, &p, &kern) != GDN_OK) return 0;
+    g_msg[0] = 0;
+    return kern == GDN_KERNEL_TC ? (uint64_t)gdn::tc_workspace_bytes(p) : 0;
+}
+
 int32_t gdn_select_kernel(const gdn_fwd_args *args) {
     gdn::FwdParams p;
     int kern = 0;
@@ -172,8 +181,16 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_args *args, void *stream) {
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
     const char *why = "";
-    if (kern == GDN_KERNEL_TC) e = gdn::launch_tc(p, st, &why);
-    else e = gdn::launch_simt(p, st);
+    if (kern == GDN_KERNEL_TC) {
+        const size_t need = gdn::tc_workspace_bytes(p);
+        if (!args->workspace || args->workspace_bytes < need)
+            return fail(GDN_ERR_INVALID_ARG, "tensor-core kernel needs a workspace of %zu bytes (got %llu)",
+                        need, (unsigned long long)args->workspace_bytes);
+        e = gdn::launch_tc(p, args->workspace, st, &why);
+    }
+    else {
+        e = gdn::launch_simt(p, st);
+    }
     if (e != cudaSuccess)
         return fail(GDN_ERR_CUDA, "%s launch: %s %s", kern == GDN_KERNEL_TC ? "tc" : "simt",
                     cudaGetErrorString(e), why);

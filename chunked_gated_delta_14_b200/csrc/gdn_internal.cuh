@@ -35,7 +35,8 @@ cudaError_t launch_simt(const FwdParams &p, cudaStream_t stream);
 // Tensor-core kernel (tcgen05 / TMEM / TMA).
 bool tc_supports(const FwdParams &p, const char **why);
 int tc_default_slices(const FwdParams &p);
-cudaError_t launch_tc(const FwdParams &p, cudaStream_t stream, const char **why);
+size_t tc_workspace_bytes(const FwdParams &p);
+cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, const char **why);
 // Synchronise `stream`, return (and clear) the tensor-core kernel's error word.
 unsigned int tc_read_and_clear_error(cudaStream_t stream, cudaError_t *err);
 

@@ -1,39 +1,40 @@
-// Tensor-core chunk kernel for the gated delta rule on sm_100a.
+// Tensor-core path of the chunkwise gated delta rule on sm_100a: two kernels.
 //
-// One CTA per (batch, head, 64-column value slice) walks the chunks of its
-// sequence in order.  The fp32 state h = S^T (128 x 64) lives in TMEM for the
-// whole sequence.  Warp roles:
-//   warp 0      TMA producer: q, k (two 64-column boxes each) and the v slice
-//               of chunk m into a 2-stage ring (128-byte swizzle).
-//   warp 1      TMEM allocation / release.
-//   warps 2-5   "key side" (depends on the chunk's keys only, runs a chunk
-//               ahead): gate scan (cumulative log2 decay), Gram MMA
-//               [Q;K] K^T (bf16 operands, exact products), in-place fp16
-//               conversion of Q (scaled by e^{g_r}), K and V, the decayed
-//               causal scores P and the strictly lower L, and the inverse
-//               T = (I + L)^-1 = (I - A)^-1 (exact blocked or masked Neumann).
-//   warps 6-9   "state chain" (serial over chunks):
-//                 h16 <- h (fp16 copy in smem);  h <- e^{g_C} h in TMEM
-//                 [Q'h ; Kh]     = [Q' ; K] h16                      (MMA)
-//                 R_r            = beta_r (v_r - e^{g_r} (K h)_r)
-//                 Delta          = T R                               (MMA)
-//                 O              = Q'h + P Delta                     (MMA)
-//                 h             += K^T (e^{g_C - g} (.) Delta)       (MMA)
-// All MMAs are tcgen05.mma kind::f16 with M = 128 (64-row operands are stacked
-// with a zero block), fp32 accumulation in TMEM.  Derived operands (h, R,
-// Delta, T, P, Q') are fp16: on this workload bf16 operands leave the outputs
-// outside the 2e-2-of-RMS accuracy bar, fp16 operands do not.
+// 1. keyside_kernel -- the chunk-local A/T builder, one CTA per (chunk, head,
+//    batch), all chunks in parallel.  TMA loads the chunk's keys; a tcgen05
+//    MMA forms the Gram matrix K K^T (bf16 operands, exact products, fp32 in
+//    TMEM); the decayed strictly lower L_ri = beta_r exp(g_r - g_i) (k_r.k_i)
+//    (A = -L) is formed on the CUDA cores and T = (I - A)^-1 is built either
+//    exactly (16 x 16 diagonal blocks by forward substitution, merged
+//    16 -> 32 -> 64 by T21 = -T22 L21 T11) or as the masked truncated Neumann
+//    series M^(N) (.) sum_{n<=N} A^n by Horner's rule on the band.  T is
+//    written in fp16 to a workspace ([B, H, chunks, 64, 64]).
 //
-// The chunk system (I + L) Delta = diag(beta)(V - diag(e^g) K h) is the WY/UT
-// form of the recurrence S_t = S_{t-1} alpha_t (I - beta_t k_t k_t^T) +
-// beta_t v_t k_t^T; its triangular inverse T = (I - A)^-1 with A = -L strictly
-// lower is the step "Quando o 'Bom o Suficiente' e Otimo: Aproximacao de
-// Inversao de Matriz Baseada Apenas em Multiplicacao para Gated DeltaNet
-// Quantizado" (section "Declaracao do Problema") singles out.  Exact mode:
-// 16 x 16 diagonal blocks by forward substitution, merged 16 -> 32 -> 64 by
-// T21 = -T22 L21 T11.  Neumann mode: the masked truncated series
-// M^(N) (.) sum_{n<=N} A^n (section "Metodologia", items 1-2) by Horner's
-// rule T <- M (.) (I + A T), keeping only the band the mask leaves non-zero.
+// 2. chain_kernel -- one CTA per (batch, head, 64-column value slice) walks
+//    the chunks in order with the fp32 state h = S^T (128 x 64) in TMEM.
+//      warp 0      TMA producer: q, k, v slice, T of chunk m (2-stage ring)
+//      warp 1      TMEM allocation
+//      warps 2-9   key side of chunk m (runs ahead of the chain): gate scan,
+//                  Gram Q K^T -> decayed causal scores P, fp16 operands
+//                  Q' = diag(e^g) Q, K, beta V, T diag(beta e^g), and the WY
+//                  products U = T (beta V), W = T diag(beta e^g) K (MMAs)
+//      warps 10-13 state chain:
+//                  h16 <- h;  h <- e^{g_C} h               (TMEM)
+//                  [-W h ; Q' h] = [-W ; Q'] h16            (MMA)
+//                  Delta = U - W h                          (CUDA cores)
+//                  O = Q'h + P Delta ; h += K^T (e^{g_C - g} Delta)   (MMAs)
+//    Every MMA is tcgen05.mma kind::f16, M = 128: a 64-row operand is paired
+//    with whatever 64 rows follow it in shared memory; the TMEM lanes those
+//    rows produce are never read (or are read before they are overwritten).
+//    Derived operands are fp16: with bf16 operands the outputs of this
+//    workload leave the 2e-2-of-RMS accuracy bar, with fp16 they stay inside.
+//
+// The recurrence is S_t = S_{t-1} alpha_t (I - beta_t k_t k_t^T) +
+// beta_t v_t k_t^T, o_t = S_t q_t; the chunk system (I - A) Delta =
+// diag(beta)(V - diag(e^g) K h) with T = (I - A)^-1 is the step "Quando o 'Bom
+// o Suficiente' e Otimo: Aproximacao de Inversao de Matriz Baseada Apenas em
+// Multiplicacao para Gated DeltaNet Quantizado" (section "Declaracao do
+// Problema") singles out; its Neumann and mask items are "Metodologia" 1, 2.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -41,7 +42,7 @@
 #include <cudaTypedefs.h>
 
 #include "gdn_internal.cuh"
-#include "sm100.cuh"
+#include "gdn_tc_common.cuh"
 
 namespace gdn {
 
@@ -50,121 +51,212 @@ __device__ unsigned int g_tc_error = 0;
 namespace {
 
 using namespace sm100;
+using tc::C;
+using tc::ChunkParams;
+using tc::DK;
+using tc::LSTR;
+using tc::pack_h2;
+using tc::st_row_f16;
+using tc::tmem_ld64;
+using tc::unpack_bf2;
+using tc::unpack_h2;
 
-constexpr int C = 64;          // chunk
-constexpr int DK = 128;        // key dim
-constexpr int DVS = 64;        // value columns per CTA
-constexpr int kThreads = 448;  // 14 warps
-constexpr int kKsThreads = 256, kChThreads = 128;
+constexpr int DVS = 64;            // value columns per chain CTA
 constexpr int kNeumannMaxN = 15;
-
-// shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t STAGE_BYTES = 40960;
-constexpr uint32_t ST_Q0 = 0, ST_K0 = 8192, ST_Q1 = 16384, ST_K1 = 24576, ST_V = 32768;
-constexpr uint32_t OFF_PZT = 2 * STAGE_BYTES;          // [P | Z | T] x 2
-constexpr uint32_t PZT_BYTES = 24576;
-constexpr uint32_t PZT_Z = 8192, PZT_T = 16384;
-constexpr uint32_t OFF_HS = OFF_PZT + 2 * PZT_BYTES;   // h fp16, 128 rows
-constexpr uint32_t OFF_RS = OFF_HS + 16384;            // R fp16
-constexpr uint32_t OFF_DS = OFF_RS + 8192;             // Delta fp16
-constexpr uint32_t OFF_DPS = OFF_DS + 8192;            // e^{g_C-g} Delta fp16
-constexpr int LSTR = 68;                               // fp32 row stride of L, T
-constexpr uint32_t MAT_BYTES = 64 * LSTR * 4;
-constexpr uint32_t OFF_LB = OFF_DPS + 8192;
-constexpr uint32_t OFF_TB = OFF_LB + MAT_BYTES;
-constexpr uint32_t OFF_YB = OFF_TB + MAT_BYTES;        // merge temporaries / Horner band
-constexpr uint32_t YB_FLOATS = 2048;
-constexpr uint32_t OFF_PAR = OFF_YB + YB_FLOATS * 4;
-
-struct ChunkParams {
-    float g2[C];    // cumulative log2 decay at each row
-    float al[C];    // alpha_r (1 on padded rows)
-    float dblk[C];  // e^{g_(end of r's 16-row block) - g_r}
-    float eg[C];    // e^{g_r}
-    float bet[C];   // beta_r (0 on padded rows)
-    float egc[C];   // e^{g_C - g_r}
-    float egC;      // e^{g_C}
-    int Cv;         // valid rows
-    float pad[2];
-};
-constexpr uint32_t PAR_BYTES = (sizeof(ChunkParams) + 15) & ~15u;
-constexpr uint32_t OFF_BAR = OFF_PAR + 3 * PAR_BYTES;   // params ring of 3
-enum { B_FULL = 0, B_EMPTY = 2, B_KSREADY = 4, B_KSFREE = 6, B_G = 8, B_X = 10, B_D = 11, B_H = 12,
-       N_BARS = 13 };
-constexpr uint32_t OFF_MISC = OFF_BAR + N_BARS * 8;    // tmem slot, abort flag, group slots
-constexpr uint32_t SMEM_USED = OFF_MISC + 32;   // tmem slot, abort flag, 3 x 2 group slots
-constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;      // slack to align the base
-static_assert(SMEM_ALLOC <= 232448, "shared memory budget of one sm_100 block");
-
-// TMEM columns
-constexpr uint32_t TM_G0 = 0, TM_G1 = 64, TM_X0 = 128, TM_X1 = 192, TM_D = 256, TM_H = 320;
-constexpr uint32_t TM_COLS = 512;
+constexpr unsigned long long kWaitLimit = 4000000000ull;   // ~2 s at the boost clock
 
 // error codes recorded in g_tc_error (first one wins)
-enum { E_FULL = 1, E_EMPTY, E_KSREADY, E_KSFREE, E_GRAM, E_X, E_D, E_H };
+enum { E_FULL = 1, E_EMPTY, E_KSREADY, E_KSFREE, E_GRAM, E_UW, E_X, E_H, E_K1_TMA, E_K1_MMA };
 
-constexpr uint32_t IDESC_GRAM = idesc_f16(128, 64, 1, 1, 0, 0);   // bf16, K-major x K-major
-constexpr uint32_t IDESC_KB = idesc_f16(128, 64, 0, 0, 0, 1);     // fp16, K-major x MN-major
-constexpr uint32_t IDESC_MB = idesc_f16(128, 64, 0, 0, 1, 1);     // fp16, MN-major x MN-major
+constexpr uint32_t IDESC_BF_KK = idesc_f16(128, 64, 1, 1, 0, 0);    // bf16, K-major x K-major, N 64
+constexpr uint32_t IDESC_KM64 = idesc_f16(128, 64, 0, 0, 0, 1);     // fp16, K-major x MN-major, N 64
+constexpr uint32_t IDESC_KM128 = idesc_f16(128, 128, 0, 0, 0, 1);   // fp16, K-major x MN-major, N 128
+constexpr uint32_t IDESC_MM64 = idesc_f16(128, 64, 0, 0, 1, 1);     // fp16, MN-major x MN-major, N 64
 
-struct TcParams {
-    int B, T, H, dv;
+// =========================================================== key-side kernel
+
+constexpr int K1_THREADS = 256;
+constexpr uint32_t K1_OFF_K = 0;                       // K tile, two 64-column boxes
+constexpr uint32_t K1_OFF_LB = 16384;                  // L fp32 (also the rows after K's 2nd box)
+constexpr uint32_t K1_MAT = 64 * LSTR * 4;
+constexpr uint32_t K1_OFF_TB = K1_OFF_LB + K1_MAT;
+constexpr uint32_t K1_OFF_YB = K1_OFF_TB + K1_MAT;
+constexpr uint32_t K1_OFF_PAR = K1_OFF_YB + 8192;
+constexpr uint32_t K1_OFF_BAR = K1_OFF_PAR + ((sizeof(ChunkParams) + 15) & ~15u);
+constexpr uint32_t K1_SMEM = K1_OFF_BAR + 64 + 1024;  // + base alignment slack
+
+struct K1Params {
+    int B, T, H, NC;
+    const float *alpha, *beta;
+    __half *Tws;
+    int neumann, N;
+};
+
+__global__ void __launch_bounds__(K1_THREADS)
+keyside_kernel(const __grid_constant__ CUtensorMap tm_k, const K1Params p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    float *Lb = reinterpret_cast<float *>(sm + K1_OFF_LB);
+    float *Tb = reinterpret_cast<float *>(sm + K1_OFF_TB);
+    float *Yb = reinterpret_cast<float *>(sm + K1_OFF_YB);
+    ChunkParams *par = reinterpret_cast<ChunkParams *>(sm + K1_OFF_PAR);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + K1_OFF_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + K1_OFF_BAR + 16);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + K1_OFF_BAR + 20);
+
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncwarp();
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 64);
+        tmem_relinquish();
+    }
+    if (!p.neumann)
+        for (int i = tid; i < 64 * LSTR; i += K1_THREADS) Tb[i] = 0.f;
+    tc_fence_before();
+    block_sync();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int t0 = n * C;
+    if (tid == 0) {
+        tma_prefetch_desc(&tm_k);
+        mbar_arrive_expect_tx(&bars[0], 16384);
+        tma_load_4d(sm + K1_OFF_K, &tm_k, &bars[0], 0, h, t0, b);
+        tma_load_4d(sm + K1_OFF_K + 8192, &tm_k, &bars[0], 64, h, t0, b);
+    }
+    __syncwarp();
+    if (warp == 1) {
+        float a0, a1, b0, b1;
+        tc::fetch_gates(p.alpha, p.beta, b, p.T, p.H, h, t0, lane, true, a0, a1, b0, b1);
+        tc::scan_gates(par, a0, a1, b0, b1, lane, min(C, p.T - t0));
+    }
+    if (tid == 0) {
+        if (mbar_wait(&bars[0], 0, abort_flag, E_K1_TMA, kWaitLimit)) {
+            // [K ; next 64 rows] K^T: lanes 0..63 of the result hold K K^T
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(sm + K1_OFF_K);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
+                umma_f16_ss(tmem, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(a0 + off, 16, 1024),
+                            IDESC_BF_KK, kk > 0);
+            }
+            umma_commit(&bars[1]);
+            if (!mbar_wait(&bars[1], 0, abort_flag, E_K1_MMA, kWaitLimit))
+                mbar_wait_drain(&bars[1], 0, kWaitLimit);
+        } else {
+            mbar_wait_drain(&bars[0], 0, kWaitLimit);
+        }
+    }
+    __syncwarp();
+    block_sync();
+    const bool go = (*abort_flag == 0);
+    if (go) {
+        mbar_try_wait(&bars[1], 0);
+        tc_fence_after();
+        // L rows: TMEM lanes 0..63 (sub-partitions 0, 1), column half hf
+        const int sp = warp & 3, hf = warp >> 2;
+        if (sp < 2) {
+            const int r = 32 * sp + lane;
+            float *Lr = Lb + r * LSTR + 32 * hf;
+            if (hf > sp) {
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4 *>(Lr + j) = make_float4(0.f, 0.f, 0.f, 0.f);
+            } else {
+                uint32_t xr[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * sp) << 16) + 32 * hf, xr);
+                float gam[32];
+                tc::decay_row(par, r, hf, hf == sp, gam);
+                tmem_wait_ld();
+                const float br = par->bet[r];
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    const int i = 32 * hf + j;
+                    float4 v;
+                    v.x = (i + 0 < r) ? br * gam[j + 0] * __uint_as_float(xr[j + 0]) : 0.f;
+                    v.y = (i + 1 < r) ? br * gam[j + 1] * __uint_as_float(xr[j + 1]) : 0.f;
+                    v.z = (i + 2 < r) ? br * gam[j + 2] * __uint_as_float(xr[j + 2]) : 0.f;
+                    v.w = (i + 3 < r) ? br * gam[j + 3] * __uint_as_float(xr[j + 3]) : 0.f;
+                    *reinterpret_cast<float4 *>(Lr + j) = v;
+                }
+            }
+        }
+        tc_fence_before();
+        named_bar(1, K1_THREADS);
+        if (p.neumann) tc::invert_neumann(Lb, Tb, Yb, tid, p.N, 1);
+        else tc::invert_exact(Lb, Tb, Yb, tid, 1);
+        // T -> fp16, row-major [64][64] per chunk
+        {
+            const int r = tid >> 2, j0 = (tid & 3) * 2;
+            const size_t row = (((size_t)b * p.H + h) * p.NC + n) * 64 + r;
+            uint4 *dst = reinterpret_cast<uint4 *>(p.Tws + row * 64);
+            const float *Tr = Tb + r * LSTR;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int j = j0 + q;
+                const float4 a = *reinterpret_cast<const float4 *>(Tr + 8 * j);
+                const float4 c = *reinterpret_cast<const float4 *>(Tr + 8 * j + 4);
+                uint4 u;
+                u.x = pack_h2(a.x, a.y); u.y = pack_h2(a.z, a.w);
+                u.z = pack_h2(c.x, c.y); u.w = pack_h2(c.z, c.w);
+                dst[j] = u;
+            }
+        }
+    }
+    tc_fence_before();
+    block_sync();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 64);
+    }
+    if (tid == 0 && *abort_flag) atomicCAS(&g_tc_error, 0u, (unsigned)*abort_flag);
+}
+
+// ============================================================ chain kernel
+
+constexpr int K2_THREADS = 448;    // 14 warps
+constexpr int KS_THREADS = 256, CH_THREADS = 128;
+// stage (x2): per 64-column key block kb: [W | Q | K] at kb * 24 KB; V, T after
+constexpr uint32_t STG = 65536;
+constexpr uint32_t S_W = 0, S_Q = 8192, S_K = 16384, S_KB = 24576, S_V = 49152, S_T = 57344;
+constexpr uint32_t OFF_TBG = 2 * STG;                  // T diag(beta e^g)
+constexpr uint32_t OFF_P = OFF_TBG + 8192;             // P x 2 (P1's preceding rows are P0)
+constexpr uint32_t OFF_HS = OFF_P + 2 * 8192;          // h fp16, 128 rows
+constexpr uint32_t OFF_DS = OFF_HS + 16384;            // Delta fp16
+constexpr uint32_t OFF_DPS = OFF_DS + 8192;            // e^{g_C - g} Delta fp16
+constexpr uint32_t OFF_PAR = OFF_DPS + 8192;
+constexpr uint32_t PAR_BYTES = (sizeof(ChunkParams) + 15) & ~15u;
+constexpr uint32_t OFF_BAR = OFF_PAR + 3 * PAR_BYTES;   // params ring of 3
+enum { B_FULL = 0, B_EMPTY = 2, B_KSREADY = 4, B_KSFREE = 6, B_G = 8, B_UW = 9, B_X = 10, B_H = 11,
+       N_BARS = 12 };
+constexpr uint32_t OFF_MISC = OFF_BAR + N_BARS * 8;     // tmem slot, abort flag, group slots
+constexpr uint32_t SMEM_USED = OFF_MISC + 32;
+constexpr uint32_t K2_SMEM = SMEM_USED + 1024;
+static_assert(K2_SMEM <= 232448, "shared memory budget of one sm_100 block");
+static_assert(K1_SMEM * 3 <= 233472, "three key-side blocks per SM");
+
+// TMEM columns
+constexpr uint32_t TM_G = 0, TM_U0 = 64, TM_U1 = 128, TM_W = 192, TM_X0 = 320, TM_X1 = 384, TM_H = 448;
+constexpr uint32_t TM_COLS = 512;
+
+struct K2Params {
+    int B, T, H, dv, NC;
     const float *alpha, *beta, *S0;
     void *o;
     float *S_T;
-    int o_bf16, neumann, N;
-    unsigned long long limit_cycles;
+    int o_bf16;
 };
 
-__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
-    __half2 h = __floats2half2_rn(a, b);
-    return *reinterpret_cast<uint32_t *>(&h);
-}
-
-__device__ __forceinline__ float2 unpack_bf2(uint32_t u) {
-    __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162 *>(&u);
-    return __bfloat1622float2(h);
-}
-
-// Write 64 fp32 values as one fp16 row of a 128-byte swizzled tile.
-__device__ __forceinline__ void st_row_f16(uint8_t *tile, int r, const float *x) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        uint4 u;
-        u.x = pack_h2(x[8 * j + 0], x[8 * j + 1]);
-        u.y = pack_h2(x[8 * j + 2], x[8 * j + 3]);
-        u.z = pack_h2(x[8 * j + 4], x[8 * j + 5]);
-        u.w = pack_h2(x[8 * j + 6], x[8 * j + 7]);
-        *reinterpret_cast<uint4 *>(tile + sw128_off(r, j)) = u;
-    }
-}
-
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float *x) {
-    uint32_t a[32], b[32];
-    tmem_ld32(taddr, a);
-    tmem_ld32(taddr + 32, b);
-    tmem_wait_ld();
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        x[i] = __uint_as_float(a[i]);
-        x[32 + i] = __uint_as_float(b[i]);
-    }
-}
-
-__device__ __forceinline__ void tmem_st64(uint32_t taddr, const float *x) {
-    uint32_t a[32], b[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        a[i] = __float_as_uint(x[i]);
-        b[i] = __float_as_uint(x[32 + i]);
-    }
-    tmem_st32(taddr, a);
-    tmem_st32(taddr + 32, b);
-}
-
-__global__ void __launch_bounds__(kThreads, 1)
-tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const TcParams p) {
+__global__ void __launch_bounds__(K2_THREADS, 1)
+chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_t,
+             const K2Params p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base for the 128-byte swizzled tiles.  The offset is
     // applied to the __shared__ array itself so that every access below stays
@@ -172,40 +264,38 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int T = p.T, H = p.H, dv = p.dv;
+    const int T = p.T, H = p.H, dv = p.dv, NC = p.NC;
     const int v0 = slice * DVS;
-    const int NC = (T + C - 1) / C;
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC + 4);
-    // Named barrier that also broadcasts the abort state, so that every thread
-    // of a role leaves its loop at the same barrier (a failed wait can never
-    // strand the others at a bar.sync).  Two alternating slots per role.
-    const unsigned long long lim = p.limit_cycles;
-    // One thread of a role waits for the phase (sleeping), the others wait at
-    // the role's named barrier and then take the acquire with one test.
-    auto group_wait = [&](uint64_t *bar, uint32_t parity, int code, int id, int nthreads, bool leader,
-                          bool sleep = true) {
-        if (leader) {
+    ChunkParams *params = reinterpret_cast<ChunkParams *>(sm + OFF_PAR);
+    const unsigned long long lim = kWaitLimit;
+
+    // One warp of a group polls the phase (all its lanes, so the warp stays
+    // converged), the other warps wait at the group's named barrier and then
+    // take the acquire with one test.
+    auto group_wait = [&](uint64_t *bar, uint32_t parity, int code, int id, int nthreads, bool leader_warp,
+                          bool sleep) {
+        if (leader_warp) {
             if (sleep) mbar_wait(bar, parity, abort_flag, code, lim);
             else mbar_wait_spin(bar, parity, abort_flag, code, lim);
+            __syncwarp();
         }
         named_bar(id, nthreads);
-        if (!leader) mbar_try_wait(bar, parity);
+        if (!leader_warp) mbar_try_wait(bar, parity);
     };
+    // Named barrier that also broadcasts the abort state, so that every thread
+    // of a group leaves its loop at the same barrier.  Two slots per barrier id.
     auto sync_ok = [&](int id, int nthreads, bool leader, int &cnt) -> bool {
         volatile int *slots = reinterpret_cast<volatile int *>(sm + OFF_MISC + 8 + 8 * (id - 1));
         const int k = cnt++ & 1;
         if (leader) slots[k] = *abort_flag;
+        __syncwarp();
         named_bar(id, nthreads);
         return slots[k] == 0;
     };
-    ChunkParams *params = reinterpret_cast<ChunkParams *>(sm + OFF_PAR);
-    float *Lb = reinterpret_cast<float *>(sm + OFF_LB);
-    float *Tb = reinterpret_cast<float *>(sm + OFF_TB);
-    float *Yb = reinterpret_cast<float *>(sm + OFF_YB);
-    const uint32_t sbase = smem_u32(sm);
 
     // ------------------------------------------------------------- setup
     if (tid == 0) {
@@ -216,26 +306,19 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(&bars[B_KSFREE + i], 1);
         }
         mbar_init(&bars[B_G], 1);
-        mbar_init(&bars[B_G + 1], 1);
+        mbar_init(&bars[B_UW], 1);
         mbar_init(&bars[B_X], 1);
-        mbar_init(&bars[B_D], 1);
         mbar_init(&bars[B_H], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
+    __syncwarp();
     if (warp == 1) {
         tmem_alloc(tmem_slot, TM_COLS);
         tmem_relinquish();
     }
-    // zero blocks of the stacked operands, upper blocks of T
-    for (int i = tid; i < 2 * 8192 / 16; i += kThreads) {
-        const int buf = i / 512, off = (i % 512) * 16;
-        *reinterpret_cast<uint4 *>(sm + OFF_PZT + buf * PZT_BYTES + PZT_Z + off) = make_uint4(0, 0, 0, 0);
-    }
-    for (int i = tid; i < 64 * LSTR; i += kThreads) Tb[i] = 0.f;
-    fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    block_sync();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
@@ -245,132 +328,90 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
+            tma_prefetch_desc(&tm_t);
             int issued = 0;
             for (int m = 0; m < NC; ++m) {
                 const int s = m & 1;
                 if (m >= 2 && !mbar_wait(&bars[B_EMPTY + s], ((m - 2) >> 1) & 1, abort_flag, E_EMPTY, lim))
                     break;
                 uint64_t *fb = &bars[B_FULL + s];
-                mbar_arrive_expect_tx(fb, STAGE_BYTES);
-                uint8_t *st = sm + s * STAGE_BYTES;
+                mbar_arrive_expect_tx(fb, 49152);
+                uint8_t *st = sm + s * STG;
                 const int t0 = m * C;
-                tma_load_4d(st + ST_Q0, &tm_q, fb, 0, h, t0, b);
-                tma_load_4d(st + ST_Q1, &tm_q, fb, 64, h, t0, b);
-                tma_load_4d(st + ST_K0, &tm_k, fb, 0, h, t0, b);
-                tma_load_4d(st + ST_K1, &tm_k, fb, 64, h, t0, b);
-                tma_load_4d(st + ST_V, &tm_v, fb, v0, h, t0, b);
+                tma_load_4d(st + S_Q, &tm_q, fb, 0, h, t0, b);
+                tma_load_4d(st + S_KB + S_Q, &tm_q, fb, 64, h, t0, b);
+                tma_load_4d(st + S_K, &tm_k, fb, 0, h, t0, b);
+                tma_load_4d(st + S_KB + S_K, &tm_k, fb, 64, h, t0, b);
+                tma_load_4d(st + S_V, &tm_v, fb, v0, h, t0, b);
+                tma_load_4d(st + S_T, &tm_t, fb, 0, 0, (((b * H) + h) * NC + m) * 64, 0);
                 issued = m + 1;
             }
             // no copy may still be in flight when the block exits
             for (int m = issued - 2 < 0 ? 0 : issued - 2; m < issued; ++m)
                 mbar_wait_drain(&bars[B_FULL + (m & 1)], (m >> 1) & 1, lim);
         }
+        __syncwarp();
     } else if (warp >= 2 && warp < 10) {
         // ========================================================= key side
-        // 8 warps: two per TMEM sub-partition; warp half hf takes columns
-        // [32 hf, 32 hf + 32) of the Gram rows its sub-partition holds.
-        const int kt = tid - 64;                 // 0..255
+        // 8 warps, two per TMEM sub-partition; warp half hf takes columns
+        // [32 hf, 32 hf + 32) of the rows its sub-partition holds.
+        const int kt = tid - 64;                  // 0..255
         const int sp = warp & 3;
         const int hf = (warp - 2) >> 2;
-        const bool leader = (kt == 0);
-        const bool scan_warp = (kt >> 5) == 2;    // not used by the diagonal-block solve
-        float a_nx0 = 1.f, a_nx1 = 1.f, b_nx0 = 0.f, b_nx1 = 0.f;
-        auto fetch_gates = [&](int m) {
-            const int t0 = m * C;
-            const int r0 = lane, r1 = lane + 32;
-            const size_t i0 = ((size_t)b * T + t0 + r0) * H + h;
-            const size_t i1 = ((size_t)b * T + t0 + r1) * H + h;
-            const bool ok0 = (m < NC) && (t0 + r0 < T), ok1 = (m < NC) && (t0 + r1 < T);
-            a_nx0 = ok0 ? (p.alpha ? __ldg(p.alpha + i0) : 1.f) : 1.f;
-            a_nx1 = ok1 ? (p.alpha ? __ldg(p.alpha + i1) : 1.f) : 1.f;
-            b_nx0 = ok0 ? (p.beta ? __ldg(p.beta + i0) : 1.f) : 0.f;
-            b_nx1 = ok1 ? (p.beta ? __ldg(p.beta + i1) : 1.f) : 0.f;
-        };
-        // per-chunk gate scan into params[m % 3] (one warp, from prefetched gates)
-        auto scan_chunk = [&](int m) {
-            ChunkParams *par = &params[m % 3];
-            const float x0i = lg2_approx(a_nx0), x1i = lg2_approx(a_nx1);
-            float x0 = x0i, x1 = x1i;
-            const float be0 = b_nx0, be1 = b_nx1, al0 = a_nx0, al1 = a_nx1;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y0 = __shfl_up_sync(0xffffffffu, x0, o);
-                const float y1 = __shfl_up_sync(0xffffffffu, x1, o);
-                if (lane >= o) { x0 += y0; x1 += y1; }
-            }
-            x1 += __shfl_sync(0xffffffffu, x0, 31);
-            const float gC = __shfl_sync(0xffffffffu, x1, 31);
-            // cumulative decay at the last row of each row's 16-row block
-            const float e0 = __shfl_sync(0xffffffffu, x0, lane | 15);
-            const float e1 = __shfl_sync(0xffffffffu, x1, lane | 15);
-            par->g2[lane] = x0;
-            par->g2[lane + 32] = x1;
-            par->al[lane] = al0;
-            par->al[lane + 32] = al1;
-            par->dblk[lane] = ex2_approx(e0 - x0);
-            par->dblk[lane + 32] = ex2_approx(e1 - x1);
-            par->eg[lane] = ex2_approx(x0);
-            par->eg[lane + 32] = ex2_approx(x1);
-            par->egc[lane] = ex2_approx(gC - x0);
-            par->egc[lane + 32] = ex2_approx(gC - x1);
-            par->bet[lane] = be0;
-            par->bet[lane + 32] = be1;
-            if (lane == 0) {
-                par->egC = ex2_approx(gC);
-                par->Cv = min(C, T - m * C);
-            }
-            fetch_gates(m + 1);
-        };
+        const bool leader = (kt == 0);           // MMA issue and flag writes
+        const bool lwarp = (kt >> 5) == 0;        // polls the group's waits
+        const bool scan_warp = (kt >> 5) == 2;
+        float ga0 = 1.f, ga1 = 1.f, gb0 = 0.f, gb1 = 0.f;
         if (scan_warp) {
-            fetch_gates(0);
-            scan_chunk(0);
+            tc::fetch_gates(p.alpha, p.beta, b, T, H, h, 0, lane, true, ga0, ga1, gb0, gb1);
+            tc::scan_gates(&params[0], ga0, ga1, gb0, gb1, lane, min(C, T));
+            tc::fetch_gates(p.alpha, p.beta, b, T, H, h, C, lane, NC > 1, ga0, ga1, gb0, gb1);
         }
-        uint32_t pk[16];        // this thread's half row of P, fp16 pairs (sub-partitions 0, 1)
         int kcnt = 0;
-        int gram_next = 0;      // leader: first chunk whose Gram is not issued yet
-        int gram_pend = -1;     // leader: chunk of the last issued Gram (for the error-path drain)
-        auto issue_gram = [&](int m) {
-            uint8_t *stg = sm + (m & 1) * STAGE_BYTES;
-            tc_fence_after();
-            const uint32_t a0 = smem_u32(stg);
-            const uint32_t dst = tmem + ((m & 1) ? TM_G1 : TM_G0);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                umma_f16_ss(dst, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(a0 + off + 8192, 16, 1024),
-                            IDESC_GRAM, kk > 0);
-            }
-            umma_commit(&bars[B_G + (m & 1)]);
-            gram_pend = m;
-            gram_next = m + 1;
-        };
-        // leader: issue the next chunk's Gram early if its tiles have landed
-        auto try_prefetch_gram = [&](int m) {
-            if (leader && gram_next == m + 1 && m + 1 < NC &&
-                mbar_try_wait(&bars[B_FULL + ((m + 1) & 1)], ((m + 1) >> 1) & 1))
-                issue_gram(m + 1);
-        };
+        int pend = -1;   // leader: barrier of the last commit not yet known complete
+        int pend_par = 0;
         for (int m = 0; m < NC; ++m) {
             const int s = m & 1;
-            ChunkParams *par = &params[m % 3];
-            uint8_t *st = sm + s * STAGE_BYTES;
-            uint8_t *pzt = sm + OFF_PZT + s * PZT_BYTES;
-            // chain finished chunk m-2: params[(m+1) % 3] and [P|Z|T][s] are free
-            if (m >= 2) group_wait(&bars[B_KSFREE + s], ((m - 2) >> 1) & 1, E_KSFREE, 1, kKsThreads, leader);
-            group_wait(&bars[B_FULL + s], (m >> 1) & 1, E_FULL, 1, kKsThreads, leader);
-            // params written; previous reads of the Gram TMEM done
-            if (!sync_ok(1, kKsThreads, leader, kcnt)) break;
-            if (leader && gram_next == m) issue_gram(m);
-            group_wait(&bars[B_G + s], (m >> 1) & 1, E_GRAM, 1, kKsThreads, leader);
-            if (!sync_ok(1, kKsThreads, leader, kcnt)) break;
-            tc_fence_after();
-            // in-place fp16 conversion of the MMA operands: Q -> e^{g_r} Q, K -> K
+            const ChunkParams *par = &params[m % 3];
+            uint8_t *st = sm + s * STG;
+            uint8_t *P = sm + OFF_P + s * 8192;
+            uint8_t *tbg = sm + OFF_TBG;
+            // chain finished chunk m-2: its P buffer, U buffer and W slots are free
+            if (m >= 2) group_wait(&bars[B_KSFREE + s], ((m - 2) >> 1) & 1, E_KSFREE, 1, KS_THREADS, lwarp, true);
+            group_wait(&bars[B_FULL + s], (m >> 1) & 1, E_FULL, 1, KS_THREADS, lwarp, true);
+            if (!sync_ok(1, KS_THREADS, leader, kcnt)) break;
+            if (leader) {
+                // [Q ; K] K^T: lanes 0..63 of the result hold Q K^T
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(st);
 #pragma unroll
-            for (int it = 0; it < 8; ++it) {
-                const int u = kt + 256 * (it & 1);             // chunk within one 8 KB tile
-                const int tile = it >> 1;                      // Q0, Q1, K0, K1
-                uint8_t *addr = st + (tile == 0 ? ST_Q0 : tile == 1 ? ST_Q1 : tile == 2 ? ST_K0 : ST_K1) + (u << 4);
-                const float sc = tile < 2 ? par->eg[u >> 3] : 1.f;
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * S_KB + (kk & 3) * 32;
+                    umma_f16_ss(tmem + TM_G, sdesc_sw128(a0 + S_Q + off, 16, 1024),
+                                sdesc_sw128(a0 + S_K + off, 16, 1024), IDESC_BF_KK, kk > 0);
+                }
+                umma_commit(&bars[B_G]);
+                pend = B_G; pend_par = m & 1;
+            }
+            __syncwarp();
+            // gates of the next chunk meanwhile
+            if (scan_warp && m + 1 < NC) {
+                tc::scan_gates(&params[(m + 1) % 3], ga0, ga1, gb0, gb1, lane, min(C, T - (m + 1) * C));
+                tc::fetch_gates(p.alpha, p.beta, b, T, H, h, (m + 2) * C, lane, m + 2 < NC, ga0, ga1, gb0, gb1);
+            }
+            group_wait(&bars[B_G], m & 1, E_GRAM, 1, KS_THREADS, lwarp, false);
+            if (!sync_ok(1, KS_THREADS, leader, kcnt)) break;
+            tc_fence_after();
+            // in-place fp16 operands: Q -> e^{g_r} Q, K -> K, V -> beta_r V
+#pragma unroll
+            for (int it = 0; it < 10; ++it) {
+                const int u = kt + 256 * (it & 1);          // 16-byte chunk within one 8 KB tile
+                const int tile = it >> 1;                   // Q0, Q1, K0, K1, V
+                const uint32_t off = tile == 0 ? S_Q : tile == 1 ? S_KB + S_Q : tile == 2 ? S_K
+                                   : tile == 3 ? S_KB + S_K : S_V;
+                uint8_t *addr = st + off + (u << 4);
+                const int row = u >> 3;
+                const float sc = tile < 2 ? par->eg[row] : (tile == 4 ? par->bet[row] : 1.f);
                 uint4 w = *reinterpret_cast<uint4 *>(addr);
                 const float2 f0 = unpack_bf2(w.x), f1 = unpack_bf2(w.y), f2 = unpack_bf2(w.z), f3 = unpack_bf2(w.w);
                 w.x = pack_h2(f0.x * sc, f0.y * sc);
@@ -379,232 +420,100 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 w.w = pack_h2(f3.x * sc, f3.y * sc);
                 *reinterpret_cast<uint4 *>(addr) = w;
             }
-            // Gram rows: sub-partitions 0,1 hold Q K^T (-> P), 2,3 hold K K^T (-> L).
-            // This warp's 32 x 32 tile: rows 32 (sp & 1) .., columns 32 hf ..
-            // Decay factors exp(g_r - g_i) without per-element exponentials:
-            // 16-blocks left of r's block as e^{g_r - g_blockend} * dblk[i],
-            // r's own block as a running product of alpha.
-            {
-                const int rh = sp & 1;                       // row half (warp-uniform)
-                const int r = 32 * rh + lane;
-                const bool is_p = sp < 2;
-                if (hf > rh) {
-                    // strictly above the diagonal: zero
-                    if (is_p) {
+            if (sp < 2) {
+                // P rows (TMEM lanes 0..63): decayed causal scores
+                const int r = 32 * sp + lane;
+                uint32_t pk[16];
+                if (hf > sp) {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) pk[j] = 0u;
-                    } else {
-                        float *Lr = Lb + r * LSTR + 32 * hf;
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4 *>(Lr + j) = make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
+                    for (int j = 0; j < 16; ++j) pk[j] = 0u;
                 } else {
                     uint32_t xr[32];
-                    tmem_ld32(tmem + ((uint32_t)(32 * sp) << 16) + (s ? TM_G1 : TM_G0) + 32 * hf, xr);
-                    const float gr = par->g2[r];
+                    tmem_ld32(tmem + ((uint32_t)(32 * sp) << 16) + TM_G + 32 * hf, xr);
                     float gam[32];
-                    if (hf < rh) {
-                        const float E0 = ex2_approx(gr - par->g2[32 * hf + 15]);
-                        const float E1 = ex2_approx(gr - par->g2[32 * hf + 31]);
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) gam[j] = (j < 16 ? E0 : E1) * par->dblk[32 * hf + j];
-                    } else {
-                        const int br = r >> 4;
-#pragma unroll
-                        for (int bb = 0; bb < 2; ++bb) {
-                            const int blk = 2 * hf + bb;
-                            const float E = ex2_approx(gr - par->g2[16 * blk + 15]);
-                            float c = 1.f;
-#pragma unroll
-                            for (int ii = 15; ii >= 0; --ii) {
-                                const int i = 16 * blk + ii;
-                                const float chain = (i <= r) ? c : 0.f;
-                                c = (i <= r) ? c * par->al[i] : c;
-                                gam[16 * bb + ii] = (blk < br) ? E * par->dblk[i] : ((blk == br) ? chain : 0.f);
-                            }
-                        }
-                    }
+                    tc::decay_row(par, r, hf, hf == sp, gam);
                     tmem_wait_ld();
-                    if (is_p) {
 #pragma unroll
-                        for (int j = 0; j < 32; j += 2)
-                            pk[j >> 1] = pack_h2(gam[j] * __uint_as_float(xr[j]), gam[j + 1] * __uint_as_float(xr[j + 1]));
-                    } else {
-                        const float br_ = par->bet[r];
-                        float *Lr = Lb + r * LSTR + 32 * hf;
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            const int i = 32 * hf + j;
-                            float4 v;
-                            v.x = (i + 0 < r) ? br_ * gam[j + 0] * __uint_as_float(xr[j + 0]) : 0.f;
-                            v.y = (i + 1 < r) ? br_ * gam[j + 1] * __uint_as_float(xr[j + 1]) : 0.f;
-                            v.z = (i + 2 < r) ? br_ * gam[j + 2] * __uint_as_float(xr[j + 2]) : 0.f;
-                            v.w = (i + 3 < r) ? br_ * gam[j + 3] * __uint_as_float(xr[j + 3]) : 0.f;
-                            *reinterpret_cast<float4 *>(Lr + j) = v;
-                        }
-                    }
+                    for (int j = 0; j < 32; j += 2)
+                        pk[j >> 1] = pack_h2(gam[j] * __uint_as_float(xr[j]), gam[j + 1] * __uint_as_float(xr[j + 1]));
                 }
-            }
-            tc_fence_before();
-            named_bar(1, kKsThreads);  // L complete, Gram buffer s read
-            try_prefetch_gram(m);
-            // gates of the next chunk, overlapping the diagonal-block solve
-            if (scan_warp && m + 1 < NC) scan_chunk(m + 1);
-            // ------------------------------------------------ T = (I + L)^-1
-            if (!p.neumann) {
-                if (kt < 64) {
-                    // 16 x 16 diagonal blocks by forward substitution, one column per
-                    // thread; each solved entry updates the rows below it at once
-                    const int c = kt, base = c & ~15, jc = c & 15;
-                    float acc[16];
 #pragma unroll
-                    for (int r = 0; r < 16; ++r) acc[r] = (r == jc) ? 1.f : 0.f;
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float xi = acc[i];
-#pragma unroll
-                        for (int r = i + 1; r < 16; ++r) acc[r] -= Lb[(base + r) * LSTR + base + i] * xi;
-                    }
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) Tb[(base + r) * LSTR + c] = acc[r];
-                }
-                named_bar(1, kKsThreads);
-                // 16 -> 32: T_{b1 b0} = -T_{b1 b1} (L_{b1 b0} T_{b0 b0}) for both 32-blocks;
-                // two adjacent columns per thread
-                {
-                    const int pr = kt >> 7, rr = (kt >> 3) & 15, c0 = (kt & 7) * 2;
-                    const int b0 = 32 * pr, b1 = b0 + 16;
-                    float y0 = 0.f, y1 = 0.f;
-                    const float *Lr = Lb + (b1 + rr) * LSTR + b0;
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const float l = Lr[k];
-                        const float2 t = *reinterpret_cast<const float2 *>(Tb + (b0 + k) * LSTR + b0 + c0);
-                        y0 += l * t.x; y1 += l * t.y;
-                    }
-                    *reinterpret_cast<float2 *>(Yb + pr * 256 + rr * 16 + c0) = make_float2(y0, y1);
-                    named_bar(1, kKsThreads);
-                    float z0 = 0.f, z1 = 0.f;
-                    const float *Tr = Tb + (b1 + rr) * LSTR + b1;
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const float t = Tr[k];   // T_{b1 b1} is lower triangular, zeros above
-                        const float2 yy = *reinterpret_cast<const float2 *>(Yb + pr * 256 + k * 16 + c0);
-                        z0 += t * yy.x; z1 += t * yy.y;
-                    }
-                    *reinterpret_cast<float2 *>(Tb + (b1 + rr) * LSTR + b0 + c0) = make_float2(-z0, -z1);
-                }
-                named_bar(1, kKsThreads);
-                // 32 -> 64: T_{10} = -T_{11} (L_{10} T_{00}) with 32 x 32 blocks.  The
-                // triangular factors make the work per output uneven; each thread
-                // takes two output pairs whose work sums to about the same.
-                {
-                    const int rr = kt >> 3, q = kt & 7;          // row of L_10, column pair group
-                    const int ca = 2 * q, cb = 30 - 2 * q;       // column pairs (ca, ca+1), (cb, cb+1)
-                    float ya0 = 0.f, ya1 = 0.f, yb0 = 0.f, yb1 = 0.f;
-                    const float *Lr = Lb + (32 + rr) * LSTR;
-                    for (int k = ca; k < 32; ++k) {
-                        const float l = Lr[k];
-                        const float2 t = *reinterpret_cast<const float2 *>(Tb + k * LSTR + ca);
-                        ya0 += l * t.x; ya1 += l * t.y;
-                    }
-                    for (int k = cb; k < 32; ++k) {
-                        const float l = Lr[k];
-                        const float2 t = *reinterpret_cast<const float2 *>(Tb + k * LSTR + cb);
-                        yb0 += l * t.x; yb1 += l * t.y;
-                    }
-                    *reinterpret_cast<float2 *>(Yb + rr * 32 + ca) = make_float2(ya0, ya1);
-                    *reinterpret_cast<float2 *>(Yb + rr * 32 + cb) = make_float2(yb0, yb1);
-                    named_bar(1, kKsThreads);
-                    // rows (ra, rb) = (p, 31 - p) pair up the triangular sums k <= row
-                    const int pp = kt >> 4, cq = (kt & 15) * 2;
-                    const int ra = pp, rb = 31 - pp;
-                    float za0 = 0.f, za1 = 0.f, zb0 = 0.f, zb1 = 0.f;
-                    const float *Ta = Tb + (32 + ra) * LSTR + 32;
-                    const float *Tbr = Tb + (32 + rb) * LSTR + 32;
-                    for (int k = 0; k <= ra; ++k) {
-                        const float t = Ta[k];
-                        const float2 yy = *reinterpret_cast<const float2 *>(Yb + k * 32 + cq);
-                        za0 += t * yy.x; za1 += t * yy.y;
-                    }
-                    for (int k = 0; k <= rb; ++k) {
-                        const float t = Tbr[k];
-                        const float2 yy = *reinterpret_cast<const float2 *>(Yb + k * 32 + cq);
-                        zb0 += t * yy.x; zb1 += t * yy.y;
-                    }
-                    *reinterpret_cast<float2 *>(Tb + (32 + ra) * LSTR + cq) = make_float2(-za0, -za1);
-                    *reinterpret_cast<float2 *>(Tb + (32 + rb) * LSTR + cq) = make_float2(-zb0, -zb1);
-                }
+                for (int jj = 0; jj < 4; ++jj)
+                    *reinterpret_cast<uint4 *>(P + sw128_off(r, 4 * hf + jj)) =
+                        make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
             } else {
-                // masked Neumann series by Horner's rule on the band (A = -L):
-                // T^(0) = I, T^(s)_ij = [i-j <= N] (delta_ij - sum_k L_ik T^(s-1)_kj).
-                // band rows are 16 wide: band[i*16 + d] = T_{i, i-d}, d <= N <= 15;
-                // thread (i, dq) owns diagonals dq, dq+4, dq+8, dq+12 of row i
-                const int N = p.N;
-                const int i = kt >> 2, dq = kt & 3;
-                float *cur = Yb, *nxt = Yb + 1024;
+                // T diag(beta e^g): the 128 threads of sub-partitions 2, 3 (warps 2, 3,
+                // 6, 7), 4 chunks each, same swizzled positions
+                const int t2 = 64 * hf + 32 * (sp - 2) + lane;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) cur[i * 16 + dq + 4 * u] = (dq + 4 * u == 0) ? 1.f : 0.f;
-                named_bar(1, kKsThreads);
-                for (int step = 0; step < N; ++step) {
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int d = dq + 4 * u, j = i - d;
-                        float val = 0.f;
-                        if (j >= 0 && d <= N) {
-                            val = (d == 0) ? 1.f : 0.f;
-                            // k from j to i-1; T_kj is in the band while k - j <= N
-                            for (int k = j; k < i; ++k) val -= Lb[i * LSTR + k] * cur[k * 16 + (k - j)];
-                        }
-                        nxt[i * 16 + d] = val;
-                    }
-                    named_bar(1, kKsThreads);
-                    float *sw = cur; cur = nxt; nxt = sw;
-                }
-#pragma unroll 4
-                for (int qq = 0; qq < 16; ++qq) {
-                    const int e = kt + 256 * qq, ii = e >> 6, j = e & 63, d = ii - j;
-                    Tb[ii * LSTR + j] = (d >= 0 && d <= N) ? cur[ii * 16 + d] : 0.f;
-                }
-            }
-            named_bar(1, kKsThreads);  // T complete
-            try_prefetch_gram(m);
-            // ------------------------------------------ T and P to fp16 operands
-            {
-                const int r = kt >> 2, j0 = (kt & 3) * 2;
-                const float *Tr = Tb + r * LSTR;
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int j = j0 + q;
-                    const float4 a = *reinterpret_cast<const float4 *>(Tr + 8 * j);
-                    const float4 c = *reinterpret_cast<const float4 *>(Tr + 8 * j + 4);
-                    uint4 u;
-                    u.x = pack_h2(a.x, a.y); u.y = pack_h2(a.z, a.w);
-                    u.z = pack_h2(c.x, c.y); u.w = pack_h2(c.z, c.w);
-                    *reinterpret_cast<uint4 *>(pzt + PZT_T + sw128_off(r, j)) = u;
-                }
-                if (sp < 2) {
-                    const int rp = 32 * sp + lane;
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj)
-                        *reinterpret_cast<uint4 *>(pzt + sw128_off(rp, 4 * hf + jj)) =
-                            make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
+                for (int q = 0; q < 4; ++q) {
+                    const int cidx = t2 + 128 * q, r = cidx >> 3, jp = cidx & 7;
+                    const int j = jp ^ (r & 7);                 // logical 8-column group
+                    const uint32_t off = (uint32_t)(r * 128 + jp * 16);
+                    uint4 w = *reinterpret_cast<const uint4 *>(st + S_T + off);
+                    const float2 f0 = unpack_h2(w.x), f1 = unpack_h2(w.y), f2 = unpack_h2(w.z), f3 = unpack_h2(w.w);
+                    const int c0 = 8 * j;
+                    w.x = pack_h2(f0.x * par->bet[c0 + 0] * par->eg[c0 + 0], f0.y * par->bet[c0 + 1] * par->eg[c0 + 1]);
+                    w.y = pack_h2(f1.x * par->bet[c0 + 2] * par->eg[c0 + 2], f1.y * par->bet[c0 + 3] * par->eg[c0 + 3]);
+                    w.z = pack_h2(f2.x * par->bet[c0 + 4] * par->eg[c0 + 4], f2.y * par->bet[c0 + 5] * par->eg[c0 + 5]);
+                    w.w = pack_h2(f3.x * par->bet[c0 + 6] * par->eg[c0 + 6], f3.y * par->bet[c0 + 7] * par->eg[c0 + 7]);
+                    *reinterpret_cast<uint4 *>(tbg + off) = w;
                 }
             }
             fence_proxy_async_smem();
-            named_bar(1, kKsThreads);
-            if (leader) mbar_arrive(&bars[B_KSREADY + s]);
+            tc_fence_before();
+            if (!sync_ok(1, KS_THREADS, leader, kcnt)) break;
+            if (leader) {
+                tc_fence_after();
+                const uint32_t at = smem_u32(st + S_T), av = smem_u32(st + S_V);
+                const uint32_t ag = smem_u32(tbg), ak = smem_u32(st + S_K);
+                const uint32_t du = tmem + (s ? TM_U1 : TM_U0);
+                // U = T (beta V): [T ; next rows] x V (MN-major), K = 64 tokens
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16_ss(du, sdesc_sw128(at + kk * 32, 16, 1024),
+                                sdesc_sw128(av + kk * 2048, 8192, 1024), IDESC_KM64, kk > 0);
+                // W = T diag(beta e^g) K: K as MN-major B with N = 128 (two key blocks)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16_ss(tmem + TM_W, sdesc_sw128(ag + kk * 32, 16, 1024),
+                                sdesc_sw128(ak + kk * 2048, S_KB, 1024), IDESC_KM128, kk > 0);
+                umma_commit(&bars[B_UW]);
+                pend = B_UW; pend_par = m & 1;
+            }
+            __syncwarp();
+            group_wait(&bars[B_UW], m & 1, E_UW, 1, KS_THREADS, lwarp, false);
+            if (!sync_ok(1, KS_THREADS, leader, kcnt)) break;
+            tc_fence_after();
+            if (sp < 2) {
+                // -W rows (TMEM lanes 0..63) -> fp16 into the W slot of key block hf
+                const int r = 32 * sp + lane;
+                float x[64];
+                tmem_ld64(tmem + ((uint32_t)(32 * sp) << 16) + TM_W + 64 * hf, x);
+#pragma unroll
+                for (int j = 0; j < 64; ++j) x[j] = -x[j];
+                st_row_f16(st + hf * S_KB + S_W, r, x);
+            }
+            fence_proxy_async_smem();
+            named_bar(1, KS_THREADS);
+            if (leader) {
+                pend = -1;
+                mbar_arrive(&bars[B_KSREADY + s]);
+            }
+            __syncwarp();
         }
-        if (leader && gram_pend >= 0 && *abort_flag)
-            mbar_wait_drain(&bars[B_G + (gram_pend & 1)], (gram_pend >> 1) & 1, lim);
+        if (leader && pend >= 0 && *abort_flag) mbar_wait_drain(&bars[pend], pend_par, lim);
+        __syncwarp();
     } else if (warp >= 10) {
         // ========================================================= state chain
         const int ct = tid - 320;          // 0..127
         const int sp = warp & 3;
         const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
-        const int hrow = 32 * sp + lane;   // dk row of h held by this thread
+        const int hrow = 32 * sp + lane;   // key row of h held by this thread
+        const bool rowpart = (sp < 2);     // Delta rows live in TMEM lanes 0..63
+        const bool issuer = (ct == 64);    // warp 12 lane 0, sub-partition 0: MMA issue
+        const bool iwarp = (ct >> 5) == 2; // warp 12 polls the chain's waits
         uint8_t *hs = sm + OFF_HS;
-        uint8_t *rs = sm + OFF_RS;
         uint8_t *ds = sm + OFF_DS;
         uint8_t *dps = sm + OFF_DPS;
         const size_t bh = (size_t)b * H + h;
@@ -616,12 +525,18 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (p.S0) v = *reinterpret_cast<const float4 *>(p.S0 + (bh * DK + hrow) * dv + v0 + j);
                 x[j] = v.x; x[j + 1] = v.y; x[j + 2] = v.z; x[j + 3] = v.w;
             }
-            tmem_st64(tmem + lane_base + TM_H, x);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t y[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) y[j] = __float_as_uint(x[32 * hh + j]);
+                tmem_st32(tmem + lane_base + TM_H + 32 * hh, y);
+            }
             tmem_wait_st();
         }
         auto store_o = [&](int n) {
-            // rows of O for chunk n live in TMEM lanes 0..63 of the X buffer
-            const int r = 32 * sp + lane;
+            // O rows of chunk n: TMEM lanes 64..127 of its X buffer
+            const int r = 32 * (sp - 2) + lane;
             float x[64];
             tmem_ld64(tmem + lane_base + ((n & 1) ? TM_X1 : TM_X0), x);
             const int t = n * C + r;
@@ -651,19 +566,16 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         };
         int ccnt = 0, dcnt = 0;
-        // issuer only: barrier index and parity of the last commit not yet known complete
-        int pend_bar = -1, pend_par = 0;
-        const bool issuer = (ct == 0);        // warp 10, sub-partition 2
-        const bool rowpart = (sp >= 2);       // R and Delta rows live in TMEM lanes 64..127
+        int pend = -1, pend_par = 0;       // issuer: last commit not yet known complete
         bool done = true;
         for (int n = 0; n < NC; ++n) {
             const int s = n & 1;
             const ChunkParams *par = &params[n % 3];
-            uint8_t *st = sm + s * STAGE_BYTES;
-            uint8_t *pzt = sm + OFF_PZT + s * PZT_BYTES;
-            const uint32_t tx = tmem + (s ? TM_X1 : TM_X0);
-            group_wait(&bars[B_KSREADY + s], (n >> 1) & 1, E_KSREADY, 2, kChThreads, issuer, true);
-            if (n > 0) group_wait(&bars[B_H], (n - 1) & 1, E_H, 2, kChThreads, issuer, false);
+            uint8_t *st = sm + s * STG;
+            uint8_t *P = sm + OFF_P + s * 8192;
+            const uint32_t xcol = s ? TM_X1 : TM_X0;
+            group_wait(&bars[B_KSREADY + s], (n >> 1) & 1, E_KSREADY, 2, CH_THREADS, iwarp, true);
+            if (n > 0) group_wait(&bars[B_H], (n - 1) & 1, E_H, 2, CH_THREADS, iwarp, false);
             tc_fence_after();
             // ---- h <- e^{g_C} h in TMEM (issued first), h -> fp16 operand
             {
@@ -682,69 +594,36 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            if (!sync_ok(2, kChThreads, issuer, ccnt)) { done = false; break; }
+            if (!sync_ok(2, CH_THREADS, issuer, ccnt)) { done = false; break; }
             if (issuer) {
+                // [-W ; Q'] h16: lanes 0..63 -W h, lanes 64..127 Q'h
                 tc_fence_after();
                 const uint32_t a0 = smem_u32(st), b0 = smem_u32(hs);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    umma_f16_ss(tx, sdesc_sw128(a0 + aoff, 16, 1024),
-                                sdesc_sw128(b0 + kk * 2048, 8192, 1024), IDESC_KB, kk > 0);
+                    const uint32_t aoff = (kk >> 2) * S_KB + (kk & 3) * 32;
+                    umma_f16_ss(tmem + xcol, sdesc_sw128(a0 + S_W + aoff, 16, 1024),
+                                sdesc_sw128(b0 + kk * 2048, 8192, 1024), IDESC_KM64, kk > 0);
                 }
                 umma_commit(&bars[B_X]);
-                pend_bar = B_X; pend_par = n & 1;
+                pend = B_X; pend_par = n & 1;
             }
+            __syncwarp();
             if (!rowpart) {
-                // sub-partitions 0, 1: output rows of the previous chunk, off the chain
+                // sub-partitions 2, 3: output rows of the previous chunk, off the chain
                 if (n > 0) store_o(n - 1);
                 continue;
             }
-            group_wait(&bars[B_X], n & 1, E_X, 3, 64, issuer, false);
+            group_wait(&bars[B_X], n & 1, E_X, 3, 64, iwarp, false);
             tc_fence_after();
-            // ---- R = beta (v - e^g K h), rows in lanes 64..127
+            // ---- Delta = U - W h (rows in lanes 0..63) -> fp16 operands
             {
-                const int r = 32 * (sp - 2) + lane;
-                float x[64];
-                tmem_ld64(tmem + lane_base + (s ? TM_X1 : TM_X0), x);
-                const float br = par->bet[r], er = par->eg[r];
-                const uint8_t *vrow = st + ST_V;
+                const int r = 32 * sp + lane;
+                float x[64], u[64];
+                tmem_ld64(tmem + lane_base + xcol, x);
+                tmem_ld64(tmem + lane_base + (s ? TM_U1 : TM_U0), u);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint4 w = *reinterpret_cast<const uint4 *>(vrow + sw128_off(r, j));
-                    const float2 f0 = unpack_bf2(w.x), f1 = unpack_bf2(w.y), f2 = unpack_bf2(w.z), f3 = unpack_bf2(w.w);
-                    x[8 * j + 0] = br * (f0.x - er * x[8 * j + 0]);
-                    x[8 * j + 1] = br * (f0.y - er * x[8 * j + 1]);
-                    x[8 * j + 2] = br * (f1.x - er * x[8 * j + 2]);
-                    x[8 * j + 3] = br * (f1.y - er * x[8 * j + 3]);
-                    x[8 * j + 4] = br * (f2.x - er * x[8 * j + 4]);
-                    x[8 * j + 5] = br * (f2.y - er * x[8 * j + 5]);
-                    x[8 * j + 6] = br * (f3.x - er * x[8 * j + 6]);
-                    x[8 * j + 7] = br * (f3.y - er * x[8 * j + 7]);
-                }
-                st_row_f16(rs, r, x);
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            // 64-thread barrier of sub-partitions 2, 3; an abort here only stops the
-            // MMAs, the loop exits at the next 128-thread barrier
-            if (sync_ok(3, 64, issuer, dcnt) && issuer) {
-                tc_fence_after();
-                const uint32_t a0 = smem_u32(pzt + PZT_Z), b0 = smem_u32(rs);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16_ss(tmem + TM_D, sdesc_sw128(a0 + kk * 32, 16, 1024),
-                                sdesc_sw128(b0 + kk * 2048, 8192, 1024), IDESC_KB, kk > 0);
-                umma_commit(&bars[B_D]);
-                pend_bar = B_D; pend_par = n & 1;
-            }
-            group_wait(&bars[B_D], n & 1, E_D, 3, 64, issuer, false);
-            tc_fence_after();
-            // ---- Delta (rows in lanes 64..127) -> fp16 operands
-            {
-                const int r = 32 * (sp - 2) + lane;
-                float x[64];
-                tmem_ld64(tmem + lane_base + TM_D, x);
+                for (int j = 0; j < 64; ++j) x[j] += u[j];
                 st_row_f16(ds, r, x);
                 const float ec = par->egc[r];
 #pragma unroll
@@ -753,28 +632,33 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             fence_proxy_async_smem();
             tc_fence_before();
+            // 64-thread barrier of sub-partitions 0, 1; an abort here only stops the
+            // MMAs, the loop exits at the next 128-thread barrier
             if (sync_ok(3, 64, issuer, dcnt) && issuer) {
                 tc_fence_after();
-                const uint32_t ap = smem_u32(pzt), bd = smem_u32(ds);
-                const uint32_t ak = smem_u32(st + ST_K0), bdp = smem_u32(dps);
+                const uint32_t ap = smem_u32(P) - 8192, bd = smem_u32(ds);
+                const uint32_t ak = smem_u32(st + S_K), bdp = smem_u32(dps);
+                // O: [preceding rows ; P] Delta -> lanes 64..127 += P Delta
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_f16_ss(tx, sdesc_sw128(ap + kk * 32, 16, 1024),
-                                sdesc_sw128(bd + kk * 2048, 8192, 1024), IDESC_KB, 1);
+                    umma_f16_ss(tmem + xcol, sdesc_sw128(ap + kk * 32, 16, 1024),
+                                sdesc_sw128(bd + kk * 2048, 8192, 1024), IDESC_KM64, 1);
+                // h += K^T (e^{g_C - g} Delta): K^T as MN-major A over the two key blocks
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_f16_ss(tmem + TM_H, sdesc_sw128(ak + kk * 2048, 16384, 1024),
-                                sdesc_sw128(bdp + kk * 2048, 8192, 1024), IDESC_MB, 1);
+                    umma_f16_ss(tmem + TM_H, sdesc_sw128(ak + kk * 2048, S_KB, 1024),
+                                sdesc_sw128(bdp + kk * 2048, 8192, 1024), IDESC_MM64, 1);
                 umma_commit(&bars[B_EMPTY + s]);
                 umma_commit(&bars[B_KSFREE + s]);
                 umma_commit(&bars[B_H]);
-                pend_bar = B_H; pend_par = n & 1;
+                pend = B_H; pend_par = n & 1;
             }
+            __syncwarp();
         }
         if (done && NC > 0) {
-            group_wait(&bars[B_H], (NC - 1) & 1, E_H, 2, kChThreads, issuer, false);
-            if (sync_ok(2, kChThreads, issuer, ccnt)) {
-                if (issuer) pend_bar = -1;
+            group_wait(&bars[B_H], (NC - 1) & 1, E_H, 2, CH_THREADS, iwarp, false);
+            if (sync_ok(2, CH_THREADS, issuer, ccnt)) {
+                if (issuer) pend = -1;
                 tc_fence_after();
                 if (!rowpart) store_o(NC - 1);
                 if (p.S_T) {
@@ -788,17 +672,20 @@ tc_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
         // error path: no MMA of this role may still be running when TMEM is released
-        if (issuer && pend_bar >= 0 && *abort_flag) mbar_wait_drain(&bars[pend_bar], pend_par, lim);
+        if (issuer && pend >= 0 && *abort_flag) mbar_wait_drain(&bars[pend], pend_par, lim);
+        __syncwarp();
     }
     // ---------------------------------------------------------- teardown
     tc_fence_before();
-    __syncthreads();
+    block_sync();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, TM_COLS);
     }
     if (tid == 0 && *abort_flag) atomicCAS(&g_tc_error, 0u, (unsigned)*abort_flag);
 }
+
+// ---------------------------------------------------------------- host side
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -813,7 +700,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // [B, T, H, D] bf16 viewed as 4-D (D, H, T, B); box 64 x 1 x 64 x 1, 128-byte swizzle.
-bool make_map(CUtensorMap *m, const void *ptr, int B, int T, int H, int D) {
+bool make_map_bthd(CUtensorMap *m, const void *ptr, int B, int T, int H, int D) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
@@ -822,6 +709,20 @@ bool make_map(CUtensorMap *m, const void *ptr, int B, int T, int H, int D) {
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box,
                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// T workspace [rows, 64] fp16 viewed as 4-D (64, 1, rows, 1); box 64 x 1 x 64 x 1.
+bool make_map_t(CUtensorMap *m, const void *ptr, size_t rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {64, 1, (cuuint64_t)rows, 1};
+    cuuint64_t strides[3] = {128, 128, (cuuint64_t)rows * 128};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)C, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -841,27 +742,42 @@ bool tc_supports(const FwdParams &p, const char **why) {
 
 int tc_default_slices(const FwdParams &p) { return p.dv / DVS; }
 
-cudaError_t launch_tc(const FwdParams &p, cudaStream_t stream, const char **why) {
-    CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, p.q, p.B, p.T, p.H, p.dk) || !make_map(&mk, p.k, p.B, p.T, p.H, p.dk) ||
-        !make_map(&mv, p.v, p.B, p.T, p.H, p.dv)) {
+size_t tc_workspace_bytes(const FwdParams &p) {
+    const size_t nc = (size_t)(p.T + C - 1) / C;
+    return (size_t)p.B * p.H * nc * 64 * 64 * sizeof(__half);
+}
+
+cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, const char **why) {
+    const int NC = (p.T + C - 1) / C;
+    CUtensorMap mq, mk, mv, mt;
+    if (!make_map_bthd(&mq, p.q, p.B, p.T, p.H, p.dk) || !make_map_bthd(&mk, p.k, p.B, p.T, p.H, p.dk) ||
+        !make_map_bthd(&mv, p.v, p.B, p.T, p.H, p.dv) ||
+        !make_map_t(&mt, workspace, (size_t)p.B * p.H * NC * 64)) {
         *why = "(tensor map encoding failed)";
         return cudaErrorInvalidValue;
     }
     static bool attr_done = false;
     if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(tc_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SMEM_ALLOC);
+        cudaError_t e = cudaFuncSetAttribute(keyside_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)K1_SMEM);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K2_SMEM);
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
-    TcParams tp;
-    tp.B = p.B; tp.T = p.T; tp.H = p.H; tp.dv = p.dv;
-    tp.alpha = p.alpha; tp.beta = p.beta; tp.S0 = p.S0; tp.o = p.o; tp.S_T = p.S_T;
-    tp.o_bf16 = p.o_bf16; tp.neumann = p.mode == GDN_INV_NEUMANN; tp.N = p.N;
-    tp.limit_cycles = 4000000000ull;  // ~2 s at the B200 boost clock
-    dim3 grid(p.slices, p.H, p.B);
-    tc_chunk_kernel<<<grid, kThreads, SMEM_ALLOC, stream>>>(mq, mk, mv, tp);
+    K1Params k1;
+    k1.B = p.B; k1.T = p.T; k1.H = p.H; k1.NC = NC;
+    k1.alpha = p.alpha; k1.beta = p.beta;
+    k1.Tws = reinterpret_cast<__half *>(workspace);
+    k1.neumann = p.mode == GDN_INV_NEUMANN; k1.N = p.N;
+    keyside_kernel<<<dim3(NC, p.H, p.B), K1_THREADS, K1_SMEM, stream>>>(mk, k1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    K2Params k2;
+    k2.B = p.B; k2.T = p.T; k2.H = p.H; k2.dv = p.dv; k2.NC = NC;
+    k2.alpha = p.alpha; k2.beta = p.beta; k2.S0 = p.S0; k2.o = p.o; k2.S_T = p.S_T;
+    k2.o_bf16 = p.o_bf16;
+    chain_kernel<<<dim3(p.slices, p.H, p.B), K2_THREADS, K2_SMEM, stream>>>(mq, mk, mv, mt, k2);
     return cudaGetLastError();
 }
 

@@ -48,39 +48,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// As mbar_try_wait, but lets the hardware suspend the thread until the phase
-// completes or about `hint_ns` elapse, so that a waiting warp does not keep
-// polling shared memory.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-        : "memory");
-    return ok != 0;
-}
-
 // Bounded wait for phase `parity` of `bar`.  Gives up (returns false) when
 // *abort is set by another role or after about `limit_cycles` SM clock
-// cycles, recording `code` in *abort in the latter case.  The clock and the
-// abort flag are only consulted every 8 (sleeping) polls so that a waiting warp costs
-// its SM sub-partition as few issue slots as possible.
+// cycles, recording `code` in *abort in the latter case.  Between rounds of
+// polls the thread backs off with __nanosleep (itself bounded), so that a
+// waiting warp costs its SM sub-partition few issue slots; the bound never
+// depends on how long the hardware may suspend a thread inside try_wait.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           int code, uint64_t limit_cycles) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = clock64();
     for (;;) {
 #pragma unroll 1
-        for (int i = 0; i < 8; ++i)
-            if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        for (int i = 0; i < 4; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
         if (static_cast<uint64_t>(clock64()) - t0 > limit_cycles) {
             atomicCAS(const_cast<int *>(abort), 0, code);
             return false;
         }
+        __nanosleep(64);
     }
 }
 
@@ -147,9 +134,23 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Named barrier over `count` threads (ids 1..15; 0 is __syncthreads).
+// Named barrier over `count` threads (ids 1..15; 0 is the whole block).
+// Callers keep warps converged around barriers: waits are polled by whole
+// warps, and lane-only work (an MMA issue, a flag write) is followed by a
+// __syncwarp.  The warp is also reconverged on both sides here, so that the
+// barrier always sees whole warps and the .sync.aligned tcgen05 instructions
+// after it run converged.
 __device__ __forceinline__ void named_bar(int id, int count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+    __syncwarp();
+    asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+    __syncwarp();
+}
+
+// Whole-block barrier with the same convergence discipline as named_bar.
+__device__ __forceinline__ void block_sync() {
+    __syncwarp();
+    asm volatile("barrier.sync 0;" ::: "memory");
+    __syncwarp();
 }
 
 // ------------------------------------------------------------------- tcgen05

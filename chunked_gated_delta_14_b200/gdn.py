@@ -31,8 +31,8 @@ KERNELS = {"auto": 0, "simt": 1, "tc": 2}
 KERNEL_NAMES = {v: k for k, v in KERNELS.items()}
 MODES = {"exact": GDN_INV_EXACT, "neumann": GDN_INV_NEUMANN}
 
-EXPORTS = ("gdn_chunk_fwd", "gdn_select_kernel", "gdn_device_check", "gdn_status_string",
-           "gdn_last_error", "gdn_abi_version")
+EXPORTS = ("gdn_chunk_fwd", "gdn_select_kernel", "gdn_workspace_bytes", "gdn_device_check",
+           "gdn_status_string", "gdn_last_error", "gdn_abi_version")
 
 
 class GDNError(RuntimeError):
@@ -55,6 +55,7 @@ class FwdArgs(ctypes.Structure):
         ("S0", ctypes.c_void_p), ("o", ctypes.c_void_p), ("S_T", ctypes.c_void_p),
         ("mode", ctypes.c_int32), ("neumann_N", ctypes.c_int32),
         ("kernel", ctypes.c_int32), ("dv_split", ctypes.c_int32),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_uint64),
     ]
 
 
@@ -75,6 +76,8 @@ def lib() -> ctypes.CDLL:
             L.gdn_chunk_fwd.restype = ctypes.c_int
             L.gdn_select_kernel.argtypes = [ctypes.POINTER(FwdArgs)]
             L.gdn_select_kernel.restype = ctypes.c_int32
+            L.gdn_workspace_bytes.argtypes = [ctypes.POINTER(FwdArgs)]
+            L.gdn_workspace_bytes.restype = ctypes.c_uint64
             L.gdn_device_check.argtypes = [ctypes.c_void_p]
             L.gdn_device_check.restype = ctypes.c_int
             L.gdn_status_string.argtypes = [ctypes.c_int]
@@ -143,6 +146,27 @@ def select_kernel(args: FwdArgs) -> int:
     return int(lib().gdn_select_kernel(ctypes.byref(args)))
 
 
+def workspace_bytes(args: FwdArgs) -> int:
+    """Device workspace gdn_chunk_fwd needs for ``args`` (host only)."""
+    return int(lib().gdn_workspace_bytes(ctypes.byref(args)))
+
+
+_ws_cache = {}
+
+
+def workspace_for(args: FwdArgs, device: torch.device) -> Optional[torch.Tensor]:
+    """A cached device buffer of at least workspace_bytes(args) bytes, or None."""
+    need = workspace_bytes(args)
+    if need == 0:
+        return None
+    key = (device.type, device.index)
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < need:
+        buf = torch.empty(need, dtype=torch.uint8, device=device)
+        _ws_cache[key] = buf
+    return buf
+
+
 def call(args: FwdArgs, stream: Optional[int] = None) -> None:
     """Raw gdn_chunk_fwd call; raises GDNError on a non-OK status."""
     s = lib().gdn_chunk_fwd(ctypes.byref(args), ctypes.c_void_p(stream or 0))
@@ -207,6 +231,10 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         neumann_N=int(N), kernel=KERNELS[kernel], dv_split=int(dv_split))
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
+    ws = workspace_for(args, q.device)
+    if ws is not None:
+        args.workspace = ws.data_ptr()
+        args.workspace_bytes = ws.numel()
     with torch.cuda.device(q.device):
         call(args, stream.cuda_stream)
     return out, S_T

@@ -45,8 +45,10 @@
  *   o        [B, T, H, dv]   o_dtype
  *
  * Ownership.  Every pointer is a DEVICE pointer owned by the caller, who
- * allocates inputs and outputs.  The library allocates no device memory and
- * keeps no state between calls.
+ * allocates inputs, outputs and the workspace.  The library allocates no
+ * device memory and keeps no state between calls.  The tensor-core kernel
+ * stores each chunk's inverse T (fp16, 8 KB per chunk and head) in the
+ * workspace between its two launches; gdn_workspace_bytes() gives the size.
  *
  * Execution and errors.  gdn_chunk_fwd validates its arguments on the host
  * and returns an error before launching anything (nothing is written) when
@@ -66,7 +68,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 1
+#define GDN_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define GDN_API __attribute__((visibility("default")))
@@ -118,10 +120,18 @@ typedef struct {
     int32_t neumann_N;          /* N for GDN_INV_NEUMANN: 0 <= N <= chunk - 1 */
     int32_t kernel;             /* gdn_kernel selection */
     int32_t dv_split;           /* value-axis slices per head (0 = choose) */
+    void *workspace;            /* device scratch of >= gdn_workspace_bytes(args) bytes,
+                                   16-byte aligned, caller-owned; may be NULL when that is 0 */
+    uint64_t workspace_bytes;   /* size of workspace */
 } gdn_fwd_args;
 
 /* Chunkwise forward: o and S_T from q, k, v, gates and S0 (see above). */
 GDN_API gdn_status gdn_chunk_fwd(const gdn_fwd_args *args, void *stream);
+
+/* Workspace bytes gdn_chunk_fwd needs for these arguments (0 for the SIMT
+ * kernel), or 0 with gdn_last_error() set if the arguments are invalid.  Host
+ * only. */
+GDN_API uint64_t gdn_workspace_bytes(const gdn_fwd_args *args);
 
 /* Which kernel gdn_chunk_fwd would launch for these arguments (gdn_kernel
  * value, never AUTO), or a negative gdn_status if they are invalid.  Host
