@@ -3,8 +3,13 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "gdn_internal.cuh"
+
+// Fixed scratch of gdn_chunk_fwd_static_scratch: the per-chunk T matrices of
+// the tensor-core path (8 KiB per chunk-head), GDN_STATIC_SCRATCH_BYTES in all.
+static __device__ __align__(256) unsigned char gdn_static_scratch[GDN_STATIC_SCRATCH_BYTES];
 
 namespace {
 
@@ -194,6 +199,50 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_args *args, void *stream) {
     if (e != cudaSuccess)
         return fail(GDN_ERR_CUDA, "%s launch: %s %s", kern == GDN_KERNEL_TC ? "tc" : "simt",
                     cudaGetErrorString(e), why);
+    g_msg[0] = 0;
+    return GDN_OK;
+}
+
+// Tensor-core path with the file's fixed scratch array in place of a caller
+// workspace: nothing is allocated.  The array's device address is looked up
+// once per device, with that device current, on the first call made there.
+gdn_status gdn_chunk_fwd_static_scratch(const gdn_fwd_args *args, void *stream) {
+    gdn::FwdParams p;
+    int kern = 0;
+    gdn_status s = resolve(args, &p, &kern);
+    if (s != GDN_OK) return s;
+    if (kern != GDN_KERNEL_TC)
+        return fail(GDN_ERR_UNSUPPORTED, "the fixed-scratch entry point runs the tensor-core kernel only");
+    if (args->workspace || args->workspace_bytes)
+        return fail(GDN_ERR_INVALID_ARG, "the fixed-scratch entry point takes no workspace (pass NULL, 0)");
+    const size_t need = gdn::tc_workspace_bytes(p);
+    if (need > (size_t)GDN_STATIC_SCRATCH_BYTES)
+        return fail(GDN_ERR_INVALID_ARG,
+                    "needs %zu bytes of scratch (8 KiB per chunk-head, B*H*ceil(T/64) = %zu); "
+                    "the fixed array holds %llu bytes",
+                    need, need / 8192, (unsigned long long)GDN_STATIC_SCRATCH_BYTES);
+    constexpr int kMaxDevices = 64;
+    static void *dev_ptr[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(GDN_ERR_UNSUPPORTED, "device index %d >= %d", dev, kMaxDevices);
+    void *scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!dev_ptr[dev]) {
+            void *ptr = nullptr;
+            e = cudaGetSymbolAddress(&ptr, gdn_static_scratch);
+            if (e != cudaSuccess)
+                return fail(GDN_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+            dev_ptr[dev] = ptr;
+        }
+        scratch = dev_ptr[dev];
+    }
+    const char *why = "";
+    e = gdn::launch_tc(p, scratch, reinterpret_cast<cudaStream_t>(stream), &why);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "tc launch: %s %s", cudaGetErrorString(e), why);
     g_msg[0] = 0;
     return GDN_OK;
 }

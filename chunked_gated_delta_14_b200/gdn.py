@@ -32,7 +32,8 @@ KERNEL_NAMES = {v: k for k, v in KERNELS.items()}
 MODES = {"exact": GDN_INV_EXACT, "neumann": GDN_INV_NEUMANN}
 
 EXPORTS = ("gdn_chunk_fwd", "gdn_select_kernel", "gdn_workspace_bytes", "gdn_device_check",
-           "gdn_status_string", "gdn_last_error", "gdn_abi_version")
+           "gdn_status_string", "gdn_last_error", "gdn_abi_version", "gdn_chunk_fwd_static_scratch")
+STATIC_SCRATCH_BYTES = 8 << 20   # GDN_STATIC_SCRATCH_BYTES
 
 
 class GDNError(RuntimeError):
@@ -86,6 +87,8 @@ def lib() -> ctypes.CDLL:
             L.gdn_last_error.restype = ctypes.c_char_p
             L.gdn_abi_version.argtypes = []
             L.gdn_abi_version.restype = ctypes.c_int32
+            L.gdn_chunk_fwd_static_scratch.argtypes = [ctypes.POINTER(FwdArgs), ctypes.c_void_p]
+            L.gdn_chunk_fwd_static_scratch.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -170,6 +173,14 @@ def workspace_for(args: FwdArgs, device: torch.device) -> Optional[torch.Tensor]
 def call(args: FwdArgs, stream: Optional[int] = None) -> None:
     """Raw gdn_chunk_fwd call; raises GDNError on a non-OK status."""
     s = lib().gdn_chunk_fwd(ctypes.byref(args), ctypes.c_void_p(stream or 0))
+    if s != GDN_OK:
+        raise GDNError(s, last_error())
+
+
+def call_static_scratch(args: FwdArgs, stream: Optional[int] = None) -> None:
+    """Raw gdn_chunk_fwd_static_scratch call (tensor-core kernel, the library's
+    fixed scratch; args.workspace must be 0); raises GDNError on a non-OK status."""
+    s = lib().gdn_chunk_fwd_static_scratch(ctypes.byref(args), ctypes.c_void_p(stream or 0))
     if s != GDN_OK:
         raise GDNError(s, last_error())
 

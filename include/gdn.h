@@ -155,6 +155,37 @@ GDN_API const char *gdn_last_error(void);
 /* GDN_ABI_VERSION of the loaded library. */
 GDN_API int32_t gdn_abi_version(void);
 
+/* Size of the fixed device scratch array of gdn_chunk_fwd_static_scratch:
+ * 8 MiB = 1024 chunk-heads of one 64 x 64 fp16 T matrix each. */
+#define GDN_STATIC_SCRATCH_BYTES (8ull << 20)
+
+/* gdn_chunk_fwd on the tensor-core kernel, with a fixed scratch array inside
+ * the library in place of args->workspace.  The pages have no counterpart:
+ * this is a calling convenience of this library, not a step of the method.
+ *
+ * For callers that cannot allocate device memory per call: a plain C host
+ * program that links only this library and the CUDA runtime and holds no
+ * allocator, or a serving loop that must not call cudaMalloc after start-up
+ * (cudaMalloc and cudaFree may synchronise the device).  The call allocates
+ * nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *
+ * Arguments as gdn_chunk_fwd, except: args->workspace must be NULL and
+ * args->workspace_bytes 0; the arguments must select the tensor-core kernel
+ * (kernel AUTO or TC with a supported shape), else GDN_ERR_UNSUPPORTED; and
+ * B * H * ceil(T / 64) * 8192 must be <= GDN_STATIC_SCRATCH_BYTES, else
+ * GDN_ERR_INVALID_ARG with the needed size in gdn_last_error().  Nothing in
+ * the scratch has to start at zero: the key-side kernel writes every T entry
+ * the chain kernel reads, in the same call.
+ *
+ * Set-up: the first call on each device, with that device current, looks up
+ * the array's address with cudaGetSymbolAddress (an error there returns
+ * GDN_ERR_CUDA).  Make that first call before any stream capture.
+ *
+ * One scratch per device: calls that overlap in time on one device (from
+ * different streams or threads) race on it and give wrong results.  Calls
+ * ordered on one stream are safe. */
+GDN_API gdn_status gdn_chunk_fwd_static_scratch(const gdn_fwd_args *args, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,63 @@
+"""gdn_chunk_fwd_static_scratch: the tensor-core path with the library's fixed
+scratch array instead of a caller workspace.  Collected last on purpose, so
+that it also runs after every other test has used the device."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import chunked_gated_delta_14_b200 as gdn
+import chunked_gated_delta_14_b200.gdn as G
+from chunked_gated_delta_14_b200.inputs import make_inputs, workload
+from gpu_util import TOL_BF16_REL_RMS
+
+
+def _args(w, d, o, S):
+    ptr = lambda t: None if t is None else t.data_ptr()
+    return G.make_args(B=w.B, T=w.T, H=w.H, dk=w.dk, dv=w.dv, chunk=w.chunk, io_dtype=1, o_dtype=0,
+                       q=ptr(d["q"]), k=ptr(d["k"]), v=ptr(d["v"]), alpha=ptr(d["alpha"]),
+                       beta=ptr(d["beta"]), S0=ptr(d["S0"]), o=o.data_ptr(), S_T=S.data_ptr(),
+                       mode=0, kernel=2)
+
+
+def test_static_scratch_rejects_oversize_and_workspace():
+    # host-side checks: they return before any device call
+    w = workload("gdn_bf16", B=2, H=16, T=4096)          # 2048 chunk-heads: 16 MiB of T
+    fake = 1 << 20
+    a = G.make_args(B=w.B, T=w.T, H=w.H, dk=128, dv=128, chunk=64, io_dtype=1, o_dtype=0,
+                    q=fake, k=fake, v=fake, alpha=fake, beta=fake, o=2 * fake, S_T=3 * fake,
+                    mode=0, kernel=2)
+    s = G.lib().gdn_chunk_fwd_static_scratch(ctypes.byref(a), None)
+    assert s == G.GDN_ERR_INVALID_ARG
+    msg = G.last_error()
+    assert "scratch" in msg and str(16 << 20) in msg, msg
+    a.B = 1                                                  # fits, but a workspace is passed
+    a.workspace, a.workspace_bytes = 4 * fake, 8 << 20
+    assert G.lib().gdn_chunk_fwd_static_scratch(ctypes.byref(a), None) == G.GDN_ERR_INVALID_ARG
+    a.workspace, a.workspace_bytes = None, 0
+    a.kernel = 1                                             # SIMT is not this entry point's kernel
+    assert G.lib().gdn_chunk_fwd_static_scratch(ctypes.byref(a), None) == G.GDN_ERR_UNSUPPORTED
+
+
+@pytest.mark.gpu
+def test_static_scratch_matches_workspace_entry():
+    # 1 x 16 heads x 64 chunks = 1024 chunk-heads: exactly the fixed maximum
+    w = workload("gdn_bf16", B=1, H=16, T=4096, s0_std=0.02)
+    assert w.B * w.H * (w.T // 64) * 8192 == G.STATIC_SCRATCH_BYTES
+    x = make_inputs(w, seed=21)
+    d = {k: (None if v is None else v.cuda()) for k, v in x.items()}
+    o_ref, s_ref = gdn.chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S0=d["S0"],
+                                 o_dtype=torch.float32, kernel="tc")
+    torch.cuda.synchronize()
+    rms_o = float(o_ref.double().pow(2).mean().sqrt())
+    rms_s = float(s_ref.double().pow(2).mean().sqrt())
+    stream = torch.cuda.current_stream().cuda_stream
+    for call in range(2):                                    # two calls in a row
+        o = torch.full_like(o_ref, float("nan"))
+        S = torch.full_like(s_ref, float("nan"))
+        G.call_static_scratch(_args(w, d, o, S), stream)
+        gdn.device_check(stream)
+        eo = float((o.double() - o_ref.double()).abs().max()) / rms_o
+        es = float((S.double() - s_ref.double()).abs().max()) / rms_s
+        assert eo <= TOL_BF16_REL_RMS and es <= TOL_BF16_REL_RMS, (call, eo, es)
