@@ -1,13 +1,15 @@
 """Benchmark of the chunkwise gated delta-rule forward on B200.
 
 Default workload: the Gated DeltaNet layer with 1.3B-class head geometry,
-B=4, H=16, T=4096, d_k=d_v=128, chunk 64, bf16 q/k/v, fp32 alpha/beta, fp32 o
-and S_T, exact blocked inversion.  One step = one gdn_chunk_fwd call over the
+B=4, H=16, T=4096, d_k=d_v=128, chunk 64, bf16 q/k/v/o, fp32 alpha/beta and
+S_T, exact blocked inversion.  One step = one gdn_chunk_fwd call over the
 whole batch (every step of the hot path: staging, gate scans, Gram, inverse,
 WY products, state passing, output).  Inputs are synthetic (seeded), resident
 in HBM when the timed region starts.
 
-  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--batch B]
+
+``--batch B`` replaces the batch size (a smaller case for profiler captures).
 
 Under torchrun each rank runs its own independent batch (weak scaling, no
 collective on the data path); the time is the max over ranks.
@@ -175,15 +177,15 @@ def run_gpu(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = workload(WORKLOAD)
+    w = workload(WORKLOAD, **({"B": args.batch} if args.batch else {}))
     x = make_inputs(w, seed=rank)   # each rank its own batch
     d = {k: (None if v is None else v.to(dev)) for k, v in x.items()}
-    o = torch.empty((w.B, w.T, w.H, w.dv), device=dev, dtype=torch.float32)
+    o = torch.empty((w.B, w.T, w.H, w.dv), device=dev, dtype=torch.bfloat16)
     S_T = torch.empty((w.B, w.H, w.dk, w.dv), device=dev, dtype=torch.float32)
     stream = torch.cuda.current_stream(dev)
     ptr = lambda t: None if t is None else t.data_ptr()
     a = gdn.make_args(B=w.B, T=w.T, H=w.H, dk=w.dk, dv=w.dv, chunk=w.chunk, io_dtype=1,
-                      o_dtype=0, q=ptr(d["q"]), k=ptr(d["k"]), v=ptr(d["v"]),
+                      o_dtype=1, q=ptr(d["q"]), k=ptr(d["k"]), v=ptr(d["v"]),
                       alpha=ptr(d["alpha"]), beta=ptr(d["beta"]), S0=None, o=o.data_ptr(),
                       S_T=S_T.data_ptr(), mode=0, kernel=0)
     ws = gdn.workspace_for(a, dev)
@@ -192,6 +194,7 @@ def run_gpu(args, rank, world, local_rank):
         a.workspace_bytes = ws.numel()
     kernel_id = gdn.select_kernel(a)
     kernel_name = {1: "simt_chunk_kernel", 2: "keyside_kernel+chain_kernel"}.get(kernel_id, "?")
+    launches_per_call = 2 if kernel_id == 2 else 1
     sh = stream.cuda_stream
 
     def step():
@@ -246,7 +249,7 @@ def run_gpu(args, rank, world, local_rank):
                 if v is not None:
                     dev_in[k].copy_(v, non_blocking=True)
             gdn.chunk_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"],
-                          dev_in["beta"], chunk=w.chunk, o_dtype=torch.float32, out=o,
+                          dev_in["beta"], chunk=w.chunk, o_dtype=torch.bfloat16, out=o,
                           S_T=S_T)
             o_host.copy_(o, non_blocking=True)
 
@@ -272,7 +275,7 @@ def run_gpu(args, rank, world, local_rank):
                    ms_per_step=ems / args.e2e_steps)
 
     pk = peaks()
-    bytes_launch = algorithmic_bytes(w, o_bytes=4)
+    bytes_launch = algorithmic_bytes(w, o_bytes=2)
     achieved = bytes_launch / (ms_step / 1e3) / 1e9
     flops = algorithmic_flops(w)
     roof = dict(bound="hbm", achieved=achieved, peak=pk["hbm_gbs"], unit="GB/s",
@@ -295,13 +298,16 @@ def run_gpu(args, rank, world, local_rank):
                     compute="bf16 q/k/v in HBM; fp16 tensor-core operands, fp32 accumulate and state",
                     data="synthetic (seeded; Gated DeltaNet layer shapes)",
                     config=dict(workload=f"{WORKLOAD}: B={w.B} H={w.H} T={w.T} dk={w.dk} "
-                                f"dv={w.dv} chunk={w.chunk} exact inverse, o fp32",
+                                f"dv={w.dv} chunk={w.chunk} exact inverse, o bf16",
                                 global_batch=w.B * world, seq_len=w.T,
                                 parallelism=f"independent batch per GPU x{world}",
-                                l2="no flush: inputs+outputs 341 MB per step > 126 MB L2",
+                                l2=(f"no flush: inputs+outputs {bytes_launch / 1e6:.0f} MB per step > 126 MB L2"
+                                    if bytes_launch > 126e6 else
+                                    f"no flush: {bytes_launch / 1e6:.0f} MB per step (fits L2; profiler case)"),
                                 kernel=kernel_name),
                     clocks=clocks.summary() if rank == 0 else None,
-                    e2e=e2e, gpu_launches=args.steps, roofline=roof, cpu_baseline=cpu)
+                    e2e=e2e, gpu_launches=args.steps * launches_per_call, roofline=roof,
+                    cpu_baseline=cpu)
         print(json.dumps(line), flush=True)
 
 
@@ -335,7 +341,7 @@ def run_reference(args, rank, world):
         return
     import oracle
     from chunked_gated_delta_14_b200.inputs import make_inputs, workload
-    w = workload(WORKLOAD)
+    w = workload(WORKLOAD, **({"B": args.batch} if args.batch else {}))
     x = make_inputs(w)
     cores = len(os.sched_getaffinity(0))
     # per-step sample: a prefix of one (batch, head) row group sized so that
@@ -366,7 +372,8 @@ def run_reference(args, rank, world):
                 higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
                 data="synthetic (seeded; Gated DeltaNet layer shapes)",
                 config=dict(workload=f"{WORKLOAD}: B={w.B} H={w.H} T={w.T} dk={w.dk} "
-                            f"dv={w.dv} chunk={w.chunk}", global_batch=w.B, seq_len=w.T,
+                            f"dv={w.dv} chunk={w.chunk} exact inverse, o bf16",
+                            global_batch=w.B, seq_len=w.T,
                             parallelism="CPU oracle, rank 0 only"),
                 cpu_baseline=dict(value=value, unit=UNIT, cores=cores, kind="oracle",
                                   sample=sample),
@@ -384,6 +391,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--ref-budget", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="replace the batch size B (profiler case)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
