@@ -104,6 +104,24 @@ def profile_traffic(kernel_name):
     return float(m_k.group(1))
 
 
+def max_over_ranks(ms, world, device=None):
+    """Slowest rank's time: every rank contributes its own event time and all
+    ranks receive the maximum (an all-reduce, so the collective is the same on
+    every rank)."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank_step, world, steps, ms_max):
+    """Whole-job rate: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank_step * world * steps / (ms_max / 1e3)
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -222,18 +240,14 @@ def run_gpu(args, rank, world, local_rank):
     t_wall1 = time.time()
     if world > 1:
         dist.barrier()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     clocks.mark(t_wall0, t_wall1)
     time.sleep(0.3)
     clocks.stop()
 
     ms_step = ms / args.steps
     tokens_step = w.B * w.T
-    value = tokens_step * world * args.steps / (ms / 1e3)
+    value = job_throughput(tokens_step, world, args.steps, ms)
 
     # end to end through the public API: pinned host inputs -> device -> kernel -> host o
     e2e = None
@@ -265,12 +279,8 @@ def run_gpu(args, rank, world, local_rank):
             e2e_step()
         f1.record(stream)
         torch.cuda.synchronize()
-        ems = f0.elapsed_time(f1)
-        if world > 1:
-            t = torch.tensor([ems], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = dict(value=tokens_step * world * args.e2e_steps / (ems / 1e3), unit=UNIT,
+        ems = max_over_ranks(f0.elapsed_time(f1), world, dev)
+        e2e = dict(value=job_throughput(tokens_step, world, args.e2e_steps, ems), unit=UNIT,
                    h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h),
                    ms_per_step=ems / args.e2e_steps)
 
