@@ -8,7 +8,7 @@
 #include "gdn_internal.cuh"
 
 // Fixed scratch of gdn_chunk_fwd_static_scratch: the per-chunk T matrices of
-// the tensor-core path (8 KiB per chunk-head), GDN_STATIC_SCRATCH_BYTES in all.
+// the tensor-core path (24 KiB per chunk-head), GDN_STATIC_SCRATCH_BYTES in all.
 static __device__ __align__(256) unsigned char gdn_static_scratch[GDN_STATIC_SCRATCH_BYTES];
 
 namespace {
@@ -218,9 +218,9 @@ gdn_status gdn_chunk_fwd_static_scratch(const gdn_fwd_args *args, void *stream) 
     const size_t need = gdn::tc_workspace_bytes(p);
     if (need > (size_t)GDN_STATIC_SCRATCH_BYTES)
         return fail(GDN_ERR_INVALID_ARG,
-                    "needs %zu bytes of scratch (8 KiB per chunk-head, B*H*ceil(T/64) = %zu); "
+                    "needs %zu bytes of scratch (24 KiB per chunk-head, B*H*ceil(T/64) = %zu); "
                     "the fixed array holds %llu bytes",
-                    need, need / 8192, (unsigned long long)GDN_STATIC_SCRATCH_BYTES);
+                    need, need / 24576, (unsigned long long)GDN_STATIC_SCRATCH_BYTES);
     constexpr int kMaxDevices = 64;
     static void *dev_ptr[kMaxDevices] = {};
     static std::mutex mu;

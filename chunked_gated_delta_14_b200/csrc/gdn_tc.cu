@@ -75,25 +75,33 @@ constexpr uint32_t IDESC_MM64 = idesc_f16(128, 64, 0, 0, 1, 1);     // fp16, MN-
 
 // =========================================================== key-side kernel
 
+// Workspace per chunk-head: three 64 x 64 fp16 row-major matrices,
+// T diag(beta), T diag(beta e^g) and the decayed causal scores P.
+constexpr int WS_ROWS = 192;                           // rows of 128 bytes per chunk-head
+constexpr size_t WS_CHUNK_BYTES = (size_t)WS_ROWS * 128;
+
 constexpr int K1_THREADS = 256;
-constexpr uint32_t K1_OFF_K = 0;                       // K tile, two 64-column boxes
-constexpr uint32_t K1_OFF_LB = 16384;                  // L fp32 (also the rows after K's 2nd box)
+constexpr uint32_t K1_OFF_QK = 0;                      // per key block kb: [Q | K] at kb * 16 KB
+constexpr uint32_t K1_OFF_YB = 0;                      // inverse scratch (8 KB), reuses the tiles
+constexpr uint32_t K1_OFF_LB = 32768;                  // L fp32
 constexpr uint32_t K1_MAT = 64 * LSTR * 4;
 constexpr uint32_t K1_OFF_TB = K1_OFF_LB + K1_MAT;
-constexpr uint32_t K1_OFF_YB = K1_OFF_TB + K1_MAT;
-constexpr uint32_t K1_OFF_PAR = K1_OFF_YB + 8192;
+constexpr uint32_t K1_OFF_PAR = K1_OFF_TB + K1_MAT;
 constexpr uint32_t K1_OFF_BAR = K1_OFF_PAR + ((sizeof(ChunkParams) + 15) & ~15u);
 constexpr uint32_t K1_SMEM = K1_OFF_BAR + 64 + 1024;  // + base alignment slack
 
 struct K1Params {
     int B, T, H, NC;
     const float *alpha, *beta;
-    __half *Tws;
+    uint8_t *ws;
     int neumann, N;
 };
 
+// One CTA per (chunk, head, batch).  [Q ; K] K^T in one MMA: TMEM lanes 0..63
+// hold Q K^T (-> P), lanes 64..127 hold K K^T (-> L -> T).
 __global__ void __launch_bounds__(K1_THREADS)
-keyside_kernel(const __grid_constant__ CUtensorMap tm_k, const K1Params p) {
+keyside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const K1Params p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -105,6 +113,7 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_k, const K1Params p) {
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + K1_OFF_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + K1_OFF_BAR + 16);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + K1_OFF_BAR + 20);
+    uint8_t *ws = p.ws + ((((size_t)b * p.H + h) * p.NC + n) * WS_CHUNK_BYTES);
 
     if (tid == 0) {
         mbar_init(&bars[0], 1);
@@ -125,10 +134,13 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_k, const K1Params p) {
     const uint32_t tmem = *tmem_slot;
     const int t0 = n * C;
     if (tid == 0) {
+        tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
-        mbar_arrive_expect_tx(&bars[0], 16384);
-        tma_load_4d(sm + K1_OFF_K, &tm_k, &bars[0], 0, h, t0, b);
-        tma_load_4d(sm + K1_OFF_K + 8192, &tm_k, &bars[0], 64, h, t0, b);
+        mbar_arrive_expect_tx(&bars[0], 32768);
+        tma_load_4d(sm + K1_OFF_QK, &tm_q, &bars[0], 0, h, t0, b);
+        tma_load_4d(sm + K1_OFF_QK + 8192, &tm_k, &bars[0], 0, h, t0, b);
+        tma_load_4d(sm + K1_OFF_QK + 16384, &tm_q, &bars[0], 64, h, t0, b);
+        tma_load_4d(sm + K1_OFF_QK + 24576, &tm_k, &bars[0], 64, h, t0, b);
     }
     __syncwarp();
     if (warp == 1) {
@@ -138,13 +150,12 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_k, const K1Params p) {
     }
     if (tid == 0) {
         if (mbar_wait(&bars[0], 0, abort_flag, E_K1_TMA, kWaitLimit)) {
-            // [K ; next 64 rows] K^T: lanes 0..63 of the result hold K K^T
             tc_fence_after();
-            const uint32_t a0 = smem_u32(sm + K1_OFF_K);
+            const uint32_t a0 = smem_u32(sm + K1_OFF_QK);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
-                umma_f16_ss(tmem, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(a0 + off, 16, 1024),
+                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                umma_f16_ss(tmem, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(a0 + off + 8192, 16, 1024),
                             IDESC_BF_KK, kk > 0);
             }
             umma_commit(&bars[1]);
@@ -160,20 +171,40 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_k, const K1Params p) {
     if (go) {
         mbar_try_wait(&bars[1], 0);
         tc_fence_after();
-        // L rows: TMEM lanes 0..63 (sub-partitions 0, 1), column half hf
+        // sub-partition sp holds rows 32 sp .. 32 sp + 31 of [Q K^T ; K K^T];
+        // warp half hf takes columns [32 hf, 32 hf + 32).
         const int sp = warp & 3, hf = warp >> 2;
+        const int r = 32 * (sp & 1) + lane;               // chunk row
+        const bool diag = (hf == (sp & 1));
+        uint32_t xr[32];
+        float gam[32];
+        if (hf <= (sp & 1)) {
+            tmem_ld32(tmem + ((uint32_t)(32 * sp) << 16) + 32 * hf, xr);
+            tc::decay_row(par, r, hf, diag, gam);
+            tmem_wait_ld();
+        }
         if (sp < 2) {
-            const int r = 32 * sp + lane;
+            // P_ri = (q_r . k_i) exp(g_r - g_i), i <= r: straight to the workspace
+            uint4 *dst = reinterpret_cast<uint4 *>(ws + (size_t)(128 + r) * 128 + 64 * hf);
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                uint4 u = make_uint4(0u, 0u, 0u, 0u);
+                if (hf <= sp) {
+                    const int j = 8 * jj;
+                    u.x = pack_h2(gam[j] * __uint_as_float(xr[j]), gam[j + 1] * __uint_as_float(xr[j + 1]));
+                    u.y = pack_h2(gam[j + 2] * __uint_as_float(xr[j + 2]), gam[j + 3] * __uint_as_float(xr[j + 3]));
+                    u.z = pack_h2(gam[j + 4] * __uint_as_float(xr[j + 4]), gam[j + 5] * __uint_as_float(xr[j + 5]));
+                    u.w = pack_h2(gam[j + 6] * __uint_as_float(xr[j + 6]), gam[j + 7] * __uint_as_float(xr[j + 7]));
+                }
+                dst[jj] = u;
+            }
+        } else {
+            // L_ri = beta_r exp(g_r - g_i) (k_r . k_i), i < r
             float *Lr = Lb + r * LSTR + 32 * hf;
-            if (hf > sp) {
+            if (hf > (sp & 1)) {
 #pragma unroll
                 for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4 *>(Lr + j) = make_float4(0.f, 0.f, 0.f, 0.f);
             } else {
-                uint32_t xr[32];
-                tmem_ld32(tmem + ((uint32_t)(32 * sp) << 16) + 32 * hf, xr);
-                float gam[32];
-                tc::decay_row(par, r, hf, hf == sp, gam);
-                tmem_wait_ld();
                 const float br = par->bet[r];
 #pragma unroll
                 for (int j = 0; j < 32; j += 4) {
@@ -191,21 +222,26 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_k, const K1Params p) {
         named_bar(1, K1_THREADS);
         if (p.neumann) tc::invert_neumann(Lb, Tb, Yb, tid, p.N, 1);
         else tc::invert_exact(Lb, Tb, Yb, tid, 1);
-        // T -> fp16, row-major [64][64] per chunk
+        // T diag(beta) and T diag(beta e^g) -> fp16, row-major
         {
-            const int r = tid >> 2, j0 = (tid & 3) * 2;
-            const size_t row = (((size_t)b * p.H + h) * p.NC + n) * 64 + r;
-            uint4 *dst = reinterpret_cast<uint4 *>(p.Tws + row * 64);
-            const float *Tr = Tb + r * LSTR;
+            const int rr = tid >> 2, j0 = (tid & 3) * 2;
+            uint4 *d1 = reinterpret_cast<uint4 *>(ws + (size_t)rr * 128);
+            uint4 *d2 = reinterpret_cast<uint4 *>(ws + (size_t)(64 + rr) * 128);
+            const float *Tr = Tb + rr * LSTR;
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 const int j = j0 + q;
-                const float4 a = *reinterpret_cast<const float4 *>(Tr + 8 * j);
-                const float4 c = *reinterpret_cast<const float4 *>(Tr + 8 * j + 4);
-                uint4 u;
-                u.x = pack_h2(a.x, a.y); u.y = pack_h2(a.z, a.w);
-                u.z = pack_h2(c.x, c.y); u.w = pack_h2(c.z, c.w);
-                dst[j] = u;
+                float t[8], sb[8], sg[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    t[e] = Tr[8 * j + e];
+                    sb[e] = t[e] * par->bet[8 * j + e];
+                    sg[e] = sb[e] * par->eg[8 * j + e];
+                }
+                d1[j] = make_uint4(pack_h2(sb[0], sb[1]), pack_h2(sb[2], sb[3]), pack_h2(sb[4], sb[5]),
+                                   pack_h2(sb[6], sb[7]));
+                d2[j] = make_uint4(pack_h2(sg[0], sg[1]), pack_h2(sg[2], sg[3]), pack_h2(sg[4], sg[5]),
+                                   pack_h2(sg[6], sg[7]));
             }
         }
     }
@@ -223,18 +259,17 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_k, const K1Params p) {
 constexpr int K2_THREADS = 448;    // 14 warps
 constexpr int KS_THREADS = 256, CH_THREADS = 128;
 // stage (x2): per 64-column key block kb: [W | Q | K] at kb * 24 KB; V, T after
-constexpr uint32_t STG = 65536;
-constexpr uint32_t S_W = 0, S_Q = 8192, S_K = 16384, S_KB = 24576, S_V = 49152, S_T = 57344;
-constexpr uint32_t OFF_TBG = 2 * STG;                  // T diag(beta e^g)
-constexpr uint32_t OFF_P = OFF_TBG + 8192;             // P x 2 (P1's preceding rows are P0)
-constexpr uint32_t OFF_HS = OFF_P + 2 * 8192;          // h fp16, 128 rows
+//   then V, then the workspace rows of the chunk: T diag(beta), T diag(beta e^g), P
+constexpr uint32_t STG = 81920;
+constexpr uint32_t S_W = 0, S_Q = 8192, S_K = 16384, S_KB = 24576, S_V = 49152;
+constexpr uint32_t S_TB = 57344, S_TBG = 65536, S_P = 73728;
+constexpr uint32_t OFF_HS = 2 * STG;                   // h fp16, 128 rows
 constexpr uint32_t OFF_DS = OFF_HS + 16384;            // Delta fp16
 constexpr uint32_t OFF_DPS = OFF_DS + 8192;            // e^{g_C - g} Delta fp16
 constexpr uint32_t OFF_PAR = OFF_DPS + 8192;
 constexpr uint32_t PAR_BYTES = (sizeof(ChunkParams) + 15) & ~15u;
 constexpr uint32_t OFF_BAR = OFF_PAR + 3 * PAR_BYTES;   // params ring of 3
-enum { B_FULL = 0, B_EMPTY = 2, B_KSREADY = 4, B_KSFREE = 6, B_G = 8, B_UW = 9, B_X = 10, B_H = 11,
-       N_BARS = 12 };
+enum { B_FULL = 0, B_EMPTY = 2, B_KSREADY = 4, B_KSFREE = 6, B_UW = 8, B_X = 9, B_H = 10, N_BARS = 11 };
 constexpr uint32_t OFF_MISC = OFF_BAR + N_BARS * 8;     // tmem slot, abort flag, group slots
 constexpr uint32_t SMEM_USED = OFF_MISC + 32;
 constexpr uint32_t K2_SMEM = SMEM_USED + 1024;
@@ -242,7 +277,7 @@ static_assert(K2_SMEM <= 232448, "shared memory budget of one sm_100 block");
 static_assert(K1_SMEM * 3 <= 233472, "three key-side blocks per SM");
 
 // TMEM columns
-constexpr uint32_t TM_G = 0, TM_U0 = 64, TM_U1 = 128, TM_W = 192, TM_X0 = 320, TM_X1 = 384, TM_H = 448;
+constexpr uint32_t TM_U0 = 0, TM_U1 = 64, TM_W = 128, TM_X0 = 256, TM_X1 = 320, TM_H = 384;
 constexpr uint32_t TM_COLS = 512;
 
 struct K2Params {
@@ -305,7 +340,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             mbar_init(&bars[B_KSREADY + i], 1);
             mbar_init(&bars[B_KSFREE + i], 1);
         }
-        mbar_init(&bars[B_G], 1);
         mbar_init(&bars[B_UW], 1);
         mbar_init(&bars[B_X], 1);
         mbar_init(&bars[B_H], 1);
@@ -335,7 +369,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 if (m >= 2 && !mbar_wait(&bars[B_EMPTY + s], ((m - 2) >> 1) & 1, abort_flag, E_EMPTY, lim))
                     break;
                 uint64_t *fb = &bars[B_FULL + s];
-                mbar_arrive_expect_tx(fb, 49152);
+                mbar_arrive_expect_tx(fb, 65536);
                 uint8_t *st = sm + s * STG;
                 const int t0 = m * C;
                 tma_load_4d(st + S_Q, &tm_q, fb, 0, h, t0, b);
@@ -343,7 +377,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 tma_load_4d(st + S_K, &tm_k, fb, 0, h, t0, b);
                 tma_load_4d(st + S_KB + S_K, &tm_k, fb, 64, h, t0, b);
                 tma_load_4d(st + S_V, &tm_v, fb, v0, h, t0, b);
-                tma_load_4d(st + S_T, &tm_t, fb, 0, 0, (((b * H) + h) * NC + m) * 64, 0);
+                tma_load_4d(st + S_TB, &tm_t, fb, 0, 0, (((b * H) + h) * NC + m) * WS_ROWS, 0);
                 issued = m + 1;
             }
             // no copy may still be in flight when the block exits
@@ -374,35 +408,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const int s = m & 1;
             const ChunkParams *par = &params[m % 3];
             uint8_t *st = sm + s * STG;
-            uint8_t *P = sm + OFF_P + s * 8192;
-            uint8_t *tbg = sm + OFF_TBG;
-            // chain finished chunk m-2: its P buffer, U buffer and W slots are free
+            // chain finished chunk m-2: its stage's W slots and U buffer are free
             if (m >= 2) group_wait(&bars[B_KSFREE + s], ((m - 2) >> 1) & 1, E_KSFREE, 1, KS_THREADS, lwarp, true);
             group_wait(&bars[B_FULL + s], (m >> 1) & 1, E_FULL, 1, KS_THREADS, lwarp, true);
             if (!sync_ok(1, KS_THREADS, leader, kcnt)) break;
-            if (leader) {
-                // [Q ; K] K^T: lanes 0..63 of the result hold Q K^T
-                tc_fence_after();
-                const uint32_t a0 = smem_u32(st);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk >> 2) * S_KB + (kk & 3) * 32;
-                    umma_f16_ss(tmem + TM_G, sdesc_sw128(a0 + S_Q + off, 16, 1024),
-                                sdesc_sw128(a0 + S_K + off, 16, 1024), IDESC_BF_KK, kk > 0);
-                }
-                umma_commit(&bars[B_G]);
-                pend = B_G; pend_par = m & 1;
-            }
-            __syncwarp();
-            // gates of the next chunk meanwhile
-            if (scan_warp && m + 1 < NC) {
-                tc::scan_gates(&params[(m + 1) % 3], ga0, ga1, gb0, gb1, lane, min(C, T - (m + 1) * C));
-                tc::fetch_gates(p.alpha, p.beta, b, T, H, h, (m + 2) * C, lane, m + 2 < NC, ga0, ga1, gb0, gb1);
-            }
-            group_wait(&bars[B_G], m & 1, E_GRAM, 1, KS_THREADS, lwarp, false);
-            if (!sync_ok(1, KS_THREADS, leader, kcnt)) break;
-            tc_fence_after();
-            // in-place fp16 operands: Q -> e^{g_r} Q, K -> K, V -> beta_r V
+            // in-place fp16 operands: Q -> e^{g_r} Q, K -> K, V -> V
 #pragma unroll
             for (int it = 0; it < 10; ++it) {
                 const int u = kt + 256 * (it & 1);          // 16-byte chunk within one 8 KB tile
@@ -411,7 +421,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                                    : tile == 3 ? S_KB + S_K : S_V;
                 uint8_t *addr = st + off + (u << 4);
                 const int row = u >> 3;
-                const float sc = tile < 2 ? par->eg[row] : (tile == 4 ? par->bet[row] : 1.f);
+                const float sc = tile < 2 ? par->eg[row] : 1.f;
                 uint4 w = *reinterpret_cast<uint4 *>(addr);
                 const float2 f0 = unpack_bf2(w.x), f1 = unpack_bf2(w.y), f2 = unpack_bf2(w.z), f3 = unpack_bf2(w.w);
                 w.x = pack_h2(f0.x * sc, f0.y * sc);
@@ -420,55 +430,15 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 w.w = pack_h2(f3.x * sc, f3.y * sc);
                 *reinterpret_cast<uint4 *>(addr) = w;
             }
-            if (sp < 2) {
-                // P rows (TMEM lanes 0..63): decayed causal scores
-                const int r = 32 * sp + lane;
-                uint32_t pk[16];
-                if (hf > sp) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) pk[j] = 0u;
-                } else {
-                    uint32_t xr[32];
-                    tmem_ld32(tmem + ((uint32_t)(32 * sp) << 16) + TM_G + 32 * hf, xr);
-                    float gam[32];
-                    tc::decay_row(par, r, hf, hf == sp, gam);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; j += 2)
-                        pk[j >> 1] = pack_h2(gam[j] * __uint_as_float(xr[j]), gam[j + 1] * __uint_as_float(xr[j + 1]));
-                }
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj)
-                    *reinterpret_cast<uint4 *>(P + sw128_off(r, 4 * hf + jj)) =
-                        make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
-            } else {
-                // T diag(beta e^g): the 128 threads of sub-partitions 2, 3 (warps 2, 3,
-                // 6, 7), 4 chunks each, same swizzled positions
-                const int t2 = 64 * hf + 32 * (sp - 2) + lane;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int cidx = t2 + 128 * q, r = cidx >> 3, jp = cidx & 7;
-                    const int j = jp ^ (r & 7);                 // logical 8-column group
-                    const uint32_t off = (uint32_t)(r * 128 + jp * 16);
-                    uint4 w = *reinterpret_cast<const uint4 *>(st + S_T + off);
-                    const float2 f0 = unpack_h2(w.x), f1 = unpack_h2(w.y), f2 = unpack_h2(w.z), f3 = unpack_h2(w.w);
-                    const int c0 = 8 * j;
-                    w.x = pack_h2(f0.x * par->bet[c0 + 0] * par->eg[c0 + 0], f0.y * par->bet[c0 + 1] * par->eg[c0 + 1]);
-                    w.y = pack_h2(f1.x * par->bet[c0 + 2] * par->eg[c0 + 2], f1.y * par->bet[c0 + 3] * par->eg[c0 + 3]);
-                    w.z = pack_h2(f2.x * par->bet[c0 + 4] * par->eg[c0 + 4], f2.y * par->bet[c0 + 5] * par->eg[c0 + 5]);
-                    w.w = pack_h2(f3.x * par->bet[c0 + 6] * par->eg[c0 + 6], f3.y * par->bet[c0 + 7] * par->eg[c0 + 7]);
-                    *reinterpret_cast<uint4 *>(tbg + off) = w;
-                }
-            }
             fence_proxy_async_smem();
             tc_fence_before();
             if (!sync_ok(1, KS_THREADS, leader, kcnt)) break;
             if (leader) {
                 tc_fence_after();
-                const uint32_t at = smem_u32(st + S_T), av = smem_u32(st + S_V);
-                const uint32_t ag = smem_u32(tbg), ak = smem_u32(st + S_K);
+                const uint32_t at = smem_u32(st + S_TB), av = smem_u32(st + S_V);
+                const uint32_t ag = smem_u32(st + S_TBG), ak = smem_u32(st + S_K);
                 const uint32_t du = tmem + (s ? TM_U1 : TM_U0);
-                // U = T (beta V): [T ; next rows] x V (MN-major), K = 64 tokens
+                // U = T diag(beta) V: [T diag(beta) ; next rows] x V (MN-major), K = 64 tokens
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     umma_f16_ss(du, sdesc_sw128(at + kk * 32, 16, 1024),
@@ -482,6 +452,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 pend = B_UW; pend_par = m & 1;
             }
             __syncwarp();
+            // gates of the next chunk meanwhile
+            if (scan_warp && m + 1 < NC) {
+                tc::scan_gates(&params[(m + 1) % 3], ga0, ga1, gb0, gb1, lane, min(C, T - (m + 1) * C));
+                tc::fetch_gates(p.alpha, p.beta, b, T, H, h, (m + 2) * C, lane, m + 2 < NC, ga0, ga1, gb0, gb1);
+            }
             group_wait(&bars[B_UW], m & 1, E_UW, 1, KS_THREADS, lwarp, false);
             if (!sync_ok(1, KS_THREADS, leader, kcnt)) break;
             tc_fence_after();
@@ -495,6 +470,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 st_row_f16(st + hf * S_KB + S_W, r, x);
             }
             fence_proxy_async_smem();
+            tc_fence_before();
             named_bar(1, KS_THREADS);
             if (leader) {
                 pend = -1;
@@ -572,7 +548,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const int s = n & 1;
             const ChunkParams *par = &params[n % 3];
             uint8_t *st = sm + s * STG;
-            uint8_t *P = sm + OFF_P + s * 8192;
             const uint32_t xcol = s ? TM_X1 : TM_X0;
             group_wait(&bars[B_KSREADY + s], (n >> 1) & 1, E_KSREADY, 2, CH_THREADS, iwarp, true);
             if (n > 0) group_wait(&bars[B_H], (n - 1) & 1, E_H, 2, CH_THREADS, iwarp, false);
@@ -636,7 +611,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             // MMAs, the loop exits at the next 128-thread barrier
             if (sync_ok(3, 64, issuer, dcnt) && issuer) {
                 tc_fence_after();
-                const uint32_t ap = smem_u32(P) - 8192, bd = smem_u32(ds);
+                const uint32_t ap = smem_u32(st + S_P) - 8192, bd = smem_u32(ds);
                 const uint32_t ak = smem_u32(st + S_K), bdp = smem_u32(dps);
                 // O: [preceding rows ; P] Delta -> lanes 64..127 += P Delta
 #pragma unroll
@@ -713,13 +688,14 @@ bool make_map_bthd(CUtensorMap *m, const void *ptr, int B, int T, int H, int D) 
     return r == CUDA_SUCCESS;
 }
 
-// T workspace [rows, 64] fp16 viewed as 4-D (64, 1, rows, 1); box 64 x 1 x 64 x 1.
+// Workspace [rows, 64] fp16 viewed as 4-D (64, 1, rows, 1); box 64 x 1 x 192 x 1
+// (the three matrices of one chunk-head).
 bool make_map_t(CUtensorMap *m, const void *ptr, size_t rows) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[4] = {64, 1, (cuuint64_t)rows, 1};
     cuuint64_t strides[3] = {128, 128, (cuuint64_t)rows * 128};
-    cuuint32_t box[4] = {64, 1, (cuuint32_t)C, 1};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)WS_ROWS, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -744,7 +720,7 @@ int tc_default_slices(const FwdParams &p) { return p.dv / DVS; }
 
 size_t tc_workspace_bytes(const FwdParams &p) {
     const size_t nc = (size_t)(p.T + C - 1) / C;
-    return (size_t)p.B * p.H * nc * 64 * 64 * sizeof(__half);
+    return (size_t)p.B * p.H * nc * WS_CHUNK_BYTES;
 }
 
 cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, const char **why) {
@@ -752,7 +728,7 @@ cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, 
     CUtensorMap mq, mk, mv, mt;
     if (!make_map_bthd(&mq, p.q, p.B, p.T, p.H, p.dk) || !make_map_bthd(&mk, p.k, p.B, p.T, p.H, p.dk) ||
         !make_map_bthd(&mv, p.v, p.B, p.T, p.H, p.dv) ||
-        !make_map_t(&mt, workspace, (size_t)p.B * p.H * NC * 64)) {
+        !make_map_t(&mt, workspace, (size_t)p.B * p.H * NC * WS_ROWS)) {
         *why = "(tensor map encoding failed)";
         return cudaErrorInvalidValue;
     }
@@ -768,9 +744,9 @@ cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, 
     K1Params k1;
     k1.B = p.B; k1.T = p.T; k1.H = p.H; k1.NC = NC;
     k1.alpha = p.alpha; k1.beta = p.beta;
-    k1.Tws = reinterpret_cast<__half *>(workspace);
+    k1.ws = reinterpret_cast<uint8_t *>(workspace);
     k1.neumann = p.mode == GDN_INV_NEUMANN; k1.N = p.N;
-    keyside_kernel<<<dim3(NC, p.H, p.B), K1_THREADS, K1_SMEM, stream>>>(mk, k1);
+    keyside_kernel<<<dim3(NC, p.H, p.B), K1_THREADS, K1_SMEM, stream>>>(mq, mk, k1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     K2Params k2;

@@ -33,7 +33,7 @@ MODES = {"exact": GDN_INV_EXACT, "neumann": GDN_INV_NEUMANN}
 
 EXPORTS = ("gdn_chunk_fwd", "gdn_select_kernel", "gdn_workspace_bytes", "gdn_device_check",
            "gdn_status_string", "gdn_last_error", "gdn_abi_version", "gdn_chunk_fwd_static_scratch")
-STATIC_SCRATCH_BYTES = 8 << 20   # GDN_STATIC_SCRATCH_BYTES
+STATIC_SCRATCH_BYTES = 24 << 20   # GDN_STATIC_SCRATCH_BYTES
 
 
 class GDNError(RuntimeError):

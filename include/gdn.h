@@ -47,8 +47,9 @@
  * Ownership.  Every pointer is a DEVICE pointer owned by the caller, who
  * allocates inputs, outputs and the workspace.  The library allocates no
  * device memory and keeps no state between calls.  The tensor-core kernel
- * stores each chunk's inverse T (fp16, 8 KB per chunk and head) in the
- * workspace between its two launches; gdn_workspace_bytes() gives the size.
+ * keeps, per chunk and head, T diag(beta), T diag(beta e^g) and the decayed
+ * causal scores P (fp16, 24 KB) in the workspace between its two launches;
+ * gdn_workspace_bytes() gives the size.
  *
  * Execution and errors.  gdn_chunk_fwd validates its arguments on the host
  * and returns an error before launching anything (nothing is written) when
@@ -156,8 +157,8 @@ GDN_API const char *gdn_last_error(void);
 GDN_API int32_t gdn_abi_version(void);
 
 /* Size of the fixed device scratch array of gdn_chunk_fwd_static_scratch:
- * 8 MiB = 1024 chunk-heads of one 64 x 64 fp16 T matrix each. */
-#define GDN_STATIC_SCRATCH_BYTES (8ull << 20)
+ * 24 MiB = 1024 chunk-heads of three 64 x 64 fp16 matrices each. */
+#define GDN_STATIC_SCRATCH_BYTES (24ull << 20)
 
 /* gdn_chunk_fwd on the tensor-core kernel, with a fixed scratch array inside
  * the library in place of args->workspace.  The pages have no counterpart:
@@ -172,9 +173,9 @@ GDN_API int32_t gdn_abi_version(void);
  * Arguments as gdn_chunk_fwd, except: args->workspace must be NULL and
  * args->workspace_bytes 0; the arguments must select the tensor-core kernel
  * (kernel AUTO or TC with a supported shape), else GDN_ERR_UNSUPPORTED; and
- * B * H * ceil(T / 64) * 8192 must be <= GDN_STATIC_SCRATCH_BYTES, else
+ * B * H * ceil(T / 64) * 24576 must be <= GDN_STATIC_SCRATCH_BYTES, else
  * GDN_ERR_INVALID_ARG with the needed size in gdn_last_error().  Nothing in
- * the scratch has to start at zero: the key-side kernel writes every T entry
+ * the scratch has to start at zero: the key-side kernel writes every entry
  * the chain kernel reads, in the same call.
  *
  * Set-up: the first call on each device, with that device current, looks up

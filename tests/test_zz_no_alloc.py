@@ -23,7 +23,7 @@ def _args(w, d, o, S):
 
 def test_static_scratch_rejects_oversize_and_workspace():
     # host-side checks: they return before any device call
-    w = workload("gdn_bf16", B=2, H=16, T=4096)          # 2048 chunk-heads: 16 MiB of T
+    w = workload("gdn_bf16", B=2, H=16, T=4096)          # 2048 chunk-heads: 48 MiB
     fake = 1 << 20
     a = G.make_args(B=w.B, T=w.T, H=w.H, dk=128, dv=128, chunk=64, io_dtype=1, o_dtype=0,
                     q=fake, k=fake, v=fake, alpha=fake, beta=fake, o=2 * fake, S_T=3 * fake,
@@ -31,9 +31,9 @@ def test_static_scratch_rejects_oversize_and_workspace():
     s = G.lib().gdn_chunk_fwd_static_scratch(ctypes.byref(a), None)
     assert s == G.GDN_ERR_INVALID_ARG
     msg = G.last_error()
-    assert "scratch" in msg and str(16 << 20) in msg, msg
+    assert "scratch" in msg and str(48 << 20) in msg, msg
     a.B = 1                                                  # fits, but a workspace is passed
-    a.workspace, a.workspace_bytes = 4 * fake, 8 << 20
+    a.workspace, a.workspace_bytes = 4 * fake, 24 << 20
     assert G.lib().gdn_chunk_fwd_static_scratch(ctypes.byref(a), None) == G.GDN_ERR_INVALID_ARG
     a.workspace, a.workspace_bytes = None, 0
     a.kernel = 1                                             # SIMT is not this entry point's kernel
@@ -44,7 +44,7 @@ def test_static_scratch_rejects_oversize_and_workspace():
 def test_static_scratch_matches_workspace_entry():
     # 1 x 16 heads x 64 chunks = 1024 chunk-heads: exactly the fixed maximum
     w = workload("gdn_bf16", B=1, H=16, T=4096, s0_std=0.02)
-    assert w.B * w.H * (w.T // 64) * 8192 == G.STATIC_SCRATCH_BYTES
+    assert w.B * w.H * (w.T // 64) * 24576 == G.STATIC_SCRATCH_BYTES
     x = make_inputs(w, seed=21)
     d = {k: (None if v is None else v.cuda()) for k, v in x.items()}
     o_ref, s_ref = gdn.chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S0=d["S0"],
