@@ -66,7 +66,7 @@ constexpr int kNeumannMaxN = 15;
 constexpr unsigned long long kWaitLimit = 4000000000ull;   // ~2 s at the boost clock
 
 // error codes recorded in g_tc_error (first one wins)
-enum { E_FULL = 1, E_EMPTY, E_KSREADY, E_KSFREE, E_GRAM, E_UW, E_X, E_H, E_K1_TMA, E_K1_MMA };
+enum { E_FULL = 1, E_EMPTY, E_KSREADY, E_KSFREE, E_O, E_UW, E_X, E_H, E_K1_TMA, E_K1_MMA };
 
 constexpr uint32_t IDESC_BF_KK = idesc_f16(128, 64, 1, 1, 0, 0);    // bf16, K-major x K-major, N 64
 constexpr uint32_t IDESC_KM64 = idesc_f16(128, 64, 0, 0, 0, 1);     // fp16, K-major x MN-major, N 64
@@ -269,7 +269,8 @@ constexpr uint32_t OFF_DPS = OFF_DS + 8192;            // e^{g_C - g} Delta fp16
 constexpr uint32_t OFF_PAR = OFF_DPS + 8192;
 constexpr uint32_t PAR_BYTES = (sizeof(ChunkParams) + 15) & ~15u;
 constexpr uint32_t OFF_BAR = OFF_PAR + 3 * PAR_BYTES;   // params ring of 3
-enum { B_FULL = 0, B_EMPTY = 2, B_KSREADY = 4, B_KSFREE = 6, B_UW = 8, B_X = 9, B_H = 10, N_BARS = 11 };
+enum { B_FULL = 0, B_EMPTY = 2, B_KSREADY = 4, B_KSFREE = 6, B_UW = 8, B_X = 9, B_H = 10, B_O = 11,
+       N_BARS = 13 };
 constexpr uint32_t OFF_MISC = OFF_BAR + N_BARS * 8;     // tmem slot, abort flag, group slots
 constexpr uint32_t SMEM_USED = OFF_MISC + 32;
 constexpr uint32_t K2_SMEM = SMEM_USED + 1024;
@@ -343,6 +344,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         mbar_init(&bars[B_UW], 1);
         mbar_init(&bars[B_X], 1);
         mbar_init(&bars[B_H], 1);
+        mbar_init(&bars[B_O], 1);
+        mbar_init(&bars[B_O + 1], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -549,10 +552,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const ChunkParams *par = &params[n % 3];
             uint8_t *st = sm + s * STG;
             const uint32_t xcol = s ? TM_X1 : TM_X0;
-            group_wait(&bars[B_KSREADY + s], (n >> 1) & 1, E_KSREADY, 2, CH_THREADS, iwarp, true);
+            // state update of the previous chunk complete (its output rows may still be running)
             if (n > 0) group_wait(&bars[B_H], (n - 1) & 1, E_H, 2, CH_THREADS, iwarp, false);
             tc_fence_after();
-            // ---- h <- e^{g_C} h in TMEM (issued first), h -> fp16 operand
+            // ---- h <- e^{g_C} h in TMEM (issued first), h -> fp16 operand.  The
+            // gates of chunk n were scanned before the key side released chunk n-1.
             {
                 float x[64];
                 tmem_ld64(tmem + lane_base + TM_H, x);
@@ -569,6 +573,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             }
             fence_proxy_async_smem();
             tc_fence_before();
+            group_wait(&bars[B_KSREADY + s], (n >> 1) & 1, E_KSREADY, 2, CH_THREADS, iwarp, false);
             if (!sync_ok(2, CH_THREADS, issuer, ccnt)) { done = false; break; }
             if (issuer) {
                 // [-W ; Q'] h16: lanes 0..63 -W h, lanes 64..127 Q'h
@@ -586,7 +591,12 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             __syncwarp();
             if (!rowpart) {
                 // sub-partitions 2, 3: output rows of the previous chunk, off the chain
-                if (n > 0) store_o(n - 1);
+                if (n > 0 && mbar_wait(&bars[B_O + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort_flag, E_O, lim)) {
+                    __syncwarp();
+                    tc_fence_after();
+                    store_o(n - 1);
+                }
+                __syncwarp();
                 continue;
             }
             group_wait(&bars[B_X], n & 1, E_X, 3, 64, iwarp, false);
@@ -613,29 +623,35 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 tc_fence_after();
                 const uint32_t ap = smem_u32(st + S_P) - 8192, bd = smem_u32(ds);
                 const uint32_t ak = smem_u32(st + S_K), bdp = smem_u32(dps);
+                // h += K^T (e^{g_C - g} Delta) first: the next chunk waits on it alone.
+                // K^T as MN-major A over the two key blocks.
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16_ss(tmem + TM_H, sdesc_sw128(ak + kk * 2048, S_KB, 1024),
+                                sdesc_sw128(bdp + kk * 2048, 8192, 1024), IDESC_MM64, 1);
+                umma_commit(&bars[B_H]);
                 // O: [preceding rows ; P] Delta -> lanes 64..127 += P Delta
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     umma_f16_ss(tmem + xcol, sdesc_sw128(ap + kk * 32, 16, 1024),
                                 sdesc_sw128(bd + kk * 2048, 8192, 1024), IDESC_KM64, 1);
-                // h += K^T (e^{g_C - g} Delta): K^T as MN-major A over the two key blocks
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16_ss(tmem + TM_H, sdesc_sw128(ak + kk * 2048, S_KB, 1024),
-                                sdesc_sw128(bdp + kk * 2048, 8192, 1024), IDESC_MM64, 1);
+                umma_commit(&bars[B_O + s]);
                 umma_commit(&bars[B_EMPTY + s]);
                 umma_commit(&bars[B_KSFREE + s]);
-                umma_commit(&bars[B_H]);
-                pend = B_H; pend_par = n & 1;
+                pend = B_O + s; pend_par = (n >> 1) & 1;
             }
             __syncwarp();
         }
         if (done && NC > 0) {
             group_wait(&bars[B_H], (NC - 1) & 1, E_H, 2, CH_THREADS, iwarp, false);
             if (sync_ok(2, CH_THREADS, issuer, ccnt)) {
-                if (issuer) pend = -1;
                 tc_fence_after();
-                if (!rowpart) store_o(NC - 1);
+                if (!rowpart && mbar_wait(&bars[B_O + ((NC - 1) & 1)], ((NC - 1) >> 1) & 1, abort_flag, E_O, lim)) {
+                    __syncwarp();
+                    tc_fence_after();
+                    store_o(NC - 1);
+                }
+                __syncwarp();
                 if (p.S_T) {
                     float x[64];
                     tmem_ld64(tmem + lane_base + TM_H, x);
