@@ -81,11 +81,12 @@ constexpr int WS_ROWS = 192;                           // rows of 128 bytes per 
 constexpr size_t WS_CHUNK_BYTES = (size_t)WS_ROWS * 128;
 
 constexpr int K1_THREADS = 256;
-constexpr uint32_t K1_OFF_QK = 0;                      // per key block kb: [Q | K] at kb * 16 KB
-constexpr uint32_t K1_OFF_YB = 0;                      // inverse scratch (8 KB), reuses the tiles
-constexpr uint32_t K1_OFF_LB = 32768;                  // L fp32
+constexpr int K1_BLOCKS_PER_SM = 3;
 constexpr uint32_t K1_MAT = 64 * LSTR * 4;
-constexpr uint32_t K1_OFF_TB = K1_OFF_LB + K1_MAT;
+constexpr uint32_t K1_OFF_QK = 0;                      // per key block kb: [Q | K] at kb * 16 KB
+constexpr uint32_t K1_OFF_LB = 0;                      // L fp32 and the inverse scratch reuse the
+constexpr uint32_t K1_OFF_YB = K1_MAT;                 // tiles once the Gram MMA has read them
+constexpr uint32_t K1_OFF_TB = 32768;
 constexpr uint32_t K1_OFF_PAR = K1_OFF_TB + K1_MAT;
 constexpr uint32_t K1_OFF_BAR = K1_OFF_PAR + ((sizeof(ChunkParams) + 15) & ~15u);
 constexpr uint32_t K1_SMEM = K1_OFF_BAR + 64 + 1024;  // + base alignment slack
@@ -99,7 +100,7 @@ struct K1Params {
 
 // One CTA per (chunk, head, batch).  [Q ; K] K^T in one MMA: TMEM lanes 0..63
 // hold Q K^T (-> P), lanes 64..127 hold K K^T (-> L -> T).
-__global__ void __launch_bounds__(K1_THREADS)
+__global__ void __launch_bounds__(K1_THREADS, K1_BLOCKS_PER_SM)
 keyside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const K1Params p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -115,11 +116,18 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + K1_OFF_BAR + 20);
     uint8_t *ws = p.ws + ((((size_t)b * p.H + h) * p.NC + n) * WS_CHUNK_BYTES);
 
+    const int t0 = n * C;
     if (tid == 0) {
         mbar_init(&bars[0], 1);
         mbar_init(&bars[1], 1);
         *abort_flag = 0;
         fence_mbar_init();
+        // the tiles first: their latency overlaps the set-up below
+        mbar_arrive_expect_tx(&bars[0], 32768);
+        tma_load_4d(sm + K1_OFF_QK, &tm_q, &bars[0], 0, h, t0, b);
+        tma_load_4d(sm + K1_OFF_QK + 8192, &tm_k, &bars[0], 0, h, t0, b);
+        tma_load_4d(sm + K1_OFF_QK + 16384, &tm_q, &bars[0], 64, h, t0, b);
+        tma_load_4d(sm + K1_OFF_QK + 24576, &tm_k, &bars[0], 64, h, t0, b);
     }
     __syncwarp();
     if (warp == 0) {
@@ -132,17 +140,6 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     block_sync();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int t0 = n * C;
-    if (tid == 0) {
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        mbar_arrive_expect_tx(&bars[0], 32768);
-        tma_load_4d(sm + K1_OFF_QK, &tm_q, &bars[0], 0, h, t0, b);
-        tma_load_4d(sm + K1_OFF_QK + 8192, &tm_k, &bars[0], 0, h, t0, b);
-        tma_load_4d(sm + K1_OFF_QK + 16384, &tm_q, &bars[0], 64, h, t0, b);
-        tma_load_4d(sm + K1_OFF_QK + 24576, &tm_k, &bars[0], 64, h, t0, b);
-    }
-    __syncwarp();
     if (warp == 1) {
         float a0, a1, b0, b1;
         tc::fetch_gates(p.alpha, p.beta, b, p.T, p.H, h, t0, lane, true, a0, a1, b0, b1);
@@ -258,15 +255,20 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
 constexpr int K2_THREADS = 448;    // 14 warps
 constexpr int KS_THREADS = 256, CH_THREADS = 128;
-// stage (x2): per 64-column key block kb: [W | Q | K] at kb * 24 KB; V, T after
-//   then V, then the workspace rows of the chunk: T diag(beta), T diag(beta e^g), P
+// stage (x2): per 64-column key block kb: [W | Q | K] at kb * 24 KB, then V,
+//   then T diag(beta), T diag(beta e^g) and P of the chunk
 constexpr uint32_t STG = 81920;
 constexpr uint32_t S_W = 0, S_Q = 8192, S_K = 16384, S_KB = 24576, S_V = 49152;
 constexpr uint32_t S_TB = 57344, S_TBG = 65536, S_P = 73728;
+constexpr uint32_t STAGE_TX = 65536;                   // bytes the producer loads per stage
+// Every M = 128 MMA whose A operand has only 64 real rows also reads the 8 KB
+// next to them; the lanes those rows produce are never read.  The neighbours
+// all lie in the same stage and are not rewritten while the stage is in use:
+// U reads T diag(beta) + T diag(beta e^g), W reads T diag(beta e^g) + P, the
+// output MMA T diag(beta e^g) + P.
 constexpr uint32_t OFF_HS = 2 * STG;                   // h fp16, 128 rows
-constexpr uint32_t OFF_DS = OFF_HS + 16384;            // Delta fp16
-constexpr uint32_t OFF_DPS = OFF_DS + 8192;            // e^{g_C - g} Delta fp16
-constexpr uint32_t OFF_PAR = OFF_DPS + 8192;
+constexpr uint32_t OFF_DS = OFF_HS + 16384;            // Delta fp16 x 2
+constexpr uint32_t OFF_PAR = OFF_DS + 2 * 8192;
 constexpr uint32_t PAR_BYTES = (sizeof(ChunkParams) + 15) & ~15u;
 constexpr uint32_t OFF_BAR = OFF_PAR + 3 * PAR_BYTES;   // params ring of 3
 enum { B_FULL = 0, B_EMPTY = 2, B_KSREADY = 4, B_KSFREE = 6, B_UW = 8, B_X = 9, B_H = 10, B_O = 11,
@@ -275,7 +277,8 @@ constexpr uint32_t OFF_MISC = OFF_BAR + N_BARS * 8;     // tmem slot, abort flag
 constexpr uint32_t SMEM_USED = OFF_MISC + 32;
 constexpr uint32_t K2_SMEM = SMEM_USED + 1024;
 static_assert(K2_SMEM <= 232448, "shared memory budget of one sm_100 block");
-static_assert(K1_SMEM * 3 <= 233472, "three key-side blocks per SM");
+static_assert(K1_SMEM * K1_BLOCKS_PER_SM <= 233472, "key-side blocks per SM");
+static_assert(K1_OFF_YB + 8192 <= K1_OFF_TB, "L and the inverse scratch fit in the tile region");
 
 // TMEM columns
 constexpr uint32_t TM_U0 = 0, TM_U1 = 64, TM_W = 128, TM_X0 = 256, TM_X1 = 320, TM_H = 384;
@@ -369,10 +372,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             int issued = 0;
             for (int m = 0; m < NC; ++m) {
                 const int s = m & 1;
+                const int wrow = (((b * H) + h) * NC + m) * WS_ROWS;
                 if (m >= 2 && !mbar_wait(&bars[B_EMPTY + s], ((m - 2) >> 1) & 1, abort_flag, E_EMPTY, lim))
                     break;
                 uint64_t *fb = &bars[B_FULL + s];
-                mbar_arrive_expect_tx(fb, 65536);
+                mbar_arrive_expect_tx(fb, STAGE_TX);
                 uint8_t *st = sm + s * STG;
                 const int t0 = m * C;
                 tma_load_4d(st + S_Q, &tm_q, fb, 0, h, t0, b);
@@ -380,7 +384,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 tma_load_4d(st + S_K, &tm_k, fb, 0, h, t0, b);
                 tma_load_4d(st + S_KB + S_K, &tm_k, fb, 64, h, t0, b);
                 tma_load_4d(st + S_V, &tm_v, fb, v0, h, t0, b);
-                tma_load_4d(st + S_TB, &tm_t, fb, 0, 0, (((b * H) + h) * NC + m) * WS_ROWS, 0);
+                tma_load_4d(st + S_TB, &tm_t, fb, 0, 0, wrow, 0);
+                tma_load_4d(st + S_TBG, &tm_t, fb, 0, 0, wrow + 64, 0);
+                tma_load_4d(st + S_P, &tm_t, fb, 0, 0, wrow + 128, 0);
                 issued = m + 1;
             }
             // no copy may still be in flight when the block exits
@@ -471,6 +477,23 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
                 for (int j = 0; j < 64; ++j) x[j] = -x[j];
                 st_row_f16(st + hf * S_KB + S_W, r, x);
+            } else {
+                // W has read K: K -> diag(e^{g_C - g}) K in place for the state update
+                const int t2 = 64 * hf + 32 * (sp - 2) + lane;
+#pragma unroll
+                for (int it = 0; it < 8; ++it) {
+                    const int idx = t2 + 128 * it;               // 16-byte chunk of the two K blocks
+                    const int u = idx & 511;
+                    uint8_t *addr = st + (idx >> 9) * S_KB + S_K + (u << 4);
+                    const float sc = par->egc[u >> 3];
+                    uint4 w = *reinterpret_cast<uint4 *>(addr);
+                    const float2 f0 = unpack_h2(w.x), f1 = unpack_h2(w.y), f2 = unpack_h2(w.z), f3 = unpack_h2(w.w);
+                    w.x = pack_h2(f0.x * sc, f0.y * sc);
+                    w.y = pack_h2(f1.x * sc, f1.y * sc);
+                    w.z = pack_h2(f2.x * sc, f2.y * sc);
+                    w.w = pack_h2(f3.x * sc, f3.y * sc);
+                    *reinterpret_cast<uint4 *>(addr) = w;
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -493,8 +516,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const bool issuer = (ct == 64);    // warp 12 lane 0, sub-partition 0: MMA issue
         const bool iwarp = (ct >> 5) == 2; // warp 12 polls the chain's waits
         uint8_t *hs = sm + OFF_HS;
-        uint8_t *ds = sm + OFF_DS;
-        uint8_t *dps = sm + OFF_DPS;
         const size_t bh = (size_t)b * H + h;
         {
             float x[64];
@@ -544,6 +565,15 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 }
             }
         };
+        // Warps 10, 11: the output rows of chunk j once its P Delta MMA is complete.
+        auto out_rows = [&](int j) {
+            if (mbar_wait(&bars[B_O + (j & 1)], (j >> 1) & 1, abort_flag, E_O, lim)) {
+                __syncwarp();
+                tc_fence_after();
+                store_o(j);
+            }
+            __syncwarp();
+        };
         int ccnt = 0, dcnt = 0;
         int pend = -1, pend_par = 0;       // issuer: last commit not yet known complete
         bool done = true;
@@ -554,9 +584,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             const uint32_t xcol = s ? TM_X1 : TM_X0;
             // state update of the previous chunk complete (its output rows may still be running)
             if (n > 0) group_wait(&bars[B_H], (n - 1) & 1, E_H, 2, CH_THREADS, iwarp, false);
+            // the gates of chunk 0 are scanned by the key side at start-up: wait for it
+            else group_wait(&bars[B_KSREADY], 0, E_KSREADY, 2, CH_THREADS, iwarp, false);
             tc_fence_after();
             // ---- h <- e^{g_C} h in TMEM (issued first), h -> fp16 operand.  The
-            // gates of chunk n were scanned before the key side released chunk n-1.
+            // gates of chunk n > 0 were scanned before the key side released chunk n-1.
             {
                 float x[64];
                 tmem_ld64(tmem + lane_base + TM_H, x);
@@ -573,7 +605,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            group_wait(&bars[B_KSREADY + s], (n >> 1) & 1, E_KSREADY, 2, CH_THREADS, iwarp, false);
+            if (n > 0) group_wait(&bars[B_KSREADY + s], (n >> 1) & 1, E_KSREADY, 2, CH_THREADS, iwarp, false);
             if (!sync_ok(2, CH_THREADS, issuer, ccnt)) { done = false; break; }
             if (issuer) {
                 // [-W ; Q'] h16: lanes 0..63 -W h, lanes 64..127 Q'h
@@ -591,12 +623,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             __syncwarp();
             if (!rowpart) {
                 // sub-partitions 2, 3: output rows of the previous chunk, off the chain
-                if (n > 0 && mbar_wait(&bars[B_O + ((n - 1) & 1)], ((n - 1) >> 1) & 1, abort_flag, E_O, lim)) {
-                    __syncwarp();
-                    tc_fence_after();
-                    store_o(n - 1);
-                }
-                __syncwarp();
+                if (n > 0) out_rows(n - 1);
                 continue;
             }
             group_wait(&bars[B_X], n & 1, E_X, 3, 64, iwarp, false);
@@ -609,11 +636,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 tmem_ld64(tmem + lane_base + (s ? TM_U1 : TM_U0), u);
 #pragma unroll
                 for (int j = 0; j < 64; ++j) x[j] += u[j];
-                st_row_f16(ds, r, x);
-                const float ec = par->egc[r];
-#pragma unroll
-                for (int j = 0; j < 64; ++j) x[j] *= ec;
-                st_row_f16(dps, r, x);
+                st_row_f16(sm + OFF_DS + s * 8192, r, x);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -621,16 +644,18 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             // MMAs, the loop exits at the next 128-thread barrier
             if (sync_ok(3, 64, issuer, dcnt) && issuer) {
                 tc_fence_after();
-                const uint32_t ap = smem_u32(st + S_P) - 8192, bd = smem_u32(ds);
-                const uint32_t ak = smem_u32(st + S_K), bdp = smem_u32(dps);
-                // h += K^T (e^{g_C - g} Delta) first: the next chunk waits on it alone.
-                // K^T as MN-major A over the two key blocks.
+                const uint32_t ak = smem_u32(st + S_K), bd = smem_u32(sm + OFF_DS + s * 8192);
+                // h += (diag(e^{g_C - g}) K)^T Delta first: the next chunk waits on it
+                // alone.  The key side rescaled K in place; K^T as MN-major A over
+                // the two key blocks.
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     umma_f16_ss(tmem + TM_H, sdesc_sw128(ak + kk * 2048, S_KB, 1024),
-                                sdesc_sw128(bdp + kk * 2048, 8192, 1024), IDESC_MM64, 1);
+                                sdesc_sw128(bd + kk * 2048, 8192, 1024), IDESC_MM64, 1);
                 umma_commit(&bars[B_H]);
-                // O: [preceding rows ; P] Delta -> lanes 64..127 += P Delta
+                // O: [preceding rows ; P] Delta -> lanes 64..127 += P Delta.  The stage and
+                // the key side's buffers are released only after these MMAs complete.
+                const uint32_t ap = smem_u32(st + S_P) - 8192;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     umma_f16_ss(tmem + xcol, sdesc_sw128(ap + kk * 32, 16, 1024),
@@ -646,12 +671,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             group_wait(&bars[B_H], (NC - 1) & 1, E_H, 2, CH_THREADS, iwarp, false);
             if (sync_ok(2, CH_THREADS, issuer, ccnt)) {
                 tc_fence_after();
-                if (!rowpart && mbar_wait(&bars[B_O + ((NC - 1) & 1)], ((NC - 1) >> 1) & 1, abort_flag, E_O, lim)) {
-                    __syncwarp();
-                    tc_fence_after();
-                    store_o(NC - 1);
-                }
-                __syncwarp();
+                if (!rowpart) out_rows(NC - 1);
                 if (p.S_T) {
                     float x[64];
                     tmem_ld64(tmem + lane_base + TM_H, x);
@@ -704,14 +724,14 @@ bool make_map_bthd(CUtensorMap *m, const void *ptr, int B, int T, int H, int D) 
     return r == CUDA_SUCCESS;
 }
 
-// Workspace [rows, 64] fp16 viewed as 4-D (64, 1, rows, 1); box 64 x 1 x 192 x 1
-// (the three matrices of one chunk-head).
+// Workspace [rows, 64] fp16 viewed as 4-D (64, 1, rows, 1); box 64 x 1 x 64 x 1
+// (one of the three matrices of a chunk-head).
 bool make_map_t(CUtensorMap *m, const void *ptr, size_t rows) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[4] = {64, 1, (cuuint64_t)rows, 1};
     cuuint64_t strides[3] = {128, 128, (cuuint64_t)rows * 128};
-    cuuint32_t box[4] = {64, 1, (cuuint32_t)WS_ROWS, 1};
+    cuuint32_t box[4] = {64, 1, 64, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

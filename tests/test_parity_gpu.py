@@ -192,3 +192,23 @@ def test_value_split_invariance(split):
     x = make_inputs(w, seed=16)
     o_ref, s_ref = run_oracle(x, w)
     _check_bf16(f"split_{split}", w, x, o_ref, s_ref, dv_split=split)
+
+
+@needs_cuda
+def test_tensor_core_repeatable_after_other_kernels():
+    """Repeated tensor-core calls, each after a SIMT call that leaves other data in
+    shared memory, give bit-identical results within the bar: no value may be read
+    before it is written, whatever a previous kernel left behind."""
+    w = workload("gdn_bf16", B=1, H=2, T=300, s0_std=0.02)
+    x = make_inputs(w, seed=16)
+    o_ref, s_ref = run_oracle(x, w)
+    first = None
+    for _ in range(6):
+        run_gpu(x, w, o_dtype=torch.float32, kernel="simt", dv_split=1)
+        o, s = run_gpu(x, w, o_dtype=torch.float32, kernel="tc")
+        if first is None:
+            first = (o, s)
+            so = stats(o, o_ref)
+            assert so["max_rel_rms"] <= TOL_BF16_REL_RMS, so
+        else:
+            assert np.array_equal(o, first[0]) and np.array_equal(s, first[1])
