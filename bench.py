@@ -104,6 +104,14 @@ def profile_traffic(kernel_name):
     return float(m_k.group(1))
 
 
+def mode_text(args):
+    if args.mode == "neumann":
+        return f"masked Neumann inverse N={args.N}"
+    if args.mode == "residual":
+        return f"masked Neumann inverse N={args.N} + {args.S} residual terms"
+    return "exact inverse"
+
+
 def max_over_ranks(ms, world, device=None):
     """Slowest rank's time: every rank contributes its own event time and all
     ranks receive the maximum (an all-reduce, so the collective is the same on
@@ -205,7 +213,8 @@ def run_gpu(args, rank, world, local_rank):
     a = gdn.make_args(B=w.B, T=w.T, H=w.H, dk=w.dk, dv=w.dv, chunk=w.chunk, io_dtype=1,
                       o_dtype=1, q=ptr(d["q"]), k=ptr(d["k"]), v=ptr(d["v"]),
                       alpha=ptr(d["alpha"]), beta=ptr(d["beta"]), S0=None, o=o.data_ptr(),
-                      S_T=S_T.data_ptr(), mode=0, kernel=0)
+                      S_T=S_T.data_ptr(), mode={"exact": 0, "neumann": 1, "residual": 2}[args.mode],
+                      neumann_N=args.N, residual_S=args.S, kernel=0)
     ws = gdn.workspace_for(a, dev)
     if ws is not None:
         a.workspace = ws.data_ptr()
@@ -263,7 +272,8 @@ def run_gpu(args, rank, world, local_rank):
                 if v is not None:
                     dev_in[k].copy_(v, non_blocking=True)
             gdn.chunk_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"],
-                          dev_in["beta"], chunk=w.chunk, o_dtype=torch.bfloat16, out=o,
+                          dev_in["beta"], chunk=w.chunk, o_dtype=torch.bfloat16, out=o, mode=args.mode,
+                          N=args.N, S=args.S,
                           S_T=S_T)
             o_host.copy_(o, non_blocking=True)
 
@@ -308,7 +318,7 @@ def run_gpu(args, rank, world, local_rank):
                     compute="bf16 q/k/v in HBM; fp16 tensor-core operands, fp32 accumulate and state",
                     data="synthetic (seeded; Gated DeltaNet layer shapes)",
                     config=dict(workload=f"{WORKLOAD}: B={w.B} H={w.H} T={w.T} dk={w.dk} "
-                                f"dv={w.dv} chunk={w.chunk} exact inverse, o bf16",
+                                f"dv={w.dv} chunk={w.chunk} {mode_text(args)}, o bf16",
                                 global_batch=w.B * world, seq_len=w.T,
                                 parallelism=f"independent batch per GPU x{world}",
                                 l2=(f"no flush: inputs+outputs {bytes_launch / 1e6:.0f} MB per step > 126 MB L2"
@@ -382,7 +392,7 @@ def run_reference(args, rank, world):
                 higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
                 data="synthetic (seeded; Gated DeltaNet layer shapes)",
                 config=dict(workload=f"{WORKLOAD}: B={w.B} H={w.H} T={w.T} dk={w.dk} "
-                            f"dv={w.dv} chunk={w.chunk} exact inverse, o bf16",
+                            f"dv={w.dv} chunk={w.chunk} {mode_text(args)}, o bf16",
                             global_batch=w.B, seq_len=w.T,
                             parallelism="CPU oracle, rank 0 only"),
                 cpu_baseline=dict(value=value, unit=UNIT, cores=cores, kind="oracle",
@@ -402,6 +412,11 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="replace the batch size B (profiler case)")
+    ap.add_argument("--mode", default="exact", choices=["exact", "neumann", "residual"],
+                    help="inverse: exact (the headline workload), masked Neumann series "
+                         "(order --N), or the series with --S residual-correction terms")
+    ap.add_argument("--N", type=int, default=3)
+    ap.add_argument("--S", type=int, default=8)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

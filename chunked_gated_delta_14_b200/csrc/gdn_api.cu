@@ -45,10 +45,12 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
         return fail(GDN_ERR_INVALID_ARG, "o_dtype %d unknown", a->o_dtype);
     if (!a->q || !a->k || !a->v || !a->o)
         return fail(GDN_ERR_INVALID_ARG, "q, k, v and o are required");
-    if (a->mode != GDN_INV_EXACT && a->mode != GDN_INV_NEUMANN)
+    if (a->mode != GDN_INV_EXACT && a->mode != GDN_INV_NEUMANN && a->mode != GDN_INV_NEUMANN_RESIDUAL)
         return fail(GDN_ERR_INVALID_ARG, "mode %d unknown", a->mode);
-    if (a->mode == GDN_INV_NEUMANN && (a->neumann_N < 0 || a->neumann_N > a->chunk - 1))
+    if (a->mode != GDN_INV_EXACT && (a->neumann_N < 0 || a->neumann_N > a->chunk - 1))
         return fail(GDN_ERR_INVALID_ARG, "neumann_N must be in [0, chunk-1] (got %d)", a->neumann_N);
+    if (a->mode == GDN_INV_NEUMANN_RESIDUAL && (a->residual_S < 0 || a->residual_S > 64))
+        return fail(GDN_ERR_INVALID_ARG, "residual_S must be in [0, 64] (got %d)", a->residual_S);
     if (a->alpha_per_channel && !a->alpha)
         return fail(GDN_ERR_INVALID_ARG, "alpha_per_channel needs alpha");
     if (a->alpha_per_channel != 0 && a->alpha_per_channel != 1)
@@ -82,7 +84,8 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
     p.alpha = a->alpha; p.alpha_pc = a->alpha_per_channel; p.beta = a->beta;
     p.precond = a->precond; p.rho_decay = a->rho_decay; p.rho_eps = a->rho_eps;
     p.erase = a->erase; p.write = a->write; p.S0 = a->S0; p.o = a->o; p.S_T = a->S_T;
-    p.mode = a->mode; p.N = a->mode == GDN_INV_NEUMANN ? a->neumann_N : 0;
+    p.mode = a->mode; p.N = a->mode != GDN_INV_EXACT ? a->neumann_N : 0;
+    p.S = a->mode == GDN_INV_NEUMANN_RESIDUAL ? a->residual_S : 0;
     p.general = general;
 
     const char *why = "";
@@ -106,6 +109,10 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
         if (!gdn::tc_supports(p, &why))
             return fail(GDN_ERR_UNSUPPORTED, "tensor-core kernel: %s", why);
     } else {
+        if (p.mode == GDN_INV_NEUMANN_RESIDUAL)
+            return fail(GDN_ERR_UNSUPPORTED,
+                        "residual correction runs on the tensor-core kernel only (bf16 q/k/v, scalar "
+                        "decay, chunk 64, dk 128)%s%s", why[0] ? ": " : "", why);
         // SIMT: widest value slice that fits shared memory, at least
         // ~one block per SM where the problem allows it.
         int slices = a->dv_split;

@@ -25,6 +25,7 @@ struct FwdParams {
     void *o;
     float *S_T;
     int mode, N;
+    int S;              // residual-correction terms (GDN_INV_NEUMANN_RESIDUAL)
     int general;        // two-gate rule (per-channel decay / gates / preconditioner)
 };
 

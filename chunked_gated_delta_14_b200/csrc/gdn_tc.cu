@@ -90,12 +90,16 @@ constexpr uint32_t K1_OFF_TB = 32768;
 constexpr uint32_t K1_OFF_PAR = K1_OFF_TB + K1_MAT;
 constexpr uint32_t K1_OFF_BAR = K1_OFF_PAR + ((sizeof(ChunkParams) + 15) & ~15u);
 constexpr uint32_t K1_SMEM = K1_OFF_BAR + 64 + 1024;  // + base alignment slack
+// residual correction: three more 64 x LSTR fp32 matrices (E, R ping-pong)
+constexpr uint32_t K1_OFF_RES = K1_OFF_BAR + 64;
+constexpr uint32_t K1_SMEM_RES = K1_OFF_RES + 3 * K1_MAT + 1024;
 
 struct K1Params {
     int B, T, H, NC;
     const float *alpha, *beta;
     uint8_t *ws;
-    int neumann, N;
+    int neumann, N;     // neumann: 1 truncated series, 2 series + residual correction
+    int S;              // residual-correction terms
 };
 
 // One CTA per (chunk, head, batch).  [Q ; K] K^T in one MMA: TMEM lanes 0..63
@@ -219,12 +223,17 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         named_bar(1, K1_THREADS);
         if (p.neumann) tc::invert_neumann(Lb, Tb, Yb, tid, p.N, 1);
         else tc::invert_exact(Lb, Tb, Yb, tid, 1);
+        const float *Tsrc = Tb;
+        if (p.neumann == 2) {
+            float *res = reinterpret_cast<float *>(sm + K1_OFF_RES);
+            Tsrc = tc::residual_correct(Lb, Tb, res, res + 64 * LSTR, res + 2 * 64 * LSTR, tid, p.S, 1);
+        }
         // T diag(beta) and T diag(beta e^g) -> fp16, row-major
         {
             const int rr = tid >> 2, j0 = (tid & 3) * 2;
             uint4 *d1 = reinterpret_cast<uint4 *>(ws + (size_t)rr * 128);
             uint4 *d2 = reinterpret_cast<uint4 *>(ws + (size_t)(64 + rr) * 128);
-            const float *Tr = Tb + rr * LSTR;
+            const float *Tr = Tsrc + rr * LSTR;
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 const int j = j0 + q;
@@ -278,6 +287,7 @@ constexpr uint32_t SMEM_USED = OFF_MISC + 32;
 constexpr uint32_t K2_SMEM = SMEM_USED + 1024;
 static_assert(K2_SMEM <= 232448, "shared memory budget of one sm_100 block");
 static_assert(K1_SMEM * K1_BLOCKS_PER_SM <= 233472, "key-side blocks per SM");
+static_assert(K1_SMEM_RES <= 232448, "residual-correction key-side block fits one SM");
 static_assert(K1_OFF_YB + 8192 <= K1_OFF_TB, "L and the inverse scratch fit in the tile region");
 
 // TMEM columns
@@ -747,7 +757,7 @@ bool tc_supports(const FwdParams &p, const char **why) {
     if (p.C != C) { *why = "needs chunk 64"; return false; }
     if (p.dk != DK) { *why = "needs dk 128"; return false; }
     if (p.dv % DVS != 0) { *why = "needs dv a multiple of 64"; return false; }
-    if (p.mode == GDN_INV_NEUMANN && p.N > kNeumannMaxN) { *why = "Neumann N > 15"; return false; }
+    if (p.mode != GDN_INV_EXACT && p.N > kNeumannMaxN) { *why = "Neumann N > 15"; return false; }
     if (p.slices && p.dvs != DVS) { *why = "value slices must be 64 columns"; return false; }
     return true;
 }
@@ -771,7 +781,7 @@ cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, 
     static bool attr_done = false;
     if (!attr_done) {
         cudaError_t e = cudaFuncSetAttribute(keyside_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)K1_SMEM);
+                                             (int)K1_SMEM_RES);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K2_SMEM);
         if (e != cudaSuccess) return e;
@@ -781,8 +791,9 @@ cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, 
     k1.B = p.B; k1.T = p.T; k1.H = p.H; k1.NC = NC;
     k1.alpha = p.alpha; k1.beta = p.beta;
     k1.ws = reinterpret_cast<uint8_t *>(workspace);
-    k1.neumann = p.mode == GDN_INV_NEUMANN; k1.N = p.N;
-    keyside_kernel<<<dim3(NC, p.H, p.B), K1_THREADS, K1_SMEM, stream>>>(mq, mk, k1);
+    k1.neumann = p.mode == GDN_INV_NEUMANN ? 1 : (p.mode == GDN_INV_NEUMANN_RESIDUAL ? 2 : 0);
+    k1.N = p.N; k1.S = p.S;
+    keyside_kernel<<<dim3(NC, p.H, p.B), K1_THREADS, k1.neumann == 2 ? K1_SMEM_RES : K1_SMEM, stream>>>(mq, mk, k1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     K2Params k2;

@@ -26,10 +26,10 @@ GDN_ERR_DEVICE_CHECK = 5
 GDN_ERR_FAULT_INJECTED = 6
 
 GDN_F32, GDN_BF16 = 0, 1
-GDN_INV_EXACT, GDN_INV_NEUMANN = 0, 1
+GDN_INV_EXACT, GDN_INV_NEUMANN, GDN_INV_NEUMANN_RESIDUAL = 0, 1, 2
 KERNELS = {"auto": 0, "simt": 1, "tc": 2}
 KERNEL_NAMES = {v: k for k, v in KERNELS.items()}
-MODES = {"exact": GDN_INV_EXACT, "neumann": GDN_INV_NEUMANN}
+MODES = {"exact": GDN_INV_EXACT, "neumann": GDN_INV_NEUMANN, "residual": GDN_INV_NEUMANN_RESIDUAL}
 
 EXPORTS = ("gdn_chunk_fwd", "gdn_select_kernel", "gdn_workspace_bytes", "gdn_device_check",
            "gdn_status_string", "gdn_last_error", "gdn_abi_version", "gdn_chunk_fwd_static_scratch")
@@ -57,6 +57,7 @@ class FwdArgs(ctypes.Structure):
         ("mode", ctypes.c_int32), ("neumann_N", ctypes.c_int32),
         ("kernel", ctypes.c_int32), ("dv_split", ctypes.c_int32),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_uint64),
+        ("residual_S", ctypes.c_int32),
     ]
 
 
@@ -197,7 +198,7 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
               erase: Optional[torch.Tensor] = None, write: Optional[torch.Tensor] = None,
               precond: bool = False, rho_decay: float = 0.99, rho_eps: float = 1e-6,
               S0: Optional[torch.Tensor] = None, chunk: int = 64, mode: str = "exact",
-              N: int = 3, o_dtype: Optional[torch.dtype] = None, kernel: str = "auto",
+              N: int = 3, S: int = 8, o_dtype: Optional[torch.dtype] = None, kernel: str = "auto",
               dv_split: int = 0, out: Optional[torch.Tensor] = None,
               final_state: bool = True, S_T: Optional[torch.Tensor] = None,
               stream: Optional[torch.cuda.Stream] = None
@@ -209,6 +210,8 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     fp32 (None = 1).  erase [B, T, H, dk], write [B, T, H, dv] gates and
     ``precond`` select the preconditioned two-gate rule.  S0 / S_T:
     [B, H, dk, dv] fp32 (h = S^T).  ``o_dtype`` defaults to q's dtype.
+    ``mode``: "exact", "neumann" (masked series to order N) or "residual" (the
+    masked series corrected with S residual terms).
     """
     if q.dim() != 4:
         raise ValueError("q must be [B, T, H, dk]")
@@ -239,7 +242,7 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         alpha_per_channel=int(per_channel), beta=_ptr(beta), precond=int(bool(precond)),
         rho_decay=float(rho_decay), rho_eps=float(rho_eps), erase=_ptr(erase),
         write=_ptr(write), S0=_ptr(S0), o=_ptr(out), S_T=_ptr(S_T), mode=MODES[mode],
-        neumann_N=int(N), kernel=KERNELS[kernel], dv_split=int(dv_split))
+        neumann_N=int(N), residual_S=int(S), kernel=KERNELS[kernel], dv_split=int(dv_split))
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     ws = workspace_for(args, q.device)

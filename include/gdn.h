@@ -69,7 +69,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 2
+#define GDN_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define GDN_API __attribute__((visibility("default")))
@@ -91,7 +91,11 @@ typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
 
 typedef enum {
     GDN_INV_EXACT = 0,          /* T = (I - A)^-1 exactly (blocked inversion) */
-    GDN_INV_NEUMANN = 1         /* T = M^(N) (.) sum_{n=0}^{N} A^n */
+    GDN_INV_NEUMANN = 1,        /* T = M^(N) (.) sum_{n=0}^{N} A^n */
+    GDN_INV_NEUMANN_RESIDUAL = 2 /* T0 = M^(N) (.) sum_{n=0}^{N} A^n, E = I - (I - A) T0,
+                                   T = T0 sum_{s=0}^{S} E^s ("Quando o 'Bom o Suficiente' e
+                                   Otimo ...", section "Metodologia", item 3); tensor-core
+                                   kernel only */
 } gdn_inv_mode;
 
 typedef enum {
@@ -124,6 +128,7 @@ typedef struct {
     void *workspace;            /* device scratch of >= gdn_workspace_bytes(args) bytes,
                                    16-byte aligned, caller-owned; may be NULL when that is 0 */
     uint64_t workspace_bytes;   /* size of workspace */
+    int32_t residual_S;         /* S for GDN_INV_NEUMANN_RESIDUAL: 0 <= S <= 64 */
 } gdn_fwd_args;
 
 /* Chunkwise forward: o and S_T from q, k, v, gates and S0 (see above). */

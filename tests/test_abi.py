@@ -25,7 +25,7 @@ def declared_functions():
 
 def test_library_builds_and_loads():
     gbuild.build()
-    assert gdn.abi_version() == 2
+    assert gdn.abi_version() == 3
 
 
 def test_exports_every_declared_symbol():
@@ -69,6 +69,12 @@ def _args(**kw):
     (dict(kernel=2, io_dtype=0), GDN_ERR_UNSUPPORTED),  # tensor cores need bf16 io
     (dict(alpha=0x70000, alpha_per_channel=1, chunk=128, kernel=1, dv_split=8),
      GDN_ERR_UNSUPPORTED),                              # two-gate SIMT at C=128 too big
+    (dict(mode=2, neumann_N=3, residual_S=65), GDN_ERR_INVALID_ARG),   # S > 64
+    (dict(mode=2, neumann_N=3, residual_S=-1), GDN_ERR_INVALID_ARG),
+    (dict(mode=2, neumann_N=64, residual_S=8), GDN_ERR_INVALID_ARG),   # N > C - 1
+    (dict(mode=2, neumann_N=3, residual_S=8, kernel=1), GDN_ERR_UNSUPPORTED),  # SIMT has no residual
+    (dict(mode=2, neumann_N=3, residual_S=8, io_dtype=0, dk=64, dv=64),
+     GDN_ERR_UNSUPPORTED),                              # fp32 io: no tensor-core kernel
 ])
 def test_invalid_arguments_rejected_on_host(kw, status):
     a = _args(**kw)
@@ -86,6 +92,7 @@ def test_null_args_pointer():
 
 def test_valid_arguments_select_a_kernel():
     assert gdn.select_kernel(_args(kernel=1)) == 1
+    assert gdn.select_kernel(_args(mode=2, neumann_N=3, residual_S=8)) == 2   # residual: tensor cores
     assert gdn.select_kernel(_args(io_dtype=0, dk=64, dv=64)) == 1   # fp32 io -> SIMT
     assert gdn.select_kernel(_args(alpha=0x70000, precond=1, erase=0x50000,
                                    write=0x58000, alpha_per_channel=1)) in (1, 2)

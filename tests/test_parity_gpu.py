@@ -89,6 +89,33 @@ def test_neumann_sweep(chunk, N):
     report(f"neumann_C{chunk}_N{N}_vs_exact_oracle", o=stats(o, o_ex), S_T=stats(s, s_ex))
 
 
+# ------------------------------------------- residual correction (next row 1)
+
+@needs_cuda
+@pytest.mark.parametrize("N,S", [(3, 8), (2, 2), (3, 0), (1, 31)])
+def test_residual_correction_small(N, S):
+    """T0 = masked series to order N, corrected with S residual terms, on a ragged
+    sequence with S0; S = 0 is the masked series itself, (N+1)(S+1) >= C exact."""
+    w = workload("gdn_bf16", B=1, H=2, T=300, s0_std=0.02)
+    x = make_inputs(w, seed=17)
+    o_ref, s_ref = cf.chunked_gated_delta_fwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"],
+                                              chunk=64, inverse=cf.residual_inverse(N, S))
+    _check_bf16(f"residual_N{N}_S{S}", w, x, o_ref, s_ref, mode="residual", N=N, S=S)
+
+
+@needs_cuda
+def test_residual_correction_full_size():
+    """N = 3, S = 8 on the bench workload: parity against the chunk model with the
+    same correction; the error against the exact recurrence is reported."""
+    w = workload("gdn_bf16")
+    x = make_inputs(w)
+    o_ref, s_ref = cf.chunked_gated_delta_fwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"],
+                                              chunk=64, inverse=cf.residual_inverse(3, 8))
+    o, s = _check_bf16("residual_N3_S8_full", w, x, o_ref, s_ref, mode="residual", N=3, S=8)
+    o_ex, s_ex = run_oracle(x, w)
+    report("residual_N3_S8_vs_exact_oracle", o=stats(o, o_ex), S_T=stats(s, s_ex))
+
+
 # ------------------------------------------------------------ configuration 5
 
 @needs_cuda
