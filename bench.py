@@ -331,6 +331,125 @@ def run_gpu(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+DECODE_METRIC = "decode tokens/s (bf16, H=16, d=128, one token per sequence, state in place) and % of HBM roofline on 1 B200"
+
+
+def decode_bytes(w):
+    """Per step: the fp32 state read and written, q, k, v in and o out (bf16), alpha, beta."""
+    return w.B * w.H * (2 * w.dk * w.dv * 4 + (2 * w.dk + w.dv) * 2 + w.dv * 2 + 8)
+
+
+def run_decode(args, rank, world, local_rank):
+    """One decode step per call: T = 1 for B sequences, the state updated in place."""
+    import torch
+    import chunked_gated_delta_14_b200 as gdn
+    from chunked_gated_delta_14_b200.inputs import make_inputs, workload
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workload(WORKLOAD, B=args.batch or 256, T=1, s0_std=0.02)
+    x = make_inputs(w, seed=rank)
+    d = {k: (None if v is None else v.to(dev)) for k, v in x.items()}
+    state = d["S0"].clone()
+    o = torch.empty((w.B, 1, w.H, w.dv), device=dev, dtype=torch.bfloat16)
+    ptr = lambda t: None if t is None else t.data_ptr()
+    a = gdn.make_args(B=w.B, T=1, H=w.H, dk=w.dk, dv=w.dv, chunk=w.chunk, io_dtype=1, o_dtype=1,
+                      q=ptr(d["q"]), k=ptr(d["k"]), v=ptr(d["v"]), alpha=ptr(d["alpha"]),
+                      beta=ptr(d["beta"]), S0=state.data_ptr(), o=o.data_ptr(), S_T=state.data_ptr(),
+                      mode=0, kernel=0)
+    assert gdn.select_kernel(a) == 3, "decode steps run on the recurrent kernel"
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    for _ in range(args.warmup):
+        gdn.call(a, sh)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    if rank == 0:
+        clocks.start()
+        time.sleep(1.0)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        gdn.call(a, sh)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    clocks.mark(t_wall0, t_wall1)
+    time.sleep(0.3)
+    clocks.stop()
+    ms_step = ms / args.steps
+    value = job_throughput(w.B, world, args.steps, ms)
+
+    # end to end: this step's q, k, v, alpha, beta from pinned host memory, o back
+    host = {k: x[k].pin_memory() for k in ("q", "k", "v", "alpha", "beta")}
+    o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_host.numel() * o_host.element_size()
+
+    def e2e_step():
+        for k, t in host.items():
+            d[k].copy_(t, non_blocking=True)
+        gdn.call(a, sh)
+        o_host.copy_(o, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    n_e2e = max(1, args.e2e_steps * 10)
+    f0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    ems = max_over_ranks(f0.elapsed_time(f1), world, dev)
+    e2e = dict(value=job_throughput(w.B, world, n_e2e, ems), unit=UNIT, h2d_bytes_per_step=int(h2d),
+               d2h_bytes_per_step=int(d2h), ms_per_step=ems / n_e2e)
+
+    pk = peaks()
+    bytes_step = decode_bytes(w)
+    achieved = bytes_step / (ms_step / 1e3) / 1e9
+    roof = dict(bound="hbm", achieved=achieved, peak=pk["hbm_gbs"], unit="GB/s",
+                frac=achieved / pk["hbm_gbs"], traffic=None,
+                peak_source=pk["source"] + " (burst copy bandwidth)",
+                algorithmic_bytes_per_launch=bytes_step,
+                roofline_ms=bytes_step / (pk["hbm_gbs"] * 1e9) * 1e3)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        cores = len(os.sched_getaffinity(0))
+        n, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < min(args.cpu_budget, 3.0):
+            oracle.gated_delta_fwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"], nthreads=cores)
+            n += 1
+        el = time.perf_counter() - t0
+        cpu = dict(value=w.B * n / el, unit=UNIT, cores=cores, kind="oracle",
+                   sample=f"{n} decode steps of all {w.B} x {w.H} heads, fp64 C oracle, {el:.1f} s")
+    if rank == 0:
+        line = dict(metric=DECODE_METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps,
+                    warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",
+                    vs_baseline=None, dtype="bf16",
+                    compute="bf16 q/k/v/o in HBM; fp32 state, fp32 arithmetic",
+                    data="synthetic (seeded; Gated DeltaNet layer shapes)",
+                    config=dict(workload=f"decode: B={w.B} H={w.H} T=1 dk={w.dk} dv={w.dv}, state in place",
+                                global_batch=w.B * world, seq_len=1,
+                                parallelism=f"independent batch per GPU x{world}",
+                                l2=f"no flush: state {w.B * w.H * w.dk * w.dv * 4 / 1e6:.0f} MB read and "
+                                   f"written per step > 126 MB L2",
+                                kernel="recurrent_kernel"),
+                    clocks=clocks.summary(), e2e=e2e, gpu_launches=args.steps, roofline=roof,
+                    cpu_baseline=cpu)
+        print(json.dumps(line), flush=True)
+
+
 def cpu_baseline(w, x, budget_s=12.0):
     """The fp64 oracle as it stands, timed on this host's cores, on whole
     (batch, head) sequences of the same workload until ~budget_s seconds."""
@@ -415,6 +534,8 @@ def main():
     ap.add_argument("--mode", default="exact", choices=["exact", "neumann", "residual"],
                     help="inverse: exact (the headline workload), masked Neumann series "
                          "(order --N), or the series with --S residual-correction terms")
+    ap.add_argument("--decode", action="store_true",
+                    help="decode steps (T = 1, state in place, B = 256 unless --batch)")
     ap.add_argument("--N", type=int, default=3)
     ap.add_argument("--S", type=int, default=8)
     args = ap.parse_args()
@@ -434,7 +555,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_gpu(args, rank, world, local_rank)
+        if args.decode:
+            run_decode(args, rank, world, local_rank)
+        else:
+            run_gpu(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

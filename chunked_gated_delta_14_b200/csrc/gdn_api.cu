@@ -71,7 +71,7 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
                         a->workspace};
     for (const void *x : al)
         if (x && !aligned16(x)) return fail(GDN_ERR_ALIGNMENT, "pointers must be 16-byte aligned");
-    if (a->kernel < GDN_KERNEL_AUTO || a->kernel > GDN_KERNEL_TC)
+    if (a->kernel < GDN_KERNEL_AUTO || a->kernel > GDN_KERNEL_RECURRENT)
         return fail(GDN_ERR_INVALID_ARG, "kernel %d unknown", a->kernel);
     if (a->dv_split < 0 || (a->dv_split > 0 && (a->dv % a->dv_split != 0 || a->dv / a->dv_split < 16)))
         return fail(GDN_ERR_INVALID_ARG, "dv_split must divide dv into slices of >= 16 columns");
@@ -90,7 +90,10 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
 
     const char *why = "";
     int kern = a->kernel;
-    if (kern == GDN_KERNEL_AUTO) {
+    if (kern == GDN_KERNEL_AUTO && p.T <= gdn::kRecurrentMaxT && gdn::recurrent_supports(p, &why)) {
+        // a few tokens (decode steps): the token recurrence beats any chunked form
+        kern = GDN_KERNEL_RECURRENT;
+    } else if (kern == GDN_KERNEL_AUTO) {
         // tensor-core kernel when it supports the call, including the requested value split
         gdn::FwdParams t = p;
         kern = GDN_KERNEL_SIMT;
@@ -100,7 +103,12 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
             if (t.dv % t.slices == 0 && gdn::tc_supports(t, &why)) kern = GDN_KERNEL_TC;
         }
     }
-    if (kern == GDN_KERNEL_TC) {
+    if (kern == GDN_KERNEL_RECURRENT) {
+        if (!gdn::recurrent_supports(p, &why))
+            return fail(GDN_ERR_UNSUPPORTED, "recurrent kernel: %s", why);
+        p.slices = p.dv / 32;
+        p.dvs = 32;
+    } else if (kern == GDN_KERNEL_TC) {
         if (!gdn::tc_supports(p, &why))
             return fail(GDN_ERR_UNSUPPORTED, "tensor-core kernel: %s", why);
         p.slices = a->dv_split ? a->dv_split : gdn::tc_default_slices(p);
@@ -199,12 +207,14 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_args *args, void *stream) {
             return fail(GDN_ERR_INVALID_ARG, "tensor-core kernel needs a workspace of %zu bytes (got %llu)",
                         need, (unsigned long long)args->workspace_bytes);
         e = gdn::launch_tc(p, args->workspace, st, &why);
-    }
-    else {
+    } else if (kern == GDN_KERNEL_RECURRENT) {
+        e = gdn::launch_recurrent(p, st);
+    } else {
         e = gdn::launch_simt(p, st);
     }
     if (e != cudaSuccess)
-        return fail(GDN_ERR_CUDA, "%s launch: %s %s", kern == GDN_KERNEL_TC ? "tc" : "simt",
+        return fail(GDN_ERR_CUDA, "%s launch: %s %s",
+                    kern == GDN_KERNEL_TC ? "tc" : (kern == GDN_KERNEL_RECURRENT ? "recurrent" : "simt"),
                     cudaGetErrorString(e), why);
     g_msg[0] = 0;
     return GDN_OK;

@@ -30,6 +30,11 @@ struct FwdParams {
 };
 
 // SIMT fp32 chunk kernel: shared-memory bytes for p, or 0 if p does not fit.
+// Token-by-token kernel (decode steps): chosen automatically for T <= kRecurrentMaxT.
+constexpr int kRecurrentMaxT = 8;
+bool recurrent_supports(const FwdParams &p, const char **why);
+cudaError_t launch_recurrent(const FwdParams &p, cudaStream_t stream);
+
 size_t simt_smem_bytes(const FwdParams &p);
 cudaError_t launch_simt(const FwdParams &p, cudaStream_t stream);
 

@@ -27,7 +27,7 @@ GDN_ERR_FAULT_INJECTED = 6
 
 GDN_F32, GDN_BF16 = 0, 1
 GDN_INV_EXACT, GDN_INV_NEUMANN, GDN_INV_NEUMANN_RESIDUAL = 0, 1, 2
-KERNELS = {"auto": 0, "simt": 1, "tc": 2}
+KERNELS = {"auto": 0, "simt": 1, "tc": 2, "recurrent": 3}
 KERNEL_NAMES = {v: k for k, v in KERNELS.items()}
 MODES = {"exact": GDN_INV_EXACT, "neumann": GDN_INV_NEUMANN, "residual": GDN_INV_NEUMANN_RESIDUAL}
 

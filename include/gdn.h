@@ -101,7 +101,10 @@ typedef enum {
 typedef enum {
     GDN_KERNEL_AUTO = 0,        /* tensor-core kernel when it supports the call, else SIMT */
     GDN_KERNEL_SIMT = 1,        /* fp32 CUDA-core chunk kernel (all variants) */
-    GDN_KERNEL_TC = 2           /* tcgen05/TMEM/TMA kernel (bf16 io, scalar decay, C = 64) */
+    GDN_KERNEL_TC = 2,          /* tcgen05/TMEM/TMA kernel (bf16 io, scalar decay, C = 64) */
+    GDN_KERNEL_RECURRENT = 3    /* token-by-token kernel for short sequences and decode steps
+                                   (scalar decay, exact mode, dk a multiple of 8, dv of 32);
+                                   AUTO picks it for T <= 8 */
 } gdn_kernel;
 
 typedef struct {

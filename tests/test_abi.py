@@ -75,6 +75,9 @@ def _args(**kw):
     (dict(mode=2, neumann_N=3, residual_S=8, kernel=1), GDN_ERR_UNSUPPORTED),  # SIMT has no residual
     (dict(mode=2, neumann_N=3, residual_S=8, io_dtype=0, dk=64, dv=64),
      GDN_ERR_UNSUPPORTED),                              # fp32 io: no tensor-core kernel
+    (dict(kernel=3, dv=16), GDN_ERR_UNSUPPORTED),       # recurrent kernel needs dv % 32 == 0
+    (dict(kernel=3, alpha=0x70000, alpha_per_channel=1), GDN_ERR_UNSUPPORTED),   # two-gate rule
+    (dict(kernel=3, mode=1, neumann_N=3), GDN_ERR_UNSUPPORTED),
 ])
 def test_invalid_arguments_rejected_on_host(kw, status):
     a = _args(**kw)
@@ -93,6 +96,10 @@ def test_null_args_pointer():
 def test_valid_arguments_select_a_kernel():
     assert gdn.select_kernel(_args(kernel=1)) == 1
     assert gdn.select_kernel(_args(mode=2, neumann_N=3, residual_S=8)) == 2   # residual: tensor cores
+    assert gdn.select_kernel(_args(T=1)) == 3                                  # decode step
+    assert gdn.select_kernel(_args(T=8, io_dtype=0, dk=64, dv=64)) == 3
+    assert gdn.select_kernel(_args(T=9)) == 2                                  # chunked from T = 9
+    assert gdn.select_kernel(_args(T=1, mode=1, neumann_N=3)) != 3             # series: chunked only
     assert gdn.select_kernel(_args(io_dtype=0, dk=64, dv=64)) == 1   # fp32 io -> SIMT
     assert gdn.select_kernel(_args(alpha=0x70000, precond=1, erase=0x50000,
                                    write=0x58000, alpha_per_channel=1)) in (1, 2)

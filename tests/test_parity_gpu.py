@@ -116,6 +116,62 @@ def test_residual_correction_full_size():
     report("residual_N3_S8_vs_exact_oracle", o=stats(o, o_ex), S_T=stats(s, s_ex))
 
 
+# ---------------------------------------------------- decode steps (next row 4)
+
+@needs_cuda
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 64), (32, 32), (16, 32), (128, 64)])
+def test_recurrent_decode_step(dk, dv):
+    """One token per call with a carried state: the token-by-token kernel (chosen
+    automatically for short T) against the oracle, bf16 and fp32 inputs."""
+    import chunked_gated_delta_14_b200 as gdn
+    for io in ("bf16", "f32"):
+        w = workload("gdn_bf16", B=3, H=4, T=1, dk=dk, dv=dv, io=io, s0_std=0.02)
+        x = make_inputs(w, seed=18)
+        o_ref, s_ref = run_oracle(x, w)
+        o, s = run_gpu(x, w, o_dtype=torch.float32)
+        if io == "f32":
+            assert np.abs(o - o_ref).max() <= TOL_F32_ABS and np.abs(s - s_ref).max() <= TOL_F32_ABS
+        else:
+            so, ss = stats(o, o_ref), stats(s, s_ref)
+            report(f"decode_{dk}_{dv}", o=so, S_T=ss)
+            assert so["max_rel_rms"] <= TOL_BF16_REL_RMS and ss["max_rel_rms"] <= TOL_BF16_REL_RMS
+        a = gdn.make_args(B=w.B, T=w.T, H=w.H, dk=dk, dv=dv, chunk=64, io_dtype=int(io == "bf16"),
+                          o_dtype=0, q=1 << 20, k=2 << 20, v=3 << 20, o=4 << 20)
+        assert gdn.select_kernel(a) == 3
+
+
+@needs_cuda
+def test_recurrent_decode_chain_equals_one_call():
+    """Six decode calls with the state updated in place (S_T aliases S0) equal one
+    chunked call over the six tokens (SIMT kernel), fp32."""
+    import chunked_gated_delta_14_b200 as gdn
+    w = workload("plain_fp32", B=2, H=3, T=6, dk=64, dv=64, decay="scalar", s0_std=0.02)
+    x = make_inputs(w, seed=19)
+    d = {k: (None if v is None else v.cuda()) for k, v in x.items()}
+    o_all, s_all = gdn.chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S0=d["S0"], kernel="simt")
+    state = d["S0"].clone()
+    outs = []
+    for t in range(w.T):
+        sl = lambda z: z[:, t:t + 1].contiguous()
+        o_t, _ = gdn.chunk_fwd(sl(d["q"]), sl(d["k"]), sl(d["v"]), sl(d["alpha"]), sl(d["beta"]),
+                               S0=state, S_T=state, kernel="recurrent")
+        outs.append(o_t)
+    torch.cuda.synchronize()
+    o_cat = torch.cat(outs, dim=1)
+    assert (o_cat - o_all).abs().max().item() <= TOL_F32_ABS
+    assert (state - s_all).abs().max().item() <= TOL_F32_ABS
+
+
+@needs_cuda
+def test_recurrent_short_sequence_bf16():
+    """T = 8, the longest sequence the automatic choice sends to the token kernel,
+    with S0: against the oracle."""
+    w = workload("gdn_bf16", B=2, H=16, T=8, s0_std=0.02)
+    x = make_inputs(w, seed=20)
+    o_ref, s_ref = run_oracle(x, w)
+    _check_bf16("recurrent_T8", w, x, o_ref, s_ref, kernel="recurrent")
+
+
 # ------------------------------------------------------------ configuration 5
 
 @needs_cuda
