@@ -118,20 +118,34 @@ void oracle_gated_delta_fwd(int B, int T, int H, int dk, int dv,
  *   q (read key), k (raw key) [B,T,H,dk]; v [B,T,H,dv];
  *   alpha [B,T,H,dk] per key channel, or NULL (=> 1);
  *   erase b_t [B,T,H,dk] or NULL (=> 1); write w_t [B,T,H,dv] or NULL (=> 1);
- *   precond != 0 enables the curvature accumulator, otherwise the write key
- *   is k_t itself.
+ *   precond selects the per-channel preconditioner f of the curvature
+ *   accumulator rho (0: none, f = 1):
+ *     1  f = 1 / sqrt(rho + eps)                      (moving-average form)
+ *     2  f = 1 / (rho + eps)                          (P_t = Diag(A_t)^-1, the
+ *        pages' diagonal approximation, "Preconditioned DeltaNet ..." Arabic
+ *        summary, section 2b)
+ *     3  f = x^tanh(ln(1 / (rho + eps)) / ln x)      (2 squashed into [1/x, x]
+ *        on a log scale, "Resumo Tecnico: Preconditioned DeltaNet", section 2,
+ *        "Estabilidade e Parametrizacao"; the squash function is not printed)
+ *   precond_query = 0 applies f to the write key (ATK), 1 to the query (ATQ)
+ *   (Arabic summary, section 2a).
  * Per token:  rho   = rho_decay * rho + k_t (.) k_t          (rho_0 = 0)
- *             kw    = k_t / sqrt(rho + rho_eps)               (write key)
- *             e     = b_t (.) kw                              (erase key)
+ *   ATK:      kw    = f (.) k_t                               (write key)
+ *             e     = b_t (.) kw  for precond 1,  b_t (.) k_t  for 2, 3
+ *                     (the pages' forms read the state with the raw key and
+ *                      write with the preconditioned one)
+ *             qe    = q_t
+ *   ATQ:      kw    = k_t,  e = b_t (.) k_t,  qe = f (.) q_t
  *             p     = S e
  *             S     = S diag(alpha_t) - p kw^T + (w_t (.) v_t) kw^T
- *             o_t   = S q_t
+ *             o_t   = S qe
  */
 void oracle_precond_two_gate_fwd(int B, int T, int H, int dk, int dv,
                                  const double *q, const double *k, const double *v,
                                  const double *alpha, const double *erase,
                                  const double *write, int precond,
-                                 double rho_decay, double rho_eps,
+                                 double rho_decay, double rho_eps, double precond_x,
+                                 int precond_query,
                                  const double *h0, double *o, double *hT,
                                  int nthreads)
 {
@@ -145,6 +159,7 @@ void oracle_precond_two_gate_fwd(int B, int T, int H, int dk, int dv,
         double *rho = (double *)calloc((size_t)dk, sizeof(double));
         double *kw = (double *)malloc((size_t)dk * sizeof(double));
         double *e = (double *)malloc((size_t)dk * sizeof(double));
+        double *qe = (double *)malloc((size_t)dk * sizeof(double));
         double *p = (double *)malloc((size_t)dv * sizeof(double));
         if (h0) {
             const double *src = h0 + (size_t)bh * dk * dv;
@@ -156,13 +171,24 @@ void oracle_precond_two_gate_fwd(int B, int T, int H, int dk, int dv,
             const size_t r = tok(b, t, h, T, H);
             const double *kt = k + r * dk, *qt = q + r * dk, *vt = v + r * dv;
             for (int i = 0; i < dk; ++i) {
+                double f = 1.0;
                 if (precond) {
                     rho[i] = rho_decay * rho[i] + kt[i] * kt[i];
-                    kw[i] = kt[i] / sqrt(rho[i] + rho_eps);
-                } else {
-                    kw[i] = kt[i];
+                    const double a = rho[i] + rho_eps;
+                    if (precond == 1) f = 1.0 / sqrt(a);
+                    else if (precond == 2) f = 1.0 / a;
+                    else f = pow(precond_x, tanh(log(1.0 / a) / log(precond_x)));
                 }
-                e[i] = (erase ? erase[r * dk + i] : 1.0) * kw[i];
+                const double b = erase ? erase[r * dk + i] : 1.0;
+                if (precond_query) {
+                    kw[i] = kt[i];
+                    e[i] = b * kt[i];
+                    qe[i] = f * qt[i];
+                } else {
+                    kw[i] = f * kt[i];
+                    e[i] = b * (precond == 1 ? kw[i] : kt[i]);
+                    qe[i] = qt[i];
+                }
             }
             for (int j = 0; j < dv; ++j) {
                 double acc = 0.0;
@@ -180,7 +206,7 @@ void oracle_precond_two_gate_fwd(int B, int T, int H, int dk, int dv,
             double *ot = o + r * dv;
             for (int j = 0; j < dv; ++j) {
                 double acc = 0.0;
-                for (int i = 0; i < dk; ++i) acc += S[(size_t)j * dk + i] * qt[i];
+                for (int i = 0; i < dk; ++i) acc += S[(size_t)j * dk + i] * qe[i];
                 ot[j] = acc;
             }
         }
@@ -194,6 +220,7 @@ void oracle_precond_two_gate_fwd(int B, int T, int H, int dk, int dv,
         free(rho);
         free(kw);
         free(e);
+        free(qe);
         free(p);
     }
 }

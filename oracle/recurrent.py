@@ -44,7 +44,8 @@ def _load():
             lib.oracle_gated_delta_fwd.restype = None
             lib.oracle_precond_two_gate_fwd.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp,
                                                         dp, i, ctypes.c_double,
-                                                        ctypes.c_double, dp, dp, dp, i]
+                                                        ctypes.c_double, ctypes.c_double, i,
+                                                        dp, dp, dp, i]
             lib.oracle_precond_two_gate_fwd.restype = None
             _lib = lib
     return _lib
@@ -92,13 +93,17 @@ def gated_delta_fwd(q, k, v, alpha=None, beta=None, h0=None, nthreads=None):
 
 
 def precond_two_gate_fwd(q, k, v, alpha=None, erase=None, write=None, precond=True,
-                         rho_decay=0.99, rho_eps=1e-6, h0=None, nthreads=None):
+                         rho_decay=0.99, rho_eps=1e-6, h0=None, nthreads=None,
+                         precond_x=2.0, precond_query=False):
     """Preconditioned write key, per-channel decay, erase/write channel gates.
 
-    rho_t = rho_decay rho_{t-1} + k_t (.) k_t; kw = k_t / sqrt(rho_t + rho_eps);
-    S_t = S_{t-1}(diag(alpha_t) - (b_t (.) kw) kw^T) + (w_t (.) v_t) kw^T;
-    o_t = S_t q_t.  alpha, erase: [B, T, H, d_k]; write: [B, T, H, d_v];
-    each may be None (meaning all ones).
+    rho_t = rho_decay rho_{t-1} + k_t (.) k_t and a per-channel factor f(rho_t):
+    precond 1 (or True) f = 1/sqrt(rho + eps); 2 f = 1/(rho + eps) (the pages'
+    Diag(A_t)^-1); 3 the latter squashed into [1/precond_x, precond_x]; 0 (False)
+    none.  ATK (precond_query False): kw = f k_t, read key e = b (.) kw for form 1,
+    b (.) k_t for forms 2, 3.  ATQ: kw = k_t, e = b (.) k_t, o_t = S_t (f (.) q_t).
+    S_t = S_{t-1}(diag(alpha_t) - e kw^T) + (w_t (.) v_t) kw^T;  o_t = S_t q_t.
+    alpha, erase: [B, T, H, d_k]; write: [B, T, H, d_v]; each may be None (ones).
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     alpha, erase, write, h0 = _f64(alpha), _f64(erase), _f64(write), _f64(h0)
@@ -112,6 +117,7 @@ def precond_two_gate_fwd(q, k, v, alpha=None, erase=None, write=None, precond=Tr
     hT = np.zeros((B, H, dk, dv))
     _load().oracle_precond_two_gate_fwd(B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v),
                                         _ptr(alpha), _ptr(erase), _ptr(write),
-                                        int(bool(precond)), float(rho_decay), float(rho_eps),
+                                        int(precond), float(rho_decay), float(rho_eps),
+                                        float(precond_x), int(bool(precond_query)),
                                         _ptr(h0), _ptr(o), _ptr(hT), _threads(nthreads))
     return o, hT

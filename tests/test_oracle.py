@@ -13,6 +13,7 @@ import pytest
 
 from oracle import chunk_forms as cf
 from oracle import recurrent as rec
+from chunked_gated_delta_14_b200.inputs import make_inputs, workload
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -344,3 +345,78 @@ def test_neumann_chunk_model_error_shrinks_with_N():
     on, _ = cf.chunked_gated_delta_fwd(q, k, v, alpha, beta, chunk=64,
                                        inverse=cf.neumann_inverse(63))
     np.testing.assert_allclose(on, ox, rtol=0, atol=1e-12)
+
+
+# --------------------------------------- page-form preconditioners (next row 3)
+
+def _one_hot_stream(T=40, d=6, dv=3, seed=0):
+    rng = np.random.default_rng(seed)
+    idx = rng.integers(0, d, size=T)
+    k = np.zeros((1, T, 1, d))
+    k[0, np.arange(T), 0, idx] = 1.0
+    v = rng.standard_normal((1, T, 1, dv))
+    q = rng.standard_normal((1, T, 1, d))
+    return idx, q, k, v
+
+
+def test_diag_preconditioner_recovers_least_squares_for_one_hot_keys():
+    """P_t = Diag(A_t)^-1 with A_t the plain sum of k (.) k: for orthogonal (one-hot)
+    keys the Gram matrix is diagonal, so the preconditioned delta rule is the exact
+    online least-squares solve: column i of S is the mean of the values written
+    with key i (pages: exact preconditioning recovers the least-squares solution)."""
+    idx, q, k, v = _one_hot_stream()
+    o, hT = rec.precond_two_gate_fwd(q, k, v, precond=2, rho_decay=1.0, rho_eps=1e-12)
+    T, d, dv = k.shape[1], k.shape[3], v.shape[3]
+    sums, counts = np.zeros((d, dv)), np.zeros(d)
+    for t in range(T):
+        sums[idx[t]] += v[0, t, 0]
+        counts[idx[t]] += 1
+        means = np.where(counts[:, None] > 0, sums / np.maximum(counts, 1)[:, None], 0.0)
+        np.testing.assert_allclose(o[0, t, 0], means.T @ q[0, t, 0], atol=1e-9)
+    np.testing.assert_allclose(hT[0, 0], means, atol=1e-9)
+
+
+def test_preconditioned_query_linear_attention_equals_preconditioned_key_deltanet():
+    """ATQ (linear attention, no erase, preconditioner on the query) and ATK
+    (delta rule, preconditioner on the write key) give the same outputs when the
+    diagonal preconditioner is exact (one-hot keys)."""
+    idx, q, k, v = _one_hot_stream(seed=1)
+    zeros = np.zeros_like(k)
+    o_atq, _ = rec.precond_two_gate_fwd(q, k, v, erase=zeros, precond=2, rho_decay=1.0,
+                                           rho_eps=1e-12, precond_query=True)
+    o_atk, _ = rec.precond_two_gate_fwd(q, k, v, precond=2, rho_decay=1.0, rho_eps=1e-12)
+    np.testing.assert_allclose(o_atq, o_atk, atol=1e-9)
+
+
+def test_squashed_preconditioner_bounds_and_monotone():
+    """Form 3 keeps the factor in [1/x, x], equals 1 at rho = 1 and decreases with
+    rho: read off S = v (f k)^T after one write with no erase (k = c e_0)."""
+    x = 2.0
+    fs = []
+    for c in (0.05, 0.3, 1.0, 3.0, 20.0):
+        k = np.zeros((1, 1, 1, 4)); k[0, 0, 0, 0] = c
+        v = np.ones((1, 1, 1, 2))
+        q = np.zeros((1, 1, 1, 4))
+        _, hT = rec.precond_two_gate_fwd(q, k, v, erase=np.zeros_like(k), precond=3, rho_decay=1.0,
+                                            rho_eps=0.0, precond_x=x)
+        f = hT[0, 0, 0, 0] / c          # S column 0 = v f c
+        fs.append(f)
+        assert 1.0 / x - 1e-12 <= f <= x + 1e-12
+    assert abs(fs[2] - 1.0) < 1e-12
+    assert all(a > b for a, b in zip(fs, fs[1:]))
+
+
+def test_squash_limits():
+    """x -> infinity recovers Diag(A)^-1 (form 2); x -> 1 removes the preconditioner.
+    eps = 1 keeps form 2's factor in (0, 1], where the log-scale squash with a huge
+    x is linear to 1e-4 (with a tiny eps form 2 is the unstable case the squash
+    exists for, and the recurrence amplifies any difference)."""
+    w = workload("precond_two_gate", B=1, H=1, T=40, dk=8, dv=4)
+    x = make_inputs(w, seed=3)
+    args = dict(alpha=x["alpha"], erase=x["erase"], write=x["write"], rho_decay=1.0, rho_eps=1.0)
+    o2, s2 = rec.precond_two_gate_fwd(x["q"], x["k"], x["v"], precond=2, **args)
+    o3, s3 = rec.precond_two_gate_fwd(x["q"], x["k"], x["v"], precond=3, precond_x=1e60, **args)
+    np.testing.assert_allclose(o3, o2, rtol=1e-3, atol=1e-6)
+    o0, _ = rec.precond_two_gate_fwd(x["q"], x["k"], x["v"], precond=0, **args)
+    o1, _ = rec.precond_two_gate_fwd(x["q"], x["k"], x["v"], precond=3, precond_x=1.0 + 1e-9, **args)
+    np.testing.assert_allclose(o1, o0, atol=1e-7)
