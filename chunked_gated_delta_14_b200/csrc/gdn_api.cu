@@ -55,8 +55,14 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
         return fail(GDN_ERR_INVALID_ARG, "alpha_per_channel needs alpha");
     if (a->alpha_per_channel != 0 && a->alpha_per_channel != 1)
         return fail(GDN_ERR_INVALID_ARG, "alpha_per_channel must be 0 or 1");
-    if (a->precond != 0 && a->precond != 1)
-        return fail(GDN_ERR_INVALID_ARG, "precond must be 0 or 1");
+    if (a->precond < 0 || a->precond > 3)
+        return fail(GDN_ERR_INVALID_ARG, "precond must be 0, 1, 2 or 3 (got %d)", a->precond);
+    if (a->precond == 3 && !(a->precond_x > 1.f))
+        return fail(GDN_ERR_INVALID_ARG, "precond 3 needs precond_x > 1 (got %g)", (double)a->precond_x);
+    if (a->precond_query != 0 && a->precond_query != 1)
+        return fail(GDN_ERR_INVALID_ARG, "precond_query must be 0 or 1");
+    if (a->precond_query && !a->precond)
+        return fail(GDN_ERR_INVALID_ARG, "precond_query needs a preconditioner (precond 1, 2 or 3)");
     const int general = a->alpha_per_channel || a->precond || a->erase || a->write;
     if (general && a->beta)
         return fail(GDN_ERR_INVALID_ARG,
@@ -82,7 +88,7 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
     p.o_bf16 = a->o_dtype == GDN_BF16;
     p.q = a->q; p.k = a->k; p.v = a->v;
     p.alpha = a->alpha; p.alpha_pc = a->alpha_per_channel; p.beta = a->beta;
-    p.precond = a->precond; p.rho_decay = a->rho_decay; p.rho_eps = a->rho_eps;
+    p.precond = a->precond; p.precond_x = a->precond_x; p.precond_query = a->precond_query; p.rho_decay = a->rho_decay; p.rho_eps = a->rho_eps;
     p.erase = a->erase; p.write = a->write; p.S0 = a->S0; p.o = a->o; p.S_T = a->S_T;
     p.mode = a->mode; p.N = a->mode != GDN_INV_EXACT ? a->neumann_N : 0;
     p.S = a->mode == GDN_INV_NEUMANN_RESIDUAL ? a->residual_S : 0;

@@ -18,8 +18,10 @@ struct FwdParams {
     const float *alpha;
     int alpha_pc;
     const float *beta;
-    int precond;
+    int precond;        // 0 none, 1 1/sqrt(rho+eps), 2 1/(rho+eps), 3 the latter squashed
     float rho_decay, rho_eps;
+    float precond_x;    // squash bound x (precond 3)
+    int precond_query;  // 1: factor on the query (ATQ) instead of the write key
     const void *erase, *write;
     const float *S0;
     void *o;

@@ -173,17 +173,31 @@ simt_chunk_kernel(const FwdParams p) {
         if (GENERAL) {
             // per channel: preconditioner EMA (carried across chunks), write
             // key, erase key, cumulative log decay
+            // preconditioner factor f(rho): 1 1/sqrt(rho+eps), 2 1/(rho+eps) (Diag(A)^-1),
+            // 3 the latter squashed into [1/x, x] on a log scale; applied to the
+            // write key (forms 2, 3 read the state with the raw key) or to the query
+            const float lnx = p.precond == 3 ? logf(p.precond_x) : 1.f;
             for (int c = tid; c < dk; c += kThreads) {
                 float rh = rho[c], G = 0.f;
                 for (int r = 0; r < C; ++r) {
                     const int idx = r * dk + c;
-                    float kv = ld_s(kx, idx);
+                    const float kv = ld_s(kx, idx);
+                    float f = 1.f;
                     if (p.precond && r < Cv) {
                         rh = p.rho_decay * rh + kv * kv;
-                        kv = kv / sqrtf(rh + p.rho_eps);
-                        st_s(kx, idx, kv);
+                        const float a = rh + p.rho_eps;
+                        f = p.precond == 1 ? rsqrtf(a)
+                          : p.precond == 2 ? 1.f / a
+                          : expf(lnx * tanhf(-logf(a) / lnx));
                     }
-                    ex[idx] *= kv;
+                    if (p.precond_query) {
+                        st_s(qx, idx, ld_s(qx, idx) * f);
+                        ex[idx] *= kv;
+                    } else {
+                        const float kw = kv * f;
+                        st_s(kx, idx, kw);
+                        ex[idx] *= (p.precond == 1 ? kw : kv);
+                    }
                     G += gx[idx];
                     gx[idx] = G;
                 }

@@ -58,6 +58,7 @@ class FwdArgs(ctypes.Structure):
         ("kernel", ctypes.c_int32), ("dv_split", ctypes.c_int32),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_uint64),
         ("residual_S", ctypes.c_int32),
+        ("precond_x", ctypes.c_float), ("precond_query", ctypes.c_int32),
     ]
 
 
@@ -196,7 +197,8 @@ def device_check(stream: Optional[int] = None) -> None:
 def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
               alpha: Optional[torch.Tensor] = None, beta: Optional[torch.Tensor] = None, *,
               erase: Optional[torch.Tensor] = None, write: Optional[torch.Tensor] = None,
-              precond: bool = False, rho_decay: float = 0.99, rho_eps: float = 1e-6,
+              precond: int = 0, rho_decay: float = 0.99, rho_eps: float = 1e-6,
+              precond_x: float = 2.0, precond_query: bool = False,
               S0: Optional[torch.Tensor] = None, chunk: int = 64, mode: str = "exact",
               N: int = 3, S: int = 8, o_dtype: Optional[torch.dtype] = None, kernel: str = "auto",
               dv_split: int = 0, out: Optional[torch.Tensor] = None,
@@ -208,7 +210,9 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     q, k: [B, T, H, dk]; v: [B, T, H, dv] (bf16 or fp32, same dtype).
     alpha: [B, T, H] or [B, T, H, dk] fp32 decay (None = 1); beta: [B, T, H]
     fp32 (None = 1).  erase [B, T, H, dk], write [B, T, H, dv] gates and
-    ``precond`` select the preconditioned two-gate rule.  S0 / S_T:
+    ``precond`` select the preconditioned two-gate rule: 1 (or True) the
+    moving-average factor 1/sqrt(rho + eps), 2 Diag(A_t)^-1, 3 that squashed into
+    [1/precond_x, precond_x]; ``precond_query`` moves the factor to the query.  S0 / S_T:
     [B, H, dk, dv] fp32 (h = S^T).  ``o_dtype`` defaults to q's dtype.
     ``mode``: "exact", "neumann" (masked series to order N) or "residual" (the
     masked series corrected with S residual terms).
@@ -239,7 +243,8 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     args = make_args(
         B=B, T=T, H=H, dk=dk, dv=dv, chunk=int(chunk), io_dtype=_dtype_code(io),
         o_dtype=_dtype_code(od), q=_ptr(q), k=_ptr(k), v=_ptr(v), alpha=_ptr(alpha),
-        alpha_per_channel=int(per_channel), beta=_ptr(beta), precond=int(bool(precond)),
+        alpha_per_channel=int(per_channel), beta=_ptr(beta), precond=int(precond),
+        precond_x=float(precond_x), precond_query=int(bool(precond_query)),
         rho_decay=float(rho_decay), rho_eps=float(rho_eps), erase=_ptr(erase),
         write=_ptr(write), S0=_ptr(S0), o=_ptr(out), S_T=_ptr(S_T), mode=MODES[mode],
         neumann_N=int(N), residual_S=int(S), kernel=KERNELS[kernel], dv_split=int(dv_split))

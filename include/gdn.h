@@ -69,7 +69,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 3
+#define GDN_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define GDN_API __attribute__((visibility("default")))
@@ -117,7 +117,14 @@ typedef struct {
     const float *alpha;         /* decay in (0, 1]; NULL => 1 */
     int32_t alpha_per_channel;  /* 0: [B,T,H]; 1: [B,T,H,dk] */
     const float *beta;          /* write strength; NULL => 1 */
-    int32_t precond;            /* 1: diagonal curvature preconditioned write key */
+    int32_t precond;            /* diagonal curvature preconditioner, a per-channel factor
+                                   f of rho_t = rho_decay rho_{t-1} + k_t (.) k_t:
+                                   0 none; 1 f = 1/sqrt(rho + eps), erase read with the
+                                   preconditioned key; 2 f = 1/(rho + eps) (P_t =
+                                   Diag(A_t)^-1); 3 form 2 squashed into [1/x, x] on a
+                                   log scale, x = precond_x ("Preconditioned DeltaNet",
+                                   Arabic summary 2b; "Resumo Tecnico" section 2).
+                                   Forms 2, 3 read the state with the raw key. */
     float rho_decay, rho_eps;   /* preconditioner EMA constant and epsilon */
     const void *erase;          /* erase gate b_t or NULL (=> 1); needs beta == NULL */
     const void *write;          /* write gate w_t or NULL (=> 1); needs beta == NULL */
@@ -132,6 +139,9 @@ typedef struct {
                                    16-byte aligned, caller-owned; may be NULL when that is 0 */
     uint64_t workspace_bytes;   /* size of workspace */
     int32_t residual_S;         /* S for GDN_INV_NEUMANN_RESIDUAL: 0 <= S <= 64 */
+    float precond_x;            /* squash bound x > 1 for precond 3 */
+    int32_t precond_query;      /* 1: apply the factor to the query (ATQ) instead of the
+                                   write key (ATK); the write key is then k_t itself */
 } gdn_fwd_args;
 
 /* Chunkwise forward: o and S_T from q, k, v, gates and S0 (see above). */

@@ -25,7 +25,7 @@ def declared_functions():
 
 def test_library_builds_and_loads():
     gbuild.build()
-    assert gdn.abi_version() == 3
+    assert gdn.abi_version() == 4
 
 
 def test_exports_every_declared_symbol():
@@ -78,6 +78,10 @@ def _args(**kw):
     (dict(kernel=3, dv=16), GDN_ERR_UNSUPPORTED),       # recurrent kernel needs dv % 32 == 0
     (dict(kernel=3, alpha=0x70000, alpha_per_channel=1), GDN_ERR_UNSUPPORTED),   # two-gate rule
     (dict(kernel=3, mode=1, neumann_N=3), GDN_ERR_UNSUPPORTED),
+    (dict(precond=4, alpha=0x70000, alpha_per_channel=1), GDN_ERR_INVALID_ARG),
+    (dict(precond=3, precond_x=1.0, alpha=0x70000, alpha_per_channel=1), GDN_ERR_INVALID_ARG),
+    (dict(precond_query=1), GDN_ERR_INVALID_ARG),       # query placement needs a preconditioner
+    (dict(precond=2, precond_query=2), GDN_ERR_INVALID_ARG),
 ])
 def test_invalid_arguments_rejected_on_host(kw, status):
     a = _args(**kw)

@@ -190,6 +190,46 @@ def test_precond_two_gate_full_size():
     _check_bf16("precond_full_auto", w, x, o_ref, s_ref)
 
 
+# ------------------------------ page-form preconditioner variants (next row 3)
+
+def _precond_case(w, x, **kw):
+    import chunked_gated_delta_14_b200 as gdn
+    import oracle
+    o_ref, s_ref = oracle.precond_two_gate_fwd(x["q"], x["k"], x["v"], x["alpha"], x["erase"],
+                                               x["write"], h0=x["S0"], **kw)
+    d = {k: (None if v is None else v.cuda()) for k, v in x.items()}
+    o, s = gdn.chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], None, erase=d["erase"], write=d["write"],
+                         S0=d["S0"], o_dtype=torch.float32, **kw)
+    torch.cuda.synchronize()
+    return o.double().cpu().numpy(), s.double().cpu().numpy(), o_ref, s_ref
+
+
+@needs_cuda
+@pytest.mark.parametrize("form,query", [(2, False), (3, False), (2, True), (3, True), (1, True)])
+def test_page_form_preconditioners(form, query):
+    """P_t = Diag(A_t)^-1 with the plain running sum (form 2; eps 1 keeps it
+    bounded), its squash into [1/2, 2] (form 3), on the write key (ATK) or the
+    query (ATQ), on the two-gate engine with per-channel decay and S0."""
+    w = workload("precond_two_gate", B=1, H=2, T=300, s0_std=0.02)
+    x = make_inputs(w, seed=21)
+    kw = dict(precond=form, rho_decay=1.0, rho_eps=1.0 if form == 2 else 1e-6, precond_x=2.0,
+              precond_query=query)
+    o, s, o_ref, s_ref = _precond_case(w, x, **kw)
+    so, ss = stats(o, o_ref), stats(s, s_ref)
+    report(f"precond_form{form}_{'atq' if query else 'atk'}", o=so, S_T=ss)
+    assert so["max_rel_rms"] <= TOL_BF16_REL_RMS and ss["max_rel_rms"] <= TOL_BF16_REL_RMS
+
+
+@needs_cuda
+def test_squashed_preconditioner_full_size():
+    w = workload("precond_two_gate")
+    x = make_inputs(w)
+    o, s, o_ref, s_ref = _precond_case(w, x, precond=3, rho_decay=1.0, rho_eps=1e-6, precond_x=2.0)
+    so, ss = stats(o, o_ref), stats(s, s_ref)
+    report("precond_form3_full", o=so, S_T=ss)
+    assert so["max_rel_rms"] <= TOL_BF16_REL_RMS and ss["max_rel_rms"] <= TOL_BF16_REL_RMS
+
+
 # ------------------------------------------------------------------ edges
 
 @needs_cuda
