@@ -82,24 +82,29 @@ def algorithmic_flops(w):
     return f * chunks * w.B * w.H
 
 
-def kernel_source_sha():
+DECODE_PROFILE = os.path.join(ROOT, "profiles", "gdn_decode_recurrent_ncu.md")
+DECODE_SOURCES = ("gdn_recurrent.cu", "gdn_internal.cuh")
+
+
+def kernel_source_sha(files=None):
+    """sha256 prefix over the kernel sources (all of csrc, or the given files)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "chunked_gated_delta_14_b200", "csrc")
     for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh")):
+        if fn.endswith((".cu", ".cuh")) and (files is None or fn in files):
             h.update(open(os.path.join(csrc, fn), "rb").read())
     return h.hexdigest()[:16]
 
 
-def profile_traffic(kernel_name):
-    """dram read+write bytes per launch from the committed ncu summary, if it was
+def profile_traffic(kernel_name, path=PROFILE, files=None):
+    """dram read+write bytes per launch from a committed ncu summary, if it was
     taken on the current kernel sources."""
-    if not os.path.exists(PROFILE):
+    if not os.path.exists(path):
         return None
-    txt = open(PROFILE).read()
+    txt = open(path).read()
     m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
     m_k = re.search(rf"traffic_bytes_per_launch\[{re.escape(kernel_name)}\]:\s*([0-9.e+]+)", txt)
-    if not (m_sha and m_k) or m_sha.group(1) != kernel_source_sha():
+    if not (m_sha and m_k) or m_sha.group(1) != kernel_source_sha(files):
         return None
     return float(m_k.group(1))
 
@@ -417,8 +422,11 @@ def run_decode(args, rank, world, local_rank):
     pk = peaks()
     bytes_step = decode_bytes(w)
     achieved = bytes_step / (ms_step / 1e3) / 1e9
+    traffic = profile_traffic("recurrent_kernel", DECODE_PROFILE, DECODE_SOURCES)
+    if traffic is not None:
+        traffic *= w.B / 128            # the summary is taken at B = 128; traffic scales with B
     roof = dict(bound="hbm", achieved=achieved, peak=pk["hbm_gbs"], unit="GB/s",
-                frac=achieved / pk["hbm_gbs"], traffic=None,
+                frac=achieved / pk["hbm_gbs"], traffic=traffic,
                 peak_source=pk["source"] + " (burst copy bandwidth)",
                 algorithmic_bytes_per_launch=bytes_step,
                 roofline_ms=bytes_step / (pk["hbm_gbs"] * 1e9) * 1e3)
