@@ -1,40 +1,40 @@
 // Tensor-core path of the chunkwise gated delta rule on sm_100a: two kernels.
 //
-// 1. keyside_kernel -- the chunk-local A/T builder, one CTA per (chunk, head,
-//    batch), all chunks in parallel.  TMA loads the chunk's keys; a tcgen05
-//    MMA forms the Gram matrix K K^T (bf16 operands, exact products, fp32 in
-//    TMEM); the decayed strictly lower L_ri = beta_r exp(g_r - g_i) (k_r.k_i)
-//    (A = -L) is formed on the CUDA cores and T = (I - A)^-1 is built either
+// 1. keyside_kernel -- the state-independent part of every chunk, one CTA per
+//    (chunk, head, batch), all chunks in parallel.  TMA loads Q and K; one
+//    tcgen05 MMA forms [Q ; K] K^T (bf16, exact products, fp32 in TMEM).  From
+//    TMEM: the decayed causal scores P_ri = (q_r.k_i) exp(g_r - g_i), i <= r,
+//    and L_ri = beta_r exp(g_r - g_i) (k_r.k_i), i < r (A = -L).  T = (I - A)^-1
 //    exactly (16 x 16 diagonal blocks by forward substitution, merged
-//    16 -> 32 -> 64 by T21 = -T22 L21 T11) or as the masked truncated Neumann
-//    series M^(N) (.) sum_{n<=N} A^n by Horner's rule on the band.  T is
-//    written in fp16 to a workspace ([B, H, chunks, 64, 64]).
-//
+//    16 -> 32 -> 64 by T21 = -T22 L21 T11), or the masked truncated Neumann
+//    series M^(N) (.) sum_{n<=N} A^n (Horner on the band), optionally followed
+//    by the residual correction T0 sum_{s<=S} E^s.  Written to the workspace
+//    as fp16: T diag(beta), T diag(beta e^g) and P, 24 KB per chunk-head.
 // 2. chain_kernel -- one CTA per (batch, head, 64-column value slice) walks
 //    the chunks in order with the fp32 state h = S^T (128 x 64) in TMEM.
-//      warp 0      TMA producer: q, k, v slice, T of chunk m (2-stage ring)
+//      warp 0      TMA producer: q, k, v slice and the workspace rows (2 stages)
 //      warp 1      TMEM allocation
 //      warps 2-9   key side of chunk m (runs ahead of the chain): gate scan,
-//                  Gram Q K^T -> decayed causal scores P, fp16 operands
-//                  Q' = diag(e^g) Q, K, beta V, T diag(beta e^g), and the WY
-//                  products U = T (beta V), W = T diag(beta e^g) K (MMAs)
+//                  fp16 operands Q' = diag(e^g) Q, K, V; U = T diag(beta) V and
+//                  W = T diag(beta e^g) K (MMAs); -W to shared memory; K
+//                  rescaled in place by e^{g_C - g} for the state update
 //      warps 10-13 state chain:
 //                  h16 <- h;  h <- e^{g_C} h               (TMEM)
 //                  [-W h ; Q' h] = [-W ; Q'] h16            (MMA)
 //                  Delta = U - W h                          (CUDA cores)
-//                  O = Q'h + P Delta ; h += K^T (e^{g_C - g} Delta)   (MMAs)
+//                  h += (e^{g_C - g} K)^T Delta, then O = Q'h + P Delta (MMAs)
 //    Every MMA is tcgen05.mma kind::f16, M = 128: a 64-row operand is paired
-//    with whatever 64 rows follow it in shared memory; the TMEM lanes those
-//    rows produce are never read (or are read before they are overwritten).
-//    Derived operands are fp16: with bf16 operands the outputs of this
-//    workload leave the 2e-2-of-RMS accuracy bar, with fp16 they stay inside.
+//    with the 64 rows that follow it in the same stage; the TMEM lanes those
+//    rows produce are never read.  Derived operands are fp16: with bf16 ones
+//    this workload's outputs leave the 2e-2-of-RMS accuracy bar.
 //
 // The recurrence is S_t = S_{t-1} alpha_t (I - beta_t k_t k_t^T) +
 // beta_t v_t k_t^T, o_t = S_t q_t; the chunk system (I - A) Delta =
 // diag(beta)(V - diag(e^g) K h) with T = (I - A)^-1 is the step "Quando o 'Bom
 // o Suficiente' e Otimo: Aproximacao de Inversao de Matriz Baseada Apenas em
 // Multiplicacao para Gated DeltaNet Quantizado" (section "Declaracao do
-// Problema") singles out; its Neumann and mask items are "Metodologia" 1, 2.
+// Problema") singles out; its Neumann, mask and residual items are
+// "Metodologia" 1-3.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
