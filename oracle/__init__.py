@@ -6,8 +6,9 @@ package imports nothing from it: the two share no code.
 
 Contents
 --------
-``recurrent``   token-by-token recurrences in plain C (fp64), loaded with
-                ctypes from ``libgdn_oracle.so`` (compiled from
+``recurrent``   token-by-token recurrences in plain C (fp64), and the
+                adjoint of the gated delta rule for its gradients, loaded
+                with ctypes from ``libgdn_oracle.so`` (compiled from
                 ``gdn_oracle.c`` with gcc on first use).
 ``chunk_forms`` the intra-chunk pieces the pages define (the triangular
                 inverse, the truncated Neumann series, the structural mask,
@@ -16,4 +17,4 @@ Contents
                 numpy.
 """
 from . import chunk_forms, recurrent  # noqa: F401
-from .recurrent import gated_delta_fwd, precond_two_gate_fwd  # noqa: F401
+from .recurrent import gated_delta_bwd, gated_delta_fwd, precond_two_gate_fwd  # noqa: F401

@@ -224,3 +224,176 @@ void oracle_precond_two_gate_fwd(int B, int T, int H, int dk, int dv,
         free(p);
     }
 }
+
+/*
+ * Reverse-mode gradient of oracle_gated_delta_fwd (the training use the pages
+ * give chunkwise forms for: "Quando o 'Bom o Suficiente' e Otimo ...",
+ * sections "Resumo" and "Declaracao do Problema").  The pages print no
+ * backward pass; this is the adjoint of the token recurrence, one token at a
+ * time in reverse order, derived by the chain rule from the forward update.
+ *
+ * Inputs as in the forward, plus
+ *   dout [B,T,H,dv]           gradient of the loss with respect to o
+ *   dhT  [B,H,dk,dv] or NULL  gradient with respect to the final state h_T
+ * Outputs (all written in full; NULL skips one)
+ *   dq, dkk [B,T,H,dk]; dvv [B,T,H,dv]; dalpha, dbeta [B,T,H]; dh0 [B,H,dk,dv]
+ *
+ * With S_t = alpha_t S_{t-1} + u_t k_t^T, u_t = beta_t (v_t - alpha_t p_t),
+ * p_t = S_{t-1} k_t, o_t = S_t q_t, and D = dL/dS_t (d_v x d_k) the gradient
+ * reaching S_t from later tokens:
+ *   D      += do_t q_t^T                    (read-out of token t)
+ *   dq_t    = S_t^T do_t
+ *   du      = D k_t
+ *   dv_t    = beta_t du
+ *   dbeta_t = du . (v_t - alpha_t p_t)
+ *   dalpha_t= <D, S_{t-1}> - beta_t du . p_t
+ *   dk_t    = D^T u_t - alpha_t beta_t S_{t-1}^T du
+ *   D      <- alpha_t D - alpha_t beta_t du k_t^T      (dL/dS_{t-1})
+ * and dh0 = D^T after the first token.
+ *
+ * The states S_{t-1} are needed in reverse order.  They are recomputed from
+ * checkpoints kept every SEG tokens: the recomputation repeats the forward's
+ * operations in the forward's order, so every state is bit-identical to the
+ * one the forward produced; only the memory footprint changes.
+ */
+#define ORACLE_SEG 64
+
+static void fwd_token(double *S, double *p, int dk, int dv, const double *kt,
+                      const double *vt, double a, double be)
+{
+    for (int j = 0; j < dv; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < dk; ++i) acc += S[(size_t)j * dk + i] * kt[i];
+        p[j] = acc;
+    }
+    for (int j = 0; j < dv; ++j) {
+        const double cp = a * be * p[j], cv = be * vt[j];
+        double *row = S + (size_t)j * dk;
+        for (int i = 0; i < dk; ++i)
+            row[i] = a * row[i] - cp * kt[i] + cv * kt[i];
+    }
+}
+
+void oracle_gated_delta_bwd(int B, int T, int H, int dk, int dv,
+                            const double *q, const double *k, const double *v,
+                            const double *alpha, const double *beta,
+                            const double *h0, const double *dout, const double *dhT,
+                            double *dq, double *dkk, double *dvv,
+                            double *dalpha, double *dbeta, double *dh0,
+                            int nthreads)
+{
+    const int nseg = (T + ORACLE_SEG - 1) / ORACLE_SEG;
+    const size_t SZ = (size_t)dv * dk;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int bh = 0; bh < B * H; ++bh) {
+        const int b = bh / H, h = bh % H;
+        /* ckpt[s] = state before token s*SEG; seg[i] = state after token s*SEG+i-1 */
+        double *ckpt = (double *)calloc((size_t)nseg * SZ, sizeof(double));
+        double *seg = (double *)malloc((size_t)(ORACLE_SEG + 1) * SZ * sizeof(double));
+        double *S = (double *)calloc(SZ, sizeof(double));
+        double *D = (double *)calloc(SZ, sizeof(double));
+        double *p = (double *)malloc((size_t)dv * sizeof(double));
+        double *u = (double *)malloc((size_t)dv * sizeof(double));
+        double *du = (double *)malloc((size_t)dv * sizeof(double));
+        if (h0) {
+            const double *src = h0 + (size_t)bh * dk * dv;
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j)
+                    S[(size_t)j * dk + i] = src[(size_t)i * dv + j];
+        }
+        /* forward sweep, keeping the checkpoints */
+        for (int t = 0; t < T; ++t) {
+            if (t % ORACLE_SEG == 0) memcpy(ckpt + (size_t)(t / ORACLE_SEG) * SZ, S, SZ * sizeof(double));
+            const size_t r = tok(b, t, h, T, H);
+            fwd_token(S, p, dk, dv, k + r * dk, v + r * dv,
+                      alpha ? alpha[r] : 1.0, beta ? beta[r] : 1.0);
+        }
+        if (dhT) {
+            const double *src = dhT + (size_t)bh * dk * dv;
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j)
+                    D[(size_t)j * dk + i] = src[(size_t)i * dv + j];
+        }
+        /* reverse sweep, one segment at a time */
+        for (int s = nseg - 1; s >= 0; --s) {
+            const int t0 = s * ORACLE_SEG;
+            const int t1 = (t0 + ORACLE_SEG < T) ? t0 + ORACLE_SEG : T;
+            memcpy(seg, ckpt + (size_t)s * SZ, SZ * sizeof(double));
+            for (int t = t0; t < t1; ++t) {
+                const size_t r = tok(b, t, h, T, H);
+                double *Sn = seg + (size_t)(t - t0 + 1) * SZ;
+                memcpy(Sn, Sn - SZ, SZ * sizeof(double));
+                fwd_token(Sn, p, dk, dv, k + r * dk, v + r * dv,
+                          alpha ? alpha[r] : 1.0, beta ? beta[r] : 1.0);
+            }
+            for (int t = t1 - 1; t >= t0; --t) {
+                const size_t r = tok(b, t, h, T, H);
+                const double *St = seg + (size_t)(t - t0 + 1) * SZ;  /* S_t */
+                const double *Sp = St - SZ;                          /* S_{t-1} */
+                const double *kt = k + r * dk, *qt = q + r * dk, *vt = v + r * dv;
+                const double *dot = dout + r * dv;
+                const double a = alpha ? alpha[r] : 1.0;
+                const double be = beta ? beta[r] : 1.0;
+                for (int j = 0; j < dv; ++j)
+                    for (int i = 0; i < dk; ++i) D[(size_t)j * dk + i] += dot[j] * qt[i];
+                if (dq)
+                    for (int i = 0; i < dk; ++i) {
+                        double acc = 0.0;
+                        for (int j = 0; j < dv; ++j) acc += St[(size_t)j * dk + i] * dot[j];
+                        dq[r * dk + i] = acc;
+                    }
+                for (int j = 0; j < dv; ++j) {
+                    double pj = 0.0, dj = 0.0;
+                    for (int i = 0; i < dk; ++i) {
+                        pj += Sp[(size_t)j * dk + i] * kt[i];
+                        dj += D[(size_t)j * dk + i] * kt[i];
+                    }
+                    p[j] = pj;
+                    du[j] = dj;
+                    u[j] = be * (vt[j] - a * pj);
+                }
+                if (dvv)
+                    for (int j = 0; j < dv; ++j) dvv[r * dv + j] = be * du[j];
+                if (dbeta) {
+                    double acc = 0.0;
+                    for (int j = 0; j < dv; ++j) acc += du[j] * (vt[j] - a * p[j]);
+                    dbeta[r] = acc;
+                }
+                if (dalpha) {
+                    double acc = 0.0;
+                    for (size_t x = 0; x < SZ; ++x) acc += D[x] * Sp[x];
+                    for (int j = 0; j < dv; ++j) acc -= be * du[j] * p[j];
+                    dalpha[r] = acc;
+                }
+                if (dkk)
+                    for (int i = 0; i < dk; ++i) {
+                        double acc = 0.0;
+                        for (int j = 0; j < dv; ++j)
+                            acc += D[(size_t)j * dk + i] * u[j] - a * be * Sp[(size_t)j * dk + i] * du[j];
+                        dkk[r * dk + i] = acc;
+                    }
+                for (int j = 0; j < dv; ++j) {
+                    double *row = D + (size_t)j * dk;
+                    const double c = a * be * du[j];
+                    for (int i = 0; i < dk; ++i) row[i] = a * row[i] - c * kt[i];
+                }
+            }
+        }
+        if (dh0) {
+            double *dst = dh0 + (size_t)bh * dk * dv;
+            for (int i = 0; i < dk; ++i)
+                for (int j = 0; j < dv; ++j)
+                    dst[(size_t)i * dv + j] = D[(size_t)j * dk + i];
+        }
+        free(ckpt);
+        free(seg);
+        free(S);
+        free(D);
+        free(p);
+        free(u);
+        free(du);
+    }
+}

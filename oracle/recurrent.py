@@ -2,9 +2,10 @@
 
 Test infrastructure only.  Inputs may be numpy arrays or CPU torch tensors of
 any float dtype; they are widened to float64 exactly as the CUDA path receives
-them (bf16 values widen losslessly).  Returns ``(o, h_T)`` as float64 numpy
-arrays with ``o`` shaped [B, T, H, d_v] and ``h_T`` shaped [B, H, d_k, d_v]
-(the transposed state h = S^T).
+them (bf16 values widen losslessly).  The forward functions return
+``(o, h_T)`` as float64 numpy arrays with ``o`` shaped [B, T, H, d_v] and
+``h_T`` shaped [B, H, d_k, d_v] (the transposed state h = S^T);
+``gated_delta_bwd`` returns the gradients of the gated delta rule.
 """
 from __future__ import annotations
 
@@ -47,6 +48,9 @@ def _load():
                                                         ctypes.c_double, ctypes.c_double, i,
                                                         dp, dp, dp, i]
             lib.oracle_precond_two_gate_fwd.restype = None
+            lib.oracle_gated_delta_bwd.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, dp, dp,
+                                                   dp, dp, dp, dp, dp, dp, dp, i]
+            lib.oracle_gated_delta_bwd.restype = None
             _lib = lib
     return _lib
 
@@ -121,3 +125,35 @@ def precond_two_gate_fwd(q, k, v, alpha=None, erase=None, write=None, precond=Tr
                                         float(precond_x), int(bool(precond_query)),
                                         _ptr(h0), _ptr(o), _ptr(hT), _threads(nthreads))
     return o, hT
+
+
+def gated_delta_bwd(q, k, v, alpha=None, beta=None, h0=None, do=None, dhT=None,
+                    nthreads=None):
+    """Gradients of the gated delta rule by the token-by-token adjoint.
+
+    ``do`` [B, T, H, d_v] is dL/do; ``dhT`` [B, H, d_k, d_v] (or None, meaning
+    0) is dL/dh_T.  Returns a dict with ``dq``, ``dk`` [B, T, H, d_k], ``dv``
+    [B, T, H, d_v], ``dalpha`` and ``dbeta`` [B, T, H] (None when the gate was
+    None) and ``dh0`` [B, H, d_k, d_v] (dL/dh_0, also when h0 is None).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    alpha, beta, h0 = _f64(alpha), _f64(beta), _f64(h0)
+    do, dhT = _f64(do), _f64(dhT)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == q.shape and v.shape[:3] == q.shape[:3] and do.shape == v.shape
+    for a in (alpha, beta):
+        assert a is None or a.shape == (B, T, H)
+    for s in (h0, dhT):
+        assert s is None or s.shape == (B, H, dk, dv)
+    out = dict(dq=np.zeros((B, T, H, dk)), dk=np.zeros((B, T, H, dk)),
+               dv=np.zeros((B, T, H, dv)),
+               dalpha=None if alpha is None else np.zeros((B, T, H)),
+               dbeta=None if beta is None else np.zeros((B, T, H)),
+               dh0=np.zeros((B, H, dk, dv)))
+    _load().oracle_gated_delta_bwd(B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                   _ptr(beta), _ptr(h0), _ptr(do), _ptr(dhT),
+                                   _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                                   _ptr(out["dalpha"]), _ptr(out["dbeta"]), _ptr(out["dh0"]),
+                                   _threads(nthreads))
+    return out
