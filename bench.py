@@ -8,8 +8,11 @@ WY products, state passing, output).  Inputs are synthetic (seeded), resident
 in HBM when the timed region starts.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--batch B]
+                  [--mode exact|neumann|residual] [--decode] [--bwd]
 
 ``--batch B`` replaces the batch size (a smaller case for profiler captures).
+``--decode`` times one-token decode steps; ``--bwd`` times the backward pass
+(gradients of q, k, v, alpha, beta) on the same workload.
 
 Under torchrun each rank runs its own independent batch (weak scaling, no
 collective on the data path); the time is the max over ranks.
@@ -82,12 +85,13 @@ def algorithmic_flops(w):
     return f * chunks * w.B * w.H
 
 
+FWD_SOURCES = ("gdn_tc.cu", "gdn_tc_common.cuh", "sm100.cuh", "gdn_internal.cuh")
 DECODE_PROFILE = os.path.join(ROOT, "profiles", "gdn_decode_recurrent_ncu.md")
 DECODE_SOURCES = ("gdn_recurrent.cu", "gdn_internal.cuh")
 
 
 def kernel_source_sha(files=None):
-    """sha256 prefix over the kernel sources (all of csrc, or the given files)."""
+    """sha256 prefix over the given kernel sources (all of csrc when None)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "chunked_gated_delta_14_b200", "csrc")
     for fn in sorted(os.listdir(csrc)):
@@ -96,7 +100,7 @@ def kernel_source_sha(files=None):
     return h.hexdigest()[:16]
 
 
-def profile_traffic(kernel_name, path=PROFILE, files=None):
+def profile_traffic(kernel_name, path=PROFILE, files=FWD_SOURCES):
     """dram read+write bytes per launch from a committed ncu summary, if it was
     taken on the current kernel sources."""
     if not os.path.exists(path):
@@ -458,6 +462,171 @@ def run_decode(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+BWD_METRIC = "backward tokens/s (bf16 in, fp32 gradients, H=16, d=128, T=4096) and % of fp32 roofline on 1 B200"
+BWD_SOURCES = ("gdn_bwd.cu", "gdn_bwd_kernels.cuh", "gdn_bwd_params.cuh")
+BWD_PROFILE = os.path.join(ROOT, "profiles", "gdn_bwd_gdn_bf16_ncu.md")
+
+
+def fp32_alu_peak_tflops(sm_mhz=1965.0):
+    """CUDA-core fp32 peak: 148 SMs x 128 fp32 lanes x 2 flops (FMA) x clock."""
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def algorithmic_flops_bwd(w):
+    """Per chunk-head, the products of the chunked backward (fp32):
+    8 state-sized products 2*C*dk*dv (Delta = U - W h, the state update; dDelta's
+    K dh', the two terms of dh; dO h^T, Y h^T, Delta dh'^T), the score-sized ones
+    C^2 (9 dk + 5 dv) (Gram and scores twice, W and U, M^T dO and T^T dDelta,
+    dO Delta^T and Y Delta^T, the four score-times-key products of dq and dk)
+    and the triangular inverse C^3 / 3."""
+    C, dk, dv = w.chunk, w.dk, w.dv
+    f = 16 * C * dk * dv + C * C * (9 * dk + 5 * dv) + C ** 3 / 3
+    return f * -(-w.T // C) * w.B * w.H
+
+
+def bwd_bytes(w):
+    """Bytes the backward must move once: q, k, v, grad_o read (io dtype), alpha,
+    beta read (fp32); dq, dk, dv, dalpha, dbeta written (fp32)."""
+    in_b = 2 if w.io == "bf16" else 4
+    per_th = (2 * w.dk + 2 * w.dv) * in_b + 8 + (2 * w.dk + w.dv) * 4 + 8
+    return w.token_heads * per_th
+
+
+def run_bwd(args, rank, world, local_rank):
+    """One gdn_chunk_bwd call per step over the whole batch."""
+    import torch
+    import chunked_gated_delta_14_b200 as gdn
+    from chunked_gated_delta_14_b200.inputs import make_cotangents, make_inputs, workload
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workload(WORKLOAD, **({"B": args.batch} if args.batch else {}))
+    x = make_inputs(w, seed=rank)
+    c = make_cotangents(w, seed=rank, grad_state=False)
+    d = {k: (None if v is None else v.to(dev)) for k, v in x.items()}
+    grad_o = c["grad_o"].to(dev)
+    f32 = dict(device=dev, dtype=torch.float32)
+    g = dict(dq=torch.empty((w.B, w.T, w.H, w.dk), **f32), dk=torch.empty((w.B, w.T, w.H, w.dk), **f32),
+             dv=torch.empty((w.B, w.T, w.H, w.dv), **f32), da=torch.empty((w.B, w.T, w.H), **f32),
+             db=torch.empty((w.B, w.T, w.H), **f32))
+    ptr = lambda t: None if t is None else t.data_ptr()
+    a = gdn.make_bwd_args(B=w.B, T=w.T, H=w.H, dk=w.dk, dv=w.dv, chunk=w.chunk, io_dtype=1,
+                          do_dtype=1, q=ptr(d["q"]), k=ptr(d["k"]), v=ptr(d["v"]),
+                          alpha=ptr(d["alpha"]), beta=ptr(d["beta"]), grad_o=ptr(grad_o),
+                          grad_q=ptr(g["dq"]), grad_k=ptr(g["dk"]), grad_v=ptr(g["dv"]),
+                          grad_alpha=ptr(g["da"]), grad_beta=ptr(g["db"]))
+    ws = gdn.workspace_for(a, dev)
+    a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    for _ in range(args.warmup):
+        gdn.call_bwd(a, sh)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    if rank == 0:
+        clocks.start()
+        time.sleep(1.0)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        gdn.call_bwd(a, sh)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    clocks.mark(t_wall0, t_wall1)
+    time.sleep(0.3)
+    clocks.stop()
+    ms_step = ms / args.steps
+    tokens_step = w.B * w.T
+    value = job_throughput(tokens_step, world, args.steps, ms)
+
+    # end to end through chunk_bwd: pinned host inputs and grad_o in, gradients back out
+    e2e = None
+    if args.e2e_steps > 0:
+        host = {k: x[k].pin_memory() for k in ("q", "k", "v", "alpha", "beta")}
+        host["grad_o"] = c["grad_o"].pin_memory()
+        dev_in = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+        outs_host = {k: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                     for k, t in (("dq", g["dq"]), ("dk", g["dk"]), ("dv", g["dv"]),
+                                  ("dalpha", g["da"]), ("dbeta", g["db"]))}
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = sum(t.numel() * t.element_size() for t in outs_host.values())
+
+        def e2e_step():
+            for k, t in host.items():
+                dev_in[k].copy_(t, non_blocking=True)
+            r = gdn.chunk_bwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"], dev_in["beta"],
+                              dev_in["grad_o"], chunk=w.chunk, want_S0=False)
+            for k, t in outs_host.items():
+                t.copy_(r[k], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        n_e2e = max(1, args.e2e_steps // 4)
+        f0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        ems = max_over_ranks(f0.elapsed_time(f1), world, dev)
+        e2e = dict(value=job_throughput(tokens_step, world, n_e2e, ems), unit=UNIT,
+                   h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h), ms_per_step=ems / n_e2e)
+
+    pk = peaks()
+    clk = clocks.summary()
+    alu_peak = fp32_alu_peak_tflops(clk["sm_max_mhz"] or 1965.0)
+    flops = algorithmic_flops_bwd(w)
+    achieved = flops / (ms_step / 1e3) / 1e12
+    nbytes = bwd_bytes(w)
+    roof = dict(bound="alu", achieved=achieved, peak=alu_peak, unit="TFLOP/s", frac=achieved / alu_peak,
+                traffic=profile_traffic("bwd_prep_kernel+bwd_state_fwd_kernel+bwd_state_rev_kernel+bwd_grad_kernel",
+                                        BWD_PROFILE, BWD_SOURCES),
+                peak_source="derived: 148 SMs x 128 fp32 lanes x 2 flops x max SM clock",
+                algorithmic_flops_per_launch=flops, algorithmic_bytes_per_launch=nbytes,
+                hbm_gbs=nbytes / (ms_step / 1e3) / 1e9, hbm_frac=nbytes / (ms_step / 1e3) / 1e9 / pk["hbm_gbs"],
+                roofline_ms=max(flops / (alu_peak * 1e12), nbytes / (pk["hbm_gbs"] * 1e9)) * 1e3)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        cores = len(os.sched_getaffinity(0))
+        Ts = min(w.T, 1024)
+        sl = lambda t: None if t is None else t[0:1, :Ts].contiguous()
+        n, t0 = 0, time.perf_counter()
+        while True:
+            oracle.gated_delta_bwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["alpha"]), sl(x["beta"]),
+                                   None, sl(c["grad_o"]), None, nthreads=cores)
+            n += 1
+            if time.perf_counter() - t0 >= min(args.cpu_budget, 10.0):
+                break
+        el = time.perf_counter() - t0
+        cpu = dict(value=Ts * n / el, unit=UNIT, cores=cores, kind="oracle",
+                   sample=f"{n} x (tokens [0,{Ts}) of one batch row, all {w.H} heads), fp64 C adjoint, {el:.1f} s")
+    if rank == 0:
+        line = dict(metric=BWD_METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps,
+                    warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",
+                    vs_baseline=None, dtype="f32",
+                    compute="bf16 q/k/v/grad_o in HBM; fp32 arithmetic on CUDA cores; fp32 gradients",
+                    data="synthetic (seeded; Gated DeltaNet layer shapes)",
+                    config=dict(workload=f"{WORKLOAD} backward: B={w.B} H={w.H} T={w.T} dk={w.dk} "
+                                f"dv={w.dv} chunk={w.chunk} exact inverse",
+                                global_batch=w.B * world, seq_len=w.T,
+                                parallelism=f"independent batch per GPU x{world}",
+                                l2=f"no flush: inputs+gradients {nbytes / 1e6:.0f} MB + workspace "
+                                   f"{ws.numel() / 1e6:.0f} MB per step > 126 MB L2",
+                                kernel="bwd_prep_kernel+bwd_state_fwd_kernel+bwd_state_rev_kernel+bwd_grad_kernel"),
+                    clocks=clk, e2e=e2e, gpu_launches=args.steps * 4, roofline=roof, cpu_baseline=cpu)
+        print(json.dumps(line), flush=True)
+
+
 def cpu_baseline(w, x, budget_s=12.0):
     """The fp64 oracle as it stands, timed on this host's cores, on whole
     (batch, head) sequences of the same workload until ~budget_s seconds."""
@@ -544,6 +713,8 @@ def main():
                          "(order --N), or the series with --S residual-correction terms")
     ap.add_argument("--decode", action="store_true",
                     help="decode steps (T = 1, state in place, B = 256 unless --batch)")
+    ap.add_argument("--bwd", action="store_true",
+                    help="the backward pass (gradients) on the same workload")
     ap.add_argument("--N", type=int, default=3)
     ap.add_argument("--S", type=int, default=8)
     args = ap.parse_args()
@@ -565,6 +736,8 @@ def main():
     try:
         if args.decode:
             run_decode(args, rank, world, local_rank)
+        elif args.bwd:
+            run_bwd(args, rank, world, local_rank)
         else:
             run_gpu(args, rank, world, local_rank)
     finally:

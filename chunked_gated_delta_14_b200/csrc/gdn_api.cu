@@ -5,6 +5,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "gdn_bwd.cuh"
 #include "gdn_internal.cuh"
 
 // Fixed scratch of gdn_chunk_fwd_static_scratch: the per-chunk T matrices of
@@ -150,6 +151,76 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
     return GDN_OK;
 }
 
+struct Span {
+    const void *p;
+    size_t bytes;
+};
+
+bool overlap(const Span &a, const Span &b) {
+    if (!a.p || !b.p || !a.bytes || !b.bytes) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a.p), y = reinterpret_cast<uintptr_t>(b.p);
+    return x < y + b.bytes && y < x + a.bytes;
+}
+
+// Validate the backward arguments; on success fills *out (workspace regions
+// not yet carved).  Never touches the GPU.
+gdn_status resolve_bwd(const gdn_bwd_args *a, gdn::BwdParams *out) {
+    if (!a) return fail(GDN_ERR_INVALID_ARG, "args is NULL");
+    if (a->B < 1 || a->H < 1 || a->T < 1)
+        return fail(GDN_ERR_INVALID_ARG, "B, T, H must be >= 1 (got %d, %d, %d)", a->B, a->T, a->H);
+    if (a->B > 65535 || a->H > 65535)
+        return fail(GDN_ERR_INVALID_ARG, "B and H must be <= 65535 (got %d, %d)", a->B, a->H);
+    if ((long long)a->B * a->T * a->H > (1ll << 40)) return fail(GDN_ERR_INVALID_ARG, "B*T*H too large");
+    if (a->io_dtype != GDN_F32 && a->io_dtype != GDN_BF16)
+        return fail(GDN_ERR_INVALID_ARG, "io_dtype %d unknown", a->io_dtype);
+    if (a->do_dtype != GDN_F32 && a->do_dtype != GDN_BF16)
+        return fail(GDN_ERR_INVALID_ARG, "do_dtype %d unknown", a->do_dtype);
+    if (!a->q || !a->k || !a->v || !a->grad_o)
+        return fail(GDN_ERR_INVALID_ARG, "q, k, v and grad_o are required");
+    if (!a->grad_q || !a->grad_k || !a->grad_v)
+        return fail(GDN_ERR_INVALID_ARG, "grad_q, grad_k and grad_v are required");
+    if (a->grad_alpha && !a->alpha) return fail(GDN_ERR_INVALID_ARG, "grad_alpha needs alpha");
+    if (a->grad_beta && !a->beta) return fail(GDN_ERR_INVALID_ARG, "grad_beta needs beta");
+    gdn::BwdParams p{};
+    p.B = a->B; p.T = a->T; p.H = a->H; p.dk = a->dk; p.dv = a->dv; p.C = a->chunk;
+    p.NC = (a->T + a->chunk - 1) / (a->chunk > 0 ? a->chunk : 1);
+    const char *why = "";
+    if (!gdn::bwd_supports(p, &why)) return fail(GDN_ERR_UNSUPPORTED, "backward: %s", why);
+
+    const size_t tok = (size_t)a->B * a->T * a->H;
+    const size_t io = a->io_dtype == GDN_BF16 ? 2 : 4, od = a->do_dtype == GDN_BF16 ? 2 : 4;
+    const size_t st = (size_t)a->B * a->H * a->dk * a->dv * 4;
+    const size_t ws = gdn::bwd_workspace_bytes(p);
+    const Span ins[] = {{a->q, tok * a->dk * io}, {a->k, tok * a->dk * io}, {a->v, tok * a->dv * io},
+                        {a->alpha, tok * 4}, {a->beta, tok * 4}, {a->S0, st},
+                        {a->grad_o, tok * a->dv * od}, {a->grad_S_T, st}};
+    const Span outs[] = {{a->grad_q, tok * a->dk * 4}, {a->grad_k, tok * a->dk * 4},
+                         {a->grad_v, tok * a->dv * 4}, {a->grad_alpha, tok * 4},
+                         {a->grad_beta, tok * 4}, {a->grad_S0, st},
+                         {a->workspace, a->workspace ? ws : 0}};
+    const int n_out = (int)(sizeof(outs) / sizeof(outs[0]));
+    for (int i = 0; i < n_out; ++i) {
+        for (const Span &x : ins)
+            if (overlap(outs[i], x)) return fail(GDN_ERR_INVALID_ARG, "an output or the workspace overlaps an input");
+        for (int j = i + 1; j < n_out; ++j)
+            if (overlap(outs[i], outs[j]))
+                return fail(GDN_ERR_INVALID_ARG, "outputs (or the workspace) overlap one another");
+    }
+    for (const Span &x : ins)
+        if (x.p && !aligned16(x.p)) return fail(GDN_ERR_ALIGNMENT, "pointers must be 16-byte aligned");
+    for (const Span &x : outs)
+        if (x.p && !aligned16(x.p)) return fail(GDN_ERR_ALIGNMENT, "pointers must be 16-byte aligned");
+
+    p.io_bf16 = a->io_dtype == GDN_BF16;
+    p.do_bf16 = a->do_dtype == GDN_BF16;
+    p.q = a->q; p.k = a->k; p.v = a->v; p.alpha = a->alpha; p.beta = a->beta; p.S0 = a->S0;
+    p.grad_o = a->grad_o; p.grad_S_T = a->grad_S_T;
+    p.grad_q = a->grad_q; p.grad_k = a->grad_k; p.grad_v = a->grad_v;
+    p.grad_alpha = a->grad_alpha; p.grad_beta = a->grad_beta; p.grad_S0 = a->grad_S0;
+    *out = p;
+    return GDN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -266,6 +337,28 @@ gdn_status gdn_chunk_fwd_static_scratch(const gdn_fwd_args *args, void *stream) 
     const char *why = "";
     e = gdn::launch_tc(p, scratch, reinterpret_cast<cudaStream_t>(stream), &why);
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "tc launch: %s %s", cudaGetErrorString(e), why);
+    g_msg[0] = 0;
+    return GDN_OK;
+}
+
+uint64_t gdn_bwd_workspace_bytes(const gdn_bwd_args *args) {
+    gdn::BwdParams p;
+    if (resolve_bwd(args, &p) != GDN_OK) return 0;
+    g_msg[0] = 0;
+    return (uint64_t)gdn::bwd_workspace_bytes(p);
+}
+
+gdn_status gdn_chunk_bwd(const gdn_bwd_args *args, void *stream) {
+    gdn::BwdParams p;
+    gdn_status s = resolve_bwd(args, &p);
+    if (s != GDN_OK) return s;
+    const size_t need = gdn::bwd_workspace_bytes(p);
+    if (!args->workspace || args->workspace_bytes < need)
+        return fail(GDN_ERR_INVALID_ARG, "backward needs a workspace of %zu bytes (got %llu)", need,
+                    (unsigned long long)args->workspace_bytes);
+    gdn::bwd_carve_workspace(p, args->workspace);
+    const cudaError_t e = gdn::launch_bwd(p, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "backward launch: %s", cudaGetErrorString(e));
     g_msg[0] = 0;
     return GDN_OK;
 }

@@ -1,0 +1,561 @@
+// Kernels of the chunked backward pass of the gated delta rule (fp32, CUDA
+// cores).  Device code only; the launchers are in gdn_bwd.cu.
+//
+// The pages give the chunkwise WY/UT form as what makes training parallel
+// ("Quando o 'Bom o Suficiente' e Otimo: Aproximacao de Inversao de Matriz
+// Baseada Apenas em Multiplicacao para Gated DeltaNet Quantizado", sections
+// "Resumo" and "Declaracao do Problema") but print no backward pass.  This is
+// the reverse-mode derivative of that chunk form, derived here.  Per chunk of
+// Cn tokens with h the state at its start (d_k x d_v, h = S^T), in-chunk
+// cumulative log decay g, Gamma_ri = e^{g_r - g_i} (i <= r):
+//
+//   forward   L_ri = beta_r Gamma_ri k_r.k_i (i < r),  T = (I + L)^-1
+//             U = T diag(beta) V,  W = T diag(beta e^g) K,  Delta = U - W h
+//             O = diag(e^g) Q h + M Delta,  M_ri = Gamma_ri q_r.k_i (i <= r)
+//             h' = e^{g_C} h + (diag(e^{g_C - g}) K)^T Delta
+//   backward  given dO and dh' (the gradient reaching h'):
+//             dDelta = M^T dO + diag(e^{g_C - g}) K dh'
+//             Y      = T^T dDelta
+//             dh     = e^{g_C} dh' + (diag(e^g) Q)^T dO - (diag(beta e^g) K)^T Y
+//             dV     = diag(beta) Y
+//             dM     = dO Delta^T (i <= r),   dL = -Y Delta^T (i < r)
+//             dQ     = diag(e^g) dO h^T + (dM (.) Gamma) K
+//             dK     = (dM (.) Gamma)^T Q + diag(e^{g_C - g}) Delta dh'^T
+//                      - diag(beta e^g) Y h^T + (dG + dG^T) K,
+//                      dG = diag(beta) (dL (.) Gamma)
+//             dbeta_r = Y_r.V_r - e^{g_r} k_r.(Y h^T)_r + sum_i dL_ri Gamma_ri k_r.k_i
+//             dg_r   = the partial derivatives of L, M, diag(e^g), W and h'
+//                      in g_r (see bwd_grad_kernel),
+//             dlog(alpha_t) = sum_{r >= t} dg_r,   dalpha_t = dlog(alpha_t) / alpha_t.
+// (dT = dDelta (Vb - Kb h)^T and dL = -T^T dT T^T collapse to -Y Delta^T
+// because T (Vb - Kb h) = Delta.)
+//
+// Four launches: prep (per chunk-head: g, L, T, M, W, U), the forward state
+// chain (per 32-column value slice: h at every chunk start, Delta), the
+// reverse chain (per slice: dh' at every chunk end, Y, dV, dS0) and the
+// key-side gradients (per chunk-head: dQ, dK, dbeta, dalpha).
+#pragma once
+
+#include "gdn_bwd_params.cuh"
+
+namespace gdn {
+namespace bwd {
+
+constexpr int kThreads = 256;
+constexpr int kCols = 32;     // value columns per block of the two chains and per tile
+constexpr int kMaxC = 64;     // largest chunk
+
+extern __shared__ float4 bwd_smem[];
+
+__device__ __forceinline__ float ld_in(const void *ptr, size_t i, int bf16) {
+    if (bf16) return __uint_as_float((unsigned int)reinterpret_cast<const uint16_t *>(ptr)[i] << 16);
+    return reinterpret_cast<const float *>(ptr)[i];
+}
+
+__device__ __forceinline__ size_t tok_index(const BwdParams &p, int b, int t, int h) {
+    return ((size_t)b * p.T + t) * p.H + h;
+}
+
+// ------------------------------------------------------------------- prep
+// One block per chunk-head.  Shared memory (floats): K, Q (C x (dk+1)),
+// V (C x (dv+1)), L, T (C x (C+1)), g, beta, beta e^g (C each).
+__host__ __device__ inline size_t prep_smem_floats(int C, int dk, int dv) {
+    return 2 * (size_t)C * (dk + 1) + (size_t)C * (dv + 1) + 2 * (size_t)C * (C + 1) + 3 * (size_t)C;
+}
+
+__global__ void __launch_bounds__(kThreads) bwd_prep_kernel(const BwdParams p) {
+    float *sm = reinterpret_cast<float *>(bwd_smem);
+    const int C = p.C, dk = p.dk, dv = p.dv;
+    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+    const int t0 = n * C;
+    const int Cn = min(C, p.T - t0);
+    const int dkp = dk + 1, dvp = dv + 1, Cp = C + 1;
+    float *Ks = sm;
+    float *Qs = Ks + C * dkp;
+    float *Vs = Qs + C * dkp;
+    float *Ls = Vs + C * dvp;
+    float *Ts = Ls + C * Cp;
+    float *g = Ts + C * Cp;
+    float *bb = g + C;
+    float *bg = bb + C;
+    const size_t ch = ((size_t)b * p.H + h) * p.NC + n;
+
+    for (int x = tid; x < C * dk; x += kThreads) {
+        const int r = x / dk, c = x % dk;
+        float kv = 0.f, qv = 0.f;
+        if (r < Cn) {
+            const size_t ti = tok_index(p, b, t0 + r, h) * dk + c;
+            kv = ld_in(p.k, ti, p.io_bf16);
+            qv = ld_in(p.q, ti, p.io_bf16);
+        }
+        Ks[r * dkp + c] = kv;
+        Qs[r * dkp + c] = qv;
+    }
+    for (int x = tid; x < C * dv; x += kThreads) {
+        const int r = x / dv, j = x % dv;
+        Vs[r * dvp + j] = r < Cn ? ld_in(p.v, tok_index(p, b, t0 + r, h) * dv + j, p.io_bf16) : 0.f;
+    }
+    for (int x = tid; x < C * C; x += kThreads) Ts[(x / C) * Cp + x % C] = 0.f;
+    if (tid == 0) {
+        float acc = 0.f;
+        for (int r = 0; r < C; ++r) {
+            float be = 0.f;
+            if (r < Cn) {
+                const size_t ti = tok_index(p, b, t0 + r, h);
+                if (p.alpha) acc += logf(p.alpha[ti]);
+                be = p.beta ? p.beta[ti] : 1.f;
+            }
+            g[r] = acc;          // rows past the tail repeat g_{Cn-1}; their beta is 0
+            bb[r] = be;
+            bg[r] = be * expf(acc);
+        }
+    }
+    __syncthreads();
+
+    // L (strictly lower) and M (lower with diagonal)
+    for (int x = tid; x < C * C; x += kThreads) {
+        const int r = x / C, i = x % C;
+        float l = 0.f, m = 0.f;
+        if (r < Cn && i <= r) {
+            float gk = 0.f, qk = 0.f;
+            for (int c = 0; c < dk; ++c) {
+                const float ki = Ks[i * dkp + c];
+                gk += Ks[r * dkp + c] * ki;
+                qk += Qs[r * dkp + c] * ki;
+            }
+            const float gam = expf(g[r] - g[i]);
+            m = gam * qk;
+            if (i < r) l = bb[r] * gam * gk;
+        }
+        Ls[r * Cp + i] = l;
+        p.ws_M[ch * C * C + x] = m;
+    }
+    __syncthreads();
+
+    // T = (I + L)^-1 one column per thread: (I + L) t = e_j by forward
+    // substitution, t_r = 0 above the diagonal.
+    if (tid < Cn) {
+        const int j = tid;
+        Ts[j * Cp + j] = 1.f;
+        for (int r = j + 1; r < Cn; ++r) {
+            float s = 0.f;
+            for (int i = j; i < r; ++i) s += Ls[r * Cp + i] * Ts[i * Cp + j];
+            Ts[r * Cp + j] = -s;
+        }
+    }
+    __syncthreads();
+
+    for (int x = tid; x < C * C; x += kThreads) p.ws_T[ch * C * C + x] = Ts[(x / C) * Cp + x % C];
+    if (tid < C) p.ws_g[ch * C + tid] = g[tid];
+    // W = T diag(beta e^g) K and U = T diag(beta) V (zero rows past the tail)
+    for (int x = tid; x < C * dk; x += kThreads) {
+        const int r = x / dk, c = x % dk;
+        float s = 0.f;
+        for (int i = 0; i <= r && i < Cn; ++i) s += Ts[r * Cp + i] * bg[i] * Ks[i * dkp + c];
+        p.ws_W[ch * C * dk + x] = s;
+    }
+    for (int x = tid; x < C * dv; x += kThreads) {
+        const int r = x / dv, j = x % dv;
+        float s = 0.f;
+        for (int i = 0; i <= r && i < Cn; ++i) s += Ts[r * Cp + i] * bb[i] * Vs[i * dvp + j];
+        p.ws_D[ch * C * dv + x] = s;
+    }
+}
+
+// ------------------------------------------------------ forward state chain
+// One block per (batch, head, 32 value columns); walks the chunks in order.
+// Shared memory: h (dk x 33), W, K e^{g_C - g} (C x (dk+1) each), Delta (C x 33).
+__host__ __device__ inline size_t state_fwd_smem_floats(int C, int dk) {
+    return (size_t)dk * 33 + 2 * (size_t)C * (dk + 1) + (size_t)C * 33;
+}
+
+__global__ void __launch_bounds__(kThreads) bwd_state_fwd_kernel(const BwdParams p) {
+    float *sm = reinterpret_cast<float *>(bwd_smem);
+    const int C = p.C, dk = p.dk, dv = p.dv;
+    const int j0 = blockIdx.x * kCols, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+    const int jj = tid & 31, rr = tid >> 5;
+    const int dkp = dk + 1;
+    float *hs = sm;
+    float *Ws = hs + dk * 33;
+    float *Ks = Ws + C * dkp;
+    float *Ds = Ks + C * dkp;
+    const size_t bh = (size_t)b * p.H + h;
+
+    for (int c = rr; c < dk; c += 8) hs[c * 33 + jj] = p.S0 ? p.S0[(bh * dk + c) * dv + j0 + jj] : 0.f;
+    for (int n = 0; n < p.NC; ++n) {
+        const int t0 = n * C, Cn = min(C, p.T - t0);
+        const size_t ch = bh * p.NC + n;
+        __syncthreads();   // h complete; the previous chunk's reads of W, K, Delta done
+        for (int c = rr; c < dk; c += 8) p.ws_h[(ch * dk + c) * dv + j0 + jj] = hs[c * 33 + jj];
+        const float glast = p.ws_g[ch * C + Cn - 1];
+        for (int x = tid; x < C * dk; x += kThreads) {
+            const int r = x / dk, c = x % dk;
+            Ws[r * dkp + c] = p.ws_W[ch * C * dk + x];
+            float kv = 0.f;
+            if (r < Cn)
+                kv = ld_in(p.k, tok_index(p, b, t0 + r, h) * dk + c, p.io_bf16) *
+                     expf(glast - p.ws_g[ch * C + r]);
+            Ks[r * dkp + c] = kv;
+        }
+        for (int r = rr; r < C; r += 8) Ds[r * 33 + jj] = p.ws_D[(ch * C + r) * dv + j0 + jj];
+        __syncthreads();
+        // Delta = U - W h
+        for (int r = rr; r < Cn; r += 8) {
+            float s = Ds[r * 33 + jj];
+            for (int c = 0; c < dk; ++c) s -= Ws[r * dkp + c] * hs[c * 33 + jj];
+            Ds[r * 33 + jj] = s;
+            p.ws_D[(ch * C + r) * dv + j0 + jj] = s;
+        }
+        __syncthreads();
+        // h <- e^{g_C} h + (diag(e^{g_C - g}) K)^T Delta
+        const float eglast = expf(glast);
+        for (int c = rr; c < dk; c += 8) {
+            float s = eglast * hs[c * 33 + jj];
+            for (int r = 0; r < Cn; ++r) s += Ks[r * dkp + c] * Ds[r * 33 + jj];
+            hs[c * 33 + jj] = s;
+        }
+    }
+}
+
+// ------------------------------------------------------ reverse state chain
+// One block per (batch, head, 32 value columns); walks the chunks backwards.
+// Shared memory: dh (dk x 33), M, T (C x (C+1) each), K, Q (C x (dk+1) each),
+// dO, X (C x 33 each), g, beta, e^g (C each).
+__host__ __device__ inline size_t state_rev_smem_floats(int C, int dk) {
+    return (size_t)dk * 33 + 2 * (size_t)C * (C + 1) + 2 * (size_t)C * (dk + 1) + 2 * (size_t)C * 33 +
+           3 * (size_t)C;
+}
+
+__global__ void __launch_bounds__(kThreads) bwd_state_rev_kernel(const BwdParams p) {
+    float *sm = reinterpret_cast<float *>(bwd_smem);
+    const int C = p.C, dk = p.dk, dv = p.dv;
+    const int j0 = blockIdx.x * kCols, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+    const int jj = tid & 31, rr = tid >> 5;
+    const int dkp = dk + 1, Cp = C + 1;
+    float *dhs = sm;
+    float *Ms = dhs + dk * 33;
+    float *Ts = Ms + C * Cp;
+    float *Ks = Ts + C * Cp;
+    float *Qs = Ks + C * dkp;
+    float *dOs = Qs + C * dkp;
+    float *Xs = dOs + C * 33;
+    float *gs = Xs + C * 33;
+    float *bs = gs + C;
+    float *egs = bs + C;
+    const size_t bh = (size_t)b * p.H + h;
+
+    for (int c = rr; c < dk; c += 8)
+        dhs[c * 33 + jj] = p.grad_S_T ? p.grad_S_T[(bh * dk + c) * dv + j0 + jj] : 0.f;
+    for (int n = p.NC - 1; n >= 0; --n) {
+        const int t0 = n * C, Cn = min(C, p.T - t0);
+        const size_t ch = bh * p.NC + n;
+        __syncthreads();   // dh complete; the previous chunk's reads done
+        for (int c = rr; c < dk; c += 8) p.ws_dh[(ch * dk + c) * dv + j0 + jj] = dhs[c * 33 + jj];
+        for (int x = tid; x < C * C; x += kThreads) {
+            const int r = x / C, i = x % C;
+            Ms[r * Cp + i] = p.ws_M[ch * C * C + x];
+            Ts[r * Cp + i] = p.ws_T[ch * C * C + x];
+        }
+        for (int x = tid; x < C * dk; x += kThreads) {
+            const int r = x / dk, c = x % dk;
+            float kv = 0.f, qv = 0.f;
+            if (r < Cn) {
+                const size_t ti = tok_index(p, b, t0 + r, h) * dk + c;
+                kv = ld_in(p.k, ti, p.io_bf16);
+                qv = ld_in(p.q, ti, p.io_bf16);
+            }
+            Ks[r * dkp + c] = kv;
+            Qs[r * dkp + c] = qv;
+        }
+        for (int r = rr; r < C; r += 8)
+            dOs[r * 33 + jj] = r < Cn ? ld_in(p.grad_o, tok_index(p, b, t0 + r, h) * dv + j0 + jj, p.do_bf16) : 0.f;
+        if (tid < C) {
+            const float gv = p.ws_g[ch * C + tid];
+            gs[tid] = gv;
+            bs[tid] = tid < Cn ? (p.beta ? p.beta[tok_index(p, b, t0 + tid, h)] : 1.f) : 0.f;
+            egs[tid] = expf(gv);
+        }
+        __syncthreads();
+        const float glast = gs[Cn - 1];
+        // dDelta = M^T dO + diag(e^{g_C - g}) K dh'
+        for (int r = rr; r < Cn; r += 8) {
+            float s = 0.f;
+            for (int r2 = r; r2 < Cn; ++r2) s += Ms[r2 * Cp + r] * dOs[r2 * 33 + jj];
+            float u = 0.f;
+            for (int c = 0; c < dk; ++c) u += Ks[r * dkp + c] * dhs[c * 33 + jj];
+            Xs[r * 33 + jj] = s + expf(glast - gs[r]) * u;
+        }
+        __syncthreads();
+        // Y = T^T dDelta (T is lower triangular)
+        float y[kMaxC / 8];
+#pragma unroll
+        for (int m = 0; m < kMaxC / 8; ++m) {
+            const int r = rr + 8 * m;
+            float s = 0.f;
+            if (r < Cn)
+                for (int r2 = r; r2 < Cn; ++r2) s += Ts[r2 * Cp + r] * Xs[r2 * 33 + jj];
+            y[m] = s;
+        }
+        __syncthreads();   // every read of dDelta done
+#pragma unroll
+        for (int m = 0; m < kMaxC / 8; ++m) {
+            const int r = rr + 8 * m;
+            if (r < C) Xs[r * 33 + jj] = y[m];
+            if (r < Cn) {
+                p.ws_Y[(ch * C + r) * dv + j0 + jj] = y[m];
+                p.grad_v[tok_index(p, b, t0 + r, h) * dv + j0 + jj] = bs[r] * y[m];
+            }
+        }
+        __syncthreads();
+        // dh <- e^{g_C} dh' + (diag(e^g) Q)^T dO - (diag(beta e^g) K)^T Y
+        const float eglast = expf(glast);
+        for (int c = rr; c < dk; c += 8) {
+            float s = eglast * dhs[c * 33 + jj];
+            for (int r = 0; r < Cn; ++r)
+                s += egs[r] * (Qs[r * dkp + c] * dOs[r * 33 + jj] - bs[r] * Ks[r * dkp + c] * Xs[r * 33 + jj]);
+            dhs[c * 33 + jj] = s;
+        }
+    }
+    __syncthreads();
+    if (p.grad_S0)
+        for (int c = rr; c < dk; c += 8) p.grad_S0[(bh * dk + c) * dv + j0 + jj] = dhs[c * 33 + jj];
+}
+
+// ------------------------------------------------------ key-side gradients
+// One block per chunk-head.  Thread (r, cq) = (tid / 4, tid % 4) owns row r
+// and key columns cq + 4m of the three C x dk products over the value axis
+// (dO h^T, Y h^T, Delta dh'^T), accumulated in registers over 32-column
+// value tiles, and entries (r, cq + 4m) of dO Delta^T and Y Delta^T in
+// shared memory.
+// Shared memory: K, Q (C x (DK+1)), two C x (C+1) score buffers, the value
+// tiles (h, dh': DK x 33; dO, Y, Delta, V: C x 33; reused afterwards for two
+// C x (C+1) buffers), g, beta, e^g (C), kThreads partials, 4 x 4 x kMaxC row
+// partials and 10 x kMaxC row values.
+__host__ __device__ inline size_t grad_smem_floats(int C, int DK) {
+    return 2 * (size_t)C * (DK + 1) + 2 * (size_t)C * (C + 1) + 2 * (size_t)DK * 33 + 4 * (size_t)C * 33 +
+           3 * (size_t)C + kThreads + 16 * kMaxC + 10 * kMaxC;
+}
+
+enum { RV_A2K = 0, RV_QA1, RV_K3, RV_YV, RV_KAP, RV_DB, RV_DG, RV_HDH };
+
+template <int DK>
+__global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
+    constexpr int MK = DK / 4;
+    constexpr int MC = kMaxC / 4;
+    constexpr int dkp = DK + 1;
+    float *sm = reinterpret_cast<float *>(bwd_smem);
+    const int C = p.C, dv = p.dv;
+    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+    const int r = tid >> 2, cq = tid & 3;
+    const int t0 = n * C, Cn = min(C, p.T - t0);
+    const int Cp = C + 1;
+    float *Ks = sm;
+    float *Qs = Ks + C * dkp;
+    float *dMs = Qs + C * dkp;
+    float *dLs = dMs + C * Cp;
+    float *tile = dLs + C * Cp;
+    float *ht = tile;
+    float *dht = ht + DK * 33;
+    float *dOt = dht + DK * 33;
+    float *Yt = dOt + C * 33;
+    float *Dt = Yt + C * 33;
+    float *Vt = Dt + C * 33;
+    float *gs = Vt + C * 33;
+    float *bs = gs + C;
+    float *egs = bs + C;
+    float *red = egs + C;
+    float *part = red + kThreads;        // [4 quantities][4 cq][kMaxC]
+    float *rowv = part + 16 * kMaxC;     // [10][kMaxC]
+    const size_t ch = ((size_t)b * p.H + h) * p.NC + n;
+
+    for (int x = tid; x < C * DK; x += kThreads) {
+        const int r2 = x / DK, c = x % DK;
+        float kv = 0.f, qv = 0.f;
+        if (r2 < Cn) {
+            const size_t ti = tok_index(p, b, t0 + r2, h) * DK + c;
+            kv = ld_in(p.k, ti, p.io_bf16);
+            qv = ld_in(p.q, ti, p.io_bf16);
+        }
+        Ks[r2 * dkp + c] = kv;
+        Qs[r2 * dkp + c] = qv;
+    }
+    for (int x = tid; x < C * Cp; x += kThreads) {
+        dMs[x] = 0.f;
+        dLs[x] = 0.f;
+    }
+    if (tid < C) {
+        const float gv = p.ws_g[ch * C + tid];
+        gs[tid] = gv;
+        bs[tid] = tid < Cn ? (p.beta ? p.beta[tok_index(p, b, t0 + tid, h)] : 1.f) : 0.f;
+        egs[tid] = expf(gv);
+    }
+
+    float A1[MK], A2[MK], A3[MK];
+#pragma unroll
+    for (int m = 0; m < MK; ++m) A1[m] = A2[m] = A3[m] = 0.f;
+    float yv = 0.f, hdh = 0.f;
+
+    for (int j0 = 0; j0 < dv; j0 += kCols) {
+        __syncthreads();   // previous tile consumed (and, first time, the set-up above)
+        for (int x = tid; x < DK * kCols; x += kThreads) {
+            const int c = x / kCols, jj = x % kCols;
+            ht[c * 33 + jj] = p.ws_h[(ch * DK + c) * dv + j0 + jj];
+            dht[c * 33 + jj] = p.ws_dh[(ch * DK + c) * dv + j0 + jj];
+        }
+        for (int x = tid; x < C * kCols; x += kThreads) {
+            const int r2 = x / kCols, jj = x % kCols;
+            float a = 0.f, y = 0.f, d = 0.f, v = 0.f;
+            if (r2 < Cn) {
+                const size_t ti = tok_index(p, b, t0 + r2, h) * dv + j0 + jj;
+                a = ld_in(p.grad_o, ti, p.do_bf16);
+                v = ld_in(p.v, ti, p.io_bf16);
+                y = p.ws_Y[(ch * C + r2) * dv + j0 + jj];
+                d = p.ws_D[(ch * C + r2) * dv + j0 + jj];
+            }
+            dOt[r2 * 33 + jj] = a;
+            Yt[r2 * 33 + jj] = y;
+            Dt[r2 * 33 + jj] = d;
+            Vt[r2 * 33 + jj] = v;
+        }
+        __syncthreads();
+        if (r < Cn) {
+            for (int jj = 0; jj < kCols; ++jj) {
+                const float a = dOt[r * 33 + jj], y = Yt[r * 33 + jj], d = Dt[r * 33 + jj];
+#pragma unroll
+                for (int m = 0; m < MK; ++m) {
+                    const int c = cq + 4 * m;
+                    const float hv = ht[c * 33 + jj];
+                    A1[m] += a * hv;
+                    A2[m] += y * hv;
+                    A3[m] += d * dht[c * 33 + jj];
+                }
+            }
+            for (int jj = cq; jj < kCols; jj += 4) yv += Yt[r * 33 + jj] * Vt[r * 33 + jj];
+            for (int m = 0; m < MC; ++m) {
+                const int i = cq + 4 * m;
+                if (i < Cn) {
+                    float s1 = 0.f, s2 = 0.f;
+                    for (int jj = 0; jj < kCols; ++jj) {
+                        const float d = Dt[i * 33 + jj];
+                        s1 += dOt[r * 33 + jj] * d;
+                        s2 += Yt[r * 33 + jj] * d;
+                    }
+                    dMs[r * Cp + i] += s1;
+                    dLs[r * Cp + i] += s2;
+                }
+            }
+        }
+        for (int x = tid; x < DK * kCols; x += kThreads) {
+            const int c = x / kCols, jj = x % kCols;
+            hdh += ht[c * 33 + jj] * dht[c * 33 + jj];
+        }
+    }
+
+    // row dot products k_r.(Y h^T)_r, q_r.(dO h^T)_r, k_r.(Delta dh'^T)_r
+    {
+        float a2k = 0.f, qa1 = 0.f, k3 = 0.f;
+        if (r < Cn) {
+#pragma unroll
+            for (int m = 0; m < MK; ++m) {
+                const int c = cq + 4 * m;
+                a2k += A2[m] * Ks[r * dkp + c];
+                qa1 += A1[m] * Qs[r * dkp + c];
+                k3 += A3[m] * Ks[r * dkp + c];
+            }
+        }
+        part[(0 * 4 + cq) * kMaxC + r] = a2k;
+        part[(1 * 4 + cq) * kMaxC + r] = qa1;
+        part[(2 * 4 + cq) * kMaxC + r] = k3;
+        part[(3 * 4 + cq) * kMaxC + r] = yv;
+        red[tid] = hdh;
+    }
+    __syncthreads();
+    if (tid < kMaxC) {
+        for (int qn = 0; qn < 4; ++qn) {
+            float s = 0.f;
+            for (int c4 = 0; c4 < 4; ++c4) s += part[(qn * 4 + c4) * kMaxC + tid];
+            rowv[qn * kMaxC + tid] = s;   // RV_A2K, RV_QA1, RV_K3, RV_YV
+        }
+    }
+    if (tid == 0) {
+        float s = 0.f;
+        for (int x = 0; x < kThreads; ++x) s += red[x];
+        rowv[RV_HDH * kMaxC] = s;
+    }
+
+    // per score entry: recompute k_r.k_i and q_r.k_i; fold in the decay
+    float *Fs = tile;             // dL (.) L + dM (.) M, the g-derivative terms of L and M
+    float *Es = tile + C * Cp;    // dL (.) Gamma (.) k_r.k_i, the beta-derivative of L
+    for (int x = tid; x < C * C; x += kThreads) {
+        const int r2 = x / C, i = x % C;
+        float F = 0.f, E = 0.f, dmg = 0.f, dgv = 0.f;
+        if (r2 < Cn && i <= r2) {
+            float gk = 0.f, qk = 0.f;
+            for (int c = 0; c < DK; ++c) {
+                const float ki = Ks[i * dkp + c];
+                gk += Ks[r2 * dkp + c] * ki;
+                qk += Qs[r2 * dkp + c] * ki;
+            }
+            const float gam = expf(gs[r2] - gs[i]);
+            const float dm = dMs[r2 * Cp + i];
+            F = dm * gam * qk;
+            dmg = dm * gam;
+            if (i < r2) {
+                const float dl = -dLs[r2 * Cp + i];
+                F += dl * bs[r2] * gam * gk;
+                E = dl * gam * gk;
+                dgv = bs[r2] * dl * gam;
+            }
+        }
+        Fs[(x / C) * Cp + x % C] = F;
+        Es[(x / C) * Cp + x % C] = E;
+        dMs[r2 * Cp + i] = dmg;   // dM (.) Gamma
+        dLs[r2 * Cp + i] = dgv;   // dG
+    }
+    __syncthreads();
+
+    if (tid < Cn) {
+        const int rr = tid;
+        float fr = 0.f, fc = 0.f, er = 0.f;
+        for (int i = 0; i < Cn; ++i) {
+            fr += Fs[rr * Cp + i];
+            fc += Fs[i * Cp + rr];
+            er += Es[rr * Cp + i];
+        }
+        const float kap = expf(gs[Cn - 1] - gs[rr]) * rowv[RV_K3 * kMaxC + rr];
+        const float a2k = rowv[RV_A2K * kMaxC + rr];
+        rowv[RV_KAP * kMaxC + rr] = kap;
+        rowv[RV_DB * kMaxC + rr] = rowv[RV_YV * kMaxC + rr] - egs[rr] * a2k + er;
+        rowv[RV_DG * kMaxC + rr] = -bs[rr] * egs[rr] * a2k + fr - fc + egs[rr] * rowv[RV_QA1 * kMaxC + rr] - kap;
+    }
+    __syncthreads();
+    if (tid < Cn) {
+        const int rr = tid;
+        // the chunk-end terms belong to g_{Cn-1}, which every suffix sum contains
+        float s = expf(gs[Cn - 1]) * rowv[RV_HDH * kMaxC];
+        for (int i = 0; i < Cn; ++i) s += rowv[RV_KAP * kMaxC + i];
+        for (int r2 = rr; r2 < Cn; ++r2) s += rowv[RV_DG * kMaxC + r2];
+        const size_t ti = tok_index(p, b, t0 + rr, h);
+        if (p.grad_alpha) p.grad_alpha[ti] = s / p.alpha[ti];
+        if (p.grad_beta) p.grad_beta[ti] = rowv[RV_DB * kMaxC + rr];
+    }
+
+    if (r < Cn) {
+        const float eg = egs[r], ebr = bs[r] * egs[r], edec = expf(gs[Cn - 1] - gs[r]);
+        const size_t out = tok_index(p, b, t0 + r, h) * DK;
+#pragma unroll
+        for (int m = 0; m < MK; ++m) {
+            const int c = cq + 4 * m;
+            float dq = eg * A1[m];
+            float dkv = edec * A3[m] - ebr * A2[m];
+            for (int i = 0; i <= r; ++i) dq += dMs[r * Cp + i] * Ks[i * dkp + c];
+            for (int r2 = r; r2 < Cn; ++r2) dkv += dMs[r2 * Cp + r] * Qs[r2 * dkp + c];
+            for (int i = 0; i < Cn; ++i) dkv += (dLs[r * Cp + i] + dLs[i * Cp + r]) * Ks[i * dkp + c];
+            p.grad_q[out + c] = dq;
+            p.grad_k[out + c] = dkv;
+        }
+    }
+}
+
+}  // namespace bwd
+}  // namespace gdn

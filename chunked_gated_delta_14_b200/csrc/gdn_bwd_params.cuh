@@ -1,0 +1,37 @@
+// Resolved arguments of the backward kernels (gradient of the gated delta
+// rule), filled by the host layer from gdn_bwd_args.  Plain data only.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gdn {
+
+struct BwdParams {
+    int B, T, H, dk, dv, C;
+    int NC;                       // chunks per sequence, ceil(T / C)
+    int io_bf16, do_bf16;         // q/k/v and grad_o element types (1 = bf16, 0 = fp32)
+    const void *q, *k, *v;        // [B, T, H, dk|dv]
+    const float *alpha, *beta;    // [B, T, H] or null (=> 1)
+    const float *S0;              // [B, H, dk, dv] or null (=> 0)
+    const void *grad_o;           // [B, T, H, dv]
+    const float *grad_S_T;        // [B, H, dk, dv] or null (=> 0)
+    float *grad_q, *grad_k, *grad_v;
+    float *grad_alpha, *grad_beta, *grad_S0;   // each may be null
+    // Workspace regions, fp32, each indexed by chunk-head (b*H + h)*NC + n:
+    float *ws_g;    // C        in-chunk cumulative log decay g
+    float *ws_T;    // C x C    T = (I + L)^-1
+    float *ws_M;    // C x C    causal decayed scores M = (Q K^T) (.) Gamma, i <= r
+    float *ws_W;    // C x dk   W = T diag(beta e^g) K
+    float *ws_D;    // C x dv   U = T diag(beta) V, overwritten with Delta = U - W h
+    float *ws_h;    // dk x dv  state h = S^T at the chunk's start
+    float *ws_dh;   // dk x dv  dL/dh at the chunk's end
+    float *ws_Y;    // C x dv   Y = T^T dDelta
+};
+
+// fp32 words of workspace per chunk-head.
+inline size_t bwd_ws_floats_per_chunk(int C, int dk, int dv) {
+    return (size_t)C + 2 * (size_t)C * C + (size_t)C * dk + 2 * (size_t)C * dv + 2 * (size_t)dk * dv;
+}
+
+}  // namespace gdn

@@ -1,7 +1,7 @@
 """Thin ctypes binding of libgdn.so (the C ABI declared in include/gdn.h).
 
-Argument marshalling only: every step of the forward pass runs in the CUDA
-kernels of libgdn.so.  PyTorch provides device memory and the current stream.
+Argument marshalling only: every step of the forward and backward passes runs
+in the CUDA kernels of libgdn.so.  PyTorch provides device memory and the current stream.
 There is no fallback: if the library is missing or the device is not a CUDA
 device, the call raises.
 """
@@ -32,7 +32,8 @@ KERNEL_NAMES = {v: k for k, v in KERNELS.items()}
 MODES = {"exact": GDN_INV_EXACT, "neumann": GDN_INV_NEUMANN, "residual": GDN_INV_NEUMANN_RESIDUAL}
 
 EXPORTS = ("gdn_chunk_fwd", "gdn_select_kernel", "gdn_workspace_bytes", "gdn_device_check",
-           "gdn_status_string", "gdn_last_error", "gdn_abi_version", "gdn_chunk_fwd_static_scratch")
+           "gdn_status_string", "gdn_last_error", "gdn_abi_version", "gdn_chunk_fwd_static_scratch",
+           "gdn_chunk_bwd", "gdn_bwd_workspace_bytes")
 STATIC_SCRATCH_BYTES = 24 << 20   # GDN_STATIC_SCRATCH_BYTES
 
 
@@ -59,6 +60,22 @@ class FwdArgs(ctypes.Structure):
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_uint64),
         ("residual_S", ctypes.c_int32),
         ("precond_x", ctypes.c_float), ("precond_query", ctypes.c_int32),
+    ]
+
+
+class BwdArgs(ctypes.Structure):
+    """Mirror of ``gdn_bwd_args``."""
+    _fields_ = [
+        ("B", ctypes.c_int32), ("T", ctypes.c_int32), ("H", ctypes.c_int32),
+        ("dk", ctypes.c_int32), ("dv", ctypes.c_int32), ("chunk", ctypes.c_int32),
+        ("io_dtype", ctypes.c_int32), ("do_dtype", ctypes.c_int32),
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("alpha", ctypes.c_void_p), ("beta", ctypes.c_void_p), ("S0", ctypes.c_void_p),
+        ("grad_o", ctypes.c_void_p), ("grad_S_T", ctypes.c_void_p),
+        ("grad_q", ctypes.c_void_p), ("grad_k", ctypes.c_void_p), ("grad_v", ctypes.c_void_p),
+        ("grad_alpha", ctypes.c_void_p), ("grad_beta", ctypes.c_void_p),
+        ("grad_S0", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_uint64),
     ]
 
 
@@ -91,6 +108,10 @@ def lib() -> ctypes.CDLL:
             L.gdn_abi_version.restype = ctypes.c_int32
             L.gdn_chunk_fwd_static_scratch.argtypes = [ctypes.POINTER(FwdArgs), ctypes.c_void_p]
             L.gdn_chunk_fwd_static_scratch.restype = ctypes.c_int
+            L.gdn_chunk_bwd.argtypes = [ctypes.POINTER(BwdArgs), ctypes.c_void_p]
+            L.gdn_chunk_bwd.restype = ctypes.c_int
+            L.gdn_bwd_workspace_bytes.argtypes = [ctypes.POINTER(BwdArgs)]
+            L.gdn_bwd_workspace_bytes.restype = ctypes.c_uint64
             _lib = L
     return _lib
 
@@ -159,12 +180,15 @@ def workspace_bytes(args: FwdArgs) -> int:
 _ws_cache = {}
 
 
-def workspace_for(args: FwdArgs, device: torch.device) -> Optional[torch.Tensor]:
-    """A cached device buffer of at least workspace_bytes(args) bytes, or None."""
-    need = workspace_bytes(args)
+def workspace_for(args, device: torch.device) -> Optional[torch.Tensor]:
+    """A cached device buffer of at least the workspace ``args`` needs, or None.
+
+    Forward (FwdArgs) and backward (BwdArgs) calls keep separate buffers."""
+    bwd = isinstance(args, BwdArgs)
+    need = bwd_workspace_bytes(args) if bwd else workspace_bytes(args)
     if need == 0:
         return None
-    key = (device.type, device.index)
+    key = (device.type, device.index, bwd)
     buf = _ws_cache.get(key)
     if buf is None or buf.numel() < need:
         buf = torch.empty(need, dtype=torch.uint8, device=device)
@@ -257,3 +281,101 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     with torch.cuda.device(q.device):
         call(args, stream.cuda_stream)
     return out, S_T
+
+
+# ------------------------------------------------------------------ backward
+
+def make_bwd_args(**kw) -> BwdArgs:
+    a = BwdArgs()
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def bwd_workspace_bytes(args: BwdArgs) -> int:
+    """Device workspace gdn_chunk_bwd needs for ``args`` (0 if invalid; host only)."""
+    return int(lib().gdn_bwd_workspace_bytes(ctypes.byref(args)))
+
+
+def call_bwd(args: BwdArgs, stream: Optional[int] = None) -> None:
+    """Raw gdn_chunk_bwd call; raises GDNError on a non-OK status."""
+    s = lib().gdn_chunk_bwd(ctypes.byref(args), ctypes.c_void_p(stream or 0))
+    if s != GDN_OK:
+        raise GDNError(s, last_error())
+
+
+def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+              alpha: Optional[torch.Tensor], beta: Optional[torch.Tensor],
+              grad_o: torch.Tensor, *, S0: Optional[torch.Tensor] = None,
+              grad_S_T: Optional[torch.Tensor] = None, chunk: int = 64,
+              want_S0: bool = True, stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """Gradients of the gated delta rule (scalar alpha and beta, exact inverse).
+
+    Inputs as ``chunk_fwd``; ``grad_o`` [B, T, H, dv] (bf16 or fp32) is dL/do
+    and ``grad_S_T`` [B, H, dk, dv] fp32 (or None) dL/dS_T.  Returns a dict of
+    fp32 tensors ``dq``, ``dk``, ``dv``, ``dalpha`` / ``dbeta`` (None when the
+    gate is None) and ``dS0`` (None unless ``want_S0``).
+    """
+    if q.dim() != 4:
+        raise ValueError("q must be [B, T, H, dk]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    io = q.dtype
+    _check(q, "q", (B, T, H, dk), io)
+    _check(k, "k", (B, T, H, dk), io)
+    _check(v, "v", (B, T, H, dv), io)
+    _check(alpha, "alpha", (B, T, H), torch.float32)
+    _check(beta, "beta", (B, T, H), torch.float32)
+    _check(S0, "S0", (B, H, dk, dv), torch.float32)
+    _check(grad_o, "grad_o", (B, T, H, dv))
+    _check(grad_S_T, "grad_S_T", (B, H, dk, dv), torch.float32)
+    f32 = dict(device=q.device, dtype=torch.float32)
+    g = dict(dq=torch.empty((B, T, H, dk), **f32), dk=torch.empty((B, T, H, dk), **f32),
+             dv=torch.empty((B, T, H, dv), **f32),
+             dalpha=None if alpha is None else torch.empty((B, T, H), **f32),
+             dbeta=None if beta is None else torch.empty((B, T, H), **f32),
+             dS0=torch.empty((B, H, dk, dv), **f32) if want_S0 else None)
+    args = make_bwd_args(
+        B=B, T=T, H=H, dk=dk, dv=dv, chunk=int(chunk), io_dtype=_dtype_code(io),
+        do_dtype=_dtype_code(grad_o.dtype), q=_ptr(q), k=_ptr(k), v=_ptr(v), alpha=_ptr(alpha),
+        beta=_ptr(beta), S0=_ptr(S0), grad_o=_ptr(grad_o), grad_S_T=_ptr(grad_S_T),
+        grad_q=_ptr(g["dq"]), grad_k=_ptr(g["dk"]), grad_v=_ptr(g["dv"]),
+        grad_alpha=_ptr(g["dalpha"]), grad_beta=_ptr(g["dbeta"]), grad_S0=_ptr(g["dS0"]))
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    ws = workspace_for(args, q.device)
+    if ws is not None:
+        args.workspace = ws.data_ptr()
+        args.workspace_bytes = ws.numel()
+    with torch.cuda.device(q.device):
+        call_bwd(args, stream.cuda_stream)
+    return g
+
+
+class GatedDeltaRule(torch.autograd.Function):
+    """Differentiable gated delta rule: forward by ``chunk_fwd`` (exact
+    inverse), backward by ``chunk_bwd``; both run in libgdn.so."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, alpha, beta, S0, chunk):
+        o, S_T = chunk_fwd(q, k, v, alpha, beta, S0=S0, chunk=chunk)
+        ctx.save_for_backward(q, k, v, alpha, beta, S0)
+        ctx.chunk = chunk
+        return o, S_T
+
+    @staticmethod
+    def backward(ctx, grad_o, grad_S_T):
+        q, k, v, alpha, beta, S0 = ctx.saved_tensors
+        if grad_o is None:
+            grad_o = torch.zeros(v.shape, device=v.device, dtype=torch.float32)
+        g = chunk_bwd(q, k, v, alpha, beta, grad_o.contiguous(), S0=S0,
+                      grad_S_T=None if grad_S_T is None else grad_S_T.float().contiguous(),
+                      chunk=ctx.chunk, want_S0=S0 is not None and ctx.needs_input_grad[5])
+        cast = lambda t, like: None if t is None else t.to(like.dtype)
+        return (cast(g["dq"], q), cast(g["dk"], k), cast(g["dv"], v), g["dalpha"], g["dbeta"],
+                g["dS0"], None)
+
+
+def gated_delta_rule(q, k, v, alpha=None, beta=None, S0=None, chunk: int = 64):
+    """``(o, S_T)`` of the gated delta rule with autograd support (see GatedDeltaRule)."""
+    return GatedDeltaRule.apply(q, k, v, alpha, beta, S0, chunk)

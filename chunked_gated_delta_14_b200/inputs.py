@@ -19,6 +19,11 @@ skipping the ones a workload does not use):
 * erase gate b and write gate w = sigmoid(N(0, 1)) in the io dtype,
   shapes [B, T, H, d_k] and [B, T, H, d_v].
 
+Cotangents for the backward pass (``make_cotangents``) come from a second
+generator, ``PCG64([seed, 1])``, so drawing them never shifts the forward
+inputs: grad_o ~ N(0, 1) rounded to the io dtype, [B, T, H, d_v]; grad_S_T ~
+N(0, 0.02^2), fp32 [B, H, d_k, d_v] (the scale of S0).
+
 The workloads are the Gated DeltaNet layer shapes the pages discuss
 (1.3B-class head geometry: H=16, d_k=d_v=128); no dataset is involved.
 """
@@ -30,7 +35,7 @@ from typing import Optional
 import numpy as np
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "workload"]
+__all__ = ["Workload", "WORKLOADS", "make_cotangents", "make_inputs", "workload"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -145,3 +150,13 @@ def make_inputs(w: Workload, seed: int = 0) -> dict:
         erase = _round_io(_sigmoid(normal((B, T, H, dk))), w.io)
         write = _round_io(_sigmoid(normal((B, T, H, dv))), w.io)
     return dict(q=q, k=k, v=v, alpha=alpha, beta=beta, S0=S0, erase=erase, write=write)
+
+
+def make_cotangents(w: Workload, seed: int = 0, grad_state: bool = True) -> dict:
+    """Draw dL/do (io dtype) and dL/dS_T (fp32, or None) for workload ``w``."""
+    rng = np.random.Generator(np.random.PCG64([seed, 1]))
+    B, T, H, dk, dv = w.B, w.T, w.H, w.dk, w.dv
+    do = _round_io(rng.standard_normal(size=(B, T, H, dv), dtype=np.float32), w.io)
+    dS = (torch.from_numpy(rng.standard_normal(size=(B, H, dk, dv), dtype=np.float32)
+                           * np.float32(0.02)) if grad_state else None)
+    return dict(grad_o=do, grad_S_T=dS)

@@ -1,6 +1,6 @@
 /*
  * gdn.h -- C ABI of libgdn.so, the B200 (sm_100a) chunkwise gated delta-rule
- * forward pass.
+ * forward pass and the backward pass of the gated delta rule.
  *
  * What it computes.  For every (batch b, head h) sequence, with the state S_t
  * a d_v x d_k matrix (keys to values):
@@ -69,7 +69,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 4
+#define GDN_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define GDN_API __attribute__((visibility("default")))
@@ -177,6 +177,63 @@ GDN_API int32_t gdn_abi_version(void);
 /* Size of the fixed device scratch array of gdn_chunk_fwd_static_scratch:
  * 24 MiB = 1024 chunk-heads of three 64 x 64 fp16 matrices each. */
 #define GDN_STATIC_SCRATCH_BYTES (24ull << 20)
+
+/* ------------------------------------------------------------ backward pass
+ *
+ * Gradient of the gated delta rule (the default rule above: scalar decay
+ * alpha, scalar beta, exact inverse) with respect to q, k, v, alpha, beta and
+ * S0, given dL/do and dL/dS_T.  The pages use chunkwise forms to make
+ * training parallel ("Quando o 'Bom o Suficiente' e Otimo ...", sections
+ * "Resumo" and "Declaracao do Problema") but print no backward pass; this is
+ * the reverse-mode derivative of the chunked WY/UT form, fp32 on CUDA cores,
+ * in four launches:
+ *   1. per chunk-head: g, L, T = (I + L)^-1, the causal scores M, W, U;
+ *   2. per 32-column value slice, chunks in order: the state at every chunk
+ *      start and Delta = U - W h;
+ *   3. per slice, chunks in reverse: dL/dh at every chunk end, Y = T^T dDelta,
+ *      dv and dS0;
+ *   4. per chunk-head: dq, dk, dbeta, dalpha.
+ * The forward is recomputed inside the call (only S0 is taken from the
+ * caller), so the call needs no saved activations.
+ *
+ * Layouts as gdn_fwd_args; every gradient is fp32 in the layout of its input
+ * (grad_S0 and grad_S_T in the h = S^T layout [B, H, dk, dv]).
+ *
+ * Shapes: chunk 16, 32 or 64; dk 16, 32, 64 or 128; dv 32, 64 or 128;
+ * B, H <= 65535.  Other shapes return GDN_ERR_UNSUPPORTED.
+ *
+ * Ownership and errors as gdn_chunk_fwd: caller-allocated device buffers,
+ * host-side validation before any launch, asynchronous on `stream`.  The
+ * outputs must not alias the inputs or one another; every output pointer
+ * given is written in full.  alpha must be in (0, 1] (its logarithm is taken).
+ */
+typedef struct {
+    int32_t B, T, H, dk, dv, chunk;
+    int32_t io_dtype;           /* gdn_dtype of q, k, v */
+    int32_t do_dtype;           /* gdn_dtype of grad_o */
+    const void *q, *k, *v;      /* [B,T,H,dk|dv] */
+    const float *alpha;         /* [B,T,H] in (0, 1], or NULL (=> 1) */
+    const float *beta;          /* [B,T,H], or NULL (=> 1) */
+    const float *S0;            /* [B,H,dk,dv] fp32, or NULL (=> 0) */
+    const void *grad_o;         /* [B,T,H,dv] dL/do, required */
+    const float *grad_S_T;      /* [B,H,dk,dv] fp32 dL/dS_T, or NULL (=> 0) */
+    float *grad_q, *grad_k;     /* [B,T,H,dk] fp32, required */
+    float *grad_v;              /* [B,T,H,dv] fp32, required */
+    float *grad_alpha;          /* [B,T,H] fp32 or NULL; NULL when alpha is NULL */
+    float *grad_beta;           /* [B,T,H] fp32 or NULL; NULL when beta is NULL */
+    float *grad_S0;             /* [B,H,dk,dv] fp32 or NULL */
+    void *workspace;            /* >= gdn_bwd_workspace_bytes(args) bytes, 16-byte aligned */
+    uint64_t workspace_bytes;
+} gdn_bwd_args;
+
+/* Backward pass (see above). */
+GDN_API gdn_status gdn_chunk_bwd(const gdn_bwd_args *args, void *stream);
+
+/* Workspace bytes gdn_chunk_bwd needs: per chunk-head, fp32 g (C), T and M
+ * (C x C), W (C x dk), U / Delta and Y (C x dv), the state and its gradient
+ * (dk x dv); 0 with gdn_last_error() set if the arguments are invalid.  Host
+ * only. */
+GDN_API uint64_t gdn_bwd_workspace_bytes(const gdn_bwd_args *args);
 
 /* gdn_chunk_fwd on the tensor-core kernel, with a fixed scratch array inside
  * the library in place of args->workspace.  The pages have no counterpart:

@@ -25,7 +25,7 @@ def declared_functions():
 
 def test_library_builds_and_loads():
     gbuild.build()
-    assert gdn.abi_version() == 4
+    assert gdn.abi_version() == 5
 
 
 def test_exports_every_declared_symbol():
@@ -127,3 +127,82 @@ def test_python_wrapper_rejects_cpu_tensors():
     q = torch.zeros(1, 4, 1, 16, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         gdn.chunk_fwd(q, q, q)
+
+
+# ------------------------------------------------------------------ backward
+
+def _bwd_args(**kw):
+    G = 1 << 32   # fake device addresses, far enough apart never to overlap
+    base = dict(B=2, T=100, H=3, dk=128, dv=128, chunk=64, io_dtype=1, do_dtype=1,
+                q=1 * G, k=2 * G, v=3 * G, alpha=4 * G, beta=5 * G, S0=6 * G, grad_o=7 * G,
+                grad_S_T=8 * G, grad_q=9 * G, grad_k=10 * G, grad_v=11 * G, grad_alpha=12 * G,
+                grad_beta=13 * G, grad_S0=14 * G)
+    base.update(kw)
+    return gdn.make_bwd_args(**base)
+
+
+def _bwd_ws_expected(B, T, H, dk, dv, C):
+    nch = B * H * -(-T // C)
+    region = lambda f: (f * nch * 4 + 255) // 256 * 256
+    return region(C) + 2 * region(C * C) + region(C * dk) + 2 * region(C * dv) + 2 * region(dk * dv)
+
+
+@pytest.mark.parametrize("shape", [(2, 100, 3, 128, 128, 64), (1, 1, 1, 16, 32, 16),
+                                   (4, 4096, 16, 128, 128, 64), (3, 77, 5, 32, 96, 32)])
+def test_bwd_workspace_size(shape):
+    B, T, H, dk, dv, C = shape
+    a = _bwd_args(B=B, T=T, H=H, dk=dk, dv=dv, chunk=C)
+    assert gdn.bwd_workspace_bytes(a) == _bwd_ws_expected(*shape), gdn.last_error()
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=0), GDN_ERR_INVALID_ARG),
+    (dict(H=70000), GDN_ERR_INVALID_ARG),
+    (dict(chunk=128), GDN_ERR_UNSUPPORTED),            # backward chunks: 16, 32, 64
+    (dict(chunk=8), GDN_ERR_UNSUPPORTED),
+    (dict(dk=48), GDN_ERR_UNSUPPORTED),
+    (dict(dv=16), GDN_ERR_UNSUPPORTED),                # value slices of 32 columns
+    (dict(io_dtype=3), GDN_ERR_INVALID_ARG),
+    (dict(do_dtype=3), GDN_ERR_INVALID_ARG),
+    (dict(grad_o=None), GDN_ERR_INVALID_ARG),
+    (dict(grad_k=None), GDN_ERR_INVALID_ARG),
+    (dict(alpha=None), GDN_ERR_INVALID_ARG),           # grad_alpha without alpha
+    (dict(beta=None), GDN_ERR_INVALID_ARG),            # grad_beta without beta
+    (dict(grad_q=(1 << 32) + 64), GDN_ERR_INVALID_ARG),  # grad_q overlaps q
+    (dict(grad_v=10 * (1 << 32) + 4096), GDN_ERR_INVALID_ARG),  # grad_v overlaps grad_k
+    (dict(grad_S0=6 * (1 << 32)), GDN_ERR_INVALID_ARG),  # grad_S0 aliases S0
+    (dict(grad_q=9 * (1 << 32) + 8), GDN_ERR_ALIGNMENT),
+])
+def test_bwd_invalid_arguments_rejected_on_host(kw, status):
+    a = _bwd_args(**kw)
+    assert gdn.bwd_workspace_bytes(a) == 0 and gdn.last_error()
+    with pytest.raises(gdn.GDNError) as ei:
+        gdn.call_bwd(a)   # returns before any CUDA call
+    assert ei.value.status == status
+
+
+def test_bwd_workspace_must_not_overlap_and_must_be_large_enough():
+    a = _bwd_args()
+    need = gdn.bwd_workspace_bytes(a)
+    a.workspace, a.workspace_bytes = 20 << 32, need - 256
+    with pytest.raises(gdn.GDNError) as ei:
+        gdn.call_bwd(a)
+    assert ei.value.status == GDN_ERR_INVALID_ARG and "workspace" in str(ei.value)
+    a.workspace, a.workspace_bytes = (11 << 32) - 4096, need   # runs into grad_v
+    with pytest.raises(gdn.GDNError) as ei:
+        gdn.call_bwd(a)
+    assert ei.value.status == GDN_ERR_INVALID_ARG
+
+
+def test_bwd_optional_gradients_may_be_null():
+    a = _bwd_args(alpha=None, beta=None, grad_alpha=None, grad_beta=None, grad_S0=None,
+                  S0=None, grad_S_T=None)
+    assert gdn.bwd_workspace_bytes(a) > 0, gdn.last_error()
+
+
+def test_python_backward_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 4, 1, 16, dtype=torch.bfloat16)
+    v = torch.zeros(1, 4, 1, 32, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        gdn.chunk_bwd(q, q, v, None, None, v)

@@ -1,0 +1,146 @@
+"""GPU parity of the backward pass: gdn_chunk_bwd, through the C ABI, against
+the fp64 adjoint oracle on the same seeded inputs and cotangents.
+
+Tolerance.  The kernels compute in fp32 from inputs the oracle sees bit for
+bit, so the gap is fp32 rounding only: each product sums at most
+d_k, d_v or C <= 128 terms per step and the state gradient is carried over
+the chunks with decays <= 1.  Unit roundoff 6e-8 times a few hundred terms
+of growth stays below 1e-4 of a gradient's RMS; the bar, max |err| <= 1e-3
+of the oracle's RMS for every gradient, leaves a tenfold margin.
+"""
+import numpy as np
+import pytest
+import torch
+
+import chunked_gated_delta_14_b200 as gdn
+import oracle
+from chunked_gated_delta_14_b200.inputs import make_cotangents, make_inputs, workload
+
+from gpu_util import bf16_allowance_ok, report, stats, to_dev
+
+pytestmark = pytest.mark.gpu
+
+needs_cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+
+TOL_BWD_REL_RMS = 1e-3
+GRADS = dict(dq="dq", dk="dk", dv="dv", dalpha="dalpha", dbeta="dbeta", dS0="dh0")
+
+
+def _run_bwd(x, c, chunk, want_S0=True):
+    d = {k: to_dev(v) for k, v in x.items()}
+    g = gdn.chunk_bwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], to_dev(c["grad_o"]),
+                      S0=d["S0"], grad_S_T=to_dev(c["grad_S_T"]), chunk=chunk,
+                      want_S0=want_S0)
+    torch.cuda.synchronize()
+    return {k: None if v is None else v.double().cpu().numpy() for k, v in g.items()}
+
+
+def _oracle_bwd(x, c):
+    return oracle.gated_delta_bwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"],
+                                  c["grad_o"], c["grad_S_T"])
+
+
+def _compare(name, got, ref, tol=TOL_BWD_REL_RMS):
+    out = {}
+    for gk, rk in GRADS.items():
+        if ref[rk] is None or got[gk] is None:
+            assert got[gk] is None and (ref[rk] is None or gk == "dS0"), gk
+            continue
+        assert np.isfinite(got[gk]).all(), gk
+        out[gk] = stats(got[gk], ref[rk])
+    report(name, **out)
+    for gk, st in out.items():
+        assert st["max_rel_rms"] <= tol, (gk, st)
+
+
+CASES = [
+    # name, workload overrides, chunk, cotangent of S_T
+    ("gdn_ragged_s0", dict(B=2, H=3, T=1000, s0_std=0.02), 64, True),
+    ("plain_fp32", dict(B=1, H=2, T=256, dk=64, dv=64, io="f32", decay="none"), 64, False),
+    ("dk16_dv32_c16_f32", dict(B=1, H=2, T=77, dk=16, dv=32, io="f32"), 16, True),
+    ("dk32_dv96_c32", dict(B=2, H=2, T=200, dk=32, dv=96), 32, True),
+    ("single_token", dict(B=3, H=2, T=1, dk=128, dv=64, s0_std=0.02), 64, True),
+    ("dk64_dv128_c16_nobeta", dict(B=1, H=2, T=129, dk=64, dv=128, beta=False), 16, True),
+    ("one_chunk_tail", dict(B=1, H=1, T=65, dk=128, dv=128, s0_std=0.02), 64, True),
+]
+
+
+@needs_cuda
+@pytest.mark.parametrize("name,over,chunk,dS", CASES, ids=[c[0] for c in CASES])
+def test_backward_matches_adjoint_oracle(name, over, chunk, dS):
+    w = workload("gdn_bf16", **over)
+    x = make_inputs(w, seed=11)
+    c = make_cotangents(w, seed=11, grad_state=dS)
+    got = _run_bwd(x, c, chunk)
+    _compare(f"bwd_{name}", got, _oracle_bwd(x, c))
+
+
+@needs_cuda
+def test_backward_is_deterministic_and_chunk_independent():
+    w = workload("gdn_bf16", B=1, H=2, T=300, dk=64, dv=64, s0_std=0.02)
+    x = make_inputs(w, seed=12)
+    c = make_cotangents(w, seed=12)
+    a = _run_bwd(x, c, 32)
+    b = _run_bwd(x, c, 32)
+    for k in a:
+        assert np.array_equal(a[k], b[k]), k        # no atomics: bit-identical reruns
+    ref = _oracle_bwd(x, c)
+    for chunk in (16, 64):
+        _compare(f"bwd_chunk{chunk}", _run_bwd(x, c, chunk), ref)
+
+
+@needs_cuda
+def test_backward_full_size_sampled_heads():
+    """The benchmark's backward configuration (B=4, H=16, T=4096, d=128, C=64,
+    bf16): every gradient finite, and three whole (batch, head) sequences
+    against the oracle (sequences are independent, so a slice is exact)."""
+    w = workload("gdn_bf16")
+    x = make_inputs(w, seed=0)
+    c = make_cotangents(w, seed=0)
+    got = _run_bwd(x, c, 64)
+    for k, v in got.items():
+        if v is not None:
+            assert np.isfinite(v).all(), k
+    for b, h in [(0, 0), (3, 15), (1, 7)]:
+        xs = {k: None if v is None else
+              (v[b:b + 1, :, h:h + 1] if v.dim() in (3, 4) and k != "S0" else v[b:b + 1, h:h + 1])
+              .contiguous() for k, v in x.items()}
+        cs = dict(grad_o=c["grad_o"][b:b + 1, :, h:h + 1].contiguous(),
+                  grad_S_T=c["grad_S_T"][b:b + 1, h:h + 1].contiguous())
+        ref = _oracle_bwd(xs, cs)
+        sl = dict(dq=got["dq"][b:b + 1, :, h:h + 1], dk=got["dk"][b:b + 1, :, h:h + 1],
+                  dv=got["dv"][b:b + 1, :, h:h + 1], dalpha=got["dalpha"][b:b + 1, :, h:h + 1],
+                  dbeta=got["dbeta"][b:b + 1, :, h:h + 1], dS0=got["dS0"][b:b + 1, h:h + 1])
+        _compare(f"bwd_full_b{b}_h{h}", sl, ref)
+
+
+@needs_cuda
+def test_backward_long_sequence_with_initial_state():
+    w = workload("long_context", T=8192, H=2)
+    x = make_inputs(w, seed=13)
+    c = make_cotangents(w, seed=13)
+    _compare("bwd_long_8192", _run_bwd(x, c, 64), _oracle_bwd(x, c))
+
+
+@needs_cuda
+def test_autograd_function_matches_oracle():
+    """gated_delta_rule under torch.autograd: forward by gdn_chunk_fwd, backward
+    by gdn_chunk_bwd; bf16 input gradients are the fp32 ones rounded."""
+    w = workload("gdn_bf16", B=2, H=2, T=333, s0_std=0.02)
+    x = make_inputs(w, seed=14)
+    c = make_cotangents(w, seed=14)
+    d = {k: None if v is None else to_dev(v).requires_grad_(True) for k, v in x.items()
+         if k in ("q", "k", "v", "alpha", "beta", "S0")}
+    o, S_T = gdn.gated_delta_rule(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"])
+    loss = (o.float() * to_dev(c["grad_o"]).float()).sum() + (S_T * to_dev(c["grad_S_T"])).sum()
+    names = ["q", "k", "v", "alpha", "beta", "S0"]
+    grads = torch.autograd.grad(loss, [d[n] for n in names])
+    ref = _oracle_bwd(x, c)
+    for n, g in zip(names, grads):
+        r = ref[dict(q="dq", k="dk", v="dv", alpha="dalpha", beta="dbeta", S0="dh0")[n]]
+        got = g.double().cpu().numpy()
+        report(f"autograd_{n}", **stats(got, r))
+        if g.dtype == torch.bfloat16:
+            assert bf16_allowance_ok(got, r, rel_rms=TOL_BWD_REL_RMS), n
+        else:
+            assert stats(got, r)["max_rel_rms"] <= TOL_BWD_REL_RMS, n
