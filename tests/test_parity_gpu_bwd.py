@@ -2,11 +2,15 @@
 the fp64 adjoint oracle on the same seeded inputs and cotangents.
 
 Tolerance.  The kernels compute in fp32 from inputs the oracle sees bit for
-bit, so the gap is fp32 rounding only: each product sums at most
-d_k, d_v or C <= 128 terms per step and the state gradient is carried over
-the chunks with decays <= 1.  Unit roundoff 6e-8 times a few hundred terms
-of growth stays below 1e-4 of a gradient's RMS; the bar, max |err| <= 1e-3
-of the oracle's RMS for every gradient, leaves a tenfold margin.
+bit, so the gap is fp32 rounding only: each product sums at most d_k, d_v or
+C <= 128 terms per step and the state gradient is carried over the chunks
+with decays <= 1, so unit roundoff 6e-8 times a few hundred terms of growth
+gives about 1e-5 of a gradient's RMS.  dalpha is the exception: it is a
+suffix sum over the chunk of per-token terms that cancel to a small
+remainder, divided by alpha_t (down to 0.006 here), so its relative error is
+larger.  Measured on a B200 with these seeds: at most 3e-5 of the RMS for dq,
+dk, dv, dbeta and dS0, at most 6.4e-4 for dalpha.  The bar for every
+gradient is max |err| <= 1e-3 of the oracle's RMS.
 """
 import numpy as np
 import pytest
