@@ -26,7 +26,8 @@
 //             dbeta_r = Y_r.V_r - e^{g_r} k_r.(Y h^T)_r + sum_i dL_ri Gamma_ri k_r.k_i
 //             dg_r   = the partial derivatives of L, M, diag(e^g), W and h'
 //                      in g_r (see bwd_grad_kernel),
-//             dlog(alpha_t) = sum_{r >= t} dg_r,   dalpha_t = dlog(alpha_t) / alpha_t.
+//             dlog(alpha_t) = sum_{r >= t} dg_r (summed without the terms that
+//                      cancel), dalpha_t = dlog(alpha_t) / alpha_t.
 // (dT = dDelta (Vb - Kb h)^T and dL = -T^T dT T^T collapse to -Y Delta^T
 // because T (Vb - Kb h) = Delta.)
 //
@@ -484,7 +485,7 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
     }
 
     // per score entry: recompute k_r.k_i and q_r.k_i; fold in the decay
-    float *Fs = tile;             // dL (.) L + dM (.) M, the g-derivative terms of L and M
+    float *Fs = tile;             // dL (.) L + dM (.) M: F_ri enters dg_r with +, dg_i with -
     float *Es = tile + C * Cp;    // dL (.) Gamma (.) k_r.k_i, the beta-derivative of L
     for (int x = tid; x < C * C; x += kThreads) {
         const int r2 = x / C, i = x % C;
@@ -516,25 +517,28 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
 
     if (tid < Cn) {
         const int rr = tid;
-        float fr = 0.f, fc = 0.f, er = 0.f;
-        for (int i = 0; i < Cn; ++i) {
-            fr += Fs[rr * Cp + i];
-            fc += Fs[i * Cp + rr];
-            er += Es[rr * Cp + i];
-        }
+        float er = 0.f;
+        for (int i = 0; i < Cn; ++i) er += Es[rr * Cp + i];
         const float kap = expf(gs[Cn - 1] - gs[rr]) * rowv[RV_K3 * kMaxC + rr];
         const float a2k = rowv[RV_A2K * kMaxC + rr];
         rowv[RV_KAP * kMaxC + rr] = kap;
         rowv[RV_DB * kMaxC + rr] = rowv[RV_YV * kMaxC + rr] - egs[rr] * a2k + er;
-        rowv[RV_DG * kMaxC + rr] = -bs[rr] * egs[rr] * a2k + fr - fc + egs[rr] * rowv[RV_QA1 * kMaxC + rr] - kap;
+        // the derivative in g_r of diag(e^g) Q h and of W (F and kappa enter below)
+        rowv[RV_DG * kMaxC + rr] = -bs[rr] * egs[rr] * a2k + egs[rr] * rowv[RV_QA1 * kMaxC + rr];
     }
     __syncthreads();
     if (tid < Cn) {
         const int rr = tid;
-        // the chunk-end terms belong to g_{Cn-1}, which every suffix sum contains
+        // d log alpha_t = sum_{r >= t} dg_r, where dg_r collects the terms above,
+        // +F_ri for every i <= r, -F_ir for every i >= r, -kappa_r, and at the
+        // chunk end e^{g_C}<h, dh'> + sum_i kappa_i.  Summed over r >= t, the F terms
+        // with both indices >= t and the kappa terms with index >= t cancel exactly;
+        // only those crossing t are added, so no large terms cancel in fp32.
         float s = expf(gs[Cn - 1]) * rowv[RV_HDH * kMaxC];
-        for (int i = 0; i < Cn; ++i) s += rowv[RV_KAP * kMaxC + i];
+        for (int i = 0; i < rr; ++i) s += rowv[RV_KAP * kMaxC + i];
         for (int r2 = rr; r2 < Cn; ++r2) s += rowv[RV_DG * kMaxC + r2];
+        for (int r2 = rr; r2 < Cn; ++r2)
+            for (int i = 0; i < rr; ++i) s += Fs[r2 * Cp + i];
         const size_t ti = tok_index(p, b, t0 + rr, h);
         if (p.grad_alpha) p.grad_alpha[ti] = s / p.alpha[ti];
         if (p.grad_beta) p.grad_beta[ti] = rowv[RV_DB * kMaxC + rr];
