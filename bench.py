@@ -12,7 +12,9 @@ in HBM when the timed region starts.
 
 ``--batch B`` replaces the batch size (a smaller case for profiler captures).
 ``--decode`` times one-token decode steps; ``--bwd`` times the backward pass
-(gradients of q, k, v, alpha, beta) on the same workload.
+(gradients of q, k, v, alpha, beta) on the same workload.  The default line
+also carries a short backward timing in its ``backward`` object
+(``--bwd-steps``, 0 to skip).
 
 Under torchrun each rank runs its own independent batch (weak scaling, no
 collective on the data path); the time is the max over ranks.
@@ -316,6 +318,14 @@ def run_gpu(args, rank, world, local_rank):
                 roofline_ms=max(bytes_launch / (pk["hbm_gbs"] * 1e9),
                                 flops / (pk["bf16_tflops"] * 1e12)) * 1e3)
 
+    clk = clocks.summary() if rank == 0 else dict(sm_max_mhz=None)
+    backward = None
+    if args.bwd_steps > 0:
+        try:
+            backward = backward_side_measure(w, x, rank, world, dev, args.bwd_steps, 3, clk["sm_max_mhz"])
+        except Exception as e:   # the forward line is printed either way, with the reason
+            backward = dict(error=f"{type(e).__name__}: {e}")
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, x, budget_s=args.cpu_budget)
@@ -334,9 +344,9 @@ def run_gpu(args, rank, world, local_rank):
                                     if bytes_launch > 126e6 else
                                     f"no flush: {bytes_launch / 1e6:.0f} MB per step (fits L2; profiler case)"),
                                 kernel=kernel_name),
-                    clocks=clocks.summary() if rank == 0 else None,
+                    clocks=clk,
                     e2e=e2e, gpu_launches=args.steps * launches_per_call, roofline=roof,
-                    cpu_baseline=cpu)
+                    cpu_baseline=cpu, backward=backward)
         print(json.dumps(line), flush=True)
 
 
@@ -492,17 +502,13 @@ def bwd_bytes(w):
     return w.token_heads * per_th
 
 
-def run_bwd(args, rank, world, local_rank):
-    """One gdn_chunk_bwd call per step over the whole batch."""
+def bwd_setup(w, x, c, dev):
+    """Device copies of the inputs and dL/do, fp32 gradient buffers and the
+    gdn_bwd_args (with workspace) of one backward call over the whole batch.
+    The args hold raw pointers: the returned dict keeps every tensor they point
+    to alive."""
     import torch
     import chunked_gated_delta_14_b200 as gdn
-    from chunked_gated_delta_14_b200.inputs import make_cotangents, make_inputs, workload
-
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    w = workload(WORKLOAD, **({"B": args.batch} if args.batch else {}))
-    x = make_inputs(w, seed=rank)
-    c = make_cotangents(w, seed=rank, grad_state=False)
     d = {k: (None if v is None else v.to(dev)) for k, v in x.items()}
     grad_o = c["grad_o"].to(dev)
     f32 = dict(device=dev, dtype=torch.float32)
@@ -517,6 +523,70 @@ def run_bwd(args, rank, world, local_rank):
                           grad_alpha=ptr(g["da"]), grad_beta=ptr(g["db"]))
     ws = gdn.workspace_for(a, dev)
     a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    g["inputs"], g["grad_o"] = d, grad_o
+    return a, g, ws
+
+
+def bwd_roofline(w, ms_step, sm_max_mhz):
+    pk = peaks()
+    alu_peak = fp32_alu_peak_tflops(sm_max_mhz or 1965.0)
+    flops = algorithmic_flops_bwd(w)
+    achieved = flops / (ms_step / 1e3) / 1e12
+    nbytes = bwd_bytes(w)
+    return dict(bound="alu", achieved=achieved, peak=alu_peak, unit="TFLOP/s", frac=achieved / alu_peak,
+                traffic=profile_traffic("bwd_prep_kernel+bwd_state_fwd_kernel+bwd_state_rev_kernel+bwd_grad_kernel",
+                                        BWD_PROFILE, BWD_SOURCES),
+                peak_source="derived: 148 SMs x 128 fp32 lanes x 2 flops x max SM clock",
+                algorithmic_flops_per_launch=flops, algorithmic_bytes_per_launch=nbytes,
+                hbm_gbs=nbytes / (ms_step / 1e3) / 1e9, hbm_frac=nbytes / (ms_step / 1e3) / 1e9 / pk["hbm_gbs"],
+                roofline_ms=max(flops / (alu_peak * 1e12), nbytes / (pk["hbm_gbs"] * 1e9)) * 1e3)
+
+
+def backward_side_measure(w, x, rank, world, dev, steps, warmup, sm_max_mhz):
+    """The backward pass timed on the forward's workload (for the forward line's
+    ``backward`` object): one gdn_chunk_bwd call per step, CUDA events, max over
+    ranks."""
+    import torch
+    import chunked_gated_delta_14_b200 as gdn
+    from chunked_gated_delta_14_b200.inputs import make_cotangents
+    c = make_cotangents(w, seed=rank, grad_state=False)
+    a, g, ws = bwd_setup(w, x, c, dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warmup):
+        gdn.call_bwd(a, stream.cuda_stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        gdn.call_bwd(a, stream.cuda_stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    ms_step = ms / steps
+    out = dict(metric=BWD_METRIC, value=job_throughput(w.B * w.T, world, steps, ms), unit=UNIT,
+               steps=steps, warmup=warmup, ms_per_step=ms_step, dtype="f32",
+               gpu_launches=4 * steps, roofline=bwd_roofline(w, ms_step, sm_max_mhz),
+               note="gradients of q, k, v, alpha, beta on the same workload; full line: bench.py --bwd")
+    del a, g, ws
+    return out
+
+
+def run_bwd(args, rank, world, local_rank):
+    """One gdn_chunk_bwd call per step over the whole batch."""
+    import torch
+    import chunked_gated_delta_14_b200 as gdn
+    from chunked_gated_delta_14_b200.inputs import make_cotangents, make_inputs, workload
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workload(WORKLOAD, **({"B": args.batch} if args.batch else {}))
+    x = make_inputs(w, seed=rank)
+    c = make_cotangents(w, seed=rank, grad_state=False)
+    a, g, ws = bwd_setup(w, x, c, dev)
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
     for _ in range(args.warmup):
@@ -581,19 +651,9 @@ def run_bwd(args, rank, world, local_rank):
         e2e = dict(value=job_throughput(tokens_step, world, n_e2e, ems), unit=UNIT,
                    h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h), ms_per_step=ems / n_e2e)
 
-    pk = peaks()
     clk = clocks.summary()
-    alu_peak = fp32_alu_peak_tflops(clk["sm_max_mhz"] or 1965.0)
-    flops = algorithmic_flops_bwd(w)
-    achieved = flops / (ms_step / 1e3) / 1e12
     nbytes = bwd_bytes(w)
-    roof = dict(bound="alu", achieved=achieved, peak=alu_peak, unit="TFLOP/s", frac=achieved / alu_peak,
-                traffic=profile_traffic("bwd_prep_kernel+bwd_state_fwd_kernel+bwd_state_rev_kernel+bwd_grad_kernel",
-                                        BWD_PROFILE, BWD_SOURCES),
-                peak_source="derived: 148 SMs x 128 fp32 lanes x 2 flops x max SM clock",
-                algorithmic_flops_per_launch=flops, algorithmic_bytes_per_launch=nbytes,
-                hbm_gbs=nbytes / (ms_step / 1e3) / 1e9, hbm_frac=nbytes / (ms_step / 1e3) / 1e9 / pk["hbm_gbs"],
-                roofline_ms=max(flops / (alu_peak * 1e12), nbytes / (pk["hbm_gbs"] * 1e9)) * 1e3)
+    roof = bwd_roofline(w, ms_step, clk["sm_max_mhz"])
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
@@ -715,6 +775,8 @@ def main():
                     help="decode steps (T = 1, state in place, B = 256 unless --batch)")
     ap.add_argument("--bwd", action="store_true",
                     help="the backward pass (gradients) on the same workload")
+    ap.add_argument("--bwd-steps", type=int, default=20,
+                    help="backward calls timed for the forward line's 'backward' object (0: none)")
     ap.add_argument("--N", type=int, default=3)
     ap.add_argument("--S", type=int, default=8)
     args = ap.parse_args()
