@@ -31,10 +31,11 @@
 // (dT = dDelta (Vb - Kb h)^T and dL = -T^T dT T^T collapse to -Y Delta^T
 // because T (Vb - Kb h) = Delta.)
 //
-// Four launches: prep (per chunk-head: g, L, T, M, W, U), the forward state
-// chain (per 32-column value slice: h at every chunk start, Delta), the
-// reverse chain (per slice: dh' at every chunk end, Y, dV, dS0) and the
-// key-side gradients (per chunk-head: dQ, dK, dbeta, dalpha).
+// Four launches: prep (per chunk-head: g, L, T, M, W, U and the
+// state-independent M^T dO and (diag(e^g) Q)^T dO), the forward state chain
+// (per 32-column value slice: h at every chunk start, Delta), the reverse chain
+// (per slice: dh' at every chunk end, Y, dV, dS0) and the key-side gradients
+// (per chunk-head: dQ, dK, dbeta, dalpha).
 #pragma once
 
 #include "gdn_bwd_params.cuh"
@@ -57,11 +58,39 @@ __device__ __forceinline__ size_t tok_index(const BwdParams &p, int b, int t, in
     return ((size_t)b * p.T + t) * p.H + h;
 }
 
+// out[r][c] = sum_{i < nterm} A(r, i) scale[i] X[i][c] for r < nrow, c < n, with
+// A(r, i) = A[r * ra + i * ia] in shared memory (so A or its transpose) and
+// scale null meaning 1; written to global memory row-major.  With
+// rstep = kThreads / n column groups, thread t < rstep n takes column t % n
+// and rows t / n + rstep m: each X[i][c] load serves all of its rows, each
+// row a separate accumulator (threads past the last full group idle).
+// 16 <= n <= 128 and ceil(nrow / rstep) <= MAXR.
+template <int MAXR>
+__device__ __forceinline__ void block_product(const float *A, int ra, int ia, int nrow, int nterm,
+                                              const float *scale, const float *X, int xp, int n,
+                                              float *out, int tid) {
+    const int c = tid % n, rg = tid / n, rstep = kThreads / n;
+    if (rg >= rstep) return;
+    const int nr = (nrow - rg + rstep - 1) / rstep;   // rows rg + rstep m < nrow
+    float acc[MAXR];
+#pragma unroll
+    for (int m = 0; m < MAXR; ++m) acc[m] = 0.f;
+    for (int i = 0; i < nterm; ++i) {
+        const float xv = scale ? scale[i] * X[i * xp + c] : X[i * xp + c];
+#pragma unroll
+        for (int m = 0; m < MAXR; ++m)
+            if (m < nr) acc[m] += A[(rg + rstep * m) * ra + i * ia] * xv;
+    }
+#pragma unroll
+    for (int m = 0; m < MAXR; ++m)
+        if (m < nr) out[(size_t)(rg + rstep * m) * n + c] = acc[m];
+}
+
 // ------------------------------------------------------------------- prep
 // One block per chunk-head.  Shared memory (floats): K, Q (C x (dk+1)),
-// V (C x (dv+1)), L, T (C x (C+1)), g, beta, beta e^g (C each).
+// V and then dO (C x (dv+1)), L, T, M (C x (C+1)), g, beta, beta e^g, e^g (C each).
 __host__ __device__ inline size_t prep_smem_floats(int C, int dk, int dv) {
-    return 2 * (size_t)C * (dk + 1) + (size_t)C * (dv + 1) + 2 * (size_t)C * (C + 1) + 3 * (size_t)C;
+    return 2 * (size_t)C * (dk + 1) + (size_t)C * (dv + 1) + 3 * (size_t)C * (C + 1) + 4 * (size_t)C;
 }
 
 __global__ void __launch_bounds__(kThreads) bwd_prep_kernel(const BwdParams p) {
@@ -76,9 +105,11 @@ __global__ void __launch_bounds__(kThreads) bwd_prep_kernel(const BwdParams p) {
     float *Vs = Qs + C * dkp;
     float *Ls = Vs + C * dvp;
     float *Ts = Ls + C * Cp;
-    float *g = Ts + C * Cp;
+    float *Ms = Ts + C * Cp;
+    float *g = Ms + C * Cp;
     float *bb = g + C;
     float *bg = bb + C;
+    float *eg = bg + C;
     const size_t ch = ((size_t)b * p.H + h) * p.NC + n;
 
     for (int x = tid; x < C * dk; x += kThreads) {
@@ -97,19 +128,29 @@ __global__ void __launch_bounds__(kThreads) bwd_prep_kernel(const BwdParams p) {
         Vs[r * dvp + j] = r < Cn ? ld_in(p.v, tok_index(p, b, t0 + r, h) * dv + j, p.io_bf16) : 0.f;
     }
     for (int x = tid; x < C * C; x += kThreads) Ts[(x / C) * Cp + x % C] = 0.f;
+    // gates: every token's log alpha and beta in parallel, then the in-chunk scan
+    if (tid < C) {
+        float la = 0.f, be = 0.f;
+        if (tid < Cn) {
+            const size_t ti = tok_index(p, b, t0 + tid, h);
+            la = p.alpha ? logf(p.alpha[ti]) : 0.f;
+            be = p.beta ? p.beta[ti] : 1.f;
+        }
+        g[tid] = la;             // rows past the tail add 0, so g repeats g_{Cn-1}; their beta is 0
+        bb[tid] = be;
+    }
+    __syncthreads();
     if (tid == 0) {
         float acc = 0.f;
         for (int r = 0; r < C; ++r) {
-            float be = 0.f;
-            if (r < Cn) {
-                const size_t ti = tok_index(p, b, t0 + r, h);
-                if (p.alpha) acc += logf(p.alpha[ti]);
-                be = p.beta ? p.beta[ti] : 1.f;
-            }
-            g[r] = acc;          // rows past the tail repeat g_{Cn-1}; their beta is 0
-            bb[r] = be;
-            bg[r] = be * expf(acc);
+            acc += g[r];
+            g[r] = acc;
         }
+    }
+    __syncthreads();
+    if (tid < C) {
+        eg[tid] = expf(g[tid]);
+        bg[tid] = bb[tid] * eg[tid];
     }
     __syncthreads();
 
@@ -129,7 +170,7 @@ __global__ void __launch_bounds__(kThreads) bwd_prep_kernel(const BwdParams p) {
             if (i < r) l = bb[r] * gam * gk;
         }
         Ls[r * Cp + i] = l;
-        p.ws_M[ch * C * C + x] = m;
+        Ms[r * Cp + i] = m;
     }
     __syncthreads();
 
@@ -149,18 +190,19 @@ __global__ void __launch_bounds__(kThreads) bwd_prep_kernel(const BwdParams p) {
     for (int x = tid; x < C * C; x += kThreads) p.ws_T[ch * C * C + x] = Ts[(x / C) * Cp + x % C];
     if (tid < C) p.ws_g[ch * C + tid] = g[tid];
     // W = T diag(beta e^g) K and U = T diag(beta) V (zero rows past the tail)
-    for (int x = tid; x < C * dk; x += kThreads) {
-        const int r = x / dk, c = x % dk;
-        float s = 0.f;
-        for (int i = 0; i <= r && i < Cn; ++i) s += Ts[r * Cp + i] * bg[i] * Ks[i * dkp + c];
-        p.ws_W[ch * C * dk + x] = s;
-    }
+    block_product<kMaxC * 128 / kThreads>(Ts, Cp, 1, C, Cn, bg, Ks, dkp, dk, p.ws_W + ch * C * dk, tid);
+    block_product<kMaxC * 128 / kThreads>(Ts, Cp, 1, C, Cn, bb, Vs, dvp, dv, p.ws_D + ch * C * dv, tid);
+    __syncthreads();   // V consumed: its buffer takes dO
+    float *dOs = Vs;
     for (int x = tid; x < C * dv; x += kThreads) {
         const int r = x / dv, j = x % dv;
-        float s = 0.f;
-        for (int i = 0; i <= r && i < Cn; ++i) s += Ts[r * Cp + i] * bb[i] * Vs[i * dvp + j];
-        p.ws_D[ch * C * dv + x] = s;
+        dOs[r * dvp + j] = r < Cn ? ld_in(p.grad_o, tok_index(p, b, t0 + r, h) * dv + j, p.do_bf16) : 0.f;
     }
+    __syncthreads();
+    // the state-independent parts of the reverse chain: M^T dO (C x dv) and
+    // (diag(e^g) Q)^T dO (dk x dv)
+    block_product<kMaxC * 128 / kThreads>(Ms, 1, Cp, C, Cn, nullptr, dOs, dvp, dv, p.ws_Y + ch * C * dv, tid);
+    block_product<128 * 128 / kThreads>(Qs, 1, dkp, dk, Cn, eg, dOs, dvp, dv, p.ws_P + ch * dk * dv, tid);
 }
 
 // ------------------------------------------------------ forward state chain
@@ -200,31 +242,54 @@ __global__ void __launch_bounds__(kThreads) bwd_state_fwd_kernel(const BwdParams
         }
         for (int r = rr; r < C; r += 8) Ds[r * 33 + jj] = p.ws_D[(ch * C + r) * dv + j0 + jj];
         __syncthreads();
-        // Delta = U - W h
-        for (int r = rr; r < Cn; r += 8) {
-            float s = Ds[r * 33 + jj];
-            for (int c = 0; c < dk; ++c) s -= Ws[r * dkp + c] * hs[c * 33 + jj];
-            Ds[r * 33 + jj] = s;
-            p.ws_D[(ch * C + r) * dv + j0 + jj] = s;
+        // Delta = U - W h; this thread's rows rr + 8m, one accumulator each
+        {
+            float acc[kMaxC / 8];
+#pragma unroll
+            for (int m = 0; m < kMaxC / 8; ++m) acc[m] = rr + 8 * m < Cn ? Ds[(rr + 8 * m) * 33 + jj] : 0.f;
+            for (int c = 0; c < dk; ++c) {
+                const float hv = hs[c * 33 + jj];
+#pragma unroll
+                for (int m = 0; m < kMaxC / 8; ++m)
+                    if (rr + 8 * m < Cn) acc[m] -= Ws[(rr + 8 * m) * dkp + c] * hv;
+            }
+#pragma unroll
+            for (int m = 0; m < kMaxC / 8; ++m) {
+                const int r = rr + 8 * m;
+                if (r < Cn) {
+                    Ds[r * 33 + jj] = acc[m];
+                    p.ws_D[(ch * C + r) * dv + j0 + jj] = acc[m];
+                }
+            }
         }
         __syncthreads();
-        // h <- e^{g_C} h + (diag(e^{g_C - g}) K)^T Delta
-        const float eglast = expf(glast);
-        for (int c = rr; c < dk; c += 8) {
-            float s = eglast * hs[c * 33 + jj];
-            for (int r = 0; r < Cn; ++r) s += Ks[r * dkp + c] * Ds[r * 33 + jj];
-            hs[c * 33 + jj] = s;
+        // h <- e^{g_C} h + (diag(e^{g_C - g}) K)^T Delta; this thread's key rows rr + 8m
+        {
+            const float eglast = expf(glast);
+            float acc[128 / 8];
+#pragma unroll
+            for (int m = 0; m < 128 / 8; ++m) acc[m] = rr + 8 * m < dk ? eglast * hs[(rr + 8 * m) * 33 + jj] : 0.f;
+            for (int r = 0; r < Cn; ++r) {
+                const float d = Ds[r * 33 + jj];
+#pragma unroll
+                for (int m = 0; m < 128 / 8; ++m)
+                    if (rr + 8 * m < dk) acc[m] += Ks[r * dkp + rr + 8 * m] * d;
+            }
+#pragma unroll
+            for (int m = 0; m < 128 / 8; ++m)
+                if (rr + 8 * m < dk) hs[(rr + 8 * m) * 33 + jj] = acc[m];
         }
     }
 }
 
 // ------------------------------------------------------ reverse state chain
 // One block per (batch, head, 32 value columns); walks the chunks backwards.
-// Shared memory: dh (dk x 33), M, T (C x (C+1) each), K, Q (C x (dk+1) each),
-// dO, X (C x 33 each), g, beta, e^g (C each).
+// The state-independent terms M^T dO and (diag(e^g) Q)^T dO come from the prep
+// kernel, so the serial step per chunk is K dh', T^T dDelta and K^T Y.
+// Shared memory: dh (dk x 33), T (C x (C+1)), K (C x (dk+1)), X (C x 33),
+// g, beta, e^g (C each).
 __host__ __device__ inline size_t state_rev_smem_floats(int C, int dk) {
-    return (size_t)dk * 33 + 2 * (size_t)C * (C + 1) + 2 * (size_t)C * (dk + 1) + 2 * (size_t)C * 33 +
-           3 * (size_t)C;
+    return (size_t)dk * 33 + (size_t)C * (C + 1) + (size_t)C * (dk + 1) + (size_t)C * 33 + 3 * (size_t)C;
 }
 
 __global__ void __launch_bounds__(kThreads) bwd_state_rev_kernel(const BwdParams p) {
@@ -234,12 +299,9 @@ __global__ void __launch_bounds__(kThreads) bwd_state_rev_kernel(const BwdParams
     const int jj = tid & 31, rr = tid >> 5;
     const int dkp = dk + 1, Cp = C + 1;
     float *dhs = sm;
-    float *Ms = dhs + dk * 33;
-    float *Ts = Ms + C * Cp;
+    float *Ts = dhs + dk * 33;
     float *Ks = Ts + C * Cp;
-    float *Qs = Ks + C * dkp;
-    float *dOs = Qs + C * dkp;
-    float *Xs = dOs + C * 33;
+    float *Xs = Ks + C * dkp;
     float *gs = Xs + C * 33;
     float *bs = gs + C;
     float *egs = bs + C;
@@ -252,24 +314,11 @@ __global__ void __launch_bounds__(kThreads) bwd_state_rev_kernel(const BwdParams
         const size_t ch = bh * p.NC + n;
         __syncthreads();   // dh complete; the previous chunk's reads done
         for (int c = rr; c < dk; c += 8) p.ws_dh[(ch * dk + c) * dv + j0 + jj] = dhs[c * 33 + jj];
-        for (int x = tid; x < C * C; x += kThreads) {
-            const int r = x / C, i = x % C;
-            Ms[r * Cp + i] = p.ws_M[ch * C * C + x];
-            Ts[r * Cp + i] = p.ws_T[ch * C * C + x];
-        }
+        for (int x = tid; x < C * C; x += kThreads) Ts[(x / C) * Cp + x % C] = p.ws_T[ch * C * C + x];
         for (int x = tid; x < C * dk; x += kThreads) {
             const int r = x / dk, c = x % dk;
-            float kv = 0.f, qv = 0.f;
-            if (r < Cn) {
-                const size_t ti = tok_index(p, b, t0 + r, h) * dk + c;
-                kv = ld_in(p.k, ti, p.io_bf16);
-                qv = ld_in(p.q, ti, p.io_bf16);
-            }
-            Ks[r * dkp + c] = kv;
-            Qs[r * dkp + c] = qv;
+            Ks[r * dkp + c] = r < Cn ? ld_in(p.k, tok_index(p, b, t0 + r, h) * dk + c, p.io_bf16) : 0.f;
         }
-        for (int r = rr; r < C; r += 8)
-            dOs[r * 33 + jj] = r < Cn ? ld_in(p.grad_o, tok_index(p, b, t0 + r, h) * dv + j0 + jj, p.do_bf16) : 0.f;
         if (tid < C) {
             const float gv = p.ws_g[ch * C + tid];
             gs[tid] = gv;
@@ -278,24 +327,34 @@ __global__ void __launch_bounds__(kThreads) bwd_state_rev_kernel(const BwdParams
         }
         __syncthreads();
         const float glast = gs[Cn - 1];
-        // dDelta = M^T dO + diag(e^{g_C - g}) K dh'
-        for (int r = rr; r < Cn; r += 8) {
-            float s = 0.f;
-            for (int r2 = r; r2 < Cn; ++r2) s += Ms[r2 * Cp + r] * dOs[r2 * 33 + jj];
-            float u = 0.f;
-            for (int c = 0; c < dk; ++c) u += Ks[r * dkp + c] * dhs[c * 33 + jj];
-            Xs[r * 33 + jj] = s + expf(glast - gs[r]) * u;
+        // dDelta = M^T dO + diag(e^{g_C - g}) K dh'; this thread's rows rr + 8m
+        {
+            float u[kMaxC / 8];
+#pragma unroll
+            for (int m = 0; m < kMaxC / 8; ++m) u[m] = 0.f;
+            for (int c = 0; c < dk; ++c) {
+                const float hv = dhs[c * 33 + jj];
+#pragma unroll
+                for (int m = 0; m < kMaxC / 8; ++m)
+                    if (rr + 8 * m < Cn) u[m] += Ks[(rr + 8 * m) * dkp + c] * hv;
+            }
+#pragma unroll
+            for (int m = 0; m < kMaxC / 8; ++m) {
+                const int r = rr + 8 * m;
+                if (r < Cn)
+                    Xs[r * 33 + jj] = p.ws_Y[(ch * C + r) * dv + j0 + jj] + expf(glast - gs[r]) * u[m];
+            }
         }
         __syncthreads();
-        // Y = T^T dDelta (T is lower triangular)
+        // Y = T^T dDelta (T is lower triangular, zero above the diagonal)
         float y[kMaxC / 8];
 #pragma unroll
-        for (int m = 0; m < kMaxC / 8; ++m) {
-            const int r = rr + 8 * m;
-            float s = 0.f;
-            if (r < Cn)
-                for (int r2 = r; r2 < Cn; ++r2) s += Ts[r2 * Cp + r] * Xs[r2 * 33 + jj];
-            y[m] = s;
+        for (int m = 0; m < kMaxC / 8; ++m) y[m] = 0.f;
+        for (int r2 = 0; r2 < Cn; ++r2) {
+            const float xv = Xs[r2 * 33 + jj];
+#pragma unroll
+            for (int m = 0; m < kMaxC / 8; ++m)
+                if (rr + 8 * m < Cn) y[m] += Ts[r2 * Cp + rr + 8 * m] * xv;
         }
         __syncthreads();   // every read of dDelta done
 #pragma unroll
@@ -303,18 +362,29 @@ __global__ void __launch_bounds__(kThreads) bwd_state_rev_kernel(const BwdParams
             const int r = rr + 8 * m;
             if (r < C) Xs[r * 33 + jj] = y[m];
             if (r < Cn) {
-                p.ws_Y[(ch * C + r) * dv + j0 + jj] = y[m];
+                p.ws_Y[(ch * C + r) * dv + j0 + jj] = y[m];   // over M^T dO, read above by this thread
                 p.grad_v[tok_index(p, b, t0 + r, h) * dv + j0 + jj] = bs[r] * y[m];
             }
         }
         __syncthreads();
-        // dh <- e^{g_C} dh' + (diag(e^g) Q)^T dO - (diag(beta e^g) K)^T Y
-        const float eglast = expf(glast);
-        for (int c = rr; c < dk; c += 8) {
-            float s = eglast * dhs[c * 33 + jj];
-            for (int r = 0; r < Cn; ++r)
-                s += egs[r] * (Qs[r * dkp + c] * dOs[r * 33 + jj] - bs[r] * Ks[r * dkp + c] * Xs[r * 33 + jj]);
-            dhs[c * 33 + jj] = s;
+        // dh <- e^{g_C} dh' + (diag(e^g) Q)^T dO - (diag(beta e^g) K)^T Y; key rows rr + 8m
+        {
+            const float eglast = expf(glast);
+            float acc[128 / 8];
+#pragma unroll
+            for (int m = 0; m < 128 / 8; ++m) {
+                const int c = rr + 8 * m;
+                acc[m] = c < dk ? eglast * dhs[c * 33 + jj] + p.ws_P[(ch * dk + c) * dv + j0 + jj] : 0.f;
+            }
+            for (int r = 0; r < Cn; ++r) {
+                const float yb = egs[r] * bs[r] * Xs[r * 33 + jj];
+#pragma unroll
+                for (int m = 0; m < 128 / 8; ++m)
+                    if (rr + 8 * m < dk) acc[m] -= Ks[r * dkp + rr + 8 * m] * yb;
+            }
+#pragma unroll
+            for (int m = 0; m < 128 / 8; ++m)
+                if (rr + 8 * m < dk) dhs[(rr + 8 * m) * 33 + jj] = acc[m];
         }
     }
     __syncthreads();
@@ -432,17 +502,27 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
                 }
             }
             for (int jj = cq; jj < kCols; jj += 4) yv += Yt[r * 33 + jj] * Vt[r * 33 + jj];
+            // this tile's part of dO Delta^T and Y Delta^T at (r, cq + 4m)
+            float s1[MC], s2[MC];
+#pragma unroll
+            for (int m = 0; m < MC; ++m) s1[m] = s2[m] = 0.f;
+            for (int jj = 0; jj < kCols; ++jj) {
+                const float a = dOt[r * 33 + jj], y = Yt[r * 33 + jj];
+#pragma unroll
+                for (int m = 0; m < MC; ++m) {
+                    if (cq + 4 * m < Cn) {
+                        const float d = Dt[(cq + 4 * m) * 33 + jj];
+                        s1[m] += a * d;
+                        s2[m] += y * d;
+                    }
+                }
+            }
+#pragma unroll
             for (int m = 0; m < MC; ++m) {
                 const int i = cq + 4 * m;
                 if (i < Cn) {
-                    float s1 = 0.f, s2 = 0.f;
-                    for (int jj = 0; jj < kCols; ++jj) {
-                        const float d = Dt[i * 33 + jj];
-                        s1 += dOt[r * 33 + jj] * d;
-                        s2 += Yt[r * 33 + jj] * d;
-                    }
-                    dMs[r * Cp + i] += s1;
-                    dLs[r * Cp + i] += s2;
+                    dMs[r * Cp + i] += s1[m];
+                    dLs[r * Cp + i] += s2[m];
                 }
             }
         }
@@ -547,16 +627,32 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
     if (r < Cn) {
         const float eg = egs[r], ebr = bs[r] * egs[r], edec = expf(gs[Cn - 1] - gs[r]);
         const size_t out = tok_index(p, b, t0 + r, h) * DK;
+        // dQ = diag(e^g) dO h^T + (dM (.) Gamma) K, accumulated into A1
+#pragma unroll
+        for (int m = 0; m < MK; ++m) A1[m] *= eg;
+        for (int i = 0; i <= r; ++i) {
+            const float dm = dMs[r * Cp + i];
+#pragma unroll
+            for (int m = 0; m < MK; ++m) A1[m] += dm * Ks[i * dkp + cq + 4 * m];
+        }
+        // dK = (dM (.) Gamma)^T Q + diag(e^{g_C-g}) Delta dh'^T - diag(beta e^g) Y h^T
+        //      + (dG + dG^T) K, accumulated into A3
+#pragma unroll
+        for (int m = 0; m < MK; ++m) A3[m] = edec * A3[m] - ebr * A2[m];
+        for (int r2 = r; r2 < Cn; ++r2) {
+            const float dm = dMs[r2 * Cp + r];
+#pragma unroll
+            for (int m = 0; m < MK; ++m) A3[m] += dm * Qs[r2 * dkp + cq + 4 * m];
+        }
+        for (int i = 0; i < Cn; ++i) {
+            const float dg2 = dLs[r * Cp + i] + dLs[i * Cp + r];
+#pragma unroll
+            for (int m = 0; m < MK; ++m) A3[m] += dg2 * Ks[i * dkp + cq + 4 * m];
+        }
 #pragma unroll
         for (int m = 0; m < MK; ++m) {
-            const int c = cq + 4 * m;
-            float dq = eg * A1[m];
-            float dkv = edec * A3[m] - ebr * A2[m];
-            for (int i = 0; i <= r; ++i) dq += dMs[r * Cp + i] * Ks[i * dkp + c];
-            for (int r2 = r; r2 < Cn; ++r2) dkv += dMs[r2 * Cp + r] * Qs[r2 * dkp + c];
-            for (int i = 0; i < Cn; ++i) dkv += (dLs[r * Cp + i] + dLs[i * Cp + r]) * Ks[i * dkp + c];
-            p.grad_q[out + c] = dq;
-            p.grad_k[out + c] = dkv;
+            p.grad_q[out + cq + 4 * m] = A1[m];
+            p.grad_k[out + cq + 4 * m] = A3[m];
         }
     }
 }

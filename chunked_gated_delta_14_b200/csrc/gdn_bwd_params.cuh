@@ -21,17 +21,18 @@ struct BwdParams {
     // Workspace regions, fp32, each indexed by chunk-head (b*H + h)*NC + n:
     float *ws_g;    // C        in-chunk cumulative log decay g
     float *ws_T;    // C x C    T = (I + L)^-1
-    float *ws_M;    // C x C    causal decayed scores M = (Q K^T) (.) Gamma, i <= r
     float *ws_W;    // C x dk   W = T diag(beta e^g) K
     float *ws_D;    // C x dv   U = T diag(beta) V, overwritten with Delta = U - W h
+    float *ws_Y;    // C x dv   M^T dO (M the causal decayed scores), overwritten with
+                    //          Y = T^T dDelta
+    float *ws_P;    // dk x dv  (diag(e^g) Q)^T dO
     float *ws_h;    // dk x dv  state h = S^T at the chunk's start
     float *ws_dh;   // dk x dv  dL/dh at the chunk's end
-    float *ws_Y;    // C x dv   Y = T^T dDelta
 };
 
 // fp32 words of workspace per chunk-head.
 inline size_t bwd_ws_floats_per_chunk(int C, int dk, int dv) {
-    return (size_t)C + 2 * (size_t)C * C + (size_t)C * dk + 2 * (size_t)C * dv + 2 * (size_t)dk * dv;
+    return (size_t)C + (size_t)C * C + (size_t)C * dk + 2 * (size_t)C * dv + 3 * (size_t)dk * dv;
 }
 
 }  // namespace gdn

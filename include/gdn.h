@@ -187,7 +187,8 @@ GDN_API int32_t gdn_abi_version(void);
  * "Resumo" and "Declaracao do Problema") but print no backward pass; this is
  * the reverse-mode derivative of the chunked WY/UT form, fp32 on CUDA cores,
  * in four launches:
- *   1. per chunk-head: g, L, T = (I + L)^-1, the causal scores M, W, U;
+ *   1. per chunk-head: g, L, T = (I + L)^-1, the causal scores M, W, U, and the
+ *      state-independent M^T dO and (diag(e^g) Q)^T dO;
  *   2. per 32-column value slice, chunks in order: the state at every chunk
  *      start and Delta = U - W h;
  *   3. per slice, chunks in reverse: dL/dh at every chunk end, Y = T^T dDelta,
@@ -229,10 +230,10 @@ typedef struct {
 /* Backward pass (see above). */
 GDN_API gdn_status gdn_chunk_bwd(const gdn_bwd_args *args, void *stream);
 
-/* Workspace bytes gdn_chunk_bwd needs: per chunk-head, fp32 g (C), T and M
- * (C x C), W (C x dk), U / Delta and Y (C x dv), the state and its gradient
- * (dk x dv); 0 with gdn_last_error() set if the arguments are invalid.  Host
- * only. */
+/* Workspace bytes gdn_chunk_bwd needs: per chunk-head, fp32 g (C), T (C x C),
+ * W (C x dk), U / Delta and M^T dO / Y (C x dv), (diag(e^g) Q)^T dO, the state
+ * and its gradient (dk x dv each); 0 with gdn_last_error() set if the
+ * arguments are invalid.  Host only. */
 GDN_API uint64_t gdn_bwd_workspace_bytes(const gdn_bwd_args *args);
 
 /* gdn_chunk_fwd on the tensor-core kernel, with a fixed scratch array inside
