@@ -30,7 +30,7 @@ bool bwd_supports(const BwdParams &p, const char **why) {
 size_t bwd_workspace_bytes(const BwdParams &p) {
     const size_t nch = (size_t)p.B * p.H * p.NC;
     const size_t C = p.C, dk = p.dk, dv = p.dv;
-    return region(C, nch) + region(C * C, nch) + region(C * dk, nch) + 2 * region(C * dv, nch) +
+    return region(C, nch) + 3 * region(C * C, nch) + region(C * dk, nch) + 2 * region(C * dv, nch) +
            3 * region(dk * dv, nch);
 }
 
@@ -40,6 +40,8 @@ void bwd_carve_workspace(BwdParams &p, void *workspace) {
     char *w = static_cast<char *>(workspace);
     p.ws_g = reinterpret_cast<float *>(w);  w += region(C, nch);
     p.ws_T = reinterpret_cast<float *>(w);  w += region(C * C, nch);
+    p.ws_S = reinterpret_cast<float *>(w);  w += region(C * C, nch);
+    p.ws_M = reinterpret_cast<float *>(w);  w += region(C * C, nch);
     p.ws_W = reinterpret_cast<float *>(w);  w += region(C * dk, nch);
     p.ws_D = reinterpret_cast<float *>(w);  w += region(C * dv, nch);
     p.ws_Y = reinterpret_cast<float *>(w);  w += region(C * dv, nch);

@@ -31,7 +31,7 @@
 // (dT = dDelta (Vb - Kb h)^T and dL = -T^T dT T^T collapse to -Y Delta^T
 // because T (Vb - Kb h) = Delta.)
 //
-// Four launches: prep (per chunk-head: g, L, T, M, W, U and the
+// Four launches: prep (per chunk-head: g, L, T, M, W, U, the decayed Gram, and the
 // state-independent M^T dO and (diag(e^g) Q)^T dO), the forward state chain
 // (per 32-column value slice: h at every chunk start, Delta), the reverse chain
 // (per slice: dh' at every chunk end, Y, dV, dS0) and the key-side gradients
@@ -60,30 +60,42 @@ __device__ __forceinline__ size_t tok_index(const BwdParams &p, int b, int t, in
 
 // out[r][c] = sum_{i < nterm} A(r, i) scale[i] X[i][c] for r < nrow, c < n, with
 // A(r, i) = A[r * ra + i * ia] in shared memory (so A or its transpose) and
-// scale null meaning 1; written to global memory row-major.  With
-// rstep = kThreads / n column groups, thread t < rstep n takes column t % n
-// and rows t / n + rstep m: each X[i][c] load serves all of its rows, each
-// row a separate accumulator (threads past the last full group idle).
-// 16 <= n <= 128 and ceil(nrow / rstep) <= MAXR.
+// scale null meaning 1; written to global memory row-major.  With half = n / 2
+// and rstep = kThreads / half row groups, thread t < rstep half takes the two
+// columns t % half and t % half + half and the rows t / half + rstep m: each A
+// load serves both columns and each X load all of the thread's rows, with a
+// separate accumulator per output (threads past the last full group idle).
+// n even, 16 <= n <= 128, and ceil(nrow / rstep) <= MAXR.
 template <int MAXR>
 __device__ __forceinline__ void block_product(const float *A, int ra, int ia, int nrow, int nterm,
                                               const float *scale, const float *X, int xp, int n,
                                               float *out, int tid) {
-    const int c = tid % n, rg = tid / n, rstep = kThreads / n;
-    if (rg >= rstep) return;
+    const int half = n / 2;
+    const int c = tid % half, rg = tid / half, rstep = kThreads / half;
+    if (rg >= rstep || rg >= nrow) return;
     const int nr = (nrow - rg + rstep - 1) / rstep;   // rows rg + rstep m < nrow
-    float acc[MAXR];
+    float acc0[MAXR], acc1[MAXR];
 #pragma unroll
-    for (int m = 0; m < MAXR; ++m) acc[m] = 0.f;
+    for (int m = 0; m < MAXR; ++m) acc0[m] = acc1[m] = 0.f;
     for (int i = 0; i < nterm; ++i) {
-        const float xv = scale ? scale[i] * X[i * xp + c] : X[i * xp + c];
+        const float sc = scale ? scale[i] : 1.f;
+        const float x0 = sc * X[i * xp + c], x1 = sc * X[i * xp + c + half];
 #pragma unroll
-        for (int m = 0; m < MAXR; ++m)
-            if (m < nr) acc[m] += A[(rg + rstep * m) * ra + i * ia] * xv;
+        for (int m = 0; m < MAXR; ++m) {
+            if (m < nr) {
+                const float a = A[(rg + rstep * m) * ra + i * ia];
+                acc0[m] += a * x0;
+                acc1[m] += a * x1;
+            }
+        }
     }
 #pragma unroll
-    for (int m = 0; m < MAXR; ++m)
-        if (m < nr) out[(size_t)(rg + rstep * m) * n + c] = acc[m];
+    for (int m = 0; m < MAXR; ++m) {
+        if (m < nr) {
+            out[(size_t)(rg + rstep * m) * n + c] = acc0[m];
+            out[(size_t)(rg + rstep * m) * n + c + half] = acc1[m];
+        }
+    }
 }
 
 // ------------------------------------------------------------------- prep
@@ -154,23 +166,41 @@ __global__ void __launch_bounds__(kThreads) bwd_prep_kernel(const BwdParams p) {
     }
     __syncthreads();
 
-    // L (strictly lower) and M (lower with diagonal)
-    for (int x = tid; x < C * C; x += kThreads) {
-        const int r = x / C, i = x % C;
-        float l = 0.f, m = 0.f;
-        if (r < Cn && i <= r) {
-            float gk = 0.f, qk = 0.f;
-            for (int c = 0; c < dk; ++c) {
-                const float ki = Ks[i * dkp + c];
-                gk += Ks[r * dkp + c] * ki;
-                qk += Qs[r * dkp + c] * ki;
+    // L (strictly lower) and M (lower with diagonal).  Thread t takes column
+    // i = t % C and rows t / C + (kThreads / C) k, one pair of accumulators each.
+    {
+        constexpr int KR = kMaxC * kMaxC / kThreads;      // rows per thread at C = 64
+        const int i = tid % C, rstep = kThreads / C, nk = C * C / kThreads;
+        float gk[KR], qk[KR];
+#pragma unroll
+        for (int k = 0; k < KR; ++k) gk[k] = qk[k] = 0.f;
+        for (int c = 0; c < dk; ++c) {
+            const float ki = Ks[i * dkp + c];
+#pragma unroll
+            for (int k = 0; k < KR; ++k) {
+                const int r = tid / C + rstep * k;
+                if (k < nk && r < Cn && i <= r) {
+                    gk[k] += Ks[r * dkp + c] * ki;
+                    qk[k] += Qs[r * dkp + c] * ki;
+                }
             }
-            const float gam = expf(g[r] - g[i]);
-            m = gam * qk;
-            if (i < r) l = bb[r] * gam * gk;
         }
-        Ls[r * Cp + i] = l;
-        Ms[r * Cp + i] = m;
+#pragma unroll
+        for (int k = 0; k < KR; ++k) {
+            const int r = tid / C + rstep * k;
+            if (k < nk) {
+                float gg = 0.f, m = 0.f;
+                if (r < Cn && i <= r) {
+                    const float gam = expf(g[r] - g[i]);
+                    m = gam * qk[k];
+                    if (i < r) gg = gam * gk[k];
+                }
+                Ls[r * Cp + i] = bb[r] * gg;
+                Ms[r * Cp + i] = m;
+                p.ws_S[ch * C * C + r * C + i] = gg;
+                p.ws_M[ch * C * C + r * C + i] = m;
+            }
+        }
     }
     __syncthreads();
 
@@ -190,8 +220,8 @@ __global__ void __launch_bounds__(kThreads) bwd_prep_kernel(const BwdParams p) {
     for (int x = tid; x < C * C; x += kThreads) p.ws_T[ch * C * C + x] = Ts[(x / C) * Cp + x % C];
     if (tid < C) p.ws_g[ch * C + tid] = g[tid];
     // W = T diag(beta e^g) K and U = T diag(beta) V (zero rows past the tail)
-    block_product<kMaxC * 128 / kThreads>(Ts, Cp, 1, C, Cn, bg, Ks, dkp, dk, p.ws_W + ch * C * dk, tid);
-    block_product<kMaxC * 128 / kThreads>(Ts, Cp, 1, C, Cn, bb, Vs, dvp, dv, p.ws_D + ch * C * dv, tid);
+    block_product<kMaxC * 64 / kThreads>(Ts, Cp, 1, C, Cn, bg, Ks, dkp, dk, p.ws_W + ch * C * dk, tid);
+    block_product<kMaxC * 64 / kThreads>(Ts, Cp, 1, C, Cn, bb, Vs, dvp, dv, p.ws_D + ch * C * dv, tid);
     __syncthreads();   // V consumed: its buffer takes dO
     float *dOs = Vs;
     for (int x = tid; x < C * dv; x += kThreads) {
@@ -201,8 +231,8 @@ __global__ void __launch_bounds__(kThreads) bwd_prep_kernel(const BwdParams p) {
     __syncthreads();
     // the state-independent parts of the reverse chain: M^T dO (C x dv) and
     // (diag(e^g) Q)^T dO (dk x dv)
-    block_product<kMaxC * 128 / kThreads>(Ms, 1, Cp, C, Cn, nullptr, dOs, dvp, dv, p.ws_Y + ch * C * dv, tid);
-    block_product<128 * 128 / kThreads>(Qs, 1, dkp, dk, Cn, eg, dOs, dvp, dv, p.ws_P + ch * dk * dv, tid);
+    block_product<kMaxC * 64 / kThreads>(Ms, 1, Cp, C, Cn, nullptr, dOs, dvp, dv, p.ws_Y + ch * C * dv, tid);
+    block_product<128 * 64 / kThreads>(Qs, 1, dkp, dk, Cn, eg, dOs, dvp, dv, p.ws_P + ch * dk * dv, tid);
 }
 
 // ------------------------------------------------------ forward state chain
@@ -393,32 +423,34 @@ __global__ void __launch_bounds__(kThreads) bwd_state_rev_kernel(const BwdParams
 }
 
 // ------------------------------------------------------ key-side gradients
-// One block per chunk-head.  Thread (r, cq) = (tid / 4, tid % 4) owns row r
-// and key columns cq + 4m of the three C x dk products over the value axis
-// (dO h^T, Y h^T, Delta dh'^T), accumulated in registers over 32-column
-// value tiles, and entries (r, cq + 4m) of dO Delta^T and Y Delta^T in
-// shared memory.
+// One block per chunk-head.  Thread (rp, c8) = (tid / 8, tid % 8) owns the two
+// rows r0 = 2 rp, r1 = 2 rp + 1 and the key columns c8 + 8m of the three
+// C x dk products over the value axis (dO h^T, Y h^T, Delta dh'^T),
+// accumulated in registers over 32-column value tiles, and the entries
+// (r0 or r1, c8 + 8m) of dO Delta^T and Y Delta^T in shared memory.  Each
+// loaded h, dh' and K element serves both rows.
 // Shared memory: K, Q (C x (DK+1)), two C x (C+1) score buffers, the value
 // tiles (h, dh': DK x 33; dO, Y, Delta, V: C x 33; reused afterwards for two
-// C x (C+1) buffers), g, beta, e^g (C), kThreads partials, 4 x 4 x kMaxC row
+// C x (C+1) buffers), g, beta, e^g (C), kThreads partials, 4 x 8 x kMaxC row
 // partials and 10 x kMaxC row values.
 __host__ __device__ inline size_t grad_smem_floats(int C, int DK) {
     return 2 * (size_t)C * (DK + 1) + 2 * (size_t)C * (C + 1) + 2 * (size_t)DK * 33 + 4 * (size_t)C * 33 +
-           3 * (size_t)C + kThreads + 16 * kMaxC + 10 * kMaxC;
+           3 * (size_t)C + kThreads + 32 * kMaxC + 10 * kMaxC;
 }
 
 enum { RV_A2K = 0, RV_QA1, RV_K3, RV_YV, RV_KAP, RV_DB, RV_DG, RV_HDH };
 
 template <int DK>
 __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
-    constexpr int MK = DK / 4;
-    constexpr int MC = kMaxC / 4;
+    constexpr int MK = DK / 8;         // key columns per thread
+    constexpr int MC = kMaxC / 8;      // score columns per thread
     constexpr int dkp = DK + 1;
     float *sm = reinterpret_cast<float *>(bwd_smem);
     const int C = p.C, dv = p.dv;
     const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-    const int r = tid >> 2, cq = tid & 3;
+    const int c8 = tid & 7, r0 = 2 * (tid >> 3), r1 = r0 + 1;
     const int t0 = n * C, Cn = min(C, p.T - t0);
+    const bool v0 = r0 < Cn, v1 = r1 < Cn;     // r1 < C whenever v0 (C is even)
     const int Cp = C + 1;
     float *Ks = sm;
     float *Qs = Ks + C * dkp;
@@ -435,8 +467,8 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
     float *bs = gs + C;
     float *egs = bs + C;
     float *red = egs + C;
-    float *part = red + kThreads;        // [4 quantities][4 cq][kMaxC]
-    float *rowv = part + 16 * kMaxC;     // [10][kMaxC]
+    float *part = red + kThreads;        // [4 quantities][8 c8][kMaxC]
+    float *rowv = part + 32 * kMaxC;     // [10][kMaxC]
     const size_t ch = ((size_t)b * p.H + h) * p.NC + n;
 
     for (int x = tid; x < C * DK; x += kThreads) {
@@ -461,10 +493,10 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
         egs[tid] = expf(gv);
     }
 
-    float A1[MK], A2[MK], A3[MK];
+    float A1[2][MK], A2[2][MK], A3[2][MK];
 #pragma unroll
-    for (int m = 0; m < MK; ++m) A1[m] = A2[m] = A3[m] = 0.f;
-    float yv = 0.f, hdh = 0.f;
+    for (int m = 0; m < MK; ++m) A1[0][m] = A2[0][m] = A3[0][m] = A1[1][m] = A2[1][m] = A3[1][m] = 0.f;
+    float yv0 = 0.f, yv1 = 0.f, hdh = 0.f;
 
     for (int j0 = 0; j0 < dv; j0 += kCols) {
         __syncthreads();   // previous tile consumed (and, first time, the set-up above)
@@ -489,40 +521,54 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
             Vt[r2 * 33 + jj] = v;
         }
         __syncthreads();
-        if (r < Cn) {
+        if (v0) {   // tile rows at and past Cn are zero, so row r1 needs no test here
             for (int jj = 0; jj < kCols; ++jj) {
-                const float a = dOt[r * 33 + jj], y = Yt[r * 33 + jj], d = Dt[r * 33 + jj];
+                const float a0 = dOt[r0 * 33 + jj], y0 = Yt[r0 * 33 + jj], d0 = Dt[r0 * 33 + jj];
+                const float a1 = dOt[r1 * 33 + jj], y1 = Yt[r1 * 33 + jj], d1 = Dt[r1 * 33 + jj];
 #pragma unroll
                 for (int m = 0; m < MK; ++m) {
-                    const int c = cq + 4 * m;
-                    const float hv = ht[c * 33 + jj];
-                    A1[m] += a * hv;
-                    A2[m] += y * hv;
-                    A3[m] += d * dht[c * 33 + jj];
+                    const int c = c8 + 8 * m;
+                    const float hv = ht[c * 33 + jj], dhv = dht[c * 33 + jj];
+                    A1[0][m] += a0 * hv;
+                    A2[0][m] += y0 * hv;
+                    A3[0][m] += d0 * dhv;
+                    A1[1][m] += a1 * hv;
+                    A2[1][m] += y1 * hv;
+                    A3[1][m] += d1 * dhv;
                 }
             }
-            for (int jj = cq; jj < kCols; jj += 4) yv += Yt[r * 33 + jj] * Vt[r * 33 + jj];
-            // this tile's part of dO Delta^T and Y Delta^T at (r, cq + 4m)
-            float s1[MC], s2[MC];
+            for (int jj = c8; jj < kCols; jj += 8) {
+                yv0 += Yt[r0 * 33 + jj] * Vt[r0 * 33 + jj];
+                yv1 += Yt[r1 * 33 + jj] * Vt[r1 * 33 + jj];
+            }
+            // this tile's part of dO Delta^T and Y Delta^T at (r0 or r1, c8 + 8m)
+            float s1[2][MC], s2[2][MC];
 #pragma unroll
-            for (int m = 0; m < MC; ++m) s1[m] = s2[m] = 0.f;
+            for (int m = 0; m < MC; ++m) s1[0][m] = s2[0][m] = s1[1][m] = s2[1][m] = 0.f;
             for (int jj = 0; jj < kCols; ++jj) {
-                const float a = dOt[r * 33 + jj], y = Yt[r * 33 + jj];
+                const float a0 = dOt[r0 * 33 + jj], y0 = Yt[r0 * 33 + jj];
+                const float a1 = dOt[r1 * 33 + jj], y1 = Yt[r1 * 33 + jj];
 #pragma unroll
                 for (int m = 0; m < MC; ++m) {
-                    if (cq + 4 * m < Cn) {
-                        const float d = Dt[(cq + 4 * m) * 33 + jj];
-                        s1[m] += a * d;
-                        s2[m] += y * d;
+                    if (c8 + 8 * m < Cn) {
+                        const float d = Dt[(c8 + 8 * m) * 33 + jj];
+                        s1[0][m] += a0 * d;
+                        s2[0][m] += y0 * d;
+                        s1[1][m] += a1 * d;
+                        s2[1][m] += y1 * d;
                     }
                 }
             }
 #pragma unroll
             for (int m = 0; m < MC; ++m) {
-                const int i = cq + 4 * m;
+                const int i = c8 + 8 * m;
                 if (i < Cn) {
-                    dMs[r * Cp + i] += s1[m];
-                    dLs[r * Cp + i] += s2[m];
+                    dMs[r0 * Cp + i] += s1[0][m];
+                    dLs[r0 * Cp + i] += s2[0][m];
+                    if (v1) {
+                        dMs[r1 * Cp + i] += s1[1][m];
+                        dLs[r1 * Cp + i] += s2[1][m];
+                    }
                 }
             }
         }
@@ -533,28 +579,30 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
     }
 
     // row dot products k_r.(Y h^T)_r, q_r.(dO h^T)_r, k_r.(Delta dh'^T)_r
-    {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const int r = r0 + e;
         float a2k = 0.f, qa1 = 0.f, k3 = 0.f;
         if (r < Cn) {
 #pragma unroll
             for (int m = 0; m < MK; ++m) {
-                const int c = cq + 4 * m;
-                a2k += A2[m] * Ks[r * dkp + c];
-                qa1 += A1[m] * Qs[r * dkp + c];
-                k3 += A3[m] * Ks[r * dkp + c];
+                const int c = c8 + 8 * m;
+                a2k += A2[e][m] * Ks[r * dkp + c];
+                qa1 += A1[e][m] * Qs[r * dkp + c];
+                k3 += A3[e][m] * Ks[r * dkp + c];
             }
         }
-        part[(0 * 4 + cq) * kMaxC + r] = a2k;
-        part[(1 * 4 + cq) * kMaxC + r] = qa1;
-        part[(2 * 4 + cq) * kMaxC + r] = k3;
-        part[(3 * 4 + cq) * kMaxC + r] = yv;
-        red[tid] = hdh;
+        part[(0 * 8 + c8) * kMaxC + r] = a2k;
+        part[(1 * 8 + c8) * kMaxC + r] = qa1;
+        part[(2 * 8 + c8) * kMaxC + r] = k3;
+        part[(3 * 8 + c8) * kMaxC + r] = e ? yv1 : yv0;
     }
+    red[tid] = hdh;
     __syncthreads();
     if (tid < kMaxC) {
         for (int qn = 0; qn < 4; ++qn) {
             float s = 0.f;
-            for (int c4 = 0; c4 < 4; ++c4) s += part[(qn * 4 + c4) * kMaxC + tid];
+            for (int k8 = 0; k8 < 8; ++k8) s += part[(qn * 8 + k8) * kMaxC + tid];
             rowv[qn * kMaxC + tid] = s;   // RV_A2K, RV_QA1, RV_K3, RV_YV
         }
     }
@@ -564,27 +612,22 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
         rowv[RV_HDH * kMaxC] = s;
     }
 
-    // per score entry: recompute k_r.k_i and q_r.k_i; fold in the decay
+    // per score entry, with the decayed Gram and scores of the prep kernel
     float *Fs = tile;             // dL (.) L + dM (.) M: F_ri enters dg_r with +, dg_i with -
     float *Es = tile + C * Cp;    // dL (.) Gamma (.) k_r.k_i, the beta-derivative of L
     for (int x = tid; x < C * C; x += kThreads) {
         const int r2 = x / C, i = x % C;
         float F = 0.f, E = 0.f, dmg = 0.f, dgv = 0.f;
         if (r2 < Cn && i <= r2) {
-            float gk = 0.f, qk = 0.f;
-            for (int c = 0; c < DK; ++c) {
-                const float ki = Ks[i * dkp + c];
-                gk += Ks[r2 * dkp + c] * ki;
-                qk += Qs[r2 * dkp + c] * ki;
-            }
             const float gam = expf(gs[r2] - gs[i]);
             const float dm = dMs[r2 * Cp + i];
-            F = dm * gam * qk;
+            F = dm * p.ws_M[ch * C * C + x];
             dmg = dm * gam;
             if (i < r2) {
                 const float dl = -dLs[r2 * Cp + i];
-                F += dl * bs[r2] * gam * gk;
-                E = dl * gam * gk;
+                const float gg = p.ws_S[ch * C * C + x];   // Gamma_ri k_r.k_i
+                F += dl * bs[r2] * gg;
+                E = dl * gg;
                 dgv = bs[r2] * dl * gam;
             }
         }
@@ -624,35 +667,62 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
         if (p.grad_beta) p.grad_beta[ti] = rowv[RV_DB * kMaxC + rr];
     }
 
-    if (r < Cn) {
-        const float eg = egs[r], ebr = bs[r] * egs[r], edec = expf(gs[Cn - 1] - gs[r]);
-        const size_t out = tok_index(p, b, t0 + r, h) * DK;
-        // dQ = diag(e^g) dO h^T + (dM (.) Gamma) K, accumulated into A1
+    if (v0) {
+        // dQ = diag(e^g) dO h^T + (dM (.) Gamma) K, accumulated into A1.  dM (.) Gamma
+        // is zero above the diagonal, so both rows run over i <= r1.
 #pragma unroll
-        for (int m = 0; m < MK; ++m) A1[m] *= eg;
-        for (int i = 0; i <= r; ++i) {
-            const float dm = dMs[r * Cp + i];
+        for (int e = 0; e < 2; ++e) {
+            const float eg = egs[r0 + e];   // row r1 past the tail: beta 0, its outputs unused
 #pragma unroll
-            for (int m = 0; m < MK; ++m) A1[m] += dm * Ks[i * dkp + cq + 4 * m];
+            for (int m = 0; m < MK; ++m) A1[e][m] *= eg;
+        }
+        for (int i = 0; i <= r1 && i < Cn; ++i) {
+            const float dm0 = dMs[r0 * Cp + i], dm1 = dMs[r1 * Cp + i];
+#pragma unroll
+            for (int m = 0; m < MK; ++m) {
+                const float kv = Ks[i * dkp + c8 + 8 * m];
+                A1[0][m] += dm0 * kv;
+                A1[1][m] += dm1 * kv;
+            }
         }
         // dK = (dM (.) Gamma)^T Q + diag(e^{g_C-g}) Delta dh'^T - diag(beta e^g) Y h^T
         //      + (dG + dG^T) K, accumulated into A3
 #pragma unroll
-        for (int m = 0; m < MK; ++m) A3[m] = edec * A3[m] - ebr * A2[m];
-        for (int r2 = r; r2 < Cn; ++r2) {
-            const float dm = dMs[r2 * Cp + r];
+        for (int e = 0; e < 2; ++e) {
+            const int r = r0 + e;
+            const float ebr = bs[r] * egs[r], edec = expf(gs[Cn - 1] - gs[r]);
 #pragma unroll
-            for (int m = 0; m < MK; ++m) A3[m] += dm * Qs[r2 * dkp + cq + 4 * m];
+            for (int m = 0; m < MK; ++m) A3[e][m] = edec * A3[e][m] - ebr * A2[e][m];
+        }
+        for (int r2 = r0; r2 < Cn; ++r2) {
+            const float dm0 = dMs[r2 * Cp + r0], dm1 = dMs[r2 * Cp + r1];   // dm1 = 0 at r2 = r0
+#pragma unroll
+            for (int m = 0; m < MK; ++m) {
+                const float qv = Qs[r2 * dkp + c8 + 8 * m];
+                A3[0][m] += dm0 * qv;
+                A3[1][m] += dm1 * qv;
+            }
         }
         for (int i = 0; i < Cn; ++i) {
-            const float dg2 = dLs[r * Cp + i] + dLs[i * Cp + r];
+            const float g0 = dLs[r0 * Cp + i] + dLs[i * Cp + r0];
+            const float g1 = dLs[r1 * Cp + i] + dLs[i * Cp + r1];
 #pragma unroll
-            for (int m = 0; m < MK; ++m) A3[m] += dg2 * Ks[i * dkp + cq + 4 * m];
+            for (int m = 0; m < MK; ++m) {
+                const float kv = Ks[i * dkp + c8 + 8 * m];
+                A3[0][m] += g0 * kv;
+                A3[1][m] += g1 * kv;
+            }
         }
 #pragma unroll
-        for (int m = 0; m < MK; ++m) {
-            p.grad_q[out + cq + 4 * m] = A1[m];
-            p.grad_k[out + cq + 4 * m] = A3[m];
+        for (int e = 0; e < 2; ++e) {
+            if (e == 0 || v1) {
+                const size_t out = tok_index(p, b, t0 + r0 + e, h) * DK;
+#pragma unroll
+                for (int m = 0; m < MK; ++m) {
+                    p.grad_q[out + c8 + 8 * m] = A1[e][m];
+                    p.grad_k[out + c8 + 8 * m] = A3[e][m];
+                }
+            }
         }
     }
 }

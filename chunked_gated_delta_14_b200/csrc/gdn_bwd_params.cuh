@@ -21,6 +21,8 @@ struct BwdParams {
     // Workspace regions, fp32, each indexed by chunk-head (b*H + h)*NC + n:
     float *ws_g;    // C        in-chunk cumulative log decay g
     float *ws_T;    // C x C    T = (I + L)^-1
+    float *ws_S;    // C x C    decayed Gram Gamma (.) K K^T, strictly lower
+    float *ws_M;    // C x C    causal decayed scores M = Gamma (.) Q K^T, lower with diagonal
     float *ws_W;    // C x dk   W = T diag(beta e^g) K
     float *ws_D;    // C x dv   U = T diag(beta) V, overwritten with Delta = U - W h
     float *ws_Y;    // C x dv   M^T dO (M the causal decayed scores), overwritten with
@@ -32,7 +34,7 @@ struct BwdParams {
 
 // fp32 words of workspace per chunk-head.
 inline size_t bwd_ws_floats_per_chunk(int C, int dk, int dv) {
-    return (size_t)C + (size_t)C * C + (size_t)C * dk + 2 * (size_t)C * dv + 3 * (size_t)dk * dv;
+    return (size_t)C + 3 * (size_t)C * C + (size_t)C * dk + 2 * (size_t)C * dv + 3 * (size_t)dk * dv;
 }
 
 }  // namespace gdn

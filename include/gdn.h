@@ -230,10 +230,11 @@ typedef struct {
 /* Backward pass (see above). */
 GDN_API gdn_status gdn_chunk_bwd(const gdn_bwd_args *args, void *stream);
 
-/* Workspace bytes gdn_chunk_bwd needs: per chunk-head, fp32 g (C), T (C x C),
- * W (C x dk), U / Delta and M^T dO / Y (C x dv), (diag(e^g) Q)^T dO, the state
- * and its gradient (dk x dv each); 0 with gdn_last_error() set if the
- * arguments are invalid.  Host only. */
+/* Workspace bytes gdn_chunk_bwd needs: per chunk-head, fp32 g (C), T, the
+ * decayed Gram and the causal scores (C x C each), W (C x dk), U / Delta and
+ * M^T dO / Y (C x dv each), (diag(e^g) Q)^T dO, the state and its gradient
+ * (dk x dv each); 0 with gdn_last_error() set if the arguments are invalid.
+ * Host only. */
 GDN_API uint64_t gdn_bwd_workspace_bytes(const gdn_bwd_args *args);
 
 /* gdn_chunk_fwd on the tensor-core kernel, with a fixed scratch array inside

@@ -144,7 +144,7 @@ def _bwd_args(**kw):
 def _bwd_ws_expected(B, T, H, dk, dv, C):
     nch = B * H * -(-T // C)
     region = lambda f: (f * nch * 4 + 255) // 256 * 256
-    return region(C) + region(C * C) + region(C * dk) + 2 * region(C * dv) + 3 * region(dk * dv)
+    return region(C) + 3 * region(C * C) + region(C * dk) + 2 * region(C * dv) + 3 * region(dk * dv)
 
 
 @pytest.mark.parametrize("shape", [(2, 100, 3, 128, 128, 64), (1, 1, 1, 16, 32, 16),
