@@ -23,7 +23,7 @@ cudaError_t launch_one(K kernel, dim3 grid, size_t smem_floats, const BwdParams 
 bool bwd_supports(const BwdParams &p, const char **why) {
     if (p.C != 16 && p.C != 32 && p.C != 64) { *why = "chunk must be 16, 32 or 64"; return false; }
     if (p.dk != 16 && p.dk != 32 && p.dk != 64 && p.dk != 128) { *why = "dk must be 16, 32, 64 or 128"; return false; }
-    if (p.dv % bwd::kCols != 0 || p.dv > 128) { *why = "dv must be 32, 64 or 128"; return false; }
+    if (p.dv % bwd::kCols != 0 || p.dv > 128) { *why = "dv must be 32, 64, 96 or 128"; return false; }
     return true;
 }
 

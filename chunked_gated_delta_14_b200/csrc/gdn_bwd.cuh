@@ -8,7 +8,7 @@
 namespace gdn {
 
 // Shapes the backward kernels take: chunk 16, 32 or 64; dk 16..128 (a power of
-// two); dv a multiple of 32.
+// two); dv a multiple of 32, at most 128.
 bool bwd_supports(const BwdParams &p, const char **why);
 // Workspace bytes for p (regions 256-byte aligned).
 size_t bwd_workspace_bytes(const BwdParams &p);

@@ -200,7 +200,7 @@ GDN_API int32_t gdn_abi_version(void);
  * Layouts as gdn_fwd_args; every gradient is fp32 in the layout of its input
  * (grad_S0 and grad_S_T in the h = S^T layout [B, H, dk, dv]).
  *
- * Shapes: chunk 16, 32 or 64; dk 16, 32, 64 or 128; dv 32, 64 or 128;
+ * Shapes: chunk 16, 32 or 64; dk 16, 32, 64 or 128; dv 32, 64, 96 or 128;
  * B, H <= 65535.  Other shapes return GDN_ERR_UNSUPPORTED.
  *
  * Ownership and errors as gdn_chunk_fwd: caller-allocated device buffers,
