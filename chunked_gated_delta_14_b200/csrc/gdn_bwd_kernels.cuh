@@ -246,7 +246,8 @@ __global__ void __launch_bounds__(kThreads) bwd_state_fwd_kernel(const BwdParams
     float *sm = reinterpret_cast<float *>(bwd_smem);
     const int C = p.C, dk = p.dk, dv = p.dv;
     const int j0 = blockIdx.x * kCols, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-    const int jj = tid & 31, rr = tid >> 5;
+    const int jj = tid & 31, rr = tid >> 5;     // loads and stores: column jj, rows rr + 8m
+    const int jp = tid & 15, rg = tid >> 4;     // products: columns jp, jp + 16, rows rg + 16m
     const int dkp = dk + 1;
     float *hs = sm;
     float *Ws = hs + dk * 33;
@@ -272,42 +273,67 @@ __global__ void __launch_bounds__(kThreads) bwd_state_fwd_kernel(const BwdParams
         }
         for (int r = rr; r < C; r += 8) Ds[r * 33 + jj] = p.ws_D[(ch * C + r) * dv + j0 + jj];
         __syncthreads();
-        // Delta = U - W h; this thread's rows rr + 8m, one accumulator each
+        // Delta = U - W h: this thread's columns jp, jp + 16 and rows rg + 16m
         {
-            float acc[kMaxC / 8];
+            float a0[kMaxC / 16], a1[kMaxC / 16];
 #pragma unroll
-            for (int m = 0; m < kMaxC / 8; ++m) acc[m] = rr + 8 * m < Cn ? Ds[(rr + 8 * m) * 33 + jj] : 0.f;
+            for (int m = 0; m < kMaxC / 16; ++m) {
+                const int r = rg + 16 * m;
+                a0[m] = r < Cn ? Ds[r * 33 + jp] : 0.f;
+                a1[m] = r < Cn ? Ds[r * 33 + jp + 16] : 0.f;
+            }
             for (int c = 0; c < dk; ++c) {
-                const float hv = hs[c * 33 + jj];
+                const float h0 = hs[c * 33 + jp], h1 = hs[c * 33 + jp + 16];
 #pragma unroll
-                for (int m = 0; m < kMaxC / 8; ++m)
-                    if (rr + 8 * m < Cn) acc[m] -= Ws[(rr + 8 * m) * dkp + c] * hv;
+                for (int m = 0; m < kMaxC / 16; ++m) {
+                    if (rg + 16 * m < Cn) {
+                        const float wv = Ws[(rg + 16 * m) * dkp + c];
+                        a0[m] -= wv * h0;
+                        a1[m] -= wv * h1;
+                    }
+                }
             }
 #pragma unroll
-            for (int m = 0; m < kMaxC / 8; ++m) {
-                const int r = rr + 8 * m;
+            for (int m = 0; m < kMaxC / 16; ++m) {
+                const int r = rg + 16 * m;
                 if (r < Cn) {
-                    Ds[r * 33 + jj] = acc[m];
-                    p.ws_D[(ch * C + r) * dv + j0 + jj] = acc[m];
+                    Ds[r * 33 + jp] = a0[m];
+                    Ds[r * 33 + jp + 16] = a1[m];
+                    p.ws_D[(ch * C + r) * dv + j0 + jp] = a0[m];
+                    p.ws_D[(ch * C + r) * dv + j0 + jp + 16] = a1[m];
                 }
             }
         }
         __syncthreads();
-        // h <- e^{g_C} h + (diag(e^{g_C - g}) K)^T Delta; this thread's key rows rr + 8m
+        // h <- e^{g_C} h + (diag(e^{g_C - g}) K)^T Delta: columns jp, jp + 16, key rows rg + 16m
         {
             const float eglast = expf(glast);
-            float acc[128 / 8];
+            float a0[128 / 16], a1[128 / 16];
 #pragma unroll
-            for (int m = 0; m < 128 / 8; ++m) acc[m] = rr + 8 * m < dk ? eglast * hs[(rr + 8 * m) * 33 + jj] : 0.f;
+            for (int m = 0; m < 128 / 16; ++m) {
+                const int c = rg + 16 * m;
+                a0[m] = c < dk ? eglast * hs[c * 33 + jp] : 0.f;
+                a1[m] = c < dk ? eglast * hs[c * 33 + jp + 16] : 0.f;
+            }
             for (int r = 0; r < Cn; ++r) {
-                const float d = Ds[r * 33 + jj];
+                const float d0 = Ds[r * 33 + jp], d1 = Ds[r * 33 + jp + 16];
 #pragma unroll
-                for (int m = 0; m < 128 / 8; ++m)
-                    if (rr + 8 * m < dk) acc[m] += Ks[r * dkp + rr + 8 * m] * d;
+                for (int m = 0; m < 128 / 16; ++m) {
+                    if (rg + 16 * m < dk) {
+                        const float kv = Ks[r * dkp + rg + 16 * m];
+                        a0[m] += kv * d0;
+                        a1[m] += kv * d1;
+                    }
+                }
             }
 #pragma unroll
-            for (int m = 0; m < 128 / 8; ++m)
-                if (rr + 8 * m < dk) hs[(rr + 8 * m) * 33 + jj] = acc[m];
+            for (int m = 0; m < 128 / 16; ++m) {
+                const int c = rg + 16 * m;
+                if (c < dk) {
+                    hs[c * 33 + jp] = a0[m];
+                    hs[c * 33 + jp + 16] = a1[m];
+                }
+            }
         }
     }
 }
@@ -326,7 +352,8 @@ __global__ void __launch_bounds__(kThreads) bwd_state_rev_kernel(const BwdParams
     float *sm = reinterpret_cast<float *>(bwd_smem);
     const int C = p.C, dk = p.dk, dv = p.dv;
     const int j0 = blockIdx.x * kCols, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-    const int jj = tid & 31, rr = tid >> 5;
+    const int jj = tid & 31, rr = tid >> 5;     // loads and stores: column jj, rows rr + 8m
+    const int jp = tid & 15, rg = tid >> 4;     // products: columns jp, jp + 16, rows rg + 16m
     const int dkp = dk + 1, Cp = C + 1;
     float *dhs = sm;
     float *Ts = dhs + dk * 33;
@@ -357,64 +384,99 @@ __global__ void __launch_bounds__(kThreads) bwd_state_rev_kernel(const BwdParams
         }
         __syncthreads();
         const float glast = gs[Cn - 1];
-        // dDelta = M^T dO + diag(e^{g_C - g}) K dh'; this thread's rows rr + 8m
+        // dDelta = M^T dO + diag(e^{g_C - g}) K dh': columns jp, jp + 16, rows rg + 16m
         {
-            float u[kMaxC / 8];
+            float u0[kMaxC / 16], u1[kMaxC / 16];
 #pragma unroll
-            for (int m = 0; m < kMaxC / 8; ++m) u[m] = 0.f;
+            for (int m = 0; m < kMaxC / 16; ++m) u0[m] = u1[m] = 0.f;
             for (int c = 0; c < dk; ++c) {
-                const float hv = dhs[c * 33 + jj];
+                const float h0 = dhs[c * 33 + jp], h1 = dhs[c * 33 + jp + 16];
 #pragma unroll
-                for (int m = 0; m < kMaxC / 8; ++m)
-                    if (rr + 8 * m < Cn) u[m] += Ks[(rr + 8 * m) * dkp + c] * hv;
+                for (int m = 0; m < kMaxC / 16; ++m) {
+                    if (rg + 16 * m < Cn) {
+                        const float kv = Ks[(rg + 16 * m) * dkp + c];
+                        u0[m] += kv * h0;
+                        u1[m] += kv * h1;
+                    }
+                }
             }
 #pragma unroll
-            for (int m = 0; m < kMaxC / 8; ++m) {
-                const int r = rr + 8 * m;
-                if (r < Cn)
-                    Xs[r * 33 + jj] = p.ws_Y[(ch * C + r) * dv + j0 + jj] + expf(glast - gs[r]) * u[m];
+            for (int m = 0; m < kMaxC / 16; ++m) {
+                const int r = rg + 16 * m;
+                if (r < Cn) {
+                    const float e = expf(glast - gs[r]);
+                    const size_t w = (ch * C + r) * dv + j0 + jp;
+                    Xs[r * 33 + jp] = p.ws_Y[w] + e * u0[m];
+                    Xs[r * 33 + jp + 16] = p.ws_Y[w + 16] + e * u1[m];
+                }
             }
         }
         __syncthreads();
         // Y = T^T dDelta (T is lower triangular, zero above the diagonal)
-        float y[kMaxC / 8];
+        float y0[kMaxC / 16], y1[kMaxC / 16];
 #pragma unroll
-        for (int m = 0; m < kMaxC / 8; ++m) y[m] = 0.f;
+        for (int m = 0; m < kMaxC / 16; ++m) y0[m] = y1[m] = 0.f;
         for (int r2 = 0; r2 < Cn; ++r2) {
-            const float xv = Xs[r2 * 33 + jj];
+            const float x0 = Xs[r2 * 33 + jp], x1 = Xs[r2 * 33 + jp + 16];
 #pragma unroll
-            for (int m = 0; m < kMaxC / 8; ++m)
-                if (rr + 8 * m < Cn) y[m] += Ts[r2 * Cp + rr + 8 * m] * xv;
+            for (int m = 0; m < kMaxC / 16; ++m) {
+                if (rg + 16 * m < Cn) {
+                    const float tv = Ts[r2 * Cp + rg + 16 * m];
+                    y0[m] += tv * x0;
+                    y1[m] += tv * x1;
+                }
+            }
         }
         __syncthreads();   // every read of dDelta done
 #pragma unroll
-        for (int m = 0; m < kMaxC / 8; ++m) {
-            const int r = rr + 8 * m;
-            if (r < C) Xs[r * 33 + jj] = y[m];
+        for (int m = 0; m < kMaxC / 16; ++m) {
+            const int r = rg + 16 * m;
+            if (r < C) {
+                Xs[r * 33 + jp] = y0[m];
+                Xs[r * 33 + jp + 16] = y1[m];
+            }
             if (r < Cn) {
-                p.ws_Y[(ch * C + r) * dv + j0 + jj] = y[m];   // over M^T dO, read above by this thread
-                p.grad_v[tok_index(p, b, t0 + r, h) * dv + j0 + jj] = bs[r] * y[m];
+                const size_t w = (ch * C + r) * dv + j0 + jp;     // over M^T dO, read above by this thread
+                p.ws_Y[w] = y0[m];
+                p.ws_Y[w + 16] = y1[m];
+                const size_t o = tok_index(p, b, t0 + r, h) * dv + j0 + jp;
+                p.grad_v[o] = bs[r] * y0[m];
+                p.grad_v[o + 16] = bs[r] * y1[m];
             }
         }
         __syncthreads();
-        // dh <- e^{g_C} dh' + (diag(e^g) Q)^T dO - (diag(beta e^g) K)^T Y; key rows rr + 8m
+        // dh <- e^{g_C} dh' + (diag(e^g) Q)^T dO - (diag(beta e^g) K)^T Y:
+        // columns jp, jp + 16, key rows rg + 16m
         {
             const float eglast = expf(glast);
-            float acc[128 / 8];
+            float a0[128 / 16], a1[128 / 16];
 #pragma unroll
-            for (int m = 0; m < 128 / 8; ++m) {
-                const int c = rr + 8 * m;
-                acc[m] = c < dk ? eglast * dhs[c * 33 + jj] + p.ws_P[(ch * dk + c) * dv + j0 + jj] : 0.f;
+            for (int m = 0; m < 128 / 16; ++m) {
+                const int c = rg + 16 * m;
+                const size_t w = (ch * dk + c) * dv + j0 + jp;
+                a0[m] = c < dk ? eglast * dhs[c * 33 + jp] + p.ws_P[w] : 0.f;
+                a1[m] = c < dk ? eglast * dhs[c * 33 + jp + 16] + p.ws_P[w + 16] : 0.f;
             }
             for (int r = 0; r < Cn; ++r) {
-                const float yb = egs[r] * bs[r] * Xs[r * 33 + jj];
+                const float eb = egs[r] * bs[r];
+                const float yb0 = eb * Xs[r * 33 + jp], yb1 = eb * Xs[r * 33 + jp + 16];
 #pragma unroll
-                for (int m = 0; m < 128 / 8; ++m)
-                    if (rr + 8 * m < dk) acc[m] -= Ks[r * dkp + rr + 8 * m] * yb;
+                for (int m = 0; m < 128 / 16; ++m) {
+                    if (rg + 16 * m < dk) {
+                        const float kv = Ks[r * dkp + rg + 16 * m];
+                        a0[m] -= kv * yb0;
+                        a1[m] -= kv * yb1;
+                    }
+                }
             }
 #pragma unroll
-            for (int m = 0; m < 128 / 8; ++m)
-                if (rr + 8 * m < dk) dhs[(rr + 8 * m) * 33 + jj] = acc[m];
+            for (int m = 0; m < 128 / 16; ++m) {
+                const int c = rg + 16 * m;
+                if (c < dk) {
+                    dhs[c * 33 + jp] = a0[m];
+                    dhs[c * 33 + jp + 16] = a1[m];
+                }
+            }
         }
     }
     __syncthreads();

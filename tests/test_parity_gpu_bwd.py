@@ -87,6 +87,10 @@ def test_backward_is_deterministic_and_chunk_independent():
     b = _run_bwd(x, c, 32)
     for k in a:
         assert np.array_equal(a[k], b[k]), k        # no atomics: bit-identical reruns
+    no_s0 = _run_bwd(x, c, 32, want_S0=False)       # grad_S0 NULL changes nothing else
+    assert no_s0["dS0"] is None
+    for k in ("dq", "dk", "dv", "dalpha", "dbeta"):
+        assert np.array_equal(a[k], no_s0[k]), k
     ref = _oracle_bwd(x, c)
     for chunk in (16, 64):
         _compare(f"bwd_chunk{chunk}", _run_bwd(x, c, chunk), ref)
