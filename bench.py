@@ -204,6 +204,72 @@ class ClockSampler:
                     reasons=sorted(reasons), samples=len(sm))
 
 
+def pipelined_e2e(host_in, run, steps, dev, warm=2, barrier=None):
+    """End-to-end steps through the public API, timed on the device clock.
+
+    Per step, every pinned host tensor of ``host_in`` is copied to the device,
+    ``run(dev_in, slot)`` computes on the current stream and returns the device
+    tensors to read back, and those are copied into pinned host buffers.
+    Uploads run on one copy stream and readbacks on another, with two slots of
+    device inputs: step i's compute and readback overlap step i+1's upload,
+    and every step still moves all of its own bytes.  Events order each reuse
+    of a slot (an upload waits for the compute that read the slot's previous
+    inputs; a compute waits for the readback of the slot's previous outputs).
+    Returns (ms per step, bytes uploaded per step, bytes read back per step).
+    """
+    import torch
+    comp = torch.cuda.current_stream(dev)
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    dev_in = [{k: torch.empty_like(v, device=dev) for k, v in host_in.items()} for _ in range(2)]
+    in_done = [torch.cuda.Event(), torch.cuda.Event()]
+    comp_done = [torch.cuda.Event(), torch.cuda.Event()]
+    out_done = [torch.cuda.Event(), torch.cuda.Event()]
+    host_out = [None, None]
+    used = [False, False]
+    nbytes = dict(h2d=sum(v.numel() * v.element_size() for v in host_in.values()), d2h=0)
+
+    def step(i):
+        b = i & 1
+        with torch.cuda.stream(s_in):
+            if used[b]:
+                s_in.wait_event(comp_done[b])
+            for k, v in host_in.items():
+                dev_in[b][k].copy_(v, non_blocking=True)
+            in_done[b].record(s_in)
+        comp.wait_event(in_done[b])
+        if used[b]:
+            comp.wait_event(out_done[b])
+        res = run(dev_in[b], b)
+        comp_done[b].record(comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[b])
+            if host_out[b] is None:
+                host_out[b] = {k: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for k, t in res.items()}
+            for k, t in res.items():
+                t.record_stream(s_out)
+                host_out[b][k].copy_(t, non_blocking=True)
+            out_done[b].record(s_out)
+        used[b] = True
+        nbytes["d2h"] = sum(t.numel() * t.element_size() for t in res.values())
+
+    for i in range(warm):
+        step(i)
+    torch.cuda.synchronize()
+    if barrier is not None:
+        barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    s_in.wait_event(e0)
+    for i in range(steps):
+        step(warm + i)
+    comp.wait_event(out_done[0])
+    comp.wait_event(out_done[1])
+    e1.record(comp)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, nbytes["h2d"], nbytes["d2h"]
+
+
 # ------------------------------------------------------------ our arm (GPU)
 
 def run_gpu(args, rank, world, local_rank):
@@ -272,38 +338,22 @@ def run_gpu(args, rank, world, local_rank):
     # end to end through the public API: pinned host inputs -> device -> kernel -> host o
     e2e = None
     if args.e2e_steps > 0:
-        host = {k: (None if v is None else v.pin_memory()) for k, v in x.items()}
-        dev_in = {k: (None if v is None else torch.empty_like(v, device=dev)) for k, v in x.items()}
-        o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-        h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
-        d2h = o_host.numel() * o_host.element_size()
+        host = {k: v.pin_memory() for k, v in x.items() if v is not None}
+        outs = [torch.empty_like(o) for _ in range(2)]
+        finals = [torch.empty_like(S_T) for _ in range(2)]
 
-        def e2e_step():
-            for k, v in host.items():
-                if v is not None:
-                    dev_in[k].copy_(v, non_blocking=True)
-            gdn.chunk_fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"],
-                          dev_in["beta"], chunk=w.chunk, o_dtype=torch.bfloat16, out=o, mode=args.mode,
-                          N=args.N, S=args.S,
-                          S_T=S_T)
-            o_host.copy_(o, non_blocking=True)
+        def run(di, slot):
+            gdn.chunk_fwd(di["q"], di["k"], di["v"], di.get("alpha"), di.get("beta"), chunk=w.chunk,
+                          o_dtype=torch.bfloat16, out=outs[slot], mode=args.mode, N=args.N, S=args.S,
+                          S_T=finals[slot])
+            return {"o": outs[slot]}
 
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        f0 = torch.cuda.Event(enable_timing=True)
-        f1 = torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        f1.record(stream)
-        torch.cuda.synchronize()
-        ems = max_over_ranks(f0.elapsed_time(f1), world, dev)
-        e2e = dict(value=job_throughput(tokens_step, world, args.e2e_steps, ems), unit=UNIT,
-                   h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h),
-                   ms_per_step=ems / args.e2e_steps)
+        ems, h2d, d2h = pipelined_e2e(host, run, args.e2e_steps, dev,
+                                      barrier=dist.barrier if world > 1 else None)
+        ems = max_over_ranks(ems, world, dev)
+        e2e = dict(value=job_throughput(tokens_step, world, 1, ems), unit=UNIT,
+                   h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h), ms_per_step=ems,
+                   pipeline="uploads, compute and readbacks on three streams, two input slots")
 
     pk = peaks()
     bytes_launch = algorithmic_bytes(w, o_bytes=2)
@@ -578,6 +628,7 @@ def backward_side_measure(w, x, rank, world, dev, steps, warmup, sm_max_mhz):
 def run_bwd(args, rank, world, local_rank):
     """One gdn_chunk_bwd call per step over the whole batch."""
     import torch
+    import torch.distributed as dist
     import chunked_gated_delta_14_b200 as gdn
     from chunked_gated_delta_14_b200.inputs import make_cotangents, make_inputs, workload
 
@@ -622,34 +673,19 @@ def run_bwd(args, rank, world, local_rank):
     if args.e2e_steps > 0:
         host = {k: x[k].pin_memory() for k in ("q", "k", "v", "alpha", "beta")}
         host["grad_o"] = c["grad_o"].pin_memory()
-        dev_in = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
-        outs_host = {k: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-                     for k, t in (("dq", g["dq"]), ("dk", g["dk"]), ("dv", g["dv"]),
-                                  ("dalpha", g["da"]), ("dbeta", g["db"]))}
-        h2d = sum(t.numel() * t.element_size() for t in host.values())
-        d2h = sum(t.numel() * t.element_size() for t in outs_host.values())
 
-        def e2e_step():
-            for k, t in host.items():
-                dev_in[k].copy_(t, non_blocking=True)
-            r = gdn.chunk_bwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"], dev_in["beta"],
-                              dev_in["grad_o"], chunk=w.chunk, want_S0=False)
-            for k, t in outs_host.items():
-                t.copy_(r[k], non_blocking=True)
+        def run(di, slot):
+            r = gdn.chunk_bwd(di["q"], di["k"], di["v"], di["alpha"], di["beta"], di["grad_o"],
+                              chunk=w.chunk, want_S0=False)
+            return {k: r[k] for k in ("dq", "dk", "dv", "dalpha", "dbeta")}
 
-        e2e_step()
-        torch.cuda.synchronize()
-        f0 = torch.cuda.Event(enable_timing=True)
-        f1 = torch.cuda.Event(enable_timing=True)
         n_e2e = max(1, args.e2e_steps // 4)
-        f0.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
-        f1.record(stream)
-        torch.cuda.synchronize()
-        ems = max_over_ranks(f0.elapsed_time(f1), world, dev)
-        e2e = dict(value=job_throughput(tokens_step, world, n_e2e, ems), unit=UNIT,
-                   h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h), ms_per_step=ems / n_e2e)
+        ems, h2d, d2h = pipelined_e2e(host, run, n_e2e, dev,
+                                      barrier=dist.barrier if world > 1 else None)
+        ems = max_over_ranks(ems, world, dev)
+        e2e = dict(value=job_throughput(tokens_step, world, 1, ems), unit=UNIT,
+                   h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h), ms_per_step=ems,
+                   pipeline="uploads, compute and readbacks on three streams, two input slots")
 
     clk = clocks.summary()
     nbytes = bwd_bytes(w)

@@ -38,6 +38,12 @@ def fake_cuda(monkeypatch):
     class Stream:
         cuda_stream = 0
 
+        def __init__(self, *a, **kw):
+            pass
+
+        def wait_event(self, ev):
+            pass
+
     calls = dict(fwd=0, bwd=0)
 
     def fwd(a, s=None):
@@ -56,6 +62,9 @@ def fake_cuda(monkeypatch):
 
     monkeypatch.setattr(torch.cuda, "Event", Event)
     monkeypatch.setattr(torch.cuda, "current_stream", lambda dev=None: Stream())
+    monkeypatch.setattr(torch.cuda, "Stream", Stream)
+    monkeypatch.setattr(torch.cuda, "stream", lambda st: contextlib.nullcontext())
+    monkeypatch.setattr(torch.Tensor, "record_stream", lambda self, st: None)
     monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
     monkeypatch.setattr(torch.cuda, "set_device", lambda *a, **k: None)
     monkeypatch.setattr(torch.cuda, "device", lambda d: contextlib.nullcontext())
@@ -94,6 +103,7 @@ def _check_contract(line):
     assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-12
     e = line["e2e"]
     assert e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] > 0 and e["unit"] == line["unit"]
+    assert e["value"] > 0 and e["ms_per_step"] > 0
     c = line["cpu_baseline"]
     assert c["kind"] == "oracle" and c["cores"] >= 1 and c["value"] > 0 and c["sample"]
     assert line["gpu_launches"] > 0
