@@ -206,3 +206,27 @@ def test_python_backward_rejects_cpu_tensors():
     v = torch.zeros(1, 4, 1, 32, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         gdn.chunk_bwd(q, q, v, None, None, v)
+
+
+def _c_layout(struct, fields, tmp_path):
+    """sizeof and offsetof of every field of a struct in include/gdn.h, from gcc."""
+    src = tmp_path / "layout.c"
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "gdn.h"', "int main(void) {",
+             f'  printf("%zu\\n", sizeof({struct}));']
+    lines += [f'  printf("%zu\\n", offsetof({struct}, {f}));' for f in fields]
+    lines += ["  return 0;", "}"]
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    vals = [int(v) for v in subprocess.check_output([str(exe)]).decode().split()]
+    return vals[0], vals[1:]
+
+
+@pytest.mark.parametrize("struct,mirror", [("gdn_fwd_args", gdn.FwdArgs), ("gdn_bwd_args", gdn.BwdArgs)])
+def test_ctypes_mirrors_match_the_c_structs(struct, mirror, tmp_path):
+    import ctypes
+    fields = [f[0] for f in mirror._fields_]
+    size, offsets = _c_layout(struct, fields, tmp_path)
+    assert ctypes.sizeof(mirror) == size
+    for name, off in zip(fields, offsets):
+        assert getattr(mirror, name).offset == off, name
