@@ -135,3 +135,13 @@ def test_decode_line(fake_cuda):
     line = _line("run_decode", batch=8)
     _check_contract(line)
     assert line["roofline"]["bound"] == "hbm" and line["config"]["seq_len"] == 1
+
+
+def test_e2e_falls_back_to_one_stream(fake_cuda, monkeypatch):
+    import bench
+
+    def broken(*a, **k):
+        raise RuntimeError("stand-in failure")
+    monkeypatch.setattr(bench, "pipelined_e2e", broken)
+    line = _line("run_gpu", bwd_steps=0, no_cpu_baseline=True)
+    assert line["e2e"]["value"] > 0 and line["e2e"]["pipeline"].startswith("one stream")
