@@ -180,18 +180,27 @@ def workspace_bytes(args: FwdArgs) -> int:
 _ws_cache = {}
 
 
-def workspace_for(args, device: torch.device) -> Optional[torch.Tensor]:
+def workspace_for(args, device: torch.device,
+                  stream: Optional[torch.cuda.Stream] = None) -> Optional[torch.Tensor]:
     """A cached device buffer of at least the workspace ``args`` needs, or None.
 
-    Forward (FwdArgs) and backward (BwdArgs) calls keep separate buffers."""
+    One buffer per (device, stream, direction): calls ordered on one stream
+    reuse it, calls on different streams never share one, and forward
+    (FwdArgs) and backward (BwdArgs) calls keep separate buffers.  ``stream``
+    is the stream the call will run on (default: the device's current one)."""
     bwd = isinstance(args, BwdArgs)
     need = bwd_workspace_bytes(args) if bwd else workspace_bytes(args)
     if need == 0:
         return None
-    key = (device.type, device.index, bwd)
+    current = torch.cuda.current_stream(device)
+    if stream is None:
+        stream = current
+    key = (device.type, device.index, stream.cuda_stream, bwd)
     buf = _ws_cache.get(key)
     if buf is None or buf.numel() < need:
         buf = torch.empty(need, dtype=torch.uint8, device=device)
+        if stream.cuda_stream != current.cuda_stream:
+            buf.record_stream(stream)   # freed blocks wait for the stream that used them
         _ws_cache[key] = buf
     return buf
 
@@ -274,7 +283,7 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         neumann_N=int(N), residual_S=int(S), kernel=KERNELS[kernel], dv_split=int(dv_split))
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
-    ws = workspace_for(args, q.device)
+    ws = workspace_for(args, q.device, stream)
     if ws is not None:
         args.workspace = ws.data_ptr()
         args.workspace_bytes = ws.numel()
@@ -343,7 +352,7 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         grad_alpha=_ptr(g["dalpha"]), grad_beta=_ptr(g["dbeta"]), grad_S0=_ptr(g["dS0"]))
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
-    ws = workspace_for(args, q.device)
+    ws = workspace_for(args, q.device, stream)
     if ws is not None:
         args.workspace = ws.data_ptr()
         args.workspace_bytes = ws.numel()
