@@ -14,7 +14,10 @@ skipping the ones a workload does not use):
 * v: N(0, 1), rounded to the io dtype.
 * beta = sigmoid(N(0, 1)), fp32, shape [B, T, H].
 * alpha = exp(-softplus(N(0, 1) + 2)), fp32, shape [B, T, H] (scalar decay)
-  or [B, T, H, d_k] (per key channel).  ``None`` means alpha == 1.
+  or [B, T, H, d_k] (per key channel).  ``None`` means alpha == 1.  The
+  "weak" scalar decay, the regime of trained Gated DeltaNet layers whose gates
+  sit close to 1, draws alpha = 0.9 + 0.1 U[0, 1) (fp32 uniform) in the same
+  slot instead.
 * S0 ~ N(0, 0.02^2) (0.02 is the standard deviation), fp32 [B, H, d_k, d_v].
 * erase gate b and write gate w = sigmoid(N(0, 1)) in the io dtype,
   shapes [B, T, H, d_k] and [B, T, H, d_v].
@@ -48,7 +51,7 @@ class Workload:
     dv: int
     chunk: int
     io: str                 # "f32" or "bf16"
-    decay: str              # "none" | "scalar" | "channel"
+    decay: str              # "none" | "scalar" | "weak" | "channel"
     beta: bool              # scalar write strength beta_t present
     s0_std: float           # 0 -> no initial state
     gates: bool             # erase/write channel gates present
@@ -139,6 +142,9 @@ def make_inputs(w: Workload, seed: int = 0) -> dict:
         alpha = None
     elif w.decay == "scalar":
         alpha = torch.from_numpy(_decay(normal((B, T, H))))
+    elif w.decay == "weak":
+        u = rng.random(size=(B, T, H), dtype=np.float32)
+        alpha = torch.from_numpy((np.float32(0.9) + np.float32(0.1) * u).astype(np.float32))
     elif w.decay == "channel":
         alpha = torch.from_numpy(_decay(normal((B, T, H, dk))))
     else:
