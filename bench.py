@@ -41,7 +41,6 @@ sys.path.insert(0, ROOT)
 WORKLOAD = "gdn_bf16"
 METRIC = "tokens/s (fwd, bf16, H=16, d=128, T=4096) and % of roofline on 1 B200"
 UNIT = "tokens/s"
-PROFILE = os.path.join(ROOT, "profiles", "gdn_fwd_gdn_bf16_ncu.md")
 
 
 # --------------------------------------------------------------------- utils
@@ -69,7 +68,7 @@ def algorithmic_bytes(w, o_bytes):
     S0 (if given) and S_T per (batch, head)."""
     in_b = 2 if w.io == "bf16" else 4
     per_th = 2 * w.dk * in_b + w.dv * in_b + w.dv * o_bytes
-    per_th += 4 if w.decay == "scalar" else (4 * w.dk if w.decay == "channel" else 0)
+    per_th += 4 if w.decay in ("scalar", "weak") else (4 * w.dk if w.decay == "channel" else 0)
     per_th += 4 if w.beta else 0
     per_th += (w.dk + w.dv) * in_b if w.gates else 0
     state = w.dk * w.dv * 4 * (2 if w.s0_std > 0 else 1)
@@ -87,9 +86,11 @@ def algorithmic_flops(w):
     return f * chunks * w.B * w.H
 
 
-FWD_SOURCES = ("gdn_tc.cu", "gdn_tc_common.cuh", "sm100.cuh", "gdn_internal.cuh")
-DECODE_PROFILE = os.path.join(ROOT, "profiles", "gdn_decode_recurrent_ncu.md")
+FWD_SOURCES = ("gdn_fused.cu", "gdn_tc_common.cuh", "sm100.cuh", "gdn_internal.cuh")
+SPLIT_SOURCES = ("gdn_tc.cu", "gdn_tc_common.cuh", "sm100.cuh", "gdn_internal.cuh")
+SIMT_SOURCES = ("gdn_simt.cu", "gdn_internal.cuh")
 DECODE_SOURCES = ("gdn_recurrent.cu", "gdn_internal.cuh")
+COUNTERS = os.path.join(ROOT, "profiles", "counters.json")
 
 
 def kernel_source_sha(files=None):
@@ -102,25 +103,20 @@ def kernel_source_sha(files=None):
     return h.hexdigest()[:16]
 
 
-def profile_traffic(kernel_name, path=PROFILE, files=FWD_SOURCES):
-    """dram read+write bytes per launch from a committed ncu summary, if it was
-    taken on the current kernel sources."""
-    if not os.path.exists(path):
+def profile_traffic(key, files, units=None):
+    """DRAM read+write bytes per launch for ``key`` (kernel@workload) from the
+    committed counter file, if its capture was taken on the current kernel
+    sources.  A capture taken on a smaller case is scaled by ``units`` (the
+    launch's units over the captured units) when given."""
+    if not os.path.exists(COUNTERS):
         return None
-    txt = open(path).read()
-    m_sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", txt)
-    m_k = re.search(rf"traffic_bytes_per_launch\[{re.escape(kernel_name)}\]:\s*([0-9.e+]+)", txt)
-    if not (m_sha and m_k) or m_sha.group(1) != kernel_source_sha(files):
+    d = json.load(open(COUNTERS)).get(key)
+    if not d or d.get("kernel_source_sha") != kernel_source_sha(files):
         return None
-    return float(m_k.group(1))
-
-
-def mode_text(args):
-    if args.mode == "neumann":
-        return f"masked Neumann inverse N={args.N}"
-    if args.mode == "residual":
-        return f"masked Neumann inverse N={args.N} + {args.S} residual terms"
-    return "exact inverse"
+    t = float(d["traffic_bytes_per_launch"])
+    if units is not None and d.get("units"):
+        t *= units / float(d["units"])
+    return t
 
 
 def max_over_ranks(ms, world, device=None):
@@ -317,7 +313,59 @@ def measure_e2e(host_in, run, steps, dev, barrier=None):
 
 # ------------------------------------------------------------ our arm (GPU)
 
-def run_gpu(args, rank, world, local_rank):
+WORKLOAD_METRICS = {
+    "gdn_bf16": METRIC,
+    "plain_fp32": "tokens/s (fwd, fp32 plain delta rule, H=1, d=64, T=256) on 1 B200",
+    "long_context": "tokens/s (fwd, bf16, H=16, d=128, T=65536, S0 carried, S_T returned) and % of roofline on 1 B200",
+    "neumann": "tokens/s (fwd, bf16, H=16, d=128, T=4096, truncated Neumann inverse) and % of roofline on 1 B200",
+    "precond_two_gate": "tokens/s (fwd, bf16, preconditioned two-gate rule, H=16, d=128, T=4096) and % of roofline on 1 B200",
+}
+KERNEL_NAMES = {1: "simt_chunk_kernel", 2: "fused_kernel", 3: "recurrent_kernel", 4: "keyside_kernel+chain_kernel"}
+KERNEL_SOURCES = {1: SIMT_SOURCES, 2: FWD_SOURCES, 3: DECODE_SOURCES, 4: SPLIT_SOURCES}
+
+
+def forward_runs(args):
+    """(workload name, overrides) of every line this invocation prints."""
+    name = args.workload
+    if name == "neumann":
+        return [(name, dict(chunk=c, mode="neumann", neumann_N=n)) for c in (64, 128) for n in (2, 3, 4)]
+    over = {}
+    if args.mode != "exact" and name == "gdn_bf16":
+        over = dict(mode=args.mode, neumann_N=args.N)
+    return [(name, over)]
+
+
+def workload_text(w, mode, N, S, o_name):
+    inv = {"exact": "exact inverse", "neumann": f"masked Neumann inverse N={N}",
+           "residual": f"masked Neumann inverse N={N} + {S} residual terms"}[mode]
+    extra = []
+    if w.s0_std > 0:
+        extra.append(f"S0~N(0,{w.s0_std}^2)")
+    if w.gates:
+        extra.append("erase/write gates, per-channel decay, preconditioned write key")
+    return (f"{w.name}: B={w.B} H={w.H} T={w.T} dk={w.dk} dv={w.dv} chunk={w.chunk} {inv}"
+            + (", " + ", ".join(extra) if extra else "") + f", o {o_name}")
+
+
+_ORACLE_CACHE = {}
+
+
+def oracle_reference(w, x):
+    """fp64 oracle output (o, S_T) of the whole workload (cached per workload shape)."""
+    import oracle
+    key = (w.name, w.B, w.H, w.T, w.dk, w.dv)
+    if key not in _ORACLE_CACHE:
+        _ORACLE_CACHE[key] = oracle.gated_delta_fwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"],
+                                                    nthreads=len(os.sched_getaffinity(0)))
+    return _ORACLE_CACHE[key]
+
+
+def max_rel_rms(got, ref):
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    return float(np.abs(got - ref).max() / rms), float(np.sqrt(np.mean((got - ref) ** 2)) / rms)
+
+
+def forward_line(args, rank, world, local_rank, name, over, timed_steps):
     import torch
     import torch.distributed as dist
     import chunked_gated_delta_14_b200 as gdn
@@ -325,25 +373,35 @@ def run_gpu(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = workload(WORKLOAD, **({"B": args.batch} if args.batch else {}))
+    kw = dict(over)
+    if args.batch:
+        kw["B"] = args.batch
+    w = workload(name, **kw)
+    mode = w.mode if name in ("neumann",) or "mode" in over else args.mode
+    N = w.neumann_N if "neumann_N" in over else args.N
     x = make_inputs(w, seed=rank)   # each rank its own batch
     d = {k: (None if v is None else v.to(dev)) for k, v in x.items()}
-    o = torch.empty((w.B, w.T, w.H, w.dv), device=dev, dtype=torch.bfloat16)
+    f32 = w.io == "f32"
+    o_dt = torch.float32 if f32 else torch.bfloat16
+    o = torch.empty((w.B, w.T, w.H, w.dv), device=dev, dtype=o_dt)
     S_T = torch.empty((w.B, w.H, w.dk, w.dv), device=dev, dtype=torch.float32)
     stream = torch.cuda.current_stream(dev)
     ptr = lambda t: None if t is None else t.data_ptr()
-    a = gdn.make_args(B=w.B, T=w.T, H=w.H, dk=w.dk, dv=w.dv, chunk=w.chunk, io_dtype=1,
-                      o_dtype=1, q=ptr(d["q"]), k=ptr(d["k"]), v=ptr(d["v"]),
-                      alpha=ptr(d["alpha"]), beta=ptr(d["beta"]), S0=None, o=o.data_ptr(),
-                      S_T=S_T.data_ptr(), mode={"exact": 0, "neumann": 1, "residual": 2}[args.mode],
-                      neumann_N=args.N, residual_S=args.S, kernel=0)
+    general = w.gates or w.precond or w.decay == "channel"
+    a = gdn.make_args(B=w.B, T=w.T, H=w.H, dk=w.dk, dv=w.dv, chunk=w.chunk, io_dtype=0 if f32 else 1,
+                      o_dtype=0 if f32 else 1, q=ptr(d["q"]), k=ptr(d["k"]), v=ptr(d["v"]),
+                      alpha=ptr(d["alpha"]), alpha_per_channel=int(w.decay == "channel"),
+                      beta=ptr(d["beta"]), erase=ptr(d["erase"]), write=ptr(d["write"]),
+                      precond=int(bool(w.precond)), S0=ptr(d["S0"]), o=o.data_ptr(),
+                      S_T=S_T.data_ptr(), mode={"exact": 0, "neumann": 1, "residual": 2}[mode],
+                      neumann_N=N, residual_S=args.S, kernel=0)
     ws = gdn.workspace_for(a, dev)
     if ws is not None:
         a.workspace = ws.data_ptr()
         a.workspace_bytes = ws.numel()
     kernel_id = gdn.select_kernel(a)
-    kernel_name = {1: "simt_chunk_kernel", 2: "keyside_kernel+chain_kernel"}.get(kernel_id, "?")
-    launches_per_call = 2 if kernel_id == 2 else 1
+    kernel_name = KERNEL_NAMES.get(kernel_id, "?")
+    launches_per_call = 2 if kernel_id == 4 else 1
     sh = stream.cuda_stream
 
     def step():
@@ -352,6 +410,18 @@ def run_gpu(args, rank, world, local_rank):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    steps = timed_steps
+    if steps is None:
+        # a line other than the headline: about two seconds of timed calls
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        steps = int(min(args.steps, max(3, 2000.0 / max(t0.elapsed_time(t1), 1e-3))))
+        if world > 1:
+            steps = int(max_over_ranks(steps, world, dev))
 
     clocks = ClockSampler(local_rank)
     if rank == 0:
@@ -364,7 +434,7 @@ def run_gpu(args, rank, world, local_rank):
     e1 = torch.cuda.Event(enable_timing=True)
     t_wall0 = time.time()
     e0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
@@ -375,12 +445,13 @@ def run_gpu(args, rank, world, local_rank):
     clocks.mark(t_wall0, t_wall1)
     time.sleep(0.3)
     clocks.stop()
+    gdn.device_check(sh)
 
-    ms_step = ms / args.steps
+    ms_step = ms / steps
     tokens_step = w.B * w.T
-    value = job_throughput(tokens_step, world, args.steps, ms)
+    value = job_throughput(tokens_step, world, steps, ms)
 
-    # end to end through the public API: pinned host inputs -> device -> kernel -> host o
+    # end to end through the public API: pinned host inputs -> device -> kernel -> host o and S_T
     e2e = None
     if args.e2e_steps > 0:
         host = {k: v.pin_memory() for k, v in x.items() if v is not None}
@@ -388,34 +459,66 @@ def run_gpu(args, rank, world, local_rank):
         finals = [torch.empty_like(S_T) for _ in range(2)]
 
         def run(di, slot):
-            gdn.chunk_fwd(di["q"], di["k"], di["v"], di.get("alpha"), di.get("beta"), chunk=w.chunk,
-                          o_dtype=torch.bfloat16, out=outs[slot], mode=args.mode, N=args.N, S=args.S,
-                          S_T=finals[slot])
-            return {"o": outs[slot]}
+            gdn.chunk_fwd(di["q"], di["k"], di["v"], di.get("alpha"), di.get("beta"), erase=di.get("erase"),
+                          write=di.get("write"), precond=int(bool(w.precond)), S0=di.get("S0"), chunk=w.chunk,
+                          o_dtype=o_dt, out=outs[slot], mode=mode, N=N, S=args.S, S_T=finals[slot])
+            return {"o": outs[slot], "S_T": finals[slot]}
 
-        ems, h2d, d2h, how = measure_e2e(host, run, args.e2e_steps, dev,
-                                         barrier=dist.barrier if world > 1 else None)
+        n_e2e = args.e2e_steps if timed_steps is not None else max(2, min(args.e2e_steps, steps))
+        if world > 1:
+            # every rank takes the same collective steps: no fallback that one rank alone could take
+            ems, h2d, d2h = pipelined_e2e(host, run, n_e2e, dev, barrier=dist.barrier)
+            how = "uploads, compute and readbacks on three streams, two input slots"
+        else:
+            ems, h2d, d2h, how = measure_e2e(host, run, n_e2e, dev)
         ems = max_over_ranks(ems, world, dev)
         e2e = dict(value=job_throughput(tokens_step, world, 1, ems), unit=UNIT,
                    h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h), ms_per_step=ems,
                    pipeline=how)
 
     pk = peaks()
-    bytes_launch = algorithmic_bytes(w, o_bytes=2)
+    bytes_launch = algorithmic_bytes(w, o_bytes=4 if f32 else 2)
     achieved = bytes_launch / (ms_step / 1e3) / 1e9
     flops = algorithmic_flops(w)
+    traffic = profile_traffic(f"{kernel_name}@{name}", KERNEL_SOURCES.get(kernel_id, ()), units=w.B)
     roof = dict(bound="hbm", achieved=achieved, peak=pk["hbm_gbs"], unit="GB/s",
-                frac=achieved / pk["hbm_gbs"], traffic=profile_traffic(kernel_name),
+                frac=achieved / pk["hbm_gbs"], traffic=traffic,
                 peak_source=pk["source"] + " (burst copy bandwidth)",
                 algorithmic_bytes_per_launch=bytes_launch,
                 tensor_tflops=flops / (ms_step / 1e3) / 1e12,
                 tensor_frac_of_bf16_peak=flops / (ms_step / 1e3) / 1e12 / pk["bf16_tflops"],
                 roofline_ms=max(bytes_launch / (pk["hbm_gbs"] * 1e9),
                                 flops / (pk["bf16_tflops"] * 1e12)) * 1e3)
+    if name == "plain_fp32":
+        roof["note"] = "0.3 MB per call: launch-latency bound, the HBM fraction is only reported"
 
     clk = clocks.summary() if rank == 0 else dict(sm_max_mhz=None)
+    accuracy = None
+    if mode == "neumann" and rank == 0 and world == 1 and not general:
+        # the truncated series against exact inversion (same kernel family, exact mode)
+        # and against the fp64 oracle, on this whole workload
+        step()
+        torch.cuda.synchronize()
+        o_n = o.double().cpu().numpy()
+        s_n = S_T.double().cpu().numpy()
+        a.mode, a.neumann_N = 0, 0
+        step()
+        torch.cuda.synchronize()
+        o_x = o.double().cpu().numpy()
+        s_x = S_T.double().cpu().numpy()
+        o_ref, s_ref = oracle_reference(w, x)
+        m_o, r_o = max_rel_rms(o_n, o_x)
+        m_s, r_s = max_rel_rms(s_n, s_x)
+        mo_o, ro_o = max_rel_rms(o_n, o_ref)
+        mo_s, ro_s = max_rel_rms(s_n, s_ref)
+        accuracy = dict(
+            vs_exact=dict(o_max_rel_rms=m_o, o_rms_rel=r_o, S_T_max_rel_rms=m_s, S_T_rms_rel=r_s,
+                          exact_kernel=kernel_name),
+            vs_oracle=dict(o_max_rel_rms=mo_o, o_rms_rel=ro_o, S_T_max_rel_rms=mo_s, S_T_rms_rel=ro_s),
+            tolerance="bf16 bar: max|err| <= 2e-2 * rms(oracle) on o and S_T (o read back in bf16 here)")
+
     backward = None
-    if args.bwd_steps > 0:
+    if name == "gdn_bf16" and args.bwd_steps > 0 and world == 1:
         try:
             backward = backward_side_measure(w, x, rank, world, dev, args.bwd_steps, 3, clk["sm_max_mhz"])
         except Exception as e:   # the forward line is printed either way, with the reason
@@ -426,23 +529,35 @@ def run_gpu(args, rank, world, local_rank):
         cpu = cpu_baseline(w, x, budget_s=args.cpu_budget)
 
     if rank == 0:
-        line = dict(metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps,
+        line = dict(metric=WORKLOAD_METRICS[name], value=value, unit=UNIT, n_gpus=world, steps=steps,
                     warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True,
-                    scaling="weak", vs_baseline=None, dtype="bf16",
-                    compute="bf16 q/k/v in HBM; fp16 tensor-core operands, fp32 accumulate and state",
+                    scaling="weak", vs_baseline=None, dtype="f32" if f32 else "bf16",
+                    compute=("fp32 CUDA cores" if kernel_id == 1 else
+                             "bf16 q/k/v in HBM; fp16 tensor-core operands, fp32 accumulate and state"),
                     data="synthetic (seeded; Gated DeltaNet layer shapes)",
-                    config=dict(workload=f"{WORKLOAD}: B={w.B} H={w.H} T={w.T} dk={w.dk} "
-                                f"dv={w.dv} chunk={w.chunk} {mode_text(args)}, o bf16",
+                    config=dict(workload=workload_text(w, mode, N, args.S, "fp32" if f32 else "bf16"),
                                 global_batch=w.B * world, seq_len=w.T,
                                 parallelism=f"independent batch per GPU x{world}",
                                 l2=(f"no flush: inputs+outputs {bytes_launch / 1e6:.0f} MB per step > 126 MB L2"
                                     if bytes_launch > 126e6 else
-                                    f"no flush: {bytes_launch / 1e6:.0f} MB per step (fits L2; profiler case)"),
+                                    f"no flush: {bytes_launch / 1e6:.1f} MB per step (fits L2)"),
                                 kernel=kernel_name),
                     clocks=clk,
-                    e2e=e2e, gpu_launches=args.steps * launches_per_call, roofline=roof,
-                    cpu_baseline=cpu, backward=backward)
+                    e2e=e2e, gpu_launches=steps * launches_per_call, roofline=roof,
+                    cpu_baseline=cpu)
+        if accuracy is not None:
+            line["accuracy"] = accuracy
+        if backward is not None:
+            line["backward"] = backward
+        if world > 1:
+            line["note"] = "multi-rank run: the backward object is measured in single-GPU runs only"
         print(json.dumps(line), flush=True)
+
+
+def run_gpu(args, rank, world, local_rank):
+    for i, (name, over) in enumerate(forward_runs(args)):
+        headline = name == "gdn_bf16"
+        forward_line(args, rank, world, local_rank, name, over, args.steps if headline else None)
 
 
 DECODE_METRIC = "decode tokens/s (bf16, H=16, d=128, one token per sequence, state in place) and % of HBM roofline on 1 B200"
@@ -531,9 +646,7 @@ def run_decode(args, rank, world, local_rank):
     pk = peaks()
     bytes_step = decode_bytes(w)
     achieved = bytes_step / (ms_step / 1e3) / 1e9
-    traffic = profile_traffic("recurrent_kernel", DECODE_PROFILE, DECODE_SOURCES)
-    if traffic is not None:
-        traffic *= w.B / 128            # the summary is taken at B = 128; traffic scales with B
+    traffic = profile_traffic("recurrent_kernel@decode", DECODE_SOURCES, units=w.B)
     roof = dict(bound="hbm", achieved=achieved, peak=pk["hbm_gbs"], unit="GB/s",
                 frac=achieved / pk["hbm_gbs"], traffic=traffic,
                 peak_source=pk["source"] + " (burst copy bandwidth)",
@@ -569,7 +682,6 @@ def run_decode(args, rank, world, local_rank):
 
 BWD_METRIC = "backward tokens/s (bf16 in, fp32 gradients, H=16, d=128, T=4096) and % of fp32 roofline on 1 B200"
 BWD_SOURCES = ("gdn_bwd.cu", "gdn_bwd_kernels.cuh", "gdn_bwd_params.cuh")
-BWD_PROFILE = os.path.join(ROOT, "profiles", "gdn_bwd_gdn_bf16_ncu.md")
 
 
 def fp32_alu_peak_tflops(sm_mhz=1965.0):
@@ -629,8 +741,7 @@ def bwd_roofline(w, ms_step, sm_max_mhz):
     achieved = flops / (ms_step / 1e3) / 1e12
     nbytes = bwd_bytes(w)
     return dict(bound="alu", achieved=achieved, peak=alu_peak, unit="TFLOP/s", frac=achieved / alu_peak,
-                traffic=profile_traffic("bwd_prep_kernel+bwd_state_fwd_kernel+bwd_state_rev_kernel+bwd_grad_kernel",
-                                        BWD_PROFILE, BWD_SOURCES),
+                traffic=profile_traffic("backward@gdn_bf16", BWD_SOURCES, units=w.B),
                 peak_source="derived: 148 SMs x 128 fp32 lanes x 2 flops x max SM clock",
                 algorithmic_flops_per_launch=flops, algorithmic_bytes_per_launch=nbytes,
                 hbm_gbs=nbytes / (ms_step / 1e3) / 1e9, hbm_frac=nbytes / (ms_step / 1e3) / 1e9 / pk["hbm_gbs"],
@@ -777,10 +888,16 @@ def cpu_baseline(w, x, budget_s=12.0):
     done_th = 0
     t0 = time.time()
     b = 0
+    two_gate = w.gates or w.precond or w.decay == "channel"
     while True:
         sl = lambda t: None if t is None else t[b:b + 1]
-        oracle.gated_delta_fwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["alpha"]),
-                               sl(x["beta"]), sl(x["S0"]), nthreads=cores)
+        if two_gate:
+            oracle.precond_two_gate_fwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["alpha"]), sl(x["erase"]),
+                                        sl(x["write"]), precond=int(bool(w.precond)), h0=sl(x["S0"]),
+                                        nthreads=cores)
+        else:
+            oracle.gated_delta_fwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["alpha"]),
+                                   sl(x["beta"]), sl(x["S0"]), nthreads=cores)
         done_th += w.T * H
         b = (b + 1) % w.B
         if time.time() - t0 >= budget_s:
@@ -788,7 +905,7 @@ def cpu_baseline(w, x, budget_s=12.0):
     el = time.time() - t0
     return dict(value=done_th / H / el, unit=UNIT, cores=cores, kind="oracle",
                 sample=f"{done_th // (w.T * H)} x (batch row of {H} heads x {w.T} tokens) "
-                       f"of {WORKLOAD}, fp64 C oracle, {el:.1f} s")
+                       f"of {w.name}, fp64 C oracle, {el:.1f} s")
 
 
 # ------------------------------------------------- reference arm (the oracle)
@@ -798,7 +915,9 @@ def run_reference(args, rank, world):
         return
     import oracle
     from chunked_gated_delta_14_b200.inputs import make_inputs, workload
-    w = workload(WORKLOAD, **({"B": args.batch} if args.batch else {}))
+    name = args.workload
+    w = workload(name, **({"B": args.batch} if args.batch else {}))
+    two_gate = w.gates or w.precond or w.decay == "channel"
     x = make_inputs(w)
     cores = len(os.sched_getaffinity(0))
     # per-step sample: a prefix of one (batch, head) row group sized so that
@@ -808,14 +927,21 @@ def run_reference(args, rank, world):
     probe_T = 256
     t0 = time.time()
     sl = lambda t, b, n: None if t is None else t[b:b + 1, :n].contiguous()
-    oracle.gated_delta_fwd(sl(x["q"], 0, probe_T), sl(x["k"], 0, probe_T), sl(x["v"], 0, probe_T),
-                           sl(x["alpha"], 0, probe_T), sl(x["beta"], 0, probe_T), nthreads=cores)
+    def run_oracle(b, n):
+        if two_gate:
+            oracle.precond_two_gate_fwd(sl(x["q"], b, n), sl(x["k"], b, n), sl(x["v"], b, n),
+                                        sl(x["alpha"], b, n), sl(x["erase"], b, n), sl(x["write"], b, n),
+                                        precond=int(bool(w.precond)), h0=x["S0"][b:b + 1] if x["S0"] is not None
+                                        else None, nthreads=cores)
+        else:
+            oracle.gated_delta_fwd(sl(x["q"], b, n), sl(x["k"], b, n), sl(x["v"], b, n), sl(x["alpha"], b, n),
+                                   sl(x["beta"], b, n), x["S0"][b:b + 1] if x["S0"] is not None else None,
+                                   nthreads=cores)
+    run_oracle(0, probe_T)
     rate = probe_T / max(time.time() - t0, 1e-6)           # tokens (all heads) per second
     Ts = int(min(w.T, max(16, rate * per_step_s)))
     def step(i):
-        b = i % w.B
-        oracle.gated_delta_fwd(sl(x["q"], b, Ts), sl(x["k"], b, Ts), sl(x["v"], b, Ts),
-                               sl(x["alpha"], b, Ts), sl(x["beta"], b, Ts), nthreads=cores)
+        run_oracle(i % w.B, Ts)
     for i in range(args.warmup):
         step(i)
     t0 = time.perf_counter()
@@ -823,13 +949,13 @@ def run_reference(args, rank, world):
         step(i)
     el = time.perf_counter() - t0
     value = Ts * args.steps / el
-    sample = f"tokens [0,{Ts}) of one batch row (all {w.H} heads) of {WORKLOAD} per step"
-    line = dict(impl="reference", metric=METRIC, value=value, unit=UNIT, n_gpus=world,
+    sample = f"tokens [0,{Ts}) of one batch row (all {w.H} heads) of {name} per step"
+    line = dict(impl="reference", metric=WORKLOAD_METRICS[name], value=value, unit=UNIT, n_gpus=world,
                 steps=args.steps, warmup=args.warmup, ms_per_step=el / args.steps * 1e3,
                 higher_is_better=True, scaling="weak", vs_baseline=None, dtype="f64",
                 data="synthetic (seeded; Gated DeltaNet layer shapes)",
-                config=dict(workload=f"{WORKLOAD}: B={w.B} H={w.H} T={w.T} dk={w.dk} "
-                            f"dv={w.dv} chunk={w.chunk} {mode_text(args)}, o bf16",
+                config=dict(workload=workload_text(w, "exact" if name != "neumann" else "neumann",
+                                                   w.neumann_N, args.S, "fp32" if w.io == "f32" else "bf16"),
                             global_batch=w.B, seq_len=w.T,
                             parallelism="CPU oracle, rank 0 only"),
                 cpu_baseline=dict(value=value, unit=UNIT, cores=cores, kind="oracle",
@@ -849,6 +975,10 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="replace the batch size B (profiler case)")
+    ap.add_argument("--workload", default="gdn_bf16", choices=sorted(WORKLOAD_METRICS),
+                    help="gdn_bf16 (the headline, default), plain_fp32, long_context, neumann "
+                         "(one line per chunk 64/128 x N 2/3/4 with its error against exact inversion "
+                         "and the oracle) or precond_two_gate")
     ap.add_argument("--mode", default="exact", choices=["exact", "neumann", "residual"],
                     help="inverse: exact (the headline workload), masked Neumann series "
                          "(order --N), or the series with --S residual-correction terms")

@@ -78,7 +78,7 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
                         a->workspace};
     for (const void *x : al)
         if (x && !aligned16(x)) return fail(GDN_ERR_ALIGNMENT, "pointers must be 16-byte aligned");
-    if (a->kernel < GDN_KERNEL_AUTO || a->kernel > GDN_KERNEL_RECURRENT)
+    if (a->kernel < GDN_KERNEL_AUTO || a->kernel > GDN_KERNEL_TC_SPLIT)
         return fail(GDN_ERR_INVALID_ARG, "kernel %d unknown", a->kernel);
     if (a->dv_split < 0 || (a->dv_split > 0 && (a->dv % a->dv_split != 0 || a->dv / a->dv_split < 16)))
         return fail(GDN_ERR_INVALID_ARG, "dv_split must divide dv into slices of >= 16 columns");
@@ -101,13 +101,16 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
         // a few tokens (decode steps): the token recurrence beats any chunked form
         kern = GDN_KERNEL_RECURRENT;
     } else if (kern == GDN_KERNEL_AUTO) {
-        // tensor-core kernel when it supports the call, including the requested value split
+        // the fused tensor-core kernel, else the split one (including the requested
+        // value split), else the SIMT kernel
         gdn::FwdParams t = p;
         kern = GDN_KERNEL_SIMT;
-        if (gdn::tc_supports(t, &why)) {
+        if (a->dv_split <= 1 && gdn::fused_supports(t, &why)) {
+            kern = GDN_KERNEL_TC;
+        } else if (gdn::tc_supports(t, &why)) {
             t.slices = a->dv_split ? a->dv_split : gdn::tc_default_slices(t);
             t.dvs = t.dv / t.slices;
-            if (t.dv % t.slices == 0 && gdn::tc_supports(t, &why)) kern = GDN_KERNEL_TC;
+            if (t.dv % t.slices == 0 && gdn::tc_supports(t, &why)) kern = GDN_KERNEL_TC_SPLIT;
         }
     }
     if (kern == GDN_KERNEL_RECURRENT) {
@@ -116,18 +119,24 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
         p.slices = p.dv / 32;
         p.dvs = 32;
     } else if (kern == GDN_KERNEL_TC) {
+        if (a->dv_split > 1) return fail(GDN_ERR_UNSUPPORTED, "fused tensor-core kernel: dv_split must be 0 or 1");
+        if (!gdn::fused_supports(p, &why))
+            return fail(GDN_ERR_UNSUPPORTED, "fused tensor-core kernel: %s", why);
+        p.slices = 1;
+        p.dvs = p.dv;
+    } else if (kern == GDN_KERNEL_TC_SPLIT) {
         if (!gdn::tc_supports(p, &why))
-            return fail(GDN_ERR_UNSUPPORTED, "tensor-core kernel: %s", why);
+            return fail(GDN_ERR_UNSUPPORTED, "split tensor-core kernels: %s", why);
         p.slices = a->dv_split ? a->dv_split : gdn::tc_default_slices(p);
         if (p.dv % p.slices) return fail(GDN_ERR_UNSUPPORTED, "dv_split does not divide dv");
         p.dvs = p.dv / p.slices;
         if (!gdn::tc_supports(p, &why))
-            return fail(GDN_ERR_UNSUPPORTED, "tensor-core kernel: %s", why);
+            return fail(GDN_ERR_UNSUPPORTED, "split tensor-core kernels: %s", why);
     } else {
         if (p.mode == GDN_INV_NEUMANN_RESIDUAL)
             return fail(GDN_ERR_UNSUPPORTED,
-                        "residual correction runs on the tensor-core kernel only (bf16 q/k/v, scalar "
-                        "decay, chunk 64, dk 128)%s%s", why[0] ? ": " : "", why);
+                        "residual correction runs on the split tensor-core kernels only (bf16 q/k/v, "
+                        "scalar decay, chunk 64, dk 128)%s%s", why[0] ? ": " : "", why);
         // SIMT: widest value slice that fits shared memory, at least
         // ~one block per SM where the problem allows it.
         int slices = a->dv_split;
@@ -247,7 +256,7 @@ uint64_t gdn_workspace_bytes(const gdn_fwd_args *args) {
     int kern = 0;
     if (resolve(args, &p, &kern) != GDN_OK) return 0;
     g_msg[0] = 0;
-    return kern == GDN_KERNEL_TC ? (uint64_t)gdn::tc_workspace_bytes(p) : 0;
+    return kern == GDN_KERNEL_TC_SPLIT ? (uint64_t)gdn::tc_workspace_bytes(p) : 0;
 }
 
 int32_t gdn_select_kernel(const gdn_fwd_args *args) {
@@ -263,7 +272,10 @@ gdn_status gdn_device_check(void *stream) {
     cudaError_t e = cudaSuccess;
     const unsigned int code = gdn::tc_read_and_clear_error(reinterpret_cast<cudaStream_t>(stream), &e);
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "device check: %s", cudaGetErrorString(e));
-    if (code) return fail(GDN_ERR_DEVICE_CHECK, "tensor-core kernel wait %u gave up", code);
+    const unsigned int fcode = gdn::fused_read_and_clear_error(&e);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "device check: %s", cudaGetErrorString(e));
+    if (code) return fail(GDN_ERR_DEVICE_CHECK, "split tensor-core kernel wait %u gave up", code);
+    if (fcode) return fail(GDN_ERR_DEVICE_CHECK, "fused tensor-core kernel wait %u gave up", fcode);
     g_msg[0] = 0;
     return GDN_OK;
 }
@@ -279,9 +291,11 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_args *args, void *stream) {
     cudaError_t e;
     const char *why = "";
     if (kern == GDN_KERNEL_TC) {
+        e = gdn::launch_fused(p, st, &why);
+    } else if (kern == GDN_KERNEL_TC_SPLIT) {
         const size_t need = gdn::tc_workspace_bytes(p);
         if (!args->workspace || args->workspace_bytes < need)
-            return fail(GDN_ERR_INVALID_ARG, "tensor-core kernel needs a workspace of %zu bytes (got %llu)",
+            return fail(GDN_ERR_INVALID_ARG, "split tensor-core kernels need a workspace of %zu bytes (got %llu)",
                         need, (unsigned long long)args->workspace_bytes);
         e = gdn::launch_tc(p, args->workspace, st, &why);
     } else if (kern == GDN_KERNEL_RECURRENT) {
@@ -291,7 +305,8 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_args *args, void *stream) {
     }
     if (e != cudaSuccess)
         return fail(GDN_ERR_CUDA, "%s launch: %s %s",
-                    kern == GDN_KERNEL_TC ? "tc" : (kern == GDN_KERNEL_RECURRENT ? "recurrent" : "simt"),
+                    kern == GDN_KERNEL_TC ? "tc" : kern == GDN_KERNEL_TC_SPLIT ? "tc_split"
+                    : (kern == GDN_KERNEL_RECURRENT ? "recurrent" : "simt"),
                     cudaGetErrorString(e), why);
     g_msg[0] = 0;
     return GDN_OK;
@@ -301,12 +316,15 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_args *args, void *stream) {
 // workspace: nothing is allocated.  The array's device address is looked up
 // once per device, with that device current, on the first call made there.
 gdn_status gdn_chunk_fwd_static_scratch(const gdn_fwd_args *args, void *stream) {
+    if (!args) return fail(GDN_ERR_INVALID_ARG, "args is NULL");
+    if (args->kernel != GDN_KERNEL_AUTO && args->kernel != GDN_KERNEL_TC && args->kernel != GDN_KERNEL_TC_SPLIT)
+        return fail(GDN_ERR_UNSUPPORTED, "the fixed-scratch entry point runs the split tensor-core kernels only");
+    gdn_fwd_args a = *args;
+    a.kernel = GDN_KERNEL_TC_SPLIT;
     gdn::FwdParams p;
     int kern = 0;
-    gdn_status s = resolve(args, &p, &kern);
+    gdn_status s = resolve(&a, &p, &kern);
     if (s != GDN_OK) return s;
-    if (kern != GDN_KERNEL_TC)
-        return fail(GDN_ERR_UNSUPPORTED, "the fixed-scratch entry point runs the tensor-core kernel only");
     if (args->workspace || args->workspace_bytes)
         return fail(GDN_ERR_INVALID_ARG, "the fixed-scratch entry point takes no workspace (pass NULL, 0)");
     const size_t need = gdn::tc_workspace_bytes(p);
@@ -336,6 +354,28 @@ gdn_status gdn_chunk_fwd_static_scratch(const gdn_fwd_args *args, void *stream) 
     }
     const char *why = "";
     e = gdn::launch_tc(p, scratch, reinterpret_cast<cudaStream_t>(stream), &why);
+    if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "tc launch: %s %s", cudaGetErrorString(e), why);
+    g_msg[0] = 0;
+    return GDN_OK;
+}
+
+gdn_status gdn_debug_chunk_T(const gdn_fwd_args *args, int32_t b, int32_t h, int32_t n, float *T_out,
+                             void *stream) {
+    gdn::FwdParams p;
+    int kern = 0;
+    gdn_status s = resolve(args, &p, &kern);
+    if (s != GDN_OK) return s;
+    if (kern != GDN_KERNEL_TC)
+        return fail(GDN_ERR_UNSUPPORTED, "gdn_debug_chunk_T inspects the fused tensor-core kernel only "
+                                         "(bf16 q/k/v, scalar decay, chunk 64, dk = dv = 128)");
+    const int NC = (p.T + p.C - 1) / p.C;
+    if (b < 0 || b >= p.B || h < 0 || h >= p.H || n < 0 || n >= NC)
+        return fail(GDN_ERR_INVALID_ARG, "(b, h, n) = (%d, %d, %d) outside B = %d, H = %d, %d chunks", b, h, n,
+                    p.B, p.H, NC);
+    if (!T_out) return fail(GDN_ERR_INVALID_ARG, "T_out is NULL");
+    if (!aligned16(T_out)) return fail(GDN_ERR_ALIGNMENT, "T_out must be 16-byte aligned");
+    const char *why = "";
+    const cudaError_t e = gdn::launch_fused(p, reinterpret_cast<cudaStream_t>(stream), &why, T_out, b, h, n);
     if (e != cudaSuccess) return fail(GDN_ERR_CUDA, "tc launch: %s %s", cudaGetErrorString(e), why);
     g_msg[0] = 0;
     return GDN_OK;

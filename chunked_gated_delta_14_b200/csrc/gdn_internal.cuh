@@ -48,4 +48,12 @@ cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, 
 // Synchronise `stream`, return (and clear) the tensor-core kernel's error word.
 unsigned int tc_read_and_clear_error(cudaStream_t stream, cudaError_t *err);
 
+// Fused tensor-core kernel: one 2-CTA cluster per (batch, head), no workspace.
+bool fused_supports(const FwdParams &p, const char **why);
+// dbg_T (device, 64 x 64 fp32) receives the T of chunk dbg_n of (dbg_b, dbg_h) when non-NULL.
+cudaError_t launch_fused(const FwdParams &p, cudaStream_t stream, const char **why, float *dbg_T = nullptr,
+                         int dbg_b = 0, int dbg_h = 0, int dbg_n = 0);
+// Return (and clear) the fused kernel's error word; the caller has synchronised.
+unsigned int fused_read_and_clear_error(cudaError_t *err);
+
 }  // namespace gdn

@@ -778,14 +778,14 @@ cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, 
         *why = "(tensor map encoding failed)";
         return cudaErrorInvalidValue;
     }
-    static bool attr_done = false;
-    if (!attr_done) {
+    // The attribute belongs to the current device: set it on every launch (cheap)
+    // rather than behind a process-wide flag that a second device would not share.
+    {
         cudaError_t e = cudaFuncSetAttribute(keyside_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)K1_SMEM_RES);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K2_SMEM);
         if (e != cudaSuccess) return e;
-        attr_done = true;
     }
     K1Params k1;
     k1.B = p.B; k1.T = p.T; k1.H = p.H; k1.NC = NC;

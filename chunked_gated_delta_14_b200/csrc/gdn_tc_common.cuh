@@ -253,6 +253,143 @@ __device__ __forceinline__ void invert_neumann(const float *Lb, float *Tb, float
     named_bar(bar_id, 256);
 }
 
+// ---------------------------------------------------- 128-thread inverses
+// The fused kernel inverts with one group of four warps per chunk (two groups
+// work on alternate chunks), so these take 128 threads.
+
+// T = (I + L)^-1 = (I - A)^-1 for strictly lower L (64 x 64 fp32, row stride
+// LSTR) by 128 threads t: the 16 x 16 diagonal blocks by forward substitution
+// (one column per thread), then T21 = -T22 L21 T11 merges 16 -> 32 -> 64.
+// Tb's entries above the diagonal blocks must be zero on entry (they are
+// never written).  Yb: 1024 floats of scratch.  Ends with a barrier.
+__device__ __forceinline__ void invert_exact128(const float *Lb, float *Tb, float *Yb, int t, int bar_id) {
+    if (t < 64) {
+        const int c = t, base = c & ~15, jc = c & 15;
+        float acc[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) acc[r] = (r == jc) ? 1.f : 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float xi = acc[i];
+#pragma unroll
+            for (int r = i + 1; r < 16; ++r) acc[r] -= Lb[(base + r) * LSTR + base + i] * xi;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Tb[(base + r) * LSTR + c] = acc[r];
+    }
+    named_bar(bar_id, 128);
+    {
+        // 16 -> 32 for both 32-blocks: Y = L21 T11, then T21 = -T22 Y; thread (row, 4 columns)
+        const int pr = t >> 6, rr = (t >> 2) & 15, c0 = (t & 3) * 4;
+        const int b0 = 32 * pr, b1 = b0 + 16;
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
+        const float *Lr = Lb + (b1 + rr) * LSTR + b0;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float l = Lr[k];
+            const float4 v = *reinterpret_cast<const float4 *>(Tb + (b0 + k) * LSTR + b0 + c0);
+            y[0] += l * v.x; y[1] += l * v.y; y[2] += l * v.z; y[3] += l * v.w;
+        }
+        *reinterpret_cast<float4 *>(Yb + pr * 256 + rr * 16 + c0) = make_float4(y[0], y[1], y[2], y[3]);
+        named_bar(bar_id, 128);
+        float z[4] = {0.f, 0.f, 0.f, 0.f};
+        const float *Tr = Tb + (b1 + rr) * LSTR + b1;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float a = Tr[k];
+            const float4 v = *reinterpret_cast<const float4 *>(Yb + pr * 256 + k * 16 + c0);
+            z[0] += a * v.x; z[1] += a * v.y; z[2] += a * v.z; z[3] += a * v.w;
+        }
+        *reinterpret_cast<float4 *>(Tb + (b1 + rr) * LSTR + b0 + c0) = make_float4(-z[0], -z[1], -z[2], -z[3]);
+    }
+    named_bar(bar_id, 128);
+    {
+        // 32 -> 64: Y = L10 T00, T10 = -T11 Y; thread (two rows, 4 columns)
+        const int rr = 2 * (t >> 3), c0 = (t & 7) * 4;
+        float y0[4] = {0.f, 0.f, 0.f, 0.f}, y1[4] = {0.f, 0.f, 0.f, 0.f};
+        const float *L0 = Lb + (32 + rr) * LSTR, *L1 = L0 + LSTR;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+            const float4 v = *reinterpret_cast<const float4 *>(Tb + k * LSTR + c0);
+            const float l0 = L0[k], l1 = L1[k];
+            y0[0] += l0 * v.x; y0[1] += l0 * v.y; y0[2] += l0 * v.z; y0[3] += l0 * v.w;
+            y1[0] += l1 * v.x; y1[1] += l1 * v.y; y1[2] += l1 * v.z; y1[3] += l1 * v.w;
+        }
+        *reinterpret_cast<float4 *>(Yb + rr * 32 + c0) = make_float4(y0[0], y0[1], y0[2], y0[3]);
+        *reinterpret_cast<float4 *>(Yb + (rr + 1) * 32 + c0) = make_float4(y1[0], y1[1], y1[2], y1[3]);
+        named_bar(bar_id, 128);
+        float z0[4] = {0.f, 0.f, 0.f, 0.f}, z1[4] = {0.f, 0.f, 0.f, 0.f};
+        const float *T0 = Tb + (32 + rr) * LSTR + 32, *T1 = T0 + LSTR;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+            const float4 v = *reinterpret_cast<const float4 *>(Yb + k * 32 + c0);
+            const float a0 = T0[k], a1 = T1[k];
+            z0[0] += a0 * v.x; z0[1] += a0 * v.y; z0[2] += a0 * v.z; z0[3] += a0 * v.w;
+            z1[0] += a1 * v.x; z1[1] += a1 * v.y; z1[2] += a1 * v.z; z1[3] += a1 * v.w;
+        }
+        *reinterpret_cast<float4 *>(Tb + (32 + rr) * LSTR + c0) = make_float4(-z0[0], -z0[1], -z0[2], -z0[3]);
+        *reinterpret_cast<float4 *>(Tb + (33 + rr) * LSTR + c0) = make_float4(-z1[0], -z1[1], -z1[2], -z1[3]);
+    }
+    named_bar(bar_id, 128);
+}
+
+// Masked truncated Neumann series M^(N) (.) sum_{n<=N} A^n with A = -L by 128
+// threads, Horner's rule T <- M (.) (I + A T).  N <= 15: on the band the mask
+// leaves, rows 16 wide in Yb (2 x 1024 floats).  N > 15: dense 64 x 64
+// steps with Yb (4096 floats, row stride 64) as the second buffer.  Writes
+// the dense T (zeros outside the band) to Tb (row stride LSTR).  Ends with a
+// barrier.
+__device__ __forceinline__ void invert_neumann128(const float *Lb, float *Tb, float *Yb, int t, int N,
+                                                  int bar_id) {
+    if (N <= 15) {
+        const int i = t >> 1, dq = t & 1;
+        float *cur = Yb, *nxt = Yb + 1024;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) cur[i * 16 + dq + 2 * u] = (dq + 2 * u == 0) ? 1.f : 0.f;
+        named_bar(bar_id, 128);
+        for (int step = 0; step < N; ++step) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int d = dq + 2 * u, j = i - d;
+                float val = 0.f;
+                if (j >= 0 && d <= N) {
+                    val = (d == 0) ? 1.f : 0.f;
+                    for (int k = j; k < i; ++k) val -= Lb[i * LSTR + k] * cur[k * 16 + (k - j)];
+                }
+                nxt[i * 16 + d] = val;
+            }
+            named_bar(bar_id, 128);
+            float *sw = cur; cur = nxt; nxt = sw;
+        }
+#pragma unroll 4
+        for (int qq = 0; qq < 32; ++qq) {
+            const int e = t + 128 * qq, ii = e >> 6, j = e & 63, d = ii - j;
+            Tb[ii * LSTR + j] = (d >= 0 && d <= N) ? cur[ii * 16 + d] : 0.f;
+        }
+        named_bar(bar_id, 128);
+        return;
+    }
+    // dense: thread t owns row i = t >> 1, columns [32 (t & 1), + 32)
+    const int i = t >> 1, j0 = 32 * (t & 1);
+    for (int jj = 0; jj < 32; ++jj) Tb[i * LSTR + j0 + jj] = (i == j0 + jj) ? 1.f : 0.f;
+    named_bar(bar_id, 128);
+    for (int step = 0; step < N; ++step) {
+        // Yb <- M (.) (I - L Tb), then copy back into Tb
+        for (int jj = 0; jj < 32; ++jj) {
+            const int j = j0 + jj, d = i - j;
+            float val = 0.f;
+            if (d >= 0 && d <= N) {
+                val = (d == 0) ? 1.f : 0.f;
+                for (int k = j; k < i; ++k) val -= Lb[i * LSTR + k] * Tb[k * LSTR + j];
+            }
+            Yb[i * 64 + j] = val;
+        }
+        named_bar(bar_id, 128);
+        for (int jj = 0; jj < 32; ++jj) Tb[i * LSTR + j0 + jj] = Yb[i * 64 + j0 + jj];
+        named_bar(bar_id, 128);
+    }
+}
+
 // Z = A + sgn * (X Y) for lower-triangular 64 x 64 fp32 matrices (row stride
 // LSTR, zeros above the diagonal stored).  A is the identity (a_kind 1),
 // I - Y (a_kind 2) or zero (a_kind 0).  256 threads, one 4 x 4 tile each;

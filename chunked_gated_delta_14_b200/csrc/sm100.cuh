@@ -88,6 +88,95 @@ __device__ __forceinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity, v
     }
 }
 
+// ------------------------------------------------------------------ clusters
+// A thread-block cluster of 2 CTAs shares its shared memory (DSMEM): a CTA
+// maps a local shared address to the peer's copy with mapa, arrives on the
+// peer's mbarriers and copies tiles into the peer's shared memory with the
+// bulk-copy engine (no multicast).
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// shared::cluster address of the same offset in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+// Whole-cluster barrier (every thread of both CTAs; warps converged).  The
+// release/acquire pair orders each CTA's earlier shared-memory writes, mbarrier
+// initialisations included, before the peer's later accesses.
+__device__ __forceinline__ void cluster_sync_all() {
+    __syncwarp();
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Arrive on an mbarrier of the peer CTA (address from mapa_shared).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster)
+                 : "memory");
+}
+
+// Arrive on the peer's mbarrier and raise its expected transaction bytes.
+__device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t bar_cluster, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;"
+                 ::"r"(bar_cluster), "r"(bytes)
+                 : "memory");
+}
+
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
+// from this CTA's shared memory into the peer's; completion is signalled on
+// the peer's mbarrier as transaction bytes.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, const void *src, uint32_t bytes,
+                                                  uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst_cluster), "r"(smem_u32(src)), "r"(bytes), "r"(bar_cluster)
+        : "memory");
+}
+
+// Store a 32-bit word into the peer's shared memory.
+__device__ __forceinline__ void st_peer_u32(uint32_t addr_cluster, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr_cluster), "r"(v) : "memory");
+}
+
+// try_wait whose acquire is cluster-scoped: for phases completed by the peer
+// CTA (a remote arrive or a bulk copy from its shared memory).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait on a phase the peer CTA completes (see mbar_wait).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, volatile int *abort, int code,
+                                                  uint64_t limit_cycles) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = clock64();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i)
+            if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (*abort) return false;
+        if (static_cast<uint64_t>(clock64()) - t0 > limit_cycles) {
+            atomicCAS(const_cast<int *>(abort), 0, code);
+            return false;
+        }
+        __nanosleep(32);
+    }
+}
+
 // Bounded wait that ignores the abort flag (drains copies or MMAs still in
 // flight before a block releases its resources on an error path).
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, uint64_t limit_cycles) {

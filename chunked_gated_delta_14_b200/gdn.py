@@ -27,13 +27,13 @@ GDN_ERR_FAULT_INJECTED = 6
 
 GDN_F32, GDN_BF16 = 0, 1
 GDN_INV_EXACT, GDN_INV_NEUMANN, GDN_INV_NEUMANN_RESIDUAL = 0, 1, 2
-KERNELS = {"auto": 0, "simt": 1, "tc": 2, "recurrent": 3}
+KERNELS = {"auto": 0, "simt": 1, "tc": 2, "recurrent": 3, "tc_split": 4}
 KERNEL_NAMES = {v: k for k, v in KERNELS.items()}
 MODES = {"exact": GDN_INV_EXACT, "neumann": GDN_INV_NEUMANN, "residual": GDN_INV_NEUMANN_RESIDUAL}
 
 EXPORTS = ("gdn_chunk_fwd", "gdn_select_kernel", "gdn_workspace_bytes", "gdn_device_check",
            "gdn_status_string", "gdn_last_error", "gdn_abi_version", "gdn_chunk_fwd_static_scratch",
-           "gdn_chunk_bwd", "gdn_bwd_workspace_bytes")
+           "gdn_chunk_bwd", "gdn_bwd_workspace_bytes", "gdn_debug_chunk_T")
 STATIC_SCRATCH_BYTES = 24 << 20   # GDN_STATIC_SCRATCH_BYTES
 
 
@@ -112,6 +112,9 @@ def lib() -> ctypes.CDLL:
             L.gdn_chunk_bwd.restype = ctypes.c_int
             L.gdn_bwd_workspace_bytes.argtypes = [ctypes.POINTER(BwdArgs)]
             L.gdn_bwd_workspace_bytes.restype = ctypes.c_uint64
+            L.gdn_debug_chunk_T.argtypes = [ctypes.POINTER(FwdArgs), ctypes.c_int32, ctypes.c_int32,
+                                            ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]
+            L.gdn_debug_chunk_T.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -168,7 +171,8 @@ def make_args(**kw) -> FwdArgs:
 
 
 def select_kernel(args: FwdArgs) -> int:
-    """Kernel gdn_chunk_fwd would launch (1 simt, 2 tc) or -status. Host only."""
+    """Kernel gdn_chunk_fwd would launch (1 simt, 2 fused tc, 3 recurrent, 4 split tc)
+    or -status. Host only."""
     return int(lib().gdn_select_kernel(ctypes.byref(args)))
 
 
@@ -180,6 +184,16 @@ def workspace_bytes(args: FwdArgs) -> int:
 _ws_cache = {}
 
 
+def clear_workspace_cache(device: Optional[torch.device] = None) -> None:
+    """Drop the cached workspaces (all devices, or one), e.g. when a stream that
+    was used for calls is retired.  Each cached buffer holds its bytes until it
+    is dropped: about 96 MiB for a split-kernel forward of the 4 x 16 x 4096
+    benchmark shape, 1.4 GB for its backward; the fused forward needs none."""
+    for key in list(_ws_cache):
+        if device is None or (key[0] == device.type and key[1] == device.index):
+            del _ws_cache[key]
+
+
 def workspace_for(args, device: torch.device,
                   stream: Optional[torch.cuda.Stream] = None) -> Optional[torch.Tensor]:
     """A cached device buffer of at least the workspace ``args`` needs, or None.
@@ -187,7 +201,8 @@ def workspace_for(args, device: torch.device,
     One buffer per (device, stream, direction): calls ordered on one stream
     reuse it, calls on different streams never share one, and forward
     (FwdArgs) and backward (BwdArgs) calls keep separate buffers.  ``stream``
-    is the stream the call will run on (default: the device's current one)."""
+    is the stream the call will run on (default: the device's current one).
+    Buffers stay cached until ``clear_workspace_cache``."""
     bwd = isinstance(args, BwdArgs)
     need = bwd_workspace_bytes(args) if bwd else workspace_bytes(args)
     if need == 0:
@@ -218,6 +233,34 @@ def call_static_scratch(args: FwdArgs, stream: Optional[int] = None) -> None:
     s = lib().gdn_chunk_fwd_static_scratch(ctypes.byref(args), ctypes.c_void_p(stream or 0))
     if s != GDN_OK:
         raise GDNError(s, last_error())
+
+
+def call_debug_chunk_T(args: FwdArgs, b: int, h: int, n: int, T_out: int,
+                       stream: Optional[int] = None) -> None:
+    """Raw gdn_debug_chunk_T call (T_out: device pointer of 4096 floats); raises
+    GDNError on a non-OK status."""
+    s = lib().gdn_debug_chunk_T(ctypes.byref(args), int(b), int(h), int(n), ctypes.c_void_p(T_out),
+                                ctypes.c_void_p(stream or 0))
+    if s != GDN_OK:
+        raise GDNError(s, last_error())
+
+
+def debug_chunk_T(q, k, v, alpha=None, beta=None, *, b: int = 0, h: int = 0, n: int = 0,
+                  mode: str = "exact", N: int = 3, S0=None) -> torch.Tensor:
+    """The 64 x 64 fp32 T the fused kernel forms for chunk n of sequence (b, h)
+    (exact inverse or masked Neumann series), from one gdn_debug_chunk_T call."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = torch.empty((B, T, H, dv), device=q.device, dtype=torch.float32)
+    S_T = torch.empty((B, H, dk, dv), device=q.device, dtype=torch.float32)
+    T_out = torch.full((64, 64), float("nan"), device=q.device, dtype=torch.float32)
+    args = make_args(B=B, T=T, H=H, dk=dk, dv=dv, chunk=64, io_dtype=_dtype_code(q.dtype), o_dtype=GDN_F32,
+                     q=_ptr(q), k=_ptr(k), v=_ptr(v), alpha=_ptr(alpha), beta=_ptr(beta), S0=_ptr(S0),
+                     o=_ptr(o), S_T=_ptr(S_T), mode=MODES[mode], neumann_N=int(N), kernel=KERNELS["tc"])
+    stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        call_debug_chunk_T(args, b, h, n, T_out.data_ptr(), stream.cuda_stream)
+    return T_out
 
 
 def device_check(stream: Optional[int] = None) -> None:

@@ -46,10 +46,13 @@
  *
  * Ownership.  Every pointer is a DEVICE pointer owned by the caller, who
  * allocates inputs, outputs and the workspace.  The library allocates no
- * device memory and keeps no state between calls.  The tensor-core kernel
- * keeps, per chunk and head, T diag(beta), T diag(beta e^g) and the decayed
- * causal scores P (fp16, 24 KB) in the workspace between its two launches;
- * gdn_workspace_bytes() gives the size.
+ * device memory and keeps no state between calls.  The fused tensor-core
+ * kernel (GDN_KERNEL_TC) needs no workspace: its per-chunk inverses move
+ * between the two CTAs of a cluster through shared memory.  The split
+ * tensor-core kernels (GDN_KERNEL_TC_SPLIT) keep, per chunk and head,
+ * T diag(beta), T diag(beta e^g) and the decayed causal scores P (fp16,
+ * 24 KB) in the workspace between their two launches; gdn_workspace_bytes()
+ * gives the size.
  *
  * Execution and errors.  gdn_chunk_fwd validates its arguments on the host
  * and returns an error before launching anything (nothing is written) when
@@ -69,7 +72,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 5
+#define GDN_ABI_VERSION 6
 
 #if defined(__GNUC__)
 #define GDN_API __attribute__((visibility("default")))
@@ -99,12 +102,21 @@ typedef enum {
 } gdn_inv_mode;
 
 typedef enum {
-    GDN_KERNEL_AUTO = 0,        /* tensor-core kernel when it supports the call, else SIMT */
+    GDN_KERNEL_AUTO = 0,        /* the first of TC, TC_SPLIT, SIMT that supports the call
+                                   (RECURRENT for T <= 8) */
     GDN_KERNEL_SIMT = 1,        /* fp32 CUDA-core chunk kernel (all variants) */
-    GDN_KERNEL_TC = 2,          /* tcgen05/TMEM/TMA kernel (bf16 io, scalar decay, C = 64) */
-    GDN_KERNEL_RECURRENT = 3    /* token-by-token kernel for short sequences and decode steps
+    GDN_KERNEL_TC = 2,          /* fused tcgen05/TMEM/TMA kernel, one launch of 2-CTA
+                                   clusters per (batch, head): bf16 q/k/v, scalar decay,
+                                   C = 64, dk = dv = 128, exact or Neumann mode (any N).
+                                   Needs no workspace (gdn_workspace_bytes() is 0). */
+    GDN_KERNEL_RECURRENT = 3,   /* token-by-token kernel for short sequences and decode steps
                                    (scalar decay, exact mode, dk a multiple of 8, dv of 32);
                                    AUTO picks it for T <= 8 */
+    GDN_KERNEL_TC_SPLIT = 4     /* the tensor-core path as two launches (a key-side kernel
+                                   per chunk, then the state chain) with the per-chunk
+                                   inverses in a caller workspace: bf16 q/k/v, scalar decay,
+                                   C = 64, dk = 128, dv a multiple of 64, all three inverse
+                                   modes (Neumann N <= 15) */
 } gdn_kernel;
 
 typedef struct {
@@ -159,11 +171,30 @@ GDN_API int32_t gdn_select_kernel(const gdn_fwd_args *args);
 
 /* Synchronises `stream` (void* cudaStream_t), then reports and clears a
  * failure recorded on the device by the kernels' own checks: a bounded wait
- * inside the tensor-core kernel that gave up (after about two seconds) makes
+ * inside a tensor-core kernel that gave up (after about two seconds) makes
  * the block skip its remaining work and record an error code; this call then
  * returns GDN_ERR_DEVICE_CHECK.  GDN_ERR_CUDA if synchronising failed, else
  * GDN_OK. */
 GDN_API gdn_status gdn_device_check(void *stream);
+
+/* Inspection entry for tests: gdn_chunk_fwd on the fused tensor-core kernel
+ * (it writes o and S_T exactly as that call does) that also copies the
+ * 64 x 64 fp32 matrix T the kernel formed for chunk n of sequence (b, h)
+ * into T_out: T = (I - A)^-1 in GDN_INV_EXACT mode, the masked truncated
+ * Neumann series M^(N) (.) sum_{n<=N} A^n in GDN_INV_NEUMANN mode ("Quando o
+ * 'Bom o Suficiente' e Otimo ...", section "Declaracao do Problema" and
+ * section "Metodologia", items 1 and 2), as it stood before its rounding to
+ * fp16 for the WY products.  A = -L with L_ri = beta_r e^{g_r - g_i}
+ * (k_r . k_i), i < r, g the in-chunk cumulative log decay.
+ *
+ * T_out: DEVICE pointer, 4096 floats, 16-byte aligned, row-major (row = token
+ * row of the chunk), written on `stream`.  In a tail chunk of Cv < 64 tokens,
+ * rows and columns past Cv hold the identity.  Errors: GDN_ERR_INVALID_ARG for
+ * (b, h, n) outside the call or a NULL T_out; GDN_ERR_UNSUPPORTED unless the
+ * arguments select the fused kernel (kernel AUTO or TC); otherwise as
+ * gdn_chunk_fwd. */
+GDN_API gdn_status gdn_debug_chunk_T(const gdn_fwd_args *args, int32_t b, int32_t h, int32_t n, float *T_out,
+                                     void *stream);
 
 /* Static string for a status code. */
 GDN_API const char *gdn_status_string(gdn_status s);
@@ -237,8 +268,8 @@ GDN_API gdn_status gdn_chunk_bwd(const gdn_bwd_args *args, void *stream);
  * Host only. */
 GDN_API uint64_t gdn_bwd_workspace_bytes(const gdn_bwd_args *args);
 
-/* gdn_chunk_fwd on the tensor-core kernel, with a fixed scratch array inside
- * the library in place of args->workspace.  The pages have no counterpart:
+/* gdn_chunk_fwd on the split tensor-core kernels (GDN_KERNEL_TC_SPLIT), with
+ * a fixed scratch array inside the library in place of args->workspace.  The pages have no counterpart:
  * this is a calling convenience of this library, not a step of the method.
  *
  * For callers that cannot allocate device memory per call: a plain C host
@@ -248,8 +279,9 @@ GDN_API uint64_t gdn_bwd_workspace_bytes(const gdn_bwd_args *args);
  * nothing (no cudaMalloc, cudaFree or allocating library routine).
  *
  * Arguments as gdn_chunk_fwd, except: args->workspace must be NULL and
- * args->workspace_bytes 0; the arguments must select the tensor-core kernel
- * (kernel AUTO or TC with a supported shape), else GDN_ERR_UNSUPPORTED; and
+ * args->workspace_bytes 0; args->kernel must be AUTO, TC or TC_SPLIT and the
+ * shape one the split tensor-core kernels support, else GDN_ERR_UNSUPPORTED
+ * (whatever the kernel field, this entry point runs the split kernels); and
  * B * H * ceil(T / 64) * 24576 must be <= GDN_STATIC_SCRATCH_BYTES, else
  * GDN_ERR_INVALID_ARG with the needed size in gdn_last_error().  Nothing in
  * the scratch has to start at zero: the key-side kernel writes every entry

@@ -25,7 +25,7 @@ def declared_functions():
 
 def test_library_builds_and_loads():
     gbuild.build()
-    assert gdn.abi_version() == 5
+    assert gdn.abi_version() == 6
 
 
 def test_exports_every_declared_symbol():
@@ -65,6 +65,10 @@ def _args(**kw):
     (dict(precond=1, rho_eps=0.0), GDN_ERR_INVALID_ARG),
     (dict(q=0x10008), GDN_ERR_ALIGNMENT),
     (dict(kernel=9), GDN_ERR_INVALID_ARG),
+    (dict(kernel=2, dv=64), GDN_ERR_UNSUPPORTED),       # fused kernel: dk = dv = 128
+    (dict(kernel=2, dv_split=2), GDN_ERR_UNSUPPORTED),  # fused kernel holds the whole head
+    (dict(kernel=2, mode=2, neumann_N=3, residual_S=8), GDN_ERR_UNSUPPORTED),   # residual: split only
+    (dict(kernel=4, mode=1, neumann_N=16), GDN_ERR_UNSUPPORTED),               # split: N <= 15
     (dict(dv_split=3), GDN_ERR_INVALID_ARG),
     (dict(kernel=2, io_dtype=0), GDN_ERR_UNSUPPORTED),  # tensor cores need bf16 io
     (dict(alpha=0x70000, alpha_per_channel=1, chunk=128, kernel=1, dv_split=8),
@@ -99,7 +103,12 @@ def test_null_args_pointer():
 
 def test_valid_arguments_select_a_kernel():
     assert gdn.select_kernel(_args(kernel=1)) == 1
-    assert gdn.select_kernel(_args(mode=2, neumann_N=3, residual_S=8)) == 2   # residual: tensor cores
+    assert gdn.select_kernel(_args()) == 2                                     # fused tensor-core kernel
+    assert gdn.select_kernel(_args(mode=1, neumann_N=63)) == 2                 # any N on the fused kernel
+    assert gdn.select_kernel(_args(mode=2, neumann_N=3, residual_S=8)) == 4   # residual: split kernels
+    assert gdn.select_kernel(_args(dv=64)) == 4                                # dv 64: split kernels
+    assert gdn.select_kernel(_args(dv_split=2)) == 4                           # a value split: split kernels
+    assert gdn.select_kernel(_args(dv_split=1)) == 2
     assert gdn.select_kernel(_args(T=1)) == 3                                  # decode step
     assert gdn.select_kernel(_args(T=8, io_dtype=0, dk=64, dv=64)) == 3
     assert gdn.select_kernel(_args(T=9)) == 2                                  # chunked from T = 9
@@ -230,3 +239,16 @@ def test_ctypes_mirrors_match_the_c_structs(struct, mirror, tmp_path):
     assert ctypes.sizeof(mirror) == size
     for name, off in zip(fields, offsets):
         assert getattr(mirror, name).offset == off, name
+
+
+def test_debug_chunk_T_rejects_on_host():
+    """gdn_debug_chunk_T validates (b, h, n), T_out and the kernel before any launch."""
+    import ctypes
+    L = gdn.lib()
+    fake = 0x90000
+    for (b, h, n) in [(-1, 0, 0), (2, 0, 0), (0, 3, 0), (0, 0, 2)]:      # B=2, H=3, T=100: 2 chunks
+        assert L.gdn_debug_chunk_T(ctypes.byref(_args()), b, h, n, ctypes.c_void_p(fake), None) == GDN_ERR_INVALID_ARG
+    assert L.gdn_debug_chunk_T(ctypes.byref(_args()), 0, 0, 0, None, None) == GDN_ERR_INVALID_ARG
+    assert L.gdn_debug_chunk_T(ctypes.byref(_args()), 0, 0, 0, ctypes.c_void_p(fake + 8), None) == GDN_ERR_ALIGNMENT
+    assert L.gdn_debug_chunk_T(ctypes.byref(_args(kernel=1)), 0, 0, 0, ctypes.c_void_p(fake), None) == GDN_ERR_UNSUPPORTED
+    assert L.gdn_debug_chunk_T(ctypes.byref(_args(dv=64)), 0, 0, 0, ctypes.c_void_p(fake), None) == GDN_ERR_UNSUPPORTED

@@ -77,12 +77,15 @@ def fake_cuda(monkeypatch):
     monkeypatch.setattr(gmod, "call_bwd", bwd)
     monkeypatch.setattr(gdn, "call_bwd", bwd)
     monkeypatch.setattr(gmod, "_check", lambda *a, **k: None)
+    monkeypatch.setattr(gmod, "device_check", lambda *a, **k: None)
+    monkeypatch.setattr(gdn, "device_check", lambda *a, **k: None)
     return calls
 
 
 def _line(fn, **over):
     import bench
     args = types.SimpleNamespace(steps=2, warmup=3, e2e_steps=4, cpu_budget=0.2, no_cpu_baseline=False,
+                                 workload="gdn_bf16",
                                  batch=1, mode="exact", N=3, S=8, bwd_steps=2, ref_budget=1.0)
     for k, v in over.items():
         setattr(args, k, v)
@@ -90,6 +93,19 @@ def _line(fn, **over):
     with contextlib.redirect_stdout(buf):
         getattr(bench, fn)(args, 0, 1, 0)
     return json.loads(buf.getvalue().strip().splitlines()[-1])
+
+
+def _lines(fn, **over):
+    import bench
+    args = types.SimpleNamespace(steps=2, warmup=3, e2e_steps=4, cpu_budget=0.2, no_cpu_baseline=False,
+                                 workload="gdn_bf16", batch=1, mode="exact", N=3, S=8, bwd_steps=0,
+                                 ref_budget=1.0)
+    for k, v in over.items():
+        setattr(args, k, v)
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        getattr(bench, fn)(args, 0, 1, 0)
+    return [json.loads(x) for x in buf.getvalue().strip().splitlines() if x.startswith("{")]
 
 
 def _check_contract(line):
@@ -112,7 +128,7 @@ def _check_contract(line):
 def test_forward_line_with_backward_object(fake_cuda):
     line = _line("run_gpu")
     _check_contract(line)
-    assert line["roofline"]["bound"] == "hbm" and line["gpu_launches"] == 2 * 2
+    assert line["roofline"]["bound"] == "hbm" and line["gpu_launches"] == 2      # fused: one launch a step
     b = line["backward"]
     assert "error" not in b, b
     assert b["value"] > 0 and b["gpu_launches"] == 4 * 2 and b["roofline"]["bound"] == "alu"
@@ -128,7 +144,7 @@ def test_backward_line(fake_cuda):
 
 def test_backward_object_can_be_skipped(fake_cuda):
     line = _line("run_gpu", bwd_steps=0, no_cpu_baseline=True)
-    assert line["backward"] is None and line["cpu_baseline"] is None
+    assert line.get("backward") is None and line["cpu_baseline"] is None
 
 
 def test_decode_line(fake_cuda):
@@ -145,3 +161,38 @@ def test_e2e_falls_back_to_one_stream(fake_cuda, monkeypatch):
     monkeypatch.setattr(bench, "pipelined_e2e", broken)
     line = _line("run_gpu", bwd_steps=0, no_cpu_baseline=True)
     assert line["e2e"]["value"] > 0 and line["e2e"]["pipeline"].startswith("one stream")
+
+
+@pytest.mark.parametrize("name,kernel", [("plain_fp32", "simt_chunk_kernel"), ("long_context", "fused_kernel"),
+                                         ("precond_two_gate", "simt_chunk_kernel")])
+def test_other_workload_lines(fake_cuda, monkeypatch, name, kernel):
+    import bench
+    # the line's assembly only: a stand-in for the oracle timing of a whole long sequence
+    from chunked_gated_delta_14_b200 import inputs
+    monkeypatch.setattr(bench, "cpu_baseline", lambda w, x, budget_s=0: dict(
+        value=1.0, unit="tokens/s", cores=1, kind="oracle", sample="stand-in"))
+    if name == "long_context":   # the same line at a shorter length: host memory and time
+        monkeypatch.setitem(inputs.WORKLOADS, name, inputs.WORKLOADS[name].replace(T=2048))
+    (line,) = _lines("run_gpu", workload=name, cpu_budget=0.05)
+    _check_contract(line)
+    assert line["config"]["kernel"] == kernel
+    assert line["config"]["workload"].startswith(name)
+    assert line["metric"] != _line("run_gpu", bwd_steps=0, no_cpu_baseline=True)["metric"]
+
+
+def test_neumann_sweep_lines(fake_cuda, monkeypatch):
+    """One line per chunk 64 / 128 and N 2 / 3 / 4, each with its error against
+    exact inversion and against the oracle."""
+    import bench
+    import numpy as np
+    monkeypatch.setattr(bench, "oracle_reference", lambda w, x: (
+        np.ones((w.B, w.T, w.H, w.dv)), np.ones((w.B, w.H, w.dk, w.dv))))
+    lines = _lines("run_gpu", workload="neumann", cpu_budget=0.05, e2e_steps=0, no_cpu_baseline=True)
+    assert len(lines) == 6
+    seen = set()
+    for ln in lines:
+        acc = ln["accuracy"]
+        assert set(acc) >= {"vs_exact", "vs_oracle", "tolerance"}
+        seen.add((ln["config"]["workload"].split("chunk=")[1].split()[0],
+                  ln["config"]["workload"].split("N=")[1].split(",")[0]))
+    assert seen == {(c, n) for c in ("64", "128") for n in ("2", "3", "4")}
