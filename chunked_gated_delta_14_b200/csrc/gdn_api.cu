@@ -101,17 +101,16 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
         // a few tokens (decode steps): the token recurrence beats any chunked form
         kern = GDN_KERNEL_RECURRENT;
     } else if (kern == GDN_KERNEL_AUTO) {
-        // the fused tensor-core kernel, else the split one (including the requested
-        // value split), else the SIMT kernel
+        // the split tensor-core kernels (the faster path on B200 at these shapes),
+        // else the fused one, else the SIMT kernel
         gdn::FwdParams t = p;
         kern = GDN_KERNEL_SIMT;
-        if (a->dv_split <= 1 && gdn::fused_supports(t, &why)) {
-            kern = GDN_KERNEL_TC;
-        } else if (gdn::tc_supports(t, &why)) {
+        if (gdn::tc_supports(t, &why)) {
             t.slices = a->dv_split ? a->dv_split : gdn::tc_default_slices(t);
             t.dvs = t.dv / t.slices;
             if (t.dv % t.slices == 0 && gdn::tc_supports(t, &why)) kern = GDN_KERNEL_TC_SPLIT;
         }
+        if (kern == GDN_KERNEL_SIMT && a->dv_split <= 1 && gdn::fused_supports(p, &why)) kern = GDN_KERNEL_TC;
     }
     if (kern == GDN_KERNEL_RECURRENT) {
         if (!gdn::recurrent_supports(p, &why))
@@ -361,9 +360,12 @@ gdn_status gdn_chunk_fwd_static_scratch(const gdn_fwd_args *args, void *stream) 
 
 gdn_status gdn_debug_chunk_T(const gdn_fwd_args *args, int32_t b, int32_t h, int32_t n, float *T_out,
                              void *stream) {
+    if (!args) return fail(GDN_ERR_INVALID_ARG, "args is NULL");
+    gdn_fwd_args a = *args;
+    if (a.kernel == GDN_KERNEL_AUTO) a.kernel = GDN_KERNEL_TC;   // this entry inspects the fused kernel
     gdn::FwdParams p;
     int kern = 0;
-    gdn_status s = resolve(args, &p, &kern);
+    gdn_status s = resolve(&a, &p, &kern);
     if (s != GDN_OK) return s;
     if (kern != GDN_KERNEL_TC)
         return fail(GDN_ERR_UNSUPPORTED, "gdn_debug_chunk_T inspects the fused tensor-core kernel only "

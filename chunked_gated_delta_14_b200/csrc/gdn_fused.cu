@@ -74,30 +74,36 @@ constexpr unsigned long long kWait = 4000000000ull;   // ~2 s at the boost clock
 
 // error codes (first one wins): key side 21.., chain side 41..
 enum {
-    E_K_QKFREE = 21, E_K_QK, E_K_GRAM, E_K_KFREE, E_K_W,
+    E_K_Q = 21, E_K_GRAM, E_K_KFREE, E_K_KRECV, E_K_INV, E_K_LFULL, E_K_LFREE, E_K_TFULL, E_K_TFREE,
     E_C_SFREE = 41, E_C_SFULL, E_C_KFULL, E_C_CVT, E_C_HREADY, E_C_HSTORED, E_C_DDONE, E_C_XDONE,
-    E_C_ZDONE, E_C_ODONE, E_C_XFREE
+    E_C_ZDONE, E_C_ODONE, E_C_XFREE, E_C_WDONE, E_C_WREADY
 };
 
 constexpr uint32_t IDESC_BF_KK = idesc_f16(128, 64, 1, 1, 0, 0);    // bf16 K-major x K-major, N 64
 constexpr uint32_t IDESC_KM128 = idesc_f16(128, 128, 0, 0, 0, 1);   // fp16 K-major x MN-major, N 128
-constexpr uint32_t IDESC_MM128 = idesc_f16(128, 128, 0, 0, 1, 1);   // fp16 MN-major x MN-major, N 128
+constexpr uint32_t IDESC_KM64 = idesc_f16(128, 64, 0, 0, 0, 1);     // fp16 K-major x MN-major, N 64
+constexpr uint32_t IDESC_MM64 = idesc_f16(128, 64, 0, 0, 1, 1);     // fp16 MN-major x MN-major, N 64
 
 constexpr uint32_t PARB = (sizeof(ChunkParams) + 15) & ~15u;
 constexpr uint32_t MAT = 64 * LSTR * 4;                 // one 64 x LSTR fp32 matrix
 
 // ------------------------------------------------ key CTA shared memory
-// stage g (chunks of parity g): [Q0 | K0 | Q1 | K1], 8 KB each (64 rows of one
-// 64-column box, 128-byte swizzle); send buffer g: [-W0 | -W1 | T diag(beta) | P].
+// stage st (chunks of parity st): [Q0 | K0 | Q1 | K1], 8 KB each (64 rows of one
+// 64-column box, 128-byte swizzle).  Send buffer sb (chunk m: sb = m % 3):
+// [T diag(beta e^g) | T diag(beta) | P], fp16.  L and T: fp32, two each.
 constexpr uint32_t K_QK = 0;
 constexpr uint32_t K_SND = 65536;
-constexpr uint32_t SND_MW0 = 0, SND_MW1 = 8192, SND_TB = 16384, SND_P = 24576;
-constexpr uint32_t K_L = 131072;
+constexpr uint32_t SNDB = 24576;
+constexpr uint32_t SND_TBG = 0, SND_TB = 8192, SND_P = 16384;
+constexpr uint32_t K_L = K_SND + 3 * SNDB;
 constexpr uint32_t K_T = K_L + 2 * MAT;
 constexpr uint32_t K_PAR = K_T + 2 * MAT;
-constexpr uint32_t K_BAR = K_PAR + 2 * PARB;
-enum { KB_QKFULL = 0, KB_QKFREE = 2, KB_GRAM = 4, KB_WDONE = 6, KB_KFREE = 8, KB_N = 10 };
-constexpr uint32_t K_MISC = K_BAR + KB_N * 8;          // tmem slot, abort flag, group sync slots
+constexpr uint32_t K_BAR = K_PAR + 3 * PARB;
+enum {
+    KB_QFULL = 0, KB_GRAM = 2, KB_LFULL = 4, KB_LFREE = 6, KB_TFULL = 8, KB_TFREE = 10, KB_INV = 12,
+    KB_KFREE = 13, KB_KRECV = 15, KB_N = 18
+};
+constexpr uint32_t K_MISC = K_BAR + KB_N * 8;          // tmem slot, abort flag, stage sync slots
 constexpr uint32_t K_END = K_MISC + 64;
 
 // ---------------------------------------------- chain CTA shared memory
@@ -113,9 +119,12 @@ constexpr uint32_t C_SLOT = 0;
 constexpr uint32_t C_HS = 2 * SLOT;                    // h16: two 64-column boxes of 128 rows
 constexpr uint32_t C_PAR = C_HS + 32768;               // gate ring of 4
 constexpr uint32_t C_BAR = C_PAR + 4 * PARB;
+// per value half j (columns 64 j .. 64 j + 63): XDONE / ODONE [buffer][half],
+// HREADY / HSTORED / DDONE / ZDONE [half]
 enum {
-    CB_SFULL = 0, CB_SFREE = 2, CB_KFULL = 4, CB_CVT = 6, CB_XDONE = 8, CB_ODONE = 11, CB_XFREE = 14,
-    CB_HREADY = 17, CB_HSTORED = 18, CB_DDONE = 19, CB_ZDONE = 20, CB_N = 21
+    CB_SFULL = 0, CB_SFREE = 2, CB_KFULL = 4, CB_CVT = 6, CB_XDONE = 8, CB_ODONE = 12, CB_XFREE = 16,
+    CB_HREADY = 18, CB_HSTORED = 20, CB_DDONE = 22, CB_ZDONE = 24, CB_WDONE = 26, CB_WREADY = 27, CB_UDONE = 28,
+    CB_N = 29
 };
 constexpr uint32_t C_MISC = C_BAR + CB_N * 8;          // tmem slot, abort, sent counts, sync slots
 constexpr uint32_t C_END = C_MISC + 64;
@@ -123,12 +132,12 @@ constexpr uint32_t C_END = C_MISC + 64;
 constexpr uint32_t SMEM_USED = (K_END > C_END ? K_END : C_END);
 constexpr uint32_t FUSED_SMEM = SMEM_USED + 1024;      // + base alignment slack
 static_assert(FUSED_SMEM <= 232448, "shared memory budget of one sm_100 block");
-static_assert(K_SND + 2 * 32768 <= K_L, "key layout");
+static_assert(K_SND + 3 * SNDB <= K_L && (K_L & 15) == 0 && (K_BAR & 7) == 0, "key layout");
 static_assert((C_HS & 1023) == 0 && (K_L & 15) == 0, "alignment");
 
-// chain TMEM: h (128 columns) and three X buffers; key TMEM: Gram x 2, W x 2
-constexpr uint32_t TM_H = 0, TM_X = 128;
-constexpr uint32_t TM_G = 0, TM_W = 128;
+// chain TMEM: h (128 columns), two X buffers, W; key TMEM: Gram x 2, inverse merge
+constexpr uint32_t TM_H = 0, TM_X = 128, TM_WC = 384;
+constexpr uint32_t TM_G = 0, TM_INV = 128;
 
 struct FusedParams {
     int B, T, H, NC;
@@ -186,96 +195,86 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 // =================================================================== key CTA
+// A pipeline of three warp groups, one chunk in each stage:
+//   A (warps 0..3):   q, k tiles (TMA), gate scan, [Q ; K] K^T (MMA), and from
+//                     it the decayed scores P (fp16, send buffer) and L (fp32)
+//   B (warps 4..11):  T = (I + L)^-1, or the masked truncated Neumann series
+//   C (warps 12..15): T diag(beta), T diag(beta e^g) (fp16), then the copy of
+//                     [T diag(beta e^g) | T diag(beta) | P] into the chain CTA
+// Stages hand over through mbarriers: A -> B (L full / free), B -> C (T full /
+// free); a send buffer is reused once the chain CTA has received its copy.
 
 __device__ __forceinline__ void key_cta(uint8_t *sm, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                                         const FusedParams &p, int b, int h, uint32_t tmem, volatile int *abort) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int NC = p.NC;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + K_BAR);
+    auto Lbuf = [&](int m) { return reinterpret_cast<float *>(sm + K_L + (m & 1) * MAT); };
+    auto Tbuf = [&](int m) { return reinterpret_cast<float *>(sm + K_T + (m & 1) * MAT); };
+    auto par_of = [&](int m) { return reinterpret_cast<ChunkParams *>(sm + K_PAR + (m % 3) * PARB); };
+    auto snd_of = [&](int m) { return sm + K_SND + (m % 3) * SNDB; };
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer: q, k
-        if (lane == 0) {
+    if (warp < 4) {
+        // ------------------------------------------------------------ stage A
+        const int sp = warp;
+        const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
+        GroupSync gs{reinterpret_cast<volatile int *>(sm + K_MISC + 16), 0, 1, 128, tid == 0, warp == 0};
+        const bool leader = (tid == 0);
+        auto load_qk = [&](int m) {
+            uint64_t *fb = &bars[KB_QFULL + (m & 1)];
+            uint8_t *st = sm + K_QK + (m & 1) * 32768;
+            mbar_arrive_expect_tx(fb, 32768);
+            tma_load_4d(st, tm_q, fb, 0, h, m * C, b);
+            tma_load_4d(st + 8192, tm_k, fb, 0, h, m * C, b);
+            tma_load_4d(st + 16384, tm_q, fb, 64, h, m * C, b);
+            tma_load_4d(st + 24576, tm_k, fb, 64, h, m * C, b);
+        };
+        int q_out[2] = {-1, -1};                   // leader: phases of loads not yet consumed
+        if (leader) {
             tma_prefetch_desc(tm_q);
             tma_prefetch_desc(tm_k);
-            int issued = 0;
-            for (int m = 0; m < NC; ++m) {
-                const int g = m & 1;
-                if (m >= 2 && !mbar_wait(&bars[KB_QKFREE + g], ((m - 2) >> 1) & 1, abort, E_K_QKFREE, kWait))
-                    break;
-                uint64_t *fb = &bars[KB_QKFULL + g];
-                uint8_t *st = sm + K_QK + g * 32768;
-                mbar_arrive_expect_tx(fb, 32768);
-                const int t0 = m * C;
-                tma_load_4d(st, tm_q, fb, 0, h, t0, b);
-                tma_load_4d(st + 8192, tm_k, fb, 0, h, t0, b);
-                tma_load_4d(st + 16384, tm_q, fb, 64, h, t0, b);
-                tma_load_4d(st + 24576, tm_k, fb, 64, h, t0, b);
-                issued = m + 1;
+            for (int m = 0; m < 2 && m < NC; ++m) { load_qk(m); q_out[m] = 0; }
+        }
+        int pend = -1, pend_par = 0;
+        for (int m = 0; m < NC; ++m) {
+            const int st = m & 1;
+            uint8_t *qk = sm + K_QK + st * 32768;
+            const uint32_t tG = tmem + TM_G + 64 * st;
+            ChunkParams *par = par_of(m);
+            uint8_t *snd = snd_of(m);
+            float *Lb = Lbuf(m);
+            // the send buffer (and the gate slot) of chunk m - 3 are free once the
+            // chain CTA has received that chunk
+            if (m >= 3 && !group_wait(gs, &bars[KB_KRECV + m % 3], ((m - 3) / 3) & 1, abort, E_K_KRECV, true))
+                break;
+            if (warp == 1) {
+                float a0, a1, b0, b1;
+                tc::fetch_gates(p.alpha, p.beta, b, p.T, p.H, h, m * C, lane, true, a0, a1, b0, b1);
+                tc::scan_gates(par, a0, a1, b0, b1, lane, min(C, p.T - m * C));
             }
-            for (int m = issued - 2 < 0 ? 0 : issued - 2; m < issued; ++m)
-                mbar_wait_drain(&bars[KB_QKFULL + (m & 1)], (m >> 1) & 1, kWait);
-        }
-        __syncwarp();
-        return;
-    }
-    if (warp < 4 || warp >= 12) return;
-
-    // ------------------------------------------ two groups, alternate chunks
-    const int g = (warp - 4) >> 2;
-    const int gt = tid - 128 - 128 * g;          // 0..127
-    const int sp = warp & 3;                      // TMEM sub-partition of this warp
-    const uint32_t lane_base = (uint32_t)(32 * sp) << 16;
-    GroupSync gs{reinterpret_cast<volatile int *>(sm + K_MISC + 16 + 8 * g), 0, 1 + g, 128, gt == 0, sp == 0};
-    const bool leader = (gt == 0);
-    ChunkParams *par = reinterpret_cast<ChunkParams *>(sm + K_PAR + g * PARB);
-    float *Lb = reinterpret_cast<float *>(sm + K_L + g * MAT);
-    float *Tb = reinterpret_cast<float *>(sm + K_T + g * MAT);
-    uint8_t *qk = sm + K_QK + g * 32768;
-    uint8_t *snd = sm + K_SND + g * 32768;
-    float *Yb = reinterpret_cast<float *>(snd);   // inverse scratch: the -W region, written later
-    const uint32_t tG = tmem + TM_G + 64 * g, tW = tmem + TM_W + 128 * g;
-    const uint32_t peer_kfull = mapa_shared(smem_u32(sm + C_BAR + 8 * (CB_KFULL + g)), 1);
-    const uint32_t peer_slot = mapa_shared(smem_u32(sm + C_SLOT + g * SLOT), 1);
-
-    // T's blocks above the diagonal stay zero for the whole sequence
-    for (int i = gt; i < 64 * LSTR; i += 128) Tb[i] = 0.f;
-    named_bar(gs.id, 128);
-
-    int sent = 0;
-    int pend = -1, pend_par = 0;                  // leader: last commit not yet known complete
-    for (int m = g; m < NC; m += 2) {
-        const int it = m >> 1;
-        const uint32_t ph = it & 1;
-        const int t0 = m * C;
-        if (sp == 1) {
-            float a0, a1, b0, b1;
-            tc::fetch_gates(p.alpha, p.beta, b, p.T, p.H, h, t0, lane, true, a0, a1, b0, b1);
-            tc::scan_gates(par, a0, a1, b0, b1, lane, min(C, p.T - t0));
-        }
-        if (!group_wait(gs, &bars[KB_QKFULL + g], ph, abort, E_K_QK, false)) break;
-        if (leader) {
-            tc_fence_after();
-            const uint32_t a0 = smem_u32(qk);
+            if (!group_wait(gs, &bars[KB_QFULL + st], (m >> 1) & 1, abort, E_K_Q, false)) break;
+            if (leader) {
+                q_out[st] = -1;
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(qk);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                umma_f16_ss(tG, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(a0 + off + 8192, 16, 1024),
-                            IDESC_BF_KK, kk > 0);
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    umma_f16_ss(tG, sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(a0 + off + 8192, 16, 1024),
+                                IDESC_BF_KK, kk > 0);
+                }
+                umma_commit(&bars[KB_GRAM + st]);
+                pend = KB_GRAM + st; pend_par = (m >> 1) & 1;
             }
-            umma_commit(&bars[KB_GRAM + g]);
-            pend = KB_GRAM + g; pend_par = ph;
-        }
-        __syncwarp();
-        // the chain has consumed chunk m - 2: this group's send buffer (and the
-        // peer's slot g) may be written again
-        if (m >= 2 && !group_wait(gs, &bars[KB_KFREE + g], (it - 1) & 1, abort, E_K_KFREE, true)) break;
-        if (!group_wait(gs, &bars[KB_GRAM + g], ph, abort, E_K_GRAM, false)) break;
-        pend = -1;
-        tc_fence_after();
-        {
-            // sub-partitions 0, 1: rows of Q K^T -> P (fp16, swizzled, send buffer)
-            // sub-partitions 2, 3: rows of K K^T -> L (fp32)
+            __syncwarp();
+            // stage B has read L of chunk m - 2
+            if (m >= 2 && !group_wait(gs, &bars[KB_LFREE + st], ((m - 2) >> 1) & 1, abort, E_K_LFREE, false))
+                break;
+            if (!group_wait(gs, &bars[KB_GRAM + st], (m >> 1) & 1, abort, E_K_GRAM, false)) break;
+            pend = -1;
+            if (leader && m + 2 < NC) { load_qk(m + 2); q_out[st] = ((m + 2) >> 1) & 1; }   // q, k are read
+            tc_fence_after();
+            // sub-partitions 0, 1: rows of Q K^T -> P; sub-partitions 2, 3: rows of K K^T -> L
             const int rb = sp & 1, r = 32 * rb + lane;
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
@@ -317,30 +316,147 @@ __device__ __forceinline__ void key_cta(uint8_t *sm, const CUtensorMap *tm_q, co
                     }
                 }
             }
+            fence_proxy_async_smem();     // P is read by the bulk copy
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[KB_LFULL + st]);
         }
-        // K -> fp16 in place (the Gram MMA has read it): B operand of the W MMA
+        if (leader) {
+            // error path: nothing of this stage may still run when the block exits
+            if (pend >= 0) mbar_wait_drain(&bars[pend], pend_par, kWait);
+            for (int i = 0; i < 2; ++i)
+                if (q_out[i] >= 0) mbar_wait_drain(&bars[KB_QFULL + i], q_out[i], kWait);
+        }
+        __syncwarp();
+        return;
+    }
+
+    if (warp < 12) {
+        // ------------------------------------------------------------ stage B
+        const int bt = tid - 128;                 // 0..255
+        const int wl = warp - 4;
+        GroupSync gs{reinterpret_cast<volatile int *>(sm + K_MISC + 24), 0, 2, 256, bt == 0, wl == 0};
+        const bool leader = (bt == 0);
+        const uint32_t tI = tmem + TM_INV;
+        // T's blocks above the diagonal stay zero for the whole sequence
+        for (int i = bt; i < 2 * 64 * LSTR; i += 256) reinterpret_cast<float *>(sm + K_T)[i] = 0.f;
+        named_bar(gs.id, 256);
+        int pend = -1, pend_par = 0;
+        for (int m = 0; m < NC; ++m) {
+            const int lb = m & 1;
+            float *Lb = Lbuf(m), *Tb = Tbuf(m);
+            uint8_t *snd = snd_of(m);
+            float *Yb = reinterpret_cast<float *>(snd + SND_TBG);   // scratch until stage C writes there
+            if (!group_wait(gs, &bars[KB_LFULL + lb], (m >> 1) & 1, abort, E_K_LFULL, false)) break;
+            if (m >= 2 && !group_wait(gs, &bars[KB_TFREE + lb], ((m - 2) >> 1) & 1, abort, E_K_TFREE, false))
+                break;
+            bool fail = false;
+            if (!p.neumann) {
+                // the 16 x 16 diagonal blocks and the 16 -> 32 merges on the CUDA
+                // cores, the 32 -> 64 merge T10 = -T11 L10 T00 as two MMAs (fp16
+                // operands, fp32 accumulate; the rounding stays below that of the
+                // fp16 copies of T that the WY products use)
+                tc::invert_exact_to32(Lb, Tb, Yb, bt, gs.id);
+                uint8_t *a1 = snd + SND_TBG, *b1 = snd + SND_TBG + 4096;   // rows: L10 | T rows 0..31
+                uint8_t *a2 = snd + SND_TB, *b2 = snd + SND_TB + 4096;     // rows: -T11 | Y
+                {
+                    const int u = bt & 127, r = u >> 2, j = u & 3;
+                    const float *src = bt < 128 ? Lb + (32 + r) * LSTR + 8 * j : Tb + (32 + r) * LSTR + 32 + 8 * j;
+                    const float sg = bt < 128 ? 1.f : -1.f;
+                    const float4 x0 = *reinterpret_cast<const float4 *>(src);
+                    const float4 x1 = *reinterpret_cast<const float4 *>(src + 4);
+                    *reinterpret_cast<uint4 *>((bt < 128 ? a1 : a2) + sw128_off(r, j)) =
+                        make_uint4(pack_h2(sg * x0.x, sg * x0.y), pack_h2(sg * x0.z, sg * x0.w),
+                                   pack_h2(sg * x1.x, sg * x1.y), pack_h2(sg * x1.z, sg * x1.w));
+                    const int k = bt >> 3, jb = bt & 7;
+                    const float *tr = Tb + k * LSTR + 8 * jb;
+                    const float4 y0 = *reinterpret_cast<const float4 *>(tr);
+                    const float4 y1 = *reinterpret_cast<const float4 *>(tr + 4);
+                    *reinterpret_cast<uint4 *>(b1 + sw128_off(k, jb)) =
+                        make_uint4(pack_h2(y0.x, y0.y), pack_h2(y0.z, y0.w), pack_h2(y1.x, y1.y), pack_h2(y1.z, y1.w));
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar(gs.id, 256);
+#pragma unroll 1
+                for (int step = 0; step < 2 && !fail; ++step) {
+                    if (leader) {
+                        // step 0: Y = [L10 ; any 96 rows] T[0..31, 0..63] (columns 32..63 of T are 0)
+                        // step 1: T10 = [-T11 ; any 96 rows] Y (B2 columns 32..63 are not used)
+                        tc_fence_after();
+                        const uint32_t aa = smem_u32(step ? a2 : a1), bb = smem_u32(step ? b2 : b1);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int u = gt + 128 * q;                  // 16-byte chunk of K0 | K1
-            uint8_t *addr = qk + ((u >> 9) ? 24576 : 8192) + ((u & 511) << 4);
-            uint4 w = *reinterpret_cast<uint4 *>(addr);
-            const float2 f0 = unpack_bf2(w.x), f1 = unpack_bf2(w.y), f2 = unpack_bf2(w.z), f3 = unpack_bf2(w.w);
-            w.x = pack_h2(f0.x, f0.y);
-            w.y = pack_h2(f1.x, f1.y);
-            w.z = pack_h2(f2.x, f2.y);
-            w.w = pack_h2(f3.x, f3.y);
-            *reinterpret_cast<uint4 *>(addr) = w;
+                        for (int kk = 0; kk < 2; ++kk)
+                            umma_f16_ss(tI, sdesc_sw128(aa + kk * 32, 16, 1024), sdesc_sw128(bb + kk * 2048, 16384, 1024),
+                                        IDESC_KM64, kk > 0);
+                        umma_commit(&bars[KB_INV]);
+                        pend = KB_INV; pend_par = step;
+                    }
+                    __syncwarp();
+                    if (!group_wait(gs, &bars[KB_INV], step, abort, E_K_INV, false)) { fail = true; break; }
+                    pend = -1;
+                    tc_fence_after();
+                    if (wl == 0) {
+                        uint32_t y[32];
+                        tmem_ld32(tI, y);
+                        tmem_wait_ld();
+                        if (step == 0) {
+                            // Y rows (TMEM lanes 0..31, columns 0..31) -> fp16 rows of B2
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                *reinterpret_cast<uint4 *>(b2 + sw128_off(lane, j)) = make_uint4(
+                                    pack_h2(__uint_as_float(y[8 * j]), __uint_as_float(y[8 * j + 1])),
+                                    pack_h2(__uint_as_float(y[8 * j + 2]), __uint_as_float(y[8 * j + 3])),
+                                    pack_h2(__uint_as_float(y[8 * j + 4]), __uint_as_float(y[8 * j + 5])),
+                                    pack_h2(__uint_as_float(y[8 * j + 6]), __uint_as_float(y[8 * j + 7])));
+                            fence_proxy_async_smem();
+                        } else {
+                            float *dst = Tb + (32 + lane) * LSTR;
+#pragma unroll
+                            for (int j = 0; j < 32; j += 4)
+                                *reinterpret_cast<float4 *>(dst + j) = make_float4(
+                                    __uint_as_float(y[j]), __uint_as_float(y[j + 1]), __uint_as_float(y[j + 2]),
+                                    __uint_as_float(y[j + 3]));
+                        }
+                    }
+                    tc_fence_before();
+                    named_bar(gs.id, 256);
+                }
+            } else if (p.N <= 15) {
+                tc::invert_neumann(Lb, Tb, Yb, bt, p.N, gs.id);
+            } else {
+                // a long series (test sizes): dense steps by the first 128 threads
+                if (bt < 128) tc::invert_neumann128(Lb, Tb, Yb, bt, p.N, 4);
+                named_bar(gs.id, 256);
+            }
+            if (fail) break;
+            if (p.dbg_T && m == p.dbg_n && b == p.dbg_b && h == p.dbg_h)
+                for (int i = bt; i < 64 * 64; i += 256) p.dbg_T[i] = Tb[(i >> 6) * LSTR + (i & 63)];
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars[KB_LFREE + lb]);
+                mbar_arrive(&bars[KB_TFULL + lb]);
+            }
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        named_bar(gs.id, 128);
-        if (p.neumann) tc::invert_neumann128(Lb, Tb, Yb, gt, p.N, gs.id);
-        else tc::invert_exact128(Lb, Tb, Yb, gt, gs.id);
-        if (p.dbg_T && m == p.dbg_n && b == p.dbg_b && h == p.dbg_h)
-            for (int i = gt; i < 64 * 64; i += 128) p.dbg_T[i] = Tb[(i >> 6) * LSTR + (i & 63)];
+        if (leader && pend >= 0) mbar_wait_drain(&bars[pend], pend_par, kWait);
+        __syncwarp();
+        return;
+    }
+
+    // ---------------------------------------------------------------- stage C
+    const int ct = tid - 384;                     // 0..127
+    GroupSync gs{reinterpret_cast<volatile int *>(sm + K_MISC + 32), 0, 3, 128, ct == 0, warp == 12};
+    const bool leader = (ct == 0);
+    int sent[2] = {0, 0};
+    for (int m = 0; m < NC; ++m) {
+        const int s = m & 1;
+        const float *Tb = Tbuf(m);
+        const ChunkParams *par = par_of(m);
+        uint8_t *snd = snd_of(m);
+        if (!group_wait(gs, &bars[KB_TFULL + s], (m >> 1) & 1, abort, E_K_TFULL, false)) break;
         {
-            // T diag(beta) -> send buffer; T diag(beta e^g) -> the -W0 region (W's A operand)
-            const int rr = gt >> 1, half = gt & 1;
+            // T diag(beta), T diag(beta e^g) -> fp16; thread: row rr, 32 columns
+            const int rr = ct >> 1, half = ct & 1;
             const float *Tr = Tb + rr * LSTR + 32 * half;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -354,59 +470,35 @@ __device__ __forceinline__ void key_cta(uint8_t *sm, const CUtensorMap *tm_q, co
                 }
                 *reinterpret_cast<uint4 *>(snd + SND_TB + sw128_off(rr, c8)) =
                     make_uint4(pack_h2(sb[0], sb[1]), pack_h2(sb[2], sb[3]), pack_h2(sb[4], sb[5]), pack_h2(sb[6], sb[7]));
-                *reinterpret_cast<uint4 *>(snd + SND_MW0 + sw128_off(rr, c8)) =
+                *reinterpret_cast<uint4 *>(snd + SND_TBG + sw128_off(rr, c8)) =
                     make_uint4(pack_h2(sg[0], sg[1]), pack_h2(sg[2], sg[3]), pack_h2(sg[4], sg[5]), pack_h2(sg[6], sg[7]));
             }
         }
         fence_proxy_async_smem();
-        tc_fence_before();
-        named_bar(gs.id, 128);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[KB_TFREE + s]);
+        // the chain has finished chunk m - 2: its slot s may be overwritten
+        if (m >= 2) {
+            if (!group_wait(gs, &bars[KB_KFREE + s], ((m - 2) >> 1) & 1, abort, E_K_KFREE, true)) break;
+        } else {
+            named_bar(gs.id, 128);
+        }
         if (leader) {
-            // W = [T diag(beta e^g) ; any 64 rows] K: K as MN-major B over the two key boxes
-            tc_fence_after();
-            const uint32_t a0 = smem_u32(snd + SND_MW0), bk = smem_u32(qk + 8192);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                umma_f16_ss(tW, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(bk + kk * 2048, 16384, 1024),
-                            IDESC_KM128, kk > 0);
-            umma_commit(&bars[KB_WDONE + g]);
-            umma_commit(&bars[KB_QKFREE + g]);
-            pend = KB_WDONE + g; pend_par = ph;
+            const uint32_t kf = mapa_shared(smem_u32(sm + C_BAR + 8 * (CB_KFULL + s)), 1);
+            const uint32_t sl = mapa_shared(smem_u32(sm + C_SLOT + s * SLOT), 1);
+            mbar_arrive_expect_tx_remote(kf, 24576);
+            bulk_copy_to_peer(sl + S_MW0, snd + SND_TBG, 8192, kf);
+            bulk_copy_to_peer(sl + S_TB, snd + SND_TB, 8192, kf);
+            bulk_copy_to_peer(sl + S_P, snd + SND_P, 8192, kf);
         }
         __syncwarp();
-        if (!group_wait(gs, &bars[KB_WDONE + g], ph, abort, E_K_W, false)) break;
-        pend = -1;
-        tc_fence_after();
-        if (sp < 2) {
-            // -W rows (TMEM lanes 0..63) -> fp16, two 64-column boxes
-            const int r = 32 * sp + lane;
-            float x[64];
-            tmem_ld64(tW + lane_base, x);
-#pragma unroll
-            for (int j = 0; j < 64; ++j) x[j] = -x[j];
-            st_row_f16(snd + SND_MW0, r, x);
-            tmem_ld64(tW + lane_base + 64, x);
-#pragma unroll
-            for (int j = 0; j < 64; ++j) x[j] = -x[j];
-            st_row_f16(snd + SND_MW1, r, x);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        named_bar(gs.id, 128);
-        if (leader) {
-            mbar_arrive_expect_tx_remote(peer_kfull, 32768);
-            bulk_copy_to_peer(peer_slot + S_MW0, snd + SND_MW0, 8192, peer_kfull);
-            bulk_copy_to_peer(peer_slot + S_MW1, snd + SND_MW1, 8192, peer_kfull);
-            bulk_copy_to_peer(peer_slot + S_TB, snd + SND_TB, 8192, peer_kfull);
-            bulk_copy_to_peer(peer_slot + S_P, snd + SND_P, 8192, peer_kfull);
-        }
-        __syncwarp();
-        ++sent;
+        ++sent[s];
     }
-    // error path: no MMA of this group may still run when TMEM is released
-    if (leader && pend >= 0) mbar_wait_drain(&bars[pend], pend_par, kWait);
-    // tell the chain CTA how many chunks this group shipped into slot g
-    if (leader) st_peer_u32(mapa_shared(smem_u32(sm + C_MISC + 8 + 4 * g), 1), (uint32_t)sent);
+    // tell the chain CTA how many chunks were shipped into each slot
+    if (leader) {
+        st_peer_u32(mapa_shared(smem_u32(sm + C_MISC + 8), 1), (uint32_t)sent[0]);
+        st_peer_u32(mapa_shared(smem_u32(sm + C_MISC + 12), 1), (uint32_t)sent[1]);
+    }
     __syncwarp();
 }
 
@@ -459,23 +551,30 @@ __device__ __forceinline__ void chain_cta(uint8_t *sm, const CUtensorMap *tm_q, 
         // ------------------------------------------------ MMA issue (one thread)
         if (lane == 0) {
             const uint32_t hs = smem_u32(sm + C_HS);
-            auto xbuf = [&](int n) { return tmem + TM_X + 128u * (uint32_t)(n % 3); };
-            // U(n): X_n = [T diag(beta) ; 0] V once the key side and the conversion are done
-            auto u_ready = [&](int n) {
-                const int s = n & 1;
-                if (!mbar_try_wait_cluster(&bars[CB_KFULL + s], (n >> 1) & 1)) return false;
-                if (!mbar_try_wait(&bars[CB_CVT + s], (n >> 1) & 1)) return false;
-                if (n >= 3 && !mbar_try_wait(&bars[CB_XFREE + n % 3], ((n - 3) / 3) & 1)) return false;
-                return true;
+            auto xbuf = [&](int n) { return tmem + TM_X + 128u * (uint32_t)(n & 1); };
+            const uint32_t peer_krecv = mapa_shared(smem_u32(sm + K_BAR + 8 * KB_KRECV), 0);
+            // W(n) = [T diag(beta e^g) ; Q'0] K16 once the key side's tiles and the
+            // conversion of chunk n are in (lanes 64..127 of W are not used)
+            auto w_ready = [&](int n) {
+                return mbar_try_wait_cluster(&bars[CB_KFULL + (n & 1)], (n >> 1) & 1) &&
+                       mbar_try_wait(&bars[CB_CVT + (n & 1)], (n >> 1) & 1);
             };
-            auto u_wait = [&](int n) {
-                const int s = n & 1;
-                if (!mbar_wait_cluster(&bars[CB_KFULL + s], (n >> 1) & 1, abort, E_C_KFULL, kWait)) return false;
-                if (!mbar_wait(&bars[CB_CVT + s], (n >> 1) & 1, abort, E_C_CVT, kWait)) return false;
-                if (n >= 3 && !mbar_wait(&bars[CB_XFREE + n % 3], ((n - 3) / 3) & 1, abort, E_C_XFREE, kWait))
-                    return false;
-                return true;
+            auto w_wait = [&](int n) {
+                return mbar_wait_cluster(&bars[CB_KFULL + (n & 1)], (n >> 1) & 1, abort, E_C_KFULL, kWait) &&
+                       mbar_wait(&bars[CB_CVT + (n & 1)], (n >> 1) & 1, abort, E_C_CVT, kWait);
             };
+            auto w_issue = [&](int n) {
+                // the key side's copy of chunk n has landed: its send buffer is free
+                mbar_arrive_remote(peer_krecv + 8 * (n % 3));
+                tc_fence_after();
+                const uint32_t st = smem_u32(slot(n & 1));
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16_ss(tmem + TM_WC, sdesc_sw128(st + S_MW0 + kk * 32, 16, 1024),
+                                sdesc_sw128(st + S_K0 + kk * 2048, 8192, 1024), IDESC_KM128, kk > 0);
+                umma_commit(&bars[CB_WDONE]);
+            };
+            // U(n): X_n = [T diag(beta) ; 0] V
             auto u_issue = [&](int n) {
                 tc_fence_after();
                 const uint32_t st = smem_u32(slot(n & 1));
@@ -486,42 +585,73 @@ __device__ __forceinline__ void chain_cta(uint8_t *sm, const CUtensorMap *tm_q, 
             };
             int pend = -1, pend_par = 0;
             int cons[2] = {0, 0};                 // key-side shipments consumed, per slot
-            bool ok = NC > 0 && u_wait(0);
-            if (ok) { u_issue(0); cons[0] = 1; }
+            int nu = 0;                           // U commits (on a barrier only the error path waits for)
+            bool ok = NC > 0 && w_wait(0);
+            if (ok) {
+                w_issue(0);
+                u_issue(0);
+                umma_commit(&bars[CB_UDONE]);
+                cons[0] = 1; pend = CB_UDONE; pend_par = nu++ & 1;
+            }
             for (int n = 0; ok && n < NC; ++n) {
-                const int s = n & 1;
+                const int s = n & 1, xb = n & 1;
+                const uint32_t par2 = (n >> 1) & 1;
                 const uint32_t st = smem_u32(slot(s));
-                // X(n): [-W ; Q'] h16 onto U
-                if (!mbar_wait_spin(&bars[CB_HREADY], n & 1, abort, E_C_HREADY, kWait)) break;
-                tc_fence_after();
+                // -W and K' of chunk n are in shared memory
+                if (!mbar_wait(&bars[CB_WREADY], n & 1, abort, E_C_WREADY, kWait)) break;
+                // X(n), one value half at a time: [-W ; Q'] h16_j onto U
+                bool fail = false;
+#pragma unroll 1
+                for (int j = 0; j < 2; ++j) {
+                    if (!mbar_wait_spin(&bars[CB_HREADY + j], n & 1, abort, E_C_HREADY, kWait)) { fail = true; break; }
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    umma_f16_ss(xbuf(n), sdesc_sw128(st + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                                sdesc_sw128(hs + kk * 2048, 16384, 1024), IDESC_KM128, 1);
-                umma_commit(&bars[CB_XDONE + n % 3]);
-                pend = CB_XDONE + n % 3; pend_par = (n / 3) & 1;
-                bool u_next = n + 1 >= NC;
-                if (!u_next && u_ready(n + 1)) { u_issue(n + 1); u_next = true; ++cons[(n + 1) & 1]; }
-                // Z(n): h += K'^T Delta16;  O(n): X_n += [0 ; P] Delta16
-                if (!mbar_wait_spin(&bars[CB_DDONE], n & 1, abort, E_C_DDONE, kWait)) break;
-                if (!mbar_wait_spin(&bars[CB_HSTORED], n & 1, abort, E_C_HSTORED, kWait)) break;
-                tc_fence_after();
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_f16_ss(xbuf(n) + 64 * j, sdesc_sw128(st + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                                    sdesc_sw128(hs + 16384 * j + kk * 2048, 16384, 1024), IDESC_KM64, 1);
+                    umma_commit(&bars[CB_XDONE + 2 * xb + j]);
+                    pend = CB_XDONE + 2 * xb + j; pend_par = par2;
+                }
+                if (fail) break;
+                // W(n+1) while the Delta epilogue runs (the tensor pipe is idle then);
+                // U(n+1) only after Z(n), O(n): an MMA issue blocks while earlier MMAs
+                // drain, so anything ahead of Z would delay the state chain
+                bool w_next = n + 1 >= NC;
+                if (!w_next && w_ready(n + 1)) { w_issue(n + 1); w_next = true; ++cons[(n + 1) & 1]; }
+                // per half: Z(n) h_j += K'^T Delta16_j;  O(n) X_n,j += [0 ; P] Delta16_j
+#pragma unroll 1
+                for (int j = 0; j < 2; ++j) {
+                    if (!mbar_wait_spin(&bars[CB_DDONE + j], n & 1, abort, E_C_DDONE, kWait)) { fail = true; break; }
+                    if (!mbar_wait_spin(&bars[CB_HSTORED + j], n & 1, abort, E_C_HSTORED, kWait)) { fail = true; break; }
+                    tc_fence_after();
+                    const uint32_t dj = st + S_V0 + 8192 * j;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16_ss(tmem + TM_H, sdesc_sw128(st + S_K0 + kk * 2048, 8192, 1024),
-                                sdesc_sw128(st + S_V0 + kk * 2048, 8192, 1024), IDESC_MM128, 1);
-                umma_commit(&bars[CB_ZDONE]);
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ss(tmem + TM_H + 64 * j, sdesc_sw128(st + S_K0 + kk * 2048, 8192, 1024),
+                                    sdesc_sw128(dj + kk * 2048, 8192, 1024), IDESC_MM64, 1);
+                    umma_commit(&bars[CB_ZDONE + j]);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16_ss(xbuf(n), sdesc_sw128(st + S_ZERO + kk * 32, 16, 1024),
-                                sdesc_sw128(st + S_V0 + kk * 2048, 8192, 1024), IDESC_KM128, 1);
-                umma_commit(&bars[CB_ODONE + n % 3]);
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ss(xbuf(n) + 64 * j, sdesc_sw128(st + S_ZERO + kk * 32, 16, 1024),
+                                    sdesc_sw128(dj + kk * 2048, 8192, 1024), IDESC_KM64, 1);
+                    umma_commit(&bars[CB_ODONE + 2 * xb + j]);
+                    pend = CB_ODONE + 2 * xb + j; pend_par = par2;
+                }
+                if (fail) break;
                 umma_commit(&bars[CB_SFREE + s]);
-                pend = CB_SFREE + s; pend_par = (n >> 1) & 1;
-                if (!u_next) {
-                    if (!u_wait(n + 1)) break;
+                pend = CB_SFREE + s; pend_par = par2;
+                if (n + 1 < NC) {
+                    if (!w_next) {
+                        if (!w_wait(n + 1)) break;
+                        w_issue(n + 1);
+                        ++cons[(n + 1) & 1];
+                    }
+                    // X buffer (n+1) & 1 is free once the output rows of chunk n - 1 are read
+                    if (n >= 1 && !mbar_wait(&bars[CB_XFREE + ((n + 1) & 1)], ((n - 1) >> 1) & 1, abort, E_C_XFREE, kWait))
+                        break;
                     u_issue(n + 1);
-                    ++cons[(n + 1) & 1];
+                    umma_commit(&bars[CB_UDONE]);
+                    pend = CB_UDONE; pend_par = nu++ & 1;
                 }
             }
             // error path: no MMA may still run when TMEM is released
@@ -535,7 +665,11 @@ __device__ __forceinline__ void chain_cta(uint8_t *sm, const CUtensorMap *tm_q, 
 
     if (warp == 2 || warp == 3 || warp >= 12) {
         // ---------------------------------------- operand conversion (6 warps)
+        // (a) q -> Q' = diag(e^g) Q, k -> K16, v -> V16 (fp16, in place);
+        // (b) once W(n) is in TMEM: -W -> fp16 over T diag(beta e^g) (warps 12, 13:
+        //     TMEM lanes 0..63) and K16 -> K' = diag(e^{g_C - g}) K in place
         const int cvi = (warp < 4 ? warp - 2 : warp - 10) * 32 + lane;   // 0..191
+        const int sp = warp & 3;
         GroupSync gs{reinterpret_cast<volatile int *>(sm + C_MISC + 16), 0, 3, 192, warp == 2 && lane == 0,
                      warp == 2};
         float ga0 = 1.f, ga1 = 1.f, gb0 = 0.f, gb1 = 0.f;
@@ -555,7 +689,7 @@ __device__ __forceinline__ void chain_cta(uint8_t *sm, const CUtensorMap *tm_q, 
                 const int tile = idx >> 9, u = idx & 511, row = u >> 3;
                 const uint32_t off = tile == 0 ? S_Q0 : tile == 1 ? S_Q1 : tile == 2 ? S_K0
                                    : tile == 3 ? S_K1 : tile == 4 ? S_V0 : S_V1;
-                const float sc = tile < 2 ? par->eg[row] : (tile < 4 ? par->egc[row] : 1.f);
+                const float sc = tile < 2 ? par->eg[row] : 1.f;
                 uint8_t *addr = st + off + (u << 4);
                 uint4 w = *reinterpret_cast<uint4 *>(addr);
                 const float2 f0 = unpack_bf2(w.x), f1 = unpack_bf2(w.y), f2 = unpack_bf2(w.z), f3 = unpack_bf2(w.w);
@@ -568,6 +702,43 @@ __device__ __forceinline__ void chain_cta(uint8_t *sm, const CUtensorMap *tm_q, 
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[CB_CVT + s]);
+            // (b)
+            if (!group_wait(gs, &bars[CB_WDONE], n & 1, abort, E_C_WDONE, false)) break;
+            tc_fence_after();
+            if (warp >= 12 && sp < 2) {
+                const uint32_t lb = (uint32_t)(32 * sp) << 16;
+                const int r = 32 * sp + lane;
+                float x[64];
+                tmem_ld64(tmem + TM_WC + lb, x);
+#pragma unroll
+                for (int j = 0; j < 64; ++j) x[j] = -x[j];
+                st_row_f16(st + S_MW0, r, x);
+                tmem_ld64(tmem + TM_WC + lb + 64, x);
+#pragma unroll
+                for (int j = 0; j < 64; ++j) x[j] = -x[j];
+                st_row_f16(st + S_MW1, r, x);
+            }
+#pragma unroll 2
+            for (int j = 0; j < 6; ++j) {
+                const int idx = cvi + 192 * j;               // 16-byte chunk of K0 K1 (1024 of them)
+                if (idx < 1024) {
+                    const int u = idx & 511;
+                    uint8_t *addr = st + ((idx >> 9) ? S_K1 : S_K0) + (u << 4);
+                    const float sc = par->egc[u >> 3];
+                    uint4 w = *reinterpret_cast<uint4 *>(addr);
+                    const float2 f0 = tc::unpack_h2(w.x), f1 = tc::unpack_h2(w.y), f2 = tc::unpack_h2(w.z),
+                                 f3 = tc::unpack_h2(w.w);
+                    w.x = pack_h2(f0.x * sc, f0.y * sc);
+                    w.y = pack_h2(f1.x * sc, f1.y * sc);
+                    w.z = pack_h2(f2.x * sc, f2.y * sc);
+                    w.w = pack_h2(f3.x * sc, f3.y * sc);
+                    *reinterpret_cast<uint4 *>(addr) = w;
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[CB_WREADY]);
         }
         return;
     }
@@ -595,16 +766,16 @@ __device__ __forceinline__ void chain_cta(uint8_t *sm, const CUtensorMap *tm_q, 
         }
         tmem_wait_st();
     }
-    auto xbuf = [&](int n) { return tmem + TM_X + 128u * (uint32_t)(n % 3); };
-    // output rows of chunk j: X_j lanes 64..127 once O(j) is complete
+    auto xbuf = [&](int n) { return tmem + TM_X + 128u * (uint32_t)(n & 1); };
+    // output rows of chunk j (this warp's value half): X_j lanes 64..127 once O(j) is complete
     auto out_rows = [&](int j) -> bool {
-        if (!warp_wait(&bars[CB_ODONE + j % 3], (j / 3) & 1, abort, E_C_ODONE, false)) return false;
+        if (!warp_wait(&bars[CB_ODONE + 2 * (j & 1) + hf], (j >> 1) & 1, abort, E_C_ODONE, false)) return false;
         tc_fence_after();
         float x[64];
         tmem_ld64(xbuf(j) + lb + 64 * hf, x);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[CB_XFREE + j % 3]);
+        if (lane == 0) mbar_arrive(&bars[CB_XFREE + (j & 1)]);
         const int t = j * C + (r - 64);
         if (t < T) {
             const size_t go = (((size_t)b * T + t) * H + h) * DV + 64 * hf;
@@ -632,12 +803,15 @@ __device__ __forceinline__ void chain_cta(uint8_t *sm, const CUtensorMap *tm_q, 
         }
         return true;
     };
+    // the two value halves are independent chains (each column of h, Delta and O
+    // depends only on the same column of U and h): warps of half hf wait only on
+    // their own half's barriers
     bool ok = true;
     for (int n = 0; n < NC; ++n) {
         const int s = n & 1;
         // the gates of chunk n are scanned before its conversion completes
         if (!warp_wait(&bars[CB_CVT + s], (n >> 1) & 1, abort, E_C_CVT, false)) { ok = false; break; }
-        if (n > 0 && !warp_wait(&bars[CB_ZDONE], (n - 1) & 1, abort, E_C_ZDONE, true)) { ok = false; break; }
+        if (n > 0 && !warp_wait(&bars[CB_ZDONE + hf], (n - 1) & 1, abort, E_C_ZDONE, true)) { ok = false; break; }
         tc_fence_after();
         {
             // h16 <- h (operand of X(n));  h <- e^{g_C} h for Z(n) to accumulate onto
@@ -655,14 +829,17 @@ __device__ __forceinline__ void chain_cta(uint8_t *sm, const CUtensorMap *tm_q, 
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[CB_HREADY]);
+        if (lane == 0) mbar_arrive(&bars[CB_HREADY + hf]);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[CB_HSTORED]);
+        if (lane == 0) mbar_arrive(&bars[CB_HSTORED + hf]);
         if (sp < 2) {
             // Delta = U - W h (X_n lanes 0..63) -> fp16 over V in slot s
-            if (!warp_wait(&bars[CB_XDONE + n % 3], (n / 3) & 1, abort, E_C_XDONE, true)) { ok = false; break; }
+            if (!warp_wait(&bars[CB_XDONE + 2 * (n & 1) + hf], (n >> 1) & 1, abort, E_C_XDONE, true)) {
+                ok = false;
+                break;
+            }
             tc_fence_after();
             float x[64];
             tmem_ld64(xbuf(n) + lb + 64 * hf, x);
@@ -670,14 +847,14 @@ __device__ __forceinline__ void chain_cta(uint8_t *sm, const CUtensorMap *tm_q, 
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[CB_DDONE]);
+            if (lane == 0) mbar_arrive(&bars[CB_DDONE + hf]);
         } else if (n > 0) {
             if (!out_rows(n - 1)) { ok = false; break; }
         }
     }
     if (ok && NC > 0) {
         if (sp >= 2) ok = out_rows(NC - 1);
-        if (ok && warp_wait(&bars[CB_ZDONE], (NC - 1) & 1, abort, E_C_ZDONE, false)) {
+        if (ok && warp_wait(&bars[CB_ZDONE + hf], (NC - 1) & 1, abort, E_C_ZDONE, false)) {
             tc_fence_after();
             float x[64];
             tmem_ld64(tmem + TM_H + lb + 64 * hf, x);
@@ -708,6 +885,12 @@ fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     if (tid == 0) {
         if (key) {
             for (int i = 0; i < KB_N; ++i) mbar_init(&bars[i], 1);
+            for (int i = 0; i < 2; ++i) {
+                mbar_init(&bars[KB_LFULL + i], 4);    // stage A warps
+                mbar_init(&bars[KB_LFREE + i], 8);    // stage B warps
+                mbar_init(&bars[KB_TFULL + i], 8);    // stage B warps
+                mbar_init(&bars[KB_TFREE + i], 4);    // stage C warps
+            }
         } else {
             for (int i = 0; i < 2; ++i) {
                 mbar_init(&bars[CB_SFULL + i], 1);
@@ -715,15 +898,20 @@ fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 mbar_init(&bars[CB_KFULL + i], 1);
                 mbar_init(&bars[CB_CVT + i], 6);
             }
-            for (int i = 0; i < 3; ++i) {
+            for (int i = 0; i < 4; ++i) {
                 mbar_init(&bars[CB_XDONE + i], 1);
                 mbar_init(&bars[CB_ODONE + i], 1);
-                mbar_init(&bars[CB_XFREE + i], 4);
             }
-            mbar_init(&bars[CB_HREADY], 8);
-            mbar_init(&bars[CB_HSTORED], 8);
-            mbar_init(&bars[CB_DDONE], 4);
-            mbar_init(&bars[CB_ZDONE], 1);
+            for (int i = 0; i < 2; ++i) mbar_init(&bars[CB_XFREE + i], 4);
+            for (int j = 0; j < 2; ++j) {
+                mbar_init(&bars[CB_HREADY + j], 4);
+                mbar_init(&bars[CB_HSTORED + j], 4);
+                mbar_init(&bars[CB_DDONE + j], 2);
+                mbar_init(&bars[CB_ZDONE + j], 1);
+            }
+            mbar_init(&bars[CB_WDONE], 1);
+            mbar_init(&bars[CB_WREADY], 6);
+            mbar_init(&bars[CB_UDONE], 1);
             // [2], [3]: chunks the key side shipped per slot; [6], [7]: chunks consumed
             for (int i = 2; i < 8; ++i) reinterpret_cast<volatile uint32_t *>(misc)[i] = 0;
         }

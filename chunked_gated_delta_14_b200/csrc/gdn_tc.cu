@@ -66,7 +66,7 @@ constexpr int kNeumannMaxN = 15;
 constexpr unsigned long long kWaitLimit = 4000000000ull;   // ~2 s at the boost clock
 
 // error codes recorded in g_tc_error (first one wins)
-enum { E_FULL = 1, E_EMPTY, E_KSREADY, E_KSFREE, E_O, E_UW, E_X, E_H, E_K1_TMA, E_K1_MMA };
+enum { E_FULL = 1, E_EMPTY, E_KSREADY, E_KSFREE, E_O, E_UW, E_X, E_H, E_K1_TMA, E_K1_MMA, E_XISS };
 
 constexpr uint32_t IDESC_BF_KK = idesc_f16(128, 64, 1, 1, 0, 0);    // bf16, K-major x K-major, N 64
 constexpr uint32_t IDESC_KM64 = idesc_f16(128, 64, 0, 0, 0, 1);     // fp16, K-major x MN-major, N 64
@@ -89,7 +89,12 @@ constexpr uint32_t K1_OFF_YB = K1_MAT;                 // tiles once the Gram MM
 constexpr uint32_t K1_OFF_TB = 32768;
 constexpr uint32_t K1_OFF_PAR = K1_OFF_TB + K1_MAT;
 constexpr uint32_t K1_OFF_BAR = K1_OFF_PAR + ((sizeof(ChunkParams) + 15) & ~15u);
-constexpr uint32_t K1_SMEM = K1_OFF_BAR + 64 + 1024;  // + base alignment slack
+// fp16 staging of the 32 -> 64 inverse merge (exact mode): B2 over the 16 -> 32
+// merge's scratch, A1 in the rest of the tile region (L occupies its start), A2
+// and B1 in a region of their own; a 64-row A operand drags 96 more rows along
+constexpr uint32_t K1_OFF_STG = (K1_OFF_BAR + 64 + 1023) & ~1023u;
+constexpr uint32_t K1_OFF_B2 = K1_OFF_YB, K1_OFF_A1 = 22528, K1_OFF_A2 = K1_OFF_STG, K1_OFF_B1 = K1_OFF_STG + 4096;
+constexpr uint32_t K1_SMEM = K1_OFF_STG + 16384 + 1024;  // + base alignment slack
 // residual correction: three more 64 x LSTR fp32 matrices (E, R ping-pong)
 constexpr uint32_t K1_OFF_RES = K1_OFF_BAR + 64;
 constexpr uint32_t K1_SMEM_RES = K1_OFF_RES + 3 * K1_MAT + 1024;
@@ -116,14 +121,16 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     float *Yb = reinterpret_cast<float *>(sm + K1_OFF_YB);
     ChunkParams *par = reinterpret_cast<ChunkParams *>(sm + K1_OFF_PAR);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + K1_OFF_BAR);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + K1_OFF_BAR + 16);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + K1_OFF_BAR + 20);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + K1_OFF_BAR + 24);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + K1_OFF_BAR + 28);
+    volatile int *okflag = reinterpret_cast<volatile int *>(sm + K1_OFF_BAR + 32);
     uint8_t *ws = p.ws + ((((size_t)b * p.H + h) * p.NC + n) * WS_CHUNK_BYTES);
 
     const int t0 = n * C;
     if (tid == 0) {
         mbar_init(&bars[0], 1);
         mbar_init(&bars[1], 1);
+        mbar_init(&bars[2], 1);
         *abort_flag = 0;
         fence_mbar_init();
         // the tiles first: their latency overlaps the set-up below
@@ -135,7 +142,7 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     __syncwarp();
     if (warp == 0) {
-        tmem_alloc(tmem_slot, 64);
+        tmem_alloc(tmem_slot, 128);      // Gram (64 columns), inverse merge (64)
         tmem_relinquish();
     }
     if (!p.neumann)
@@ -221,15 +228,92 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         tc_fence_before();
         named_bar(1, K1_THREADS);
-        if (p.neumann) tc::invert_neumann(Lb, Tb, Yb, tid, p.N, 1);
-        else tc::invert_exact(Lb, Tb, Yb, tid, 1);
+        bool inv_ok = true;
+        if (p.neumann) {
+            tc::invert_neumann(Lb, Tb, Yb, tid, p.N, 1);
+        } else {
+            // T = (I + L)^-1: the 16 x 16 diagonal blocks and the 16 -> 32 merges on
+            // the CUDA cores, the 32 -> 64 merge T10 = -T11 L10 T00 as two MMAs (fp16
+            // operands, fp32 accumulate).  Staging tiles in the free part of the q/k
+            // tile region and the scratch of the 16 -> 32 merge; the 96 rows each
+            // 64-row A operand drags along lie in tiles that stay unchanged while it runs.
+            tc::invert_exact_to32(Lb, Tb, Yb, tid, 1);
+            uint8_t *a1 = sm + K1_OFF_A1, *b1 = sm + K1_OFF_B1, *a2 = sm + K1_OFF_A2, *b2 = sm + K1_OFF_B2;
+            const uint32_t tI = tmem + 64;
+            {
+                const int u = tid & 127, rw = u >> 2, j = u & 3;
+                const float *src = tid < 128 ? Lb + (32 + rw) * LSTR + 8 * j : Tb + (32 + rw) * LSTR + 32 + 8 * j;
+                const float sg = tid < 128 ? 1.f : -1.f;
+                const float4 x0 = *reinterpret_cast<const float4 *>(src);
+                const float4 x1 = *reinterpret_cast<const float4 *>(src + 4);
+                *reinterpret_cast<uint4 *>((tid < 128 ? a1 : a2) + sw128_off(rw, j)) =
+                    make_uint4(pack_h2(sg * x0.x, sg * x0.y), pack_h2(sg * x0.z, sg * x0.w),
+                               pack_h2(sg * x1.x, sg * x1.y), pack_h2(sg * x1.z, sg * x1.w));
+                const int k = tid >> 3, jb = tid & 7;
+                const float *tr = Tb + k * LSTR + 8 * jb;
+                const float4 y0 = *reinterpret_cast<const float4 *>(tr);
+                const float4 y1 = *reinterpret_cast<const float4 *>(tr + 4);
+                *reinterpret_cast<uint4 *>(b1 + sw128_off(k, jb)) =
+                    make_uint4(pack_h2(y0.x, y0.y), pack_h2(y0.z, y0.w), pack_h2(y1.x, y1.y), pack_h2(y1.z, y1.w));
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(1, K1_THREADS);
+#pragma unroll 1
+            for (int step = 0; step < 2; ++step) {
+                if (tid == 0) {
+                    // step 0: Y = [L10 ; any 96 rows] T[0..31, 0..63] (columns 32..63 of T are 0)
+                    // step 1: T10 = [-T11 ; any 96 rows] Y (columns 32..63 of B2 are not used)
+                    tc_fence_after();
+                    const uint32_t aa = smem_u32(step ? a2 : a1), bb = smem_u32(step ? b2 : b1);
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk)
+                        umma_f16_ss(tI, sdesc_sw128(aa + kk * 32, 16, 1024), sdesc_sw128(bb + kk * 2048, 16384, 1024),
+                                    IDESC_KM64, kk > 0);
+                    umma_commit(&bars[2]);
+                    const bool w = mbar_wait(&bars[2], step, abort_flag, E_K1_MMA, kWaitLimit);
+                    if (!w) mbar_wait_drain(&bars[2], step, kWaitLimit);
+                    *okflag = w ? 1 : 0;
+                }
+                __syncwarp();
+                named_bar(1, K1_THREADS);
+                if (!*okflag) { inv_ok = false; break; }
+                mbar_try_wait(&bars[2], step);
+                tc_fence_after();
+                if (warp == 0) {
+                    uint32_t y[32];
+                    tmem_ld32(tI, y);
+                    tmem_wait_ld();
+                    if (step == 0) {
+                        // Y rows (TMEM lanes 0..31, columns 0..31) -> fp16 rows of B2
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            *reinterpret_cast<uint4 *>(b2 + sw128_off(lane, j)) = make_uint4(
+                                pack_h2(__uint_as_float(y[8 * j]), __uint_as_float(y[8 * j + 1])),
+                                pack_h2(__uint_as_float(y[8 * j + 2]), __uint_as_float(y[8 * j + 3])),
+                                pack_h2(__uint_as_float(y[8 * j + 4]), __uint_as_float(y[8 * j + 5])),
+                                pack_h2(__uint_as_float(y[8 * j + 6]), __uint_as_float(y[8 * j + 7])));
+                        fence_proxy_async_smem();
+                    } else {
+                        float *dst = Tb + (32 + lane) * LSTR;
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4)
+                            *reinterpret_cast<float4 *>(dst + j) = make_float4(
+                                __uint_as_float(y[j]), __uint_as_float(y[j + 1]), __uint_as_float(y[j + 2]),
+                                __uint_as_float(y[j + 3]));
+                    }
+                }
+                tc_fence_before();
+                named_bar(1, K1_THREADS);
+            }
+        }
         const float *Tsrc = Tb;
         if (p.neumann == 2) {
             float *res = reinterpret_cast<float *>(sm + K1_OFF_RES);
             Tsrc = tc::residual_correct(Lb, Tb, res, res + 64 * LSTR, res + 2 * 64 * LSTR, tid, p.S, 1);
         }
         // T diag(beta) and T diag(beta e^g) -> fp16, row-major
-        {
+        if (inv_ok) {
             const int rr = tid >> 2, j0 = (tid & 3) * 2;
             uint4 *d1 = reinterpret_cast<uint4 *>(ws + (size_t)rr * 128);
             uint4 *d2 = reinterpret_cast<uint4 *>(ws + (size_t)(64 + rr) * 128);
@@ -255,7 +339,7 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     block_sync();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 64);
+        tmem_dealloc(tmem, 128);
     }
     if (tid == 0 && *abort_flag) atomicCAS(&g_tc_error, 0u, (unsigned)*abort_flag);
 }
@@ -281,7 +365,7 @@ constexpr uint32_t OFF_PAR = OFF_DS + 2 * 8192;
 constexpr uint32_t PAR_BYTES = (sizeof(ChunkParams) + 15) & ~15u;
 constexpr uint32_t OFF_BAR = OFF_PAR + 3 * PAR_BYTES;   // params ring of 3
 enum { B_FULL = 0, B_EMPTY = 2, B_KSREADY = 4, B_KSFREE = 6, B_UW = 8, B_X = 9, B_H = 10, B_O = 11,
-       N_BARS = 13 };
+       B_XISS = 13, N_BARS = 14 };
 constexpr uint32_t OFF_MISC = OFF_BAR + N_BARS * 8;     // tmem slot, abort flag, group slots
 constexpr uint32_t SMEM_USED = OFF_MISC + 32;
 constexpr uint32_t K2_SMEM = SMEM_USED + 1024;
@@ -289,6 +373,10 @@ static_assert(K2_SMEM <= 232448, "shared memory budget of one sm_100 block");
 static_assert(K1_SMEM * K1_BLOCKS_PER_SM <= 233472, "key-side blocks per SM");
 static_assert(K1_SMEM_RES <= 232448, "residual-correction key-side block fits one SM");
 static_assert(K1_OFF_YB + 8192 <= K1_OFF_TB, "L and the inverse scratch fit in the tile region");
+static_assert(K1_OFF_LB + K1_MAT <= K1_OFF_B2 && K1_OFF_B2 + 4096 <= K1_OFF_A1 && K1_OFF_A1 + 4096 <= K1_OFF_TB &&
+              K1_OFF_A1 + 16384 <= K1_OFF_TB + K1_MAT && (K1_OFF_B2 & 1023) == 0 && (K1_OFF_A1 & 1023) == 0 &&
+              K1_OFF_A2 + 16384 + 1024 <= K1_SMEM,
+              "inverse merge staging: tiles apart, 64-row operands' padding rows inside the block");
 
 // TMEM columns
 constexpr uint32_t TM_U0 = 0, TM_U1 = 64, TM_W = 128, TM_X0 = 256, TM_X1 = 320, TM_H = 384;
@@ -359,6 +447,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         mbar_init(&bars[B_H], 1);
         mbar_init(&bars[B_O], 1);
         mbar_init(&bars[B_O + 1], 1);
+        mbar_init(&bars[B_XISS], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -452,7 +541,12 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             fence_proxy_async_smem();
             tc_fence_before();
             if (!sync_ok(1, KS_THREADS, leader, kcnt)) break;
-            if (leader) {
+            // the U and W MMAs of chunk m go into the tensor pipe right after the
+            // chain has issued X(m - 1): they run while its Delta epilogue does,
+            // instead of landing ahead of the state update it waits for
+            if (leader && m >= 1 && !mbar_wait(&bars[B_XISS], (m - 1) & 1, abort_flag, E_XISS, lim)) {
+                // abort: the group leaves at the next wait
+            } else if (leader) {
                 tc_fence_after();
                 const uint32_t at = smem_u32(st + S_TB), av = smem_u32(st + S_V);
                 const uint32_t ag = smem_u32(st + S_TBG), ak = smem_u32(st + S_K);
@@ -628,6 +722,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                                 sdesc_sw128(b0 + kk * 2048, 8192, 1024), IDESC_KM64, kk > 0);
                 }
                 umma_commit(&bars[B_X]);
+                mbar_arrive(&bars[B_XISS]);
                 pend = B_X; pend_par = n & 1;
             }
             __syncwarp();

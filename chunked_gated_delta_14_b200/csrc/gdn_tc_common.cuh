@@ -151,7 +151,10 @@ constexpr int LSTR = 68;   // fp32 row stride of the L and T work matrices
 // LSTR) by 256 threads: 16 x 16 diagonal blocks by forward substitution, then
 // T21 = -T22 L21 T11 merges 16 -> 32 -> 64.  Tb's entries above the diagonal
 // blocks must be zero on entry.  Yb: 1024 floats.  Ends with a barrier.
-__device__ __forceinline__ void invert_exact(const float *Lb, float *Tb, float *Yb, int kt, int bar_id) {
+// The first two levels of invert_exact: the 16 x 16 diagonal blocks and the
+// 16 -> 32 merges (T00 and T11 of the two 32-blocks complete).  Yb: 512 floats.
+// Ends with a barrier.
+__device__ __forceinline__ void invert_exact_to32(const float *Lb, float *Tb, float *Yb, int kt, int bar_id) {
     if (kt < 64) {
         // one column per thread; each solved entry updates the rows below it at once
         const int c = kt, base = c & ~15, jc = c & 15;
@@ -193,6 +196,10 @@ __device__ __forceinline__ void invert_exact(const float *Lb, float *Tb, float *
         *reinterpret_cast<float2 *>(Tb + (b1 + rr) * LSTR + b0 + c0) = make_float2(-z0, -z1);
     }
     named_bar(bar_id, 256);
+}
+
+__device__ __forceinline__ void invert_exact(const float *Lb, float *Tb, float *Yb, int kt, int bar_id) {
+    invert_exact_to32(Lb, Tb, Yb, kt, bar_id);
     {
         // 32 -> 64: Y = L10 T00, T10 = -T11 Y; thread (row, 4 columns), full unroll
         const int rr = kt >> 3, c0 = (kt & 7) * 4;

@@ -102,7 +102,7 @@ typedef enum {
 } gdn_inv_mode;
 
 typedef enum {
-    GDN_KERNEL_AUTO = 0,        /* the first of TC, TC_SPLIT, SIMT that supports the call
+    GDN_KERNEL_AUTO = 0,        /* the first of TC_SPLIT, TC, SIMT that supports the call
                                    (RECURRENT for T <= 8) */
     GDN_KERNEL_SIMT = 1,        /* fp32 CUDA-core chunk kernel (all variants) */
     GDN_KERNEL_TC = 2,          /* fused tcgen05/TMEM/TMA kernel, one launch of 2-CTA

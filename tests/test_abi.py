@@ -103,20 +103,21 @@ def test_null_args_pointer():
 
 def test_valid_arguments_select_a_kernel():
     assert gdn.select_kernel(_args(kernel=1)) == 1
-    assert gdn.select_kernel(_args()) == 2                                     # fused tensor-core kernel
-    assert gdn.select_kernel(_args(mode=1, neumann_N=63)) == 2                 # any N on the fused kernel
+    assert gdn.select_kernel(_args()) == 4                                     # split tensor-core kernels
+    assert gdn.select_kernel(_args(kernel=2)) == 2                             # the fused kernel on request
+    assert gdn.select_kernel(_args(mode=1, neumann_N=63)) == 2                 # N > 15: the fused kernel
     assert gdn.select_kernel(_args(mode=2, neumann_N=3, residual_S=8)) == 4   # residual: split kernels
     assert gdn.select_kernel(_args(dv=64)) == 4                                # dv 64: split kernels
     assert gdn.select_kernel(_args(dv_split=2)) == 4                           # a value split: split kernels
-    assert gdn.select_kernel(_args(dv_split=1)) == 2
+    assert gdn.select_kernel(_args(dv_split=1)) == 2                           # one slice: the fused kernel
     assert gdn.select_kernel(_args(T=1)) == 3                                  # decode step
     assert gdn.select_kernel(_args(T=8, io_dtype=0, dk=64, dv=64)) == 3
-    assert gdn.select_kernel(_args(T=9)) == 2                                  # chunked from T = 9
+    assert gdn.select_kernel(_args(T=9)) == 4                                  # chunked from T = 9
     assert gdn.select_kernel(_args(T=1, mode=1, neumann_N=3)) != 3             # series: chunked only
     assert gdn.select_kernel(_args(io_dtype=0, dk=64, dv=64)) == 1   # fp32 io -> SIMT
     assert gdn.select_kernel(_args(alpha=0x70000, precond=1, erase=0x50000,
                                    write=0x58000, alpha_per_channel=1)) in (1, 2)
-    assert gdn.select_kernel(_args(S0=0x80000, S_T=0x80000)) in (1, 2)  # S_T may alias S0
+    assert gdn.select_kernel(_args(S0=0x80000, S_T=0x80000)) in (1, 2, 4)  # S_T may alias S0
 
 
 def test_fault_injection_env(monkeypatch):

@@ -128,7 +128,7 @@ def _check_contract(line):
 def test_forward_line_with_backward_object(fake_cuda):
     line = _line("run_gpu")
     _check_contract(line)
-    assert line["roofline"]["bound"] == "hbm" and line["gpu_launches"] == 2      # fused: one launch a step
+    assert line["roofline"]["bound"] == "hbm" and line["gpu_launches"] == 2 * 2  # split kernels: two a step
     b = line["backward"]
     assert "error" not in b, b
     assert b["value"] > 0 and b["gpu_launches"] == 4 * 2 and b["roofline"]["bound"] == "alu"
@@ -163,7 +163,8 @@ def test_e2e_falls_back_to_one_stream(fake_cuda, monkeypatch):
     assert line["e2e"]["value"] > 0 and line["e2e"]["pipeline"].startswith("one stream")
 
 
-@pytest.mark.parametrize("name,kernel", [("plain_fp32", "simt_chunk_kernel"), ("long_context", "fused_kernel"),
+@pytest.mark.parametrize("name,kernel", [("plain_fp32", "simt_chunk_kernel"),
+                                         ("long_context", "keyside_kernel+chain_kernel"),
                                          ("precond_two_gate", "simt_chunk_kernel")])
 def test_other_workload_lines(fake_cuda, monkeypatch, name, kernel):
     import bench

@@ -318,7 +318,8 @@ def test_value_split_invariance(split):
 
 
 @needs_cuda
-def test_tensor_core_repeatable_after_other_kernels():
+@pytest.mark.parametrize("tc_kernel", ["tc_split", "tc"])
+def test_tensor_core_repeatable_after_other_kernels(tc_kernel):
     """Repeated tensor-core calls, each after a SIMT call that leaves other data in
     shared memory, give bit-identical results within the bar: no value may be read
     before it is written, whatever a previous kernel left behind."""
@@ -328,7 +329,7 @@ def test_tensor_core_repeatable_after_other_kernels():
     first = None
     for _ in range(6):
         run_gpu(x, w, o_dtype=torch.float32, kernel="simt", dv_split=1)
-        o, s = run_gpu(x, w, o_dtype=torch.float32, kernel="tc")
+        o, s = run_gpu(x, w, o_dtype=torch.float32, kernel=tc_kernel)
         if first is None:
             first = (o, s)
             so = stats(o, o_ref)

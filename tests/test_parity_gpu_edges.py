@@ -27,45 +27,52 @@ pytestmark = pytest.mark.gpu
 needs_cuda = pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
 
 
-def _check_tc(name, w, seed, **kw):
+KERNELS = ["tc_split", "tc"]   # the split kernels (what AUTO picks here) and the fused one
+
+
+def _check_tc(name, w, seed, kernel, **kw):
     import chunked_gated_delta_14_b200 as gdn
     x = make_inputs(w, seed=seed)
     a = gdn.make_args(B=w.B, T=w.T, H=w.H, dk=w.dk, dv=w.dv, chunk=w.chunk, io_dtype=1, o_dtype=0,
-                      q=1 << 20, k=2 << 20, v=3 << 20, o=4 << 20, kernel=0,
+                      q=1 << 20, k=2 << 20, v=3 << 20, o=4 << 20, kernel=gdn.gdn.KERNELS[kernel],
                       alpha=(5 << 20) if x["alpha"] is not None else None,
                       beta=(6 << 20) if x["beta"] is not None else None)
-    assert gdn.select_kernel(a) == 2, "this case must run on the tensor-core kernel"
+    assert gdn.select_kernel(a) == gdn.gdn.KERNELS[kernel], "this case must run on that tensor-core kernel"
     o_ref, s_ref = run_oracle(x, w)
-    o, s = run_gpu(x, w, o_dtype=torch.float32, kernel="tc", **kw)
+    o, s = run_gpu(x, w, o_dtype=torch.float32, kernel=kernel, **kw)
     so, ss = stats(o, o_ref), stats(s, s_ref)
-    report(name, o=so, S_T=ss)
+    report(f"{name}_{kernel}", o=so, S_T=ss)
     assert so["max_rel_rms"] <= TOL_BF16_REL_RMS, so
     assert ss["max_rel_rms"] <= TOL_BF16_REL_RMS, ss
 
 
 @needs_cuda
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("decay", ["weak", "none"])
 @pytest.mark.parametrize("s0", [0.0, 0.02])
-def test_tc_weak_and_unit_decay(decay, s0):
+def test_tc_weak_and_unit_decay(decay, s0, kernel):
     w = workload("gdn_bf16", B=1, H=16, T=4096, decay=decay, s0_std=s0)
-    _check_tc(f"tc_decay_{decay}_s0_{s0}", w, seed=31)
+    _check_tc(f"tc_decay_{decay}_s0_{s0}", w, 31, kernel)
 
 
 @needs_cuda
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("decay", ["scalar", "weak"])
-def test_tc_unit_beta(decay):
+def test_tc_unit_beta(decay, kernel):
     w = workload("gdn_bf16", B=1, H=16, T=4096, decay=decay, beta=False, s0_std=0.02)
-    _check_tc(f"tc_beta1_decay_{decay}", w, seed=32)
+    _check_tc(f"tc_beta1_decay_{decay}", w, 32, kernel)
 
 
 @needs_cuda
-def test_tc_long_context_weak_decay():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_tc_long_context_weak_decay(kernel):
     w = workload("long_context", decay="weak")
-    _check_tc("tc_long_context_weak", w, seed=33)
+    _check_tc("tc_long_context_weak", w, 33, kernel)
 
 
 @needs_cuda
-def test_tc_ragged_weak_decay():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_tc_ragged_weak_decay(kernel):
     """A ragged length (tail chunk of 17 tokens) with weak decay and S0."""
     w = workload("gdn_bf16", B=2, H=3, T=1041, decay="weak", s0_std=0.02)
-    _check_tc("tc_ragged_weak", w, seed=34)
+    _check_tc("tc_ragged_weak", w, 34, kernel)
