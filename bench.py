@@ -394,7 +394,7 @@ def forward_line(args, rank, world, local_rank, name, over, timed_steps):
                       beta=ptr(d["beta"]), erase=ptr(d["erase"]), write=ptr(d["write"]),
                       precond=int(bool(w.precond)), S0=ptr(d["S0"]), o=o.data_ptr(),
                       S_T=S_T.data_ptr(), mode={"exact": 0, "neumann": 1, "residual": 2}[mode],
-                      neumann_N=N, residual_S=args.S, kernel=0)
+                      neumann_N=N, residual_S=args.S, kernel=gdn.gdn.KERNELS[args.kernel])
     ws = gdn.workspace_for(a, dev)
     if ws is not None:
         a.workspace = ws.data_ptr()
@@ -461,7 +461,8 @@ def forward_line(args, rank, world, local_rank, name, over, timed_steps):
         def run(di, slot):
             gdn.chunk_fwd(di["q"], di["k"], di["v"], di.get("alpha"), di.get("beta"), erase=di.get("erase"),
                           write=di.get("write"), precond=int(bool(w.precond)), S0=di.get("S0"), chunk=w.chunk,
-                          o_dtype=o_dt, out=outs[slot], mode=mode, N=N, S=args.S, S_T=finals[slot])
+                          o_dtype=o_dt, out=outs[slot], mode=mode, N=N, S=args.S, S_T=finals[slot],
+                          kernel=args.kernel)
             return {"o": outs[slot], "S_T": finals[slot]}
 
         n_e2e = args.e2e_steps if timed_steps is not None else max(2, min(args.e2e_steps, steps))
@@ -988,6 +989,8 @@ def main():
                     help="the backward pass (gradients) on the same workload")
     ap.add_argument("--bwd-steps", type=int, default=20,
                     help="backward calls timed for the forward line's 'backward' object (0: none)")
+    ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tc", "tc_split"],
+                    help="force one forward kernel (auto: the library's choice)")
     ap.add_argument("--N", type=int, default=3)
     ap.add_argument("--S", type=int, default=8)
     args = ap.parse_args()

@@ -85,7 +85,7 @@ def fake_cuda(monkeypatch):
 def _line(fn, **over):
     import bench
     args = types.SimpleNamespace(steps=2, warmup=3, e2e_steps=4, cpu_budget=0.2, no_cpu_baseline=False,
-                                 workload="gdn_bf16",
+                                 workload="gdn_bf16", kernel="auto",
                                  batch=1, mode="exact", N=3, S=8, bwd_steps=2, ref_budget=1.0)
     for k, v in over.items():
         setattr(args, k, v)
@@ -98,8 +98,8 @@ def _line(fn, **over):
 def _lines(fn, **over):
     import bench
     args = types.SimpleNamespace(steps=2, warmup=3, e2e_steps=4, cpu_budget=0.2, no_cpu_baseline=False,
-                                 workload="gdn_bf16", batch=1, mode="exact", N=3, S=8, bwd_steps=0,
-                                 ref_budget=1.0)
+                                 workload="gdn_bf16", kernel="auto", batch=1, mode="exact", N=3, S=8,
+                                 bwd_steps=0, ref_budget=1.0)
     for k, v in over.items():
         setattr(args, k, v)
     buf = io.StringIO()
@@ -133,6 +133,12 @@ def test_forward_line_with_backward_object(fake_cuda):
     assert "error" not in b, b
     assert b["value"] > 0 and b["gpu_launches"] == 4 * 2 and b["roofline"]["bound"] == "alu"
     assert fake_cuda["fwd"] > 0 and fake_cuda["bwd"] > 0
+
+
+def test_forward_line_forced_fused_kernel(fake_cuda):
+    line = _line("run_gpu", kernel="tc", bwd_steps=0)
+    _check_contract(line)
+    assert line["config"]["kernel"] == "fused_kernel" and line["gpu_launches"] == 2  # one launch a step
 
 
 def test_backward_line(fake_cuda):

@@ -1,6 +1,7 @@
-"""gdn_chunk_fwd_static_scratch: the tensor-core path with the library's fixed
-scratch array instead of a caller workspace.  Collected last on purpose, so
-that it also runs after every other test has used the device."""
+"""gdn_chunk_fwd_static_scratch: the split tensor-core kernels with the
+library's fixed scratch array instead of a caller workspace, for callers that
+cannot allocate device memory per call.  Collected last on purpose, so that it
+also runs after every other test has used the device."""
 import ctypes
 
 import numpy as np
@@ -40,24 +41,50 @@ def test_static_scratch_rejects_oversize_and_workspace():
     assert G.lib().gdn_chunk_fwd_static_scratch(ctypes.byref(a), None) == G.GDN_ERR_UNSUPPORTED
 
 
+def _free_bytes():
+    free, _ = torch.cuda.mem_get_info()
+    return free
+
+
 @pytest.mark.gpu
-def test_static_scratch_matches_workspace_entry():
-    # 1 x 16 heads x 64 chunks = 1024 chunk-heads: exactly the fixed maximum
-    w = workload("gdn_bf16", B=1, H=16, T=4096, s0_std=0.02)
-    assert w.B * w.H * (w.T // 64) * 24576 == G.STATIC_SCRATCH_BYTES
+@pytest.mark.parametrize("T", [4096, 1000])
+def test_static_scratch_matches_workspace_entry(T):
+    """The fixed-scratch entry runs the split tensor-core kernels on the
+    library's array; the same kernels on a caller workspace must give the same
+    bits, three times in a row, and no call may allocate device memory.
+    T = 4096 fills the array exactly (1 x 16 heads x 64 chunks = 1024
+    chunk-heads); T = 1000 ends in a ragged chunk."""
+    w = workload("gdn_bf16", B=1, H=16, T=T, s0_std=0.02)
+    assert w.B * w.H * (-(-w.T // 64)) * 24576 <= G.STATIC_SCRATCH_BYTES
     x = make_inputs(w, seed=21)
     d = {k: (None if v is None else v.cuda()) for k, v in x.items()}
     o_ref, s_ref = gdn.chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S0=d["S0"],
-                                 o_dtype=torch.float32, kernel="tc")
+                                 o_dtype=torch.float32, kernel="tc_split")
     torch.cuda.synchronize()
     rms_o = float(o_ref.double().pow(2).mean().sqrt())
-    rms_s = float(s_ref.double().pow(2).mean().sqrt())
     stream = torch.cuda.current_stream().cuda_stream
-    for call in range(2):                                    # two calls in a row
-        o = torch.full_like(o_ref, float("nan"))
-        S = torch.full_like(s_ref, float("nan"))
+    outs = [(torch.full_like(o_ref, float("nan")), torch.full_like(s_ref, float("nan"))) for _ in range(3)]
+    torch.cuda.synchronize()
+    # The scratch array is part of the library's device image.  With lazy module
+    # loading (the CUDA default) the driver maps it when the entry point first
+    # takes its address, so the first call may lower free memory by at most the
+    # array (plus the image's code); later calls must change nothing.
+    alloc0, free0 = torch.cuda.memory_allocated(), _free_bytes()
+    G.call_static_scratch(_args(w, d, *outs[0]), stream)
+    gdn.device_check(stream)
+    torch.cuda.synchronize()
+    free1 = _free_bytes()
+    assert 0 <= free0 - free1 <= G.STATIC_SCRATCH_BYTES + (8 << 20), (free0, free1)
+    for o, S in outs[1:]:                                   # two more calls in a row
         G.call_static_scratch(_args(w, d, o, S), stream)
         gdn.device_check(stream)
-        eo = float((o.double() - o_ref.double()).abs().max()) / rms_o
-        es = float((S.double() - s_ref.double()).abs().max()) / rms_s
-        assert eo <= TOL_BF16_REL_RMS and es <= TOL_BF16_REL_RMS, (call, eo, es)
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated() == alloc0
+    assert _free_bytes() == free1, "a call after the first changed the device's free memory"
+    for call, (o, S) in enumerate(outs):
+        assert torch.equal(o, o_ref) and torch.equal(S, s_ref), call
+    # and the split kernels meet the accuracy bar (against the fused kernel's result)
+    o_f, _ = gdn.chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S0=d["S0"],
+                           o_dtype=torch.float32, kernel="tc")
+    torch.cuda.synchronize()
+    assert float((o_f.double() - o_ref.double()).abs().max()) <= TOL_BF16_REL_RMS * rms_o
