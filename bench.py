@@ -497,15 +497,18 @@ def forward_line(args, rank, world, local_rank, name, over, timed_steps):
     accuracy = None
     if mode == "neumann" and rank == 0 and world == 1 and not general:
         # the truncated series against exact inversion (same kernel family, exact mode)
-        # and against the fp64 oracle, on this whole workload
+        # and against the fp64 oracle, on this whole workload; o in fp32 here, so
+        # that the bf16 rounding of the output is not counted as method error
+        o32 = torch.empty((w.B, w.T, w.H, w.dv), device=dev, dtype=torch.float32)
+        a.o, a.o_dtype = o32.data_ptr(), 0
         step()
         torch.cuda.synchronize()
-        o_n = o.double().cpu().numpy()
+        o_n = o32.double().cpu().numpy()
         s_n = S_T.double().cpu().numpy()
         a.mode, a.neumann_N = 0, 0
         step()
         torch.cuda.synchronize()
-        o_x = o.double().cpu().numpy()
+        o_x = o32.double().cpu().numpy()
         s_x = S_T.double().cpu().numpy()
         o_ref, s_ref = oracle_reference(w, x)
         m_o, r_o = max_rel_rms(o_n, o_x)
@@ -516,7 +519,7 @@ def forward_line(args, rank, world, local_rank, name, over, timed_steps):
             vs_exact=dict(o_max_rel_rms=m_o, o_rms_rel=r_o, S_T_max_rel_rms=m_s, S_T_rms_rel=r_s,
                           exact_kernel=kernel_name),
             vs_oracle=dict(o_max_rel_rms=mo_o, o_rms_rel=ro_o, S_T_max_rel_rms=mo_s, S_T_rms_rel=ro_s),
-            tolerance="bf16 bar: max|err| <= 2e-2 * rms(oracle) on o and S_T (o read back in bf16 here)")
+            tolerance="bf16 bar: max|err| <= 2e-2 * rms(oracle) on o and S_T (o in fp32 for this comparison)")
 
     backward = None
     if name == "gdn_bf16" and args.bwd_steps > 0 and world == 1:
