@@ -12,8 +12,9 @@
 //    as fp16: T diag(beta), T diag(beta e^g) and P, 24 KB per chunk-head.
 // 2. chain_kernel -- one CTA per (batch, head, 64-column value slice) walks
 //    the chunks in order with the fp32 state h = S^T (128 x 64) in TMEM.
-//      warp 0      TMA producer: q, k, v slice and the workspace rows (2 stages)
-//      warp 1      TMEM allocation
+//      warp 0      TMA producer: q, k and P into a ring of three stages; the
+//                  v slice, T diag(beta), T diag(beta e^g) into one early slot
+//      warp 1      TMEM allocation, then the output MMAs O += P Delta
 //      warps 2-9   key side of chunk m (runs ahead of the chain): gate scan,
 //                  fp16 operands Q' = diag(e^g) Q, K, V; U = T diag(beta) V and
 //                  W = T diag(beta e^g) K (MMAs); -W to shared memory; K
@@ -22,7 +23,8 @@
 //                  h16 <- h;  h <- e^{g_C} h               (TMEM)
 //                  [-W h ; Q' h] = [-W ; Q'] h16            (MMA)
 //                  Delta = U - W h                          (CUDA cores)
-//                  h += (e^{g_C - g} K)^T Delta, then O = Q'h + P Delta (MMAs)
+//                  h += (e^{g_C - g} K)^T Delta                (MMA)
+//                  O = Q'h + P Delta is finished by warp 1 off the chain
 //    Every MMA is tcgen05.mma kind::f16, M = 128: a 64-row operand is paired
 //    with the 64 rows that follow it in the same stage; the TMEM lanes those
 //    rows produce are never read.  Derived operands are fp16: with bf16 ones
@@ -66,7 +68,7 @@ constexpr int kNeumannMaxN = 15;
 constexpr unsigned long long kWaitLimit = 4000000000ull;   // ~2 s at the boost clock
 
 // error codes recorded in g_tc_error (first one wins)
-enum { E_FULL = 1, E_EMPTY, E_KSREADY, E_KSFREE, E_O, E_UW, E_X, E_H, E_K1_TMA, E_K1_MMA, E_XISS };
+enum { E_FULL = 1, E_EMPTY, E_KSREADY, E_KSFREE, E_O, E_UW, E_X, E_H, E_K1_TMA, E_K1_MMA, E_XISS, E_DREADY };
 
 constexpr uint32_t IDESC_BF_KK = idesc_f16(128, 64, 1, 1, 0, 0);    // bf16, K-major x K-major, N 64
 constexpr uint32_t IDESC_KM64 = idesc_f16(128, 64, 0, 0, 0, 1);     // fp16, K-major x MN-major, N 64
@@ -348,24 +350,32 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
 constexpr int K2_THREADS = 448;    // 14 warps
 constexpr int KS_THREADS = 256, CH_THREADS = 128;
-// stage (x2): per 64-column key block kb: [W | Q | K] at kb * 24 KB, then V,
-//   then T diag(beta), T diag(beta e^g) and P of the chunk
-constexpr uint32_t STG = 81920;
-constexpr uint32_t S_W = 0, S_Q = 8192, S_K = 16384, S_KB = 24576, S_V = 49152;
-constexpr uint32_t S_TB = 57344, S_TBG = 65536, S_P = 73728;
-constexpr uint32_t STAGE_TX = 65536;                   // bytes the producer loads per stage
+// Main stage (x3): per 64-column key block kb: [W | Q | K] at kb * 24 KB, then
+// P.  It holds a chunk from its load until the chain's MMAs of the chunk are
+// complete; three of them let the load of chunk m + 2 start while the key side
+// works on m + 1 and the chain on m.
+constexpr int NSTAGE = 3;
+constexpr uint32_t MSTG = 57344;
+constexpr uint32_t S_W = 0, S_Q = 8192, S_K = 16384, S_KB = 24576, S_P = 49152;
+constexpr uint32_t MAIN_TX = 40960;                    // bytes loaded per main stage: Q, K, P
+// Early slot (x1): T diag(beta), T diag(beta e^g) and the V slice, read only by
+// the U and W MMAs and reloaded as soon as those are complete.
+constexpr uint32_t OFF_EARLY = NSTAGE * MSTG;
+constexpr uint32_t ES_TB = 0, ES_TBG = 8192, ES_V = 16384;
+constexpr uint32_t EARLY_TX = 24576;
 // Every M = 128 MMA whose A operand has only 64 real rows also reads the 8 KB
 // next to them; the lanes those rows produce are never read.  The neighbours
-// all lie in the same stage and are not rewritten while the stage is in use:
-// U reads T diag(beta) + T diag(beta e^g), W reads T diag(beta e^g) + P, the
-// output MMA T diag(beta e^g) + P.
-constexpr uint32_t OFF_HS = 2 * STG;                   // h fp16, 128 rows
+// are not rewritten while the MMA runs: U reads T diag(beta) + T diag(beta e^g),
+// W reads T diag(beta e^g) + V, the output MMA the second K block + P.
+constexpr uint32_t OFF_HS = OFF_EARLY + EARLY_TX;      // h fp16, 128 rows
 constexpr uint32_t OFF_DS = OFF_HS + 16384;            // Delta fp16 x 2
 constexpr uint32_t OFF_PAR = OFF_DS + 2 * 8192;
-constexpr uint32_t PAR_BYTES = (sizeof(ChunkParams) + 15) & ~15u;
-constexpr uint32_t OFF_BAR = OFF_PAR + 3 * PAR_BYTES;   // params ring of 3
-enum { B_FULL = 0, B_EMPTY = 2, B_KSREADY = 4, B_KSFREE = 6, B_UW = 8, B_X = 9, B_H = 10, B_O = 11,
-       B_XISS = 13, N_BARS = 14 };
+constexpr uint32_t PAR_BYTES = (sizeof(tc::ChainParams) + 15) & ~15u;
+constexpr uint32_t OFF_BAR = OFF_PAR + 3 * PAR_BYTES;   // gate ring of 3
+enum { B_FULL = 0, B_EMPTY = 3, B_EFULL = 6, B_EEMPTY = 7, B_KSREADY = 8, B_KSFREE = 10, B_UW = 12, B_X = 13,
+       B_H = 14, B_O = 15, B_XISS = 17, B_DREADY = 18, N_BARS = 20 };
+static_assert((MSTG & 1023) == 0 && (OFF_EARLY & 1023) == 0 && (OFF_HS & 1023) == 0 && (OFF_DS & 1023) == 0,
+              "swizzled tiles on 1024-byte boundaries");
 constexpr uint32_t OFF_MISC = OFF_BAR + N_BARS * 8;     // tmem slot, abort flag, group slots
 constexpr uint32_t SMEM_USED = OFF_MISC + 32;
 constexpr uint32_t K2_SMEM = SMEM_USED + 1024;
@@ -407,7 +417,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC + 4);
-    ChunkParams *params = reinterpret_cast<ChunkParams *>(sm + OFF_PAR);
+    tc::ChainParams *params = reinterpret_cast<tc::ChainParams *>(sm + OFF_PAR);
     const unsigned long long lim = kWaitLimit;
 
     // One warp of a group polls the phase (all its lanes, so the warp stays
@@ -436,12 +446,19 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 
     // ------------------------------------------------------------- setup
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NSTAGE; ++i) {
             mbar_init(&bars[B_FULL + i], 1);
-            mbar_init(&bars[B_EMPTY + i], 1);
+            // a stage is free once the chain's MMAs (X, state update) and warp 1's
+            // output MMAs that read it are complete: one commit from each issuer
+            mbar_init(&bars[B_EMPTY + i], 2);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&bars[B_KSREADY + i], 1);
             mbar_init(&bars[B_KSFREE + i], 1);
+            mbar_init(&bars[B_DREADY + i], 1);
         }
+        mbar_init(&bars[B_EFULL], 1);
+        mbar_init(&bars[B_EEMPTY], 1);
         mbar_init(&bars[B_UW], 1);
         mbar_init(&bars[B_X], 1);
         mbar_init(&bars[B_H], 1);
@@ -468,29 +485,66 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             tma_prefetch_desc(&tm_t);
-            int issued = 0;
+            int issued = 0, issued_early = 0;
             for (int m = 0; m < NC; ++m) {
-                const int s = m & 1;
+                const int ms = m % NSTAGE;
                 const int wrow = (((b * H) + h) * NC + m) * WS_ROWS;
-                if (m >= 2 && !mbar_wait(&bars[B_EMPTY + s], ((m - 2) >> 1) & 1, abort_flag, E_EMPTY, lim))
-                    break;
-                uint64_t *fb = &bars[B_FULL + s];
-                mbar_arrive_expect_tx(fb, STAGE_TX);
-                uint8_t *st = sm + s * STG;
                 const int t0 = m * C;
+                // main stage: free once the chain's MMAs of chunk m - 3 are complete
+                if (m >= NSTAGE &&
+                    !mbar_wait(&bars[B_EMPTY + ms], ((m / NSTAGE) - 1) & 1, abort_flag, E_EMPTY, lim))
+                    break;
+                uint64_t *fb = &bars[B_FULL + ms];
+                mbar_arrive_expect_tx(fb, MAIN_TX);
+                uint8_t *st = sm + ms * MSTG;
                 tma_load_4d(st + S_Q, &tm_q, fb, 0, h, t0, b);
                 tma_load_4d(st + S_KB + S_Q, &tm_q, fb, 64, h, t0, b);
                 tma_load_4d(st + S_K, &tm_k, fb, 0, h, t0, b);
                 tma_load_4d(st + S_KB + S_K, &tm_k, fb, 64, h, t0, b);
-                tma_load_4d(st + S_V, &tm_v, fb, v0, h, t0, b);
-                tma_load_4d(st + S_TB, &tm_t, fb, 0, 0, wrow, 0);
-                tma_load_4d(st + S_TBG, &tm_t, fb, 0, 0, wrow + 64, 0);
                 tma_load_4d(st + S_P, &tm_t, fb, 0, 0, wrow + 128, 0);
                 issued = m + 1;
+                // early slot: free once the U and W MMAs of chunk m - 1 are complete
+                if (m >= 1 && !mbar_wait(&bars[B_EEMPTY], (m - 1) & 1, abort_flag, E_EMPTY, lim)) break;
+                uint64_t *eb = &bars[B_EFULL];
+                mbar_arrive_expect_tx(eb, EARLY_TX);
+                uint8_t *es = sm + OFF_EARLY;
+                tma_load_4d(es + ES_V, &tm_v, eb, v0, h, t0, b);
+                tma_load_4d(es + ES_TB, &tm_t, eb, 0, 0, wrow, 0);
+                tma_load_4d(es + ES_TBG, &tm_t, eb, 0, 0, wrow + 64, 0);
+                issued_early = m + 1;
             }
-            // no copy may still be in flight when the block exits
-            for (int m = issued - 2 < 0 ? 0 : issued - 2; m < issued; ++m)
-                mbar_wait_drain(&bars[B_FULL + (m & 1)], (m >> 1) & 1, lim);
+            // no copy may still be in flight when the block exits: the last load of
+            // each stage, and of the early slot
+            for (int m = issued - NSTAGE < 0 ? 0 : issued - NSTAGE; m < issued; ++m)
+                mbar_wait_drain(&bars[B_FULL + m % NSTAGE], (m / NSTAGE) & 1, lim);
+            if (issued_early > 0) mbar_wait_drain(&bars[B_EFULL], (issued_early - 1) & 1, lim);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ========================================================= output MMAs
+        // O(n) += [preceding rows ; P] Delta(n) into lanes 64..127 of X(n)'s
+        // buffer, once the chain has stored Delta(n) and issued its state update.
+        // Off the chain: its issue no longer holds up the chain's own warps.
+        if (lane == 0) {
+            int opend = -1, opar = 0;
+            for (int n = 0; n < NC; ++n) {
+                const int s = n & 1;
+                if (!mbar_wait_spin(&bars[B_DREADY + s], (n >> 1) & 1, abort_flag, E_DREADY, lim)) break;
+                tc_fence_after();
+                uint8_t *st = sm + (n % NSTAGE) * MSTG;
+                const uint32_t ap = smem_u32(st + S_P) - 8192, bd = smem_u32(sm + OFF_DS + s * 8192);
+                const uint32_t xcol = s ? TM_X1 : TM_X0;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f16_ss(tmem + xcol, sdesc_sw128(ap + kk * 32, 16, 1024),
+                                sdesc_sw128(bd + kk * 2048, 8192, 1024), IDESC_KM64, 1);
+                umma_commit(&bars[B_O + s]);
+                umma_commit(&bars[B_EMPTY + n % NSTAGE]);
+                opend = B_O + s;
+                opar = (n >> 1) & 1;
+            }
+            // error path: no MMA of this role may still be running when TMEM is released
+            if (opend >= 0 && *abort_flag) mbar_wait_drain(&bars[opend], opar, lim);
         }
         __syncwarp();
     } else if (warp >= 2 && warp < 10) {
@@ -506,28 +560,32 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         float ga0 = 1.f, ga1 = 1.f, gb0 = 0.f, gb1 = 0.f;
         if (scan_warp) {
             tc::fetch_gates(p.alpha, p.beta, b, T, H, h, 0, lane, true, ga0, ga1, gb0, gb1);
-            tc::scan_gates(&params[0], ga0, ga1, gb0, gb1, lane, min(C, T));
+            tc::scan_gates_chain(&params[0], ga0, ga1, lane);
             tc::fetch_gates(p.alpha, p.beta, b, T, H, h, C, lane, NC > 1, ga0, ga1, gb0, gb1);
         }
         int kcnt = 0;
         int pend = -1;   // leader: barrier of the last commit not yet known complete
         int pend_par = 0;
         for (int m = 0; m < NC; ++m) {
-            const int s = m & 1;
-            const ChunkParams *par = &params[m % 3];
-            uint8_t *st = sm + s * STG;
-            // chain finished chunk m-2: its stage's W slots and U buffer are free
+            const int s = m & 1, ms = m % NSTAGE;
+            const tc::ChainParams *par = &params[m % 3];
+            uint8_t *st = sm + ms * MSTG;
+            uint8_t *es = sm + OFF_EARLY;
+            // chain finished chunk m-2: the U buffer s is free (the stage's W slots
+            // came free with the stage itself)
             if (m >= 2) group_wait(&bars[B_KSFREE + s], ((m - 2) >> 1) & 1, E_KSFREE, 1, KS_THREADS, lwarp, true);
-            group_wait(&bars[B_FULL + s], (m >> 1) & 1, E_FULL, 1, KS_THREADS, lwarp, true);
+            group_wait(&bars[B_FULL + ms], (m / NSTAGE) & 1, E_FULL, 1, KS_THREADS, lwarp, true);
             if (!sync_ok(1, KS_THREADS, leader, kcnt)) break;
-            // in-place fp16 operands: Q -> e^{g_r} Q, K -> K, V -> V
+            // in-place fp16 operands: Q -> e^{g_r} Q, K -> K in the main stage, then
+            // V in the early slot once it has landed
 #pragma unroll
             for (int it = 0; it < 10; ++it) {
+                if (it == 8) group_wait(&bars[B_EFULL], m & 1, E_FULL, 1, KS_THREADS, lwarp, true);
                 const int u = kt + 256 * (it & 1);          // 16-byte chunk within one 8 KB tile
                 const int tile = it >> 1;                   // Q0, Q1, K0, K1, V
                 const uint32_t off = tile == 0 ? S_Q : tile == 1 ? S_KB + S_Q : tile == 2 ? S_K
-                                   : tile == 3 ? S_KB + S_K : S_V;
-                uint8_t *addr = st + off + (u << 4);
+                                   : tile == 3 ? S_KB + S_K : ES_V;
+                uint8_t *addr = (tile < 4 ? st : es) + off + (u << 4);
                 const int row = u >> 3;
                 const float sc = tile < 2 ? par->eg[row] : 1.f;
                 uint4 w = *reinterpret_cast<uint4 *>(addr);
@@ -548,8 +606,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 // abort: the group leaves at the next wait
             } else if (leader) {
                 tc_fence_after();
-                const uint32_t at = smem_u32(st + S_TB), av = smem_u32(st + S_V);
-                const uint32_t ag = smem_u32(st + S_TBG), ak = smem_u32(st + S_K);
+                const uint32_t at = smem_u32(es + ES_TB), av = smem_u32(es + ES_V);
+                const uint32_t ag = smem_u32(es + ES_TBG), ak = smem_u32(st + S_K);
                 const uint32_t du = tmem + (s ? TM_U1 : TM_U0);
                 // U = T diag(beta) V: [T diag(beta) ; next rows] x V (MN-major), K = 64 tokens
 #pragma unroll
@@ -562,12 +620,13 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     umma_f16_ss(tmem + TM_W, sdesc_sw128(ag + kk * 32, 16, 1024),
                                 sdesc_sw128(ak + kk * 2048, S_KB, 1024), IDESC_KM128, kk > 0);
                 umma_commit(&bars[B_UW]);
+                umma_commit(&bars[B_EEMPTY]);       // the early slot reloads once U and W are formed
                 pend = B_UW; pend_par = m & 1;
             }
             __syncwarp();
             // gates of the next chunk meanwhile
             if (scan_warp && m + 1 < NC) {
-                tc::scan_gates(&params[(m + 1) % 3], ga0, ga1, gb0, gb1, lane, min(C, T - (m + 1) * C));
+                tc::scan_gates_chain(&params[(m + 1) % 3], ga0, ga1, lane);
                 tc::fetch_gates(p.alpha, p.beta, b, T, H, h, (m + 2) * C, lane, m + 2 < NC, ga0, ga1, gb0, gb1);
             }
             group_wait(&bars[B_UW], m & 1, E_UW, 1, KS_THREADS, lwarp, false);
@@ -678,18 +737,24 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             }
             __syncwarp();
         };
+        // every chain warp polls a phase itself (all lanes, so the warp stays converged)
+        auto warp_wait = [&](uint64_t *bar, uint32_t parity, int code) {
+            const bool ok = mbar_wait_spin(bar, parity, abort_flag, code, lim);
+            __syncwarp();
+            return ok;
+        };
         int ccnt = 0, dcnt = 0;
         int pend = -1, pend_par = 0;       // issuer: last commit not yet known complete
         bool done = true;
         for (int n = 0; n < NC; ++n) {
             const int s = n & 1;
-            const ChunkParams *par = &params[n % 3];
-            uint8_t *st = sm + s * STG;
+            const tc::ChainParams *par = &params[n % 3];
+            uint8_t *st = sm + (n % NSTAGE) * MSTG;
             const uint32_t xcol = s ? TM_X1 : TM_X0;
             // state update of the previous chunk complete (its output rows may still be running)
-            if (n > 0) group_wait(&bars[B_H], (n - 1) & 1, E_H, 2, CH_THREADS, iwarp, false);
+            if (n > 0) warp_wait(&bars[B_H], (n - 1) & 1, E_H);
             // the gates of chunk 0 are scanned by the key side at start-up: wait for it
-            else group_wait(&bars[B_KSREADY], 0, E_KSREADY, 2, CH_THREADS, iwarp, false);
+            else warp_wait(&bars[B_KSREADY], 0, E_KSREADY);
             tc_fence_after();
             // ---- h <- e^{g_C} h in TMEM (issued first), h -> fp16 operand.  The
             // gates of chunk n > 0 were scanned before the key side released chunk n-1.
@@ -709,7 +774,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            if (n > 0) group_wait(&bars[B_KSREADY + s], (n >> 1) & 1, E_KSREADY, 2, CH_THREADS, iwarp, false);
+            // Only the MMAs read the key side's operands of chunk n: the issuing warp
+            // waits for them, and the barrier then orders every chain warp after that
+            // acquire (the gates of chunk n + 1, which the next c1 reads, were scanned
+            // before the key side released chunk n).
+            if (iwarp) warp_wait(&bars[B_KSREADY + s], (n >> 1) & 1, E_KSREADY);
             if (!sync_ok(2, CH_THREADS, issuer, ccnt)) { done = false; break; }
             if (issuer) {
                 // [-W ; Q'] h16: lanes 0..63 -W h, lanes 64..127 Q'h
@@ -731,7 +800,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 if (n > 0) out_rows(n - 1);
                 continue;
             }
-            group_wait(&bars[B_X], n & 1, E_X, 3, 64, iwarp, false);
+            warp_wait(&bars[B_X], n & 1, E_X);
             tc_fence_after();
             // ---- Delta = U - W h (rows in lanes 0..63) -> fp16 operands
             {
@@ -750,30 +819,24 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             if (sync_ok(3, 64, issuer, dcnt) && issuer) {
                 tc_fence_after();
                 const uint32_t ak = smem_u32(st + S_K), bd = smem_u32(sm + OFF_DS + s * 8192);
-                // h += (diag(e^{g_C - g}) K)^T Delta first: the next chunk waits on it
-                // alone.  The key side rescaled K in place; K^T as MN-major A over
-                // the two key blocks.
+                // h += (diag(e^{g_C - g}) K)^T Delta: the next chunk waits on it alone.
+                // The key side rescaled K in place; K^T as MN-major A over the two key
+                // blocks.  The output MMAs of this chunk are warp 1's.
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     umma_f16_ss(tmem + TM_H, sdesc_sw128(ak + kk * 2048, S_KB, 1024),
                                 sdesc_sw128(bd + kk * 2048, 8192, 1024), IDESC_MM64, 1);
                 umma_commit(&bars[B_H]);
-                // O: [preceding rows ; P] Delta -> lanes 64..127 += P Delta.  The stage and
-                // the key side's buffers are released only after these MMAs complete.
-                const uint32_t ap = smem_u32(st + S_P) - 8192;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16_ss(tmem + xcol, sdesc_sw128(ap + kk * 32, 16, 1024),
-                                sdesc_sw128(bd + kk * 2048, 8192, 1024), IDESC_KM64, 1);
-                umma_commit(&bars[B_O + s]);
-                umma_commit(&bars[B_EMPTY + s]);
-                umma_commit(&bars[B_KSFREE + s]);
-                pend = B_O + s; pend_par = (n >> 1) & 1;
+                umma_commit(&bars[B_EMPTY + n % NSTAGE]);   // X and the state update have read the stage
+                umma_commit(&bars[B_KSFREE + s]);            // and Delta has read U
+                tc_fence_before();
+                mbar_arrive(&bars[B_DREADY + s]);
+                pend = B_H; pend_par = n & 1;
             }
             __syncwarp();
         }
         if (done && NC > 0) {
-            group_wait(&bars[B_H], (NC - 1) & 1, E_H, 2, CH_THREADS, iwarp, false);
+            warp_wait(&bars[B_H], (NC - 1) & 1, E_H);
             if (sync_ok(2, CH_THREADS, issuer, ccnt)) {
                 tc_fence_after();
                 if (!rowpart) out_rows(NC - 1);

@@ -115,6 +115,32 @@ __device__ __forceinline__ void scan_gates(ChunkParams *par, float a0, float a1,
     }
 }
 
+// The gate factors the chain kernel reads: e^{g_r} (Q'), e^{g_C - g_r} (K') and
+// e^{g_C} (the state decay), the same arithmetic as scan_gates.
+struct ChainParams {
+    float eg[C];
+    float egc[C];
+    float egC;
+    float pad[3];
+};
+
+__device__ __forceinline__ void scan_gates_chain(ChainParams *par, float a0, float a1, int lane) {
+    float x0 = lg2_approx(a0), x1 = lg2_approx(a1);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y0 = __shfl_up_sync(0xffffffffu, x0, o);
+        const float y1 = __shfl_up_sync(0xffffffffu, x1, o);
+        if (lane >= o) { x0 += y0; x1 += y1; }
+    }
+    x1 += __shfl_sync(0xffffffffu, x0, 31);
+    const float gC = __shfl_sync(0xffffffffu, x1, 31);
+    par->eg[lane] = ex2_approx(x0);
+    par->eg[lane + 32] = ex2_approx(x1);
+    par->egc[lane] = ex2_approx(gC - x0);
+    par->egc[lane + 32] = ex2_approx(gC - x1);
+    if (lane == 0) par->egC = ex2_approx(gC);
+}
+
 // Decay factors exp(g_r - g_i) of row r for the 32 columns [32 hf, 32 hf + 32),
 // columns right of r zero.  No per-element exponential: 16-blocks left of r's
 // block as 2^(g_r - g_blockend) * dblk[i], r's own block as a running product
