@@ -573,28 +573,61 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             uint8_t *es = sm + OFF_EARLY;
             // chain finished chunk m-2: the U buffer s is free (the stage's W slots
             // came free with the stage itself)
-            if (m >= 2) group_wait(&bars[B_KSFREE + s], ((m - 2) >> 1) & 1, E_KSFREE, 1, KS_THREADS, lwarp, true);
-            group_wait(&bars[B_FULL + ms], (m / NSTAGE) & 1, E_FULL, 1, KS_THREADS, lwarp, true);
+            // one warp polls both phases, one barrier releases the group; the other
+            // warps then take the acquire of the loaded tiles with one test
+            if (lwarp) {
+                if (m >= 2) mbar_wait(&bars[B_KSFREE + s], ((m - 2) >> 1) & 1, abort_flag, E_KSFREE, lim);
+                mbar_wait(&bars[B_FULL + ms], (m / NSTAGE) & 1, abort_flag, E_FULL, lim);
+                __syncwarp();
+            }
             if (!sync_ok(1, KS_THREADS, leader, kcnt)) break;
+            if (!lwarp) mbar_try_wait(&bars[B_FULL + ms], (m / NSTAGE) & 1);
             // in-place fp16 operands: Q -> e^{g_r} Q, K -> K in the main stage, then
-            // V in the early slot once it has landed
+            // V in the early slot once it has landed.  Every load of a pass is
+            // issued before the first store, so they overlap instead of waiting on
+            // one another.
+            auto convert = [&](uint8_t *const (&addr)[8], const float (&sc)[8], int cnt) {
+                uint4 w[8];
 #pragma unroll
-            for (int it = 0; it < 10; ++it) {
-                if (it == 8) group_wait(&bars[B_EFULL], m & 1, E_FULL, 1, KS_THREADS, lwarp, true);
-                const int u = kt + 256 * (it & 1);          // 16-byte chunk within one 8 KB tile
-                const int tile = it >> 1;                   // Q0, Q1, K0, K1, V
-                const uint32_t off = tile == 0 ? S_Q : tile == 1 ? S_KB + S_Q : tile == 2 ? S_K
-                                   : tile == 3 ? S_KB + S_K : ES_V;
-                uint8_t *addr = (tile < 4 ? st : es) + off + (u << 4);
-                const int row = u >> 3;
-                const float sc = tile < 2 ? par->eg[row] : 1.f;
-                uint4 w = *reinterpret_cast<uint4 *>(addr);
-                const float2 f0 = unpack_bf2(w.x), f1 = unpack_bf2(w.y), f2 = unpack_bf2(w.z), f3 = unpack_bf2(w.w);
-                w.x = pack_h2(f0.x * sc, f0.y * sc);
-                w.y = pack_h2(f1.x * sc, f1.y * sc);
-                w.z = pack_h2(f2.x * sc, f2.y * sc);
-                w.w = pack_h2(f3.x * sc, f3.y * sc);
-                *reinterpret_cast<uint4 *>(addr) = w;
+                for (int i = 0; i < 8; ++i)
+                    if (i < cnt) w[i] = *reinterpret_cast<const uint4 *>(addr[i]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (i < cnt) {
+                        const float2 f0 = unpack_bf2(w[i].x), f1 = unpack_bf2(w[i].y);
+                        const float2 f2 = unpack_bf2(w[i].z), f3 = unpack_bf2(w[i].w);
+                        uint4 o;
+                        o.x = pack_h2(f0.x * sc[i], f0.y * sc[i]);
+                        o.y = pack_h2(f1.x * sc[i], f1.y * sc[i]);
+                        o.z = pack_h2(f2.x * sc[i], f2.y * sc[i]);
+                        o.w = pack_h2(f3.x * sc[i], f3.y * sc[i]);
+                        *reinterpret_cast<uint4 *>(addr[i]) = o;
+                    }
+                }
+            };
+            {
+                uint8_t *addr[8];
+                float sc[8];
+#pragma unroll
+                for (int it = 0; it < 8; ++it) {
+                    const int u = kt + 256 * (it & 1);      // 16-byte chunk within one 8 KB tile
+                    const int tile = it >> 1;               // Q0, Q1, K0, K1
+                    const uint32_t off = tile == 0 ? S_Q : tile == 1 ? S_KB + S_Q : tile == 2 ? S_K : S_KB + S_K;
+                    addr[it] = st + off + (u << 4);
+                    sc[it] = tile < 2 ? par->eg[u >> 3] : 1.f;
+                }
+                convert(addr, sc, 8);
+            }
+            group_wait(&bars[B_EFULL], m & 1, E_FULL, 1, KS_THREADS, lwarp, true);
+            {
+                uint8_t *addr[8];
+                float sc[8];
+#pragma unroll
+                for (int it = 0; it < 8; ++it) {
+                    addr[it] = es + ES_V + ((kt + 256 * (it & 1)) << 4);
+                    sc[it] = 1.f;
+                }
+                convert(addr, sc, 2);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -643,19 +676,25 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             } else {
                 // W has read K: K -> diag(e^{g_C - g}) K in place for the state update
                 const int t2 = 64 * hf + 32 * (sp - 2) + lane;
+                uint8_t *addr[8];
+                uint4 w[8];
 #pragma unroll
                 for (int it = 0; it < 8; ++it) {
                     const int idx = t2 + 128 * it;               // 16-byte chunk of the two K blocks
-                    const int u = idx & 511;
-                    uint8_t *addr = st + (idx >> 9) * S_KB + S_K + (u << 4);
-                    const float sc = par->egc[u >> 3];
-                    uint4 w = *reinterpret_cast<uint4 *>(addr);
-                    const float2 f0 = unpack_h2(w.x), f1 = unpack_h2(w.y), f2 = unpack_h2(w.z), f3 = unpack_h2(w.w);
-                    w.x = pack_h2(f0.x * sc, f0.y * sc);
-                    w.y = pack_h2(f1.x * sc, f1.y * sc);
-                    w.z = pack_h2(f2.x * sc, f2.y * sc);
-                    w.w = pack_h2(f3.x * sc, f3.y * sc);
-                    *reinterpret_cast<uint4 *>(addr) = w;
+                    addr[it] = st + (idx >> 9) * S_KB + S_K + ((idx & 511) << 4);
+                    w[it] = *reinterpret_cast<const uint4 *>(addr[it]);
+                }
+#pragma unroll
+                for (int it = 0; it < 8; ++it) {
+                    const float sc = par->egc[((t2 + 128 * it) & 511) >> 3];
+                    const float2 f0 = unpack_h2(w[it].x), f1 = unpack_h2(w[it].y);
+                    const float2 f2 = unpack_h2(w[it].z), f3 = unpack_h2(w[it].w);
+                    uint4 o;
+                    o.x = pack_h2(f0.x * sc, f0.y * sc);
+                    o.y = pack_h2(f1.x * sc, f1.y * sc);
+                    o.z = pack_h2(f2.x * sc, f2.y * sc);
+                    o.w = pack_h2(f3.x * sc, f3.y * sc);
+                    *reinterpret_cast<uint4 *>(addr[it]) = o;
                 }
             }
             fence_proxy_async_smem();
