@@ -255,7 +255,9 @@ uint64_t gdn_workspace_bytes(const gdn_fwd_args *args) {
     int kern = 0;
     if (resolve(args, &p, &kern) != GDN_OK) return 0;
     g_msg[0] = 0;
-    return kern == GDN_KERNEL_TC_SPLIT ? (uint64_t)gdn::tc_workspace_bytes(p) : 0;
+    if (kern == GDN_KERNEL_TC_SPLIT) return (uint64_t)gdn::tc_workspace_bytes(p);
+    if (kern == GDN_KERNEL_SIMT) return (uint64_t)gdn::simt_workspace_bytes(p);
+    return 0;
 }
 
 int32_t gdn_select_kernel(const gdn_fwd_args *args) {
@@ -300,7 +302,11 @@ gdn_status gdn_chunk_fwd(const gdn_fwd_args *args, void *stream) {
     } else if (kern == GDN_KERNEL_RECURRENT) {
         e = gdn::launch_recurrent(p, st);
     } else {
-        e = gdn::launch_simt(p, st);
+        const size_t need = gdn::simt_workspace_bytes(p);
+        if (!args->workspace || args->workspace_bytes < need)
+            return fail(GDN_ERR_INVALID_ARG, "the SIMT kernels need a workspace of %zu bytes (got %llu)", need,
+                        (unsigned long long)args->workspace_bytes);
+        e = gdn::launch_simt(p, args->workspace, st);
     }
     if (e != cudaSuccess)
         return fail(GDN_ERR_CUDA, "%s launch: %s %s",

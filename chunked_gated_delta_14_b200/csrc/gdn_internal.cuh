@@ -38,7 +38,10 @@ bool recurrent_supports(const FwdParams &p, const char **why);
 cudaError_t launch_recurrent(const FwdParams &p, cudaStream_t stream);
 
 size_t simt_smem_bytes(const FwdParams &p);
-cudaError_t launch_simt(const FwdParams &p, cudaStream_t stream);
+// Workspace of the SIMT path: per chunk-head the state-independent matrices
+// (fp32), plus the preconditioner's running average at chunk starts.
+size_t simt_workspace_bytes(const FwdParams &p);
+cudaError_t launch_simt(const FwdParams &p, void *workspace, cudaStream_t stream);
 
 // Tensor-core kernel (tcgen05 / TMEM / TMA).
 bool tc_supports(const FwdParams &p, const char **why);

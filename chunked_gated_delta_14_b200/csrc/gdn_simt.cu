@@ -1,7 +1,7 @@
-// fp32 CUDA-core chunk kernel for every variant of the chunkwise gated
-// delta rule.  One block per (batch, head, value slice) walks the chunks of
-// its sequence in order and carries the fp32 state h = S^T (dk x dvs) in
-// shared memory.  Per chunk of C tokens (local rows r, keys i):
+// fp32 CUDA-core path of the chunkwise gated delta rule, for every variant
+// (any chunk 16-128, d 16-128, fp32 io, the two-gate rule with per-channel
+// decay, gates and the preconditioner).  Per chunk of C tokens (local rows r,
+// keys i):
 //
 //   scalar decay (gated delta rule):
 //     g_r = sum_{i<=r} log alpha_i
@@ -18,6 +18,18 @@
 //     R_r  = u_r - h^T (e_r (.) e^{G_{r-1}})
 //     O_r  = h^T (q_r (.) e^{G_r}) + sum_{i<=r} [sum_c q_rc kw_ic exp(G_rc - G_ic)] Delta_i
 //     h   <- diag(e^{G_last}) h + sum_r (kw_r (.) e^{G_last - G_r}) Delta_r^T
+//
+// Both are one form, Delta = TB (U - E h), O = Q' h + P Delta,
+// h <- diag(d) h + K''^T Delta, whose matrices TB (T diag(beta), or T), P, E,
+// Q', K'' and d depend on the keys and gates only.  So the path is two kernels:
+//
+// 1. simt_prep_kernel -- one block per (chunk, head, batch), all chunks at
+//    once: gates, L, T, and the six matrices into the workspace (fp32).  The
+//    preconditioner's running average is carried across chunks; a scan kernel
+//    (rho_scan_kernel) gives each chunk its value at the chunk start first.
+// 2. simt_chain_kernel -- one block per (batch, head, value slice) walks the
+//    chunks in order with the fp32 state h = S^T (dk x dvs) in shared memory,
+//    reading each matrix once per chunk.
 //
 // The triangular inverse T = (I - A)^-1 with A strictly lower triangular and
 // its truncated Neumann form with the structural mask follow "Quando o 'Bom o
@@ -54,31 +66,71 @@ __device__ __forceinline__ void st_s(S *a, int i, float x) {
     else a[i] = x;
 }
 
-// Shared-memory carve-up, identical on host and device.
-struct SimtLayout {
-    size_t kx, qx, ex, gx, tp, band, hs, ux, dx, rows, rho, total;
-};
-
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
 
-__host__ __device__ inline SimtLayout simt_layout(int C, int dk, int dvs, int N, int neumann,
-                                                  int general, int key_bytes) {
-    SimtLayout L{};
+// Workspace: per chunk-head, fp32 [TB C x C | P C x C | E C x dk | Q' C x dk |
+// K'' C x dk | d dk], padded to 16 bytes; then, for the preconditioned two-gate
+// rule, the running average at every chunk start, [B, H, chunks, dk].
+struct SimtWs {
+    size_t tb, pp, e, q, k, d, stride;   // floats
+};
+
+__host__ __device__ inline SimtWs simt_ws(int C, int dk) {
+    SimtWs w;
+    w.tb = 0;
+    w.pp = (size_t)C * C;
+    w.e = 2 * (size_t)C * C;
+    w.q = w.e + (size_t)C * dk;
+    w.k = w.q + (size_t)C * dk;
+    w.d = w.k + (size_t)C * dk;
+    w.stride = (w.d + dk + 3) & ~size_t(3);
+    return w;
+}
+
+// Row stride (elements) of a C x dk key matrix in shared memory: one extra
+// 32-bit word per row, so that a warp reading channel c of 32 consecutive rows
+// touches 32 distinct banks.
+__host__ __device__ inline int key_stride(int dk, int elem_bytes) { return dk + 4 / elem_bytes; }
+
+// Shared-memory carve-up of the prep kernel, identical on host and device.
+struct PrepLayout {
+    size_t kx, qx, ex, gx, tp, band, rows, total;
+};
+
+__host__ __device__ inline PrepLayout prep_layout(int C, int dk, int N, int neumann, int general,
+                                                  int key_bytes) {
+    PrepLayout L{};
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t at = off; off = align16(off + bytes); return at; };
     // general: kw, q, e, G all fp32; scalar: k, q stored in the io dtype
     const size_t kb = general ? 4 : (size_t)key_bytes;
-    L.kx = take((size_t)C * dk * kb);
-    L.qx = take((size_t)C * dk * kb);
-    L.ex = general ? take((size_t)C * dk * 4) : off;
-    L.gx = general ? take((size_t)C * dk * 4) : off;
+    const size_t ks = key_stride(dk, (int)kb);
+    L.kx = take((size_t)C * ks * kb);
+    L.qx = take((size_t)C * ks * kb);
+    L.ex = general ? take((size_t)C * ks * 4) : off;
+    L.gx = general ? take((size_t)C * ks * 4) : off;
     L.tp = take((size_t)C * C * 4);
     L.band = neumann ? take((size_t)2 * C * (N + 1) * 4) : off;
+    L.rows = take((size_t)4 * C * 4);        // g / log alpha, beta, lrow, spare
+    L.total = off;
+    return L;
+}
+
+// Shared-memory carve-up of the chain kernel.
+struct ChainLayout {
+    size_t hs, ux, dx, ox, mat, dl, total;
+};
+
+__host__ __device__ inline ChainLayout chain_layout(int C, int dk, int dvs) {
+    ChainLayout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t at = off; off = align16(off + bytes); return at; };
     L.hs = take((size_t)dk * dvs * 4);
     L.ux = take((size_t)C * dvs * 4);
     L.dx = take((size_t)C * dvs * 4);
-    L.rows = take((size_t)4 * C * 4);        // g / log alpha, beta, lrow, spare
-    L.rho = general ? take((size_t)dk * 4) : off;
+    L.ox = take((size_t)C * dvs * 4);
+    L.mat = take((size_t)C * (C > dk ? C : dk) * 4);
+    L.dl = take((size_t)dk * 4);
     L.total = off;
     return L;
 }
@@ -100,57 +152,253 @@ __device__ void warp0_inclusive_scan(float *x, int n) {
     }
 }
 
+// The preconditioner's running average rho_t = decay rho_{t-1} + k_t (.) k_t,
+// per (batch, head, key channel), recorded at every chunk start.
+__global__ void rho_scan_kernel(const FwdParams p, float *rho_start) {
+    const int h = blockIdx.x, b = blockIdx.y, c = threadIdx.x;
+    if (c >= p.dk) return;
+    const int NC = (p.T + p.C - 1) / p.C;
+    float rh = 0.f;
+    for (int n = 0; n < NC; ++n) {
+        rho_start[(((size_t)b * p.H + h) * NC + n) * p.dk + c] = rh;
+        const int t0 = n * p.C, t1 = min(p.T, t0 + p.C);
+#pragma unroll 4
+        for (int t = t0; t < t1; ++t) {
+            const float kv = load_in(p.k, (((size_t)b * p.T + t) * p.H + h) * p.dk + c, p.io_bf16);
+            rh = p.rho_decay * rh + kv * kv;
+        }
+    }
+}
+
+// One block per (chunk, head, batch): the state-independent matrices of one chunk.
 template <typename KS, bool GENERAL>
 __global__ void __launch_bounds__(kThreads)
-simt_chunk_kernel(const FwdParams p) {
+simt_prep_kernel(const FwdParams p, float *ws) {
     extern __shared__ __align__(16) unsigned char smem[];
-    const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int C = p.C, dk = p.dk, dv = p.dv, dvs = p.dvs, H = p.H, T = p.T;
-    const int v0 = slice * dvs;
+    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int C = p.C, dk = p.dk, H = p.H, T = p.T;
+    const int NC = (T + C - 1) / C;
+    const int t0 = n * C, Cv = min(C, T - t0);
     const int tid = threadIdx.x;
     const int neumann = (p.mode == GDN_INV_NEUMANN);
     const int N = p.N;
-    const SimtLayout Ly = simt_layout(C, dk, dvs, N, neumann, GENERAL ? 1 : 0,
-                                      (int)sizeof(KS));
+    const PrepLayout Ly = prep_layout(C, dk, N, neumann, GENERAL ? 1 : 0, (int)sizeof(KS));
+    // key rows padded by one word: threads that read the same channel of
+    // consecutive rows then hit distinct banks
+    const int ks = key_stride(dk, GENERAL ? 4 : (int)sizeof(KS));
     KS *kx = reinterpret_cast<KS *>(smem + Ly.kx);       // keys (write keys kw)
     KS *qx = reinterpret_cast<KS *>(smem + Ly.qx);       // read keys
     float *ex = reinterpret_cast<float *>(smem + Ly.ex); // erase keys (two-gate)
     float *gx = reinterpret_cast<float *>(smem + Ly.gx); // per-channel cumulative log decay
-    float *tp = reinterpret_cast<float *>(smem + Ly.tp); // L -> T -> P, C x C
+    float *tp = reinterpret_cast<float *>(smem + Ly.tp); // L -> T, C x C
     float *band = reinterpret_cast<float *>(smem + Ly.band);
-    float *hs = reinterpret_cast<float *>(smem + Ly.hs); // state h, dk x dvs
-    float *ux = reinterpret_cast<float *>(smem + Ly.ux); // values -> R
-    float *dx = reinterpret_cast<float *>(smem + Ly.dx); // Delta
     float *rows = reinterpret_cast<float *>(smem + Ly.rows);
     float *g = rows;                 // scalar: log alpha -> cumulative g
     float *bet = rows + C;           // scalar: beta
     float *lrow = rows + 2 * C;      // forward-substitution row copy
-    float *rho = reinterpret_cast<float *>(smem + Ly.rho);
-
     const size_t bh = (size_t)b * H + h;
-    // initial state
+    const SimtWs W = simt_ws(C, dk);
+    float *out = ws + (bh * NC + n) * W.stride;
+
+    // ---------------------------------------------------------- load
+    for (int idx = tid; idx < C * dk; idx += kThreads) {
+        const int r = idx / dk, c = idx % dk;
+        const size_t gi = (((size_t)b * T + t0 + r) * H + h) * dk + c;
+        const bool ok = r < Cv;
+        const int si = r * ks + c;
+        st_s(kx, si, ok ? load_in(p.k, gi, p.io_bf16) : 0.f);
+        st_s(qx, si, ok ? load_in(p.q, gi, p.io_bf16) : 0.f);
+        if (GENERAL) {
+            ex[si] = ok ? (p.erase ? load_in(p.erase, gi, p.io_bf16) : 1.f) : 0.f;
+            gx[si] = (ok && p.alpha) ? logf(p.alpha[p.alpha_pc ? gi : gi / dk]) : 0.f;
+        }
+    }
+    if (!GENERAL) {
+        for (int r = tid; r < C; r += kThreads) {
+            const size_t ti = ((size_t)b * T + t0 + r) * H + h;
+            g[r] = (r < Cv && p.alpha) ? logf(p.alpha[ti]) : 0.f;
+            bet[r] = (r < Cv) ? (p.beta ? p.beta[ti] : 1.f) : 0.f;
+        }
+    }
+    __syncthreads();
+    // ------------------------------------------- gates and scans
+    if (GENERAL) {
+        // per channel: preconditioner average (from the chunk start), write
+        // key, erase key, cumulative log decay.  Preconditioner factor f(rho):
+        // 1 1/sqrt(rho+eps), 2 1/(rho+eps) (Diag(A)^-1), 3 the latter squashed
+        // into [1/x, x] on a log scale; applied to the write key (forms 2, 3
+        // read the state with the raw key) or to the query
+        const float lnx = p.precond == 3 ? logf(p.precond_x) : 1.f;
+        const float *rho0 = ws + (size_t)p.B * H * NC * W.stride;
+        for (int c = tid; c < dk; c += kThreads) {
+            float rh = p.precond ? rho0[(bh * NC + n) * dk + c] : 0.f, G = 0.f;
+            for (int r = 0; r < C; ++r) {
+                const int idx = r * ks + c;
+                const float kv = ld_s(kx, idx);
+                float f = 1.f;
+                if (p.precond && r < Cv) {
+                    rh = p.rho_decay * rh + kv * kv;
+                    const float a = rh + p.rho_eps;
+                    f = p.precond == 1 ? rsqrtf(a)
+                      : p.precond == 2 ? 1.f / a
+                      : expf(lnx * tanhf(-logf(a) / lnx));
+                }
+                if (p.precond_query) {
+                    st_s(qx, idx, ld_s(qx, idx) * f);
+                    ex[idx] *= kv;
+                } else {
+                    const float kw = kv * f;
+                    st_s(kx, idx, kw);
+                    ex[idx] *= (p.precond == 1 ? kw : kv);
+                }
+                G += gx[idx];
+                gx[idx] = G;
+            }
+        }
+    } else {
+        warp0_inclusive_scan(g, C);
+    }
+    __syncthreads();
+    // ------------------------------------------------ L (strictly lower)
+    for (int idx = tid; idx < C * C; idx += kThreads) {
+        const int r = idx / C, i = idx % C;
+        float val = 0.f;
+        if (i < r) {
+            float acc = 0.f;
+            if (GENERAL) {
+                for (int c = 0; c < dk; ++c)
+                    acc += ex[r * ks + c] * ld_s(kx, i * ks + c) *
+                           expf(gx[(r - 1) * ks + c] - gx[i * ks + c]);
+                val = acc;
+            } else {
+                for (int c = 0; c < dk; ++c) acc += ld_s(kx, r * ks + c) * ld_s(kx, i * ks + c);
+                val = bet[r] * expf(g[r] - g[i]) * acc;
+            }
+        }
+        tp[idx] = val;
+    }
+    __syncthreads();
+    // ------------------------------------------------ T = (I + L)^-1
+    if (!neumann) {
+        // forward substitution, one row at a time: T_rc = -sum_{c<=i<r} L_ri T_ic
+        for (int r = 1; r < C; ++r) {
+            if (tid < r) lrow[tid] = tp[r * C + tid];
+            __syncthreads();
+            if (tid < r) {
+                const int c = tid;
+                float s = lrow[c];
+                for (int i = c + 1; i < r; ++i) s += lrow[i] * tp[i * C + c];
+                tp[r * C + c] = -s;
+            }
+            __syncthreads();
+        }
+        for (int r = tid; r < C; r += kThreads) tp[r * C + r] = 1.f;
+    } else {
+        // Horner on the band: T <- M (.) (I + A T), A = -L, T^(0) = I.
+        // band[i*(N+1)+d] holds T_{i,i-d}.
+        const int Wd = N + 1;
+        float *cur = band, *nxt = band + (size_t)C * Wd;
+        for (int idx = tid; idx < C * Wd; idx += kThreads) cur[idx] = (idx % Wd == 0) ? 1.f : 0.f;
+        __syncthreads();
+        for (int step = 0; step < N; ++step) {
+            for (int idx = tid; idx < C * Wd; idx += kThreads) {
+                const int i = idx / Wd, d = idx % Wd, j = i - d;
+                float val = 0.f;
+                if (j >= 0) {
+                    val = (d == 0) ? 1.f : 0.f;
+                    // sum_{k=j}^{i-1} A_ik T_kj with T_kj in band (k - j <= N)
+                    const int kmax = min(i - 1, j + N);
+                    for (int kk = j; kk <= kmax; ++kk) val -= tp[i * C + kk] * cur[kk * Wd + (kk - j)];
+                }
+                nxt[idx] = val;
+            }
+            __syncthreads();
+            float *sw = cur; cur = nxt; nxt = sw;
+        }
+        for (int idx = tid; idx < C * C; idx += kThreads) {
+            const int i = idx / C, j = idx % C, d = i - j;
+            tp[idx] = (d >= 0 && d <= N) ? cur[i * Wd + d] : 0.f;
+        }
+    }
+    __syncthreads();
+    // ------------------------------------------------ the chunk's matrices
+    // TB = T diag(beta) (scalar rule; the two-gate rule has no beta)
+    for (int idx = tid; idx < C * C; idx += kThreads)
+        out[W.tb + idx] = GENERAL ? tp[idx] : tp[idx] * bet[idx % C];
+    // P: decayed causal scores
+    for (int idx = tid; idx < C * C; idx += kThreads) {
+        const int r = idx / C, i = idx % C;
+        float val = 0.f;
+        if (i <= r) {
+            float acc = 0.f;
+            if (GENERAL) {
+                for (int c = 0; c < dk; ++c)
+                    acc += ld_s(qx, r * ks + c) * ld_s(kx, i * ks + c) *
+                           expf(gx[r * ks + c] - gx[i * ks + c]);
+                val = acc;
+            } else {
+                for (int c = 0; c < dk; ++c) acc += ld_s(qx, r * ks + c) * ld_s(kx, i * ks + c);
+                val = expf(g[r] - g[i]) * acc;
+            }
+        }
+        out[W.pp + idx] = val;
+    }
+    // E (the state read), Q' (the output read), K'' (the state write)
+    for (int idx = tid; idx < C * dk; idx += kThreads) {
+        const int r = idx / dk, c = idx % dk, si = r * ks + c;
+        if (GENERAL) {
+            const float Gl = gx[(C - 1) * ks + c];
+            out[W.e + idx] = ex[si] * ((r > 0) ? expf(gx[si - ks]) : 1.f);
+            out[W.q + idx] = ld_s(qx, si) * expf(gx[si]);
+            out[W.k + idx] = ld_s(kx, si) * expf(Gl - gx[si]);
+        } else {
+            const float gl = g[C - 1];
+            out[W.e + idx] = ld_s(kx, si) * expf(g[r]);
+            out[W.q + idx] = ld_s(qx, si) * expf(g[r]);
+            out[W.k + idx] = ld_s(kx, si) * expf(gl - g[r]);
+        }
+    }
+    // d: the state's decay over the chunk
+    for (int c = tid; c < dk; c += kThreads)
+        out[W.d + c] = GENERAL ? expf(gx[(C - 1) * ks + c]) : expf(g[C - 1]);
+}
+
+// Copy n floats (n a multiple of 4, both 16-byte aligned) from the workspace to shared memory.
+__device__ __forceinline__ void stage(float *dst, const float *src, int n) {
+    const float4 *s = reinterpret_cast<const float4 *>(src);
+    float4 *d = reinterpret_cast<float4 *>(dst);
+    for (int i = threadIdx.x; i < n / 4; i += kThreads) d[i] = __ldg(s + i);
+}
+
+// One block per (value slice, head, batch): the chunks of one sequence in order.
+template <bool GENERAL>
+__global__ void __launch_bounds__(kThreads)
+simt_chain_kernel(const FwdParams p, const float *ws) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int C = p.C, dk = p.dk, dv = p.dv, dvs = p.dvs, H = p.H, T = p.T;
+    const int NC = (T + C - 1) / C;
+    const int v0 = slice * dvs;
+    const int tid = threadIdx.x;
+    const ChainLayout Ly = chain_layout(C, dk, dvs);
+    float *hs = reinterpret_cast<float *>(smem + Ly.hs);   // state h, dk x dvs
+    float *ux = reinterpret_cast<float *>(smem + Ly.ux);   // values -> R
+    float *dx = reinterpret_cast<float *>(smem + Ly.dx);   // Delta
+    float *ox = reinterpret_cast<float *>(smem + Ly.ox);   // Q' h
+    float *mat = reinterpret_cast<float *>(smem + Ly.mat); // the chunk matrix of each step
+    float *dl = reinterpret_cast<float *>(smem + Ly.dl);   // the state's decay
+    const size_t bh = (size_t)b * H + h;
+    const SimtWs W = simt_ws(C, dk);
+
     for (int idx = tid; idx < dk * dvs; idx += kThreads) {
         const int c = idx / dvs, j = idx % dvs;
         hs[idx] = p.S0 ? p.S0[(bh * dk + c) * dv + v0 + j] : 0.f;
     }
-    if (GENERAL)
-        for (int c = tid; c < dk; c += kThreads) rho[c] = 0.f;
-
-    for (int t0 = 0; t0 < T; t0 += C) {
-        const int Cv = min(C, T - t0);
+    for (int n = 0; n < NC; ++n) {
+        const int t0 = n * C, Cv = min(C, T - t0);
+        const float *src = ws + (bh * NC + n) * W.stride;
         __syncthreads();  // previous chunk fully consumed
-        // ---------------------------------------------------------- load
-        for (int idx = tid; idx < C * dk; idx += kThreads) {
-            const int r = idx / dk, c = idx % dk;
-            const size_t gi = (((size_t)b * T + t0 + r) * H + h) * dk + c;
-            const bool ok = r < Cv;
-            st_s(kx, idx, ok ? load_in(p.k, gi, p.io_bf16) : 0.f);
-            st_s(qx, idx, ok ? load_in(p.q, gi, p.io_bf16) : 0.f);
-            if (GENERAL) {
-                ex[idx] = ok ? (p.erase ? load_in(p.erase, gi, p.io_bf16) : 1.f) : 0.f;
-                gx[idx] = (ok && p.alpha) ? logf(p.alpha[p.alpha_pc ? gi : gi / dk]) : 0.f;
-            }
-        }
+        // ---------------------------------------------- U and E
         for (int idx = tid; idx < C * dvs; idx += kThreads) {
             const int r = idx / dvs, j = idx % dvs;
             const size_t gi = (((size_t)b * T + t0 + r) * H + h) * dv + v0 + j;
@@ -161,200 +409,57 @@ simt_chunk_kernel(const FwdParams p) {
             }
             ux[idx] = u;
         }
-        if (!GENERAL) {
-            for (int r = tid; r < C; r += kThreads) {
-                const size_t ti = ((size_t)b * T + t0 + r) * H + h;
-                g[r] = (r < Cv && p.alpha) ? logf(p.alpha[ti]) : 0.f;
-                bet[r] = (r < Cv) ? (p.beta ? p.beta[ti] : 1.f) : 0.f;
-            }
-        }
+        stage(mat, src + W.e, C * dk);
+        stage(dl, src + W.d, dk);
         __syncthreads();
-        // ------------------------------------------- gates and scans
-        if (GENERAL) {
-            // per channel: preconditioner EMA (carried across chunks), write
-            // key, erase key, cumulative log decay
-            // preconditioner factor f(rho): 1 1/sqrt(rho+eps), 2 1/(rho+eps) (Diag(A)^-1),
-            // 3 the latter squashed into [1/x, x] on a log scale; applied to the
-            // write key (forms 2, 3 read the state with the raw key) or to the query
-            const float lnx = p.precond == 3 ? logf(p.precond_x) : 1.f;
-            for (int c = tid; c < dk; c += kThreads) {
-                float rh = rho[c], G = 0.f;
-                for (int r = 0; r < C; ++r) {
-                    const int idx = r * dk + c;
-                    const float kv = ld_s(kx, idx);
-                    float f = 1.f;
-                    if (p.precond && r < Cv) {
-                        rh = p.rho_decay * rh + kv * kv;
-                        const float a = rh + p.rho_eps;
-                        f = p.precond == 1 ? rsqrtf(a)
-                          : p.precond == 2 ? 1.f / a
-                          : expf(lnx * tanhf(-logf(a) / lnx));
-                    }
-                    if (p.precond_query) {
-                        st_s(qx, idx, ld_s(qx, idx) * f);
-                        ex[idx] *= kv;
-                    } else {
-                        const float kw = kv * f;
-                        st_s(kx, idx, kw);
-                        ex[idx] *= (p.precond == 1 ? kw : kv);
-                    }
-                    G += gx[idx];
-                    gx[idx] = G;
-                }
-                rho[c] = rh;
-            }
-        } else {
-            warp0_inclusive_scan(g, C);
-        }
-        __syncthreads();
-        // ------------------------------------------------ L (strictly lower)
-        for (int idx = tid; idx < C * C; idx += kThreads) {
-            const int r = idx / C, i = idx % C;
-            float val = 0.f;
-            if (i < r) {
-                float acc = 0.f;
-                if (GENERAL) {
-                    for (int c = 0; c < dk; ++c)
-                        acc += ex[r * dk + c] * ld_s(kx, i * dk + c) *
-                               expf(gx[(r - 1) * dk + c] - gx[i * dk + c]);
-                    val = acc;
-                } else {
-                    for (int c = 0; c < dk; ++c) acc += ld_s(kx, r * dk + c) * ld_s(kx, i * dk + c);
-                    val = bet[r] * expf(g[r] - g[i]) * acc;
-                }
-            }
-            tp[idx] = val;
-        }
-        __syncthreads();
-        // ------------------------------------------------ T = (I + L)^-1
-        if (!neumann) {
-            // forward substitution, one row at a time: T_rc = -sum_{c<=i<r} L_ri T_ic
-            for (int r = 1; r < C; ++r) {
-                if (tid < r) lrow[tid] = tp[r * C + tid];
-                __syncthreads();
-                if (tid < r) {
-                    const int c = tid;
-                    float s = lrow[c];
-                    for (int i = c + 1; i < r; ++i) s += lrow[i] * tp[i * C + c];
-                    tp[r * C + c] = -s;
-                }
-                __syncthreads();
-            }
-            for (int r = tid; r < C; r += kThreads) tp[r * C + r] = 1.f;
-        } else {
-            // Horner on the band: T <- M (.) (I + A T), A = -L, T^(0) = I.
-            // band[i*(N+1)+d] holds T_{i,i-d}.
-            const int W = N + 1;
-            float *cur = band, *nxt = band + (size_t)C * W;
-            for (int idx = tid; idx < C * W; idx += kThreads) cur[idx] = (idx % W == 0) ? 1.f : 0.f;
-            __syncthreads();
-            for (int step = 0; step < N; ++step) {
-                for (int idx = tid; idx < C * W; idx += kThreads) {
-                    const int i = idx / W, d = idx % W, j = i - d;
-                    float val = 0.f;
-                    if (j >= 0) {
-                        val = (d == 0) ? 1.f : 0.f;
-                        // sum_{k=j}^{i-1} A_ik T_kj with T_kj in band (k - j <= N)
-                        const int kmax = min(i - 1, j + N);
-                        for (int kk = j; kk <= kmax; ++kk) val -= tp[i * C + kk] * cur[kk * W + (kk - j)];
-                    }
-                    nxt[idx] = val;
-                }
-                __syncthreads();
-                float *sw = cur; cur = nxt; nxt = sw;
-            }
-            for (int idx = tid; idx < C * C; idx += kThreads) {
-                const int i = idx / C, j = idx % C, d = i - j;
-                tp[idx] = (d >= 0 && d <= N) ? cur[i * W + d] : 0.f;
-            }
-        }
-        __syncthreads();
-        // ------------------------------------------------ R = u - h^T e'
-        if (GENERAL) {
-            // e'_rc = e_rc exp(G_{r-1,c})
-            for (int idx = tid; idx < C * dk; idx += kThreads) {
-                const int r = idx / dk;
-                ex[idx] *= (r > 0) ? expf(gx[idx - dk]) : 1.f;
-            }
-            __syncthreads();
-        }
+        // ---------------------------------------------- R = U - E h
         for (int idx = tid; idx < C * dvs; idx += kThreads) {
             const int r = idx / dvs, j = idx % dvs;
             float acc = 0.f;
-            if (GENERAL) {
-                for (int c = 0; c < dk; ++c) acc += ex[r * dk + c] * hs[c * dvs + j];
-                ux[idx] = ux[idx] - acc;
-            } else {
-                for (int c = 0; c < dk; ++c) acc += ld_s(kx, r * dk + c) * hs[c * dvs + j];
-                ux[idx] = bet[r] * (ux[idx] - expf(g[r]) * acc);
-            }
+            for (int c = 0; c < dk; ++c) acc += mat[r * dk + c] * hs[c * dvs + j];
+            ux[idx] -= acc;
         }
         __syncthreads();
-        // ------------------------------------------------ Delta = T R
+        stage(mat, src + W.tb, C * C);
+        __syncthreads();
+        // ---------------------------------------------- Delta = TB R
         for (int idx = tid; idx < C * dvs; idx += kThreads) {
             const int r = idx / dvs, j = idx % dvs;
             float acc = 0.f;
-            for (int i = 0; i <= r; ++i) acc += tp[r * C + i] * ux[i * dvs + j];
+            for (int i = 0; i <= r; ++i) acc += mat[r * C + i] * ux[i * dvs + j];
             dx[idx] = acc;
         }
         __syncthreads();
-        // ------------------------------------------------ P (causal, decayed)
-        for (int idx = tid; idx < C * C; idx += kThreads) {
-            const int r = idx / C, i = idx % C;
-            float val = 0.f;
-            if (i <= r) {
-                float acc = 0.f;
-                if (GENERAL) {
-                    for (int c = 0; c < dk; ++c)
-                        acc += ld_s(qx, r * dk + c) * ld_s(kx, i * dk + c) *
-                               expf(gx[r * dk + c] - gx[i * dk + c]);
-                    val = acc;
-                } else {
-                    for (int c = 0; c < dk; ++c) acc += ld_s(qx, r * dk + c) * ld_s(kx, i * dk + c);
-                    val = expf(g[r] - g[i]) * acc;
-                }
-            }
-            tp[idx] = val;
+        stage(mat, src + W.q, C * dk);
+        __syncthreads();
+        // ---------------------------------------------- O = Q' h + P Delta
+        for (int idx = tid; idx < C * dvs; idx += kThreads) {
+            const int r = idx / dvs, j = idx % dvs;
+            float acc = 0.f;
+            for (int c = 0; c < dk; ++c) acc += mat[r * dk + c] * hs[c * dvs + j];
+            ox[idx] = acc;
         }
         __syncthreads();
-        if (GENERAL) {
-            // q <- q (.) e^{G_r};  kw <- kw (.) e^{G_last - G_r}
-            for (int idx = tid; idx < C * dk; idx += kThreads) {
-                const int c = idx % dk;
-                const float Gl = gx[(C - 1) * dk + c];
-                st_s(qx, idx, ld_s(qx, idx) * expf(gx[idx]));
-                st_s(kx, idx, ld_s(kx, idx) * expf(Gl - gx[idx]));
-            }
-            __syncthreads();
-        }
-        // ------------------------------------------------ O
+        stage(mat, src + W.pp, C * C);
+        __syncthreads();
         for (int idx = tid; idx < C * dvs; idx += kThreads) {
             const int r = idx / dvs, j = idx % dvs;
             if (r >= Cv) continue;
-            float acc = 0.f;
-            for (int c = 0; c < dk; ++c) acc += ld_s(qx, r * dk + c) * hs[c * dvs + j];
-            if (!GENERAL) acc *= expf(g[r]);
-            for (int i = 0; i <= r; ++i) acc += tp[r * C + i] * dx[i * dvs + j];
+            float acc = ox[idx];
+            for (int i = 0; i <= r; ++i) acc += mat[r * C + i] * dx[i * dvs + j];
             const size_t go = (((size_t)b * T + t0 + r) * H + h) * dv + v0 + j;
             if (p.o_bf16) reinterpret_cast<__nv_bfloat16 *>(p.o)[go] = __float2bfloat16_rn(acc);
             else reinterpret_cast<float *>(p.o)[go] = acc;
         }
         __syncthreads();
-        // ------------------------------------------------ state update
+        stage(mat, src + W.k, C * dk);
+        __syncthreads();
+        // ---------------------------------------------- h <- diag(d) h + K''^T Delta
         for (int idx = tid; idx < dk * dvs; idx += kThreads) {
             const int c = idx / dvs, j = idx % dvs;
             float acc = 0.f;
-            float decay;
-            if (GENERAL) {
-                for (int r = 0; r < C; ++r) acc += ld_s(kx, r * dk + c) * dx[r * dvs + j];
-                decay = expf(gx[(C - 1) * dk + c]);
-            } else {
-                const float gl = g[C - 1];
-                for (int r = 0; r < C; ++r)
-                    acc += ld_s(kx, r * dk + c) * expf(gl - g[r]) * dx[r * dvs + j];
-                decay = expf(gl);
-            }
-            hs[idx] = decay * hs[idx] + acc;
+            for (int r = 0; r < C; ++r) acc += mat[r * dk + c] * dx[r * dvs + j];
+            hs[idx] = dl[c] * hs[idx] + acc;
         }
     }
     __syncthreads();
@@ -366,36 +471,48 @@ simt_chunk_kernel(const FwdParams p) {
     }
 }
 
+template <typename KS, bool GENERAL>
+cudaError_t launch_pair(const FwdParams &p, float *ws, cudaStream_t stream) {
+    const int NC = (p.T + p.C - 1) / p.C;
+    const PrepLayout pl = prep_layout(p.C, p.dk, p.N, p.mode == GDN_INV_NEUMANN, GENERAL ? 1 : 0, (int)sizeof(KS));
+    const ChainLayout cl = chain_layout(p.C, p.dk, p.dvs);
+    auto prep = simt_prep_kernel<KS, GENERAL>;
+    auto chain = simt_chain_kernel<GENERAL>;
+    cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.total);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(chain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cl.total);
+    if (e != cudaSuccess) return e;
+    if (GENERAL && p.precond) {
+        float *rho0 = ws + (size_t)p.B * p.H * NC * simt_ws(p.C, p.dk).stride;
+        rho_scan_kernel<<<dim3(p.H, p.B), 128, 0, stream>>>(p, rho0);
+    }
+    prep<<<dim3(NC, p.H, p.B), kThreads, pl.total, stream>>>(p, ws);
+    chain<<<dim3(p.slices, p.H, p.B), kThreads, cl.total, stream>>>(p, ws);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t simt_smem_bytes(const FwdParams &p) {
     const int key_bytes = (p.io_bf16 && !p.general) ? 2 : 4;
-    const SimtLayout L = simt_layout(p.C, p.dk, p.dvs, p.N, p.mode == GDN_INV_NEUMANN,
-                                     p.general, key_bytes);
-    return L.total;
+    const PrepLayout pl = prep_layout(p.C, p.dk, p.N, p.mode == GDN_INV_NEUMANN, p.general, key_bytes);
+    const ChainLayout cl = chain_layout(p.C, p.dk, p.dvs);
+    return pl.total > cl.total ? pl.total : cl.total;
 }
 
-cudaError_t launch_simt(const FwdParams &p, cudaStream_t stream) {
-    const size_t smem = simt_smem_bytes(p);
-    dim3 grid(p.slices, p.H, p.B);
-    cudaError_t e;
-    if (p.general) {
-        auto kern = simt_chunk_kernel<float, true>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        kern<<<grid, kThreads, smem, stream>>>(p);
-    } else if (p.io_bf16) {
-        auto kern = simt_chunk_kernel<__nv_bfloat16, false>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        kern<<<grid, kThreads, smem, stream>>>(p);
-    } else {
-        auto kern = simt_chunk_kernel<float, false>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        kern<<<grid, kThreads, smem, stream>>>(p);
-    }
-    return cudaGetLastError();
+size_t simt_workspace_bytes(const FwdParams &p) {
+    const size_t NC = (size_t)(p.T + p.C - 1) / p.C;
+    const size_t chunks = (size_t)p.B * p.H * NC;
+    size_t floats = chunks * simt_ws(p.C, p.dk).stride;
+    if (p.general && p.precond) floats += chunks * p.dk;
+    return floats * sizeof(float);
+}
+
+cudaError_t launch_simt(const FwdParams &p, void *workspace, cudaStream_t stream) {
+    float *ws = reinterpret_cast<float *>(workspace);
+    if (p.general) return launch_pair<float, true>(p, ws, stream);
+    if (p.io_bf16) return launch_pair<__nv_bfloat16, false>(p, ws, stream);
+    return launch_pair<float, false>(p, ws, stream);
 }
 
 }  // namespace gdn

@@ -51,8 +51,12 @@
  * between the two CTAs of a cluster through shared memory.  The split
  * tensor-core kernels (GDN_KERNEL_TC_SPLIT) keep, per chunk and head,
  * T diag(beta), T diag(beta e^g) and the decayed causal scores P (fp16,
- * 24 KB) in the workspace between their two launches; gdn_workspace_bytes()
- * gives the size.
+ * 24 KB) in the workspace between their two launches.  The SIMT kernels
+ * (GDN_KERNEL_SIMT) keep, per chunk and head, the state-independent fp32
+ * matrices of the chunk (T diag(beta), the decayed scores, the decayed keys
+ * and queries, 2 C^2 + 3 C dk + dk floats) and, for the preconditioned
+ * two-gate rule, the running average at every chunk start (dk floats).
+ * gdn_workspace_bytes() gives the size.
  *
  * Execution and errors.  gdn_chunk_fwd validates its arguments on the host
  * and returns an error before launching anything (nothing is written) when
@@ -72,7 +76,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 6
+#define GDN_ABI_VERSION 7
 
 #if defined(__GNUC__)
 #define GDN_API __attribute__((visibility("default")))
@@ -104,7 +108,9 @@ typedef enum {
 typedef enum {
     GDN_KERNEL_AUTO = 0,        /* the first of TC_SPLIT, TC, SIMT that supports the call
                                    (RECURRENT for T <= 8) */
-    GDN_KERNEL_SIMT = 1,        /* fp32 CUDA-core chunk kernel (all variants) */
+    GDN_KERNEL_SIMT = 1,        /* fp32 CUDA-core kernels (all variants): the chunk matrices
+                                   of every chunk at once into the workspace, then the
+                                   state chain */
     GDN_KERNEL_TC = 2,          /* fused tcgen05/TMEM/TMA kernel, one launch of 2-CTA
                                    clusters per (batch, head): bf16 q/k/v, scalar decay,
                                    C = 64, dk = dv = 128, exact or Neumann mode (any N).
@@ -159,9 +165,9 @@ typedef struct {
 /* Chunkwise forward: o and S_T from q, k, v, gates and S0 (see above). */
 GDN_API gdn_status gdn_chunk_fwd(const gdn_fwd_args *args, void *stream);
 
-/* Workspace bytes gdn_chunk_fwd needs for these arguments (0 for the SIMT
- * kernel), or 0 with gdn_last_error() set if the arguments are invalid.  Host
- * only. */
+/* Workspace bytes gdn_chunk_fwd needs for these arguments (0 for the fused
+ * and the recurrent kernels), or 0 with gdn_last_error() set if the arguments
+ * are invalid.  Host only. */
 GDN_API uint64_t gdn_workspace_bytes(const gdn_fwd_args *args);
 
 /* Which kernel gdn_chunk_fwd would launch for these arguments (gdn_kernel
