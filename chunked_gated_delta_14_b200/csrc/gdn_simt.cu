@@ -25,8 +25,9 @@
 //
 // 1. simt_prep_kernel -- one block per (chunk, head, batch), all chunks at
 //    once: gates, L, T, and the six matrices into the workspace (fp32).  The
-//    preconditioner's running average is carried across chunks; a scan kernel
-//    (rho_scan_kernel) gives each chunk its value at the chunk start first.
+//    preconditioner's running average is carried across chunks; two small
+//    kernels (rho_local_kernel, rho_combine_kernel) give each chunk its value
+//    at the chunk start first.
 // 2. simt_chain_kernel -- one block per (batch, head, value slice) walks the
 //    chunks in order with the fp32 state h = S^T (dk x dvs) in shared memory,
 //    reading each matrix once per chunk.
@@ -68,9 +69,19 @@ __device__ __forceinline__ void st_s(S *a, int i, float x) {
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
 
+// 2^x on the special-function unit (PTX ex2.approx.ftz.f32, relative error
+// about 2^-22): the per-channel decay ratios of the two-gate rule, kept in
+// log2 form.
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Workspace: per chunk-head, fp32 [TB C x C | P C x C | E C x dk | Q' C x dk |
 // K'' C x dk | d dk], padded to 16 bytes; then, for the preconditioned two-gate
-// rule, the running average at every chunk start, [B, H, chunks, dk].
+// rule, the running average at every chunk start, each chunk's own sum and the
+// decay's power over the chunk, three times [B, H, chunks, dk].
 struct SimtWs {
     size_t tb, pp, e, q, k, d, stride;   // floats
 };
@@ -129,7 +140,7 @@ __host__ __device__ inline ChainLayout chain_layout(int C, int dk, int dvs) {
     L.ux = take((size_t)C * dvs * 4);
     L.dx = take((size_t)C * dvs * 4);
     L.ox = take((size_t)C * dvs * 4);
-    L.mat = take((size_t)C * (C > dk ? C : dk) * 4);
+    L.mat = take((size_t)C * ((C > dk ? C : dk) + 4) * 4);   // rows padded by 4 floats
     L.dl = take((size_t)dk * 4);
     L.total = off;
     return L;
@@ -153,20 +164,36 @@ __device__ void warp0_inclusive_scan(float *x, int n) {
 }
 
 // The preconditioner's running average rho_t = decay rho_{t-1} + k_t (.) k_t,
-// per (batch, head, key channel), recorded at every chunk start.
-__global__ void rho_scan_kernel(const FwdParams p, float *rho_start) {
+// per (batch, head, key channel), at every chunk start.  Over a chunk of Cv
+// tokens rho_end = decay^Cv rho_start + sum_r decay^(Cv-1-r) k_r (.) k_r, so the
+// chunks' own sums come first, in parallel (rho_local_kernel), and a short
+// pass over the chunks chains them (rho_combine_kernel).
+__global__ void rho_local_kernel(const FwdParams p, float *sums, float *pows) {
+    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, c = threadIdx.x;
+    if (c >= p.dk) return;
+    const int NC = (p.T + p.C - 1) / p.C;
+    const int t0 = n * p.C, t1 = min(p.T, t0 + p.C);
+    float s = 0.f, a = 1.f;
+#pragma unroll 4
+    for (int t = t0; t < t1; ++t) {
+        const float kv = load_in(p.k, (((size_t)b * p.T + t) * p.H + h) * p.dk + c, p.io_bf16);
+        s = p.rho_decay * s + kv * kv;
+        a *= p.rho_decay;
+    }
+    const size_t o = (((size_t)b * p.H + h) * NC + n) * p.dk + c;
+    sums[o] = s;
+    pows[o] = a;
+}
+
+__global__ void rho_combine_kernel(const FwdParams p, const float *sums, const float *pows, float *rho_start) {
     const int h = blockIdx.x, b = blockIdx.y, c = threadIdx.x;
     if (c >= p.dk) return;
     const int NC = (p.T + p.C - 1) / p.C;
     float rh = 0.f;
     for (int n = 0; n < NC; ++n) {
-        rho_start[(((size_t)b * p.H + h) * NC + n) * p.dk + c] = rh;
-        const int t0 = n * p.C, t1 = min(p.T, t0 + p.C);
-#pragma unroll 4
-        for (int t = t0; t < t1; ++t) {
-            const float kv = load_in(p.k, (((size_t)b * p.T + t) * p.H + h) * p.dk + c, p.io_bf16);
-            rh = p.rho_decay * rh + kv * kv;
-        }
+        const size_t o = (((size_t)b * p.H + h) * NC + n) * p.dk + c;
+        rho_start[o] = rh;
+        rh = pows[o] * rh + sums[o];
     }
 }
 
@@ -189,7 +216,7 @@ simt_prep_kernel(const FwdParams p, float *ws) {
     KS *kx = reinterpret_cast<KS *>(smem + Ly.kx);       // keys (write keys kw)
     KS *qx = reinterpret_cast<KS *>(smem + Ly.qx);       // read keys
     float *ex = reinterpret_cast<float *>(smem + Ly.ex); // erase keys (two-gate)
-    float *gx = reinterpret_cast<float *>(smem + Ly.gx); // per-channel cumulative log decay
+    float *gx = reinterpret_cast<float *>(smem + Ly.gx); // per-channel cumulative log2 decay
     float *tp = reinterpret_cast<float *>(smem + Ly.tp); // L -> T, C x C
     float *band = reinterpret_cast<float *>(smem + Ly.band);
     float *rows = reinterpret_cast<float *>(smem + Ly.rows);
@@ -210,7 +237,7 @@ simt_prep_kernel(const FwdParams p, float *ws) {
         st_s(qx, si, ok ? load_in(p.q, gi, p.io_bf16) : 0.f);
         if (GENERAL) {
             ex[si] = ok ? (p.erase ? load_in(p.erase, gi, p.io_bf16) : 1.f) : 0.f;
-            gx[si] = (ok && p.alpha) ? logf(p.alpha[p.alpha_pc ? gi : gi / dk]) : 0.f;
+            gx[si] = (ok && p.alpha) ? log2f(p.alpha[p.alpha_pc ? gi : gi / dk]) : 0.f;
         }
     }
     if (!GENERAL) {
@@ -260,22 +287,50 @@ simt_prep_kernel(const FwdParams p, float *ws) {
     }
     __syncthreads();
     // ------------------------------------------------ L (strictly lower)
-    for (int idx = tid; idx < C * C; idx += kThreads) {
-        const int r = idx / C, i = idx % C;
-        float val = 0.f;
-        if (i < r) {
-            float acc = 0.f;
+    // 4 x 4 register tiles (rows r0.., keys i0..): 8 loads per 16 products
+    for (int t = tid; t < (C / 4) * (C / 4); t += kThreads) {
+        const int r0 = 4 * (t / (C / 4)), i0 = 4 * (t % (C / 4));
+        float acc[4][4] = {};
+        if (i0 < r0 + 3) {
             if (GENERAL) {
-                for (int c = 0; c < dk; ++c)
-                    acc += ex[r * ks + c] * ld_s(kx, i * ks + c) *
-                           expf(gx[(r - 1) * ks + c] - gx[i * ks + c]);
-                val = acc;
+                for (int c = 0; c < dk; ++c) {
+                    float er[4], gr[4], ki[4], gi[4];
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) {
+                        er[a] = ex[(r0 + a) * ks + c];
+                        gr[a] = (r0 + a > 0) ? gx[(r0 + a - 1) * ks + c] : 0.f;
+                        ki[a] = ld_s(kx, (i0 + a) * ks + c);
+                        gi[a] = gx[(i0 + a) * ks + c];
+                    }
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) acc[a][e] += er[a] * ki[e] * fast_exp2(gr[a] - gi[e]);
+                }
             } else {
-                for (int c = 0; c < dk; ++c) acc += ld_s(kx, r * ks + c) * ld_s(kx, i * ks + c);
-                val = bet[r] * expf(g[r] - g[i]) * acc;
+                for (int c = 0; c < dk; ++c) {
+                    float kr[4], ki[4];
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) {
+                        kr[a] = ld_s(kx, (r0 + a) * ks + c);
+                        ki[a] = ld_s(kx, (i0 + a) * ks + c);
+                    }
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) acc[a][e] += kr[a] * ki[e];
+                }
             }
         }
-        tp[idx] = val;
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = r0 + a, i = i0 + e;
+                float val = 0.f;
+                if (i < r) val = GENERAL ? acc[a][e] : bet[r] * expf(g[r] - g[i]) * acc[a][e];
+                tp[r * C + i] = val;
+            }
     }
     __syncthreads();
     // ------------------------------------------------ T = (I + L)^-1
@@ -325,32 +380,59 @@ simt_prep_kernel(const FwdParams p, float *ws) {
     // TB = T diag(beta) (scalar rule; the two-gate rule has no beta)
     for (int idx = tid; idx < C * C; idx += kThreads)
         out[W.tb + idx] = GENERAL ? tp[idx] : tp[idx] * bet[idx % C];
-    // P: decayed causal scores
-    for (int idx = tid; idx < C * C; idx += kThreads) {
-        const int r = idx / C, i = idx % C;
-        float val = 0.f;
-        if (i <= r) {
-            float acc = 0.f;
+    // P: decayed causal scores, 4 x 4 register tiles
+    for (int t = tid; t < (C / 4) * (C / 4); t += kThreads) {
+        const int r0 = 4 * (t / (C / 4)), i0 = 4 * (t % (C / 4));
+        float acc[4][4] = {};
+        if (i0 <= r0 + 3) {
             if (GENERAL) {
-                for (int c = 0; c < dk; ++c)
-                    acc += ld_s(qx, r * ks + c) * ld_s(kx, i * ks + c) *
-                           expf(gx[r * ks + c] - gx[i * ks + c]);
-                val = acc;
+                for (int c = 0; c < dk; ++c) {
+                    float qr[4], gr[4], ki[4], gi[4];
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) {
+                        qr[a] = ld_s(qx, (r0 + a) * ks + c);
+                        gr[a] = gx[(r0 + a) * ks + c];
+                        ki[a] = ld_s(kx, (i0 + a) * ks + c);
+                        gi[a] = gx[(i0 + a) * ks + c];
+                    }
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) acc[a][e] += qr[a] * ki[e] * fast_exp2(gr[a] - gi[e]);
+                }
             } else {
-                for (int c = 0; c < dk; ++c) acc += ld_s(qx, r * ks + c) * ld_s(kx, i * ks + c);
-                val = expf(g[r] - g[i]) * acc;
+                for (int c = 0; c < dk; ++c) {
+                    float qr[4], ki[4];
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) {
+                        qr[a] = ld_s(qx, (r0 + a) * ks + c);
+                        ki[a] = ld_s(kx, (i0 + a) * ks + c);
+                    }
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) acc[a][e] += qr[a] * ki[e];
+                }
             }
         }
-        out[W.pp + idx] = val;
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int r = r0 + a, i = i0 + e;
+                float val = 0.f;
+                if (i <= r) val = GENERAL ? acc[a][e] : expf(g[r] - g[i]) * acc[a][e];
+                out[W.pp + r * C + i] = val;
+            }
     }
     // E (the state read), Q' (the output read), K'' (the state write)
     for (int idx = tid; idx < C * dk; idx += kThreads) {
         const int r = idx / dk, c = idx % dk, si = r * ks + c;
         if (GENERAL) {
             const float Gl = gx[(C - 1) * ks + c];
-            out[W.e + idx] = ex[si] * ((r > 0) ? expf(gx[si - ks]) : 1.f);
-            out[W.q + idx] = ld_s(qx, si) * expf(gx[si]);
-            out[W.k + idx] = ld_s(kx, si) * expf(Gl - gx[si]);
+            out[W.e + idx] = ex[si] * ((r > 0) ? fast_exp2(gx[si - ks]) : 1.f);
+            out[W.q + idx] = ld_s(qx, si) * fast_exp2(gx[si]);
+            out[W.k + idx] = ld_s(kx, si) * fast_exp2(Gl - gx[si]);
         } else {
             const float gl = g[C - 1];
             out[W.e + idx] = ld_s(kx, si) * expf(g[r]);
@@ -360,15 +442,25 @@ simt_prep_kernel(const FwdParams p, float *ws) {
     }
     // d: the state's decay over the chunk
     for (int c = tid; c < dk; c += kThreads)
-        out[W.d + c] = GENERAL ? expf(gx[(C - 1) * ks + c]) : expf(g[C - 1]);
+        out[W.d + c] = GENERAL ? fast_exp2(gx[(C - 1) * ks + c]) : expf(g[C - 1]);
 }
 
-// Copy n floats (n a multiple of 4, both 16-byte aligned) from the workspace to shared memory.
-__device__ __forceinline__ void stage(float *dst, const float *src, int n) {
+// Copy a rows x cols matrix (cols a multiple of 4, 16-byte aligned) from the
+// workspace into shared memory with rows cols + 4 floats apart, so that the
+// row reads of one warp fall into different banks.
+__device__ __forceinline__ void stage(float *dst, const float *src, int rows, int cols) {
+    const int q = cols / 4;
     const float4 *s = reinterpret_cast<const float4 *>(src);
-    float4 *d = reinterpret_cast<float4 *>(dst);
-    for (int i = threadIdx.x; i < n / 4; i += kThreads) d[i] = __ldg(s + i);
+    for (int i = threadIdx.x; i < rows * q; i += kThreads) {
+        const int r = i / q, c = i % q;
+        *reinterpret_cast<float4 *>(dst + (size_t)r * (cols + 4) + 4 * c) = __ldg(s + i);
+    }
 }
+
+// 2 x 2 output tiles of a rows x dvs product: rows r0, r0 + 1, columns j0, j0 + 1.
+#define FOR_TILES(rows, dvs)                                                         \
+    for (int t_ = threadIdx.x; t_ < ((rows) / 2) * ((dvs) / 2); t_ += kThreads)      \
+        if (const int r0 = 2 * (t_ / ((dvs) / 2)), j0 = 2 * (t_ % ((dvs) / 2)); true)
 
 // One block per (value slice, head, batch): the chunks of one sequence in order.
 template <bool GENERAL>
@@ -387,8 +479,10 @@ simt_chain_kernel(const FwdParams p, const float *ws) {
     float *ox = reinterpret_cast<float *>(smem + Ly.ox);   // Q' h
     float *mat = reinterpret_cast<float *>(smem + Ly.mat); // the chunk matrix of each step
     float *dl = reinterpret_cast<float *>(smem + Ly.dl);   // the state's decay
+    const int mk = dk + 4, mc = C + 4;                     // staged row strides
     const size_t bh = (size_t)b * H + h;
     const SimtWs W = simt_ws(C, dk);
+    auto ld2 = [](const float *x) { return *reinterpret_cast<const float2 *>(x); };
 
     for (int idx = tid; idx < dk * dvs; idx += kThreads) {
         const int c = idx / dvs, j = idx % dvs;
@@ -409,57 +503,90 @@ simt_chain_kernel(const FwdParams p, const float *ws) {
             }
             ux[idx] = u;
         }
-        stage(mat, src + W.e, C * dk);
-        stage(dl, src + W.d, dk);
+        stage(mat, src + W.e, C, dk);
+        for (int c = tid; c < dk; c += kThreads) dl[c] = src[W.d + c];
         __syncthreads();
         // ---------------------------------------------- R = U - E h
-        for (int idx = tid; idx < C * dvs; idx += kThreads) {
-            const int r = idx / dvs, j = idx % dvs;
-            float acc = 0.f;
-            for (int c = 0; c < dk; ++c) acc += mat[r * dk + c] * hs[c * dvs + j];
-            ux[idx] -= acc;
+        FOR_TILES(C, dvs) {
+            float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+            for (int c = 0; c < dk; ++c) {
+                const float e0 = mat[r0 * mk + c], e1 = mat[(r0 + 1) * mk + c];
+                const float2 hv = ld2(hs + c * dvs + j0);
+                a00 += e0 * hv.x; a01 += e0 * hv.y; a10 += e1 * hv.x; a11 += e1 * hv.y;
+            }
+            ux[r0 * dvs + j0] -= a00; ux[r0 * dvs + j0 + 1] -= a01;
+            ux[(r0 + 1) * dvs + j0] -= a10; ux[(r0 + 1) * dvs + j0 + 1] -= a11;
         }
         __syncthreads();
-        stage(mat, src + W.tb, C * C);
+        stage(mat, src + W.tb, C, C);
         __syncthreads();
-        // ---------------------------------------------- Delta = TB R
-        for (int idx = tid; idx < C * dvs; idx += kThreads) {
-            const int r = idx / dvs, j = idx % dvs;
-            float acc = 0.f;
-            for (int i = 0; i <= r; ++i) acc += mat[r * C + i] * ux[i * dvs + j];
-            dx[idx] = acc;
+        // ---------------------------------------------- Delta = TB R (TB lower triangular)
+        FOR_TILES(C, dvs) {
+            float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+            for (int i = 0; i < r0 + 2; ++i) {
+                const float t0v = mat[r0 * mc + i], t1v = mat[(r0 + 1) * mc + i];
+                const float2 rv = ld2(ux + i * dvs + j0);
+                a00 += t0v * rv.x; a01 += t0v * rv.y; a10 += t1v * rv.x; a11 += t1v * rv.y;
+            }
+            dx[r0 * dvs + j0] = a00; dx[r0 * dvs + j0 + 1] = a01;
+            dx[(r0 + 1) * dvs + j0] = a10; dx[(r0 + 1) * dvs + j0 + 1] = a11;
         }
         __syncthreads();
-        stage(mat, src + W.q, C * dk);
+        stage(mat, src + W.q, C, dk);
         __syncthreads();
         // ---------------------------------------------- O = Q' h + P Delta
-        for (int idx = tid; idx < C * dvs; idx += kThreads) {
-            const int r = idx / dvs, j = idx % dvs;
-            float acc = 0.f;
-            for (int c = 0; c < dk; ++c) acc += mat[r * dk + c] * hs[c * dvs + j];
-            ox[idx] = acc;
+        FOR_TILES(C, dvs) {
+            float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+            for (int c = 0; c < dk; ++c) {
+                const float q0 = mat[r0 * mk + c], q1 = mat[(r0 + 1) * mk + c];
+                const float2 hv = ld2(hs + c * dvs + j0);
+                a00 += q0 * hv.x; a01 += q0 * hv.y; a10 += q1 * hv.x; a11 += q1 * hv.y;
+            }
+            ox[r0 * dvs + j0] = a00; ox[r0 * dvs + j0 + 1] = a01;
+            ox[(r0 + 1) * dvs + j0] = a10; ox[(r0 + 1) * dvs + j0 + 1] = a11;
         }
         __syncthreads();
-        stage(mat, src + W.pp, C * C);
+        stage(mat, src + W.pp, C, C);
         __syncthreads();
-        for (int idx = tid; idx < C * dvs; idx += kThreads) {
-            const int r = idx / dvs, j = idx % dvs;
-            if (r >= Cv) continue;
-            float acc = ox[idx];
-            for (int i = 0; i <= r; ++i) acc += mat[r * C + i] * dx[i * dvs + j];
-            const size_t go = (((size_t)b * T + t0 + r) * H + h) * dv + v0 + j;
-            if (p.o_bf16) reinterpret_cast<__nv_bfloat16 *>(p.o)[go] = __float2bfloat16_rn(acc);
-            else reinterpret_cast<float *>(p.o)[go] = acc;
+        FOR_TILES(C, dvs) {
+            float a[2][2] = {{ox[r0 * dvs + j0], ox[r0 * dvs + j0 + 1]},
+                             {ox[(r0 + 1) * dvs + j0], ox[(r0 + 1) * dvs + j0 + 1]}};
+            for (int i = 0; i < r0 + 2; ++i) {
+                const float p0 = mat[r0 * mc + i], p1 = mat[(r0 + 1) * mc + i];
+                const float2 dv2 = ld2(dx + i * dvs + j0);
+                a[0][0] += p0 * dv2.x; a[0][1] += p0 * dv2.y; a[1][0] += p1 * dv2.x; a[1][1] += p1 * dv2.y;
+            }
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int r = r0 + e;
+                if (r >= Cv) continue;
+                const size_t go = (((size_t)b * T + t0 + r) * H + h) * dv + v0 + j0;
+                if (p.o_bf16) {
+                    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.o) + go;
+                    o[0] = __float2bfloat16_rn(a[e][0]);
+                    o[1] = __float2bfloat16_rn(a[e][1]);
+                } else {
+                    float *o = reinterpret_cast<float *>(p.o) + go;
+                    o[0] = a[e][0];
+                    o[1] = a[e][1];
+                }
+            }
         }
         __syncthreads();
-        stage(mat, src + W.k, C * dk);
+        stage(mat, src + W.k, C, dk);
         __syncthreads();
         // ---------------------------------------------- h <- diag(d) h + K''^T Delta
-        for (int idx = tid; idx < dk * dvs; idx += kThreads) {
-            const int c = idx / dvs, j = idx % dvs;
-            float acc = 0.f;
-            for (int r = 0; r < C; ++r) acc += mat[r * dk + c] * dx[r * dvs + j];
-            hs[idx] = dl[c] * hs[idx] + acc;
+        FOR_TILES(dk, dvs) {
+            const int c0 = r0;
+            float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+            for (int r = 0; r < C; ++r) {
+                const float2 kv = ld2(mat + r * mk + c0);
+                const float2 dv2 = ld2(dx + r * dvs + j0);
+                a00 += kv.x * dv2.x; a01 += kv.x * dv2.y; a10 += kv.y * dv2.x; a11 += kv.y * dv2.y;
+            }
+            float *h0 = hs + c0 * dvs + j0, *h1 = hs + (c0 + 1) * dvs + j0;
+            h0[0] = dl[c0] * h0[0] + a00; h0[1] = dl[c0] * h0[1] + a01;
+            h1[0] = dl[c0 + 1] * h1[0] + a10; h1[1] = dl[c0 + 1] * h1[1] + a11;
         }
     }
     __syncthreads();
@@ -470,6 +597,7 @@ simt_chain_kernel(const FwdParams p, const float *ws) {
         }
     }
 }
+#undef FOR_TILES
 
 template <typename KS, bool GENERAL>
 cudaError_t launch_pair(const FwdParams &p, float *ws, cudaStream_t stream) {
@@ -483,8 +611,11 @@ cudaError_t launch_pair(const FwdParams &p, float *ws, cudaStream_t stream) {
     e = cudaFuncSetAttribute(chain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cl.total);
     if (e != cudaSuccess) return e;
     if (GENERAL && p.precond) {
-        float *rho0 = ws + (size_t)p.B * p.H * NC * simt_ws(p.C, p.dk).stride;
-        rho_scan_kernel<<<dim3(p.H, p.B), 128, 0, stream>>>(p, rho0);
+        const size_t chunks = (size_t)p.B * p.H * NC;
+        float *rho0 = ws + chunks * simt_ws(p.C, p.dk).stride;
+        float *sums = rho0 + chunks * p.dk, *pows = sums + chunks * p.dk;
+        rho_local_kernel<<<dim3(NC, p.H, p.B), 128, 0, stream>>>(p, sums, pows);
+        rho_combine_kernel<<<dim3(p.H, p.B), 128, 0, stream>>>(p, sums, pows, rho0);
     }
     prep<<<dim3(NC, p.H, p.B), kThreads, pl.total, stream>>>(p, ws);
     chain<<<dim3(p.slices, p.H, p.B), kThreads, cl.total, stream>>>(p, ws);
@@ -504,7 +635,7 @@ size_t simt_workspace_bytes(const FwdParams &p) {
     const size_t NC = (size_t)(p.T + p.C - 1) / p.C;
     const size_t chunks = (size_t)p.B * p.H * NC;
     size_t floats = chunks * simt_ws(p.C, p.dk).stride;
-    if (p.general && p.precond) floats += chunks * p.dk;
+    if (p.general && p.precond) floats += 3 * chunks * p.dk;   // start values, chunk sums, decay powers
     return floats * sizeof(float);
 }
 
