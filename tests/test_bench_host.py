@@ -169,10 +169,10 @@ def test_e2e_falls_back_to_one_stream(fake_cuda, monkeypatch):
     assert line["e2e"]["value"] > 0 and line["e2e"]["pipeline"].startswith("one stream")
 
 
-@pytest.mark.parametrize("name,kernel", [("plain_fp32", "simt_chunk_kernel"),
-                                         ("long_context", "keyside_kernel+chain_kernel"),
-                                         ("precond_two_gate", "simt_chunk_kernel")])
-def test_other_workload_lines(fake_cuda, monkeypatch, name, kernel):
+@pytest.mark.parametrize("name,kernel,launches", [("plain_fp32", "simt_prep_kernel+simt_chain_kernel", 2),
+                                                  ("long_context", "keyside_kernel+chain_kernel", 2),
+                                                  ("precond_two_gate", "simt_prep_kernel+simt_chain_kernel", 4)])
+def test_other_workload_lines(fake_cuda, monkeypatch, name, kernel, launches):
     import bench
     # the line's assembly only: a stand-in for the oracle timing of a whole long sequence
     from chunked_gated_delta_14_b200 import inputs
@@ -183,6 +183,7 @@ def test_other_workload_lines(fake_cuda, monkeypatch, name, kernel):
     (line,) = _lines("run_gpu", workload=name, cpu_budget=0.05)
     _check_contract(line)
     assert line["config"]["kernel"] == kernel
+    assert line["gpu_launches"] == launches * line["steps"]
     assert line["config"]["workload"].startswith(name)
     assert line["metric"] != _line("run_gpu", bwd_steps=0, no_cpu_baseline=True)["metric"]
 
