@@ -253,3 +253,34 @@ def test_debug_chunk_T_rejects_on_host():
     assert L.gdn_debug_chunk_T(ctypes.byref(_args()), 0, 0, 0, ctypes.c_void_p(fake + 8), None) == GDN_ERR_ALIGNMENT
     assert L.gdn_debug_chunk_T(ctypes.byref(_args(kernel=1)), 0, 0, 0, ctypes.c_void_p(fake), None) == GDN_ERR_UNSUPPORTED
     assert L.gdn_debug_chunk_T(ctypes.byref(_args(dv=64)), 0, 0, 0, ctypes.c_void_p(fake), None) == GDN_ERR_UNSUPPORTED
+
+
+def test_workspace_sizes_per_kernel():
+    """The SIMT kernels keep, per chunk-head, the fp32 matrices TB, P (C x C), E, Q',
+    K'' (C x dk) and the decay d (dk), padded to 16 bytes; the preconditioned two-gate
+    rule adds three dk arrays per chunk-head.  The split tensor-core kernels keep
+    24 KiB per chunk-head, the fused and the recurrent kernels nothing."""
+    B, T, H, C, dk = 2, 100, 3, 64, 128
+    chunks = B * H * (-(-T // C))
+    per = 2 * C * C + 3 * C * dk + dk
+    per = (per + 3) // 4 * 4
+    assert gdn.workspace_bytes(_args(kernel=1)) == chunks * per * 4
+    two_gate = _args(kernel=1, alpha=0x70000, alpha_per_channel=1, precond=1, erase=0x50000, write=0x58000)
+    assert gdn.workspace_bytes(two_gate) == chunks * (per + 3 * dk) * 4
+    assert gdn.workspace_bytes(_args(kernel=4)) == chunks * 24576
+    assert gdn.workspace_bytes(_args(kernel=2)) == 0
+    assert gdn.workspace_bytes(_args(T=4, kernel=3)) == 0
+    c128 = _args(kernel=1, chunk=128, mode=1, neumann_N=3)
+    per128 = 2 * 128 * 128 + 3 * 128 * dk + dk
+    assert gdn.workspace_bytes(c128) == B * H * 1 * per128 * 4
+
+
+def test_simt_call_without_workspace_rejected_on_host():
+    a = _args(kernel=1)
+    with pytest.raises(gdn.GDNError) as ei:
+        gdn.call(a)   # returns before any CUDA call
+    assert ei.value.status == GDN_ERR_INVALID_ARG and "workspace" in str(ei.value)
+    a.workspace, a.workspace_bytes = 0x900000, gdn.workspace_bytes(a) - 16
+    with pytest.raises(gdn.GDNError) as ei:
+        gdn.call(a)
+    assert ei.value.status == GDN_ERR_INVALID_ARG and "workspace" in str(ei.value)

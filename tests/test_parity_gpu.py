@@ -190,6 +190,18 @@ def test_precond_two_gate_full_size():
     _check_bf16("precond_full_auto", w, x, o_ref, s_ref)
 
 
+@needs_cuda
+@pytest.mark.parametrize("chunk,T", [(16, 301), (32, 1000), (64, 65)])
+def test_precond_two_gate_chunks_ragged(chunk, T):
+    """The preconditioner's running average crosses every chunk boundary (chunk
+    sums chained over many chunks, a ragged last chunk); the chain kernel runs
+    with several value slices."""
+    w = workload("precond_two_gate", B=1, H=2, T=T, chunk=chunk)
+    x = make_inputs(w, seed=6 + chunk)
+    o_ref, s_ref = run_oracle(x, w)
+    _check_bf16(f"precond_C{chunk}_T{T}", w, x, o_ref, s_ref)
+
+
 # ------------------------------ page-form preconditioner variants (next row 3)
 
 def _precond_case(w, x, **kw):
