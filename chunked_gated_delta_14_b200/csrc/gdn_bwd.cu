@@ -10,11 +10,12 @@ size_t region(size_t floats_per_chunk, size_t chunks) {
 }
 
 template <class K>
-cudaError_t launch_one(K kernel, dim3 grid, size_t smem_floats, const BwdParams &p, cudaStream_t stream) {
+cudaError_t launch_one(K kernel, dim3 grid, size_t smem_floats, const BwdParams &p, cudaStream_t stream,
+                       int threads = bwd::kThreads) {
     const size_t bytes = smem_floats * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
-    kernel<<<grid, bwd::kThreads, bytes, stream>>>(p);
+    kernel<<<grid, threads, bytes, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -53,7 +54,8 @@ void bwd_carve_workspace(BwdParams &p, void *workspace) {
 cudaError_t launch_bwd(const BwdParams &p, cudaStream_t stream) {
     const dim3 per_chunk(p.NC, p.H, p.B);
     const dim3 per_slice(p.dv / bwd::kCols, p.H, p.B);
-    cudaError_t e = launch_one(bwd::bwd_prep_kernel, per_chunk, bwd::prep_smem_floats(p.C, p.dk, p.dv), p, stream);
+    cudaError_t e = launch_one(bwd::bwd_prep_kernel, per_chunk, bwd::prep_smem_floats(p.C, p.dk, p.dv), p, stream,
+                               bwd::kPrepThreads);
     if (e != cudaSuccess) return e;
     e = launch_one(bwd::bwd_state_fwd_kernel, per_slice, bwd::state_fwd_smem_floats(p.C, p.dk), p, stream);
     if (e != cudaSuccess) return e;

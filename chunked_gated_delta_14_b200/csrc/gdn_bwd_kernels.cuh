@@ -44,6 +44,7 @@ namespace gdn {
 namespace bwd {
 
 constexpr int kThreads = 256;
+constexpr int kPrepThreads = 512;   // the prep kernel: one block per SM (shared memory), 16 warps
 constexpr int kCols = 32;     // value columns per block of the two chains and per tile
 constexpr int kMaxC = 64;     // largest chunk
 
@@ -61,17 +62,17 @@ __device__ __forceinline__ size_t tok_index(const BwdParams &p, int b, int t, in
 // out[r][c] = sum_{i < nterm} A(r, i) scale[i] X[i][c] for r < nrow, c < n, with
 // A(r, i) = A[r * ra + i * ia] in shared memory (so A or its transpose) and
 // scale null meaning 1; written to global memory row-major.  With half = n / 2
-// and rstep = kThreads / half row groups, thread t < rstep half takes the two
+// and rstep = NT / half row groups, thread t < rstep half takes the two
 // columns t % half and t % half + half and the rows t / half + rstep m: each A
 // load serves both columns and each X load all of the thread's rows, with a
 // separate accumulator per output (threads past the last full group idle).
 // n even, 16 <= n <= 128, and ceil(nrow / rstep) <= MAXR.
-template <int MAXR>
+template <int MAXR, int NT = kThreads>
 __device__ __forceinline__ void block_product(const float *A, int ra, int ia, int nrow, int nterm,
                                               const float *scale, const float *X, int xp, int n,
                                               float *out, int tid) {
     const int half = n / 2;
-    const int c = tid % half, rg = tid / half, rstep = kThreads / half;
+    const int c = tid % half, rg = tid / half, rstep = NT / half;
     if (rg >= rstep || rg >= nrow) return;
     const int nr = (nrow - rg + rstep - 1) / rstep;   // rows rg + rstep m < nrow
     float acc0[MAXR], acc1[MAXR];
@@ -105,7 +106,7 @@ __host__ __device__ inline size_t prep_smem_floats(int C, int dk, int dv) {
     return 2 * (size_t)C * (dk + 1) + (size_t)C * (dv + 1) + 3 * (size_t)C * (C + 1) + 4 * (size_t)C;
 }
 
-__global__ void __launch_bounds__(kThreads) bwd_prep_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(const BwdParams p) {
     float *sm = reinterpret_cast<float *>(bwd_smem);
     const int C = p.C, dk = p.dk, dv = p.dv;
     const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(kThreads) bwd_prep_kernel(const BwdParams p) {
     float *eg = bg + C;
     const size_t ch = ((size_t)b * p.H + h) * p.NC + n;
 
-    for (int x = tid; x < C * dk; x += kThreads) {
+    for (int x = tid; x < C * dk; x += kPrepThreads) {
         const int r = x / dk, c = x % dk;
         float kv = 0.f, qv = 0.f;
         if (r < Cn) {
@@ -135,11 +136,11 @@ __global__ void __launch_bounds__(kThreads) bwd_prep_kernel(const BwdParams p) {
         Ks[r * dkp + c] = kv;
         Qs[r * dkp + c] = qv;
     }
-    for (int x = tid; x < C * dv; x += kThreads) {
+    for (int x = tid; x < C * dv; x += kPrepThreads) {
         const int r = x / dv, j = x % dv;
         Vs[r * dvp + j] = r < Cn ? ld_in(p.v, tok_index(p, b, t0 + r, h) * dv + j, p.io_bf16) : 0.f;
     }
-    for (int x = tid; x < C * C; x += kThreads) Ts[(x / C) * Cp + x % C] = 0.f;
+    for (int x = tid; x < C * C; x += kPrepThreads) Ts[(x / C) * Cp + x % C] = 0.f;
     // gates: every token's log alpha and beta in parallel, then the in-chunk scan
     if (tid < C) {
         float la = 0.f, be = 0.f;
@@ -167,10 +168,12 @@ __global__ void __launch_bounds__(kThreads) bwd_prep_kernel(const BwdParams p) {
     __syncthreads();
 
     // L (strictly lower) and M (lower with diagonal).  Thread t takes column
-    // i = t % C and rows t / C + (kThreads / C) k, one pair of accumulators each.
+    // i = t % C and rows t / C + (kPrepThreads / C) k, one pair of accumulators each
+    // (at C = 16 the threads past row 15 have none).
     {
-        constexpr int KR = kMaxC * kMaxC / kThreads;      // rows per thread at C = 64
-        const int i = tid % C, rstep = kThreads / C, nk = C * C / kThreads;
+        constexpr int KR = kMaxC * kMaxC / kPrepThreads;  // rows per thread at C = 64
+        const int i = tid % C, rstep = kPrepThreads / C;
+        const int nk = C * C >= kPrepThreads ? C * C / kPrepThreads : 1;
         float gk[KR], qk[KR];
 #pragma unroll
         for (int k = 0; k < KR; ++k) gk[k] = qk[k] = 0.f;
@@ -188,7 +191,7 @@ __global__ void __launch_bounds__(kThreads) bwd_prep_kernel(const BwdParams p) {
 #pragma unroll
         for (int k = 0; k < KR; ++k) {
             const int r = tid / C + rstep * k;
-            if (k < nk) {
+            if (k < nk && r < C) {
                 float gg = 0.f, m = 0.f;
                 if (r < Cn && i <= r) {
                     const float gam = expf(g[r] - g[i]);
@@ -217,22 +220,26 @@ __global__ void __launch_bounds__(kThreads) bwd_prep_kernel(const BwdParams p) {
     }
     __syncthreads();
 
-    for (int x = tid; x < C * C; x += kThreads) p.ws_T[ch * C * C + x] = Ts[(x / C) * Cp + x % C];
+    for (int x = tid; x < C * C; x += kPrepThreads) p.ws_T[ch * C * C + x] = Ts[(x / C) * Cp + x % C];
     if (tid < C) p.ws_g[ch * C + tid] = g[tid];
     // W = T diag(beta e^g) K and U = T diag(beta) V (zero rows past the tail)
-    block_product<kMaxC * 64 / kThreads>(Ts, Cp, 1, C, Cn, bg, Ks, dkp, dk, p.ws_W + ch * C * dk, tid);
-    block_product<kMaxC * 64 / kThreads>(Ts, Cp, 1, C, Cn, bb, Vs, dvp, dv, p.ws_D + ch * C * dv, tid);
+    block_product<kMaxC * 64 / kPrepThreads, kPrepThreads>(Ts, Cp, 1, C, Cn, bg, Ks, dkp, dk, p.ws_W + ch * C * dk,
+                                                           tid);
+    block_product<kMaxC * 64 / kPrepThreads, kPrepThreads>(Ts, Cp, 1, C, Cn, bb, Vs, dvp, dv, p.ws_D + ch * C * dv,
+                                                           tid);
     __syncthreads();   // V consumed: its buffer takes dO
     float *dOs = Vs;
-    for (int x = tid; x < C * dv; x += kThreads) {
+    for (int x = tid; x < C * dv; x += kPrepThreads) {
         const int r = x / dv, j = x % dv;
         dOs[r * dvp + j] = r < Cn ? ld_in(p.grad_o, tok_index(p, b, t0 + r, h) * dv + j, p.do_bf16) : 0.f;
     }
     __syncthreads();
     // the state-independent parts of the reverse chain: M^T dO (C x dv) and
     // (diag(e^g) Q)^T dO (dk x dv)
-    block_product<kMaxC * 64 / kThreads>(Ms, 1, Cp, C, Cn, nullptr, dOs, dvp, dv, p.ws_Y + ch * C * dv, tid);
-    block_product<128 * 64 / kThreads>(Qs, 1, dkp, dk, Cn, eg, dOs, dvp, dv, p.ws_P + ch * dk * dv, tid);
+    block_product<kMaxC * 64 / kPrepThreads, kPrepThreads>(Ms, 1, Cp, C, Cn, nullptr, dOs, dvp, dv,
+                                                           p.ws_Y + ch * C * dv, tid);
+    block_product<128 * 64 / kPrepThreads, kPrepThreads>(Qs, 1, dkp, dk, Cn, eg, dOs, dvp, dv,
+                                                         p.ws_P + ch * dk * dv, tid);
 }
 
 // ------------------------------------------------------ forward state chain

@@ -1,6 +1,6 @@
 // Test infrastructure: runs the four backward kernels of gdn_bwd_kernels.cuh on
-// the host (see cuda_host_shim.h), grid block by grid block, 256 threads per
-// block.  Before each block the shared-memory array is filled with NaN; after
+// the host (see cuda_host_shim.h), grid block by grid block, with each kernel's
+// block size (512 threads for the prep kernel, 256 for the others).  Before each block the shared-memory array is filled with NaN; after
 // it, every word past the kernel's requested size must still be NaN (nothing
 // wrote past its allocation).  The workspace starts NaN-filled too, so a read
 // of an entry no kernel wrote shows up in the outputs.  Exposes one C entry:
@@ -20,16 +20,16 @@ static void fill_nan(void *p, size_t bytes) {
 static int g_overrun = 0;
 
 template <class F>
-static void run_grid(F kernel, dim3h grid, const BwdParams &p, size_t smem_floats) {
+static void run_grid(F kernel, dim3h grid, const BwdParams &p, size_t smem_floats, int nthreads = bwd::kThreads) {
     for (unsigned z = 0; z < grid.z; ++z)
         for (unsigned y = 0; y < grid.y; ++y)
             for (unsigned x = 0; x < grid.x; ++x) {
                 blockIdx = {x, y, z};
                 fill_nan(bwd::bwd_smem, sizeof(bwd::bwd_smem));
-                std::barrier<> bar(bwd::kThreads);
+                std::barrier<> bar(nthreads);
                 g_block_barrier = &bar;
                 std::vector<std::thread> th;
-                for (int t = 0; t < bwd::kThreads; ++t)
+                for (int t = 0; t < nthreads; ++t)
                     th.emplace_back([&, t] { threadIdx = {(unsigned)t, 0, 0}; kernel(p); });
                 for (auto &t : th) t.join();
                 const uint32_t *u = reinterpret_cast<const uint32_t *>(bwd::bwd_smem);
@@ -70,7 +70,7 @@ extern "C" int host_bwd(int B, int T, int H, int dk, int dv, int C, int io_bf16,
     g_overrun = 0;
     const dim3h per_chunk{(unsigned)p.NC, (unsigned)H, (unsigned)B};
     const dim3h per_slice{(unsigned)(dv / bwd::kCols), (unsigned)H, (unsigned)B};
-    run_grid(bwd::bwd_prep_kernel, per_chunk, p, bwd::prep_smem_floats(C, dk, dv));
+    run_grid(bwd::bwd_prep_kernel, per_chunk, p, bwd::prep_smem_floats(C, dk, dv), bwd::kPrepThreads);
     run_grid(bwd::bwd_state_fwd_kernel, per_slice, p, bwd::state_fwd_smem_floats(C, dk));
     run_grid(bwd::bwd_state_rev_kernel, per_slice, p, bwd::state_rev_smem_floats(C, dk));
     const size_t gs = bwd::grad_smem_floats(C, dk);
