@@ -55,6 +55,20 @@ __device__ __forceinline__ float ld_in(const void *ptr, size_t i, int bf16) {
     return reinterpret_cast<const float *>(ptr)[i];
 }
 
+// Four consecutive inputs from element i (i a multiple of 4; bf16 or fp32).
+__device__ __forceinline__ float4 ld4_in(const void *ptr, size_t i, int bf16) {
+    float4 v;
+    if (bf16) {
+        const uint32_t *u = reinterpret_cast<const uint32_t *>(ptr) + i / 2;
+        const uint32_t a = u[0], b = u[1];
+        v.x = __uint_as_float(a << 16); v.y = __uint_as_float(a & 0xffff0000u);
+        v.z = __uint_as_float(b << 16); v.w = __uint_as_float(b & 0xffff0000u);
+    } else {
+        v = *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(ptr) + i);
+    }
+    return v;
+}
+
 __device__ __forceinline__ size_t tok_index(const BwdParams &p, int b, int t, int h) {
     return ((size_t)b * p.T + t) * p.H + h;
 }
@@ -244,9 +258,9 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(const BwdParams 
 
 // ------------------------------------------------------ forward state chain
 // One block per (batch, head, 32 value columns); walks the chunks in order.
-// Shared memory: h (dk x 33), W, K e^{g_C - g} (C x (dk+1) each), Delta (C x 33).
+// Shared memory: h (dk x 33), W, K (C x (dk+1) each), Delta (C x 33), e^{g_C - g} (C).
 __host__ __device__ inline size_t state_fwd_smem_floats(int C, int dk) {
-    return (size_t)dk * 33 + 2 * (size_t)C * (dk + 1) + (size_t)C * 33;
+    return (size_t)dk * 33 + 2 * (size_t)C * (dk + 1) + (size_t)C * 33 + (size_t)C;
 }
 
 __global__ void __launch_bounds__(kThreads) bwd_state_fwd_kernel(const BwdParams p) {
@@ -260,6 +274,7 @@ __global__ void __launch_bounds__(kThreads) bwd_state_fwd_kernel(const BwdParams
     float *Ws = hs + dk * 33;
     float *Ks = Ws + C * dkp;
     float *Ds = Ks + C * dkp;
+    float *es = Ds + C * 33;
     const size_t bh = (size_t)b * p.H + h;
 
     for (int c = rr; c < dk; c += 8) hs[c * 33 + jj] = p.S0 ? p.S0[(bh * dk + c) * dv + j0 + jj] : 0.f;
@@ -269,15 +284,18 @@ __global__ void __launch_bounds__(kThreads) bwd_state_fwd_kernel(const BwdParams
         __syncthreads();   // h complete; the previous chunk's reads of W, K, Delta done
         for (int c = rr; c < dk; c += 8) p.ws_h[(ch * dk + c) * dv + j0 + jj] = hs[c * 33 + jj];
         const float glast = p.ws_g[ch * C + Cn - 1];
-        for (int x = tid; x < C * dk; x += kThreads) {
-            const int r = x / dk, c = x % dk;
-            Ws[r * dkp + c] = p.ws_W[ch * C * dk + x];
-            float kv = 0.f;
-            if (r < Cn)
-                kv = ld_in(p.k, tok_index(p, b, t0 + r, h) * dk + c, p.io_bf16) *
-                     expf(glast - p.ws_g[ch * C + r]);
-            Ks[r * dkp + c] = kv;
+        // W and the raw keys, four elements a load; the decay e^{g_C - g} goes on the
+        // rows of Delta in the state update instead of on every key element
+        for (int x = tid; x < C * dk / 4; x += kThreads) {
+            const int r = 4 * x / dk, c = 4 * x % dk;
+            const float4 w = *reinterpret_cast<const float4 *>(p.ws_W + ch * C * dk + 4 * x);
+            float4 kv = {0.f, 0.f, 0.f, 0.f};
+            if (r < Cn) kv = ld4_in(p.k, tok_index(p, b, t0 + r, h) * dk + c, p.io_bf16);
+            float *wr = Ws + r * dkp + c, *kr = Ks + r * dkp + c;
+            wr[0] = w.x; wr[1] = w.y; wr[2] = w.z; wr[3] = w.w;
+            kr[0] = kv.x; kr[1] = kv.y; kr[2] = kv.z; kr[3] = kv.w;
         }
+        if (tid < C) es[tid] = tid < Cn ? expf(glast - p.ws_g[ch * C + tid]) : 0.f;
         for (int r = rr; r < C; r += 8) Ds[r * 33 + jj] = p.ws_D[(ch * C + r) * dv + j0 + jj];
         __syncthreads();
         // Delta = U - W h: this thread's columns jp, jp + 16 and rows rg + 16m
@@ -323,7 +341,7 @@ __global__ void __launch_bounds__(kThreads) bwd_state_fwd_kernel(const BwdParams
                 a1[m] = c < dk ? eglast * hs[c * 33 + jp + 16] : 0.f;
             }
             for (int r = 0; r < Cn; ++r) {
-                const float d0 = Ds[r * 33 + jp], d1 = Ds[r * 33 + jp + 16];
+                const float d0 = es[r] * Ds[r * 33 + jp], d1 = es[r] * Ds[r * 33 + jp + 16];
 #pragma unroll
                 for (int m = 0; m < 128 / 16; ++m) {
                     if (rg + 16 * m < dk) {
@@ -378,10 +396,18 @@ __global__ void __launch_bounds__(kThreads) bwd_state_rev_kernel(const BwdParams
         const size_t ch = bh * p.NC + n;
         __syncthreads();   // dh complete; the previous chunk's reads done
         for (int c = rr; c < dk; c += 8) p.ws_dh[(ch * dk + c) * dv + j0 + jj] = dhs[c * 33 + jj];
-        for (int x = tid; x < C * C; x += kThreads) Ts[(x / C) * Cp + x % C] = p.ws_T[ch * C * C + x];
-        for (int x = tid; x < C * dk; x += kThreads) {
-            const int r = x / dk, c = x % dk;
-            Ks[r * dkp + c] = r < Cn ? ld_in(p.k, tok_index(p, b, t0 + r, h) * dk + c, p.io_bf16) : 0.f;
+        for (int x = tid; x < C * C / 4; x += kThreads) {
+            const int r = 4 * x / C, c = 4 * x % C;
+            const float4 t = *reinterpret_cast<const float4 *>(p.ws_T + ch * C * C + 4 * x);
+            float *tr = Ts + r * Cp + c;
+            tr[0] = t.x; tr[1] = t.y; tr[2] = t.z; tr[3] = t.w;
+        }
+        for (int x = tid; x < C * dk / 4; x += kThreads) {
+            const int r = 4 * x / dk, c = 4 * x % dk;
+            float4 kv = {0.f, 0.f, 0.f, 0.f};
+            if (r < Cn) kv = ld4_in(p.k, tok_index(p, b, t0 + r, h) * dk + c, p.io_bf16);
+            float *kr = Ks + r * dkp + c;
+            kr[0] = kv.x; kr[1] = kv.y; kr[2] = kv.z; kr[3] = kv.w;
         }
         if (tid < C) {
             const float gv = p.ws_g[ch * C + tid];
