@@ -188,7 +188,9 @@ def clear_workspace_cache(device: Optional[torch.device] = None) -> None:
     """Drop the cached workspaces (all devices, or one), e.g. when a stream that
     was used for calls is retired.  Each cached buffer holds its bytes until it
     is dropped: about 96 MiB for a split-kernel forward of the 4 x 16 x 4096
-    benchmark shape, 1.4 GB for its backward; the fused forward needs none."""
+    benchmark shape, 263 MB for the SIMT two-gate forward of 2 x 16 x 4096,
+    1.4 GB for the scalar-rule backward of the benchmark shape; the fused and
+    the recurrent forward need none."""
     for key in list(_ws_cache):
         if device is None or (key[0] == device.type and key[1] == device.index):
             del _ws_cache[key]
