@@ -6,9 +6,10 @@
 //    TMEM: the decayed causal scores P_ri = (q_r.k_i) exp(g_r - g_i), i <= r,
 //    and L_ri = beta_r exp(g_r - g_i) (k_r.k_i), i < r (A = -L).  T = (I - A)^-1
 //    exactly (16 x 16 diagonal blocks by forward substitution, merged
-//    16 -> 32 -> 64 by T21 = -T22 L21 T11), or the masked truncated Neumann
-//    series M^(N) (.) sum_{n<=N} A^n (Horner on the band), optionally followed
-//    by the residual correction T0 sum_{s<=S} E^s.  Written to the workspace
+//    16 -> 32 -> 64 by T21 = -T22 L21 T11, the last merge on the tensor cores),
+//    or the masked truncated Neumann series M^(N) (.) sum_{n<=N} A^n by Horner's
+//    rule as N - 1 masked MMAs, or (with the residual correction T0 sum_{s<=S}
+//    E^s) its band form on the CUDA cores.  Written to the workspace
 //    as fp16: T diag(beta), T diag(beta e^g) and P, 24 KB per chunk-head.
 // 2. chain_kernel -- one CTA per (batch, head, 64-column value slice) walks
 //    the chunks in order with the fp32 state h = S^T (128 x 64) in TMEM.
@@ -231,7 +232,93 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tc_fence_before();
         named_bar(1, K1_THREADS);
         bool inv_ok = true;
-        if (p.neumann) {
+        if (p.neumann == 1) {
+            // The masked truncated Neumann series by Horner's rule, T <- M (.) (I + A T),
+            // with the products on the tensor cores: T1 = M (.) (I + A) from L, then
+            // N - 1 steps of one MMA (A and T fp16, fp32 accumulate) and the mask.
+            // A = -L sits in the staging region (its 64 padding rows stay inside the
+            // block), T in the inverse scratch.
+            uint8_t *aS = sm + K1_OFF_STG, *bS = sm + K1_OFF_YB;
+            const uint32_t tI = tmem + 64;
+            const int N = p.N;
+            {
+                const int r = tid >> 2, j0 = (tid & 3) * 2;     // row r, 16-byte chunks j0, j0 + 1
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int j = j0 + q;
+                    float a[8], t[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int c = 8 * j + e, d = r - c;
+                        const float l = Lb[r * LSTR + c];
+                        a[e] = -l;
+                        t[e] = d == 0 ? 1.f : (d > 0 && d <= N ? -l : 0.f);
+                    }
+                    *reinterpret_cast<uint4 *>(aS + sw128_off(r, j)) =
+                        make_uint4(pack_h2(a[0], a[1]), pack_h2(a[2], a[3]), pack_h2(a[4], a[5]), pack_h2(a[6], a[7]));
+                    *reinterpret_cast<uint4 *>(bS + sw128_off(r, j)) =
+                        make_uint4(pack_h2(t[0], t[1]), pack_h2(t[2], t[3]), pack_h2(t[4], t[5]), pack_h2(t[6], t[7]));
+                    if (N <= 1) {
+                        *reinterpret_cast<float4 *>(Tb + r * LSTR + 8 * j) = make_float4(t[0], t[1], t[2], t[3]);
+                        *reinterpret_cast<float4 *>(Tb + r * LSTR + 8 * j + 4) = make_float4(t[4], t[5], t[6], t[7]);
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(1, K1_THREADS);
+#pragma unroll 1
+            for (int step = 1; step < N; ++step) {
+                if (tid == 0) {
+                    // D = [A ; any 64 rows] T (TMEM lanes 0..63 real), K = 64 in four MMAs
+                    tc_fence_after();
+                    const uint32_t aa = smem_u32(aS), bb = smem_u32(bS);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ss(tI, sdesc_sw128(aa + kk * 32, 16, 1024), sdesc_sw128(bb + kk * 2048, 16384, 1024),
+                                    IDESC_KM64, kk > 0);
+                    umma_commit(&bars[2]);
+                    const bool w = mbar_wait(&bars[2], (step - 1) & 1, abort_flag, E_K1_MMA, kWaitLimit);
+                    if (!w) mbar_wait_drain(&bars[2], (step - 1) & 1, kWaitLimit);
+                    *okflag = w ? 1 : 0;
+                }
+                __syncwarp();
+                named_bar(1, K1_THREADS);
+                if (!*okflag) { inv_ok = false; break; }
+                mbar_try_wait(&bars[2], (step - 1) & 1);
+                tc_fence_after();
+                if ((warp & 3) < 2) {
+                    // warps 0, 1, 4, 5: rows 32 sp + lane, columns [32 hf, 32 hf + 32)
+                    const int sp = warp & 3, hf = warp >> 2, r = 32 * sp + lane;
+                    const bool last = (step == N - 1);
+                    uint32_t x[32];
+                    tmem_ld32(tI + ((uint32_t)(32 * sp) << 16) + 32 * hf, x);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        float t[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int c = 32 * hf + 8 * jj + e, d = r - c;
+                            t[e] = d == 0 ? 1.f : (d > 0 && d <= N ? __uint_as_float(x[8 * jj + e]) : 0.f);
+                        }
+                        if (last) {
+                            float *dst = Tb + r * LSTR + 32 * hf + 8 * jj;
+                            *reinterpret_cast<float4 *>(dst) = make_float4(t[0], t[1], t[2], t[3]);
+                            *reinterpret_cast<float4 *>(dst + 4) = make_float4(t[4], t[5], t[6], t[7]);
+                        } else {
+                            *reinterpret_cast<uint4 *>(bS + sw128_off(r, 4 * hf + jj)) =
+                                make_uint4(pack_h2(t[0], t[1]), pack_h2(t[2], t[3]), pack_h2(t[4], t[5]),
+                                           pack_h2(t[6], t[7]));
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar(1, K1_THREADS);
+            }
+        } else if (p.neumann) {
+            // the residual-corrected series keeps the band form on the CUDA cores
             tc::invert_neumann(Lb, Tb, Yb, tid, p.N, 1);
         } else {
             // T = (I + L)^-1: the 16 x 16 diagonal blocks and the 16 -> 32 merges on
