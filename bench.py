@@ -519,6 +519,10 @@ def forward_line(args, rank, world, local_rank, name, over, timed_steps):
         o_n = o32.double().cpu().numpy()
         s_n = S_T.double().cpu().numpy()
         a.mode, a.neumann_N = 0, 0
+        ws_x = gdn.workspace_for(a, dev)    # exact inversion may run on another kernel
+        if ws_x is not None:
+            a.workspace, a.workspace_bytes = ws_x.data_ptr(), ws_x.numel()
+        exact_kernel = KERNEL_NAMES.get(gdn.select_kernel(a), "?")
         step()
         torch.cuda.synchronize()
         o_x = o32.double().cpu().numpy()
@@ -529,10 +533,12 @@ def forward_line(args, rank, world, local_rank, name, over, timed_steps):
         mo_o, ro_o = max_rel_rms(o_n, o_ref)
         mo_s, ro_s = max_rel_rms(s_n, s_ref)
         accuracy = dict(
-            vs_exact=dict(o_max_rel_rms=m_o, o_rms_rel=r_o, S_T_max_rel_rms=m_s, S_T_rms_rel=r_s,
-                          exact_kernel=kernel_name),
-            vs_oracle=dict(o_max_rel_rms=mo_o, o_rms_rel=ro_o, S_T_max_rel_rms=mo_s, S_T_rms_rel=ro_s),
-            tolerance="bf16 bar: max|err| <= 2e-2 * rms(oracle) on o and S_T (o in fp32 for this comparison)")
+            vs_exact_inverse=dict(o_max_rel_rms=m_o, o_rms_rel=r_o, S_T_max_rel_rms=m_s, S_T_rms_rel=r_s,
+                                  exact_kernel=exact_kernel),
+            vs_exact_oracle=dict(o_max_rel_rms=mo_o, o_rms_rel=ro_o, S_T_max_rel_rms=mo_s, S_T_rms_rel=ro_s),
+            note="the truncated series' method error against exact inversion (this library in exact "
+                 "mode) and against the fp64 token recurrence, o in fp32; parity with the masked-series "
+                 "oracle (max|err| <= 2e-2 * rms) is the tests' check, not this one")
 
     backward = None
     if name == "gdn_bf16" and args.bwd_steps > 0 and world == 1:

@@ -29,6 +29,7 @@ struct FwdParams {
     int mode, N;
     int S;              // residual-correction terms (GDN_INV_NEUMANN_RESIDUAL)
     int general;        // two-gate rule (per-channel decay / gates / preconditioner)
+    int pair;           // tensor-core path: a 128-token chunk of the masked series run as two 64-token halves
 };
 
 // SIMT fp32 chunk kernel: shared-memory bytes for p, or 0 if p does not fit.

@@ -105,10 +105,21 @@ constexpr uint32_t K1_SMEM_RES = K1_OFF_RES + 3 * K1_MAT + 1024;
 struct K1Params {
     int B, T, H, NC;
     const float *alpha, *beta;
+    const void *k;      // bf16 [B, T, H, DK] (the boundary window of a 128-token chunk)
     uint8_t *ws;
+    float *pair_ws;     // chunk 128 as two halves: per chunk-head, C1 and C2' (second halves only)
     int neumann, N;     // neumann: 1 truncated series, 2 series + residual correction
     int S;              // residual-correction terms
 };
+
+// Chunk 128 of the masked series as two 64-token halves a, b.  The second half's
+// Delta differs from that of a 64-token chunk only through the band's corner T_ba
+// (rows 0..N-1 of b, columns 64-N..63 of a) and through the state at the start of
+// the 128-token chunk: Delta_b = U_b - (W_b + C2') e^{g_aC} h_a + C1 V_a, with
+// C1 = T_ba diag(beta_a) (N x N over a's last N rows) and
+// C2' = T_ba diag(beta_a e^{g_a - g_aC}) K_a (N x DK).  Per chunk-head, fp32:
+constexpr int PAIR_MAXN = 16;
+constexpr int PAIR_C1 = 0, PAIR_C2 = PAIR_MAXN * PAIR_MAXN, PAIR_STRIDE = PAIR_C2 + PAIR_MAXN * 128;
 
 // One CTA per (chunk, head, batch).  [Q ; K] K^T in one MMA: TMEM lanes 0..63
 // hold Q K^T (-> P), lanes 64..127 hold K K^T (-> L -> T).
@@ -424,6 +435,99 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
         }
     }
+    if (p.pair_ws && (n & 1)) block_sync();
+    if (p.pair_ws && (n & 1) && *abort_flag == 0) {
+        // Second half of a 128-token chunk: the corner of the 128-token chunk's masked
+        // series from the 2N-token window around the halves' boundary (window rows
+        // w < N: a's rows 64 - N + w; w >= N: b's rows w - N), then C1 and C2'.
+        // The tile region is free by now (the series' MMAs and the stores are done).
+        const int N = p.N, NW = 2 * N;
+        float *kw = Lb;                          // NW x 129
+        float *aw = Lb + 32 * 129;               // NW x 33: A of the window, then T
+        float *tw = aw + 32 * 33;                // NW x 33
+        float *gw = tw + 32 * 33;                // NW: cumulative log decay over the window
+        float *bw = gw + 32;                     // NW: beta
+        float *ew = bw + 32;                     // N: e^{g_j - g_{N-1}}, decay to the first half's end
+        float *cw = ew + 32;                     // N x N: C1
+        for (int x = tid; x < NW * 128; x += K1_THREADS) {
+            const int w = x >> 7, c = x & 127, t = t0 - N + w;
+            float kv = 0.f;
+            if (t < p.T) {
+                const uint16_t u = reinterpret_cast<const uint16_t *>(p.k)[(((size_t)b * p.T + t) * p.H + h) * 128 + c];
+                kv = __uint_as_float((uint32_t)u << 16);
+            }
+            kw[w * 129 + c] = kv;
+        }
+        if (warp == 0) {
+            // window gates: log alpha (0 past the end) scanned over the window, beta (0 past the end)
+            float la = 0.f, be = 0.f;
+            if (lane < NW) {
+                const int t = t0 - N + lane;
+                if (t < p.T) {
+                    const size_t ti = ((size_t)b * p.T + t) * p.H + h;
+                    la = p.alpha ? logf(p.alpha[ti]) : 0.f;
+                    be = p.beta ? p.beta[ti] : 1.f;
+                }
+            }
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, la, o);
+                if (lane >= o) la += y;
+            }
+            if (lane < NW) { gw[lane] = la; bw[lane] = be; }
+        }
+        block_sync();
+        // A_ij = -beta_i exp(g_i - g_j) k_i.k_j (i > j) over the window; T = M (.) (I + A T), N steps
+        for (int x = tid; x < NW * NW; x += K1_THREADS) {
+            const int i = x / NW, j = x % NW;
+            float a = 0.f;
+            if (j < i) {
+                float d = 0.f;
+                for (int c = 0; c < 128; ++c) d += kw[i * 129 + c] * kw[j * 129 + c];
+                a = -bw[i] * expf(gw[i] - gw[j]) * d;
+            }
+            aw[i * 33 + j] = a;
+            tw[i * 33 + j] = (i == j) ? 1.f : 0.f;
+        }
+        block_sync();
+        for (int step = 0; step < N; ++step) {
+            float val[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int x = tid + K1_THREADS * q, i = x / NW, j = x % NW;
+                val[q] = 0.f;
+                if (x < NW * NW && i - j >= 0 && i - j <= N) {
+                    float sacc = (i == j) ? 1.f : 0.f;
+                    for (int kk = j; kk < i; ++kk) sacc += aw[i * 33 + kk] * tw[kk * 33 + j];
+                    val[q] = sacc;
+                }
+            }
+            block_sync();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int x = tid + K1_THREADS * q;
+                if (x < NW * NW) tw[(x / NW) * 33 + x % NW] = val[q];
+            }
+            block_sync();
+        }
+        // C1[i][j] = T[N + i][j] beta_j;  C2'[i][c] = sum_j C1[i][j] e^{g_j - g_{N-1}} k_j[c]
+        float *dst = p.pair_ws + (((size_t)b * p.H + h) * p.NC + n) * PAIR_STRIDE;
+        if (tid < N) ew[tid] = expf(gw[tid] - gw[N - 1]);
+        for (int x = tid; x < PAIR_MAXN * PAIR_MAXN; x += K1_THREADS) {
+            const int i = x / PAIR_MAXN, j = x % PAIR_MAXN;
+            const float c1 = (i < N && j < N) ? tw[(N + i) * 33 + j] * bw[j] : 0.f;
+            cw[x] = c1;
+            dst[PAIR_C1 + x] = c1;
+        }
+        block_sync();
+        for (int x = tid; x < PAIR_MAXN * 128; x += K1_THREADS) {
+            const int i = x >> 7, c = x & 127;
+            float acc = 0.f;
+            if (i < N)
+                for (int j = 0; j < N; ++j) acc += cw[i * PAIR_MAXN + j] * ew[j] * kw[j * 129 + c];
+            dst[PAIR_C2 + x] = acc;
+        }
+    }
     tc_fence_before();
     block_sync();
     if (warp == 0) {
@@ -440,36 +544,45 @@ constexpr int KS_THREADS = 256, CH_THREADS = 128;
 // Main stage (x3): per 64-column key block kb: [W | Q | K] at kb * 24 KB, then
 // P.  It holds a chunk from its load until the chain's MMAs of the chunk are
 // complete; three of them let the load of chunk m + 2 start while the key side
-// works on m + 1 and the chain on m.
-constexpr int NSTAGE = 3;
+// works on m + 1 and the chain on m.  A 128-token chunk of the masked series,
+// run as two 64-token halves, keeps two stages: its extra tiles take the third.
 constexpr uint32_t MSTG = 57344;
 constexpr uint32_t S_W = 0, S_Q = 8192, S_K = 16384, S_KB = 24576, S_P = 49152;
 constexpr uint32_t MAIN_TX = 40960;                    // bytes loaded per main stage: Q, K, P
 // Early slot (x1): T diag(beta), T diag(beta e^g) and the V slice, read only by
 // the U and W MMAs and reloaded as soon as those are complete.
-constexpr uint32_t OFF_EARLY = NSTAGE * MSTG;
 constexpr uint32_t ES_TB = 0, ES_TBG = 8192, ES_V = 16384;
 constexpr uint32_t EARLY_TX = 24576;
 // Every M = 128 MMA whose A operand has only 64 real rows also reads the 8 KB
 // next to them; the lanes those rows produce are never read.  The neighbours
 // are not rewritten while the MMA runs: U reads T diag(beta) + T diag(beta e^g),
 // W reads T diag(beta e^g) + V, the output MMA the second K block + P.
-constexpr uint32_t OFF_HS = OFF_EARLY + EARLY_TX;      // h fp16, 128 rows
-constexpr uint32_t OFF_DS = OFF_HS + 16384;            // Delta fp16 x 2
-constexpr uint32_t OFF_PAR = OFF_DS + 2 * 8192;
 constexpr uint32_t PAR_BYTES = (sizeof(tc::ChainParams) + 15) & ~15u;
-constexpr uint32_t OFF_BAR = OFF_PAR + 3 * PAR_BYTES;   // gate ring of 3
 enum { B_FULL = 0, B_EMPTY = 3, B_EFULL = 6, B_EEMPTY = 7, B_KSREADY = 8, B_KSFREE = 10, B_UW = 12, B_X = 13,
        B_H = 14, B_O = 15, B_XISS = 17, B_DREADY = 18, N_BARS = 20 };
-static_assert((MSTG & 1023) == 0 && (OFF_EARLY & 1023) == 0 && (OFF_HS & 1023) == 0 && (OFF_DS & 1023) == 0,
-              "swizzled tiles on 1024-byte boundaries");
-constexpr uint32_t OFF_MISC = OFF_BAR + N_BARS * 8;     // tmem slot, abort flag, group slots
-constexpr uint32_t SMEM_USED = OFF_MISC + 32;
-constexpr uint32_t K2_SMEM = SMEM_USED + 1024;
-static_assert(K2_SMEM <= 232448, "shared memory budget of one sm_100 block");
+// Shared-memory layout of the chain kernel; PAIR: 128-token chunks as two halves.
+template <bool PAIR> struct K2Layout {
+    static constexpr int NSTAGE = PAIR ? 2 : 3;
+    static constexpr uint32_t EARLY = NSTAGE * MSTG;
+    static constexpr uint32_t HS = EARLY + EARLY_TX;            // h fp16, 128 rows
+    static constexpr uint32_t HH = HS + 16384;                  // PAIR: e^{g_C} h of a first half, fp16
+    static constexpr uint32_t DS = HH + (PAIR ? 16384 : 0);     // Delta fp16 x 2
+    static constexpr uint32_t CORNER = DS + 2 * 8192;           // PAIR: C1 V_a, 16 x 64 fp32
+    static constexpr uint32_t C2S = CORNER + (PAIR ? 4096 : 0); // PAIR: C2', 16 x 128 fp32
+    static constexpr uint32_t PAR = C2S + (PAIR ? 8192 : 0);
+    static constexpr uint32_t BAR = PAR + 3 * PAR_BYTES;        // gate ring of 3
+    static constexpr uint32_t MISC = BAR + N_BARS * 8;          // tmem slot, abort flag, group slots
+    static constexpr uint32_t SMEM = MISC + 32 + 1024;
+    static_assert((EARLY & 1023) == 0 && (HS & 1023) == 0 && (HH & 1023) == 0 && (DS & 1023) == 0,
+                  "swizzled tiles on 1024-byte boundaries");
+    static_assert(SMEM <= 232448, "shared memory budget of one sm_100 block");
+};
+static_assert((MSTG & 1023) == 0, "swizzled tiles on 1024-byte boundaries");
 static_assert(K1_SMEM * K1_BLOCKS_PER_SM <= 233472, "key-side blocks per SM");
 static_assert(K1_SMEM_RES <= 232448, "residual-correction key-side block fits one SM");
 static_assert(K1_OFF_YB + 8192 <= K1_OFF_TB, "L and the inverse scratch fit in the tile region");
+static_assert((32 * 129 + 2 * 32 * 33 + 3 * 32 + PAIR_MAXN * PAIR_MAXN) * 4 <= K1_OFF_TB,
+              "the boundary window of a 128-token chunk fits in the tile region");
 static_assert(K1_OFF_LB + K1_MAT <= K1_OFF_B2 && K1_OFF_B2 + 4096 <= K1_OFF_A1 && K1_OFF_A1 + 4096 <= K1_OFF_TB &&
               K1_OFF_A1 + 16384 <= K1_OFF_TB + K1_MAT && (K1_OFF_B2 & 1023) == 0 && (K1_OFF_A1 & 1023) == 0 &&
               K1_OFF_A2 + 16384 + 1024 <= K1_SMEM,
@@ -477,16 +590,21 @@ static_assert(K1_OFF_LB + K1_MAT <= K1_OFF_B2 && K1_OFF_B2 + 4096 <= K1_OFF_A1 &
 
 // TMEM columns
 constexpr uint32_t TM_U0 = 0, TM_U1 = 64, TM_W = 128, TM_X0 = 256, TM_X1 = 320, TM_H = 384;
+constexpr uint32_t TM_XB = 448;     // PAIR, second halves: [-(W + C2') ; Q'] e^{g_C} h of the first half
 constexpr uint32_t TM_COLS = 512;
 
 struct K2Params {
     int B, T, H, dv, NC;
     const float *alpha, *beta, *S0;
+    const void *v;          // bf16 [B, T, H, dv] (PAIR: the first half's last N rows)
+    const float *pair_ws;   // PAIR: C1 and C2' of every second half
+    int N;                  // PAIR: band of the masked series
     void *o;
     float *S_T;
     int o_bf16;
 };
 
+template <bool PAIR>
 __global__ void __launch_bounds__(K2_THREADS, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_t,
@@ -500,6 +618,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int T = p.T, H = p.H, dv = p.dv, NC = p.NC;
     const int v0 = slice * DVS;
+    using L = K2Layout<PAIR>;
+    constexpr int NSTAGE = L::NSTAGE;
+    constexpr uint32_t OFF_EARLY = L::EARLY, OFF_HS = L::HS, OFF_DS = L::DS, OFF_PAR = L::PAR, OFF_BAR = L::BAR,
+                       OFF_MISC = L::MISC;
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC);
@@ -669,6 +791,15 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             }
             if (!sync_ok(1, KS_THREADS, leader, kcnt)) break;
             if (!lwarp) mbar_try_wait(&bars[B_FULL + ms], (m / NSTAGE) & 1);
+            // second half of a 128-token chunk: C2' (16 x 128) -> shared memory; the
+            // loads are in flight while the operands below are converted
+            float4 c2a = make_float4(0.f, 0.f, 0.f, 0.f), c2b = c2a;
+            if (PAIR && (m & 1)) {
+                const float4 *src = reinterpret_cast<const float4 *>(
+                    p.pair_ws + (((size_t)b * H + h) * NC + m) * PAIR_STRIDE + PAIR_C2);
+                c2a = src[kt];
+                c2b = src[kt + 256];
+            }
             // in-place fp16 operands: Q -> e^{g_r} Q, K -> K in the main stage, then
             // V in the early slot once it has landed.  Every load of a pass is
             // issued before the first store, so they overlap instead of waiting on
@@ -716,6 +847,11 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 }
                 convert(addr, sc, 2);
             }
+            if (PAIR && (m & 1)) {
+                float4 *dst = reinterpret_cast<float4 *>(sm + L::C2S);
+                dst[kt] = c2a;
+                dst[kt + 256] = c2b;
+            }
             fence_proxy_async_smem();
             tc_fence_before();
             if (!sync_ok(1, KS_THREADS, leader, kcnt)) break;
@@ -757,8 +893,15 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 const int r = 32 * sp + lane;
                 float x[64];
                 tmem_ld64(tmem + ((uint32_t)(32 * sp) << 16) + TM_W + 64 * hf, x);
+                if (PAIR && (m & 1) && r < PAIR_MAXN) {
+                    // -(W + C2'): the band corner's key part of a second half
+                    const float *c2 = reinterpret_cast<const float *>(sm + L::C2S) + r * 128 + 64 * hf;
 #pragma unroll
-                for (int j = 0; j < 64; ++j) x[j] = -x[j];
+                    for (int j = 0; j < 64; ++j) x[j] = -x[j] - c2[j];
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) x[j] = -x[j];
+                }
                 st_row_f16(st + hf * S_KB + S_W, r, x);
             } else {
                 // W has read K: K -> diag(e^{g_C - g}) K in place for the state update
@@ -896,6 +1039,13 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     tmem_st32(tmem + lane_base + TM_H + 32 * hh, y);
                 }
                 st_row_f16(hs, hrow, x);
+                if (PAIR && !(n & 1) && n + 1 < NC) {
+                    // first half of a 128-token chunk: e^{g_C} h, the state the second
+                    // half's Delta is formed from
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) x[j] *= egC;
+                    st_row_f16(sm + L::HH, hrow, x);
+                }
                 tmem_wait_st();
             }
             fence_proxy_async_smem();
@@ -916,12 +1066,42 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     umma_f16_ss(tmem + xcol, sdesc_sw128(a0 + S_W + aoff, 16, 1024),
                                 sdesc_sw128(b0 + kk * 2048, 8192, 1024), IDESC_KM64, kk > 0);
                 }
+                if (PAIR && (n & 1)) {
+                    // second half: [-(W + C2') ; Q'] (e^{g_C} h of the first half); only
+                    // its lanes 0..63 are read
+                    const uint32_t b1 = smem_u32(sm + L::HH);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t aoff = (kk >> 2) * S_KB + (kk & 3) * 32;
+                        umma_f16_ss(tmem + TM_XB, sdesc_sw128(a0 + S_W + aoff, 16, 1024),
+                                    sdesc_sw128(b1 + kk * 2048, 8192, 1024), IDESC_KM64, kk > 0);
+                    }
+                }
                 umma_commit(&bars[B_X]);
                 mbar_arrive(&bars[B_XISS]);
                 pend = B_X; pend_par = n & 1;
             }
             __syncwarp();
             if (!rowpart) {
+                if (PAIR && !(n & 1) && n + 1 < NC) {
+                    // first half of a 128-token chunk: the corner's value part of the
+                    // second half, C1 V_a (V_a: this chunk's last N rows), column ct
+                    const float *c1 = p.pair_ws + (bh * NC + n + 1) * PAIR_STRIDE + PAIR_C1;
+                    const uint16_t *vp = reinterpret_cast<const uint16_t *>(p.v) +
+                                         (((size_t)b * T + (n * C + C - p.N)) * H + h) * dv + v0 + ct;
+                    float vv[PAIR_MAXN];
+#pragma unroll
+                    for (int j = 0; j < PAIR_MAXN; ++j)
+                        vv[j] = j < p.N ? __uint_as_float((uint32_t)vp[(size_t)j * H * dv] << 16) : 0.f;
+                    float *cr = reinterpret_cast<float *>(sm + L::CORNER);
+#pragma unroll 4
+                    for (int i = 0; i < PAIR_MAXN; ++i) {
+                        float acc = 0.f;
+#pragma unroll
+                        for (int j = 0; j < PAIR_MAXN; ++j) acc += c1[i * PAIR_MAXN + j] * vv[j];
+                        cr[i * 64 + ct] = acc;
+                    }
+                }
                 // sub-partitions 2, 3: output rows of the previous chunk, off the chain
                 if (n > 0) out_rows(n - 1);
                 continue;
@@ -932,10 +1112,16 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             {
                 const int r = 32 * sp + lane;
                 float x[64], u[64];
-                tmem_ld64(tmem + lane_base + xcol, x);
+                tmem_ld64(tmem + lane_base + ((PAIR && s) ? TM_XB : xcol), x);
                 tmem_ld64(tmem + lane_base + (s ? TM_U1 : TM_U0), u);
 #pragma unroll
                 for (int j = 0; j < 64; ++j) x[j] += u[j];
+                if (PAIR && s && r < PAIR_MAXN) {
+                    // second half: + C1 V_a, the corner's value part
+                    const float *cr = reinterpret_cast<const float *>(sm + L::CORNER) + r * 64;
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) x[j] += cr[j];
+                }
                 st_row_f16(sm + OFF_DS + s * 8192, r, x);
             }
             fence_proxy_async_smem();
@@ -1038,7 +1224,10 @@ bool make_map_t(CUtensorMap *m, const void *ptr, size_t rows) {
 bool tc_supports(const FwdParams &p, const char **why) {
     if (!p.io_bf16) { *why = "needs bf16 q/k/v"; return false; }
     if (p.general) { *why = "two-gate rule runs on the SIMT kernel"; return false; }
-    if (p.C != C) { *why = "needs chunk 64"; return false; }
+    if (p.C != C && !(p.C == 2 * C && p.mode == GDN_INV_NEUMANN)) {
+        *why = "needs chunk 64 (or 128 with the masked series)";
+        return false;
+    }
     if (p.dk != DK) { *why = "needs dk 128"; return false; }
     if (p.dv % DVS != 0) { *why = "needs dv a multiple of 64"; return false; }
     if (p.mode != GDN_INV_EXACT && p.N > kNeumannMaxN) { *why = "Neumann N > 15"; return false; }
@@ -1050,7 +1239,8 @@ int tc_default_slices(const FwdParams &p) { return p.dv / DVS; }
 
 size_t tc_workspace_bytes(const FwdParams &p) {
     const size_t nc = (size_t)(p.T + C - 1) / C;
-    return (size_t)p.B * p.H * nc * WS_CHUNK_BYTES;
+    const size_t per = WS_CHUNK_BYTES + (p.C == 2 * C ? (size_t)PAIR_STRIDE * 4 : 0);
+    return (size_t)p.B * p.H * nc * per;
 }
 
 cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, const char **why) {
@@ -1064,16 +1254,27 @@ cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, 
     }
     // The attribute belongs to the current device: set it on every launch (cheap)
     // rather than behind a process-wide flag that a second device would not share.
+    // A 128-token chunk of the masked series runs as two 64-token halves ("pair"):
+    // the second halves' band corners go to the workspace after the T matrices.
+    const bool pair = p.C == 2 * C;
+    float *pair_ws = pair ? reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) +
+                                                      (size_t)p.B * p.H * NC * WS_CHUNK_BYTES)
+                          : nullptr;
     {
         cudaError_t e = cudaFuncSetAttribute(keyside_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)K1_SMEM_RES);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K2_SMEM);
+        e = pair ? cudaFuncSetAttribute(chain_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)K2Layout<true>::SMEM)
+                 : cudaFuncSetAttribute(chain_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)K2Layout<false>::SMEM);
         if (e != cudaSuccess) return e;
     }
     K1Params k1;
     k1.B = p.B; k1.T = p.T; k1.H = p.H; k1.NC = NC;
     k1.alpha = p.alpha; k1.beta = p.beta;
+    k1.k = p.k;
+    k1.pair_ws = pair_ws;
     k1.ws = reinterpret_cast<uint8_t *>(workspace);
     k1.neumann = p.mode == GDN_INV_NEUMANN ? 1 : (p.mode == GDN_INV_NEUMANN_RESIDUAL ? 2 : 0);
     k1.N = p.N; k1.S = p.S;
@@ -1083,8 +1284,14 @@ cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, 
     K2Params k2;
     k2.B = p.B; k2.T = p.T; k2.H = p.H; k2.dv = p.dv; k2.NC = NC;
     k2.alpha = p.alpha; k2.beta = p.beta; k2.S0 = p.S0; k2.o = p.o; k2.S_T = p.S_T;
+    k2.v = p.v; k2.pair_ws = pair_ws; k2.N = p.N;
     k2.o_bf16 = p.o_bf16;
-    chain_kernel<<<dim3(p.slices, p.H, p.B), K2_THREADS, K2_SMEM, stream>>>(mq, mk, mv, mt, k2);
+    if (pair)
+        chain_kernel<true><<<dim3(p.slices, p.H, p.B), K2_THREADS, K2Layout<true>::SMEM, stream>>>(mq, mk, mv, mt,
+                                                                                                  k2);
+    else
+        chain_kernel<false><<<dim3(p.slices, p.H, p.B), K2_THREADS, K2Layout<false>::SMEM, stream>>>(mq, mk, mv,
+                                                                                                    mt, k2);
     return cudaGetLastError();
 }
 

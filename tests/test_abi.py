@@ -118,6 +118,13 @@ def test_valid_arguments_select_a_kernel():
     assert gdn.select_kernel(_args(alpha=0x70000, precond=1, erase=0x50000,
                                    write=0x58000, alpha_per_channel=1)) in (1, 2)
     assert gdn.select_kernel(_args(S0=0x80000, S_T=0x80000)) in (1, 2, 4)  # S_T may alias S0
+    # chunk 128: the masked series (N <= 15) on the split kernels as two 64-token
+    # halves; the exact inverse and wider bands on the SIMT kernel
+    assert gdn.select_kernel(_args(chunk=128, mode=1, neumann_N=3)) == 4
+    assert gdn.select_kernel(_args(chunk=128, mode=1, neumann_N=15)) == 4
+    assert gdn.select_kernel(_args(chunk=128, mode=1, neumann_N=16)) == 1
+    assert gdn.select_kernel(_args(chunk=128)) == 1
+    assert gdn.select_kernel(_args(chunk=128, mode=2, neumann_N=3, residual_S=8)) < 0
 
 
 def test_fault_injection_env(monkeypatch):
@@ -273,6 +280,10 @@ def test_workspace_sizes_per_kernel():
     c128 = _args(kernel=1, chunk=128, mode=1, neumann_N=3)
     per128 = 2 * 128 * 128 + 3 * 128 * dk + dk
     assert gdn.workspace_bytes(c128) == B * H * 1 * per128 * 4
+    # chunk 128 on the split kernels: per 64-token half the 24 KiB of T matrices and
+    # the band corner (C1: 16 x 16, C2': 16 x dk, fp32)
+    assert gdn.workspace_bytes(_args(kernel=4, chunk=128, mode=1, neumann_N=3)) == \
+        chunks * (24576 + (16 * 16 + 16 * dk) * 4)
 
 
 def test_simt_call_without_workspace_rejected_on_host():

@@ -200,7 +200,7 @@ def test_neumann_sweep_lines(fake_cuda, monkeypatch):
     seen = set()
     for ln in lines:
         acc = ln["accuracy"]
-        assert set(acc) >= {"vs_exact", "vs_oracle", "tolerance"}
+        assert set(acc) >= {"vs_exact_inverse", "vs_exact_oracle", "note"}
         seen.add((ln["config"]["workload"].split("chunk=")[1].split()[0],
                   ln["config"]["workload"].split("N=")[1].split(",")[0]))
     assert seen == {(c, n) for c in ("64", "128") for n in ("2", "3", "4")}

@@ -89,6 +89,20 @@ def test_neumann_sweep(chunk, N):
     report(f"neumann_C{chunk}_N{N}_vs_exact_oracle", o=stats(o, o_ex), S_T=stats(s, s_ex))
 
 
+@needs_cuda
+@pytest.mark.parametrize("T,N,s0", [(1000, 15, 0.02), (900, 1, 0.0), (129, 7, 0.02), (640, 0, 0.02),
+                                    (4096, 3, 0.02)])
+def test_neumann_chunk128_halves_ragged(T, N, s0):
+    """Chunk 128 of the masked series on the split tensor-core kernels: each
+    128-token chunk runs as two 64-token halves plus the band's corner between
+    them.  Ragged ends (a partial second half; a lone first half), the widest band
+    (N = 15), N = 0 (T = I: no corner) and a nonzero initial state."""
+    w = workload("neumann", B=2, H=2, T=T, chunk=128, neumann_N=N, s0_std=s0)
+    x = make_inputs(w, seed=40 + N)
+    o_ref, s_ref = run_oracle(x, w)
+    _check_bf16(f"neumann_C128_halves_T{T}_N{N}", w, x, o_ref, s_ref, kernel="tc_split")
+
+
 # ------------------------------------------- residual correction (next row 1)
 
 @needs_cuda
