@@ -328,11 +328,15 @@ KERNEL_SOURCES = {1: SIMT_SOURCES, 2: FWD_SOURCES, 3: DECODE_SOURCES, 4: SPLIT_S
 def forward_runs(args):
     """(workload name, overrides) of every line this invocation prints."""
     name = args.workload
+    chunk = getattr(args, "chunk", 0)
     if name == "neumann":
-        return [(name, dict(chunk=c, mode="neumann", neumann_N=n)) for c in (64, 128) for n in (2, 3, 4)]
+        return [(name, dict(chunk=c, mode="neumann", neumann_N=n)) for c in ((chunk,) if chunk else (64, 128))
+                for n in (2, 3, 4)]
     over = {}
     if args.mode != "exact" and name == "gdn_bf16":
         over = dict(mode=args.mode, neumann_N=args.N)
+    if chunk:
+        over["chunk"] = chunk
     return [(name, over)]
 
 
@@ -402,9 +406,13 @@ def forward_line(args, rank, world, local_rank, name, over, timed_steps):
         a.workspace_bytes = ws.numel()
     kernel_id = gdn.select_kernel(a)
     kernel_name = KERNEL_NAMES.get(kernel_id, "?")
-    # split tensor-core path: key side + chain; SIMT path: prep + chain, plus the two
-    # scan kernels of the preconditioner's running average
-    launches_per_call = {4: 2, 1: 4 if (w.precond and general) else 2}.get(kernel_id, 1)
+    # split tensor-core path: key side + chain (chunk 128: the band-corner kernel first
+    # when there is a second half); SIMT path: prep + chain, plus the two scan kernels
+    # of the preconditioner's running average
+    pair = kernel_id == 4 and w.chunk == 128 and w.T > 64
+    if pair:
+        kernel_name = "pair_corner_kernel+" + kernel_name
+    launches_per_call = {4: 3 if pair else 2, 1: 4 if (w.precond and general) else 2}.get(kernel_id, 1)
     sh = stream.cuda_stream
 
     def step():
@@ -1017,6 +1025,8 @@ def main():
                     help="backward calls timed for the forward line's 'backward' object (0: none)")
     ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tc", "tc_split"],
                     help="force one forward kernel (auto: the library's choice)")
+    ap.add_argument("--chunk", type=int, default=0,
+                    help="chunk length (0: the workload's own; for --workload neumann, the lines of that chunk only)")
     ap.add_argument("--N", type=int, default=3)
     ap.add_argument("--S", type=int, default=8)
     args = ap.parse_args()

@@ -105,9 +105,7 @@ constexpr uint32_t K1_SMEM_RES = K1_OFF_RES + 3 * K1_MAT + 1024;
 struct K1Params {
     int B, T, H, NC;
     const float *alpha, *beta;
-    const void *k;      // bf16 [B, T, H, DK] (the boundary window of a 128-token chunk)
     uint8_t *ws;
-    float *pair_ws;     // chunk 128 as two halves: per chunk-head, C1 and C2' (second halves only)
     int neumann, N;     // neumann: 1 truncated series, 2 series + residual correction
     int S;              // residual-correction terms
 };
@@ -117,9 +115,165 @@ struct K1Params {
 // (rows 0..N-1 of b, columns 64-N..63 of a) and through the state at the start of
 // the 128-token chunk: Delta_b = U_b - (W_b + C2') e^{g_aC} h_a + C1 V_a, with
 // C1 = T_ba diag(beta_a) (N x N over a's last N rows) and
-// C2' = T_ba diag(beta_a e^{g_a - g_aC}) K_a (N x DK).  Per chunk-head, fp32:
+// C2' = T_ba diag(beta_a e^{g_a - g_aC}) K_a (N x DK).  Per second half and head,
+// fp32: C2' (16 x DK), then C1 V_a as one 16 x 64 block per 64-column value slice;
+// rows N..15 zero.
 constexpr int PAIR_MAXN = 16;
-constexpr int PAIR_C1 = 0, PAIR_C2 = PAIR_MAXN * PAIR_MAXN, PAIR_STRIDE = PAIR_C2 + PAIR_MAXN * 128;
+constexpr size_t pair_stride(int dv) { return (size_t)PAIR_MAXN * (DK + dv); }
+
+struct PairParams {
+    int B, T, H, dv, NC, N;
+    const void *k, *v;          // bf16 [B, T, H, DK], [B, T, H, dv]
+    const float *alpha, *beta;  // [B, T, H] (nullptr: 1)
+    float *pair_ws;
+};
+
+constexpr int PAIR_THREADS = 128;
+
+// One CTA per (second half, head, batch): the band corner of a 128-token chunk.  The
+// entries of the masked series within the band equal those of the exact inverse
+// (A is strictly lower triangular, so A^n vanishes more than n - 1 below the
+// diagonal), and an entry (r, c) depends only on the tokens between c and r: T_ba
+// is the exact inverse of the 2N-token window around the halves' boundary, read
+// in the band.  Window row w < N is the first half's row 64 - N + w, row N + i
+// the second half's row i.  Small and latency-bound: many CTAs per SM, the band N
+// a template argument so that every loop has its exact trip count.
+template <int N>
+__global__ void __launch_bounds__(PAIR_THREADS)
+pair_corner_kernel(const PairParams p) {
+    constexpr int NW = 2 * N, NWP = NW > 0 ? NW : 1, NP = N > 0 ? N : 1;
+    __shared__ float kw[NWP][DK + 1];            // window keys, fp32
+    __shared__ float aw[NWP][NWP + 1];           // A of the window (band)
+    __shared__ float gw[NWP], bw[NWP], ew[NP];
+    __shared__ float cw[NP][NP];                 // C1 = T_ba diag(beta_a)
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n = 2 * blockIdx.x + 1, h = blockIdx.y, b = blockIdx.z;
+    const int t0 = n * C - N;                    // window start token
+    const int rs = p.H * DK;
+    const uint16_t *kg = reinterpret_cast<const uint16_t *>(p.k) + (((size_t)b * p.T + t0) * p.H + h) * DK;
+    const uint16_t *vg = reinterpret_cast<const uint16_t *>(p.v) + (((size_t)b * p.T + t0) * p.H + h) * p.dv;
+    float *dst = p.pair_ws + (((size_t)b * p.H + h) * p.NC + n) * pair_stride(p.dv);
+
+    // every global load of the window first, so that their latencies overlap:
+    // keys as 16-byte pieces (16 per row), the first value column of this thread,
+    // the gates (warp 0)
+    constexpr int KQ = (NW * 16 + PAIR_THREADS - 1) / PAIR_THREADS;
+    uint4 kr[KQ > 0 ? KQ : 1];
+#pragma unroll
+    for (int q = 0; q < KQ; ++q) {
+        const int x = tid + PAIR_THREADS * q, w = x >> 4;
+        kr[q] = make_uint4(0u, 0u, 0u, 0u);
+        if (w < NW && t0 + w < p.T) kr[q] = *reinterpret_cast<const uint4 *>(kg + (size_t)w * rs + 8 * (x & 15));
+    }
+    float vj[NP];
+#pragma unroll
+    for (int j = 0; j < N; ++j)
+        vj[j] = tid < p.dv ? __uint_as_float((uint32_t)vg[(size_t)j * p.H * p.dv + tid] << 16) : 0.f;
+    float la = 0.f, be = 0.f;
+    if (warp == 0 && lane < NW && t0 + lane < p.T) {
+        const size_t ti = ((size_t)b * p.T + t0 + lane) * p.H + h;
+        la = p.alpha ? logf(p.alpha[ti]) : 0.f;
+        be = p.beta ? p.beta[ti] : 1.f;
+    }
+#pragma unroll
+    for (int q = 0; q < KQ; ++q) {
+        const int x = tid + PAIR_THREADS * q, w = x >> 4;
+        if (w < NW) {
+            float *d = &kw[w][8 * (x & 15)];
+            const uint32_t u[4] = {kr[q].x, kr[q].y, kr[q].z, kr[q].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                d[2 * e] = __uint_as_float(u[e] << 16);
+                d[2 * e + 1] = __uint_as_float(u[e] & 0xffff0000u);
+            }
+        }
+    }
+    if (warp == 0) {
+        // cumulative log decay over the window (only differences are used)
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, la, o);
+            if (lane >= o) la += y;
+        }
+        if (lane < NW) { gw[lane] = la; bw[lane] = be; }
+    }
+    __syncthreads();
+    // A_ij = -beta_i e^{g_i - g_j} k_i.k_j for 0 < i - j <= N: four lanes per entry,
+    // 32 channels each (rotated by 8 per lane so that the four do not share banks)
+    constexpr int TOTAL = NW * NW * 4;
+    for (int q0 = warp * 32; q0 < TOTAL; q0 += PAIR_THREADS) {
+        const int q = q0 + lane, e = q >> 2, part = q & 3;
+        const int i = e / NWP, j = e - i * NWP;
+        const bool need = q < TOTAL && j < i && i - j <= N;
+        float d = 0.f;
+        if (need) {
+#pragma unroll 8
+            for (int cc = 0; cc < 32; ++cc) {
+                const int c = 32 * part + ((cc + 8 * part) & 31);
+                d += kw[i][c] * kw[j][c];
+            }
+        }
+        d += __shfl_xor_sync(0xffffffffu, d, 1);
+        d += __shfl_xor_sync(0xffffffffu, d, 2);
+        if (need && part == 0) aw[i][j] = -bw[i] * expf(gw[i] - gw[j]) * d;
+    }
+    __syncthreads();
+    if (tid < N) {
+        // column j = tid of the window's inverse by forward substitution, rows j..N+j
+        // (every A entry it reads lies in the band); C1 = T_ba diag(beta_a) in the
+        // band (i <= j), zero below it
+        const int j = tid;
+        float t[NWP];
+#pragma unroll
+        for (int k = 0; k < NW; ++k) {
+            float acc = (k == j) ? 1.f : 0.f;
+            if (k > j && k <= N + j) {
+#pragma unroll
+                for (int m = 0; m < k; ++m)
+                    if (m >= j) acc += aw[k][m] * t[m];
+            }
+            t[k] = acc;
+        }
+#pragma unroll
+        for (int i = 0; i < N; ++i) cw[i][j] = i <= j ? t[N + i] * bw[j] : 0.f;
+        ew[j] = expf(gw[j] - gw[N - 1]);
+    }
+    __syncthreads();
+    {
+        // C2'[i][c] = sum_j C1[i][j] e^{g_j - g_{N-1}} k_j[c], column c = tid; rows >= N zero
+        const int c = tid;
+        float kc[NP];
+#pragma unroll
+        for (int j = 0; j < N; ++j) kc[j] = ew[j] * kw[j][c];
+#pragma unroll 4
+        for (int i = 0; i < PAIR_MAXN; ++i) {
+            float acc = 0.f;
+            if (i < N) {
+#pragma unroll
+                for (int j = 0; j < N; ++j) acc += cw[i < N ? i : 0][j] * kc[j];
+            }
+            dst[i * DK + c] = acc;
+        }
+    }
+    // C1 V_a, column c of the value rows t0 .. t0 + N - 1, one 16 x 64 block per
+    // 64-column value slice
+    for (int c = tid; c < p.dv; c += PAIR_THREADS) {
+        if (c != tid) {
+#pragma unroll
+            for (int j = 0; j < N; ++j) vj[j] = __uint_as_float((uint32_t)vg[(size_t)j * p.H * p.dv + c] << 16);
+        }
+        float *dc = dst + PAIR_MAXN * DK + (c >> 6) * (PAIR_MAXN * 64) + (c & 63);
+#pragma unroll 4
+        for (int i = 0; i < PAIR_MAXN; ++i) {
+            float acc = 0.f;
+            if (i < N) {
+#pragma unroll
+                for (int j = 0; j < N; ++j) acc += cw[i < N ? i : 0][j] * vj[j];
+            }
+            dc[i * 64] = acc;
+        }
+    }
+}
 
 // One CTA per (chunk, head, batch).  [Q ; K] K^T in one MMA: TMEM lanes 0..63
 // hold Q K^T (-> P), lanes 64..127 hold K K^T (-> L -> T).
@@ -435,99 +589,6 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
         }
     }
-    if (p.pair_ws && (n & 1)) block_sync();
-    if (p.pair_ws && (n & 1) && *abort_flag == 0) {
-        // Second half of a 128-token chunk: the corner of the 128-token chunk's masked
-        // series from the 2N-token window around the halves' boundary (window rows
-        // w < N: a's rows 64 - N + w; w >= N: b's rows w - N), then C1 and C2'.
-        // The tile region is free by now (the series' MMAs and the stores are done).
-        const int N = p.N, NW = 2 * N;
-        float *kw = Lb;                          // NW x 129
-        float *aw = Lb + 32 * 129;               // NW x 33: A of the window, then T
-        float *tw = aw + 32 * 33;                // NW x 33
-        float *gw = tw + 32 * 33;                // NW: cumulative log decay over the window
-        float *bw = gw + 32;                     // NW: beta
-        float *ew = bw + 32;                     // N: e^{g_j - g_{N-1}}, decay to the first half's end
-        float *cw = ew + 32;                     // N x N: C1
-        for (int x = tid; x < NW * 128; x += K1_THREADS) {
-            const int w = x >> 7, c = x & 127, t = t0 - N + w;
-            float kv = 0.f;
-            if (t < p.T) {
-                const uint16_t u = reinterpret_cast<const uint16_t *>(p.k)[(((size_t)b * p.T + t) * p.H + h) * 128 + c];
-                kv = __uint_as_float((uint32_t)u << 16);
-            }
-            kw[w * 129 + c] = kv;
-        }
-        if (warp == 0) {
-            // window gates: log alpha (0 past the end) scanned over the window, beta (0 past the end)
-            float la = 0.f, be = 0.f;
-            if (lane < NW) {
-                const int t = t0 - N + lane;
-                if (t < p.T) {
-                    const size_t ti = ((size_t)b * p.T + t) * p.H + h;
-                    la = p.alpha ? logf(p.alpha[ti]) : 0.f;
-                    be = p.beta ? p.beta[ti] : 1.f;
-                }
-            }
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, la, o);
-                if (lane >= o) la += y;
-            }
-            if (lane < NW) { gw[lane] = la; bw[lane] = be; }
-        }
-        block_sync();
-        // A_ij = -beta_i exp(g_i - g_j) k_i.k_j (i > j) over the window; T = M (.) (I + A T), N steps
-        for (int x = tid; x < NW * NW; x += K1_THREADS) {
-            const int i = x / NW, j = x % NW;
-            float a = 0.f;
-            if (j < i) {
-                float d = 0.f;
-                for (int c = 0; c < 128; ++c) d += kw[i * 129 + c] * kw[j * 129 + c];
-                a = -bw[i] * expf(gw[i] - gw[j]) * d;
-            }
-            aw[i * 33 + j] = a;
-            tw[i * 33 + j] = (i == j) ? 1.f : 0.f;
-        }
-        block_sync();
-        for (int step = 0; step < N; ++step) {
-            float val[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int x = tid + K1_THREADS * q, i = x / NW, j = x % NW;
-                val[q] = 0.f;
-                if (x < NW * NW && i - j >= 0 && i - j <= N) {
-                    float sacc = (i == j) ? 1.f : 0.f;
-                    for (int kk = j; kk < i; ++kk) sacc += aw[i * 33 + kk] * tw[kk * 33 + j];
-                    val[q] = sacc;
-                }
-            }
-            block_sync();
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int x = tid + K1_THREADS * q;
-                if (x < NW * NW) tw[(x / NW) * 33 + x % NW] = val[q];
-            }
-            block_sync();
-        }
-        // C1[i][j] = T[N + i][j] beta_j;  C2'[i][c] = sum_j C1[i][j] e^{g_j - g_{N-1}} k_j[c]
-        float *dst = p.pair_ws + (((size_t)b * p.H + h) * p.NC + n) * PAIR_STRIDE;
-        if (tid < N) ew[tid] = expf(gw[tid] - gw[N - 1]);
-        for (int x = tid; x < PAIR_MAXN * PAIR_MAXN; x += K1_THREADS) {
-            const int i = x / PAIR_MAXN, j = x % PAIR_MAXN;
-            const float c1 = (i < N && j < N) ? tw[(N + i) * 33 + j] * bw[j] : 0.f;
-            cw[x] = c1;
-            dst[PAIR_C1 + x] = c1;
-        }
-        block_sync();
-        for (int x = tid; x < PAIR_MAXN * 128; x += K1_THREADS) {
-            const int i = x >> 7, c = x & 127;
-            float acc = 0.f;
-            if (i < N)
-                for (int j = 0; j < N; ++j) acc += cw[i * PAIR_MAXN + j] * ew[j] * kw[j * 129 + c];
-            dst[PAIR_C2 + x] = acc;
-        }
-    }
     tc_fence_before();
     block_sync();
     if (warp == 0) {
@@ -567,8 +628,8 @@ template <bool PAIR> struct K2Layout {
     static constexpr uint32_t HS = EARLY + EARLY_TX;            // h fp16, 128 rows
     static constexpr uint32_t HH = HS + 16384;                  // PAIR: e^{g_C} h of a first half, fp16
     static constexpr uint32_t DS = HH + (PAIR ? 16384 : 0);     // Delta fp16 x 2
-    static constexpr uint32_t CORNER = DS + 2 * 8192;           // PAIR: C1 V_a, 16 x 64 fp32
-    static constexpr uint32_t C2S = CORNER + (PAIR ? 4096 : 0); // PAIR: C2', 16 x 128 fp32
+    static constexpr uint32_t CORNER = DS + 2 * 8192;           // PAIR: C1 V_a, 16 x 64 fp32, x 2
+    static constexpr uint32_t C2S = CORNER + (PAIR ? 8192 : 0); // PAIR: C2', 16 x 128 fp32
     static constexpr uint32_t PAR = C2S + (PAIR ? 8192 : 0);
     static constexpr uint32_t BAR = PAR + 3 * PAR_BYTES;        // gate ring of 3
     static constexpr uint32_t MISC = BAR + N_BARS * 8;          // tmem slot, abort flag, group slots
@@ -581,8 +642,6 @@ static_assert((MSTG & 1023) == 0, "swizzled tiles on 1024-byte boundaries");
 static_assert(K1_SMEM * K1_BLOCKS_PER_SM <= 233472, "key-side blocks per SM");
 static_assert(K1_SMEM_RES <= 232448, "residual-correction key-side block fits one SM");
 static_assert(K1_OFF_YB + 8192 <= K1_OFF_TB, "L and the inverse scratch fit in the tile region");
-static_assert((32 * 129 + 2 * 32 * 33 + 3 * 32 + PAIR_MAXN * PAIR_MAXN) * 4 <= K1_OFF_TB,
-              "the boundary window of a 128-token chunk fits in the tile region");
 static_assert(K1_OFF_LB + K1_MAT <= K1_OFF_B2 && K1_OFF_B2 + 4096 <= K1_OFF_A1 && K1_OFF_A1 + 4096 <= K1_OFF_TB &&
               K1_OFF_A1 + 16384 <= K1_OFF_TB + K1_MAT && (K1_OFF_B2 & 1023) == 0 && (K1_OFF_A1 & 1023) == 0 &&
               K1_OFF_A2 + 16384 + 1024 <= K1_SMEM,
@@ -596,9 +655,7 @@ constexpr uint32_t TM_COLS = 512;
 struct K2Params {
     int B, T, H, dv, NC;
     const float *alpha, *beta, *S0;
-    const void *v;          // bf16 [B, T, H, dv] (PAIR: the first half's last N rows)
-    const float *pair_ws;   // PAIR: C1 and C2' of every second half
-    int N;                  // PAIR: band of the masked series
+    const float *pair_ws;   // PAIR: C2' and C1 V_a of every second half
     void *o;
     float *S_T;
     int o_bf16;
@@ -715,11 +772,21 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 // early slot: free once the U and W MMAs of chunk m - 1 are complete
                 if (m >= 1 && !mbar_wait(&bars[B_EEMPTY], (m - 1) & 1, abort_flag, E_EMPTY, lim)) break;
                 uint64_t *eb = &bars[B_EFULL];
-                mbar_arrive_expect_tx(eb, EARLY_TX);
+                const bool second = PAIR && (m & 1);
+                mbar_arrive_expect_tx(eb, EARLY_TX + (second ? 8192u + 4096u : 0u));
                 uint8_t *es = sm + OFF_EARLY;
                 tma_load_4d(es + ES_V, &tm_v, eb, v0, h, t0, b);
                 tma_load_4d(es + ES_TB, &tm_t, eb, 0, 0, wrow, 0);
                 tma_load_4d(es + ES_TBG, &tm_t, eb, 0, 0, wrow + 64, 0);
+                if (second) {
+                    // second half of a 128-token chunk: C2' for the key side and this
+                    // slice's C1 V_a for the chain (two buffers: the chain may still be
+                    // reading the previous pair's while this one lands)
+                    const float *src = p.pair_ws + (((size_t)b * H + h) * NC + m) * pair_stride(dv);
+                    bulk_load_g2s(sm + L::C2S, src, 8192u, eb);
+                    bulk_load_g2s(sm + L::CORNER + ((m >> 1) & 1) * 4096u, src + PAIR_MAXN * DK + slice * (PAIR_MAXN * 64),
+                                  4096u, eb);
+                }
                 issued_early = m + 1;
             }
             // no copy may still be in flight when the block exits: the last load of
@@ -791,15 +858,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             }
             if (!sync_ok(1, KS_THREADS, leader, kcnt)) break;
             if (!lwarp) mbar_try_wait(&bars[B_FULL + ms], (m / NSTAGE) & 1);
-            // second half of a 128-token chunk: C2' (16 x 128) -> shared memory; the
-            // loads are in flight while the operands below are converted
-            float4 c2a = make_float4(0.f, 0.f, 0.f, 0.f), c2b = c2a;
-            if (PAIR && (m & 1)) {
-                const float4 *src = reinterpret_cast<const float4 *>(
-                    p.pair_ws + (((size_t)b * H + h) * NC + m) * PAIR_STRIDE + PAIR_C2);
-                c2a = src[kt];
-                c2b = src[kt + 256];
-            }
             // in-place fp16 operands: Q -> e^{g_r} Q, K -> K in the main stage, then
             // V in the early slot once it has landed.  Every load of a pass is
             // issued before the first store, so they overlap instead of waiting on
@@ -846,11 +904,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     sc[it] = 1.f;
                 }
                 convert(addr, sc, 2);
-            }
-            if (PAIR && (m & 1)) {
-                float4 *dst = reinterpret_cast<float4 *>(sm + L::C2S);
-                dst[kt] = c2a;
-                dst[kt + 256] = c2b;
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -1083,25 +1136,6 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             }
             __syncwarp();
             if (!rowpart) {
-                if (PAIR && !(n & 1) && n + 1 < NC) {
-                    // first half of a 128-token chunk: the corner's value part of the
-                    // second half, C1 V_a (V_a: this chunk's last N rows), column ct
-                    const float *c1 = p.pair_ws + (bh * NC + n + 1) * PAIR_STRIDE + PAIR_C1;
-                    const uint16_t *vp = reinterpret_cast<const uint16_t *>(p.v) +
-                                         (((size_t)b * T + (n * C + C - p.N)) * H + h) * dv + v0 + ct;
-                    float vv[PAIR_MAXN];
-#pragma unroll
-                    for (int j = 0; j < PAIR_MAXN; ++j)
-                        vv[j] = j < p.N ? __uint_as_float((uint32_t)vp[(size_t)j * H * dv] << 16) : 0.f;
-                    float *cr = reinterpret_cast<float *>(sm + L::CORNER);
-#pragma unroll 4
-                    for (int i = 0; i < PAIR_MAXN; ++i) {
-                        float acc = 0.f;
-#pragma unroll
-                        for (int j = 0; j < PAIR_MAXN; ++j) acc += c1[i * PAIR_MAXN + j] * vv[j];
-                        cr[i * 64 + ct] = acc;
-                    }
-                }
                 // sub-partitions 2, 3: output rows of the previous chunk, off the chain
                 if (n > 0) out_rows(n - 1);
                 continue;
@@ -1118,7 +1152,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 for (int j = 0; j < 64; ++j) x[j] += u[j];
                 if (PAIR && s && r < PAIR_MAXN) {
                     // second half: + C1 V_a, the corner's value part
-                    const float *cr = reinterpret_cast<const float *>(sm + L::CORNER) + r * 64;
+                    const float *cr = reinterpret_cast<const float *>(sm + L::CORNER + ((n >> 1) & 1) * 4096u) + r * 64;
 #pragma unroll
                     for (int j = 0; j < 64; ++j) x[j] += cr[j];
                 }
@@ -1239,7 +1273,7 @@ int tc_default_slices(const FwdParams &p) { return p.dv / DVS; }
 
 size_t tc_workspace_bytes(const FwdParams &p) {
     const size_t nc = (size_t)(p.T + C - 1) / C;
-    const size_t per = WS_CHUNK_BYTES + (p.C == 2 * C ? (size_t)PAIR_STRIDE * 4 : 0);
+    const size_t per = WS_CHUNK_BYTES + (p.C == 2 * C ? pair_stride(p.dv) * 4 : 0);
     return (size_t)p.B * p.H * nc * per;
 }
 
@@ -1255,7 +1289,8 @@ cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, 
     // The attribute belongs to the current device: set it on every launch (cheap)
     // rather than behind a process-wide flag that a second device would not share.
     // A 128-token chunk of the masked series runs as two 64-token halves ("pair"):
-    // the second halves' band corners go to the workspace after the T matrices.
+    // the second halves' band corners (a third kernel) go to the workspace after the
+    // T matrices.
     const bool pair = p.C == 2 * C;
     float *pair_ws = pair ? reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) +
                                                       (size_t)p.B * p.H * NC * WS_CHUNK_BYTES)
@@ -1270,11 +1305,27 @@ cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, 
                                         (int)K2Layout<false>::SMEM);
         if (e != cudaSuccess) return e;
     }
+    if (pair && NC / 2 > 0) {
+        PairParams pp;
+        pp.B = p.B; pp.T = p.T; pp.H = p.H; pp.dv = p.dv; pp.NC = NC; pp.N = p.N;
+        pp.k = p.k; pp.v = p.v; pp.alpha = p.alpha; pp.beta = p.beta; pp.pair_ws = pair_ws;
+        const dim3 grid(NC / 2, p.H, p.B);
+        switch (p.N) {
+#define GDN_PAIR_CASE(n) \
+    case n: pair_corner_kernel<n><<<grid, PAIR_THREADS, 0, stream>>>(pp); break;
+            GDN_PAIR_CASE(0) GDN_PAIR_CASE(1) GDN_PAIR_CASE(2) GDN_PAIR_CASE(3) GDN_PAIR_CASE(4)
+            GDN_PAIR_CASE(5) GDN_PAIR_CASE(6) GDN_PAIR_CASE(7) GDN_PAIR_CASE(8) GDN_PAIR_CASE(9)
+            GDN_PAIR_CASE(10) GDN_PAIR_CASE(11) GDN_PAIR_CASE(12) GDN_PAIR_CASE(13) GDN_PAIR_CASE(14)
+            GDN_PAIR_CASE(15)
+#undef GDN_PAIR_CASE
+            default: *why = "(band N > 15 with chunk 128)"; return cudaErrorInvalidValue;
+        }
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
     K1Params k1;
     k1.B = p.B; k1.T = p.T; k1.H = p.H; k1.NC = NC;
     k1.alpha = p.alpha; k1.beta = p.beta;
-    k1.k = p.k;
-    k1.pair_ws = pair_ws;
     k1.ws = reinterpret_cast<uint8_t *>(workspace);
     k1.neumann = p.mode == GDN_INV_NEUMANN ? 1 : (p.mode == GDN_INV_NEUMANN_RESIDUAL ? 2 : 0);
     k1.N = p.N; k1.S = p.S;
@@ -1284,7 +1335,7 @@ cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, 
     K2Params k2;
     k2.B = p.B; k2.T = p.T; k2.H = p.H; k2.dv = p.dv; k2.NC = NC;
     k2.alpha = p.alpha; k2.beta = p.beta; k2.S0 = p.S0; k2.o = p.o; k2.S_T = p.S_T;
-    k2.v = p.v; k2.pair_ws = pair_ws; k2.N = p.N;
+    k2.pair_ws = pair_ws;
     k2.o_bf16 = p.o_bf16;
     if (pair)
         chain_kernel<true><<<dim3(p.slices, p.H, p.B), K2_THREADS, K2Layout<true>::SMEM, stream>>>(mq, mk, mv, mt,

@@ -281,9 +281,10 @@ def test_workspace_sizes_per_kernel():
     per128 = 2 * 128 * 128 + 3 * 128 * dk + dk
     assert gdn.workspace_bytes(c128) == B * H * 1 * per128 * 4
     # chunk 128 on the split kernels: per 64-token half the 24 KiB of T matrices and
-    # the band corner (C1: 16 x 16, C2': 16 x dk, fp32)
+    # the band corner's two parts (C2': 16 x dk, C1 V_a: 16 x dv, fp32)
+    dv = 128
     assert gdn.workspace_bytes(_args(kernel=4, chunk=128, mode=1, neumann_N=3)) == \
-        chunks * (24576 + (16 * 16 + 16 * dk) * 4)
+        chunks * (24576 + 16 * (dk + dv) * 4)
 
 
 def test_simt_call_without_workspace_rejected_on_host():
