@@ -410,9 +410,15 @@ def forward_line(args, rank, world, local_rank, name, over, timed_steps):
     # when there is a second half); SIMT path: prep + chain, plus the two scan kernels
     # of the preconditioner's running average
     pair = kernel_id == 4 and w.chunk == 128 and w.T > 64
+    # the two-gate rule on the split path: the SIMT prep writes fp16 rows, the
+    # tensor-core chain reads them (no key-side kernel)
+    gen = kernel_id == 4 and general
     if pair:
         kernel_name = "pair_corner_kernel+" + kernel_name
-    launches_per_call = {4: 3 if pair else 2, 1: 4 if (w.precond and general) else 2}.get(kernel_id, 1)
+    if gen:
+        kernel_name = "simt_prep_kernel+chain_kernel"
+    scans = 2 if (w.precond and general) else 0    # the preconditioner's running-average kernels
+    launches_per_call = {4: 3 if pair else 2 + scans, 1: 2 + scans}.get(kernel_id, 1)
     sh = stream.cuda_stream
 
     def step():
@@ -492,7 +498,8 @@ def forward_line(args, rank, world, local_rank, name, over, timed_steps):
     bytes_launch = algorithmic_bytes(w, o_bytes=4 if f32 else 2)
     achieved = bytes_launch / (ms_step / 1e3) / 1e9
     flops = algorithmic_flops(w)
-    traffic = profile_traffic(f"{kernel_name}@{name}", KERNEL_SOURCES.get(kernel_id, ()), units=w.B)
+    sources = SPLIT_SOURCES + SIMT_SOURCES if gen else KERNEL_SOURCES.get(kernel_id, ())
+    traffic = profile_traffic(f"{kernel_name}@{name}", sources, units=w.B)
     roof = dict(bound="hbm", achieved=achieved, peak=pk["hbm_gbs"], unit="GB/s",
                 frac=achieved / pk["hbm_gbs"], traffic=traffic,
                 peak_source=pk["source"] + " (burst copy bandwidth)",
@@ -501,9 +508,10 @@ def forward_line(args, rank, world, local_rank, name, over, timed_steps):
                 tensor_frac_of_bf16_peak=flops / (ms_step / 1e3) / 1e12 / pk["bf16_tflops"],
                 roofline_ms=max(bytes_launch / (pk["hbm_gbs"] * 1e9),
                                 flops / (pk["bf16_tflops"] * 1e12)) * 1e3)
-    if kernel_id == 1:
+    if kernel_id == 1 or gen:
         # the SIMT path computes in fp32 on the CUDA cores: its bound is the fp32
-        # arithmetic of the chunk algebra, not HBM (the HBM figures stay alongside)
+        # arithmetic of the chunk algebra, not HBM (the HBM figures stay alongside);
+        # so does the two-gate rule's prep, the larger part of its split path
         alu_peak = fp32_alu_peak_tflops(1965.0)
         ach = flops / (ms_step / 1e3) / 1e12
         roof = dict(bound="alu", achieved=ach, peak=alu_peak, unit="TFLOP/s", frac=ach / alu_peak,
@@ -564,6 +572,8 @@ def forward_line(args, rank, world, local_rank, name, over, timed_steps):
                     warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True,
                     scaling="weak", vs_baseline=None, dtype="f32" if f32 else "bf16",
                     compute=("fp32 CUDA cores" if kernel_id == 1 else
+                             "fp32 CUDA-core prep; fp16 tensor-core chain operands, fp32 accumulate and state"
+                             if gen else
                              "bf16 q/k/v in HBM; fp16 tensor-core operands, fp32 accumulate and state"),
                     data="synthetic (seeded; Gated DeltaNet layer shapes)",
                     parity=("o and S_T meet max|err| <= 2e-2 * rms(oracle) with an fp32 o (the parity tests); "

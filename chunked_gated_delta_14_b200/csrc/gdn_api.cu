@@ -335,9 +335,9 @@ gdn_status gdn_chunk_fwd_static_scratch(const gdn_fwd_args *args, void *stream) 
     const size_t need = gdn::tc_workspace_bytes(p);
     if (need > (size_t)GDN_STATIC_SCRATCH_BYTES)
         return fail(GDN_ERR_INVALID_ARG,
-                    "needs %zu bytes of scratch (24 KiB per chunk-head, B*H*ceil(T/64) = %zu); "
+                    "needs %zu bytes of scratch (gdn_workspace_bytes of the split tensor-core kernels); "
                     "the fixed array holds %llu bytes",
-                    need, need / 24576, (unsigned long long)GDN_STATIC_SCRATCH_BYTES);
+                    need, (unsigned long long)GDN_STATIC_SCRATCH_BYTES);
     constexpr int kMaxDevices = 64;
     static void *dev_ptr[kMaxDevices] = {};
     static std::mutex mu;

@@ -29,7 +29,6 @@ struct FwdParams {
     int mode, N;
     int S;              // residual-correction terms (GDN_INV_NEUMANN_RESIDUAL)
     int general;        // two-gate rule (per-channel decay / gates / preconditioner)
-    int pair;           // tensor-core path: a 128-token chunk of the masked series run as two 64-token halves
 };
 
 // SIMT fp32 chunk kernel: shared-memory bytes for p, or 0 if p does not fit.
@@ -43,6 +42,27 @@ size_t simt_smem_bytes(const FwdParams &p);
 // (fp32), plus the preconditioner's running average at chunk starts.
 size_t simt_workspace_bytes(const FwdParams &p);
 cudaError_t launch_simt(const FwdParams &p, void *workspace, cudaStream_t stream);
+
+// The two-gate rule on the tensor-core chain: the SIMT prep kernel's matrices as
+// fp16 rows of 64 (128 B) per chunk-head, ready for the chain kernel's TMA loads.
+// TB, P and U = w (.) v go as hi/lo fp16 pairs (x = hi + lo to about 2^-22): with
+// the preconditioned write keys the first tokens' outputs are hundreds of times
+// the sequence's RMS, and one fp16 rounding of those operands would leave the
+// accuracy bar there.  E, Q', K'' are 64-column blocks (channels 0..63, 64..127),
+// U one block per 64 value columns, d (the state's decay) fp32.  Chunk 64, d_k 128.
+struct GenRows {
+    int tb, tbl, pp, ppl, e, q, k, u, ul, d, rows;
+};
+__host__ __device__ inline GenRows gen_rows(int dv) {
+    GenRows g;
+    g.tb = 0; g.tbl = 64; g.pp = 128; g.ppl = 192; g.e = 256; g.q = 384; g.k = 512; g.u = 640;
+    g.ul = 640 + dv; g.d = 640 + 2 * dv; g.rows = g.d + 4;
+    return g;
+}
+// Workspace of that prep (rows for every chunk-head, then the preconditioner's
+// running averages) and its launch: the running-average kernels and the prep.
+size_t gen_prep_workspace_bytes(const FwdParams &p);
+cudaError_t launch_gen_prep(const FwdParams &p, void *workspace, cudaStream_t stream);
 
 // Tensor-core kernel (tcgen05 / TMEM / TMA).
 bool tc_supports(const FwdParams &p, const char **why);

@@ -42,6 +42,7 @@
 // Decay ratios are always exp(later - earlier) <= 1.
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "gdn_internal.cuh"
 
@@ -198,9 +199,12 @@ __global__ void rho_combine_kernel(const FwdParams p, const float *sums, const f
 }
 
 // One block per (chunk, head, batch): the state-independent matrices of one chunk.
-template <typename KS, bool GENERAL>
+// TCOUT (two-gate rule, chunk 64, d_k 128): written as fp16 rows for the
+// tensor-core chain (gen_rows), together with U = w (.) v, instead of fp32.
+// rho0: the preconditioner's running average at every chunk start.
+template <typename KS, bool GENERAL, bool TCOUT = false>
 __global__ void __launch_bounds__(kThreads)
-simt_prep_kernel(const FwdParams p, float *ws) {
+simt_prep_kernel(const FwdParams p, float *ws, const float *rho0) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int C = p.C, dk = p.dk, H = p.H, T = p.T;
@@ -226,6 +230,8 @@ simt_prep_kernel(const FwdParams p, float *ws) {
     const size_t bh = (size_t)b * H + h;
     const SimtWs W = simt_ws(C, dk);
     float *out = ws + (bh * NC + n) * W.stride;
+    const GenRows GR = gen_rows(p.dv);
+    __half *ob = reinterpret_cast<__half *>(ws) + (bh * NC + n) * (size_t)GR.rows * 64;   // TCOUT rows
 
     // ---------------------------------------------------------- load
     for (int idx = tid; idx < C * dk; idx += kThreads) {
@@ -256,7 +262,6 @@ simt_prep_kernel(const FwdParams p, float *ws) {
         // into [1/x, x] on a log scale; applied to the write key (forms 2, 3
         // read the state with the raw key) or to the query
         const float lnx = p.precond == 3 ? logf(p.precond_x) : 1.f;
-        const float *rho0 = ws + (size_t)p.B * H * NC * W.stride;
         for (int c = tid; c < dk; c += kThreads) {
             float rh = p.precond ? rho0[(bh * NC + n) * dk + c] : 0.f, G = 0.f;
             for (int r = 0; r < C; ++r) {
@@ -378,8 +383,16 @@ simt_prep_kernel(const FwdParams p, float *ws) {
     __syncthreads();
     // ------------------------------------------------ the chunk's matrices
     // TB = T diag(beta) (scalar rule; the two-gate rule has no beta)
-    for (int idx = tid; idx < C * C; idx += kThreads)
-        out[W.tb + idx] = GENERAL ? tp[idx] : tp[idx] * bet[idx % C];
+    for (int idx = tid; idx < C * C; idx += kThreads) {
+        const float tb = GENERAL ? tp[idx] : tp[idx] * bet[idx % C];
+        if (TCOUT) {
+            const __half hi = __float2half_rn(tb);
+            ob[(size_t)GR.tb * 64 + idx] = hi;
+            ob[(size_t)GR.tbl * 64 + idx] = __float2half_rn(tb - __half2float(hi));
+        } else {
+            out[W.tb + idx] = tb;
+        }
+    }
     // P: decayed causal scores, 4 x 4 register tiles
     for (int t = tid; t < (C / 4) * (C / 4); t += kThreads) {
         const int r0 = 4 * (t / (C / 4)), i0 = 4 * (t % (C / 4));
@@ -422,13 +435,26 @@ simt_prep_kernel(const FwdParams p, float *ws) {
                 const int r = r0 + a, i = i0 + e;
                 float val = 0.f;
                 if (i <= r) val = GENERAL ? acc[a][e] : expf(g[r] - g[i]) * acc[a][e];
-                out[W.pp + r * C + i] = val;
+                if (TCOUT) {
+                    const __half hi = __float2half_rn(val);
+                    ob[(size_t)(GR.pp + r) * 64 + i] = hi;
+                    ob[(size_t)(GR.ppl + r) * 64 + i] = __float2half_rn(val - __half2float(hi));
+                } else {
+                    out[W.pp + r * C + i] = val;
+                }
             }
     }
     // E (the state read), Q' (the output read), K'' (the state write)
     for (int idx = tid; idx < C * dk; idx += kThreads) {
         const int r = idx / dk, c = idx % dk, si = r * ks + c;
-        if (GENERAL) {
+        if (TCOUT) {
+            // 64-column blocks: channel c of row r at row (block base + 64 (c / 64) + r)
+            const float Gl = gx[(C - 1) * ks + c];
+            const size_t o = (size_t)(64 * (c >> 6) + r) * 64 + (c & 63);
+            ob[(size_t)GR.e * 64 + o] = __float2half_rn(ex[si] * ((r > 0) ? fast_exp2(gx[si - ks]) : 1.f));
+            ob[(size_t)GR.q * 64 + o] = __float2half_rn(ld_s(qx, si) * fast_exp2(gx[si]));
+            ob[(size_t)GR.k * 64 + o] = __float2half_rn(ld_s(kx, si) * fast_exp2(Gl - gx[si]));
+        } else if (GENERAL) {
             const float Gl = gx[(C - 1) * ks + c];
             out[W.e + idx] = ex[si] * ((r > 0) ? fast_exp2(gx[si - ks]) : 1.f);
             out[W.q + idx] = ld_s(qx, si) * fast_exp2(gx[si]);
@@ -441,8 +467,27 @@ simt_prep_kernel(const FwdParams p, float *ws) {
         }
     }
     // d: the state's decay over the chunk
-    for (int c = tid; c < dk; c += kThreads)
-        out[W.d + c] = GENERAL ? fast_exp2(gx[(C - 1) * ks + c]) : expf(g[C - 1]);
+    for (int c = tid; c < dk; c += kThreads) {
+        const float dc = GENERAL ? fast_exp2(gx[(C - 1) * ks + c]) : expf(g[C - 1]);
+        if (TCOUT) reinterpret_cast<float *>(ob + (size_t)GR.d * 64)[c] = dc;
+        else out[W.d + c] = dc;
+    }
+    if (TCOUT) {
+        // U = w (.) v (hi, lo), one 64-column block per value slice; zero past the end
+        for (int idx = tid; idx < C * p.dv; idx += kThreads) {
+            const int r = idx / p.dv, j = idx % p.dv;
+            float u = 0.f;
+            if (r < Cv) {
+                const size_t gi = (((size_t)b * T + t0 + r) * H + h) * p.dv + j;
+                u = load_in(p.v, gi, p.io_bf16);
+                if (p.write) u *= load_in(p.write, gi, p.io_bf16);
+            }
+            const size_t o = (size_t)(64 * (j >> 6) + r) * 64 + (j & 63);
+            const __half hi = __float2half_rn(u);
+            ob[(size_t)GR.u * 64 + o] = hi;
+            ob[(size_t)GR.ul * 64 + o] = __float2half_rn(u - __half2float(hi));
+        }
+    }
 }
 
 // Copy a rows x cols matrix (cols a multiple of 4, 16-byte aligned) from the
@@ -610,14 +655,14 @@ cudaError_t launch_pair(const FwdParams &p, float *ws, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(chain, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cl.total);
     if (e != cudaSuccess) return e;
+    const size_t chunks = (size_t)p.B * p.H * NC;
+    float *rho0 = ws + chunks * simt_ws(p.C, p.dk).stride;
     if (GENERAL && p.precond) {
-        const size_t chunks = (size_t)p.B * p.H * NC;
-        float *rho0 = ws + chunks * simt_ws(p.C, p.dk).stride;
         float *sums = rho0 + chunks * p.dk, *pows = sums + chunks * p.dk;
         rho_local_kernel<<<dim3(NC, p.H, p.B), 128, 0, stream>>>(p, sums, pows);
         rho_combine_kernel<<<dim3(p.H, p.B), 128, 0, stream>>>(p, sums, pows, rho0);
     }
-    prep<<<dim3(NC, p.H, p.B), kThreads, pl.total, stream>>>(p, ws);
+    prep<<<dim3(NC, p.H, p.B), kThreads, pl.total, stream>>>(p, ws, rho0);
     chain<<<dim3(p.slices, p.H, p.B), kThreads, cl.total, stream>>>(p, ws);
     return cudaGetLastError();
 }
@@ -637,6 +682,33 @@ size_t simt_workspace_bytes(const FwdParams &p) {
     size_t floats = chunks * simt_ws(p.C, p.dk).stride;
     if (p.general && p.precond) floats += 3 * chunks * p.dk;   // start values, chunk sums, decay powers
     return floats * sizeof(float);
+}
+
+size_t gen_prep_workspace_bytes(const FwdParams &p) {
+    const size_t NC = (size_t)(p.T + p.C - 1) / p.C;
+    const size_t chunks = (size_t)p.B * p.H * NC;
+    size_t bytes = chunks * (size_t)gen_rows(p.dv).rows * 128;
+    if (p.precond) bytes += 3 * chunks * p.dk * sizeof(float);
+    return bytes;
+}
+
+cudaError_t launch_gen_prep(const FwdParams &p, void *workspace, cudaStream_t stream) {
+    const int NC = (p.T + p.C - 1) / p.C;
+    const size_t chunks = (size_t)p.B * p.H * NC;
+    float *ws = reinterpret_cast<float *>(workspace);
+    float *rho0 = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(workspace) +
+                                            chunks * (size_t)gen_rows(p.dv).rows * 128);
+    const PrepLayout pl = prep_layout(p.C, p.dk, p.N, p.mode == GDN_INV_NEUMANN, 1, 4);
+    auto prep = simt_prep_kernel<float, true, true>;
+    cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.total);
+    if (e != cudaSuccess) return e;
+    if (p.precond) {
+        float *sums = rho0 + chunks * p.dk, *pows = sums + chunks * p.dk;
+        rho_local_kernel<<<dim3(NC, p.H, p.B), 128, 0, stream>>>(p, sums, pows);
+        rho_combine_kernel<<<dim3(p.H, p.B), 128, 0, stream>>>(p, sums, pows, rho0);
+    }
+    prep<<<dim3(NC, p.H, p.B), kThreads, pl.total, stream>>>(p, ws, rho0);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_simt(const FwdParams &p, void *workspace, cudaStream_t stream) {

@@ -621,20 +621,32 @@ constexpr uint32_t EARLY_TX = 24576;
 constexpr uint32_t PAR_BYTES = (sizeof(tc::ChainParams) + 15) & ~15u;
 enum { B_FULL = 0, B_EMPTY = 3, B_EFULL = 6, B_EEMPTY = 7, B_KSREADY = 8, B_KSFREE = 10, B_UW = 12, B_X = 13,
        B_H = 14, B_O = 15, B_XISS = 17, B_DREADY = 18, N_BARS = 20 };
-// Shared-memory layout of the chain kernel; PAIR: 128-token chunks as two halves.
-template <bool PAIR> struct K2Layout {
-    static constexpr int NSTAGE = PAIR ? 2 : 3;
-    static constexpr uint32_t EARLY = NSTAGE * MSTG;
-    static constexpr uint32_t HS = EARLY + EARLY_TX;            // h fp16, 128 rows
+// Modes of the chain kernel: the gated delta rule at chunk 64, chunk 128 as two
+// halves (the masked series), the two-gate rule (every operand from the prep's
+// fp16 rows: Q', K'' in the Q and K slots, P as hi, lo; early slot TB hi, lo,
+// U hi, lo, E; Delta kept as hi, lo).
+enum { K2_PLAIN = 0, K2_PAIR = 1, K2_GEN = 2 };
+constexpr uint32_t S_PL = S_P + 8192;                  // K2_GEN: P lo after P hi
+constexpr uint32_t ES_VL = 24576, ES_E = 32768;        // K2_GEN: U lo, E (two 64-column blocks)
+constexpr uint32_t GEN_MAIN_TX = 6 * 8192;             // Q', K'' (two blocks each), P hi, lo
+constexpr uint32_t GEN_EARLY_TX = 6 * 8192;            // TB hi, lo, U hi, lo, E
+// Shared-memory layout of the chain kernel.
+template <int MODE> struct K2Layout {
+    static constexpr bool PAIR = MODE == K2_PAIR, GEN = MODE == K2_GEN;
+    static constexpr int NSTAGE = (PAIR || GEN) ? 2 : 3;
+    static constexpr uint32_t STG = GEN ? MSTG + 8192 : MSTG;
+    static constexpr uint32_t EARLY = NSTAGE * STG;
+    static constexpr uint32_t HS = EARLY + (GEN ? GEN_EARLY_TX : EARLY_TX);   // h fp16, 128 rows
     static constexpr uint32_t HH = HS + 16384;                  // PAIR: e^{g_C} h of a first half, fp16
-    static constexpr uint32_t DS = HH + (PAIR ? 16384 : 0);     // Delta fp16 x 2
-    static constexpr uint32_t CORNER = DS + 2 * 8192;           // PAIR: C1 V_a, 16 x 64 fp32, x 2
+    static constexpr uint32_t DS = HH + (PAIR ? 16384 : 0);     // Delta fp16 x 2 (GEN: hi x 2, lo x 2)
+    static constexpr uint32_t CORNER = DS + (GEN ? 4 : 2) * 8192; // PAIR: C1 V_a, 16 x 64 fp32, x 2
     static constexpr uint32_t C2S = CORNER + (PAIR ? 8192 : 0); // PAIR: C2', 16 x 128 fp32
     static constexpr uint32_t PAR = C2S + (PAIR ? 8192 : 0);
     static constexpr uint32_t BAR = PAR + 3 * PAR_BYTES;        // gate ring of 3
     static constexpr uint32_t MISC = BAR + N_BARS * 8;          // tmem slot, abort flag, group slots
     static constexpr uint32_t SMEM = MISC + 32 + 1024;
-    static_assert((EARLY & 1023) == 0 && (HS & 1023) == 0 && (HH & 1023) == 0 && (DS & 1023) == 0,
+    static_assert((STG & 1023) == 0 && (EARLY & 1023) == 0 && (HS & 1023) == 0 && (HH & 1023) == 0 &&
+                      (DS & 1023) == 0,
                   "swizzled tiles on 1024-byte boundaries");
     static_assert(SMEM <= 232448, "shared memory budget of one sm_100 block");
 };
@@ -656,12 +668,14 @@ struct K2Params {
     int B, T, H, dv, NC;
     const float *alpha, *beta, *S0;
     const float *pair_ws;   // PAIR: C2' and C1 V_a of every second half
+    const uint8_t *gen_ws;  // GEN: the prep's rows (gen_rows), ws_rows per chunk-head
+    int ws_rows;            // rows of 128 B per chunk-head in the workspace map
     void *o;
     float *S_T;
     int o_bf16;
 };
 
-template <bool PAIR>
+template <int MODE>
 __global__ void __launch_bounds__(K2_THREADS, 1)
 chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_t,
@@ -675,8 +689,10 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int T = p.T, H = p.H, dv = p.dv, NC = p.NC;
     const int v0 = slice * DVS;
-    using L = K2Layout<PAIR>;
+    using L = K2Layout<MODE>;
+    constexpr bool PAIR = L::PAIR, GEN = L::GEN;
     constexpr int NSTAGE = L::NSTAGE;
+    constexpr uint32_t MSTG = L::STG;   // main stage stride of this mode
     constexpr uint32_t OFF_EARLY = L::EARLY, OFF_HS = L::HS, OFF_DS = L::DS, OFF_PAR = L::PAR, OFF_BAR = L::BAR,
                        OFF_MISC = L::MISC;
 
@@ -754,30 +770,55 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             int issued = 0, issued_early = 0;
             for (int m = 0; m < NC; ++m) {
                 const int ms = m % NSTAGE;
-                const int wrow = (((b * H) + h) * NC + m) * WS_ROWS;
+                const int wrow = (((b * H) + h) * NC + m) * p.ws_rows;
                 const int t0 = m * C;
                 // main stage: free once the chain's MMAs of chunk m - 3 are complete
                 if (m >= NSTAGE &&
                     !mbar_wait(&bars[B_EMPTY + ms], ((m / NSTAGE) - 1) & 1, abort_flag, E_EMPTY, lim))
                     break;
                 uint64_t *fb = &bars[B_FULL + ms];
-                mbar_arrive_expect_tx(fb, MAIN_TX);
                 uint8_t *st = sm + ms * MSTG;
-                tma_load_4d(st + S_Q, &tm_q, fb, 0, h, t0, b);
-                tma_load_4d(st + S_KB + S_Q, &tm_q, fb, 64, h, t0, b);
-                tma_load_4d(st + S_K, &tm_k, fb, 0, h, t0, b);
-                tma_load_4d(st + S_KB + S_K, &tm_k, fb, 64, h, t0, b);
-                tma_load_4d(st + S_P, &tm_t, fb, 0, 0, wrow + 128, 0);
+                if (GEN) {
+                    // the prep's fp16 rows: Q', K'' (two key blocks each), P hi, lo
+                    const GenRows G = gen_rows(dv);
+                    mbar_arrive_expect_tx(fb, GEN_MAIN_TX);
+                    tma_load_4d(st + S_Q, &tm_t, fb, 0, 0, wrow + G.q, 0);
+                    tma_load_4d(st + S_KB + S_Q, &tm_t, fb, 0, 0, wrow + G.q + 64, 0);
+                    tma_load_4d(st + S_K, &tm_t, fb, 0, 0, wrow + G.k, 0);
+                    tma_load_4d(st + S_KB + S_K, &tm_t, fb, 0, 0, wrow + G.k + 64, 0);
+                    tma_load_4d(st + S_P, &tm_t, fb, 0, 0, wrow + G.pp, 0);
+                    tma_load_4d(st + S_PL, &tm_t, fb, 0, 0, wrow + G.ppl, 0);
+                } else {
+                    mbar_arrive_expect_tx(fb, MAIN_TX);
+                    tma_load_4d(st + S_Q, &tm_q, fb, 0, h, t0, b);
+                    tma_load_4d(st + S_KB + S_Q, &tm_q, fb, 64, h, t0, b);
+                    tma_load_4d(st + S_K, &tm_k, fb, 0, h, t0, b);
+                    tma_load_4d(st + S_KB + S_K, &tm_k, fb, 64, h, t0, b);
+                    tma_load_4d(st + S_P, &tm_t, fb, 0, 0, wrow + 128, 0);
+                }
                 issued = m + 1;
                 // early slot: free once the U and W MMAs of chunk m - 1 are complete
                 if (m >= 1 && !mbar_wait(&bars[B_EEMPTY], (m - 1) & 1, abort_flag, E_EMPTY, lim)) break;
                 uint64_t *eb = &bars[B_EFULL];
                 const bool second = PAIR && (m & 1);
-                mbar_arrive_expect_tx(eb, EARLY_TX + (second ? 8192u + 4096u : 0u));
                 uint8_t *es = sm + OFF_EARLY;
-                tma_load_4d(es + ES_V, &tm_v, eb, v0, h, t0, b);
-                tma_load_4d(es + ES_TB, &tm_t, eb, 0, 0, wrow, 0);
-                tma_load_4d(es + ES_TBG, &tm_t, eb, 0, 0, wrow + 64, 0);
+                if (GEN) {
+                    // TB hi, lo, this slice's U = w (.) v hi, lo, and E (read only by the
+                    // U and W products, like the rest of the early slot)
+                    const GenRows G = gen_rows(dv);
+                    mbar_arrive_expect_tx(eb, GEN_EARLY_TX);
+                    tma_load_4d(es + ES_TB, &tm_t, eb, 0, 0, wrow + G.tb, 0);
+                    tma_load_4d(es + ES_TBG, &tm_t, eb, 0, 0, wrow + G.tbl, 0);
+                    tma_load_4d(es + ES_V, &tm_t, eb, 0, 0, wrow + G.u + 64 * slice, 0);
+                    tma_load_4d(es + ES_VL, &tm_t, eb, 0, 0, wrow + G.ul + 64 * slice, 0);
+                    tma_load_4d(es + ES_E, &tm_t, eb, 0, 0, wrow + G.e, 0);
+                    tma_load_4d(es + ES_E + 8192, &tm_t, eb, 0, 0, wrow + G.e + 64, 0);
+                } else {
+                    mbar_arrive_expect_tx(eb, EARLY_TX + (second ? 8192u + 4096u : 0u));
+                    tma_load_4d(es + ES_V, &tm_v, eb, v0, h, t0, b);
+                    tma_load_4d(es + ES_TB, &tm_t, eb, 0, 0, wrow, 0);
+                    tma_load_4d(es + ES_TBG, &tm_t, eb, 0, 0, wrow + 64, 0);
+                }
                 if (second) {
                     // second half of a 128-token chunk: C2' for the key side and this
                     // slice's C1 V_a for the chain (two buffers: the chain may still be
@@ -814,6 +855,19 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 for (int kk = 0; kk < 4; ++kk)
                     umma_f16_ss(tmem + xcol, sdesc_sw128(ap + kk * 32, 16, 1024),
                                 sdesc_sw128(bd + kk * 2048, 8192, 1024), IDESC_KM64, 1);
+                if (GEN) {
+                    // P and Delta as hi + lo: + P_hi Delta_lo, + P_lo Delta_hi ([P_hi ; P_lo]:
+                    // its top half lands in lanes 0..63, whose -W h the chain has read)
+                    const uint32_t bdl = bd + 16384;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ss(tmem + xcol, sdesc_sw128(ap + kk * 32, 16, 1024),
+                                    sdesc_sw128(bdl + kk * 2048, 8192, 1024), IDESC_KM64, 1);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ss(tmem + xcol, sdesc_sw128(ap + 8192 + kk * 32, 16, 1024),
+                                    sdesc_sw128(bd + kk * 2048, 8192, 1024), IDESC_KM64, 1);
+                }
                 umma_commit(&bars[B_O + s]);
                 umma_commit(&bars[B_EMPTY + n % NSTAGE]);
                 opend = B_O + s;
@@ -834,10 +888,23 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         const bool lwarp = (kt >> 5) == 0;        // polls the group's waits
         const bool scan_warp = (kt >> 5) == 2;
         float ga0 = 1.f, ga1 = 1.f, gb0 = 0.f, gb1 = 0.f;
+        // GEN: the state's per-channel decay d of chunk mm (128 floats) into the
+        // gate record (channels 0..63 in eg, 64..127 in egc), by the scan warp
+        auto load_d = [&](int mm, tc::ChainParams *dst) {
+            const GenRows G = gen_rows(dv);
+            const float4 v = *reinterpret_cast<const float4 *>(
+                p.gen_ws + ((((size_t)b * H + h) * NC + mm) * p.ws_rows + G.d) * 128 + 16 * lane);
+            float *dd = lane < 16 ? dst->eg + 4 * lane : dst->egc + 4 * (lane - 16);
+            dd[0] = v.x; dd[1] = v.y; dd[2] = v.z; dd[3] = v.w;
+        };
         if (scan_warp) {
-            tc::fetch_gates(p.alpha, p.beta, b, T, H, h, 0, lane, true, ga0, ga1, gb0, gb1);
-            tc::scan_gates_chain(&params[0], ga0, ga1, lane);
-            tc::fetch_gates(p.alpha, p.beta, b, T, H, h, C, lane, NC > 1, ga0, ga1, gb0, gb1);
+            if (GEN) {
+                load_d(0, &params[0]);
+            } else {
+                tc::fetch_gates(p.alpha, p.beta, b, T, H, h, 0, lane, true, ga0, ga1, gb0, gb1);
+                tc::scan_gates_chain(&params[0], ga0, ga1, lane);
+                tc::fetch_gates(p.alpha, p.beta, b, T, H, h, C, lane, NC > 1, ga0, ga1, gb0, gb1);
+            }
         }
         int kcnt = 0;
         int pend = -1;   // leader: barrier of the last commit not yet known complete
@@ -881,7 +948,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     }
                 }
             };
-            {
+            if (!GEN) {
                 uint8_t *addr[8];
                 float sc[8];
 #pragma unroll
@@ -895,7 +962,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 convert(addr, sc, 8);
             }
             group_wait(&bars[B_EFULL], m & 1, E_FULL, 1, KS_THREADS, lwarp, true);
-            {
+            if (!GEN) {
                 uint8_t *addr[8];
                 float sc[8];
 #pragma unroll
@@ -916,18 +983,46 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             } else if (leader) {
                 tc_fence_after();
                 const uint32_t at = smem_u32(es + ES_TB), av = smem_u32(es + ES_V);
-                const uint32_t ag = smem_u32(es + ES_TBG), ak = smem_u32(st + S_K);
                 const uint32_t du = tmem + (s ? TM_U1 : TM_U0);
-                // U = T diag(beta) V: [T diag(beta) ; next rows] x V (MN-major), K = 64 tokens
+                if (GEN) {
+                    // U = TB U_in and W = TB E with TB, U_in as hi + lo (the lo x lo
+                    // product, about 2^-22 relative, dropped).  A = TB hi or lo with the
+                    // 8 KiB after it as padding rows; E two 64-column blocks 8 KiB apart.
+                    const uint32_t atl = smem_u32(es + ES_TBG), avl = smem_u32(es + ES_VL);
+                    const uint32_t ae = smem_u32(es + ES_E);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16_ss(du, sdesc_sw128(at + kk * 32, 16, 1024),
-                                sdesc_sw128(av + kk * 2048, 8192, 1024), IDESC_KM64, kk > 0);
-                // W = T diag(beta e^g) K: K as MN-major B with N = 128 (two key blocks)
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ss(du, sdesc_sw128(at + kk * 32, 16, 1024),
+                                    sdesc_sw128(av + kk * 2048, 8192, 1024), IDESC_KM64, kk > 0);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    umma_f16_ss(tmem + TM_W, sdesc_sw128(ag + kk * 32, 16, 1024),
-                                sdesc_sw128(ak + kk * 2048, S_KB, 1024), IDESC_KM128, kk > 0);
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ss(du, sdesc_sw128(at + kk * 32, 16, 1024),
+                                    sdesc_sw128(avl + kk * 2048, 8192, 1024), IDESC_KM64, 1);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ss(du, sdesc_sw128(atl + kk * 32, 16, 1024),
+                                    sdesc_sw128(av + kk * 2048, 8192, 1024), IDESC_KM64, 1);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ss(tmem + TM_W, sdesc_sw128(at + kk * 32, 16, 1024),
+                                    sdesc_sw128(ae + kk * 2048, 8192, 1024), IDESC_KM128, kk > 0);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ss(tmem + TM_W, sdesc_sw128(atl + kk * 32, 16, 1024),
+                                    sdesc_sw128(ae + kk * 2048, 8192, 1024), IDESC_KM128, 1);
+                } else {
+                    const uint32_t ag = smem_u32(es + ES_TBG), ak = smem_u32(st + S_K);
+                    // U = T diag(beta) V: [T diag(beta) ; next rows] x V (MN-major), K = 64 tokens
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ss(du, sdesc_sw128(at + kk * 32, 16, 1024),
+                                    sdesc_sw128(av + kk * 2048, 8192, 1024), IDESC_KM64, kk > 0);
+                    // W = T diag(beta e^g) K: K as MN-major B with N = 128 (two key blocks)
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ss(tmem + TM_W, sdesc_sw128(ag + kk * 32, 16, 1024),
+                                    sdesc_sw128(ak + kk * 2048, S_KB, 1024), IDESC_KM128, kk > 0);
+                }
                 umma_commit(&bars[B_UW]);
                 umma_commit(&bars[B_EEMPTY]);       // the early slot reloads once U and W are formed
                 pend = B_UW; pend_par = m & 1;
@@ -935,8 +1030,12 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             __syncwarp();
             // gates of the next chunk meanwhile
             if (scan_warp && m + 1 < NC) {
-                tc::scan_gates_chain(&params[(m + 1) % 3], ga0, ga1, lane);
-                tc::fetch_gates(p.alpha, p.beta, b, T, H, h, (m + 2) * C, lane, m + 2 < NC, ga0, ga1, gb0, gb1);
+                if (GEN) {
+                    load_d(m + 1, &params[(m + 1) % 3]);
+                } else {
+                    tc::scan_gates_chain(&params[(m + 1) % 3], ga0, ga1, lane);
+                    tc::fetch_gates(p.alpha, p.beta, b, T, H, h, (m + 2) * C, lane, m + 2 < NC, ga0, ga1, gb0, gb1);
+                }
             }
             group_wait(&bars[B_UW], m & 1, E_UW, 1, KS_THREADS, lwarp, false);
             if (!sync_ok(1, KS_THREADS, leader, kcnt)) break;
@@ -956,8 +1055,9 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     for (int j = 0; j < 64; ++j) x[j] = -x[j];
                 }
                 st_row_f16(st + hf * S_KB + S_W, r, x);
-            } else {
+            } else if (!GEN) {
                 // W has read K: K -> diag(e^{g_C - g}) K in place for the state update
+                // (GEN: K'' comes scaled from the prep)
                 const int t2 = 64 * hf + 32 * (sp - 2) + lane;
                 uint8_t *addr[8];
                 uint4 w[8];
@@ -1083,7 +1183,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             {
                 float x[64];
                 tmem_ld64(tmem + lane_base + TM_H, x);
-                const float egC = par->egC;
+                // the state's decay over the chunk: e^{g_C}, or per key channel (GEN)
+                const float egC = GEN ? (hrow < 64 ? par->eg[hrow] : par->egc[hrow - 64]) : par->egC;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     uint32_t y[32];
@@ -1156,6 +1257,12 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
                     for (int j = 0; j < 64; ++j) x[j] += cr[j];
                 }
+                if (GEN) {
+                    // Delta as hi + lo fp16 (u reused for the low parts)
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) u[j] = x[j] - __half2float(__float2half_rn(x[j]));
+                    st_row_f16(sm + OFF_DS + 16384 + s * 8192, r, u);
+                }
                 st_row_f16(sm + OFF_DS + s * 8192, r, x);
             }
             fence_proxy_async_smem();
@@ -1172,6 +1279,12 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                 for (int kk = 0; kk < 4; ++kk)
                     umma_f16_ss(tmem + TM_H, sdesc_sw128(ak + kk * 2048, S_KB, 1024),
                                 sdesc_sw128(bd + kk * 2048, 8192, 1024), IDESC_MM64, 1);
+                if (GEN) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_f16_ss(tmem + TM_H, sdesc_sw128(ak + kk * 2048, S_KB, 1024),
+                                    sdesc_sw128(bd + 16384 + kk * 2048, 8192, 1024), IDESC_MM64, 1);
+                }
                 umma_commit(&bars[B_H]);
                 umma_commit(&bars[B_EMPTY + n % NSTAGE]);   // X and the state update have read the stage
                 umma_commit(&bars[B_KSFREE + s]);            // and Delta has read U
@@ -1257,7 +1370,19 @@ bool make_map_t(CUtensorMap *m, const void *ptr, size_t rows) {
 
 bool tc_supports(const FwdParams &p, const char **why) {
     if (!p.io_bf16) { *why = "needs bf16 q/k/v"; return false; }
-    if (p.general) { *why = "two-gate rule runs on the SIMT kernel"; return false; }
+    if (p.general) {
+        // the two-gate rule: the SIMT prep's matrices in fp16 for the chain kernel
+        if (p.C != C) { *why = "two-gate rule: needs chunk 64"; return false; }
+        if (p.mode == GDN_INV_NEUMANN_RESIDUAL) { *why = "two-gate rule: no residual correction"; return false; }
+        if (p.precond > 1) {
+            *why = "two-gate rule: preconditioner forms 2 and 3 (unbounded write keys) run on the SIMT kernel";
+            return false;
+        }
+        if (p.dk != DK) { *why = "needs dk 128"; return false; }
+        if (p.dv % DVS != 0) { *why = "needs dv a multiple of 64"; return false; }
+        if (p.slices && p.dvs != DVS) { *why = "value slices must be 64 columns"; return false; }
+        return true;
+    }
     if (p.C != C && !(p.C == 2 * C && p.mode == GDN_INV_NEUMANN)) {
         *why = "needs chunk 64 (or 128 with the masked series)";
         return false;
@@ -1272,6 +1397,7 @@ bool tc_supports(const FwdParams &p, const char **why) {
 int tc_default_slices(const FwdParams &p) { return p.dv / DVS; }
 
 size_t tc_workspace_bytes(const FwdParams &p) {
+    if (p.general) return gen_prep_workspace_bytes(p);
     const size_t nc = (size_t)(p.T + C - 1) / C;
     const size_t per = WS_CHUNK_BYTES + (p.C == 2 * C ? pair_stride(p.dv) * 4 : 0);
     return (size_t)p.B * p.H * nc * per;
@@ -1280,6 +1406,28 @@ size_t tc_workspace_bytes(const FwdParams &p) {
 cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, const char **why) {
     const int NC = (p.T + C - 1) / C;
     CUtensorMap mq, mk, mv, mt;
+    if (p.general) {
+        // the two-gate rule: the prep's fp16 rows, then the chain kernel (every
+        // operand from the workspace through one map)
+        const GenRows G = gen_rows(p.dv);
+        if (!make_map_t(&mt, workspace, (size_t)p.B * p.H * NC * G.rows)) {
+            *why = "(tensor map encoding failed)";
+            return cudaErrorInvalidValue;
+        }
+        cudaError_t e = launch_gen_prep(p, workspace, stream);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(chain_kernel<K2_GEN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)K2Layout<K2_GEN>::SMEM);
+        if (e != cudaSuccess) return e;
+        K2Params k2{};
+        k2.B = p.B; k2.T = p.T; k2.H = p.H; k2.dv = p.dv; k2.NC = NC;
+        k2.S0 = p.S0; k2.o = p.o; k2.S_T = p.S_T; k2.o_bf16 = p.o_bf16;
+        k2.gen_ws = reinterpret_cast<const uint8_t *>(workspace);
+        k2.ws_rows = G.rows;
+        chain_kernel<K2_GEN><<<dim3(p.slices, p.H, p.B), K2_THREADS, K2Layout<K2_GEN>::SMEM, stream>>>(mt, mt, mt,
+                                                                                                      mt, k2);
+        return cudaGetLastError();
+    }
     if (!make_map_bthd(&mq, p.q, p.B, p.T, p.H, p.dk) || !make_map_bthd(&mk, p.k, p.B, p.T, p.H, p.dk) ||
         !make_map_bthd(&mv, p.v, p.B, p.T, p.H, p.dv) ||
         !make_map_t(&mt, workspace, (size_t)p.B * p.H * NC * WS_ROWS)) {
@@ -1299,10 +1447,10 @@ cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, 
         cudaError_t e = cudaFuncSetAttribute(keyside_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)K1_SMEM_RES);
         if (e != cudaSuccess) return e;
-        e = pair ? cudaFuncSetAttribute(chain_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)K2Layout<true>::SMEM)
-                 : cudaFuncSetAttribute(chain_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)K2Layout<false>::SMEM);
+        e = pair ? cudaFuncSetAttribute(chain_kernel<K2_PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)K2Layout<K2_PAIR>::SMEM)
+                 : cudaFuncSetAttribute(chain_kernel<K2_PLAIN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)K2Layout<K2_PLAIN>::SMEM);
         if (e != cudaSuccess) return e;
     }
     if (pair && NC / 2 > 0) {
@@ -1332,16 +1480,17 @@ cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, 
     keyside_kernel<<<dim3(NC, p.H, p.B), K1_THREADS, k1.neumann == 2 ? K1_SMEM_RES : K1_SMEM, stream>>>(mq, mk, k1);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    K2Params k2;
+    K2Params k2{};
+    k2.ws_rows = WS_ROWS;
     k2.B = p.B; k2.T = p.T; k2.H = p.H; k2.dv = p.dv; k2.NC = NC;
     k2.alpha = p.alpha; k2.beta = p.beta; k2.S0 = p.S0; k2.o = p.o; k2.S_T = p.S_T;
     k2.pair_ws = pair_ws;
     k2.o_bf16 = p.o_bf16;
     if (pair)
-        chain_kernel<true><<<dim3(p.slices, p.H, p.B), K2_THREADS, K2Layout<true>::SMEM, stream>>>(mq, mk, mv, mt,
+        chain_kernel<K2_PAIR><<<dim3(p.slices, p.H, p.B), K2_THREADS, K2Layout<K2_PAIR>::SMEM, stream>>>(mq, mk, mv, mt,
                                                                                                   k2);
     else
-        chain_kernel<false><<<dim3(p.slices, p.H, p.B), K2_THREADS, K2Layout<false>::SMEM, stream>>>(mq, mk, mv,
+        chain_kernel<K2_PLAIN><<<dim3(p.slices, p.H, p.B), K2_THREADS, K2Layout<K2_PLAIN>::SMEM, stream>>>(mq, mk, mv,
                                                                                                     mt, k2);
     return cudaGetLastError();
 }

@@ -115,8 +115,14 @@ def test_valid_arguments_select_a_kernel():
     assert gdn.select_kernel(_args(T=9)) == 4                                  # chunked from T = 9
     assert gdn.select_kernel(_args(T=1, mode=1, neumann_N=3)) != 3             # series: chunked only
     assert gdn.select_kernel(_args(io_dtype=0, dk=64, dv=64)) == 1   # fp32 io -> SIMT
-    assert gdn.select_kernel(_args(alpha=0x70000, precond=1, erase=0x50000,
-                                   write=0x58000, alpha_per_channel=1)) in (1, 2)
+    # the two-gate rule: split tensor-core kernels (SIMT prep in fp16 rows + chain) at
+    # chunk 64 with preconditioner forms 0 and 1; forms 2, 3, other chunks: SIMT
+    two_gate = dict(alpha=0x70000, erase=0x50000, write=0x58000, alpha_per_channel=1)
+    assert gdn.select_kernel(_args(precond=1, **two_gate)) == 4
+    assert gdn.select_kernel(_args(precond=0, **two_gate)) == 4
+    assert gdn.select_kernel(_args(precond=2, **two_gate)) == 1
+    assert gdn.select_kernel(_args(precond=1, chunk=32, **two_gate)) == 1
+    assert gdn.select_kernel(_args(precond=1, kernel=2, **two_gate)) < 0     # not on the fused kernel
     assert gdn.select_kernel(_args(S0=0x80000, S_T=0x80000)) in (1, 2, 4)  # S_T may alias S0
     # chunk 128: the masked series (N <= 15) on the split kernels as two 64-token
     # halves; the exact inverse and wider bands on the SIMT kernel
@@ -274,6 +280,11 @@ def test_workspace_sizes_per_kernel():
     assert gdn.workspace_bytes(_args(kernel=1)) == chunks * per * 4
     two_gate = _args(kernel=1, alpha=0x70000, alpha_per_channel=1, precond=1, erase=0x50000, write=0x58000)
     assert gdn.workspace_bytes(two_gate) == chunks * (per + 3 * dk) * 4
+    # the two-gate rule on the split tensor-core kernels: fp16 rows of 128 B per
+    # chunk-head (TB, P as hi + lo: 4 x 64; E, Q', K'': 128 each; U as hi + lo: 2 d_v;
+    # d: 4), then the preconditioner's three running-average arrays
+    two_gate_tc = _args(kernel=4, alpha=0x70000, alpha_per_channel=1, precond=1, erase=0x50000, write=0x58000)
+    assert gdn.workspace_bytes(two_gate_tc) == chunks * ((640 + 2 * 128 + 4) * 128 + 3 * dk * 4)
     assert gdn.workspace_bytes(_args(kernel=4)) == chunks * 24576
     assert gdn.workspace_bytes(_args(kernel=2)) == 0
     assert gdn.workspace_bytes(_args(T=4, kernel=3)) == 0

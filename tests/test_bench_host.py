@@ -171,7 +171,7 @@ def test_e2e_falls_back_to_one_stream(fake_cuda, monkeypatch):
 
 @pytest.mark.parametrize("name,kernel,launches", [("plain_fp32", "simt_prep_kernel+simt_chain_kernel", 2),
                                                   ("long_context", "keyside_kernel+chain_kernel", 2),
-                                                  ("precond_two_gate", "simt_prep_kernel+simt_chain_kernel", 4)])
+                                                  ("precond_two_gate", "simt_prep_kernel+chain_kernel", 4)])
 def test_other_workload_lines(fake_cuda, monkeypatch, name, kernel, launches):
     import bench
     # the line's assembly only: a stand-in for the oracle timing of a whole long sequence

@@ -189,19 +189,34 @@ def test_recurrent_short_sequence_bf16():
 # ------------------------------------------------------------ configuration 5
 
 @needs_cuda
-def test_precond_two_gate_small():
+@pytest.mark.parametrize("kernel", ["auto", "simt", "tc_split"])
+def test_precond_two_gate_small(kernel):
+    """auto and tc_split: the SIMT prep writes fp16 rows for the tensor-core chain;
+    simt: the fp32 chain."""
     w = workload("precond_two_gate", B=1, H=2, T=300)
     x = make_inputs(w, seed=5)
     o_ref, s_ref = run_oracle(x, w)
-    _check_bf16("precond_small", w, x, o_ref, s_ref)
+    _check_bf16(f"precond_small_{kernel}", w, x, o_ref, s_ref, kernel=kernel)
 
 
 @needs_cuda
-def test_precond_two_gate_full_size():
+@pytest.mark.parametrize("kernel", ["auto", "simt"])
+def test_precond_two_gate_full_size(kernel):
     w = workload("precond_two_gate")
     x = make_inputs(w)
     o_ref, s_ref = run_oracle(x, w)
-    _check_bf16("precond_full_auto", w, x, o_ref, s_ref)
+    _check_bf16(f"precond_full_{kernel}", w, x, o_ref, s_ref, kernel=kernel)
+
+
+@needs_cuda
+@pytest.mark.parametrize("T,s0,dv", [(1000, 0.02, 128), (4096, 0.0, 64), (65, 0.02, 128)])
+def test_precond_two_gate_tensor_cores(T, s0, dv):
+    """The two-gate rule on the tensor-core chain: ragged tails (a one-token last
+    chunk), an initial state, d_v 64 (one value slice), against the oracle."""
+    w = workload("precond_two_gate", B=2, H=2, T=T, s0_std=s0, dv=dv)
+    x = make_inputs(w, seed=30 + T)
+    o_ref, s_ref = run_oracle(x, w)
+    _check_bf16(f"precond_tc_T{T}_dv{dv}", w, x, o_ref, s_ref, kernel="tc_split")
 
 
 @needs_cuda
