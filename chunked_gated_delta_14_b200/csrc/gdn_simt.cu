@@ -50,10 +50,21 @@ namespace gdn {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kPrepThreads = 512;   // prep kernel: one block per SM by shared memory, so 16 warps
 
 __device__ __forceinline__ float load_in(const void *p, size_t i, int bf16) {
     if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
     return reinterpret_cast<const float *>(p)[i];
+}
+
+// Four consecutive inputs from element i (i a multiple of 4; bf16 or fp32).
+__device__ __forceinline__ float4 load4_in(const void *p, size_t i, int bf16) {
+    if (bf16) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(reinterpret_cast<const __nv_bfloat16 *>(p) + i);
+        return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                           __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+    }
+    return *reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(p) + i);
 }
 
 template <typename S>
@@ -203,7 +214,7 @@ __global__ void rho_combine_kernel(const FwdParams p, const float *sums, const f
 // tensor-core chain (gen_rows), together with U = w (.) v, instead of fp32.
 // rho0: the preconditioner's running average at every chunk start.
 template <typename KS, bool GENERAL, bool TCOUT = false>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kPrepThreads)
 simt_prep_kernel(const FwdParams p, float *ws, const float *rho0) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -234,20 +245,63 @@ simt_prep_kernel(const FwdParams p, float *ws, const float *rho0) {
     __half *ob = reinterpret_cast<__half *>(ws) + (bh * NC + n) * (size_t)GR.rows * 64;   // TCOUT rows
 
     // ---------------------------------------------------------- load
-    for (int idx = tid; idx < C * dk; idx += kThreads) {
-        const int r = idx / dk, c = idx % dk;
-        const size_t gi = (((size_t)b * T + t0 + r) * H + h) * dk + c;
-        const bool ok = r < Cv;
-        const int si = r * ks + c;
-        st_s(kx, si, ok ? load_in(p.k, gi, p.io_bf16) : 0.f);
-        st_s(qx, si, ok ? load_in(p.q, gi, p.io_bf16) : 0.f);
-        if (GENERAL) {
-            ex[si] = ok ? (p.erase ? load_in(p.erase, gi, p.io_bf16) : 1.f) : 0.f;
-            gx[si] = (ok && p.alpha) ? log2f(p.alpha[p.alpha_pc ? gi : gi / dk]) : 0.f;
+    // four consecutive channels per item, four items' loads issued before the
+    // first store, so that their latencies overlap
+    {
+        constexpr int UNR = 4;
+        const int n4 = C * dk / 4;
+        const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f), one4 = make_float4(1.f, 1.f, 1.f, 1.f);
+        for (int base = tid; base < n4; base += kPrepThreads * UNR) {
+            float4 kv[UNR], qv[UNR], ev[UNR], av[UNR];
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int i4 = base + kPrepThreads * u;
+                kv[u] = qv[u] = ev[u] = zero4;
+                av[u] = one4;
+                if (i4 < n4) {
+                    const int r = (4 * i4) / dk, c = (4 * i4) % dk;
+                    if (r < Cv) {
+                        const size_t gi = (((size_t)b * T + t0 + r) * H + h) * dk + c;
+                        kv[u] = load4_in(p.k, gi, p.io_bf16);
+                        qv[u] = load4_in(p.q, gi, p.io_bf16);
+                        if (GENERAL) {
+                            ev[u] = p.erase ? load4_in(p.erase, gi, p.io_bf16) : one4;
+                            if (p.alpha) {
+                                if (p.alpha_pc) {
+                                    av[u] = *reinterpret_cast<const float4 *>(p.alpha + gi);
+                                } else {
+                                    const float a = p.alpha[gi / dk];
+                                    av[u] = make_float4(a, a, a, a);
+                                }
+                            }
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int i4 = base + kPrepThreads * u;
+                if (i4 < n4) {
+                    const int r = (4 * i4) / dk, c = (4 * i4) % dk, si = r * ks + c;
+                    const float kk[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+                    const float qq[4] = {qv[u].x, qv[u].y, qv[u].z, qv[u].w};
+                    const float ee[4] = {ev[u].x, ev[u].y, ev[u].z, ev[u].w};
+                    const float aa[4] = {av[u].x, av[u].y, av[u].z, av[u].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        st_s(kx, si + e, kk[e]);
+                        st_s(qx, si + e, qq[e]);
+                        if (GENERAL) {
+                            ex[si + e] = ee[e];
+                            gx[si + e] = log2f(aa[e]);   // 0 past the end and without a decay
+                        }
+                    }
+                }
+            }
         }
     }
     if (!GENERAL) {
-        for (int r = tid; r < C; r += kThreads) {
+        for (int r = tid; r < C; r += kPrepThreads) {
             const size_t ti = ((size_t)b * T + t0 + r) * H + h;
             g[r] = (r < Cv && p.alpha) ? logf(p.alpha[ti]) : 0.f;
             bet[r] = (r < Cv) ? (p.beta ? p.beta[ti] : 1.f) : 0.f;
@@ -262,7 +316,7 @@ simt_prep_kernel(const FwdParams p, float *ws, const float *rho0) {
         // into [1/x, x] on a log scale; applied to the write key (forms 2, 3
         // read the state with the raw key) or to the query
         const float lnx = p.precond == 3 ? logf(p.precond_x) : 1.f;
-        for (int c = tid; c < dk; c += kThreads) {
+        for (int c = tid; c < dk; c += kPrepThreads) {
             float rh = p.precond ? rho0[(bh * NC + n) * dk + c] : 0.f, G = 0.f;
             for (int r = 0; r < C; ++r) {
                 const int idx = r * ks + c;
@@ -291,28 +345,63 @@ simt_prep_kernel(const FwdParams p, float *ws, const float *rho0) {
         warp0_inclusive_scan(g, C);
     }
     __syncthreads();
-    // ------------------------------------------------ L (strictly lower)
-    // 4 x 4 register tiles (rows r0.., keys i0..): 8 loads per 16 products
-    for (int t = tid; t < (C / 4) * (C / 4); t += kThreads) {
-        const int r0 = 4 * (t / (C / 4)), i0 = 4 * (t % (C / 4));
-        float acc[4][4] = {};
-        if (i0 < r0 + 3) {
-            if (GENERAL) {
-                for (int c = 0; c < dk; ++c) {
-                    float er[4], gr[4], ki[4], gi[4];
+    // The two-gate rule's decayed Gram sums_c X[r][c] kw[i][c] 2^{GX[r][c] - G[i][c]}
+    // over the lower 4 x 4 tiles (r-block >= i-block), four lanes per tile on
+    // interleaved channel quarters (c = 4 cc + part), reduced with shuffles: every
+    // warp of the block has work and each chain is a quarter as long.  GX is G_r,
+    // or G_{r-1} (shift 1, G_{-1} = 0).  store(r0, i0, acc) writes one tile.
+    auto decayed_gram = [&](const float *X, int shift, auto &&store) {
+        const int nT = C / 4, tiles = nT * (nT + 1) / 2, items = ((4 * tiles + 31) / 32) * 32;
+        for (int w = tid; w < items; w += kPrepThreads) {
+            const int part = w & 3, tix = w >> 2;
+            const bool need = tix < tiles;
+            int R = 0;
+            while ((R + 1) * (R + 2) / 2 <= tix) ++R;
+            const int r0 = 4 * R, i0 = 4 * (tix - R * (R + 1) / 2);
+            float acc[4][4] = {};
+            if (need) {
+                for (int cc = 0; cc < dk / 4; ++cc) {
+                    const int c = 4 * cc + part;
+                    float xr[4], gr[4], yi[4], gi[4];
 #pragma unroll
                     for (int a = 0; a < 4; ++a) {
-                        er[a] = ex[(r0 + a) * ks + c];
-                        gr[a] = (r0 + a > 0) ? gx[(r0 + a - 1) * ks + c] : 0.f;
-                        ki[a] = ld_s(kx, (i0 + a) * ks + c);
+                        xr[a] = X[(r0 + a) * ks + c];
+                        gr[a] = (shift && r0 + a == 0) ? 0.f : gx[(r0 + a - shift) * ks + c];
+                        yi[a] = ld_s(kx, (i0 + a) * ks + c);
                         gi[a] = gx[(i0 + a) * ks + c];
                     }
 #pragma unroll
                     for (int a = 0; a < 4; ++a)
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) acc[a][e] += er[a] * ki[e] * fast_exp2(gr[a] - gi[e]);
+                        for (int e = 0; e < 4; ++e) acc[a][e] += xr[a] * yi[e] * fast_exp2(gr[a] - gi[e]);
                 }
-            } else {
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    acc[a][e] += __shfl_xor_sync(0xffffffffu, acc[a][e], 1);
+                    acc[a][e] += __shfl_xor_sync(0xffffffffu, acc[a][e], 2);
+                }
+            if (need && part == 0) store(r0, i0, acc);
+        }
+    };
+    // ------------------------------------------------ L (strictly lower)
+    if (GENERAL) {
+        decayed_gram(reinterpret_cast<const float *>(ex), 1, [&](int r0, int i0, const float (&acc)[4][4]) {
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) tp[(r0 + a) * C + i0 + e] = (i0 + e < r0 + a) ? acc[a][e] : 0.f;
+        });
+        for (int idx = tid; idx < C * C; idx += kPrepThreads)
+            if (((idx % C) >> 2) > ((idx / C) >> 2)) tp[idx] = 0.f;   // tiles above the diagonal
+    } else {
+        // 4 x 4 register tiles (rows r0.., keys i0..): 8 loads per 16 products
+        for (int t = tid; t < (C / 4) * (C / 4); t += kPrepThreads) {
+            const int r0 = 4 * (t / (C / 4)), i0 = 4 * (t % (C / 4));
+            float acc[4][4] = {};
+            if (i0 < r0 + 3) {
                 for (int c = 0; c < dk; ++c) {
                     float kr[4], ki[4];
 #pragma unroll
@@ -326,16 +415,14 @@ simt_prep_kernel(const FwdParams p, float *ws, const float *rho0) {
                         for (int e = 0; e < 4; ++e) acc[a][e] += kr[a] * ki[e];
                 }
             }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int r = r0 + a, i = i0 + e;
+                    tp[r * C + i] = (i < r) ? bet[r] * expf(g[r] - g[i]) * acc[a][e] : 0.f;
+                }
         }
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int r = r0 + a, i = i0 + e;
-                float val = 0.f;
-                if (i < r) val = GENERAL ? acc[a][e] : bet[r] * expf(g[r] - g[i]) * acc[a][e];
-                tp[r * C + i] = val;
-            }
     }
     __syncthreads();
     // ------------------------------------------------ T = (I + L)^-1
@@ -352,16 +439,16 @@ simt_prep_kernel(const FwdParams p, float *ws, const float *rho0) {
             }
             __syncthreads();
         }
-        for (int r = tid; r < C; r += kThreads) tp[r * C + r] = 1.f;
+        for (int r = tid; r < C; r += kPrepThreads) tp[r * C + r] = 1.f;
     } else {
         // Horner on the band: T <- M (.) (I + A T), A = -L, T^(0) = I.
         // band[i*(N+1)+d] holds T_{i,i-d}.
         const int Wd = N + 1;
         float *cur = band, *nxt = band + (size_t)C * Wd;
-        for (int idx = tid; idx < C * Wd; idx += kThreads) cur[idx] = (idx % Wd == 0) ? 1.f : 0.f;
+        for (int idx = tid; idx < C * Wd; idx += kPrepThreads) cur[idx] = (idx % Wd == 0) ? 1.f : 0.f;
         __syncthreads();
         for (int step = 0; step < N; ++step) {
-            for (int idx = tid; idx < C * Wd; idx += kThreads) {
+            for (int idx = tid; idx < C * Wd; idx += kPrepThreads) {
                 const int i = idx / Wd, d = idx % Wd, j = i - d;
                 float val = 0.f;
                 if (j >= 0) {
@@ -375,7 +462,7 @@ simt_prep_kernel(const FwdParams p, float *ws, const float *rho0) {
             __syncthreads();
             float *sw = cur; cur = nxt; nxt = sw;
         }
-        for (int idx = tid; idx < C * C; idx += kThreads) {
+        for (int idx = tid; idx < C * C; idx += kPrepThreads) {
             const int i = idx / C, j = idx % C, d = i - j;
             tp[idx] = (d >= 0 && d <= N) ? cur[i * Wd + d] : 0.f;
         }
@@ -383,7 +470,7 @@ simt_prep_kernel(const FwdParams p, float *ws, const float *rho0) {
     __syncthreads();
     // ------------------------------------------------ the chunk's matrices
     // TB = T diag(beta) (scalar rule; the two-gate rule has no beta)
-    for (int idx = tid; idx < C * C; idx += kThreads) {
+    for (int idx = tid; idx < C * C; idx += kPrepThreads) {
         const float tb = GENERAL ? tp[idx] : tp[idx] * bet[idx % C];
         if (TCOUT) {
             const __half hi = __float2half_rn(tb);
@@ -393,27 +480,31 @@ simt_prep_kernel(const FwdParams p, float *ws, const float *rho0) {
             out[W.tb + idx] = tb;
         }
     }
-    // P: decayed causal scores, 4 x 4 register tiles
-    for (int t = tid; t < (C / 4) * (C / 4); t += kThreads) {
-        const int r0 = 4 * (t / (C / 4)), i0 = 4 * (t % (C / 4));
-        float acc[4][4] = {};
-        if (i0 <= r0 + 3) {
-            if (GENERAL) {
-                for (int c = 0; c < dk; ++c) {
-                    float qr[4], gr[4], ki[4], gi[4];
+    // P: decayed causal scores
+    auto store_p = [&](int r, int i, float val) {
+        if (TCOUT) {
+            const __half hi = __float2half_rn(val);
+            ob[(size_t)(GR.pp + r) * 64 + i] = hi;
+            ob[(size_t)(GR.ppl + r) * 64 + i] = __float2half_rn(val - __half2float(hi));
+        } else {
+            out[W.pp + r * C + i] = val;
+        }
+    };
+    if (GENERAL) {
+        decayed_gram(reinterpret_cast<const float *>(qx), 0, [&](int r0, int i0, const float (&acc)[4][4]) {
 #pragma unroll
-                    for (int a = 0; a < 4; ++a) {
-                        qr[a] = ld_s(qx, (r0 + a) * ks + c);
-                        gr[a] = gx[(r0 + a) * ks + c];
-                        ki[a] = ld_s(kx, (i0 + a) * ks + c);
-                        gi[a] = gx[(i0 + a) * ks + c];
-                    }
+            for (int a = 0; a < 4; ++a)
 #pragma unroll
-                    for (int a = 0; a < 4; ++a)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) acc[a][e] += qr[a] * ki[e] * fast_exp2(gr[a] - gi[e]);
-                }
-            } else {
+                for (int e = 0; e < 4; ++e) store_p(r0 + a, i0 + e, (i0 + e <= r0 + a) ? acc[a][e] : 0.f);
+        });
+        for (int idx = tid; idx < C * C; idx += kPrepThreads)
+            if (((idx % C) >> 2) > ((idx / C) >> 2)) store_p(idx / C, idx % C, 0.f);   // above the diagonal
+    } else {
+        // 4 x 4 register tiles
+        for (int t = tid; t < (C / 4) * (C / 4); t += kPrepThreads) {
+            const int r0 = 4 * (t / (C / 4)), i0 = 4 * (t % (C / 4));
+            float acc[4][4] = {};
+            if (i0 <= r0 + 3) {
                 for (int c = 0; c < dk; ++c) {
                     float qr[4], ki[4];
 #pragma unroll
@@ -427,34 +518,38 @@ simt_prep_kernel(const FwdParams p, float *ws, const float *rho0) {
                         for (int e = 0; e < 4; ++e) acc[a][e] += qr[a] * ki[e];
                 }
             }
-        }
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < 4; ++a)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int r = r0 + a, i = i0 + e;
-                float val = 0.f;
-                if (i <= r) val = GENERAL ? acc[a][e] : expf(g[r] - g[i]) * acc[a][e];
-                if (TCOUT) {
-                    const __half hi = __float2half_rn(val);
-                    ob[(size_t)(GR.pp + r) * 64 + i] = hi;
-                    ob[(size_t)(GR.ppl + r) * 64 + i] = __float2half_rn(val - __half2float(hi));
-                } else {
-                    out[W.pp + r * C + i] = val;
+                for (int e = 0; e < 4; ++e) {
+                    const int r = r0 + a, i = i0 + e;
+                    store_p(r, i, (i <= r) ? expf(g[r] - g[i]) * acc[a][e] : 0.f);
                 }
-            }
+        }
     }
     // E (the state read), Q' (the output read), K'' (the state write)
-    for (int idx = tid; idx < C * dk; idx += kThreads) {
-        const int r = idx / dk, c = idx % dk, si = r * ks + c;
-        if (TCOUT) {
-            // 64-column blocks: channel c of row r at row (block base + 64 (c / 64) + r)
-            const float Gl = gx[(C - 1) * ks + c];
+    if (TCOUT) {
+        // 64-column blocks: channel c of row r at row (block base + 64 (c / 64) + r);
+        // two channels per item, stored as one fp16 pair
+        for (int idx = tid; idx < C * dk / 2; idx += kPrepThreads) {
+            const int r = (2 * idx) / dk, c = (2 * idx) % dk, si = r * ks + c;
+            float e2[2], q2[2], k2[2];
+#pragma unroll
+            for (int z = 0; z < 2; ++z) {
+                const float Gl = gx[(C - 1) * ks + c + z];
+                e2[z] = ex[si + z] * ((r > 0) ? fast_exp2(gx[si + z - ks]) : 1.f);
+                q2[z] = ld_s(qx, si + z) * fast_exp2(gx[si + z]);
+                k2[z] = ld_s(kx, si + z) * fast_exp2(Gl - gx[si + z]);
+            }
             const size_t o = (size_t)(64 * (c >> 6) + r) * 64 + (c & 63);
-            ob[(size_t)GR.e * 64 + o] = __float2half_rn(ex[si] * ((r > 0) ? fast_exp2(gx[si - ks]) : 1.f));
-            ob[(size_t)GR.q * 64 + o] = __float2half_rn(ld_s(qx, si) * fast_exp2(gx[si]));
-            ob[(size_t)GR.k * 64 + o] = __float2half_rn(ld_s(kx, si) * fast_exp2(Gl - gx[si]));
-        } else if (GENERAL) {
+            *reinterpret_cast<__half2 *>(ob + (size_t)GR.e * 64 + o) = __floats2half2_rn(e2[0], e2[1]);
+            *reinterpret_cast<__half2 *>(ob + (size_t)GR.q * 64 + o) = __floats2half2_rn(q2[0], q2[1]);
+            *reinterpret_cast<__half2 *>(ob + (size_t)GR.k * 64 + o) = __floats2half2_rn(k2[0], k2[1]);
+        }
+    }
+    for (int idx = tid; idx < (TCOUT ? 0 : C * dk); idx += kPrepThreads) {
+        const int r = idx / dk, c = idx % dk, si = r * ks + c;
+        if (GENERAL) {
             const float Gl = gx[(C - 1) * ks + c];
             out[W.e + idx] = ex[si] * ((r > 0) ? fast_exp2(gx[si - ks]) : 1.f);
             out[W.q + idx] = ld_s(qx, si) * fast_exp2(gx[si]);
@@ -467,25 +562,51 @@ simt_prep_kernel(const FwdParams p, float *ws, const float *rho0) {
         }
     }
     // d: the state's decay over the chunk
-    for (int c = tid; c < dk; c += kThreads) {
+    for (int c = tid; c < dk; c += kPrepThreads) {
         const float dc = GENERAL ? fast_exp2(gx[(C - 1) * ks + c]) : expf(g[C - 1]);
         if (TCOUT) reinterpret_cast<float *>(ob + (size_t)GR.d * 64)[c] = dc;
         else out[W.d + c] = dc;
     }
     if (TCOUT) {
-        // U = w (.) v (hi, lo), one 64-column block per value slice; zero past the end
-        for (int idx = tid; idx < C * p.dv; idx += kThreads) {
-            const int r = idx / p.dv, j = idx % p.dv;
-            float u = 0.f;
-            if (r < Cv) {
-                const size_t gi = (((size_t)b * T + t0 + r) * H + h) * p.dv + j;
-                u = load_in(p.v, gi, p.io_bf16);
-                if (p.write) u *= load_in(p.write, gi, p.io_bf16);
+        // U = w (.) v (hi, lo), one 64-column block per value slice; zero past the
+        // end.  Four values per item, four items' loads in flight together.
+        constexpr int UNR = 4;
+        const int n4 = C * p.dv / 4;
+        for (int base = tid; base < n4; base += kPrepThreads * UNR) {
+            float4 vv[UNR], ww[UNR];
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int i4 = base + kPrepThreads * u;
+                vv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                ww[u] = make_float4(1.f, 1.f, 1.f, 1.f);
+                if (i4 < n4) {
+                    const int r = (4 * i4) / p.dv, j = (4 * i4) % p.dv;
+                    if (r < Cv) {
+                        const size_t gi = (((size_t)b * T + t0 + r) * H + h) * p.dv + j;
+                        vv[u] = load4_in(p.v, gi, p.io_bf16);
+                        if (p.write) ww[u] = load4_in(p.write, gi, p.io_bf16);
+                    }
+                }
             }
-            const size_t o = (size_t)(64 * (j >> 6) + r) * 64 + (j & 63);
-            const __half hi = __float2half_rn(u);
-            ob[(size_t)GR.u * 64 + o] = hi;
-            ob[(size_t)GR.ul * 64 + o] = __float2half_rn(u - __half2float(hi));
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int i4 = base + kPrepThreads * u;
+                if (i4 < n4) {
+                    const int r = (4 * i4) / p.dv, j = (4 * i4) % p.dv;
+                    const float x[4] = {vv[u].x * ww[u].x, vv[u].y * ww[u].y, vv[u].z * ww[u].z, vv[u].w * ww[u].w};
+                    __half hi[4], lo[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        hi[e] = __float2half_rn(x[e]);
+                        lo[e] = __float2half_rn(x[e] - __half2float(hi[e]));
+                    }
+                    const size_t o = (size_t)(64 * (j >> 6) + r) * 64 + (j & 63);
+                    *reinterpret_cast<__half2 *>(ob + (size_t)GR.u * 64 + o) = __halves2half2(hi[0], hi[1]);
+                    *reinterpret_cast<__half2 *>(ob + (size_t)GR.u * 64 + o + 2) = __halves2half2(hi[2], hi[3]);
+                    *reinterpret_cast<__half2 *>(ob + (size_t)GR.ul * 64 + o) = __halves2half2(lo[0], lo[1]);
+                    *reinterpret_cast<__half2 *>(ob + (size_t)GR.ul * 64 + o + 2) = __halves2half2(lo[2], lo[3]);
+                }
+            }
         }
     }
 }
@@ -662,7 +783,7 @@ cudaError_t launch_pair(const FwdParams &p, float *ws, cudaStream_t stream) {
         rho_local_kernel<<<dim3(NC, p.H, p.B), 128, 0, stream>>>(p, sums, pows);
         rho_combine_kernel<<<dim3(p.H, p.B), 128, 0, stream>>>(p, sums, pows, rho0);
     }
-    prep<<<dim3(NC, p.H, p.B), kThreads, pl.total, stream>>>(p, ws, rho0);
+    prep<<<dim3(NC, p.H, p.B), kPrepThreads, pl.total, stream>>>(p, ws, rho0);
     chain<<<dim3(p.slices, p.H, p.B), kThreads, cl.total, stream>>>(p, ws);
     return cudaGetLastError();
 }
@@ -707,7 +828,7 @@ cudaError_t launch_gen_prep(const FwdParams &p, void *workspace, cudaStream_t st
         rho_local_kernel<<<dim3(NC, p.H, p.B), 128, 0, stream>>>(p, sums, pows);
         rho_combine_kernel<<<dim3(p.H, p.B), 128, 0, stream>>>(p, sums, pows, rho0);
     }
-    prep<<<dim3(NC, p.H, p.B), kThreads, pl.total, stream>>>(p, ws, rho0);
+    prep<<<dim3(NC, p.H, p.B), kPrepThreads, pl.total, stream>>>(p, ws, rho0);
     return cudaGetLastError();
 }
 
