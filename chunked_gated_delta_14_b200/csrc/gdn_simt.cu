@@ -45,6 +45,7 @@
 #include <cuda_fp16.h>
 
 #include "gdn_internal.cuh"
+#include "gdn_tc_common.cuh"
 
 namespace gdn {
 namespace {
@@ -117,7 +118,7 @@ __host__ __device__ inline int key_stride(int dk, int elem_bytes) { return dk + 
 
 // Shared-memory carve-up of the prep kernel, identical on host and device.
 struct PrepLayout {
-    size_t kx, qx, ex, gx, tp, band, rows, total;
+    size_t kx, qx, ex, gx, tp, band, rows, inv, total;
 };
 
 __host__ __device__ inline PrepLayout prep_layout(int C, int dk, int N, int neumann, int general,
@@ -135,6 +136,8 @@ __host__ __device__ inline PrepLayout prep_layout(int C, int dk, int N, int neum
     L.tp = take((size_t)C * C * 4);
     L.band = neumann ? take((size_t)2 * C * (N + 1) * 4) : off;
     L.rows = take((size_t)4 * C * 4);        // g / log alpha, beta, lrow, spare
+    // chunk 64, exact: the blocked inverse's L and T (row stride LSTR) and scratch
+    L.inv = (C == 64 && !neumann) ? take((size_t)(2 * 64 * tc::LSTR + 1024) * 4) : off;
     L.total = off;
     return L;
 }
@@ -351,15 +354,40 @@ simt_prep_kernel(const FwdParams p, float *ws, const float *rho0) {
     // warp of the block has work and each chain is a quarter as long.  GX is G_r,
     // or G_{r-1} (shift 1, G_{-1} = 0).  store(r0, i0, acc) writes one tile.
     auto decayed_gram = [&](const float *X, int shift, auto &&store) {
-        const int nT = C / 4, tiles = nT * (nT + 1) / 2, items = ((4 * tiles + 31) / 32) * 32;
+        // tiles below the diagonal first (4 (nT (nT - 1) / 2) items, whole warps at
+        // C = 64), then the diagonal ones, so that no warp mixes the two forms
+        const int nT = C / 4, offd = nT * (nT - 1) / 2, tiles = offd + nT;
+        const int items = ((4 * tiles + 31) / 32) * 32;
         for (int w = tid; w < items; w += kPrepThreads) {
             const int part = w & 3, tix = w >> 2;
-            const bool need = tix < tiles;
-            int R = 0;
-            while ((R + 1) * (R + 2) / 2 <= tix) ++R;
-            const int r0 = 4 * R, i0 = 4 * (tix - R * (R + 1) / 2);
+            const bool need = tix < tiles, diag = tix >= offd;
+            int R = tix - offd, I = R;
+            if (!diag) {
+                R = 1;
+                while ((R + 1) * R / 2 <= tix) ++R;
+                I = tix - R * (R - 1) / 2;
+            }
+            const int r0 = 4 * R, i0 = 4 * I;
             float acc[4][4] = {};
-            if (need) {
+            if (need && !diag) {
+                // every row's exponent point lies after the tile's last key m = i0 + 3:
+                // 2^{GX_r - G_i} = 2^{GX_r - G_m} 2^{G_m - G_i}, both factors <= 1,
+                // 8 exponentials per 16 products
+                for (int cc = 0; cc < dk / 4; ++cc) {
+                    const int c = 4 * cc + part;
+                    const float gm = gx[(i0 + 3) * ks + c];
+                    float xr[4], yi[4];
+#pragma unroll
+                    for (int a = 0; a < 4; ++a) {
+                        xr[a] = X[(r0 + a) * ks + c] * fast_exp2(gx[(r0 + a - shift) * ks + c] - gm);
+                        yi[a] = ld_s(kx, (i0 + a) * ks + c) * fast_exp2(gm - gx[(i0 + a) * ks + c]);
+                    }
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) acc[a][e] += xr[a] * yi[e];
+                }
+            } else if (need) {
                 for (int cc = 0; cc < dk / 4; ++cc) {
                     const int c = 4 * cc + part;
                     float xr[4], gr[4], yi[4], gi[4];
@@ -426,7 +454,23 @@ simt_prep_kernel(const FwdParams p, float *ws, const float *rho0) {
     }
     __syncthreads();
     // ------------------------------------------------ T = (I + L)^-1
-    if (!neumann) {
+    if (!neumann && C == 64) {
+        // blocked: 16 x 16 diagonal blocks by forward substitution, merged
+        // 16 -> 32 -> 64 by T21 = -T22 L21 T11, by the first 256 threads
+        float *Lb = reinterpret_cast<float *>(smem + Ly.inv), *Tb = Lb + 64 * tc::LSTR, *Yb = Tb + 64 * tc::LSTR;
+        for (int idx = tid; idx < 64 * 64; idx += kPrepThreads) {
+            const int r = idx >> 6, c = idx & 63;
+            Lb[r * tc::LSTR + c] = tp[idx];
+            Tb[r * tc::LSTR + c] = 0.f;
+        }
+        __syncthreads();
+        if (tid < 256) tc::invert_exact(Lb, Tb, Yb, tid, 1);
+        __syncthreads();
+        for (int idx = tid; idx < 64 * 64; idx += kPrepThreads) {
+            const int r = idx >> 6, c = idx & 63;
+            tp[idx] = (c <= r) ? Tb[r * tc::LSTR + c] : 0.f;
+        }
+    } else if (!neumann) {
         // forward substitution, one row at a time: T_rc = -sum_{c<=i<r} L_ri T_ic
         for (int r = 1; r < C; ++r) {
             if (tid < r) lrow[tid] = tp[r * C + tid];
