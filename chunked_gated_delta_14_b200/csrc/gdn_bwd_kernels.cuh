@@ -73,6 +73,47 @@ __device__ __forceinline__ size_t tok_index(const BwdParams &p, int b, int t, in
     return ((size_t)b * p.T + t) * p.H + h;
 }
 
+// C rows of D values of [B, T, H, D] inputs (tokens t0.., head h; zero rows from
+// Cn on) into shared memory with row stride Dp, from one source (src1 null) or two
+// with the same shape.  Four consecutive values per item, and four items' loads
+// in flight before the first store: the loads' latencies overlap.
+template <int NT>
+__device__ __forceinline__ void load_rows(const BwdParams &p, int b, int h, int t0, int C, int Cn, int D, int Dp,
+                                          const void *src0, int bf0, float *dst0, const void *src1, int bf1,
+                                          float *dst1, int tid) {
+    constexpr int UNR = 4;
+    const int n4 = C * D / 4;
+    for (int base = tid; base < n4; base += NT * UNR) {
+        float4 v0[UNR], v1[UNR];
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+            const int i4 = base + NT * u;
+            v0[u] = v1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i4 < n4) {
+                const int r = (4 * i4) / D, c = (4 * i4) % D;
+                if (r < Cn) {
+                    const size_t gi = tok_index(p, b, t0 + r, h) * D + c;
+                    v0[u] = ld4_in(src0, gi, bf0);
+                    if (src1) v1[u] = ld4_in(src1, gi, bf1);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+            const int i4 = base + NT * u;
+            if (i4 < n4) {
+                const int r = (4 * i4) / D, c = (4 * i4) % D;
+                float *d0 = dst0 + r * Dp + c;
+                d0[0] = v0[u].x; d0[1] = v0[u].y; d0[2] = v0[u].z; d0[3] = v0[u].w;
+                if (src1) {
+                    float *d1 = dst1 + r * Dp + c;
+                    d1[0] = v1[u].x; d1[1] = v1[u].y; d1[2] = v1[u].z; d1[3] = v1[u].w;
+                }
+            }
+        }
+    }
+}
+
 // out[r][c] = sum_{i < nterm} A(r, i) scale[i] X[i][c] for r < nrow, c < n, with
 // A(r, i) = A[r * ra + i * ia] in shared memory (so A or its transpose) and
 // scale null meaning 1; written to global memory row-major.  With half = n / 2
@@ -139,21 +180,8 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(const BwdParams 
     float *eg = bg + C;
     const size_t ch = ((size_t)b * p.H + h) * p.NC + n;
 
-    for (int x = tid; x < C * dk; x += kPrepThreads) {
-        const int r = x / dk, c = x % dk;
-        float kv = 0.f, qv = 0.f;
-        if (r < Cn) {
-            const size_t ti = tok_index(p, b, t0 + r, h) * dk + c;
-            kv = ld_in(p.k, ti, p.io_bf16);
-            qv = ld_in(p.q, ti, p.io_bf16);
-        }
-        Ks[r * dkp + c] = kv;
-        Qs[r * dkp + c] = qv;
-    }
-    for (int x = tid; x < C * dv; x += kPrepThreads) {
-        const int r = x / dv, j = x % dv;
-        Vs[r * dvp + j] = r < Cn ? ld_in(p.v, tok_index(p, b, t0 + r, h) * dv + j, p.io_bf16) : 0.f;
-    }
+    load_rows<kPrepThreads>(p, b, h, t0, C, Cn, dk, dkp, p.k, p.io_bf16, Ks, p.q, p.io_bf16, Qs, tid);
+    load_rows<kPrepThreads>(p, b, h, t0, C, Cn, dv, dvp, p.v, p.io_bf16, Vs, nullptr, 0, nullptr, tid);
     for (int x = tid; x < C * C; x += kPrepThreads) Ts[(x / C) * Cp + x % C] = 0.f;
     // gates: every token's log alpha and beta in parallel, then the in-chunk scan
     if (tid < C) {
@@ -243,10 +271,7 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(const BwdParams 
                                                            tid);
     __syncthreads();   // V consumed: its buffer takes dO
     float *dOs = Vs;
-    for (int x = tid; x < C * dv; x += kPrepThreads) {
-        const int r = x / dv, j = x % dv;
-        dOs[r * dvp + j] = r < Cn ? ld_in(p.grad_o, tok_index(p, b, t0 + r, h) * dv + j, p.do_bf16) : 0.f;
-    }
+    load_rows<kPrepThreads>(p, b, h, t0, C, Cn, dv, dvp, p.grad_o, p.do_bf16, dOs, nullptr, 0, nullptr, tid);
     __syncthreads();
     // the state-independent parts of the reverse chain: M^T dO (C x dv) and
     // (diag(e^g) Q)^T dO (dk x dv)
@@ -566,17 +591,7 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
     float *rowv = part + 32 * kMaxC;     // [10][kMaxC]
     const size_t ch = ((size_t)b * p.H + h) * p.NC + n;
 
-    for (int x = tid; x < C * DK; x += kThreads) {
-        const int r2 = x / DK, c = x % DK;
-        float kv = 0.f, qv = 0.f;
-        if (r2 < Cn) {
-            const size_t ti = tok_index(p, b, t0 + r2, h) * DK + c;
-            kv = ld_in(p.k, ti, p.io_bf16);
-            qv = ld_in(p.q, ti, p.io_bf16);
-        }
-        Ks[r2 * dkp + c] = kv;
-        Qs[r2 * dkp + c] = qv;
-    }
+    load_rows<kThreads>(p, b, h, t0, C, Cn, DK, dkp, p.k, p.io_bf16, Ks, p.q, p.io_bf16, Qs, tid);
     for (int x = tid; x < C * Cp; x += kThreads) {
         dMs[x] = 0.f;
         dLs[x] = 0.f;
@@ -595,25 +610,56 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
 
     for (int j0 = 0; j0 < dv; j0 += kCols) {
         __syncthreads();   // previous tile consumed (and, first time, the set-up above)
-        for (int x = tid; x < DK * kCols; x += kThreads) {
-            const int c = x / kCols, jj = x % kCols;
-            ht[c * 33 + jj] = p.ws_h[(ch * DK + c) * dv + j0 + jj];
-            dht[c * 33 + jj] = p.ws_dh[(ch * DK + c) * dv + j0 + jj];
-        }
-        for (int x = tid; x < C * kCols; x += kThreads) {
-            const int r2 = x / kCols, jj = x % kCols;
-            float a = 0.f, y = 0.f, d = 0.f, v = 0.f;
-            if (r2 < Cn) {
-                const size_t ti = tok_index(p, b, t0 + r2, h) * dv + j0 + jj;
-                a = ld_in(p.grad_o, ti, p.do_bf16);
-                v = ld_in(p.v, ti, p.io_bf16);
-                y = p.ws_Y[(ch * C + r2) * dv + j0 + jj];
-                d = p.ws_D[(ch * C + r2) * dv + j0 + jj];
+        // the tile's inputs four values at a time, every load of a pass issued
+        // before its first store
+        {
+            constexpr int NH = DK * (kCols / 4);                      // float4 items (h, dh)
+            constexpr int HQ = (NH + kThreads - 1) / kThreads;        // per thread
+            float4 hv[HQ], dhv[HQ];
+#pragma unroll
+            for (int u = 0; u < HQ; ++u) {
+                const int x = tid + kThreads * u, c = x / (kCols / 4), q4 = x % (kCols / 4);
+                if (x < NH) {
+                    const size_t o = (ch * DK + c) * dv + j0 + 4 * q4;
+                    hv[u] = *reinterpret_cast<const float4 *>(p.ws_h + o);
+                    dhv[u] = *reinterpret_cast<const float4 *>(p.ws_dh + o);
+                }
             }
-            dOt[r2 * 33 + jj] = a;
-            Yt[r2 * 33 + jj] = y;
-            Dt[r2 * 33 + jj] = d;
-            Vt[r2 * 33 + jj] = v;
+#pragma unroll
+            for (int u = 0; u < HQ; ++u) {
+                const int x = tid + kThreads * u, c = x / (kCols / 4), q4 = x % (kCols / 4);
+                if (x < NH) {
+                    float *hd = ht + c * 33 + 4 * q4, *dd = dht + c * 33 + 4 * q4;
+                    hd[0] = hv[u].x; hd[1] = hv[u].y; hd[2] = hv[u].z; hd[3] = hv[u].w;
+                    dd[0] = dhv[u].x; dd[1] = dhv[u].y; dd[2] = dhv[u].z; dd[3] = dhv[u].w;
+                }
+            }
+        }
+        for (int base = tid; base < C * (kCols / 4); base += 2 * kThreads) {
+            float4 a4[2], v4[2], y4[2], d4[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int x = base + kThreads * u, r2 = x / (kCols / 4), q4 = x % (kCols / 4);
+                a4[u] = v4[u] = y4[u] = d4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (x < C * (kCols / 4) && r2 < Cn) {
+                    const size_t ti = tok_index(p, b, t0 + r2, h) * dv + j0 + 4 * q4;
+                    a4[u] = ld4_in(p.grad_o, ti, p.do_bf16);
+                    v4[u] = ld4_in(p.v, ti, p.io_bf16);
+                    y4[u] = *reinterpret_cast<const float4 *>(p.ws_Y + (ch * C + r2) * dv + j0 + 4 * q4);
+                    d4[u] = *reinterpret_cast<const float4 *>(p.ws_D + (ch * C + r2) * dv + j0 + 4 * q4);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int x = base + kThreads * u, r2 = x / (kCols / 4), q4 = x % (kCols / 4);
+                if (x < C * (kCols / 4)) {
+                    const int o = r2 * 33 + 4 * q4;
+                    dOt[o] = a4[u].x; dOt[o + 1] = a4[u].y; dOt[o + 2] = a4[u].z; dOt[o + 3] = a4[u].w;
+                    Vt[o] = v4[u].x; Vt[o + 1] = v4[u].y; Vt[o + 2] = v4[u].z; Vt[o + 3] = v4[u].w;
+                    Yt[o] = y4[u].x; Yt[o + 1] = y4[u].y; Yt[o + 2] = y4[u].z; Yt[o + 3] = y4[u].w;
+                    Dt[o] = d4[u].x; Dt[o + 1] = d4[u].y; Dt[o + 2] = d4[u].z; Dt[o + 3] = d4[u].w;
+                }
+            }
         }
         __syncthreads();
         if (v0) {   // tile rows at and past Cn are zero, so row r1 needs no test here

@@ -17,6 +17,7 @@
 
 struct dim3h { unsigned x, y, z; };
 struct float4 { float x, y, z, w; };
+inline float4 make_float4(float x, float y, float z, float w) { return float4{x, y, z, w}; }
 inline thread_local dim3h threadIdx;
 inline dim3h blockIdx;
 #define __global__
