@@ -51,7 +51,11 @@
  * between the two CTAs of a cluster through shared memory.  The split
  * tensor-core kernels (GDN_KERNEL_TC_SPLIT) keep, per chunk and head,
  * T diag(beta), T diag(beta e^g) and the decayed causal scores P (fp16,
- * 24 KB) in the workspace between their two launches.  The SIMT kernels
+ * 24 KB) in the workspace between their two launches; at C = 128 also, per
+ * second 64-token half, the band corner's two parts (16 (dk + dv) fp32); for
+ * the two-gate rule instead the prep's operands as fp16 rows (TB, P, U as
+ * hi + lo pairs, E, Q', K'', the decay; (640 + 2 dv + 4) x 128 B) and the
+ * preconditioner's running averages.  The SIMT kernels
  * (GDN_KERNEL_SIMT) keep, per chunk and head, the state-independent fp32
  * matrices of the chunk (T diag(beta), the decayed scores, the decayed keys
  * and queries, 2 C^2 + 3 C dk + dk floats) and, for the preconditioned
@@ -120,9 +124,18 @@ typedef enum {
                                    AUTO picks it for T <= 8 */
     GDN_KERNEL_TC_SPLIT = 4     /* the tensor-core path as two launches (a key-side kernel
                                    per chunk, then the state chain) with the per-chunk
-                                   inverses in a caller workspace: bf16 q/k/v, scalar decay,
-                                   C = 64, dk = 128, dv a multiple of 64, all three inverse
-                                   modes (Neumann N <= 15) */
+                                   inverses in a caller workspace: bf16 q/k/v, dk = 128,
+                                   dv a multiple of 64, and
+                                   - the scalar rule at C = 64, all three inverse modes
+                                     (Neumann N <= 15);
+                                   - the scalar rule at C = 128 with the masked series
+                                     (N <= 15): each 128-token chunk as two 64-token
+                                     halves plus the band's corner (a third launch);
+                                   - the two-gate rule at C = 64, exact or Neumann, with
+                                     preconditioner form 0 or 1: the SIMT kernels' prep
+                                     writes fp16 operands for the tensor-core chain
+                                     (the preconditioner's running-average kernels
+                                     first, when it is on) */
 } gdn_kernel;
 
 typedef struct {
@@ -288,10 +301,11 @@ GDN_API uint64_t gdn_bwd_workspace_bytes(const gdn_bwd_args *args);
  * args->workspace_bytes 0; args->kernel must be AUTO, TC or TC_SPLIT and the
  * shape one the split tensor-core kernels support, else GDN_ERR_UNSUPPORTED
  * (whatever the kernel field, this entry point runs the split kernels); and
- * B * H * ceil(T / 64) * 24576 must be <= GDN_STATIC_SCRATCH_BYTES, else
- * GDN_ERR_INVALID_ARG with the needed size in gdn_last_error().  Nothing in
- * the scratch has to start at zero: the key-side kernel writes every entry
- * the chain kernel reads, in the same call.
+ * the workspace the call needs there (gdn_workspace_bytes with kernel
+ * TC_SPLIT: B * H * ceil(T / 64) * 24576 for the scalar rule at C = 64) must
+ * be <= GDN_STATIC_SCRATCH_BYTES, else GDN_ERR_INVALID_ARG with the needed
+ * size in gdn_last_error().  Nothing in the scratch has to start at zero: the
+ * call's first kernels write every entry the chain kernel reads.
  *
  * Set-up: the first call on each device, with that device current, looks up
  * the array's address with cudaGetSymbolAddress (an error there returns
