@@ -91,12 +91,14 @@ def test_neumann_sweep(chunk, N):
 
 @needs_cuda
 @pytest.mark.parametrize("T,N,s0", [(1000, 15, 0.02), (900, 1, 0.0), (129, 7, 0.02), (640, 0, 0.02),
-                                    (4096, 3, 0.02)])
+                                    (4096, 3, 0.02), (64, 3, 0.02), (65, 2, 0.02), (128, 15, 0.0)])
 def test_neumann_chunk128_halves_ragged(T, N, s0):
     """Chunk 128 of the masked series on the split tensor-core kernels: each
     128-token chunk runs as two 64-token halves plus the band's corner between
-    them.  Ragged ends (a partial second half; a lone first half), the widest band
-    (N = 15), N = 0 (T = I: no corner) and a nonzero initial state."""
+    them.  Ragged ends (a partial second half; a lone first half), a sequence of one
+    half (T = 64: no corner launch), a one-token second half (T = 65), exactly one
+    128-token chunk, the widest band (N = 15), N = 0 (T = I: no corner) and a
+    nonzero initial state."""
     w = workload("neumann", B=2, H=2, T=T, chunk=128, neumann_N=N, s0_std=s0)
     x = make_inputs(w, seed=40 + N)
     o_ref, s_ref = run_oracle(x, w)
@@ -209,10 +211,12 @@ def test_precond_two_gate_full_size(kernel):
 
 
 @needs_cuda
-@pytest.mark.parametrize("T,s0,dv", [(1000, 0.02, 128), (4096, 0.0, 64), (65, 0.02, 128)])
+@pytest.mark.parametrize("T,s0,dv", [(1000, 0.02, 128), (4096, 0.0, 64), (65, 0.02, 128), (1, 0.02, 128),
+                                     (64, 0.0, 64)])
 def test_precond_two_gate_tensor_cores(T, s0, dv):
     """The two-gate rule on the tensor-core chain: ragged tails (a one-token last
-    chunk), an initial state, d_v 64 (one value slice), against the oracle."""
+    chunk), a single token, one full chunk, an initial state, d_v 64 (one value
+    slice), against the oracle."""
     w = workload("precond_two_gate", B=2, H=2, T=T, s0_std=s0, dv=dv)
     x = make_inputs(w, seed=30 + T)
     o_ref, s_ref = run_oracle(x, w)
