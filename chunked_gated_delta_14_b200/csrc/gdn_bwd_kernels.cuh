@@ -219,12 +219,15 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(const BwdParams 
         float gk[KR], qk[KR];
 #pragma unroll
         for (int k = 0; k < KR; ++k) gk[k] = qk[k] = 0.f;
+        // every (r, i) pair of the chunk accumulates; the ones outside the lower
+        // triangle or the sequence are dropped when written (no divergent branch in
+        // the loop at C >= 32; the rows it reads past the tail are the zero rows)
         for (int c = 0; c < dk; ++c) {
             const float ki = Ks[i * dkp + c];
 #pragma unroll
             for (int k = 0; k < KR; ++k) {
                 const int r = tid / C + rstep * k;
-                if (k < nk && r < Cn && i <= r) {
+                if (k < nk && r < C) {
                     gk[k] += Ks[r * dkp + c] * ki;
                     qk[k] += Qs[r * dkp + c] * ki;
                 }
