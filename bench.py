@@ -300,14 +300,15 @@ def serial_e2e(host_in, run, steps, dev, warm=2, barrier=None):
     return e0.elapsed_time(e1) / steps, nbytes["h2d"], nbytes["d2h"]
 
 
-def measure_e2e(host_in, run, steps, dev, barrier=None):
+def measure_e2e(host_in, run, steps, dev):
     """pipelined_e2e, or serial_e2e if the pipelined form raises; returns
-    (ms per step, h2d bytes, d2h bytes, description)."""
+    (ms per step, h2d bytes, d2h bytes, description).  Single-process runs only:
+    a fallback taken by one rank alone would desynchronise the ranks' collectives."""
     try:
-        ms, h2d, d2h = pipelined_e2e(host_in, run, steps, dev, barrier=barrier)
+        ms, h2d, d2h = pipelined_e2e(host_in, run, steps, dev)
         return ms, h2d, d2h, "uploads, compute and readbacks on three streams, two input slots"
     except Exception as e:   # keep the line: time the steps on one stream instead
-        ms, h2d, d2h = serial_e2e(host_in, run, steps, dev, barrier=barrier)
+        ms, h2d, d2h = serial_e2e(host_in, run, steps, dev)
         return ms, h2d, d2h, f"one stream (pipelined form failed: {type(e).__name__}: {e})"
 
 
@@ -881,8 +882,12 @@ def run_bwd(args, rank, world, local_rank):
             return {k: r[k] for k in ("dq", "dk", "dv", "dalpha", "dbeta")}
 
         n_e2e = max(1, args.e2e_steps // 4)
-        ems, h2d, d2h, how = measure_e2e(host, run, n_e2e, dev,
-                                         barrier=dist.barrier if world > 1 else None)
+        if world > 1:
+            # every rank takes the same collective steps: no fallback that one rank alone could take
+            ems, h2d, d2h = pipelined_e2e(host, run, n_e2e, dev, barrier=dist.barrier)
+            how = "uploads, compute and readbacks on three streams, two input slots"
+        else:
+            ems, h2d, d2h, how = measure_e2e(host, run, n_e2e, dev)
         ems = max_over_ranks(ems, world, dev)
         e2e = dict(value=job_throughput(tokens_step, world, 1, ems), unit=UNIT,
                    h2d_bytes_per_step=int(h2d), d2h_bytes_per_step=int(d2h), ms_per_step=ems,
