@@ -400,7 +400,8 @@ def forward_line(args, rank, world, local_rank, name, over, timed_steps):
                       beta=ptr(d["beta"]), erase=ptr(d["erase"]), write=ptr(d["write"]),
                       precond=int(bool(w.precond)), S0=ptr(d["S0"]), o=o.data_ptr(),
                       S_T=S_T.data_ptr(), mode={"exact": 0, "neumann": 1, "residual": 2}[mode],
-                      neumann_N=N, residual_S=args.S, kernel=gdn.gdn.KERNELS[args.kernel])
+                      neumann_N=N, residual_S=args.S, kernel=gdn.gdn.KERNELS[args.kernel],
+                      seq_segments=getattr(args, "segments", 0))
     ws = gdn.workspace_for(a, dev)
     if ws is not None:
         a.workspace = ws.data_ptr()
@@ -420,6 +421,11 @@ def forward_line(args, rank, world, local_rank, name, over, timed_steps):
         kernel_name = "simt_prep_kernel+chain_kernel"
     scans = 2 if (w.precond and general) else 0    # the preconditioner's running-average kernels
     launches_per_call = {4: 3 if pair else 2 + scans, 1: 2 + scans}.get(kernel_id, 1)
+    segments = gdn.select_segments(a) if kernel_id == 4 else 1
+    if segments == 3:
+        # three key-side launches, five chain runs (two passes), the identity and the composition
+        launches_per_call = 10
+        kernel_name += "+seg_identity_kernel+seg_compose_kernel (3 sequence segments)"
     sh = stream.cuda_stream
 
     def step():
@@ -480,6 +486,7 @@ def forward_line(args, rank, world, local_rank, name, over, timed_steps):
             gdn.chunk_fwd(di["q"], di["k"], di["v"], di.get("alpha"), di.get("beta"), erase=di.get("erase"),
                           write=di.get("write"), precond=int(bool(w.precond)), S0=di.get("S0"), chunk=w.chunk,
                           o_dtype=o_dt, out=outs[slot], mode=mode, N=N, S=args.S, S_T=finals[slot],
+                          segments=getattr(args, "segments", 0),
                           kernel=args.kernel)
             return {"o": outs[slot], "S_T": finals[slot]}
 
@@ -1038,6 +1045,8 @@ def main():
                     help="the backward pass (gradients) on the same workload")
     ap.add_argument("--bwd-steps", type=int, default=20,
                     help="backward calls timed for the forward line's 'backward' object (0: none)")
+    ap.add_argument("--segments", type=int, default=0, choices=[0, 1, 3],
+                    help="sequence segments of the split tensor-core path (0: the library's choice)")
     ap.add_argument("--kernel", default="auto", choices=["auto", "simt", "tc", "tc_split"],
                     help="force one forward kernel (auto: the library's choice)")
     ap.add_argument("--chunk", type=int, default=0,

@@ -8,9 +8,9 @@ the benchmark.  Build the library with
 from .gdn import (GDNError, BwdArgs, FwdArgs, GatedDeltaRule, abi_version,  # noqa: F401
                   bwd_workspace_bytes, call, call_bwd, chunk_bwd, chunk_fwd, clear_workspace_cache,
                   debug_chunk_T, device_check,
-                  gated_delta_rule, last_error, lib, make_args, make_bwd_args, select_kernel,
+                  gated_delta_rule, last_error, lib, make_args, make_bwd_args, select_kernel, select_segments,
                   status_string, workspace_bytes, workspace_for)
 
 __all__ = ["chunk_fwd", "chunk_bwd", "gated_delta_rule", "GatedDeltaRule", "BwdArgs",
-           "make_bwd_args", "call_bwd", "bwd_workspace_bytes", "device_check", "workspace_bytes", "workspace_for", "GDNError", "FwdArgs", "make_args", "call", "select_kernel",
+           "make_bwd_args", "call_bwd", "bwd_workspace_bytes", "device_check", "workspace_bytes", "workspace_for", "GDNError", "FwdArgs", "make_args", "call", "select_kernel", "select_segments",
            "abi_version", "last_error", "status_string", "lib", "debug_chunk_T", "clear_workspace_cache"]

@@ -82,6 +82,8 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
         return fail(GDN_ERR_INVALID_ARG, "kernel %d unknown", a->kernel);
     if (a->dv_split < 0 || (a->dv_split > 0 && (a->dv % a->dv_split != 0 || a->dv / a->dv_split < 16)))
         return fail(GDN_ERR_INVALID_ARG, "dv_split must divide dv into slices of >= 16 columns");
+    if (a->seq_segments != 0 && a->seq_segments != 1 && a->seq_segments != 3)
+        return fail(GDN_ERR_INVALID_ARG, "seq_segments must be 0, 1 or 3 (got %d)", a->seq_segments);
 
     gdn::FwdParams p{};
     p.B = a->B; p.T = a->T; p.H = a->H; p.dk = a->dk; p.dv = a->dv; p.C = a->chunk;
@@ -112,6 +114,9 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
         }
         if (kern == GDN_KERNEL_SIMT && a->dv_split <= 1 && gdn::fused_supports(p, &why)) kern = GDN_KERNEL_TC;
     }
+    p.segments = 1;
+    if (a->seq_segments == 3 && kern != GDN_KERNEL_TC_SPLIT)
+        return fail(GDN_ERR_UNSUPPORTED, "seq_segments 3 runs on the split tensor-core kernels only");
     if (kern == GDN_KERNEL_RECURRENT) {
         if (!gdn::recurrent_supports(p, &why))
             return fail(GDN_ERR_UNSUPPORTED, "recurrent kernel: %s", why);
@@ -131,6 +136,9 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
         p.dvs = p.dv / p.slices;
         if (!gdn::tc_supports(p, &why))
             return fail(GDN_ERR_UNSUPPORTED, "split tensor-core kernels: %s", why);
+        if (a->seq_segments == 3 && !gdn::tc_segments_support(p, &why))
+            return fail(GDN_ERR_UNSUPPORTED, "split tensor-core kernels: %s", why);
+        p.segments = a->seq_segments ? a->seq_segments : gdn::tc_auto_segments(p);
     } else {
         if (p.mode == GDN_INV_NEUMANN_RESIDUAL)
             return fail(GDN_ERR_UNSUPPORTED,
@@ -269,6 +277,15 @@ int32_t gdn_select_kernel(const gdn_fwd_args *args) {
     return kern;
 }
 
+int32_t gdn_select_segments(const gdn_fwd_args *args) {
+    gdn::FwdParams p;
+    int kern = 0;
+    gdn_status s = resolve(args, &p, &kern);
+    if (s != GDN_OK) return -(int32_t)s;
+    g_msg[0] = 0;
+    return p.segments;
+}
+
 gdn_status gdn_device_check(void *stream) {
     cudaError_t e = cudaSuccess;
     const unsigned int code = gdn::tc_read_and_clear_error(reinterpret_cast<cudaStream_t>(stream), &e);
@@ -332,6 +349,7 @@ gdn_status gdn_chunk_fwd_static_scratch(const gdn_fwd_args *args, void *stream) 
     if (s != GDN_OK) return s;
     if (args->workspace || args->workspace_bytes)
         return fail(GDN_ERR_INVALID_ARG, "the fixed-scratch entry point takes no workspace (pass NULL, 0)");
+    p.segments = 1;     // one pass: the segment schedule's streams and states are not for this entry
     const size_t need = gdn::tc_workspace_bytes(p);
     if (need > (size_t)GDN_STATIC_SCRATCH_BYTES)
         return fail(GDN_ERR_INVALID_ARG,

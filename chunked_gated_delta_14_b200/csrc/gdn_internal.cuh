@@ -29,6 +29,7 @@ struct FwdParams {
     int mode, N;
     int S;              // residual-correction terms (GDN_INV_NEUMANN_RESIDUAL)
     int general;        // two-gate rule (per-channel decay / gates / preconditioner)
+    int segments;       // split tensor-core path: 1 one pass, 3 three sequence segments
 };
 
 // SIMT fp32 chunk kernel: shared-memory bytes for p, or 0 if p does not fit.
@@ -68,6 +69,10 @@ cudaError_t launch_gen_prep(const FwdParams &p, void *workspace, cudaStream_t st
 bool tc_supports(const FwdParams &p, const char **why);
 int tc_default_slices(const FwdParams &p);
 size_t tc_workspace_bytes(const FwdParams &p);
+// Sequence segments of the split path (B = 1, scalar rule, chunk 64): whether p
+// allows them, and the count chosen when the caller leaves it to the library.
+bool tc_segments_support(const FwdParams &p, const char **why);
+int tc_auto_segments(const FwdParams &p);
 cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, const char **why);
 // Synchronise `stream`, return (and clear) the tensor-core kernel's error word.
 unsigned int tc_read_and_clear_error(cudaStream_t stream, cudaError_t *err);

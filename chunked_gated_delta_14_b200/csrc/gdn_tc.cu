@@ -44,6 +44,8 @@
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "gdn_internal.cuh"
 #include "gdn_tc_common.cuh"
 
@@ -65,6 +67,8 @@ using tc::unpack_bf2;
 using tc::unpack_h2;
 
 constexpr int DVS = 64;            // value columns per chain CTA
+constexpr int kSMs = 148;          // B200
+constexpr int kSegAutoMinChunks = 256;   // sequence segments by default from 16384 tokens
 constexpr int kNeumannMaxN = 15;
 constexpr unsigned long long kWaitLimit = 4000000000ull;   // ~2 s at the boost clock
 
@@ -670,9 +674,10 @@ struct K2Params {
     const float *pair_ws;   // PAIR: C2' and C1 V_a of every second half
     const uint8_t *gen_ws;  // GEN: the prep's rows (gen_rows), ws_rows per chunk-head
     int ws_rows;            // rows of 128 B per chunk-head in the workspace map
-    void *o;
+    void *o;                // nullptr: the outputs are not stored (a state-only run)
     float *S_T;
     int o_bf16;
+    int v_zero;             // PLAIN: V = 0 (no V loads), the state map's linear part
 };
 
 template <int MODE>
@@ -755,6 +760,12 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         tmem_alloc(tmem_slot, TM_COLS);
         tmem_relinquish();
     }
+    if (!PAIR && !GEN && p.v_zero) {
+        // V = 0: the V tile is never loaded; its in-place conversion keeps zeros
+        uint4 *z = reinterpret_cast<uint4 *>(sm + OFF_EARLY + ES_V);
+        for (int i = tid; i < 8192 / 16; i += K2_THREADS) z[i] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
     block_sync();
     tc_fence_after();
@@ -814,8 +825,8 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                     tma_load_4d(es + ES_E, &tm_t, eb, 0, 0, wrow + G.e, 0);
                     tma_load_4d(es + ES_E + 8192, &tm_t, eb, 0, 0, wrow + G.e + 64, 0);
                 } else {
-                    mbar_arrive_expect_tx(eb, EARLY_TX + (second ? 8192u + 4096u : 0u));
-                    tma_load_4d(es + ES_V, &tm_v, eb, v0, h, t0, b);
+                    mbar_arrive_expect_tx(eb, EARLY_TX - (p.v_zero ? 8192u : 0u) + (second ? 8192u + 4096u : 0u));
+                    if (!p.v_zero) tma_load_4d(es + ES_V, &tm_v, eb, v0, h, t0, b);
                     tma_load_4d(es + ES_TB, &tm_t, eb, 0, 0, wrow, 0);
                     tma_load_4d(es + ES_TBG, &tm_t, eb, 0, 0, wrow + 64, 0);
                 }
@@ -1125,7 +1136,7 @@ chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             float x[64];
             tmem_ld64(tmem + lane_base + ((n & 1) ? TM_X1 : TM_X0), x);
             const int t = n * C + r;
-            if (t < T) {
+            if (t < T && p.o) {
                 const size_t go = (((size_t)b * T + t) * H + h) * dv + v0;
                 if (p.o_bf16) {
                     __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(p.o) + go;
@@ -1366,6 +1377,205 @@ bool make_map_t(CUtensorMap *m, const void *ptr, size_t rows) {
     return r == CUDA_SUCCESS;
 }
 
+
+// ------------------------------------------------- sequence segments (B = 1)
+//
+// The recurrence is affine in the state: over any run of tokens the final h is
+// M h_start + N, M (d_k x d_k) the run's product of transitions and N its final
+// state from h_start = 0.  A long sequence is cut into three segments s0, s1,
+// s2.  Pass 1 runs s0 from S0, s1 from 0 (-> N) and s1 with V = 0 from the
+// identity (-> M) side by side; then h(s2 start) = M h(s1 start) + N; pass 2
+// runs s1 and s2 from their true starts.  Two chain passes of a third of the
+// chunks each, instead of one pass over all of them, when the per-head chains
+// alone cannot fill the SMs.
+
+// h = S^T of every head set to the identity (d_k x d_k): the start of M's run.
+__global__ void seg_identity_kernel(float *I, int dk) {
+    const int h = blockIdx.y, r = blockIdx.x;
+    for (int c = threadIdx.x; c < dk; c += blockDim.x) I[((size_t)h * dk + r) * dk + c] = r == c ? 1.f : 0.f;
+}
+
+// out = M h1 + N per head: M [H, dk, dk], h1, N, out [H, dk, dv]; one block per
+// (row, head), one thread per value column.
+__global__ void seg_compose_kernel(const float *M, const float *h1, const float *N, float *out, int dk, int dv) {
+    __shared__ float mr[DK];
+    const int h = blockIdx.y, r = blockIdx.x;
+    for (int i = threadIdx.x; i < dk; i += blockDim.x) mr[i] = M[((size_t)h * dk + r) * dk + i];
+    __syncthreads();
+    const float *hh = h1 + (size_t)h * dk * dv;
+    for (int c = threadIdx.x; c < dv; c += blockDim.x) {
+        float acc = N[((size_t)h * dk + r) * dv + c];
+        for (int i = 0; i < dk; ++i) acc = fmaf(mr[i], hh[(size_t)i * dv + c], acc);
+        out[((size_t)h * dk + r) * dv + c] = acc;
+    }
+}
+
+// The key-side kernel over p's tokens, T matrices into ws.
+cudaError_t launch_k1_plain(const FwdParams &p, void *ws, cudaStream_t stream) {
+    CUtensorMap mq, mk;
+    if (!make_map_bthd(&mq, p.q, p.B, p.T, p.H, p.dk) || !make_map_bthd(&mk, p.k, p.B, p.T, p.H, p.dk))
+        return cudaErrorInvalidValue;
+    const int NC = (p.T + C - 1) / C;
+    K1Params k1;
+    k1.B = p.B; k1.T = p.T; k1.H = p.H; k1.NC = NC;
+    k1.alpha = p.alpha; k1.beta = p.beta;
+    k1.ws = reinterpret_cast<uint8_t *>(ws);
+    k1.neumann = p.mode == GDN_INV_NEUMANN ? 1 : (p.mode == GDN_INV_NEUMANN_RESIDUAL ? 2 : 0);
+    k1.N = p.N; k1.S = p.S;
+    keyside_kernel<<<dim3(NC, p.H, p.B), K1_THREADS, k1.neumann == 2 ? K1_SMEM_RES : K1_SMEM, stream>>>(mq, mk, k1);
+    return cudaGetLastError();
+}
+
+// The chain kernel (chunk 64) over p's tokens, reading the T matrices from ws;
+// p.v == nullptr runs it with V = 0.
+cudaError_t launch_k2_plain(const FwdParams &p, const void *ws, cudaStream_t stream) {
+    CUtensorMap mq, mk, mv, mt;
+    const int NC = (p.T + C - 1) / C;
+    if (!make_map_bthd(&mq, p.q, p.B, p.T, p.H, p.dk) || !make_map_bthd(&mk, p.k, p.B, p.T, p.H, p.dk) ||
+        !make_map_t(&mt, ws, (size_t)p.B * p.H * NC * WS_ROWS))
+        return cudaErrorInvalidValue;
+    if (p.v) {
+        if (!make_map_bthd(&mv, p.v, p.B, p.T, p.H, p.dv)) return cudaErrorInvalidValue;
+    } else {
+        mv = mq;    // never read: the kernel loads no V
+    }
+    K2Params k2{};
+    k2.ws_rows = WS_ROWS;
+    k2.B = p.B; k2.T = p.T; k2.H = p.H; k2.dv = p.dv; k2.NC = NC;
+    k2.alpha = p.alpha; k2.beta = p.beta; k2.S0 = p.S0; k2.o = p.o; k2.S_T = p.S_T;
+    k2.o_bf16 = p.o_bf16;
+    k2.v_zero = p.v ? 0 : 1;
+    chain_kernel<K2_PLAIN><<<dim3(p.dv / DVS, p.H, p.B), K2_THREADS, K2Layout<K2_PLAIN>::SMEM, stream>>>(mq, mk, mv, mt,
+                                                                                                  k2);
+    return cudaGetLastError();
+}
+
+// Streams and events of the segment schedule, one set per device, made on first
+// use with that device current.  The chain runs go to high-priority streams so
+// that their blocks are placed ahead of the key-side blocks running beside them.
+struct SegStreams {
+    bool ready = false;
+    cudaStream_t run[3] = {};
+    cudaStream_t side = nullptr;
+    cudaEvent_t ev[8] = {};
+};
+constexpr int kSegMaxDevices = 64;
+SegStreams g_seg[kSegMaxDevices];
+std::mutex g_seg_mu;
+
+cudaError_t seg_streams(int dev, SegStreams **out) {
+    SegStreams &S = g_seg[dev];
+    if (!S.ready) {
+        int lo = 0, hi = 0;
+        cudaError_t e = cudaDeviceGetStreamPriorityRange(&lo, &hi);
+        if (e != cudaSuccess) return e;
+        for (auto &r : S.run)
+            if ((e = cudaStreamCreateWithPriority(&r, cudaStreamNonBlocking, hi)) != cudaSuccess) return e;
+        if ((e = cudaStreamCreateWithPriority(&S.side, cudaStreamNonBlocking, lo)) != cudaSuccess) return e;
+        for (auto &v : S.ev)
+            if ((e = cudaEventCreateWithFlags(&v, cudaEventDisableTiming)) != cudaSuccess) return e;
+        S.ready = true;
+    }
+    *out = &S;
+    return cudaSuccess;
+}
+
+// p with its token range cut to [t0, t0 + T) (B = 1: every [B, T, H, *] tensor
+// is contiguous in t).
+FwdParams seg_view(const FwdParams &p, int t0, int T) {
+    FwdParams s = p;
+    const size_t r = (size_t)t0 * p.H;
+    s.T = T;
+    s.q = reinterpret_cast<const uint8_t *>(p.q) + r * p.dk * 2;
+    s.k = reinterpret_cast<const uint8_t *>(p.k) + r * p.dk * 2;
+    s.v = reinterpret_cast<const uint8_t *>(p.v) + r * p.dv * 2;
+    s.alpha = p.alpha ? p.alpha + r : nullptr;
+    s.beta = p.beta ? p.beta + r : nullptr;
+    s.o = reinterpret_cast<uint8_t *>(p.o) + r * p.dv * (p.o_bf16 ? 2 : 4);
+    return s;
+}
+
+// Workspace of the segment schedule: the T matrices of every chunk-head (as one
+// pass), then the identity, M, N, h(s1 start) and h(s2 start) per head.
+size_t seg_state_floats(const FwdParams &p) { return (size_t)p.H * p.dk * (2 * (size_t)p.dk + 3 * (size_t)p.dv); }
+
+cudaError_t launch_tc_segments(const FwdParams &p, void *workspace, cudaStream_t stream) {
+    const int NC = (p.T + C - 1) / C;
+    const int L = NC / 3;                   // chunks of s0 and of s1; s2 takes the rest
+    const int T0 = L * C;
+    const int t0[3] = {0, T0, 2 * T0}, Ts[3] = {T0, T0, p.T - 2 * T0};
+    const size_t per_seg = (size_t)p.H * L * WS_CHUNK_BYTES;
+    uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
+    uint8_t *wsg[3] = {ws, ws + per_seg, ws + 2 * per_seg};
+    float *sI = reinterpret_cast<float *>(ws + (size_t)p.H * NC * WS_CHUNK_BYTES);
+    const size_t kk = (size_t)p.H * p.dk * p.dk, kv = (size_t)p.H * p.dk * p.dv;
+    float *sM = sI + kk, *sN = sM + kk, *sH1 = sN + kv, *sH2 = sH1 + kv;
+
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kSegMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_seg_mu);   // one schedule at a time uses the set
+    SegStreams *S = nullptr;
+    if ((e = seg_streams(dev, &S)) != cudaSuccess) return e;
+    cudaEvent_t ev_k1 = S->ev[0], ev_n = S->ev[1], ev_m = S->ev[2], ev_h1 = S->ev[3], ev_k1b = S->ev[4],
+                ev_s1 = S->ev[5], ev_s2 = S->ev[6];
+    cudaStream_t r0 = S->run[0], r1 = S->run[1], r2 = S->run[2], side = S->side;
+#define GDN_SEG_TRY(x) \
+    do { if ((e = (x)) != cudaSuccess) return e; } while (0)
+
+    // key side of s0 and s1, and the identity, on the caller's stream
+    const FwdParams v0 = seg_view(p, t0[0], Ts[0]), v1 = seg_view(p, t0[1], Ts[1]), v2 = seg_view(p, t0[2], Ts[2]);
+    GDN_SEG_TRY(launch_k1_plain(v0, wsg[0], stream));
+    GDN_SEG_TRY(launch_k1_plain(v1, wsg[1], stream));
+    seg_identity_kernel<<<dim3(p.dk, p.H), 128, 0, stream>>>(sI, p.dk);
+    GDN_SEG_TRY(cudaGetLastError());
+    GDN_SEG_TRY(cudaEventRecord(ev_k1, stream));
+
+    // pass 1: s0 from S0 (its outputs; h at s1's start), s1 from 0 (N), s1 with
+    // V = 0 from the identity (M, a d_k-column state); the key side of s2 beside them
+    FwdParams a0 = v0;
+    a0.S_T = sH1;
+    FwdParams an = v1;
+    an.S0 = nullptr; an.o = nullptr; an.S_T = sN;
+    FwdParams am = v1;
+    am.v = nullptr; am.dv = p.dk; am.S0 = sI; am.o = nullptr; am.S_T = sM;
+    GDN_SEG_TRY(cudaStreamWaitEvent(r0, ev_k1, 0));
+    GDN_SEG_TRY(cudaStreamWaitEvent(r1, ev_k1, 0));
+    GDN_SEG_TRY(cudaStreamWaitEvent(r2, ev_k1, 0));
+    GDN_SEG_TRY(cudaStreamWaitEvent(side, ev_k1, 0));
+    GDN_SEG_TRY(launch_k2_plain(a0, wsg[0], r0));
+    GDN_SEG_TRY(launch_k2_plain(an, wsg[1], r1));
+    GDN_SEG_TRY(launch_k2_plain(am, wsg[1], r2));
+    GDN_SEG_TRY(launch_k1_plain(v2, wsg[2], side));
+    GDN_SEG_TRY(cudaEventRecord(ev_h1, r0));
+    GDN_SEG_TRY(cudaEventRecord(ev_n, r1));
+    GDN_SEG_TRY(cudaEventRecord(ev_m, r2));
+    GDN_SEG_TRY(cudaEventRecord(ev_k1b, side));
+
+    // pass 2: s1 from h(s1 start); h(s2 start) = M h(s1 start) + N, then s2 from it
+    FwdParams a1 = v1;
+    a1.S0 = sH1; a1.S_T = nullptr;
+    GDN_SEG_TRY(cudaStreamWaitEvent(r1, ev_h1, 0));
+    GDN_SEG_TRY(launch_k2_plain(a1, wsg[1], r1));
+    GDN_SEG_TRY(cudaEventRecord(ev_s1, r1));
+    GDN_SEG_TRY(cudaStreamWaitEvent(r0, ev_n, 0));
+    GDN_SEG_TRY(cudaStreamWaitEvent(r0, ev_m, 0));
+    seg_compose_kernel<<<dim3(p.dk, p.H), 128, 0, r0>>>(sM, sH1, sN, sH2, p.dk, p.dv);
+    GDN_SEG_TRY(cudaGetLastError());
+    FwdParams a2 = v2;
+    a2.S0 = sH2;    // S_T: the caller's (it may alias S0, which pass 1 has read)
+    GDN_SEG_TRY(cudaStreamWaitEvent(r0, ev_k1b, 0));
+    GDN_SEG_TRY(launch_k2_plain(a2, wsg[2], r0));
+    GDN_SEG_TRY(cudaEventRecord(ev_s2, r0));
+
+    // join: the caller's stream continues after both pass-2 runs
+    GDN_SEG_TRY(cudaStreamWaitEvent(stream, ev_s1, 0));
+    GDN_SEG_TRY(cudaStreamWaitEvent(stream, ev_s2, 0));
+#undef GDN_SEG_TRY
+    return cudaSuccess;
+}
+
 }  // namespace
 
 bool tc_supports(const FwdParams &p, const char **why) {
@@ -1400,11 +1610,37 @@ size_t tc_workspace_bytes(const FwdParams &p) {
     if (p.general) return gen_prep_workspace_bytes(p);
     const size_t nc = (size_t)(p.T + C - 1) / C;
     const size_t per = WS_CHUNK_BYTES + (p.C == 2 * C ? pair_stride(p.dv) * 4 : 0);
-    return (size_t)p.B * p.H * nc * per;
+    return (size_t)p.B * p.H * nc * per + (p.segments == 3 ? seg_state_floats(p) * 4 : 0);
+}
+
+bool tc_segments_support(const FwdParams &p, const char **why) {
+    if (p.B != 1) { *why = "sequence segments need B = 1"; return false; }
+    if (p.general || p.C != C) { *why = "sequence segments: the scalar rule at chunk 64 only"; return false; }
+    if ((p.T + C - 1) / C < 3) { *why = "sequence segments need at least 3 chunks"; return false; }
+    return true;
+}
+
+int tc_auto_segments(const FwdParams &p) {
+    const char *why = "";
+    if (!tc_segments_support(p, &why)) return 1;
+    // a long sequence whose chains fill under a third of the SMs: three chain runs
+    // side by side in the first pass still fit in one wave
+    const int NC = (p.T + C - 1) / C;
+    return (NC >= kSegAutoMinChunks && 3 * p.H * (p.dv / DVS) <= kSMs) ? 3 : 1;
 }
 
 cudaError_t launch_tc(const FwdParams &p, void *workspace, cudaStream_t stream, const char **why) {
     const int NC = (p.T + C - 1) / C;
+    if (p.segments == 3) {
+        cudaError_t e = cudaFuncSetAttribute(keyside_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)K1_SMEM_RES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(chain_kernel<K2_PLAIN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)K2Layout<K2_PLAIN>::SMEM);
+        if (e == cudaSuccess) e = launch_tc_segments(p, workspace, stream);
+        if (e != cudaSuccess) *why = "(sequence segments)";
+        return e;
+    }
     CUtensorMap mq, mk, mv, mt;
     if (p.general) {
         // the two-gate rule: the prep's fp16 rows, then the chain kernel (every

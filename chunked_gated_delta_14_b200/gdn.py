@@ -33,7 +33,7 @@ MODES = {"exact": GDN_INV_EXACT, "neumann": GDN_INV_NEUMANN, "residual": GDN_INV
 
 EXPORTS = ("gdn_chunk_fwd", "gdn_select_kernel", "gdn_workspace_bytes", "gdn_device_check",
            "gdn_status_string", "gdn_last_error", "gdn_abi_version", "gdn_chunk_fwd_static_scratch",
-           "gdn_chunk_bwd", "gdn_bwd_workspace_bytes", "gdn_debug_chunk_T")
+           "gdn_chunk_bwd", "gdn_bwd_workspace_bytes", "gdn_debug_chunk_T", "gdn_select_segments")
 STATIC_SCRATCH_BYTES = 24 << 20   # GDN_STATIC_SCRATCH_BYTES
 
 
@@ -60,6 +60,7 @@ class FwdArgs(ctypes.Structure):
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_uint64),
         ("residual_S", ctypes.c_int32),
         ("precond_x", ctypes.c_float), ("precond_query", ctypes.c_int32),
+        ("seq_segments", ctypes.c_int32),
     ]
 
 
@@ -96,6 +97,8 @@ def lib() -> ctypes.CDLL:
             L.gdn_chunk_fwd.restype = ctypes.c_int
             L.gdn_select_kernel.argtypes = [ctypes.POINTER(FwdArgs)]
             L.gdn_select_kernel.restype = ctypes.c_int32
+            L.gdn_select_segments.argtypes = [ctypes.POINTER(FwdArgs)]
+            L.gdn_select_segments.restype = ctypes.c_int32
             L.gdn_workspace_bytes.argtypes = [ctypes.POINTER(FwdArgs)]
             L.gdn_workspace_bytes.restype = ctypes.c_uint64
             L.gdn_device_check.argtypes = [ctypes.c_void_p]
@@ -174,6 +177,11 @@ def select_kernel(args: FwdArgs) -> int:
     """Kernel gdn_chunk_fwd would launch (1 simt, 2 fused tc, 3 recurrent, 4 split tc)
     or -status. Host only."""
     return int(lib().gdn_select_kernel(ctypes.byref(args)))
+
+
+def select_segments(args: FwdArgs) -> int:
+    """Sequence segments gdn_chunk_fwd would use (1 or 3) or -status. Host only."""
+    return int(lib().gdn_select_segments(ctypes.byref(args)))
 
 
 def workspace_bytes(args: FwdArgs) -> int:
@@ -279,7 +287,7 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
               precond_x: float = 2.0, precond_query: bool = False,
               S0: Optional[torch.Tensor] = None, chunk: int = 64, mode: str = "exact",
               N: int = 3, S: int = 8, o_dtype: Optional[torch.dtype] = None, kernel: str = "auto",
-              dv_split: int = 0, out: Optional[torch.Tensor] = None,
+              dv_split: int = 0, segments: int = 0, out: Optional[torch.Tensor] = None,
               final_state: bool = True, S_T: Optional[torch.Tensor] = None,
               stream: Optional[torch.cuda.Stream] = None
               ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
@@ -293,7 +301,9 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     [1/precond_x, precond_x]; ``precond_query`` moves the factor to the query.  S0 / S_T:
     [B, H, dk, dv] fp32 (h = S^T).  ``o_dtype`` defaults to q's dtype.
     ``mode``: "exact", "neumann" (masked series to order N) or "residual" (the
-    masked series corrected with S residual terms).
+    masked series corrected with S residual terms).  ``segments``: 0 lets the
+    library choose, 1 forces one pass over the chunks, 3 three sequence segments
+    (split tensor-core kernels, scalar rule, chunk 64, B = 1).
     """
     if q.dim() != 4:
         raise ValueError("q must be [B, T, H, dk]")
@@ -325,7 +335,8 @@ def chunk_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         precond_x=float(precond_x), precond_query=int(bool(precond_query)),
         rho_decay=float(rho_decay), rho_eps=float(rho_eps), erase=_ptr(erase),
         write=_ptr(write), S0=_ptr(S0), o=_ptr(out), S_T=_ptr(S_T), mode=MODES[mode],
-        neumann_N=int(N), residual_S=int(S), kernel=KERNELS[kernel], dv_split=int(dv_split))
+        neumann_N=int(N), residual_S=int(S), kernel=KERNELS[kernel], dv_split=int(dv_split),
+        seq_segments=int(segments))
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     ws = workspace_for(args, q.device, stream)

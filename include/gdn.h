@@ -80,7 +80,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 7
+#define GDN_ABI_VERSION 8
 
 #if defined(__GNUC__)
 #define GDN_API __attribute__((visibility("default")))
@@ -173,6 +173,11 @@ typedef struct {
     float precond_x;            /* squash bound x > 1 for precond 3 */
     int32_t precond_query;      /* 1: apply the factor to the query (ATQ) instead of the
                                    write key (ATK); the write key is then k_t itself */
+    int32_t seq_segments;       /* split tensor-core path, scalar rule, chunk 64, B = 1:
+                                   0 = the library chooses (3 from 256 chunks when three
+                                   rows of chains, H * dv / 64 each, fit the 148 SMs),
+                                   1 = one pass over the chunks, 3 = three sequence
+                                   segments (see gdn_select_segments) */
 } gdn_fwd_args;
 
 /* Chunkwise forward: o and S_T from q, k, v, gates and S0 (see above). */
@@ -187,6 +192,28 @@ GDN_API uint64_t gdn_workspace_bytes(const gdn_fwd_args *args);
  * value, never AUTO), or a negative gdn_status if they are invalid.  Host
  * only; launches nothing. */
 GDN_API int32_t gdn_select_kernel(const gdn_fwd_args *args);
+
+/* Sequence segments gdn_chunk_fwd would use for these arguments (1 or 3), or
+ * a negative gdn_status if they are invalid.  Host only; launches nothing.
+ *
+ * The state update is affine in the state (S_t = S_{t-1} alpha_t (I - beta_t
+ * k_t k_t^T) + beta_t v_t k_t^T, "Resumo Tecnico: Preconditioned DeltaNet",
+ * section 1), so over any run of chunks h_end = M h_start + N, with M the
+ * run's d_k x d_k product of transitions (the run from h = I with v = 0) and N
+ * its end state from h = 0.  With 3 segments s0, s1, s2 (s0 and s1 of
+ * floor(chunks / 3) chunks each) the call runs, on three library-owned
+ * high-priority streams joined back into `stream`: s0 from S0, s1 from 0 and
+ * s1 with v = 0 from the identity side by side (the key-side kernel of s2
+ * beside them on a fourth, low-priority stream); then h(s2) = M h(s1) + N and
+ * s1, s2 from their true starts.  Two chain passes of a third of the chunks
+ * each replace one over all of them: the serial chain per (head, value slice)
+ * is the cost when B * H * dv / 64 chains fill few of the SMs.  The schedule
+ * is this library's, not the pages'.  The workspace grows by
+ * H * dk * (2 dk + 3 dv) floats (identity, M, N, two start states).  The
+ * streams and events are made on the first such call on each device (with
+ * that device current) and kept until exit; concurrent calls from several
+ * host threads take turns enqueueing. */
+GDN_API int32_t gdn_select_segments(const gdn_fwd_args *args);
 
 /* Synchronises `stream` (void* cudaStream_t), then reports and clears a
  * failure recorded on the device by the kernels' own checks: a bounded wait
