@@ -136,6 +136,11 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
         p.dvs = p.dv / p.slices;
         if (!gdn::tc_supports(p, &why))
             return fail(GDN_ERR_UNSUPPORTED, "split tensor-core kernels: %s", why);
+        // Exact inversion at chunk 128 as two 64-token chunks: T = (I - A)^-1 of a
+        // 128-token chunk is block lower triangular with the two halves' inverses on
+        // its diagonal, and its off-diagonal block is what the state carried from
+        // the first half to the second applies, so o and S_T are those of chunk 64.
+        if (p.C == 128 && p.mode == GDN_INV_EXACT && !p.general) p.C = 64;
         if (a->seq_segments == 3 && !gdn::tc_segments_support(p, &why))
             return fail(GDN_ERR_UNSUPPORTED, "split tensor-core kernels: %s", why);
         p.segments = a->seq_segments ? a->seq_segments : gdn::tc_auto_segments(p);

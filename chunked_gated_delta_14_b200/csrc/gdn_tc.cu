@@ -1593,8 +1593,8 @@ bool tc_supports(const FwdParams &p, const char **why) {
         if (p.slices && p.dvs != DVS) { *why = "value slices must be 64 columns"; return false; }
         return true;
     }
-    if (p.C != C && !(p.C == 2 * C && p.mode == GDN_INV_NEUMANN)) {
-        *why = "needs chunk 64 (or 128 with the masked series)";
+    if (p.C != C && !(p.C == 2 * C && (p.mode == GDN_INV_NEUMANN || p.mode == GDN_INV_EXACT))) {
+        *why = "needs chunk 64 (or 128, exact or with the masked series)";
         return false;
     }
     if (p.dk != DK) { *why = "needs dk 128"; return false; }

@@ -125,11 +125,13 @@ def test_valid_arguments_select_a_kernel():
     assert gdn.select_kernel(_args(precond=1, kernel=2, **two_gate)) < 0     # not on the fused kernel
     assert gdn.select_kernel(_args(S0=0x80000, S_T=0x80000)) in (1, 2, 4)  # S_T may alias S0
     # chunk 128: the masked series (N <= 15) on the split kernels as two 64-token
-    # halves; the exact inverse and wider bands on the SIMT kernel
+    # halves; wider bands on the SIMT kernel
     assert gdn.select_kernel(_args(chunk=128, mode=1, neumann_N=3)) == 4
     assert gdn.select_kernel(_args(chunk=128, mode=1, neumann_N=15)) == 4
     assert gdn.select_kernel(_args(chunk=128, mode=1, neumann_N=16)) == 1
-    assert gdn.select_kernel(_args(chunk=128)) == 1
+    # exact inversion at chunk 128: the split kernels, as 64-token chunks (the same o, S_T)
+    assert gdn.select_kernel(_args(chunk=128)) == 4
+    assert gdn.workspace_bytes(_args(chunk=128)) == gdn.workspace_bytes(_args(chunk=64))
     assert gdn.select_kernel(_args(chunk=128, mode=2, neumann_N=3, residual_S=8)) < 0
 
 

@@ -76,3 +76,16 @@ def test_tc_ragged_weak_decay(kernel):
     """A ragged length (tail chunk of 17 tokens) with weak decay and S0."""
     w = workload("gdn_bf16", B=2, H=3, T=1041, decay="weak", s0_std=0.02)
     _check_tc("tc_ragged_weak", w, 34, kernel)
+
+
+@needs_cuda
+def test_tc_exact_chunk128():
+    """Exact inversion at chunk 128 on the split kernels: against the fp64 oracle at
+    the bar, and identical to chunk 64 (a 128-token chunk's exact inverse is block
+    lower triangular; the state between its halves applies the off-diagonal block)."""
+    w = workload("gdn_bf16", B=2, H=4, T=1000, chunk=128, decay="weak", s0_std=0.02)
+    _check_tc("tc_exact_chunk128", w, 35, "tc_split")
+    x = make_inputs(w, seed=35)
+    o128, s128 = run_gpu(x, w, o_dtype=torch.float32, kernel="tc_split")
+    o64, s64 = run_gpu(x, w.replace(chunk=64), o_dtype=torch.float32, kernel="tc_split")
+    assert (o128 == o64).all() and (s128 == s64).all()
