@@ -313,21 +313,29 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tma_load_4d(sm + K1_OFF_QK + 24576, &tm_k, &bars[0], 64, h, t0, b);
     }
     __syncwarp();
-    if (warp == 0) {
-        tmem_alloc(tmem_slot, 128);      // Gram (64 columns), inverse merge (64)
-        tmem_relinquish();
-    }
-    if (!p.neumann)
-        for (int i = tid; i < 64 * LSTR; i += K1_THREADS) Tb[i] = 0.f;
-    tc_fence_before();
-    block_sync();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
+    // set-up in parallel: warp 0 has issued the tile loads, warp 1 fetches and scans
+    // the gates (their global loads are the longest wait before the Gram), warp 2
+    // allocates TMEM, everyone clears the two upper 16 x 16 blocks of the inverse's
+    // 32-blocks (the 32 -> 64 merge reads them as zeros; the rest of T above the
+    // diagonal is never read as anything but zero: the final writes mask it)
     if (warp == 1) {
         float a0, a1, b0, b1;
         tc::fetch_gates(p.alpha, p.beta, b, p.T, p.H, h, t0, lane, true, a0, a1, b0, b1);
         tc::scan_gates(par, a0, a1, b0, b1, lane, min(C, p.T - t0));
     }
+    if (warp == 2) {
+        tmem_alloc(tmem_slot, 128);      // Gram (64 columns), inverse merge (64)
+        tmem_relinquish();
+    }
+    if (!p.neumann) {
+        const int blk = tid >> 7, u = tid & 127;
+        *reinterpret_cast<float2 *>(Tb + (32 * blk + (u >> 3)) * LSTR + 32 * blk + 16 + 2 * (u & 7)) =
+            make_float2(0.f, 0.f);
+    }
+    tc_fence_before();
+    block_sync();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
     if (tid == 0) {
         if (mbar_wait(&bars[0], 0, abort_flag, E_K1_TMA, kWaitLimit)) {
             tc_fence_after();
@@ -582,7 +590,7 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 float t[8], sb[8], sg[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    t[e] = Tr[8 * j + e];
+                    t[e] = 8 * j + e <= rr ? Tr[8 * j + e] : 0.f;    // T is lower triangular
                     sb[e] = t[e] * par->bet[8 * j + e];
                     sg[e] = sb[e] * par->eg[8 * j + e];
                 }
@@ -595,7 +603,7 @@ keyside_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     tc_fence_before();
     block_sync();
-    if (warp == 0) {
+    if (warp == 2) {
         tc_fence_after();
         tmem_dealloc(tmem, 128);
     }

@@ -164,3 +164,25 @@ def test_segments_repeat_alias_and_one_pass():
     _check("segments_vs_one_pass", o1, S1, op.double().cpu().numpy(), Sp.double().cpu().numpy())
     o_ref, s_ref = oracle.gated_delta_fwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"])
     _check("segments_alias", o3, S3, o_ref, s_ref)
+
+
+@pytest.mark.gpu
+@needs_cuda
+def test_segments_long_context_bf16_output():
+    """The timed long-context configuration (bf16 o, the library's choice of
+    segments) against the fp64 oracle: every element within the bar plus one bf16
+    rounding of the reference, and S_T (fp32) at the bar."""
+    from gpu_util import bf16_allowance_ok
+    w = workload("long_context")
+    x = make_inputs(w)
+    d = {k: (None if v is None else v.to("cuda").contiguous()) for k, v in x.items()}
+    a = _args(T=w.T, H=w.H, o_dtype=1)
+    assert gdn.select_segments(a) == 3
+    o, S = gdn.chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S0=d["S0"], chunk=64)
+    torch.cuda.synchronize()
+    assert o.dtype == torch.bfloat16
+    o_ref, s_ref = oracle.gated_delta_fwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"])
+    got = o.double().cpu().numpy()
+    report("segments_long_context_bf16_o", o=stats(got, o_ref), S_T=stats(S.double().cpu().numpy(), s_ref))
+    assert bf16_allowance_ok(got, o_ref)
+    assert stats(S.double().cpu().numpy(), s_ref)["max_rel_rms"] <= TOL_BF16_REL_RMS
