@@ -158,7 +158,8 @@ __device__ __forceinline__ void block_product(const float *A, int ra, int ia, in
 // One block per chunk-head.  Shared memory (floats): K, Q (C x (dk+1)),
 // V and then dO (C x (dv+1)), L, T, M (C x (C+1)), g, beta, beta e^g, e^g (C each).
 __host__ __device__ inline size_t prep_smem_floats(int C, int dk, int dv) {
-    return 2 * (size_t)C * (dk + 1) + (size_t)C * (dv + 1) + 3 * (size_t)C * (C + 1) + 4 * (size_t)C;
+    return 2 * (size_t)C * (dk + 1) + (size_t)C * (dv + 1) + 3 * (size_t)C * (C + 1) + 4 * (size_t)C +
+           (size_t)C * C / 4;   // + the inverse's merge scratch
 }
 
 __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(const BwdParams p) {
@@ -178,6 +179,7 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(const BwdParams 
     float *bb = g + C;
     float *bg = bb + C;
     float *eg = bg + C;
+    float *Ys = eg + C;        // C/2 x C/2: the inverse's merge scratch
     const size_t ch = ((size_t)b * p.H + h) * p.NC + n;
 
     load_rows<kPrepThreads>(p, b, h, t0, C, Cn, dk, dkp, p.k, p.io_bf16, Ks, p.q, p.io_bf16, Qs, tid);
@@ -209,60 +211,105 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(const BwdParams 
     }
     __syncthreads();
 
-    // L (strictly lower) and M (lower with diagonal).  Thread t takes column
-    // i = t % C and rows t / C + (kPrepThreads / C) k, one pair of accumulators each
-    // (at C = 16 the threads past row 15 have none).
+    // L (strictly lower) and M (lower with diagonal) in 4 x 4 register tiles of
+    // (rows r0.., keys i0..): per channel the tile's four key rows, query rows and
+    // column keys (12 loads per 32 products).  Two neighbouring lanes take the even
+    // and odd channels of one tile and add their sums with a shuffle.  Tiles above
+    // the diagonal only write zeros; the rows past the tail are the zero rows.
     {
-        constexpr int KR = kMaxC * kMaxC / kPrepThreads;  // rows per thread at C = 64
-        const int i = tid % C, rstep = kPrepThreads / C;
-        const int nk = C * C >= kPrepThreads ? C * C / kPrepThreads : 1;
-        float gk[KR], qk[KR];
+        const int nt = C / 4, tiles = nt * nt;
+        for (int w = tid; w < 2 * tiles; w += kPrepThreads) {
+            const int part = w & 1, t = w >> 1;
+            const int r0 = 4 * (t / nt), i0 = 4 * (t % nt);
+            float gk[4][4] = {}, qk[4][4] = {};
+            if (i0 <= r0 + 3) {
+                for (int c = part; c < dk; c += 2) {
+                    float kr[4], qr[4], ki[4];
 #pragma unroll
-        for (int k = 0; k < KR; ++k) gk[k] = qk[k] = 0.f;
-        // every (r, i) pair of the chunk accumulates; the ones outside the lower
-        // triangle or the sequence are dropped when written (no divergent branch in
-        // the loop at C >= 32; the rows it reads past the tail are the zero rows)
-        for (int c = 0; c < dk; ++c) {
-            const float ki = Ks[i * dkp + c];
+                    for (int a = 0; a < 4; ++a) {
+                        kr[a] = Ks[(r0 + a) * dkp + c];
+                        qr[a] = Qs[(r0 + a) * dkp + c];
+                        ki[a] = Ks[(i0 + a) * dkp + c];
+                    }
 #pragma unroll
-            for (int k = 0; k < KR; ++k) {
-                const int r = tid / C + rstep * k;
-                if (k < nk && r < C) {
-                    gk[k] += Ks[r * dkp + c] * ki;
-                    qk[k] += Qs[r * dkp + c] * ki;
+                    for (int a = 0; a < 4; ++a)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            gk[a][e] += kr[a] * ki[e];
+                            qk[a][e] += qr[a] * ki[e];
+                        }
                 }
             }
-        }
 #pragma unroll
-        for (int k = 0; k < KR; ++k) {
-            const int r = tid / C + rstep * k;
-            if (k < nk && r < C) {
-                float gg = 0.f, m = 0.f;
-                if (r < Cn && i <= r) {
-                    const float gam = expf(g[r] - g[i]);
-                    m = gam * qk[k];
-                    if (i < r) gg = gam * gk[k];
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    gk[a][e] += __shfl_xor_sync(0xffffffffu, gk[a][e], 1);
+                    qk[a][e] += __shfl_xor_sync(0xffffffffu, qk[a][e], 1);
                 }
-                Ls[r * Cp + i] = bb[r] * gg;
-                Ms[r * Cp + i] = m;
-                p.ws_S[ch * C * C + r * C + i] = gg;
-                p.ws_M[ch * C * C + r * C + i] = m;
+            if (part == 0) {
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int r = r0 + a, i = i0 + e;
+                        float gg = 0.f, m = 0.f;
+                        if (r < Cn && i <= r) {
+                            const float gam = expf(g[r] - g[i]);
+                            m = gam * qk[a][e];
+                            if (i < r) gg = gam * gk[a][e];
+                        }
+                        Ls[r * Cp + i] = bb[r] * gg;
+                        Ms[r * Cp + i] = m;
+                        p.ws_S[ch * C * C + r * C + i] = gg;
+                        p.ws_M[ch * C * C + r * C + i] = m;
+                    }
             }
         }
     }
     __syncthreads();
 
-    // T = (I + L)^-1 one column per thread: (I + L) t = e_j by forward
-    // substitution, t_r = 0 above the diagonal.
-    if (tid < Cn) {
-        const int j = tid;
-        Ts[j * Cp + j] = 1.f;
-        for (int r = j + 1; r < Cn; ++r) {
-            float s = 0.f;
-            for (int i = j; i < r; ++i) s += Ls[r * Cp + i] * Ts[i * Cp + j];
-            Ts[r * Cp + j] = -s;
+    // T = (I + L)^-1, blocked: the 16 x 16 diagonal blocks by forward substitution
+    // (one column per thread; each solved entry updates the rows below it), then
+    // the merges 16 -> 32 -> 64 of neighbouring blocks, T21 = -T22 L21 T11, with
+    // every thread.  T starts at zero, so the blocks above the diagonal stay zero.
+    // Rows past the tail have zero L rows; their diagonal is cleared at the end, so
+    // that T is zero outside the sequence as the chains expect.
+    if (tid < C) {
+        const int c = tid, base = c & ~15, jc = c & 15;
+        float acc[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) acc[r] = (r == jc) ? 1.f : 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float xi = acc[i];
+#pragma unroll
+            for (int r = i + 1; r < 16; ++r) acc[r] -= Ls[(base + r) * Cp + base + i] * xi;
         }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Ts[(base + r) * Cp + c] = acc[r];
     }
+    __syncthreads();
+    for (int sz = 16; sz < C; sz *= 2) {
+        const int work = (C / (2 * sz)) * sz * sz;      // outputs of one product, all pairs
+        for (int o = tid; o < work; o += kPrepThreads) {
+            const int pr = o / (sz * sz), rr = (o / sz) % sz, cc = o % sz;
+            const int b0 = 2 * sz * pr, b1 = b0 + sz;
+            float y = 0.f;
+            for (int k = 0; k < sz; ++k) y += Ls[(b1 + rr) * Cp + b0 + k] * Ts[(b0 + k) * Cp + b0 + cc];
+            Ys[o] = y;
+        }
+        __syncthreads();
+        for (int o = tid; o < work; o += kPrepThreads) {
+            const int pr = o / (sz * sz), rr = (o / sz) % sz, cc = o % sz;
+            const int b0 = 2 * sz * pr, b1 = b0 + sz;
+            float z = 0.f;
+            for (int k = 0; k < sz; ++k) z += Ts[(b1 + rr) * Cp + b1 + k] * Ys[pr * sz * sz + k * sz + cc];
+            Ts[(b1 + rr) * Cp + b0 + cc] = -z;
+        }
+        __syncthreads();
+    }
+    if (tid < C && tid >= Cn) Ts[tid * Cp + tid] = 0.f;
     __syncthreads();
 
     for (int x = tid; x < C * C; x += kPrepThreads) p.ws_T[ch * C * C + x] = Ts[(x / C) * Cp + x % C];

@@ -28,10 +28,14 @@ static void run_grid(F kernel, dim3h grid, const BwdParams &p, size_t smem_float
                 fill_nan(bwd::bwd_smem, sizeof(bwd::bwd_smem));
                 std::barrier<> bar(nthreads);
                 g_block_barrier = &bar;
+                std::vector<std::barrier<> *> warps;
+                for (int w = 0; w < (nthreads + 31) / 32; ++w) warps.push_back(new std::barrier<>(32));
+                g_warp_barriers = warps.data();
                 std::vector<std::thread> th;
                 for (int t = 0; t < nthreads; ++t)
                     th.emplace_back([&, t] { threadIdx = {(unsigned)t, 0, 0}; kernel(p); });
                 for (auto &t : th) t.join();
+                for (auto *w : warps) delete w;
                 const uint32_t *u = reinterpret_cast<const uint32_t *>(bwd::bwd_smem);
                 for (size_t i = smem_floats; i < sizeof(bwd::bwd_smem) / 4; ++i)
                     if (u[i] != 0x7fc00000u) { ++g_overrun; break; }
