@@ -116,40 +116,46 @@ __device__ __forceinline__ void load_rows(const BwdParams &p, int b, int h, int 
 
 // out[r][c] = sum_{i < nterm} A(r, i) scale[i] X[i][c] for r < nrow, c < n, with
 // A(r, i) = A[r * ra + i * ia] in shared memory (so A or its transpose) and
-// scale null meaning 1; written to global memory row-major.  With half = n / 2
-// and rstep = NT / half row groups, thread t < rstep half takes the two
-// columns t % half and t % half + half and the rows t / half + rstep m: each A
-// load serves both columns and each X load all of the thread's rows, with a
-// separate accumulator per output (threads past the last full group idle).
-// n even, 16 <= n <= 128, and ceil(nrow / rstep) <= MAXR.
+// scale null meaning 1; written to global memory row-major.  With q = n / 4 and
+// rstep = NT / q row groups, thread t < rstep q takes the four columns t % q + q j
+// (j < 4) and the rows t / q + rstep m: each A load serves four columns and each
+// X load all of the thread's rows, with a separate accumulator per output
+// (threads past the last full group idle).  n a multiple of 4, 16 <= n <= 128,
+// and ceil(nrow / rstep) <= MAXR.
 template <int MAXR, int NT = kThreads>
 __device__ __forceinline__ void block_product(const float *A, int ra, int ia, int nrow, int nterm,
                                               const float *scale, const float *X, int xp, int n,
                                               float *out, int tid) {
-    const int half = n / 2;
-    const int c = tid % half, rg = tid / half, rstep = NT / half;
+    const int q = n / 4;
+    const int c = tid % q, rg = tid / q, rstep = NT / q;
     if (rg >= rstep || rg >= nrow) return;
     const int nr = (nrow - rg + rstep - 1) / rstep;   // rows rg + rstep m < nrow
-    float acc0[MAXR], acc1[MAXR];
+    float acc[MAXR][4];
 #pragma unroll
-    for (int m = 0; m < MAXR; ++m) acc0[m] = acc1[m] = 0.f;
+    for (int m = 0; m < MAXR; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.f;
     for (int i = 0; i < nterm; ++i) {
         const float sc = scale ? scale[i] : 1.f;
-        const float x0 = sc * X[i * xp + c], x1 = sc * X[i * xp + c + half];
+        const float *xr = X + i * xp + c;
+        const float x0 = sc * xr[0], x1 = sc * xr[q], x2 = sc * xr[2 * q], x3 = sc * xr[3 * q];
 #pragma unroll
         for (int m = 0; m < MAXR; ++m) {
             if (m < nr) {
                 const float a = A[(rg + rstep * m) * ra + i * ia];
-                acc0[m] += a * x0;
-                acc1[m] += a * x1;
+                acc[m][0] += a * x0;
+                acc[m][1] += a * x1;
+                acc[m][2] += a * x2;
+                acc[m][3] += a * x3;
             }
         }
     }
 #pragma unroll
     for (int m = 0; m < MAXR; ++m) {
         if (m < nr) {
-            out[(size_t)(rg + rstep * m) * n + c] = acc0[m];
-            out[(size_t)(rg + rstep * m) * n + c + half] = acc1[m];
+            float *o = out + (size_t)(rg + rstep * m) * n + c;
+            o[0] = acc[m][0];
+            o[q] = acc[m][1];
+            o[2 * q] = acc[m][2];
+            o[3 * q] = acc[m][3];
         }
     }
 }
@@ -315,9 +321,9 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(const BwdParams 
     for (int x = tid; x < C * C; x += kPrepThreads) p.ws_T[ch * C * C + x] = Ts[(x / C) * Cp + x % C];
     if (tid < C) p.ws_g[ch * C + tid] = g[tid];
     // W = T diag(beta e^g) K and U = T diag(beta) V (zero rows past the tail)
-    block_product<kMaxC * 64 / kPrepThreads, kPrepThreads>(Ts, Cp, 1, C, Cn, bg, Ks, dkp, dk, p.ws_W + ch * C * dk,
+    block_product<kMaxC / 16, kPrepThreads>(Ts, Cp, 1, C, Cn, bg, Ks, dkp, dk, p.ws_W + ch * C * dk,
                                                            tid);
-    block_product<kMaxC * 64 / kPrepThreads, kPrepThreads>(Ts, Cp, 1, C, Cn, bb, Vs, dvp, dv, p.ws_D + ch * C * dv,
+    block_product<kMaxC / 16, kPrepThreads>(Ts, Cp, 1, C, Cn, bb, Vs, dvp, dv, p.ws_D + ch * C * dv,
                                                            tid);
     __syncthreads();   // V consumed: its buffer takes dO
     float *dOs = Vs;
@@ -325,9 +331,9 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(const BwdParams 
     __syncthreads();
     // the state-independent parts of the reverse chain: M^T dO (C x dv) and
     // (diag(e^g) Q)^T dO (dk x dv)
-    block_product<kMaxC * 64 / kPrepThreads, kPrepThreads>(Ms, 1, Cp, C, Cn, nullptr, dOs, dvp, dv,
+    block_product<kMaxC / 16, kPrepThreads>(Ms, 1, Cp, C, Cn, nullptr, dOs, dvp, dv,
                                                            p.ws_Y + ch * C * dv, tid);
-    block_product<128 * 64 / kPrepThreads, kPrepThreads>(Qs, 1, dkp, dk, Cn, eg, dOs, dvp, dv,
+    block_product<128 / 16, kPrepThreads>(Qs, 1, dkp, dk, Cn, eg, dOs, dvp, dv,
                                                          p.ws_P + ch * dk * dv, tid);
 }
 
