@@ -63,10 +63,10 @@ cudaError_t launch_bwd(const BwdParams &p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     const size_t gs = bwd::grad_smem_floats(p.C, p.dk);
     switch (p.dk) {
-        case 16: return launch_one(bwd::bwd_grad_kernel<16>, per_chunk, gs, p, stream);
-        case 32: return launch_one(bwd::bwd_grad_kernel<32>, per_chunk, gs, p, stream);
-        case 64: return launch_one(bwd::bwd_grad_kernel<64>, per_chunk, gs, p, stream);
-        case 128: return launch_one(bwd::bwd_grad_kernel<128>, per_chunk, gs, p, stream);
+        case 16: return launch_one(bwd::bwd_grad_kernel<16>, per_chunk, gs, p, stream, bwd::kGradThreads);
+        case 32: return launch_one(bwd::bwd_grad_kernel<32>, per_chunk, gs, p, stream, bwd::kGradThreads);
+        case 64: return launch_one(bwd::bwd_grad_kernel<64>, per_chunk, gs, p, stream, bwd::kGradThreads);
+        case 128: return launch_one(bwd::bwd_grad_kernel<128>, per_chunk, gs, p, stream, bwd::kGradThreads);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -45,6 +45,8 @@ namespace bwd {
 
 constexpr int kThreads = 256;
 constexpr int kPrepThreads = 512;   // the prep kernel: one block per SM (shared memory), 16 warps
+constexpr int kGradThreads = 512;   // the key-side gradient kernel, likewise
+constexpr int kGradGroups = kGradThreads / 32;   // its key-column groups (32 row pairs)
 constexpr int kCols = 32;     // value columns per block of the two chains and per tile
 constexpr int kMaxC = 64;     // largest chunk
 
@@ -599,32 +601,36 @@ __global__ void __launch_bounds__(kThreads) bwd_state_rev_kernel(const BwdParams
 }
 
 // ------------------------------------------------------ key-side gradients
-// One block per chunk-head.  Thread (rp, c8) = (tid / 8, tid % 8) owns the two
-// rows r0 = 2 rp, r1 = 2 rp + 1 and the key columns c8 + 8m of the three
+// One block per chunk-head of kGradThreads threads (16 warps: the block holds
+// 170 KB of shared memory, so one block per SM; the warps hide each other's
+// shared-memory latency).  With NG = kGradThreads / 32 column groups, thread
+// (rp, cg) = (tid / NG, tid % NG) owns the two rows r0 = 2 rp, r1 = 2 rp + 1 and
+// the key columns cg + NG m of the three
 // C x dk products over the value axis (dO h^T, Y h^T, Delta dh'^T),
 // accumulated in registers over 32-column value tiles, and the entries
-// (r0 or r1, c8 + 8m) of dO Delta^T and Y Delta^T in shared memory.  Each
+// (r0 or r1, cg + NG m) of dO Delta^T and Y Delta^T in shared memory.  Each
 // loaded h, dh' and K element serves both rows.
 // Shared memory: K, Q (C x (DK+1)), two C x (C+1) score buffers, the value
 // tiles (h, dh': DK x 33; dO, Y, Delta, V: C x 33; reused afterwards for two
-// C x (C+1) buffers), g, beta, e^g (C), kThreads partials, 4 x 8 x kMaxC row
-// partials and 10 x kMaxC row values.
+// C x (C+1) buffers), g, beta, e^g (C), kGradThreads partials, 4 x NG x kMaxC
+// row partials and 10 x kMaxC row values.
 __host__ __device__ inline size_t grad_smem_floats(int C, int DK) {
     return 2 * (size_t)C * (DK + 1) + 2 * (size_t)C * (C + 1) + 2 * (size_t)DK * 33 + 4 * (size_t)C * 33 +
-           3 * (size_t)C + kThreads + 32 * kMaxC + 10 * kMaxC;
+           3 * (size_t)C + kGradThreads + 4 * (size_t)kGradGroups * kMaxC + 10 * kMaxC;
 }
 
 enum { RV_A2K = 0, RV_QA1, RV_K3, RV_YV, RV_KAP, RV_DB, RV_DG, RV_HDH };
 
 template <int DK>
-__global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
-    constexpr int MK = DK / 8;         // key columns per thread
-    constexpr int MC = kMaxC / 8;      // score columns per thread
+__global__ void __launch_bounds__(kGradThreads) bwd_grad_kernel(const BwdParams p) {
+    constexpr int NT = kGradThreads, NG = kGradGroups;
+    constexpr int MK = DK / NG;        // key columns per thread
+    constexpr int MC = kMaxC / NG;     // score columns per thread
     constexpr int dkp = DK + 1;
     float *sm = reinterpret_cast<float *>(bwd_smem);
     const int C = p.C, dv = p.dv;
     const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-    const int c8 = tid & 7, r0 = 2 * (tid >> 3), r1 = r0 + 1;
+    const int cg = tid % NG, r0 = 2 * (tid / NG), r1 = r0 + 1;
     const int t0 = n * C, Cn = min(C, p.T - t0);
     const bool v0 = r0 < Cn, v1 = r1 < Cn;     // r1 < C whenever v0 (C is even)
     const int Cp = C + 1;
@@ -643,12 +649,12 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
     float *bs = gs + C;
     float *egs = bs + C;
     float *red = egs + C;
-    float *part = red + kThreads;        // [4 quantities][8 c8][kMaxC]
-    float *rowv = part + 32 * kMaxC;     // [10][kMaxC]
+    float *part = red + NT;              // [4 quantities][NG cg][kMaxC]
+    float *rowv = part + 4 * NG * kMaxC; // [10][kMaxC]
     const size_t ch = ((size_t)b * p.H + h) * p.NC + n;
 
-    load_rows<kThreads>(p, b, h, t0, C, Cn, DK, dkp, p.k, p.io_bf16, Ks, p.q, p.io_bf16, Qs, tid);
-    for (int x = tid; x < C * Cp; x += kThreads) {
+    load_rows<NT>(p, b, h, t0, C, Cn, DK, dkp, p.k, p.io_bf16, Ks, p.q, p.io_bf16, Qs, tid);
+    for (int x = tid; x < C * Cp; x += NT) {
         dMs[x] = 0.f;
         dLs[x] = 0.f;
     }
@@ -670,11 +676,11 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
         // before its first store
         {
             constexpr int NH = DK * (kCols / 4);                      // float4 items (h, dh)
-            constexpr int HQ = (NH + kThreads - 1) / kThreads;        // per thread
+            constexpr int HQ = (NH + NT - 1) / NT;        // per thread
             float4 hv[HQ], dhv[HQ];
 #pragma unroll
             for (int u = 0; u < HQ; ++u) {
-                const int x = tid + kThreads * u, c = x / (kCols / 4), q4 = x % (kCols / 4);
+                const int x = tid + NT * u, c = x / (kCols / 4), q4 = x % (kCols / 4);
                 if (x < NH) {
                     const size_t o = (ch * DK + c) * dv + j0 + 4 * q4;
                     hv[u] = *reinterpret_cast<const float4 *>(p.ws_h + o);
@@ -683,7 +689,7 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
             }
 #pragma unroll
             for (int u = 0; u < HQ; ++u) {
-                const int x = tid + kThreads * u, c = x / (kCols / 4), q4 = x % (kCols / 4);
+                const int x = tid + NT * u, c = x / (kCols / 4), q4 = x % (kCols / 4);
                 if (x < NH) {
                     float *hd = ht + c * 33 + 4 * q4, *dd = dht + c * 33 + 4 * q4;
                     hd[0] = hv[u].x; hd[1] = hv[u].y; hd[2] = hv[u].z; hd[3] = hv[u].w;
@@ -691,11 +697,11 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
                 }
             }
         }
-        for (int base = tid; base < C * (kCols / 4); base += 2 * kThreads) {
+        for (int base = tid; base < C * (kCols / 4); base += 2 * NT) {
             float4 a4[2], v4[2], y4[2], d4[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
-                const int x = base + kThreads * u, r2 = x / (kCols / 4), q4 = x % (kCols / 4);
+                const int x = base + NT * u, r2 = x / (kCols / 4), q4 = x % (kCols / 4);
                 a4[u] = v4[u] = y4[u] = d4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (x < C * (kCols / 4) && r2 < Cn) {
                     const size_t ti = tok_index(p, b, t0 + r2, h) * dv + j0 + 4 * q4;
@@ -707,7 +713,7 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
             }
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
-                const int x = base + kThreads * u, r2 = x / (kCols / 4), q4 = x % (kCols / 4);
+                const int x = base + NT * u, r2 = x / (kCols / 4), q4 = x % (kCols / 4);
                 if (x < C * (kCols / 4)) {
                     const int o = r2 * 33 + 4 * q4;
                     dOt[o] = a4[u].x; dOt[o + 1] = a4[u].y; dOt[o + 2] = a4[u].z; dOt[o + 3] = a4[u].w;
@@ -724,7 +730,7 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
                 const float a1 = dOt[r1 * 33 + jj], y1 = Yt[r1 * 33 + jj], d1 = Dt[r1 * 33 + jj];
 #pragma unroll
                 for (int m = 0; m < MK; ++m) {
-                    const int c = c8 + 8 * m;
+                    const int c = cg + NG * m;
                     const float hv = ht[c * 33 + jj], dhv = dht[c * 33 + jj];
                     A1[0][m] += a0 * hv;
                     A2[0][m] += y0 * hv;
@@ -734,11 +740,11 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
                     A3[1][m] += d1 * dhv;
                 }
             }
-            for (int jj = c8; jj < kCols; jj += 8) {
+            for (int jj = cg; jj < kCols; jj += NG) {
                 yv0 += Yt[r0 * 33 + jj] * Vt[r0 * 33 + jj];
                 yv1 += Yt[r1 * 33 + jj] * Vt[r1 * 33 + jj];
             }
-            // this tile's part of dO Delta^T and Y Delta^T at (r0 or r1, c8 + 8m)
+            // this tile's part of dO Delta^T and Y Delta^T at (r0 or r1, cg + NG m)
             float s1[2][MC], s2[2][MC];
 #pragma unroll
             for (int m = 0; m < MC; ++m) s1[0][m] = s2[0][m] = s1[1][m] = s2[1][m] = 0.f;
@@ -747,8 +753,8 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
                 const float a1 = dOt[r1 * 33 + jj], y1 = Yt[r1 * 33 + jj];
 #pragma unroll
                 for (int m = 0; m < MC; ++m) {
-                    if (c8 + 8 * m < Cn) {
-                        const float d = Dt[(c8 + 8 * m) * 33 + jj];
+                    if (cg + NG * m < Cn) {
+                        const float d = Dt[(cg + NG * m) * 33 + jj];
                         s1[0][m] += a0 * d;
                         s2[0][m] += y0 * d;
                         s1[1][m] += a1 * d;
@@ -758,7 +764,7 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
             }
 #pragma unroll
             for (int m = 0; m < MC; ++m) {
-                const int i = c8 + 8 * m;
+                const int i = cg + NG * m;
                 if (i < Cn) {
                     dMs[r0 * Cp + i] += s1[0][m];
                     dLs[r0 * Cp + i] += s2[0][m];
@@ -769,7 +775,7 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
                 }
             }
         }
-        for (int x = tid; x < DK * kCols; x += kThreads) {
+        for (int x = tid; x < DK * kCols; x += NT) {
             const int c = x / kCols, jj = x % kCols;
             hdh += ht[c * 33 + jj] * dht[c * 33 + jj];
         }
@@ -783,36 +789,36 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
         if (r < Cn) {
 #pragma unroll
             for (int m = 0; m < MK; ++m) {
-                const int c = c8 + 8 * m;
+                const int c = cg + NG * m;
                 a2k += A2[e][m] * Ks[r * dkp + c];
                 qa1 += A1[e][m] * Qs[r * dkp + c];
                 k3 += A3[e][m] * Ks[r * dkp + c];
             }
         }
-        part[(0 * 8 + c8) * kMaxC + r] = a2k;
-        part[(1 * 8 + c8) * kMaxC + r] = qa1;
-        part[(2 * 8 + c8) * kMaxC + r] = k3;
-        part[(3 * 8 + c8) * kMaxC + r] = e ? yv1 : yv0;
+        part[(0 * NG + cg) * kMaxC + r] = a2k;
+        part[(1 * NG + cg) * kMaxC + r] = qa1;
+        part[(2 * NG + cg) * kMaxC + r] = k3;
+        part[(3 * NG + cg) * kMaxC + r] = e ? yv1 : yv0;
     }
     red[tid] = hdh;
     __syncthreads();
     if (tid < kMaxC) {
         for (int qn = 0; qn < 4; ++qn) {
             float s = 0.f;
-            for (int k8 = 0; k8 < 8; ++k8) s += part[(qn * 8 + k8) * kMaxC + tid];
+            for (int k = 0; k < NG; ++k) s += part[(qn * NG + k) * kMaxC + tid];
             rowv[qn * kMaxC + tid] = s;   // RV_A2K, RV_QA1, RV_K3, RV_YV
         }
     }
     if (tid == 0) {
         float s = 0.f;
-        for (int x = 0; x < kThreads; ++x) s += red[x];
+        for (int x = 0; x < NT; ++x) s += red[x];
         rowv[RV_HDH * kMaxC] = s;
     }
 
     // per score entry, with the decayed Gram and scores of the prep kernel
     float *Fs = tile;             // dL (.) L + dM (.) M: F_ri enters dg_r with +, dg_i with -
     float *Es = tile + C * Cp;    // dL (.) Gamma (.) k_r.k_i, the beta-derivative of L
-    for (int x = tid; x < C * C; x += kThreads) {
+    for (int x = tid; x < C * C; x += NT) {
         const int r2 = x / C, i = x % C;
         float F = 0.f, E = 0.f, dmg = 0.f, dgv = 0.f;
         if (r2 < Cn && i <= r2) {
@@ -877,7 +883,7 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
             const float dm0 = dMs[r0 * Cp + i], dm1 = dMs[r1 * Cp + i];
 #pragma unroll
             for (int m = 0; m < MK; ++m) {
-                const float kv = Ks[i * dkp + c8 + 8 * m];
+                const float kv = Ks[i * dkp + cg + NG * m];
                 A1[0][m] += dm0 * kv;
                 A1[1][m] += dm1 * kv;
             }
@@ -895,7 +901,7 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
             const float dm0 = dMs[r2 * Cp + r0], dm1 = dMs[r2 * Cp + r1];   // dm1 = 0 at r2 = r0
 #pragma unroll
             for (int m = 0; m < MK; ++m) {
-                const float qv = Qs[r2 * dkp + c8 + 8 * m];
+                const float qv = Qs[r2 * dkp + cg + NG * m];
                 A3[0][m] += dm0 * qv;
                 A3[1][m] += dm1 * qv;
             }
@@ -905,7 +911,7 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
             const float g1 = dLs[r1 * Cp + i] + dLs[i * Cp + r1];
 #pragma unroll
             for (int m = 0; m < MK; ++m) {
-                const float kv = Ks[i * dkp + c8 + 8 * m];
+                const float kv = Ks[i * dkp + cg + NG * m];
                 A3[0][m] += g0 * kv;
                 A3[1][m] += g1 * kv;
             }
@@ -916,8 +922,8 @@ __global__ void __launch_bounds__(kThreads) bwd_grad_kernel(const BwdParams p) {
                 const size_t out = tok_index(p, b, t0 + r0 + e, h) * DK;
 #pragma unroll
                 for (int m = 0; m < MK; ++m) {
-                    p.grad_q[out + c8 + 8 * m] = A1[e][m];
-                    p.grad_k[out + c8 + 8 * m] = A3[e][m];
+                    p.grad_q[out + cg + NG * m] = A1[e][m];
+                    p.grad_k[out + cg + NG * m] = A3[e][m];
                 }
             }
         }

@@ -79,10 +79,10 @@ extern "C" int host_bwd(int B, int T, int H, int dk, int dv, int C, int io_bf16,
     run_grid(bwd::bwd_state_rev_kernel, per_slice, p, bwd::state_rev_smem_floats(C, dk));
     const size_t gs = bwd::grad_smem_floats(C, dk);
     switch (dk) {
-        case 16: run_grid(bwd::bwd_grad_kernel<16>, per_chunk, p, gs); break;
-        case 32: run_grid(bwd::bwd_grad_kernel<32>, per_chunk, p, gs); break;
-        case 64: run_grid(bwd::bwd_grad_kernel<64>, per_chunk, p, gs); break;
-        case 128: run_grid(bwd::bwd_grad_kernel<128>, per_chunk, p, gs); break;
+        case 16: run_grid(bwd::bwd_grad_kernel<16>, per_chunk, p, gs, bwd::kGradThreads); break;
+        case 32: run_grid(bwd::bwd_grad_kernel<32>, per_chunk, p, gs, bwd::kGradThreads); break;
+        case 64: run_grid(bwd::bwd_grad_kernel<64>, per_chunk, p, gs, bwd::kGradThreads); break;
+        case 128: run_grid(bwd::bwd_grad_kernel<128>, per_chunk, p, gs, bwd::kGradThreads); break;
         default: return 1;
     }
     return g_overrun ? 100 + g_overrun : 0;
