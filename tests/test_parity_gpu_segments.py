@@ -186,3 +186,33 @@ def test_segments_long_context_bf16_output():
     report("segments_long_context_bf16_o", o=stats(got, o_ref), S_T=stats(S.double().cpu().numpy(), s_ref))
     assert bf16_allowance_ok(got, o_ref)
     assert stats(S.double().cpu().numpy(), s_ref)["max_rel_rms"] <= TOL_BF16_REL_RMS
+
+
+@pytest.mark.gpu
+@needs_cuda
+def test_segments_residual_mode_and_narrow_values():
+    """The residual-corrected series through the segments (against its chunk model),
+    and d_v = 64 (one value slice per head) without a final state."""
+    w = workload("gdn_bf16", B=1, H=3, T=64 * 33 + 9, decay="weak", s0_std=0.02)
+    x = make_inputs(w, seed=45)
+    d = {k: (None if v is None else v.to("cuda").contiguous()) for k, v in x.items()}
+    o, S = gdn.chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S0=d["S0"], chunk=64, mode="residual",
+                         N=3, S=8, o_dtype=torch.float32, kernel="tc_split", segments=3)
+    torch.cuda.synchronize()
+    o_ref, s_ref = cf.chunked_gated_delta_fwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"], chunk=64,
+                                              inverse=cf.residual_inverse(3, 8))
+    _check("segments_residual", o, S, o_ref, s_ref)
+
+    w64 = workload("gdn_bf16", B=1, H=5, T=64 * 40, dv=64, decay="none", s0_std=0.02)
+    x = make_inputs(w64, seed=46)
+    d = {k: (None if v is None else v.to("cuda").contiguous()) for k, v in x.items()}
+    a = _args(T=w64.T, H=5, dv=64, seq_segments=3)
+    assert gdn.select_segments(a) == 3
+    o, S = gdn.chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S0=d["S0"], chunk=64,
+                         o_dtype=torch.float32, kernel="tc_split", segments=3, final_state=False)
+    torch.cuda.synchronize()
+    assert S is None
+    o_ref, _ = oracle.gated_delta_fwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"])
+    so = stats(o.double().cpu().numpy(), o_ref)
+    report("segments_dv64_no_state", o=so)
+    assert so["max_rel_rms"] <= TOL_BF16_REL_RMS, so
