@@ -354,6 +354,8 @@ gdn_status gdn_chunk_fwd_static_scratch(const gdn_fwd_args *args, void *stream) 
     if (s != GDN_OK) return s;
     if (args->workspace || args->workspace_bytes)
         return fail(GDN_ERR_INVALID_ARG, "the fixed-scratch entry point takes no workspace (pass NULL, 0)");
+    if (args->seq_segments == 3)
+        return fail(GDN_ERR_UNSUPPORTED, "the fixed-scratch entry point runs one pass over the chunks (seq_segments 0 or 1)");
     p.segments = 1;     // one pass: the segment schedule's streams and states are not for this entry
     const size_t need = gdn::tc_workspace_bytes(p);
     if (need > (size_t)GDN_STATIC_SCRATCH_BYTES)

@@ -325,11 +325,13 @@ GDN_API uint64_t gdn_bwd_workspace_bytes(const gdn_bwd_args *args);
  * nothing (no cudaMalloc, cudaFree or allocating library routine).
  *
  * Arguments as gdn_chunk_fwd, except: args->workspace must be NULL and
- * args->workspace_bytes 0; args->kernel must be AUTO, TC or TC_SPLIT and the
- * shape one the split tensor-core kernels support, else GDN_ERR_UNSUPPORTED
- * (whatever the kernel field, this entry point runs the split kernels); and
- * the workspace the call needs there (gdn_workspace_bytes with kernel
- * TC_SPLIT: B * H * ceil(T / 64) * 24576 for the scalar rule at C = 64) must
+ * args->workspace_bytes 0; the call runs one pass over the chunks (seq_segments
+ * 3 returns GDN_ERR_UNSUPPORTED, 0 means one pass here); args->kernel must be
+ * AUTO, TC or TC_SPLIT and the shape one the split tensor-core kernels support,
+ * else GDN_ERR_UNSUPPORTED (whatever the kernel field, this entry point runs
+ * the split kernels); and the workspace the call needs there
+ * (gdn_workspace_bytes with kernel TC_SPLIT and seq_segments 1:
+ * B * H * ceil(T / 64) * 24576 for the scalar rule at C = 64) must
  * be <= GDN_STATIC_SCRATCH_BYTES, else GDN_ERR_INVALID_ARG with the needed
  * size in gdn_last_error().  Nothing in the scratch has to start at zero: the
  * call's first kernels write every entry the chain kernel reads.

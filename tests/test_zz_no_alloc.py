@@ -39,6 +39,9 @@ def test_static_scratch_rejects_oversize_and_workspace():
     a.workspace, a.workspace_bytes = None, 0
     a.kernel = 1                                             # SIMT is not this entry point's kernel
     assert G.lib().gdn_chunk_fwd_static_scratch(ctypes.byref(a), None) == G.GDN_ERR_UNSUPPORTED
+    a.kernel = 2
+    a.T, a.H, a.seq_segments = 64 * 300, 1, 3                # sequence segments: not this entry point's
+    assert G.lib().gdn_chunk_fwd_static_scratch(ctypes.byref(a), None) == G.GDN_ERR_UNSUPPORTED
 
 
 def _free_bytes():
