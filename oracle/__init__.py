@@ -15,6 +15,9 @@ Contents
                 the parallel residual correction) and a plain fp64 chunked
                 forward that takes the inverse as a parameter, written with
                 numpy.
+``chunk_grad``  the gradient of the chunked form with the masked truncated
+                Neumann inverse: the chunk model written in plain fp64
+                PyTorch ops, differentiated by autograd.
 """
-from . import chunk_forms, recurrent  # noqa: F401
+from . import chunk_forms, chunk_grad, recurrent  # noqa: F401
 from .recurrent import gated_delta_bwd, gated_delta_fwd, precond_two_gate_fwd  # noqa: F401

@@ -159,3 +159,63 @@ def test_gradient_is_linear_in_the_cotangents():
     g12 = rec.gated_delta_bwd(do=do1 + 2 * do2, dhT=dh1 + 2 * dh2, **x)
     for n in ("dq", "dk", "dv", "dalpha", "dbeta", "dh0"):
         np.testing.assert_allclose(g12[n], g1[n] + 2 * g2[n], atol=1e-12, err_msg=n)
+
+
+# ------------------------------------------- masked Neumann series (chunk model)
+
+from oracle import chunk_forms as cf  # noqa: E402
+from oracle import chunk_grad as cg  # noqa: E402
+
+
+def test_neumann_chunk_model_forward_matches_numpy_chunk_model():
+    """The autograd oracle's forward is the numpy chunk model with the masked
+    series, operation for operation."""
+    rng = np.random.default_rng(11)
+    x, _, _ = _inputs(rng, T=21, dk=6, dv=5)
+    o1, s1 = cg.neumann_fwd(chunk=8, N=2, **x)
+    o2, s2 = cf.chunked_gated_delta_fwd(chunk=8, inverse=cf.neumann_inverse(2), **x)
+    assert np.abs(o1 - o2).max() <= 1e-12 and np.abs(s1 - s2).max() <= 1e-12
+
+
+@pytest.mark.parametrize("gates", [True, False])
+def test_neumann_gradient_at_full_order_is_the_exact_adjoint(gates):
+    """At N = C - 1 the masked series is the exact inverse (A is nilpotent), so
+    the chunk model's gradient must equal the token-by-token adjoint."""
+    rng = np.random.default_rng(12)
+    x, do, dhT = _inputs(rng, T=19, dk=5, dv=4, gates=gates)
+    C = 8
+    g = cg.neumann_bwd(do=do, dhT=dhT, chunk=C, N=C - 1, **x)
+    ref = rec.gated_delta_bwd(do=do, dhT=dhT, **x)
+    for name, key in (("dq", "dq"), ("dk", "dk"), ("dv", "dv"), ("dalpha", "dalpha"), ("dbeta", "dbeta"),
+                      ("dh0", "dh0")):
+        if ref[key] is None:
+            assert g[name] is None
+            continue
+        assert np.abs(g[name] - ref[key]).max() <= 1e-9 * max(1.0, np.abs(ref[key]).max()), name
+
+
+def test_neumann_gradient_matches_finite_differences():
+    """N = 2 (the series truncated well below the chunk length): central finite
+    differences of the numpy chunk model, element by element on a sample."""
+    rng = np.random.default_rng(13)
+    x, do, dhT = _inputs(rng, T=13, dk=4, dv=3)
+    C, N = 8, 2
+    g = cg.neumann_bwd(do=do, dhT=dhT, chunk=C, N=N, **x)
+
+    def loss(xx):
+        o, hT = cf.chunked_gated_delta_fwd(chunk=C, inverse=cf.neumann_inverse(N), **xx)
+        return float((o * do).sum() + (hT * dhT).sum())
+
+    for name, key in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("alpha", "dalpha"), ("beta", "dbeta"),
+                      ("h0", "dh0")):
+        arr = x[name]
+        for flat in rng.choice(arr.size, size=6, replace=False):
+            idx = np.unravel_index(flat, arr.shape)
+            xp = dict(x)
+            xp[name] = arr.copy()
+            xp[name][idx] += 1e-6
+            lp = loss(xp)
+            xp[name][idx] -= 2e-6
+            lm = loss(xp)
+            fd = (lp - lm) / 2e-6
+            assert abs(g[key][idx] - fd) <= 1e-6 * max(1.0, abs(fd)), (name, idx, g[key][idx], fd)
