@@ -25,6 +25,7 @@ bool bwd_supports(const BwdParams &p, const char **why) {
     if (p.C != 16 && p.C != 32 && p.C != 64) { *why = "chunk must be 16, 32 or 64"; return false; }
     if (p.dk != 16 && p.dk != 32 && p.dk != 64 && p.dk != 128) { *why = "dk must be 16, 32, 64 or 128"; return false; }
     if (p.dv % bwd::kCols != 0 || p.dv > 128) { *why = "dv must be 32, 64, 96 or 128"; return false; }
+    if (p.neumann && (p.N < 0 || p.N > p.C - 1)) { *why = "neumann_N must be in [0, chunk - 1]"; return false; }
     return true;
 }
 
@@ -32,7 +33,7 @@ size_t bwd_workspace_bytes(const BwdParams &p) {
     const size_t nch = (size_t)p.B * p.H * p.NC;
     const size_t C = p.C, dk = p.dk, dv = p.dv;
     return region(C, nch) + 3 * region(C * C, nch) + region(C * dk, nch) + 2 * region(C * dv, nch) +
-           3 * region(dk * dv, nch);
+           3 * region(dk * dv, nch) + (p.neumann ? region(C * C, nch) : 0);
 }
 
 void bwd_carve_workspace(BwdParams &p, void *workspace) {
@@ -48,7 +49,8 @@ void bwd_carve_workspace(BwdParams &p, void *workspace) {
     p.ws_Y = reinterpret_cast<float *>(w);  w += region(C * dv, nch);
     p.ws_P = reinterpret_cast<float *>(w);  w += region(dk * dv, nch);
     p.ws_h = reinterpret_cast<float *>(w);  w += region(dk * dv, nch);
-    p.ws_dh = reinterpret_cast<float *>(w);
+    p.ws_dh = reinterpret_cast<float *>(w);  w += region(dk * dv, nch);
+    p.ws_dA = p.neumann ? reinterpret_cast<float *>(w) : nullptr;
 }
 
 cudaError_t launch_bwd(const BwdParams &p, cudaStream_t stream) {
@@ -61,6 +63,11 @@ cudaError_t launch_bwd(const BwdParams &p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     e = launch_one(bwd::bwd_state_rev_kernel, per_slice, bwd::state_rev_smem_floats(p.C, p.dk), p, stream);
     if (e != cudaSuccess) return e;
+    if (p.neumann) {
+        e = launch_one(bwd::bwd_neumann_kernel, per_chunk, bwd::neumann_smem_floats(p.C, p.dv), p, stream,
+                       bwd::kPrepThreads);
+        if (e != cudaSuccess) return e;
+    }
     const size_t gs = bwd::grad_smem_floats(p.C, p.dk);
     switch (p.dk) {
         case 16: return launch_one(bwd::bwd_grad_kernel<16>, per_chunk, gs, p, stream, bwd::kGradThreads);

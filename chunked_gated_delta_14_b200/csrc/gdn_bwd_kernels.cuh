@@ -162,6 +162,50 @@ __device__ __forceinline__ void block_product(const float *A, int ra, int ia, in
     }
 }
 
+// T = (I + L)^-1 for strictly lower L (C x C in shared memory, row stride Cp),
+// blocked: the 16 x 16 diagonal blocks by forward substitution (one column per
+// thread; each solved entry updates the rows below it), then the merges
+// 16 -> 32 -> 64 of neighbouring blocks, T21 = -T22 L21 T11, with every thread.
+// T must be zero on entry (the blocks above the diagonal stay zero); Ys holds
+// C * C / 4 floats of scratch.  Ends with a barrier.
+template <int NT>
+__device__ __forceinline__ void block_inverse(const float *Ls, float *Ts, float *Ys, int C, int Cp, int tid) {
+    if (tid < C) {
+        const int c = tid, base = c & ~15, jc = c & 15;
+        float acc[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) acc[r] = (r == jc) ? 1.f : 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float xi = acc[i];
+#pragma unroll
+            for (int r = i + 1; r < 16; ++r) acc[r] -= Ls[(base + r) * Cp + base + i] * xi;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Ts[(base + r) * Cp + c] = acc[r];
+    }
+    __syncthreads();
+    for (int sz = 16; sz < C; sz *= 2) {
+        const int work = (C / (2 * sz)) * sz * sz;      // outputs of one product, all pairs
+        for (int o = tid; o < work; o += NT) {
+            const int pr = o / (sz * sz), rr = (o / sz) % sz, cc = o % sz;
+            const int b0 = 2 * sz * pr, b1 = b0 + sz;
+            float y = 0.f;
+            for (int k = 0; k < sz; ++k) y += Ls[(b1 + rr) * Cp + b0 + k] * Ts[(b0 + k) * Cp + b0 + cc];
+            Ys[o] = y;
+        }
+        __syncthreads();
+        for (int o = tid; o < work; o += NT) {
+            const int pr = o / (sz * sz), rr = (o / sz) % sz, cc = o % sz;
+            const int b0 = 2 * sz * pr, b1 = b0 + sz;
+            float z = 0.f;
+            for (int k = 0; k < sz; ++k) z += Ts[(b1 + rr) * Cp + b1 + k] * Ys[pr * sz * sz + k * sz + cc];
+            Ts[(b1 + rr) * Cp + b0 + cc] = -z;
+        }
+        __syncthreads();
+    }
+}
+
 // ------------------------------------------------------------------- prep
 // One block per chunk-head.  Shared memory (floats): K, Q (C x (dk+1)),
 // V and then dO (C x (dv+1)), L, T, M (C x (C+1)), g, beta, beta e^g, e^g (C each).
@@ -277,48 +321,27 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(const BwdParams 
     }
     __syncthreads();
 
-    // T = (I + L)^-1, blocked: the 16 x 16 diagonal blocks by forward substitution
-    // (one column per thread; each solved entry updates the rows below it), then
-    // the merges 16 -> 32 -> 64 of neighbouring blocks, T21 = -T22 L21 T11, with
-    // every thread.  T starts at zero, so the blocks above the diagonal stay zero.
-    // Rows past the tail have zero L rows; their diagonal is cleared at the end, so
-    // that T is zero outside the sequence as the chains expect.
-    if (tid < C) {
-        const int c = tid, base = c & ~15, jc = c & 15;
-        float acc[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) acc[r] = (r == jc) ? 1.f : 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float xi = acc[i];
-#pragma unroll
-            for (int r = i + 1; r < 16; ++r) acc[r] -= Ls[(base + r) * Cp + base + i] * xi;
-        }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) Ts[(base + r) * Cp + c] = acc[r];
-    }
-    __syncthreads();
-    for (int sz = 16; sz < C; sz *= 2) {
-        const int work = (C / (2 * sz)) * sz * sz;      // outputs of one product, all pairs
-        for (int o = tid; o < work; o += kPrepThreads) {
-            const int pr = o / (sz * sz), rr = (o / sz) % sz, cc = o % sz;
-            const int b0 = 2 * sz * pr, b1 = b0 + sz;
-            float y = 0.f;
-            for (int k = 0; k < sz; ++k) y += Ls[(b1 + rr) * Cp + b0 + k] * Ts[(b0 + k) * Cp + b0 + cc];
-            Ys[o] = y;
-        }
-        __syncthreads();
-        for (int o = tid; o < work; o += kPrepThreads) {
-            const int pr = o / (sz * sz), rr = (o / sz) % sz, cc = o % sz;
-            const int b0 = 2 * sz * pr, b1 = b0 + sz;
-            float z = 0.f;
-            for (int k = 0; k < sz; ++k) z += Ts[(b1 + rr) * Cp + b1 + k] * Ys[pr * sz * sz + k * sz + cc];
-            Ts[(b1 + rr) * Cp + b0 + cc] = -z;
-        }
-        __syncthreads();
-    }
+    block_inverse<kPrepThreads>(Ls, Ts, Ys, C, Cp, tid);
+    // Rows past the tail have zero L rows; their diagonal is cleared, so that T is
+    // zero outside the sequence as the chains expect.
     if (tid < C && tid >= Cn) Ts[tid * Cp + tid] = 0.f;
     __syncthreads();
+    if (p.neumann) {
+        // The masked truncated series M^(N) (.) sum_{n<=N} A^n: A is strictly lower,
+        // so A^n vanishes within n - 1 of the diagonal and the series agrees with the
+        // exact inverse on the band i - j <= N; outside it the mask gives zero.  The
+        // exact inverse goes to the adjoint kernel, which needs it for the gradient.
+        for (int x = tid; x < C * C; x += kPrepThreads) {
+            const int r = x / C, c = x % C;
+            p.ws_dA[ch * C * C + x] = Ts[r * Cp + c];
+        }
+        __syncthreads();
+        for (int x = tid; x < C * C; x += kPrepThreads) {
+            const int r = x / C, c = x % C;
+            if (r - c > p.N) Ts[r * Cp + c] = 0.f;
+        }
+        __syncthreads();
+    }
 
     for (int x = tid; x < C * C; x += kPrepThreads) p.ws_T[ch * C * C + x] = Ts[(x / C) * Cp + x % C];
     if (tid < C) p.ws_g[ch * C + tid] = g[tid];
@@ -337,6 +360,108 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(const BwdParams 
                                                            p.ws_Y + ch * C * dv, tid);
     block_product<128 / 16, kPrepThreads>(Qs, 1, dkp, dk, Cn, eg, dOs, dvp, dv,
                                                          p.ws_P + ch * dk * dv, tid);
+}
+
+// ------------------------------------------------- masked-series adjoint
+// With the masked truncated series T_N = M^(N) (.) sum_{n<=N} A^n as the chunk
+// inverse ("Quando o 'Bom o Suficiente' e Otimo ...", section "Metodologia",
+// items 1 and 2), the gradient reaching L differs from the exact inverse's
+// -Y Delta^T.  Per chunk-head, from the reverse chain's Y = T_N^T dDelta and the
+// forward chain's Delta = T_N R (R = diag(beta) V - diag(beta e^g) K h):
+//   dT_N = dDelta R^T = T_N^-T (Y Delta^T) T_N^-T;
+// T_N equals M (.) (I - A)^-1 for every strictly lower A (the series and the
+// exact inverse agree on the band, the mask zeroes the rest), so
+//   dA = T^T (M (.) dT_N) T^T,  T = (I - A)^-1 exact,  dL = -dA,
+// written to ws_dA (over the exact inverse the prep left there) for the
+// key-side gradient kernel.  All products C x C (the first over d_v), fp32.
+__host__ __device__ inline size_t neumann_smem_floats(int C, int dv) {
+    return 2 * (size_t)C * (dv + 1) + 5 * (size_t)C * (C + 1) + (size_t)C * C / 4;
+}
+
+// out(r, c) = sum_{k < K} A(r, k) B(k, c) for r, c < C, A(r, k) = A[r ra + k ia],
+// B(k, c) = B[k rb + c ib], out(r, c) = out[r os + c].  4 x 4 register tiles,
+// two lanes per tile on the even and odd k, summed with a shuffle.  Ends with a
+// barrier.
+template <int NT>
+__device__ __forceinline__ void tile_product(const float *A, int ra, int ia, const float *B, int rb, int ib, int K,
+                                             float *out, int os, int C, int tid) {
+    const int nt = C / 4, items = 2 * nt * nt;
+    for (int w = tid; w < items; w += NT) {
+        const int part = w & 1, t = w >> 1;
+        const int r0 = 4 * (t / nt), c0 = 4 * (t % nt);
+        float acc[4][4] = {};
+        for (int k = part; k < K; k += 2) {
+            float a[4], bb[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                a[e] = A[(r0 + e) * ra + k * ia];
+                bb[e] = B[k * rb + (c0 + e) * ib];
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+#pragma unroll
+                for (int f = 0; f < 4; ++f) acc[e][f] += a[e] * bb[f];
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+#pragma unroll
+            for (int f = 0; f < 4; ++f) acc[e][f] += __shfl_xor_sync(0xffffffffu, acc[e][f], 1);
+        if (part == 0) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+#pragma unroll
+                for (int f = 0; f < 4; ++f) out[(r0 + e) * os + c0 + f] = acc[e][f];
+        }
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(kPrepThreads) bwd_neumann_kernel(const BwdParams p) {
+    constexpr int NT = kPrepThreads;
+    float *sm = reinterpret_cast<float *>(bwd_smem);
+    const int C = p.C, dv = p.dv, dvp = dv + 1, Cp = C + 1;
+    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+    const size_t ch = ((size_t)b * p.H + h) * p.NC + n;
+    float *Yt = sm;                 // Y, C x dv
+    float *Dt = Yt + C * dvp;       // Delta, C x dv
+    float *Ss = Dt + C * dvp;       // Y Delta^T, then M (.) dT_N
+    float *Bs = Ss + C * Cp;        // T_N without its diagonal
+    float *Ti = Bs + C * Cp;        // T_N^-1
+    float *Tx = Ti + C * Cp;        // the exact inverse
+    float *Tm = Tx + C * Cp;        // products in between
+    float *Ys = Tm + C * Cp;        // scratch of the inverse, C * C / 4
+
+    for (int x = tid; x < C * dv / 4; x += NT) {
+        const int r = 4 * x / dv, c = 4 * x % dv;
+        const float4 y = *reinterpret_cast<const float4 *>(p.ws_Y + ch * C * dv + 4 * x);
+        const float4 d = *reinterpret_cast<const float4 *>(p.ws_D + ch * C * dv + 4 * x);
+        float *yr = Yt + r * dvp + c, *dr = Dt + r * dvp + c;
+        yr[0] = y.x; yr[1] = y.y; yr[2] = y.z; yr[3] = y.w;
+        dr[0] = d.x; dr[1] = d.y; dr[2] = d.z; dr[3] = d.w;
+    }
+    for (int x = tid; x < C * C; x += NT) {
+        const int r = x / C, c = x % C;
+        const float tn = p.ws_T[ch * C * C + x];
+        Bs[r * Cp + c] = c < r ? tn : 0.f;      // rows past the tail are zero: T_N^-1 is 1 there
+        Ti[r * Cp + c] = 0.f;
+        Tx[r * Cp + c] = p.ws_dA[ch * C * C + x];
+    }
+    __syncthreads();
+    // S = Y Delta^T (over d_v), T_N^-1
+    tile_product<NT>(Yt, dvp, 1, Dt, 1, dvp, dv, Ss, Cp, C, tid);
+    block_inverse<NT>(Bs, Ti, Ys, C, Cp, tid);
+    // dT_N = T_N^-T S T_N^-T, masked to the band (its entries farther below the
+    // diagonal are not functions of A; those above it add nothing to the lower dA)
+    tile_product<NT>(Ss, Cp, 1, Ti, 1, Cp, C, Tm, Cp, C, tid);     // S T_N^-T
+    tile_product<NT>(Ti, 1, Cp, Tm, Cp, 1, C, Ss, Cp, C, tid);     // T_N^-T (S T_N^-T)
+    for (int x = tid; x < C * C; x += NT) {
+        const int r = x / C, c = x % C;
+        if (r - c > p.N) Ss[r * Cp + c] = 0.f;
+    }
+    __syncthreads();
+    // dA = T^T G T^T with the exact inverse, to the workspace
+    tile_product<NT>(Ss, Cp, 1, Tx, 1, Cp, C, Tm, Cp, C, tid);     // G T^T
+    tile_product<NT>(Tx, 1, Cp, Tm, Cp, 1, C, p.ws_dA + ch * C * C, C, C, tid);
 }
 
 // ------------------------------------------------------ forward state chain
@@ -654,9 +779,12 @@ __global__ void __launch_bounds__(kGradThreads) bwd_grad_kernel(const BwdParams 
     const size_t ch = ((size_t)b * p.H + h) * p.NC + n;
 
     load_rows<NT>(p, b, h, t0, C, Cn, DK, dkp, p.k, p.io_bf16, Ks, p.q, p.io_bf16, Qs, tid);
+    // dLs accumulates -dL: Y Delta^T over the value tiles, or (masked series) the
+    // adjoint kernel's dA
     for (int x = tid; x < C * Cp; x += NT) {
+        const int r = x / Cp, c = x % Cp;
         dMs[x] = 0.f;
-        dLs[x] = 0.f;
+        dLs[x] = (p.neumann && c < C) ? p.ws_dA[ch * C * C + r * C + c] : 0.f;
     }
     if (tid < C) {
         const float gv = p.ws_g[ch * C + tid];
@@ -767,10 +895,10 @@ __global__ void __launch_bounds__(kGradThreads) bwd_grad_kernel(const BwdParams 
                 const int i = cg + NG * m;
                 if (i < Cn) {
                     dMs[r0 * Cp + i] += s1[0][m];
-                    dLs[r0 * Cp + i] += s2[0][m];
+                    if (!p.neumann) dLs[r0 * Cp + i] += s2[0][m];
                     if (v1) {
                         dMs[r1 * Cp + i] += s1[1][m];
-                        dLs[r1 * Cp + i] += s2[1][m];
+                        if (!p.neumann) dLs[r1 * Cp + i] += s2[1][m];
                     }
                 }
             }

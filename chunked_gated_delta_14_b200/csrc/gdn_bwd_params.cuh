@@ -18,6 +18,7 @@ struct BwdParams {
     const float *grad_S_T;        // [B, H, dk, dv] or null (=> 0)
     float *grad_q, *grad_k, *grad_v;
     float *grad_alpha, *grad_beta, *grad_S0;   // each may be null
+    int neumann, N;               // chunk inverse: 0 exact; 1 the masked truncated series of order N
     // Workspace regions, fp32, each indexed by chunk-head (b*H + h)*NC + n:
     float *ws_g;    // C        in-chunk cumulative log decay g
     float *ws_T;    // C x C    T = (I + L)^-1
@@ -30,6 +31,7 @@ struct BwdParams {
     float *ws_P;    // dk x dv  (diag(e^g) Q)^T dO
     float *ws_h;    // dk x dv  state h = S^T at the chunk's start
     float *ws_dh;   // dk x dv  dL/dh at the chunk's end
+    float *ws_dA;   // C x C    masked series only: the exact inverse (prep), then dA = -dL
 };
 
 // fp32 words of workspace per chunk-head.

@@ -80,7 +80,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 8
+#define GDN_ABI_VERSION 9
 
 #if defined(__GNUC__)
 #define GDN_API __attribute__((visibility("default")))
@@ -274,6 +274,15 @@ GDN_API int32_t gdn_abi_version(void);
  * The forward is recomputed inside the call (only S0 is taken from the
  * caller), so the call needs no saved activations.
  *
+ * With mode GDN_INV_NEUMANN it is the gradient of the forward whose chunk
+ * inverse is the masked truncated series T_N = M^(N) (.) sum_{n<=N} A^n (same
+ * page, section "Metodologia", items 1 and 2): launch 1 forms T_N (on the band
+ * it equals the exact inverse, off it the mask gives zero) and keeps the exact
+ * inverse, and a launch between 3 and 4 forms, per chunk-head,
+ * dA = T^T (M (.) dT_N) T^T with dT_N = T_N^-T (Y Delta^T) T_N^-T, the gradient
+ * reaching A = -L through the series (the workspace grows by C x C floats per
+ * chunk-head).  GDN_INV_NEUMANN_RESIDUAL returns GDN_ERR_INVALID_ARG.
+ *
  * Layouts as gdn_fwd_args; every gradient is fp32 in the layout of its input
  * (grad_S0 and grad_S_T in the h = S^T layout [B, H, dk, dv]).
  *
@@ -302,6 +311,10 @@ typedef struct {
     float *grad_S0;             /* [B,H,dk,dv] fp32 or NULL */
     void *workspace;            /* >= gdn_bwd_workspace_bytes(args) bytes, 16-byte aligned */
     uint64_t workspace_bytes;
+    int32_t mode;               /* the chunk inverse of the forward being differentiated:
+                                   GDN_INV_EXACT, or GDN_INV_NEUMANN (the masked truncated
+                                   series of order neumann_N, 0 <= N <= chunk - 1) */
+    int32_t neumann_N;
 } gdn_bwd_args;
 
 /* Backward pass (see above). */

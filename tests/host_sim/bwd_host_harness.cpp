@@ -47,8 +47,9 @@ static size_t region(size_t floats, size_t n) { return (floats * n * sizeof(floa
 extern "C" int host_bwd(int B, int T, int H, int dk, int dv, int C, int io_bf16, int do_bf16,
                         const void *q, const void *k, const void *v, const float *alpha,
                         const float *beta, const float *S0, const void *grad_o, const float *grad_S_T,
-                        float *gq, float *gk, float *gv, float *ga, float *gb, float *gS0) {
+                        float *gq, float *gk, float *gv, float *ga, float *gb, float *gS0, int neumann, int N) {
     BwdParams p{};
+    p.neumann = neumann; p.N = N;
     p.B = B; p.T = T; p.H = H; p.dk = dk; p.dv = dv; p.C = C; p.NC = (T + C - 1) / C;
     p.io_bf16 = io_bf16; p.do_bf16 = do_bf16;
     p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.beta = beta; p.S0 = S0;
@@ -57,7 +58,7 @@ extern "C" int host_bwd(int B, int T, int H, int dk, int dv, int C, int io_bf16,
     // the same regions, in the same order, as gdn::bwd_carve_workspace
     const size_t n = (size_t)B * H * p.NC, Cs = C, dks = dk, dvs = dv;
     const size_t bytes = region(Cs, n) + 3 * region(Cs * Cs, n) + region(Cs * dks, n) +
-                         2 * region(Cs * dvs, n) + 3 * region(dks * dvs, n);
+                         2 * region(Cs * dvs, n) + 3 * region(dks * dvs, n) + (neumann ? region(Cs * Cs, n) : 0);
     std::vector<char> ws(bytes);
     fill_nan(ws.data(), bytes);
     char *w = ws.data();
@@ -70,13 +71,15 @@ extern "C" int host_bwd(int B, int T, int H, int dk, int dv, int C, int io_bf16,
     p.ws_Y = reinterpret_cast<float *>(w);  w += region(Cs * dvs, n);
     p.ws_P = reinterpret_cast<float *>(w);  w += region(dks * dvs, n);
     p.ws_h = reinterpret_cast<float *>(w);  w += region(dks * dvs, n);
-    p.ws_dh = reinterpret_cast<float *>(w);
+    p.ws_dh = reinterpret_cast<float *>(w);  w += region(dks * dvs, n);
+    p.ws_dA = neumann ? reinterpret_cast<float *>(w) : nullptr;
     g_overrun = 0;
     const dim3h per_chunk{(unsigned)p.NC, (unsigned)H, (unsigned)B};
     const dim3h per_slice{(unsigned)(dv / bwd::kCols), (unsigned)H, (unsigned)B};
     run_grid(bwd::bwd_prep_kernel, per_chunk, p, bwd::prep_smem_floats(C, dk, dv), bwd::kPrepThreads);
     run_grid(bwd::bwd_state_fwd_kernel, per_slice, p, bwd::state_fwd_smem_floats(C, dk));
     run_grid(bwd::bwd_state_rev_kernel, per_slice, p, bwd::state_rev_smem_floats(C, dk));
+    if (neumann) run_grid(bwd::bwd_neumann_kernel, per_chunk, p, bwd::neumann_smem_floats(C, dv), bwd::kPrepThreads);
     const size_t gs = bwd::grad_smem_floats(C, dk);
     switch (dk) {
         case 16: run_grid(bwd::bwd_grad_kernel<16>, per_chunk, p, gs, bwd::kGradThreads); break;

@@ -25,7 +25,7 @@ def declared_functions():
 
 def test_library_builds_and_loads():
     gbuild.build()
-    assert gdn.abi_version() == 8
+    assert gdn.abi_version() == 9
 
 
 def test_exports_every_declared_symbol():

@@ -19,6 +19,7 @@ import numpy as np
 import pytest
 import torch
 
+from oracle import chunk_grad as cg
 from oracle import recurrent as rec
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -52,8 +53,28 @@ CASES = [  # B, T, H, dk, dv, C, gates, S0 and dS_T, bf16 inputs
 ]
 
 
+NEUMANN_CASES = [  # ..., N: the masked truncated series of order N as the chunk inverse
+    (1, 70, 2, 16, 32, 16, True, True, False, 2),
+    (1, 100, 1, 32, 96, 32, True, True, False, 3),
+    (1, 77, 1, 128, 128, 64, True, True, True, 4),
+    (2, 130, 1, 64, 32, 64, False, False, False, 1),
+    (1, 64, 1, 32, 32, 64, True, True, False, 63),
+]
+
+
 @pytest.mark.parametrize("B,T,H,dk,dv,C,gates,state,bf16", CASES)
 def test_backward_kernel_source_on_host(host_lib, B, T, H, dk, dv, C, gates, state, bf16):
+    _run_case(host_lib, B, T, H, dk, dv, C, gates, state, bf16, None)
+
+
+@pytest.mark.parametrize("B,T,H,dk,dv,C,gates,state,bf16,N", NEUMANN_CASES)
+def test_backward_kernel_source_on_host_masked_series(host_lib, B, T, H, dk, dv, C, gates, state, bf16, N):
+    """The gradient of the forward with the masked truncated series as the chunk
+    inverse, against the fp64 autograd of the chunk model (N = C - 1: exact)."""
+    _run_case(host_lib, B, T, H, dk, dv, C, gates, state, bf16, N)
+
+
+def _run_case(host_lib, B, T, H, dk, dv, C, gates, state, bf16, N):
     g = torch.Generator().manual_seed(B * 1000 + T)
     def nrm(*s):
         return torch.randn(*s, generator=g)
@@ -72,9 +93,12 @@ def test_backward_kernel_source_on_host(host_lib, B, T, H, dk, dv, C, gates, sta
     gb = nan(B, T, H) if gates else None
     rc = host_lib.host_bwd(B, T, H, dk, dv, C, int(bf16), int(bf16), _p(q), _p(k), _p(v), _p(alpha),
                            _p(beta), _p(S0), _p(do), _p(dS), _p(gq), _p(gk), _p(gv), _p(ga), _p(gb),
-                           _p(gS0))
+                           _p(gS0), ctypes.c_int(0 if N is None else 1), ctypes.c_int(N or 0))
     assert rc == 0, f"a block wrote past its shared memory ({rc - 100} blocks)" if rc >= 100 else rc
-    ref = rec.gated_delta_bwd(q, k, v, alpha, beta, S0, do, dS)
+    if N is None:
+        ref = rec.gated_delta_bwd(q, k, v, alpha, beta, S0, do, dS)
+    else:
+        ref = cg.neumann_bwd(q, k, v, alpha, beta, S0, do, dS, chunk=C, N=N)
     for name, got in (("dq", gq), ("dk", gk), ("dv", gv), ("dalpha", ga), ("dbeta", gb), ("dh0", gS0)):
         if ref[name] is None:
             continue

@@ -153,3 +153,44 @@ def test_autograd_function_matches_oracle():
             assert bf16_allowance_ok(got, r, rel_rms=TOL_BWD_REL_RMS), n
         else:
             assert stats(got, r)["max_rel_rms"] <= TOL_BWD_REL_RMS, n
+
+
+# ------------------------------------------- masked truncated Neumann series
+
+def _run_bwd_neumann(x, c, chunk, N):
+    d = {k: to_dev(v) for k, v in x.items()}
+    g = gdn.chunk_bwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], to_dev(c["grad_o"]),
+                      S0=d["S0"], grad_S_T=to_dev(c["grad_S_T"]), chunk=chunk, mode="neumann", N=N)
+    torch.cuda.synchronize()
+    return {k: None if v is None else v.double().cpu().numpy() for k, v in g.items()}
+
+
+@needs_cuda
+@pytest.mark.parametrize("chunk,N,T", [(64, 2, 300), (64, 3, 257), (64, 4, 64), (32, 3, 100), (16, 1, 37),
+                                       (64, 63, 200)])
+def test_backward_masked_series(chunk, N, T):
+    """The gradient of the forward whose chunk inverse is the masked truncated series
+    of order N, against the fp64 autograd of that chunk model (N = C - 1 is the exact
+    inverse); ragged tails, bf16 inputs, S0 and dS_T."""
+    from oracle import chunk_grad as cg
+    w = workload("gdn_bf16", B=1, H=2, T=T, chunk=chunk, decay="weak", s0_std=0.02)
+    x = make_inputs(w, seed=51)
+    c = make_cotangents(w, seed=51)
+    got = _run_bwd_neumann(x, c, chunk, N)
+    ref = cg.neumann_bwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"], c["grad_o"], c["grad_S_T"],
+                         chunk=chunk, N=N)
+    _compare(f"bwd_neumann_C{chunk}_N{N}_T{T}", got, ref)
+
+
+@needs_cuda
+def test_backward_masked_series_full_order_equals_exact():
+    """N = C - 1: the masked series is the exact inverse, so the two modes of the
+    kernels must agree to fp32 rounding."""
+    w = workload("gdn_bf16", B=2, H=3, T=333, decay="scalar", s0_std=0.02)
+    x = make_inputs(w, seed=52)
+    c = make_cotangents(w, seed=52)
+    gx = _run_bwd(x, c, 64)
+    gn = _run_bwd_neumann(x, c, 64, 63)
+    for k in ("dq", "dk", "dv", "dalpha", "dbeta", "dS0"):
+        rms = np.sqrt(np.mean(gx[k] ** 2))
+        assert np.abs(gn[k] - gx[k]).max() <= 1e-4 * rms, k
