@@ -423,14 +423,15 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
 
 
 class GatedDeltaRule(torch.autograd.Function):
-    """Differentiable gated delta rule: forward by ``chunk_fwd`` (exact
-    inverse), backward by ``chunk_bwd``; both run in libgdn.so."""
+    """Differentiable gated delta rule: forward by ``chunk_fwd``, backward by
+    ``chunk_bwd``, both with the same chunk inverse (``mode`` "exact" or
+    "neumann" of order ``N``); both run in libgdn.so."""
 
     @staticmethod
-    def forward(ctx, q, k, v, alpha, beta, S0, chunk):
-        o, S_T = chunk_fwd(q, k, v, alpha, beta, S0=S0, chunk=chunk)
+    def forward(ctx, q, k, v, alpha, beta, S0, chunk, mode="exact", N=3):
+        o, S_T = chunk_fwd(q, k, v, alpha, beta, S0=S0, chunk=chunk, mode=mode, N=N)
         ctx.save_for_backward(q, k, v, alpha, beta, S0)
-        ctx.chunk = chunk
+        ctx.chunk, ctx.mode, ctx.N = chunk, mode, N
         return o, S_T
 
     @staticmethod
@@ -440,12 +441,18 @@ class GatedDeltaRule(torch.autograd.Function):
             grad_o = torch.zeros(v.shape, device=v.device, dtype=torch.float32)
         g = chunk_bwd(q, k, v, alpha, beta, grad_o.contiguous(), S0=S0,
                       grad_S_T=None if grad_S_T is None else grad_S_T.float().contiguous(),
-                      chunk=ctx.chunk, want_S0=S0 is not None and ctx.needs_input_grad[5])
+                      chunk=ctx.chunk, want_S0=S0 is not None and ctx.needs_input_grad[5],
+                      mode=ctx.mode, N=ctx.N)
         cast = lambda t, like: None if t is None else t.to(like.dtype)
         return (cast(g["dq"], q), cast(g["dk"], k), cast(g["dv"], v), g["dalpha"], g["dbeta"],
-                g["dS0"], None)
+                g["dS0"], None, None, None)
 
 
-def gated_delta_rule(q, k, v, alpha=None, beta=None, S0=None, chunk: int = 64):
-    """``(o, S_T)`` of the gated delta rule with autograd support (see GatedDeltaRule)."""
-    return GatedDeltaRule.apply(q, k, v, alpha, beta, S0, chunk)
+def gated_delta_rule(q, k, v, alpha=None, beta=None, S0=None, chunk: int = 64, mode: str = "exact",
+                     N: int = 3):
+    """``(o, S_T)`` of the gated delta rule with autograd support (see GatedDeltaRule);
+    ``mode`` "neumann" uses the masked truncated series of order ``N`` as the chunk
+    inverse in both passes."""
+    if mode not in ("exact", "neumann"):
+        raise ValueError("gated_delta_rule: mode must be 'exact' or 'neumann'")
+    return GatedDeltaRule.apply(q, k, v, alpha, beta, S0, chunk, mode, N)
