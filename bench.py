@@ -762,9 +762,10 @@ def bwd_bytes(w):
     return w.token_heads * per_th
 
 
-def bwd_setup(w, x, c, dev):
+def bwd_setup(w, x, c, dev, mode="exact", N=3):
     """Device copies of the inputs and dL/do, fp32 gradient buffers and the
-    gdn_bwd_args (with workspace) of one backward call over the whole batch.
+    gdn_bwd_args (with workspace) of one backward call over the whole batch
+    (``mode`` "neumann": the gradient of the masked truncated series of order N).
     The args hold raw pointers: the returned dict keeps every tensor they point
     to alive."""
     import torch
@@ -780,21 +781,25 @@ def bwd_setup(w, x, c, dev):
                           do_dtype=1, q=ptr(d["q"]), k=ptr(d["k"]), v=ptr(d["v"]),
                           alpha=ptr(d["alpha"]), beta=ptr(d["beta"]), grad_o=ptr(grad_o),
                           grad_q=ptr(g["dq"]), grad_k=ptr(g["dk"]), grad_v=ptr(g["dv"]),
-                          grad_alpha=ptr(g["da"]), grad_beta=ptr(g["db"]))
+                          grad_alpha=ptr(g["da"]), grad_beta=ptr(g["db"]),
+                          mode=1 if mode == "neumann" else 0, neumann_N=int(N) if mode == "neumann" else 0)
     ws = gdn.workspace_for(a, dev)
     a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
     g["inputs"], g["grad_o"] = d, grad_o
     return a, g, ws
 
 
-def bwd_roofline(w, ms_step, sm_max_mhz):
+def bwd_roofline(w, ms_step, sm_max_mhz, neumann=False):
+    """ALU roofline of one backward call.  With the masked series the FLOP count is
+    the exact mode's (the adjoint kernel's C x C products are not counted) and no
+    traffic is reported (the committed capture is of the exact mode)."""
     pk = peaks()
     alu_peak = fp32_alu_peak_tflops(sm_max_mhz or 1965.0)
     flops = algorithmic_flops_bwd(w)
     achieved = flops / (ms_step / 1e3) / 1e12
     nbytes = bwd_bytes(w)
     return dict(bound="alu", achieved=achieved, peak=alu_peak, unit="TFLOP/s", frac=achieved / alu_peak,
-                traffic=profile_traffic("backward@gdn_bf16", BWD_SOURCES, units=w.B),
+                traffic=None if neumann else profile_traffic("backward@gdn_bf16", BWD_SOURCES, units=w.B),
                 peak_source="derived: 148 SMs x 128 fp32 lanes x 2 flops x max SM clock",
                 algorithmic_flops_per_launch=flops, algorithmic_bytes_per_launch=nbytes,
                 hbm_gbs=nbytes / (ms_step / 1e3) / 1e9, hbm_frac=nbytes / (ms_step / 1e3) / 1e9 / pk["hbm_gbs"],
@@ -846,7 +851,10 @@ def run_bwd(args, rank, world, local_rank):
     w = workload(WORKLOAD, **({"B": args.batch} if args.batch else {}))
     x = make_inputs(w, seed=rank)
     c = make_cotangents(w, seed=rank, grad_state=False)
-    a, g, ws = bwd_setup(w, x, c, dev)
+    neumann = args.mode == "neumann"
+    if args.mode == "residual":
+        raise SystemExit("bench.py --bwd: the backward takes --mode exact or neumann")
+    a, g, ws = bwd_setup(w, x, c, dev, mode=args.mode, N=args.N)
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
     for _ in range(args.warmup):
@@ -885,6 +893,7 @@ def run_bwd(args, rank, world, local_rank):
 
         def run(di, slot):
             r = gdn.chunk_bwd(di["q"], di["k"], di["v"], di["alpha"], di["beta"], di["grad_o"],
+                              mode="neumann" if neumann else "exact", N=args.N,
                               chunk=w.chunk, want_S0=False)
             return {k: r[k] for k in ("dq", "dk", "dv", "dalpha", "dbeta")}
 
@@ -902,23 +911,29 @@ def run_bwd(args, rank, world, local_rank):
 
     clk = clocks.summary()
     nbytes = bwd_bytes(w)
-    roof = bwd_roofline(w, ms_step, clk["sm_max_mhz"])
+    roof = bwd_roofline(w, ms_step, clk["sm_max_mhz"], neumann=neumann)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
         cores = len(os.sched_getaffinity(0))
-        Ts = min(w.T, 1024)
+        Ts = min(w.T, 256 if neumann else 1024)
         sl = lambda t: None if t is None else t[0:1, :Ts].contiguous()
         n, t0 = 0, time.perf_counter()
         while True:
-            oracle.gated_delta_bwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["alpha"]), sl(x["beta"]),
+            if neumann:
+                from oracle import chunk_grad
+                chunk_grad.neumann_bwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["alpha"]), sl(x["beta"]), None,
+                                       sl(c["grad_o"]), None, chunk=w.chunk, N=args.N)
+            else:
+                oracle.gated_delta_bwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["alpha"]), sl(x["beta"]),
                                    None, sl(c["grad_o"]), None, nthreads=cores)
             n += 1
             if time.perf_counter() - t0 >= min(args.cpu_budget, 10.0):
                 break
         el = time.perf_counter() - t0
-        cpu = dict(value=Ts * n / el, unit=UNIT, cores=cores, kind="oracle",
-                   sample=f"{n} x (tokens [0,{Ts}) of one batch row, all {w.H} heads), fp64 C adjoint, {el:.1f} s")
+        how = "fp64 autograd of the masked-series chunk model (torch CPU ops)" if neumann else "fp64 C adjoint"
+        cpu = dict(value=Ts * n / el, unit=UNIT, cores=torch.get_num_threads() if neumann else cores, kind="oracle",
+                   sample=f"{n} x (tokens [0,{Ts}) of one batch row, all {w.H} heads), {how}, {el:.1f} s")
     if rank == 0:
         line = dict(metric=BWD_METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps,
                     warmup=args.warmup, ms_per_step=ms_step, higher_is_better=True, scaling="weak",
@@ -926,13 +941,16 @@ def run_bwd(args, rank, world, local_rank):
                     compute="bf16 q/k/v/grad_o in HBM; fp32 arithmetic on CUDA cores; fp32 gradients",
                     data="synthetic (seeded; Gated DeltaNet layer shapes)",
                     config=dict(workload=f"{WORKLOAD} backward: B={w.B} H={w.H} T={w.T} dk={w.dk} "
-                                f"dv={w.dv} chunk={w.chunk} exact inverse",
+                                f"dv={w.dv} chunk={w.chunk} "
+                                + (f"masked truncated Neumann inverse N={args.N}" if neumann else "exact inverse"),
                                 global_batch=w.B * world, seq_len=w.T,
                                 parallelism=f"independent batch per GPU x{world}",
                                 l2=f"no flush: inputs+gradients {nbytes / 1e6:.0f} MB + workspace "
                                    f"{ws.numel() / 1e6:.0f} MB per step > 126 MB L2",
-                                kernel="bwd_prep_kernel+bwd_state_fwd_kernel+bwd_state_rev_kernel+bwd_grad_kernel"),
-                    clocks=clk, e2e=e2e, gpu_launches=args.steps * 4, roofline=roof, cpu_baseline=cpu)
+                                kernel="bwd_prep_kernel+bwd_state_fwd_kernel+bwd_state_rev_kernel+"
+                                       + ("bwd_neumann_kernel+" if neumann else "") + "bwd_grad_kernel"),
+                    clocks=clk, e2e=e2e, gpu_launches=args.steps * (5 if neumann else 4), roofline=roof,
+                    cpu_baseline=cpu)
         print(json.dumps(line), flush=True)
 
 
