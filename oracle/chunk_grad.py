@@ -16,6 +16,8 @@ Nothing here is shared with the CUDA library.
 """
 from __future__ import annotations
 
+from typing import Optional
+
 import numpy as np
 import torch
 
@@ -41,10 +43,25 @@ def masked_neumann(A: torch.Tensor, N: int) -> torch.Tensor:
     return torch.where(i - j <= N, total, torch.zeros_like(total))
 
 
-def chunk_model(q, k, v, log_alpha, beta, h0, chunk: int, N: int):
+def residual_corrected(A: torch.Tensor, N: int, S: int) -> torch.Tensor:
+    """T0 sum_{s=0}^{S} E^s with T0 the masked series and E = I - (I - A) T0
+    ("Metodologia", item 3)."""
+    k = A.shape[0]
+    eye = torch.eye(k, dtype=A.dtype)
+    T0 = masked_neumann(A, N)
+    E = eye - (eye - A) @ T0
+    power, acc = eye, eye
+    for _ in range(S):
+        power = power @ E
+        acc = acc + power
+    return T0 @ acc
+
+
+def chunk_model(q, k, v, log_alpha, beta, h0, chunk: int, N: int, S: Optional[int] = None):
     """o [B, T, H, dv] and h_T [B, H, dk, dv] of the chunked form with the masked
-    series of order N as the chunk inverse; every input a float64 tensor
-    (log_alpha and beta [B, T, H], h0 [B, H, dk, dv])."""
+    series of order N as the chunk inverse (with S residual-correction terms when S
+    is given); every input a float64 tensor (log_alpha and beta [B, T, H], h0
+    [B, H, dk, dv])."""
     B, Tn, H, dk = q.shape
     dv = v.shape[-1]
     outs, finals = [], []
@@ -66,7 +83,7 @@ def chunk_model(q, k, v, log_alpha, beta, h0, chunk: int, N: int):
                 # A_ri = -beta_r e^{g_r - g_i} (k_r . k_i), i < r
                 A = torch.where(below, -bet[:, None] * torch.exp(torch.where(below, diff, 0.0 * diff)) * (K @ K.T),
                                 torch.zeros(C, C, dtype=q.dtype))
-                Tm = masked_neumann(A, N)
+                Tm = masked_neumann(A, N) if S is None else residual_corrected(A, N, S)
                 U = Tm @ (bet[:, None] * V)
                 W = Tm @ ((bet * torch.exp(g))[:, None] * K)
                 Delta = U - W @ h
@@ -81,7 +98,7 @@ def chunk_model(q, k, v, log_alpha, beta, h0, chunk: int, N: int):
     return torch.stack(outs, 0), torch.stack(finals, 0)
 
 
-def neumann_fwd(q, k, v, alpha=None, beta=None, h0=None, chunk: int = 64, N: int = 3):
+def neumann_fwd(q, k, v, alpha=None, beta=None, h0=None, chunk: int = 64, N: int = 3, S: Optional[int] = None):
     """(o, h_T) as float64 numpy arrays."""
     q, k, v = _t(q), _t(k), _t(v)
     B, Tn, H, dk = q.shape
@@ -90,12 +107,14 @@ def neumann_fwd(q, k, v, alpha=None, beta=None, h0=None, chunk: int = 64, N: int
     bt = torch.ones(B, Tn, H, dtype=torch.float64) if beta is None else _t(beta)
     hz = torch.zeros(B, H, dk, dv, dtype=torch.float64) if h0 is None else _t(h0)
     with torch.no_grad():
-        o, hT = chunk_model(q, k, v, la, bt, hz, chunk, N)
+        o, hT = chunk_model(q, k, v, la, bt, hz, chunk, N, S)
     return o.numpy(), hT.numpy()
 
 
-def neumann_bwd(q, k, v, alpha=None, beta=None, h0=None, do=None, dhT=None, chunk: int = 64, N: int = 3):
-    """Gradients of L = <o, do> + <h_T, dhT> through the masked-series chunk model:
+def neumann_bwd(q, k, v, alpha=None, beta=None, h0=None, do=None, dhT=None, chunk: int = 64, N: int = 3,
+                S: Optional[int] = None):
+    """Gradients of L = <o, do> + <h_T, dhT> through the masked-series chunk model
+    (with S residual-correction terms when S is given):
     a dict with dq, dk, dv, dalpha, dbeta (None when that gate is None) and dh0,
     float64 numpy arrays in the layouts of the inputs."""
     q, k, v = _t(q), _t(k), _t(v)
@@ -109,7 +128,7 @@ def neumann_bwd(q, k, v, alpha=None, beta=None, h0=None, do=None, dhT=None, chun
         x.requires_grad_(True)
     la = torch.zeros(B, Tn, H, dtype=torch.float64) if a is None else torch.log(a)
     bb = torch.ones(B, Tn, H, dtype=torch.float64) if bt is None else bt
-    o, hT = chunk_model(q, k, v, la, bb, hz, chunk, N)
+    o, hT = chunk_model(q, k, v, la, bb, hz, chunk, N, S)
     loss = (o * _t(do)).sum()
     if dhT is not None:
         loss = loss + (hT * _t(dhT)).sum()

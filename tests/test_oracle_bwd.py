@@ -219,3 +219,49 @@ def test_neumann_gradient_matches_finite_differences():
             lm = loss(xp)
             fd = (lp - lm) / 2e-6
             assert abs(g[key][idx] - fd) <= 1e-6 * max(1.0, abs(fd)), (name, idx, g[key][idx], fd)
+
+
+def test_residual_chunk_model_forward_matches_numpy_chunk_model():
+    rng = np.random.default_rng(14)
+    x, _, _ = _inputs(rng, T=21, dk=6, dv=5)
+    o1, s1 = cg.neumann_fwd(chunk=8, N=2, S=3, **x)
+    o2, s2 = cf.chunked_gated_delta_fwd(chunk=8, inverse=cf.residual_inverse(2, 3), **x)
+    assert np.abs(o1 - o2).max() <= 1e-12 and np.abs(s1 - s2).max() <= 1e-12
+
+
+def test_residual_gradient_at_exact_orders_is_the_exact_adjoint():
+    """(N + 1)(S + 1) >= C makes the corrected series exact (the residual E
+    vanishes within (N + 1)(S + 1) of the diagonal), so the gradient must be the
+    token-by-token adjoint."""
+    rng = np.random.default_rng(15)
+    x, do, dhT = _inputs(rng, T=19, dk=5, dv=4)
+    g = cg.neumann_bwd(do=do, dhT=dhT, chunk=8, N=1, S=3, **x)
+    ref = rec.gated_delta_bwd(do=do, dhT=dhT, **x)
+    for name, key in (("dq", "dq"), ("dk", "dk"), ("dv", "dv"), ("dalpha", "dalpha"), ("dbeta", "dbeta"),
+                      ("dh0", "dh0")):
+        assert np.abs(g[name] - ref[key]).max() <= 1e-9 * max(1.0, np.abs(ref[key]).max()), name
+
+
+def test_residual_gradient_matches_finite_differences():
+    rng = np.random.default_rng(16)
+    x, do, dhT = _inputs(rng, T=13, dk=4, dv=3)
+    C, N, S = 8, 1, 1
+    g = cg.neumann_bwd(do=do, dhT=dhT, chunk=C, N=N, S=S, **x)
+
+    def loss(xx):
+        o, hT = cf.chunked_gated_delta_fwd(chunk=C, inverse=cf.residual_inverse(N, S), **xx)
+        return float((o * do).sum() + (hT * dhT).sum())
+
+    for name, key in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("alpha", "dalpha"), ("beta", "dbeta"),
+                      ("h0", "dh0")):
+        arr = x[name]
+        for flat in rng.choice(arr.size, size=6, replace=False):
+            idx = np.unravel_index(flat, arr.shape)
+            xp = dict(x)
+            xp[name] = arr.copy()
+            xp[name][idx] += 1e-6
+            lp = loss(xp)
+            xp[name][idx] -= 2e-6
+            lm = loss(xp)
+            fd = (lp - lm) / 2e-6
+            assert abs(g[key][idx] - fd) <= 1e-6 * max(1.0, abs(fd)), (name, idx, g[key][idx], fd)
