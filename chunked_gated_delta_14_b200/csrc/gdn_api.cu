@@ -202,13 +202,18 @@ gdn_status resolve_bwd(const gdn_bwd_args *a, gdn::BwdParams *out) {
         return fail(GDN_ERR_INVALID_ARG, "grad_q, grad_k and grad_v are required");
     if (a->grad_alpha && !a->alpha) return fail(GDN_ERR_INVALID_ARG, "grad_alpha needs alpha");
     if (a->grad_beta && !a->beta) return fail(GDN_ERR_INVALID_ARG, "grad_beta needs beta");
-    if (a->mode != GDN_INV_EXACT && a->mode != GDN_INV_NEUMANN)
-        return fail(GDN_ERR_INVALID_ARG, "backward mode must be GDN_INV_EXACT or GDN_INV_NEUMANN (got %d)", a->mode);
+    if (a->mode != GDN_INV_EXACT && a->mode != GDN_INV_NEUMANN && a->mode != GDN_INV_NEUMANN_RESIDUAL)
+        return fail(GDN_ERR_INVALID_ARG, "backward mode %d unknown", a->mode);
+    if (a->mode == GDN_INV_NEUMANN_RESIDUAL && (a->residual_S < 0 || a->residual_S > 64))
+        return fail(GDN_ERR_INVALID_ARG, "residual_S must be in [0, 64] (got %d)", a->residual_S);
     gdn::BwdParams p{};
     p.B = a->B; p.T = a->T; p.H = a->H; p.dk = a->dk; p.dv = a->dv; p.C = a->chunk;
     p.NC = (a->T + a->chunk - 1) / (a->chunk > 0 ? a->chunk : 1);
-    p.neumann = a->mode == GDN_INV_NEUMANN;
+    p.neumann = a->mode == GDN_INV_NEUMANN || a->mode == GDN_INV_NEUMANN_RESIDUAL;
     p.N = p.neumann ? a->neumann_N : 0;
+    // S = 0 terms of the correction leave the masked series itself
+    p.residual = a->mode == GDN_INV_NEUMANN_RESIDUAL && a->residual_S > 0;
+    p.S = p.residual ? a->residual_S : 0;
     const char *why = "";
     if (!gdn::bwd_supports(p, &why)) return fail(GDN_ERR_UNSUPPORTED, "backward: %s", why);
 

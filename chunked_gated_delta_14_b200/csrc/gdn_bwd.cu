@@ -26,6 +26,7 @@ bool bwd_supports(const BwdParams &p, const char **why) {
     if (p.dk != 16 && p.dk != 32 && p.dk != 64 && p.dk != 128) { *why = "dk must be 16, 32, 64 or 128"; return false; }
     if (p.dv % bwd::kCols != 0 || p.dv > 128) { *why = "dv must be 32, 64, 96 or 128"; return false; }
     if (p.neumann && (p.N < 0 || p.N > p.C - 1)) { *why = "neumann_N must be in [0, chunk - 1]"; return false; }
+    if (p.residual && (p.S < 1 || p.S > 64)) { *why = "residual_S must be in [0, 64]"; return false; }
     return true;
 }
 
@@ -56,7 +57,7 @@ void bwd_carve_workspace(BwdParams &p, void *workspace) {
 cudaError_t launch_bwd(const BwdParams &p, cudaStream_t stream) {
     const dim3 per_chunk(p.NC, p.H, p.B);
     const dim3 per_slice(p.dv / bwd::kCols, p.H, p.B);
-    cudaError_t e = launch_one(bwd::bwd_prep_kernel, per_chunk, bwd::prep_smem_floats(p.C, p.dk, p.dv), p, stream,
+    cudaError_t e = launch_one(bwd::bwd_prep_kernel, per_chunk, bwd::prep_smem_floats(p.C, p.dk, p.dv, p.residual), p, stream,
                                bwd::kPrepThreads);
     if (e != cudaSuccess) return e;
     e = launch_one(bwd::bwd_state_fwd_kernel, per_slice, bwd::state_fwd_smem_floats(p.C, p.dk), p, stream);
@@ -64,7 +65,7 @@ cudaError_t launch_bwd(const BwdParams &p, cudaStream_t stream) {
     e = launch_one(bwd::bwd_state_rev_kernel, per_slice, bwd::state_rev_smem_floats(p.C, p.dk), p, stream);
     if (e != cudaSuccess) return e;
     if (p.neumann) {
-        e = launch_one(bwd::bwd_neumann_kernel, per_chunk, bwd::neumann_smem_floats(p.C, p.dv), p, stream,
+        e = launch_one(bwd::bwd_neumann_kernel, per_chunk, bwd::neumann_smem_floats(p.C, p.dv, p.residual), p, stream,
                        bwd::kPrepThreads);
         if (e != cudaSuccess) return e;
     }

@@ -162,6 +162,47 @@ __device__ __forceinline__ void block_product(const float *A, int ra, int ia, in
     }
 }
 
+// out(r, c) = sum_{k < K} A(r, k) B(k, c) for r, c < C (or out += that with
+// `accumulate`), A(r, k) = A[r ra + k ia], B(k, c) = B[k rb + c ib],
+// out(r, c) = out[r os + c].  4 x 4 register tiles, two lanes per tile on the even
+// and odd k, summed with a shuffle.  out must not be A or B.  Ends with a barrier.
+template <int NT>
+__device__ __forceinline__ void tile_product(const float *A, int ra, int ia, const float *B, int rb, int ib, int K,
+                                             float *out, int os, int C, int tid, bool accumulate = false) {
+    const int nt = C / 4, items = 2 * nt * nt;
+    for (int w = tid; w < items; w += NT) {
+        const int part = w & 1, t = w >> 1;
+        const int r0 = 4 * (t / nt), c0 = 4 * (t % nt);
+        float acc[4][4] = {};
+        for (int k = part; k < K; k += 2) {
+            float a[4], bb[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                a[e] = A[(r0 + e) * ra + k * ia];
+                bb[e] = B[k * rb + (c0 + e) * ib];
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+#pragma unroll
+                for (int f = 0; f < 4; ++f) acc[e][f] += a[e] * bb[f];
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+#pragma unroll
+            for (int f = 0; f < 4; ++f) acc[e][f] += __shfl_xor_sync(0xffffffffu, acc[e][f], 1);
+        if (part == 0) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+#pragma unroll
+                for (int f = 0; f < 4; ++f) {
+                    float *o = out + (r0 + e) * os + c0 + f;
+                    *o = accumulate ? *o + acc[e][f] : acc[e][f];
+                }
+        }
+    }
+    __syncthreads();
+}
+
 // T = (I + L)^-1 for strictly lower L (C x C in shared memory, row stride Cp),
 // blocked: the 16 x 16 diagonal blocks by forward substitution (one column per
 // thread; each solved entry updates the rows below it), then the merges
@@ -209,9 +250,10 @@ __device__ __forceinline__ void block_inverse(const float *Ls, float *Ts, float 
 // ------------------------------------------------------------------- prep
 // One block per chunk-head.  Shared memory (floats): K, Q (C x (dk+1)),
 // V and then dO (C x (dv+1)), L, T, M (C x (C+1)), g, beta, beta e^g, e^g (C each).
-__host__ __device__ inline size_t prep_smem_floats(int C, int dk, int dv) {
+__host__ __device__ inline size_t prep_smem_floats(int C, int dk, int dv, int residual = 0) {
     return 2 * (size_t)C * (dk + 1) + (size_t)C * (dv + 1) + 3 * (size_t)C * (C + 1) + 4 * (size_t)C +
-           (size_t)C * C / 4;   // + the inverse's merge scratch
+           (size_t)C * C / 4 +                        // the inverse's merge scratch
+           (residual ? 3 * (size_t)C * (C + 1) : 0);  // the residual correction's products
 }
 
 __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(const BwdParams p) {
@@ -232,6 +274,7 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(const BwdParams 
     float *bg = bb + C;
     float *eg = bg + C;
     float *Ys = eg + C;        // C/2 x C/2: the inverse's merge scratch
+    float *Rs = Ys + C * C / 4;   // residual correction: 3 x C x (C+1)
     const size_t ch = ((size_t)b * p.H + h) * p.NC + n;
 
     load_rows<kPrepThreads>(p, b, h, t0, C, Cn, dk, dkp, p.k, p.io_bf16, Ks, p.q, p.io_bf16, Qs, tid);
@@ -336,11 +379,34 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(const BwdParams 
             p.ws_dA[ch * C * C + x] = Ts[r * Cp + c];
         }
         __syncthreads();
-        for (int x = tid; x < C * C; x += kPrepThreads) {
-            const int r = x / C, c = x % C;
-            if (r - c > p.N) Ts[r * Cp + c] = 0.f;
+        if (!p.residual) {
+            for (int x = tid; x < C * C; x += kPrepThreads) {
+                const int r = x / C, c = x % C;
+                if (r - c > p.N) Ts[r * Cp + c] = 0.f;
+            }
+            __syncthreads();
+        } else {
+            // The residual-corrected series T0 sum_{s<=S} E^s, E = I - (I - A) T0,
+            // T0 the masked series ("Metodologia", item 3), is T - T_out E^S with
+            // T_out = T - T0 (T's entries below the band) and E = T^-1 T_out =
+            // (I + L) T_out: W_0 = T_out, W_{s+1} = (W_s + W_s L) T_out, T_res = T - W_S.
+            float *Os = Rs, *Wt = Rs + C * Cp, *Xt = Rs + 2 * C * Cp;
+            for (int x = tid; x < C * C; x += kPrepThreads) {
+                const int r = x / C, c = x % C;
+                const float t = r - c > p.N ? Ts[r * Cp + c] : 0.f;
+                Os[r * Cp + c] = t;
+                Wt[r * Cp + c] = t;
+            }
+            __syncthreads();
+            for (int it = 0; it < p.S; ++it) {
+                tile_product<kPrepThreads>(Wt, Cp, 1, Ls, Cp, 1, C, Xt, Cp, C, tid);     // W L
+                for (int x = tid; x < C * C; x += kPrepThreads) Xt[(x / C) * Cp + x % C] += Wt[(x / C) * Cp + x % C];
+                __syncthreads();
+                tile_product<kPrepThreads>(Xt, Cp, 1, Os, Cp, 1, C, Wt, Cp, C, tid);     // (W + W L) T_out
+            }
+            for (int x = tid; x < C * C; x += kPrepThreads) Ts[(x / C) * Cp + x % C] -= Wt[(x / C) * Cp + x % C];
+            __syncthreads();
         }
-        __syncthreads();
     }
 
     for (int x = tid; x < C * C; x += kPrepThreads) p.ws_T[ch * C * C + x] = Ts[(x / C) * Cp + x % C];
@@ -373,94 +439,106 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(const BwdParams 
 // exact inverse agree on the band, the mask zeroes the rest), so
 //   dA = T^T (M (.) dT_N) T^T,  T = (I - A)^-1 exact,  dL = -dA,
 // written to ws_dA (over the exact inverse the prep left there) for the
-// key-side gradient kernel.  All products C x C (the first over d_v), fp32.
-__host__ __device__ inline size_t neumann_smem_floats(int C, int dv) {
-    return 2 * (size_t)C * (dv + 1) + 5 * (size_t)C * (C + 1) + (size_t)C * C / 4;
-}
-
-// out(r, c) = sum_{k < K} A(r, k) B(k, c) for r, c < C, A(r, k) = A[r ra + k ia],
-// B(k, c) = B[k rb + c ib], out(r, c) = out[r os + c].  4 x 4 register tiles,
-// two lanes per tile on the even and odd k, summed with a shuffle.  Ends with a
-// barrier.
-template <int NT>
-__device__ __forceinline__ void tile_product(const float *A, int ra, int ia, const float *B, int rb, int ib, int K,
-                                             float *out, int os, int C, int tid) {
-    const int nt = C / 4, items = 2 * nt * nt;
-    for (int w = tid; w < items; w += NT) {
-        const int part = w & 1, t = w >> 1;
-        const int r0 = 4 * (t / nt), c0 = 4 * (t % nt);
-        float acc[4][4] = {};
-        for (int k = part; k < K; k += 2) {
-            float a[4], bb[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                a[e] = A[(r0 + e) * ra + k * ia];
-                bb[e] = B[k * rb + (c0 + e) * ib];
-            }
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-#pragma unroll
-                for (int f = 0; f < 4; ++f) acc[e][f] += a[e] * bb[f];
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-#pragma unroll
-            for (int f = 0; f < 4; ++f) acc[e][f] += __shfl_xor_sync(0xffffffffu, acc[e][f], 1);
-        if (part == 0) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-#pragma unroll
-                for (int f = 0; f < 4; ++f) out[(r0 + e) * os + c0 + f] = acc[e][f];
-        }
-    }
-    __syncthreads();
+// key-side gradient kernel.  With the residual correction (item 3) the forward's
+// inverse is T_res = T - T_out E^S (T_out the part of T below the band,
+// E = T^-1 T_out) and the gradient reaching T follows from that form (below).
+// All products C x C (the first over d_v), fp32.
+__host__ __device__ inline size_t neumann_smem_floats(int C, int dv, int residual = 0) {
+    (void)dv;
+    return 2 * (size_t)C * 33 + (residual ? 9 : 5) * (size_t)C * (C + 1) + (size_t)C * C / 4;
 }
 
 __global__ void __launch_bounds__(kPrepThreads) bwd_neumann_kernel(const BwdParams p) {
     constexpr int NT = kPrepThreads;
     float *sm = reinterpret_cast<float *>(bwd_smem);
-    const int C = p.C, dv = p.dv, dvp = dv + 1, Cp = C + 1;
+    const int C = p.C, dv = p.dv, Cp = C + 1;
     const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
     const size_t ch = ((size_t)b * p.H + h) * p.NC + n;
-    float *Yt = sm;                 // Y, C x dv
-    float *Dt = Yt + C * dvp;       // Delta, C x dv
-    float *Ss = Dt + C * dvp;       // Y Delta^T, then M (.) dT_N
-    float *Bs = Ss + C * Cp;        // T_N without its diagonal
-    float *Ti = Bs + C * Cp;        // T_N^-1
+    float *Yt = sm;                 // a 32-column tile of Y, C x 32
+    float *Dt = Yt + C * 33;        // the same tile of Delta
+    float *Ss = Dt + C * 33;        // Y Delta^T, then dT, then the gradient reaching T
+    float *Bs = Ss + C * Cp;        // strictly lower parts to invert; later T_out, powers of E
+    float *Ti = Bs + C * Cp;        // T_N^-1 (or T_res^-1), then T^-1
     float *Tx = Ti + C * Cp;        // the exact inverse
-    float *Tm = Tx + C * Cp;        // products in between
+    float *Tm = Tx + C * Cp;        // products in between; E
     float *Ys = Tm + C * Cp;        // scratch of the inverse, C * C / 4
+    float *R1 = Ys + C * C / 4;     // residual correction only: K, Q2
+    float *R2 = R1 + C * Cp, *R3 = R2 + C * Cp, *R4 = R3 + C * Cp;
 
-    for (int x = tid; x < C * dv / 4; x += NT) {
-        const int r = 4 * x / dv, c = 4 * x % dv;
-        const float4 y = *reinterpret_cast<const float4 *>(p.ws_Y + ch * C * dv + 4 * x);
-        const float4 d = *reinterpret_cast<const float4 *>(p.ws_D + ch * C * dv + 4 * x);
-        float *yr = Yt + r * dvp + c, *dr = Dt + r * dvp + c;
-        yr[0] = y.x; yr[1] = y.y; yr[2] = y.z; yr[3] = y.w;
-        dr[0] = d.x; dr[1] = d.y; dr[2] = d.z; dr[3] = d.w;
-    }
     for (int x = tid; x < C * C; x += NT) {
         const int r = x / C, c = x % C;
         const float tn = p.ws_T[ch * C * C + x];
-        Bs[r * Cp + c] = c < r ? tn : 0.f;      // rows past the tail are zero: T_N^-1 is 1 there
+        Bs[r * Cp + c] = c < r ? tn : 0.f;      // rows past the tail are zero: the inverse is 1 there
         Ti[r * Cp + c] = 0.f;
         Tx[r * Cp + c] = p.ws_dA[ch * C * C + x];
     }
-    __syncthreads();
-    // S = Y Delta^T (over d_v), T_N^-1
-    tile_product<NT>(Yt, dvp, 1, Dt, 1, dvp, dv, Ss, Cp, C, tid);
-    block_inverse<NT>(Bs, Ti, Ys, C, Cp, tid);
-    // dT_N = T_N^-T S T_N^-T, masked to the band (its entries farther below the
-    // diagonal are not functions of A; those above it add nothing to the lower dA)
-    tile_product<NT>(Ss, Cp, 1, Ti, 1, Cp, C, Tm, Cp, C, tid);     // S T_N^-T
-    tile_product<NT>(Ti, 1, Cp, Tm, Cp, 1, C, Ss, Cp, C, tid);     // T_N^-T (S T_N^-T)
-    for (int x = tid; x < C * C; x += NT) {
-        const int r = x / C, c = x % C;
-        if (r - c > p.N) Ss[r * Cp + c] = 0.f;
+    // S = Y Delta^T over d_v, 32 columns at a time
+    for (int j0 = 0; j0 < dv; j0 += 32) {
+        __syncthreads();
+        for (int x = tid; x < C * 32; x += NT) {
+            const int r = x / 32, c = x % 32;
+            Yt[r * 33 + c] = p.ws_Y[(ch * C + r) * dv + j0 + c];
+            Dt[r * 33 + c] = p.ws_D[(ch * C + r) * dv + j0 + c];
+        }
+        __syncthreads();
+        tile_product<NT>(Yt, 33, 1, Dt, 1, 33, 32, Ss, Cp, C, tid, j0 > 0);
     }
-    __syncthreads();
-    // dA = T^T G T^T with the exact inverse, to the workspace
-    tile_product<NT>(Ss, Cp, 1, Tx, 1, Cp, C, Tm, Cp, C, tid);     // G T^T
+    // dT = T_^-T S T_^-T for the truncated inverse T_ the forward used
+    block_inverse<NT>(Bs, Ti, Ys, C, Cp, tid);
+    tile_product<NT>(Ss, Cp, 1, Ti, 1, Cp, C, Tm, Cp, C, tid);     // S T_^-T
+    tile_product<NT>(Ti, 1, Cp, Tm, Cp, 1, C, Ss, Cp, C, tid);     // T_^-T (S T_^-T) = G
+    if (!p.residual) {
+        // T_N = M (.) T: the gradient reaching T is M (.) G (entries above the
+        // diagonal add nothing to the strictly lower dA)
+        for (int x = tid; x < C * C; x += NT) {
+            const int r = x / C, c = x % C;
+            if (r - c > p.N) Ss[r * Cp + c] = 0.f;
+        }
+        __syncthreads();
+    } else {
+        // T_res = T - T_out E^S, T_out = (1 - M) (.) T, E = T^-1 T_out.  With
+        // K = T_out^T G and H = sum_{j<S} (E^T)^j K (E^T)^{S-1-j}, the gradient
+        // reaching T is G - (1 - M) (.) (G (E^S)^T + T^-T H) + T^-T H E^T.
+        for (int x = tid; x < C * C; x += NT) {
+            const int r = x / C, c = x % C;
+            Bs[r * Cp + c] = c < r ? Tx[r * Cp + c] : 0.f;
+            Ti[r * Cp + c] = 0.f;
+        }
+        __syncthreads();
+        block_inverse<NT>(Bs, Ti, Ys, C, Cp, tid);                   // T^-1
+        for (int x = tid; x < C * C; x += NT) {
+            const int r = x / C, c = x % C;
+            Bs[r * Cp + c] = r - c > p.N ? Tx[r * Cp + c] : 0.f;     // T_out
+        }
+        __syncthreads();
+        tile_product<NT>(Ti, Cp, 1, Bs, Cp, 1, C, Tm, Cp, C, tid);     // E = T^-1 T_out
+        tile_product<NT>(Bs, 1, Cp, Ss, Cp, 1, C, R1, Cp, C, tid);     // K = T_out^T G
+        for (int x = tid; x < C * Cp; x += NT) {
+            Bs[x] = Tm[x];                                              // P = E^1
+            R2[x] = R1[x];                                              // X_0 = K
+        }
+        __syncthreads();
+        float *P = Bs, *Pn = R4, *X = R2, *Xn = R3;
+        for (int m = 1; m < p.S; ++m) {
+            tile_product<NT>(Tm, 1, Cp, X, Cp, 1, C, Xn, Cp, C, tid);          // E^T X_{m-1}
+            tile_product<NT>(R1, Cp, 1, P, 1, Cp, C, Xn, Cp, C, tid, true);    // + K (E^m)^T
+            tile_product<NT>(P, Cp, 1, Tm, Cp, 1, C, Pn, Cp, C, tid);          // E^{m+1}
+            float *t = X; X = Xn; Xn = t;
+            t = P; P = Pn; Pn = t;
+        }
+        // X = H, P = E^S; Pn and Xn are free
+        tile_product<NT>(Ss, Cp, 1, P, 1, Cp, C, Pn, Cp, C, tid);     // Q1 = G (E^S)^T
+        tile_product<NT>(Ti, 1, Cp, X, Cp, 1, C, R1, Cp, C, tid);      // Q2 = T^-T H
+        tile_product<NT>(R1, Cp, 1, Tm, 1, Cp, C, Xn, Cp, C, tid);     // Q3 = Q2 E^T
+        for (int x = tid; x < C * C; x += NT) {
+            const int r = x / C, c = x % C, i = r * Cp + c;
+            const float out = r - c > p.N ? Pn[i] + R1[i] : 0.f;
+            Ss[i] = Ss[i] - out + Xn[i];
+        }
+        __syncthreads();
+    }
+    // dA = T^T (gradient reaching T) T^T with the exact inverse, to the workspace
+    tile_product<NT>(Ss, Cp, 1, Tx, 1, Cp, C, Tm, Cp, C, tid);
     tile_product<NT>(Tx, 1, Cp, Tm, Cp, 1, C, p.ws_dA + ch * C * C, C, C, tid);
 }
 

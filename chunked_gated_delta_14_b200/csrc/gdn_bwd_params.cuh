@@ -19,6 +19,7 @@ struct BwdParams {
     float *grad_q, *grad_k, *grad_v;
     float *grad_alpha, *grad_beta, *grad_S0;   // each may be null
     int neumann, N;               // chunk inverse: 0 exact; 1 the masked truncated series of order N
+    int residual, S;              // with neumann: the series with S residual-correction terms
     // Workspace regions, fp32, each indexed by chunk-head (b*H + h)*NC + n:
     float *ws_g;    // C        in-chunk cumulative log decay g
     float *ws_T;    // C x C    T = (I + L)^-1

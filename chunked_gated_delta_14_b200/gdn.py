@@ -77,7 +77,7 @@ class BwdArgs(ctypes.Structure):
         ("grad_alpha", ctypes.c_void_p), ("grad_beta", ctypes.c_void_p),
         ("grad_S0", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_uint64),
-        ("mode", ctypes.c_int32), ("neumann_N", ctypes.c_int32),
+        ("mode", ctypes.c_int32), ("neumann_N", ctypes.c_int32), ("residual_S", ctypes.c_int32),
     ]
 
 
@@ -374,7 +374,7 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
               alpha: Optional[torch.Tensor], beta: Optional[torch.Tensor],
               grad_o: torch.Tensor, *, S0: Optional[torch.Tensor] = None,
               grad_S_T: Optional[torch.Tensor] = None, chunk: int = 64,
-              want_S0: bool = True, mode: str = "exact", N: int = 3,
+              want_S0: bool = True, mode: str = "exact", N: int = 3, S: int = 8,
               stream: Optional[torch.cuda.Stream] = None) -> dict:
     """Gradients of the gated delta rule (scalar alpha and beta, exact inverse).
 
@@ -382,8 +382,9 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     and ``grad_S_T`` [B, H, dk, dv] fp32 (or None) dL/dS_T.  Returns a dict of
     fp32 tensors ``dq``, ``dk``, ``dv``, ``dalpha`` / ``dbeta`` (None when the
     gate is None) and ``dS0`` (None unless ``want_S0``).  ``mode`` is the chunk
-    inverse of the forward being differentiated: "exact" or "neumann" (the
-    masked truncated series of order ``N``).
+    inverse of the forward being differentiated: "exact", "neumann" (the
+    masked truncated series of order ``N``) or "residual" (that series with ``S``
+    correction terms).
     """
     if q.dim() != 4:
         raise ValueError("q must be [B, T, H, dk]")
@@ -410,7 +411,7 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         beta=_ptr(beta), S0=_ptr(S0), grad_o=_ptr(grad_o), grad_S_T=_ptr(grad_S_T),
         grad_q=_ptr(g["dq"]), grad_k=_ptr(g["dk"]), grad_v=_ptr(g["dv"]),
         grad_alpha=_ptr(g["dalpha"]), grad_beta=_ptr(g["dbeta"]), grad_S0=_ptr(g["dS0"]),
-        mode={"exact": GDN_INV_EXACT, "neumann": GDN_INV_NEUMANN}[mode], neumann_N=int(N))
+        mode=MODES[mode], neumann_N=int(N), residual_S=int(S))
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     ws = workspace_for(args, q.device, stream)

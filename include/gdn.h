@@ -281,7 +281,11 @@ GDN_API int32_t gdn_abi_version(void);
  * inverse, and a launch between 3 and 4 forms, per chunk-head,
  * dA = T^T (M (.) dT_N) T^T with dT_N = T_N^-T (Y Delta^T) T_N^-T, the gradient
  * reaching A = -L through the series (the workspace grows by C x C floats per
- * chunk-head).  GDN_INV_NEUMANN_RESIDUAL returns GDN_ERR_INVALID_ARG.
+ * chunk-head).  With GDN_INV_NEUMANN_RESIDUAL (same section, item 3) the
+ * forward's inverse T0 sum_{s<=S} E^s equals T - T_out E^S (T_out the part of the
+ * exact T below the band, E = T^-1 T_out); launch 1 forms it with 2 S products
+ * per chunk-head and the extra launch applies the adjoint of that form
+ * (3 S + 9 products).
  *
  * Layouts as gdn_fwd_args; every gradient is fp32 in the layout of its input
  * (grad_S0 and grad_S_T in the h = S^T layout [B, H, dk, dv]).
@@ -312,9 +316,13 @@ typedef struct {
     void *workspace;            /* >= gdn_bwd_workspace_bytes(args) bytes, 16-byte aligned */
     uint64_t workspace_bytes;
     int32_t mode;               /* the chunk inverse of the forward being differentiated:
-                                   GDN_INV_EXACT, or GDN_INV_NEUMANN (the masked truncated
-                                   series of order neumann_N, 0 <= N <= chunk - 1) */
+                                   GDN_INV_EXACT, GDN_INV_NEUMANN (the masked truncated
+                                   series of order neumann_N, 0 <= N <= chunk - 1), or
+                                   GDN_INV_NEUMANN_RESIDUAL (that series corrected with
+                                   residual_S terms) */
     int32_t neumann_N;
+    int32_t residual_S;         /* GDN_INV_NEUMANN_RESIDUAL: the series of order neumann_N
+                                   with residual_S (0..64) correction terms */
 } gdn_bwd_args;
 
 /* Backward pass (see above). */

@@ -47,9 +47,10 @@ static size_t region(size_t floats, size_t n) { return (floats * n * sizeof(floa
 extern "C" int host_bwd(int B, int T, int H, int dk, int dv, int C, int io_bf16, int do_bf16,
                         const void *q, const void *k, const void *v, const float *alpha,
                         const float *beta, const float *S0, const void *grad_o, const float *grad_S_T,
-                        float *gq, float *gk, float *gv, float *ga, float *gb, float *gS0, int neumann, int N) {
+                        float *gq, float *gk, float *gv, float *ga, float *gb, float *gS0, int neumann, int N,
+                        int S) {
     BwdParams p{};
-    p.neumann = neumann; p.N = N;
+    p.neumann = neumann; p.N = N; p.residual = S > 0; p.S = S;
     p.B = B; p.T = T; p.H = H; p.dk = dk; p.dv = dv; p.C = C; p.NC = (T + C - 1) / C;
     p.io_bf16 = io_bf16; p.do_bf16 = do_bf16;
     p.q = q; p.k = k; p.v = v; p.alpha = alpha; p.beta = beta; p.S0 = S0;
@@ -76,10 +77,10 @@ extern "C" int host_bwd(int B, int T, int H, int dk, int dv, int C, int io_bf16,
     g_overrun = 0;
     const dim3h per_chunk{(unsigned)p.NC, (unsigned)H, (unsigned)B};
     const dim3h per_slice{(unsigned)(dv / bwd::kCols), (unsigned)H, (unsigned)B};
-    run_grid(bwd::bwd_prep_kernel, per_chunk, p, bwd::prep_smem_floats(C, dk, dv), bwd::kPrepThreads);
+    run_grid(bwd::bwd_prep_kernel, per_chunk, p, bwd::prep_smem_floats(C, dk, dv, p.residual), bwd::kPrepThreads);
     run_grid(bwd::bwd_state_fwd_kernel, per_slice, p, bwd::state_fwd_smem_floats(C, dk));
     run_grid(bwd::bwd_state_rev_kernel, per_slice, p, bwd::state_rev_smem_floats(C, dk));
-    if (neumann) run_grid(bwd::bwd_neumann_kernel, per_chunk, p, bwd::neumann_smem_floats(C, dv), bwd::kPrepThreads);
+    if (neumann) run_grid(bwd::bwd_neumann_kernel, per_chunk, p, bwd::neumann_smem_floats(C, dv, p.residual), bwd::kPrepThreads);
     const size_t gs = bwd::grad_smem_floats(C, dk);
     switch (dk) {
         case 16: run_grid(bwd::bwd_grad_kernel<16>, per_chunk, p, gs, bwd::kGradThreads); break;

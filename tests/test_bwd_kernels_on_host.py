@@ -61,6 +61,13 @@ NEUMANN_CASES = [  # ..., N: the masked truncated series of order N as the chunk
     (1, 64, 1, 32, 32, 64, True, True, False, 63),
 ]
 
+RESIDUAL_CASES = [  # ..., N, S: the masked series of order N with S correction terms
+    (1, 70, 2, 16, 32, 16, True, True, False, 1, 2),
+    (1, 77, 1, 128, 128, 64, True, True, True, 3, 8),
+    (1, 100, 1, 32, 64, 32, True, False, False, 2, 1),
+    (1, 64, 1, 32, 32, 64, True, True, False, 1, 31),
+]
+
 
 @pytest.mark.parametrize("B,T,H,dk,dv,C,gates,state,bf16", CASES)
 def test_backward_kernel_source_on_host(host_lib, B, T, H, dk, dv, C, gates, state, bf16):
@@ -74,7 +81,14 @@ def test_backward_kernel_source_on_host_masked_series(host_lib, B, T, H, dk, dv,
     _run_case(host_lib, B, T, H, dk, dv, C, gates, state, bf16, N)
 
 
-def _run_case(host_lib, B, T, H, dk, dv, C, gates, state, bf16, N):
+@pytest.mark.parametrize("B,T,H,dk,dv,C,gates,state,bf16,N,S", RESIDUAL_CASES)
+def test_backward_kernel_source_on_host_residual(host_lib, B, T, H, dk, dv, C, gates, state, bf16, N, S):
+    """The gradient of the forward with the residual-corrected series, against the
+    fp64 autograd of that chunk model ((N + 1)(S + 1) = C: exact)."""
+    _run_case(host_lib, B, T, H, dk, dv, C, gates, state, bf16, N, S)
+
+
+def _run_case(host_lib, B, T, H, dk, dv, C, gates, state, bf16, N, S=0):
     g = torch.Generator().manual_seed(B * 1000 + T)
     def nrm(*s):
         return torch.randn(*s, generator=g)
@@ -93,12 +107,12 @@ def _run_case(host_lib, B, T, H, dk, dv, C, gates, state, bf16, N):
     gb = nan(B, T, H) if gates else None
     rc = host_lib.host_bwd(B, T, H, dk, dv, C, int(bf16), int(bf16), _p(q), _p(k), _p(v), _p(alpha),
                            _p(beta), _p(S0), _p(do), _p(dS), _p(gq), _p(gk), _p(gv), _p(ga), _p(gb),
-                           _p(gS0), ctypes.c_int(0 if N is None else 1), ctypes.c_int(N or 0))
+                           _p(gS0), ctypes.c_int(0 if N is None else 1), ctypes.c_int(N or 0), ctypes.c_int(S))
     assert rc == 0, f"a block wrote past its shared memory ({rc - 100} blocks)" if rc >= 100 else rc
     if N is None:
         ref = rec.gated_delta_bwd(q, k, v, alpha, beta, S0, do, dS)
     else:
-        ref = cg.neumann_bwd(q, k, v, alpha, beta, S0, do, dS, chunk=C, N=N)
+        ref = cg.neumann_bwd(q, k, v, alpha, beta, S0, do, dS, chunk=C, N=N, S=S if S else None)
     for name, got in (("dq", gq), ("dk", gk), ("dv", gv), ("dalpha", ga), ("dbeta", gb), ("dh0", gS0)):
         if ref[name] is None:
             continue

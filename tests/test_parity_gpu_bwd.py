@@ -224,3 +224,23 @@ def test_autograd_masked_series():
             assert bf16_allowance_ok(got, r, rel_rms=TOL_BWD_REL_RMS), n
         else:
             assert stats(got, r)["max_rel_rms"] <= TOL_BWD_REL_RMS, n
+
+
+@needs_cuda
+@pytest.mark.parametrize("chunk,N,S,T", [(64, 3, 8, 300), (64, 2, 1, 129), (32, 1, 15, 100), (16, 2, 2, 37)])
+def test_backward_residual_corrected_series(chunk, N, S, T):
+    """The gradient of the forward with the residual-corrected series (N, S) as the
+    chunk inverse, against the fp64 autograd of that chunk model; (N + 1)(S + 1) = C
+    (the 32-chunk case) makes it exact."""
+    from oracle import chunk_grad as cg
+    w = workload("gdn_bf16", B=1, H=2, T=T, chunk=chunk, decay="weak", s0_std=0.02)
+    x = make_inputs(w, seed=54)
+    c = make_cotangents(w, seed=54)
+    d = {k: to_dev(v) for k, v in x.items()}
+    g = gdn.chunk_bwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], to_dev(c["grad_o"]), S0=d["S0"],
+                      grad_S_T=to_dev(c["grad_S_T"]), chunk=chunk, mode="residual", N=N, S=S)
+    torch.cuda.synchronize()
+    got = {k: None if v is None else v.double().cpu().numpy() for k, v in g.items()}
+    ref = cg.neumann_bwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"], c["grad_o"], c["grad_S_T"],
+                         chunk=chunk, N=N, S=S)
+    _compare(f"bwd_residual_C{chunk}_N{N}_S{S}_T{T}", got, ref)
