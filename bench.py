@@ -762,10 +762,11 @@ def bwd_bytes(w):
     return w.token_heads * per_th
 
 
-def bwd_setup(w, x, c, dev, mode="exact", N=3):
+def bwd_setup(w, x, c, dev, mode="exact", N=3, S=8):
     """Device copies of the inputs and dL/do, fp32 gradient buffers and the
     gdn_bwd_args (with workspace) of one backward call over the whole batch
-    (``mode`` "neumann": the gradient of the masked truncated series of order N).
+    (``mode`` "neumann": the gradient of the masked truncated series of order N;
+    "residual": of that series with S correction terms).
     The args hold raw pointers: the returned dict keeps every tensor they point
     to alive."""
     import torch
@@ -782,7 +783,8 @@ def bwd_setup(w, x, c, dev, mode="exact", N=3):
                           alpha=ptr(d["alpha"]), beta=ptr(d["beta"]), grad_o=ptr(grad_o),
                           grad_q=ptr(g["dq"]), grad_k=ptr(g["dk"]), grad_v=ptr(g["dv"]),
                           grad_alpha=ptr(g["da"]), grad_beta=ptr(g["db"]),
-                          mode=1 if mode == "neumann" else 0, neumann_N=int(N) if mode == "neumann" else 0)
+                          mode={"exact": 0, "neumann": 1, "residual": 2}[mode],
+                          neumann_N=int(N) if mode != "exact" else 0, residual_S=int(S) if mode == "residual" else 0)
     ws = gdn.workspace_for(a, dev)
     a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
     g["inputs"], g["grad_o"] = d, grad_o
@@ -851,10 +853,8 @@ def run_bwd(args, rank, world, local_rank):
     w = workload(WORKLOAD, **({"B": args.batch} if args.batch else {}))
     x = make_inputs(w, seed=rank)
     c = make_cotangents(w, seed=rank, grad_state=False)
-    neumann = args.mode == "neumann"
-    if args.mode == "residual":
-        raise SystemExit("bench.py --bwd: the backward takes --mode exact or neumann")
-    a, g, ws = bwd_setup(w, x, c, dev, mode=args.mode, N=args.N)
+    neumann = args.mode in ("neumann", "residual")
+    a, g, ws = bwd_setup(w, x, c, dev, mode=args.mode, N=args.N, S=args.S)
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
     for _ in range(args.warmup):
@@ -893,7 +893,7 @@ def run_bwd(args, rank, world, local_rank):
 
         def run(di, slot):
             r = gdn.chunk_bwd(di["q"], di["k"], di["v"], di["alpha"], di["beta"], di["grad_o"],
-                              mode="neumann" if neumann else "exact", N=args.N,
+                              mode=args.mode, N=args.N, S=args.S,
                               chunk=w.chunk, want_S0=False)
             return {k: r[k] for k in ("dq", "dk", "dv", "dalpha", "dbeta")}
 
@@ -923,7 +923,8 @@ def run_bwd(args, rank, world, local_rank):
             if neumann:
                 from oracle import chunk_grad
                 chunk_grad.neumann_bwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["alpha"]), sl(x["beta"]), None,
-                                       sl(c["grad_o"]), None, chunk=w.chunk, N=args.N)
+                                       sl(c["grad_o"]), None, chunk=w.chunk, N=args.N,
+                                       S=args.S if args.mode == "residual" else None)
             else:
                 oracle.gated_delta_bwd(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["alpha"]), sl(x["beta"]),
                                    None, sl(c["grad_o"]), None, nthreads=cores)
@@ -931,7 +932,7 @@ def run_bwd(args, rank, world, local_rank):
             if time.perf_counter() - t0 >= min(args.cpu_budget, 10.0):
                 break
         el = time.perf_counter() - t0
-        how = "fp64 autograd of the masked-series chunk model (torch CPU ops)" if neumann else "fp64 C adjoint"
+        how = "fp64 autograd of the series' chunk model (torch CPU ops)" if neumann else "fp64 C adjoint"
         cpu = dict(value=Ts * n / el, unit=UNIT, cores=torch.get_num_threads() if neumann else cores, kind="oracle",
                    sample=f"{n} x (tokens [0,{Ts}) of one batch row, all {w.H} heads), {how}, {el:.1f} s")
     if rank == 0:
@@ -942,7 +943,9 @@ def run_bwd(args, rank, world, local_rank):
                     data="synthetic (seeded; Gated DeltaNet layer shapes)",
                     config=dict(workload=f"{WORKLOAD} backward: B={w.B} H={w.H} T={w.T} dk={w.dk} "
                                 f"dv={w.dv} chunk={w.chunk} "
-                                + (f"masked truncated Neumann inverse N={args.N}" if neumann else "exact inverse"),
+                                + ("exact inverse" if not neumann else
+                                   f"masked truncated Neumann inverse N={args.N}"
+                                   + (f" with {args.S} residual-correction terms" if args.mode == "residual" else "")),
                                 global_batch=w.B * world, seq_len=w.T,
                                 parallelism=f"independent batch per GPU x{world}",
                                 l2=f"no flush: inputs+gradients {nbytes / 1e6:.0f} MB + workspace "
