@@ -425,14 +425,15 @@ def chunk_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
 
 class GatedDeltaRule(torch.autograd.Function):
     """Differentiable gated delta rule: forward by ``chunk_fwd``, backward by
-    ``chunk_bwd``, both with the same chunk inverse (``mode`` "exact" or
-    "neumann" of order ``N``); both run in libgdn.so."""
+    ``chunk_bwd``, both with the same chunk inverse (``mode`` "exact", "neumann"
+    of order ``N``, or "residual" with ``S`` correction terms); both run in
+    libgdn.so."""
 
     @staticmethod
-    def forward(ctx, q, k, v, alpha, beta, S0, chunk, mode="exact", N=3):
-        o, S_T = chunk_fwd(q, k, v, alpha, beta, S0=S0, chunk=chunk, mode=mode, N=N)
+    def forward(ctx, q, k, v, alpha, beta, S0, chunk, mode="exact", N=3, S=8):
+        o, S_T = chunk_fwd(q, k, v, alpha, beta, S0=S0, chunk=chunk, mode=mode, N=N, S=S)
         ctx.save_for_backward(q, k, v, alpha, beta, S0)
-        ctx.chunk, ctx.mode, ctx.N = chunk, mode, N
+        ctx.chunk, ctx.mode, ctx.N, ctx.S = chunk, mode, N, S
         return o, S_T
 
     @staticmethod
@@ -443,17 +444,17 @@ class GatedDeltaRule(torch.autograd.Function):
         g = chunk_bwd(q, k, v, alpha, beta, grad_o.contiguous(), S0=S0,
                       grad_S_T=None if grad_S_T is None else grad_S_T.float().contiguous(),
                       chunk=ctx.chunk, want_S0=S0 is not None and ctx.needs_input_grad[5],
-                      mode=ctx.mode, N=ctx.N)
+                      mode=ctx.mode, N=ctx.N, S=ctx.S)
         cast = lambda t, like: None if t is None else t.to(like.dtype)
         return (cast(g["dq"], q), cast(g["dk"], k), cast(g["dv"], v), g["dalpha"], g["dbeta"],
-                g["dS0"], None, None, None)
+                g["dS0"], None, None, None, None)
 
 
 def gated_delta_rule(q, k, v, alpha=None, beta=None, S0=None, chunk: int = 64, mode: str = "exact",
-                     N: int = 3):
+                     N: int = 3, S: int = 8):
     """``(o, S_T)`` of the gated delta rule with autograd support (see GatedDeltaRule);
     ``mode`` "neumann" uses the masked truncated series of order ``N`` as the chunk
-    inverse in both passes."""
-    if mode not in ("exact", "neumann"):
-        raise ValueError("gated_delta_rule: mode must be 'exact' or 'neumann'")
-    return GatedDeltaRule.apply(q, k, v, alpha, beta, S0, chunk, mode, N)
+    inverse in both passes, "residual" that series with ``S`` correction terms."""
+    if mode not in ("exact", "neumann", "residual"):
+        raise ValueError("gated_delta_rule: mode must be 'exact', 'neumann' or 'residual'")
+    return GatedDeltaRule.apply(q, k, v, alpha, beta, S0, chunk, mode, N, S)
