@@ -197,9 +197,11 @@ def test_backward_masked_series_full_order_equals_exact():
 
 
 @needs_cuda
-def test_autograd_masked_series():
-    """gated_delta_rule with the masked series (N = 3) in both passes, against the
-    fp64 autograd of the chunk model; the forward against the numpy chunk model."""
+@pytest.mark.parametrize("mode,S", [("neumann", None), ("residual", 4)])
+def test_autograd_masked_series(mode, S):
+    """gated_delta_rule with the masked series (N = 3; with S correction terms in
+    the residual mode) in both passes, against the fp64 autograd of the chunk
+    model; the forward against the numpy chunk model."""
     from oracle import chunk_forms as cf
     from oracle import chunk_grad as cg
     w = workload("gdn_bf16", B=1, H=2, T=200, decay="weak", s0_std=0.02)
@@ -207,19 +209,20 @@ def test_autograd_masked_series():
     c = make_cotangents(w, seed=53)
     d = {k: None if v is None else to_dev(v).requires_grad_(True) for k, v in x.items()
          if k in ("q", "k", "v", "alpha", "beta", "S0")}
-    o, S_T = gdn.gated_delta_rule(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], mode="neumann", N=3)
+    o, S_T = gdn.gated_delta_rule(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], mode=mode, N=3,
+                                  S=S or 0)
     o_ref, _ = cf.chunked_gated_delta_fwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"], chunk=64,
-                                          inverse=cf.neumann_inverse(3))
+                                          inverse=cf.neumann_inverse(3) if S is None else cf.residual_inverse(3, S))
     assert bf16_allowance_ok(o.detach().double().cpu().numpy(), o_ref)
     loss = (o.float() * to_dev(c["grad_o"]).float()).sum() + (S_T * to_dev(c["grad_S_T"])).sum()
     names = ["q", "k", "v", "alpha", "beta", "S0"]
     grads = torch.autograd.grad(loss, [d[n] for n in names])
     ref = cg.neumann_bwd(x["q"], x["k"], x["v"], x["alpha"], x["beta"], x["S0"], c["grad_o"], c["grad_S_T"],
-                         chunk=64, N=3)
+                         chunk=64, N=3, S=S)
     for n, g in zip(names, grads):
         r = ref[dict(q="dq", k="dk", v="dv", alpha="dalpha", beta="dbeta", S0="dh0")[n]]
         got = g.double().cpu().numpy()
-        report(f"autograd_neumann_{n}", **stats(got, r))
+        report(f"autograd_{mode}_{n}", **stats(got, r))
         if g.dtype == torch.bfloat16:
             assert bf16_allowance_ok(got, r, rel_rms=TOL_BWD_REL_RMS), n
         else:
