@@ -52,6 +52,8 @@ gdn_status resolve(const gdn_fwd_args *a, gdn::FwdParams *out, int *kernel) {
         return fail(GDN_ERR_INVALID_ARG, "neumann_N must be in [0, chunk-1] (got %d)", a->neumann_N);
     if (a->mode == GDN_INV_NEUMANN_RESIDUAL && (a->residual_S < 0 || a->residual_S > 64))
         return fail(GDN_ERR_INVALID_ARG, "residual_S must be in [0, 64] (got %d)", a->residual_S);
+    if (a->mode != GDN_INV_EXACT && (a->neumann_N < 0 || a->neumann_N > a->chunk - 1))
+        return fail(GDN_ERR_INVALID_ARG, "neumann_N must be in [0, chunk-1] (got %d)", a->neumann_N);
     if (a->alpha_per_channel && !a->alpha)
         return fail(GDN_ERR_INVALID_ARG, "alpha_per_channel needs alpha");
     if (a->alpha_per_channel != 0 && a->alpha_per_channel != 1)
@@ -206,6 +208,8 @@ gdn_status resolve_bwd(const gdn_bwd_args *a, gdn::BwdParams *out) {
         return fail(GDN_ERR_INVALID_ARG, "backward mode %d unknown", a->mode);
     if (a->mode == GDN_INV_NEUMANN_RESIDUAL && (a->residual_S < 0 || a->residual_S > 64))
         return fail(GDN_ERR_INVALID_ARG, "residual_S must be in [0, 64] (got %d)", a->residual_S);
+    if (a->mode != GDN_INV_EXACT && (a->neumann_N < 0 || a->neumann_N > a->chunk - 1))
+        return fail(GDN_ERR_INVALID_ARG, "neumann_N must be in [0, chunk-1] (got %d)", a->neumann_N);
     gdn::BwdParams p{};
     p.B = a->B; p.T = a->T; p.H = a->H; p.dk = a->dk; p.dv = a->dv; p.C = a->chunk;
     p.NC = (a->T + a->chunk - 1) / (a->chunk > 0 ? a->chunk : 1);

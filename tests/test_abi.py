@@ -180,6 +180,15 @@ def test_bwd_workspace_size(shape):
     assert gdn.bwd_workspace_bytes(a) == _bwd_ws_expected(*shape), gdn.last_error()
 
 
+def test_bwd_workspace_size_with_the_series():
+    # the masked series (and its residual form) add one C x C region per chunk-head
+    nch = 2 * 3 * 2
+    extra = (64 * 64 * nch * 4 + 255) // 256 * 256
+    base = _bwd_ws_expected(2, 100, 3, 128, 128, 64)
+    assert gdn.bwd_workspace_bytes(_bwd_args(mode=1, neumann_N=3)) == base + extra
+    assert gdn.bwd_workspace_bytes(_bwd_args(mode=2, neumann_N=3, residual_S=8)) == base + extra
+
+
 @pytest.mark.parametrize("kw,status", [
     (dict(B=0), GDN_ERR_INVALID_ARG),
     (dict(H=70000), GDN_ERR_INVALID_ARG),
@@ -197,6 +206,9 @@ def test_bwd_workspace_size(shape):
     (dict(grad_v=10 * (1 << 32) + 4096), GDN_ERR_INVALID_ARG),  # grad_v overlaps grad_k
     (dict(grad_S0=6 * (1 << 32)), GDN_ERR_INVALID_ARG),  # grad_S0 aliases S0
     (dict(grad_q=9 * (1 << 32) + 8), GDN_ERR_ALIGNMENT),
+    (dict(mode=7), GDN_ERR_INVALID_ARG),
+    (dict(mode=1, neumann_N=64), GDN_ERR_INVALID_ARG),      # the series' order: 0 .. chunk - 1
+    (dict(mode=2, neumann_N=3, residual_S=65), GDN_ERR_INVALID_ARG),
 ])
 def test_bwd_invalid_arguments_rejected_on_host(kw, status):
     a = _bwd_args(**kw)
