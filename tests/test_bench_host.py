@@ -148,6 +148,17 @@ def test_backward_line(fake_cuda):
     assert line["dtype"] == "f32"
 
 
+@pytest.mark.parametrize("mode", ["neumann", "residual"])
+def test_backward_line_of_the_series(fake_cuda, mode):
+    line = _line("run_bwd", mode=mode, S=2)
+    _check_contract(line)
+    assert line["gpu_launches"] == 5 * 2 and "bwd_neumann_kernel" in line["config"]["kernel"]
+    assert "masked truncated Neumann inverse N=3" in line["config"]["workload"]
+    assert ("residual" in line["config"]["workload"]) == (mode == "residual")
+    assert line["roofline"]["traffic"] is None          # the committed capture is of the exact mode
+    assert "autograd" in line["cpu_baseline"]["sample"]
+
+
 def test_backward_object_can_be_skipped(fake_cuda):
     line = _line("run_gpu", bwd_steps=0, no_cpu_baseline=True)
     assert line.get("backward") is None and line["cpu_baseline"] is None
