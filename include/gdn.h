@@ -258,12 +258,13 @@ GDN_API int32_t gdn_abi_version(void);
 /* ------------------------------------------------------------ backward pass
  *
  * Gradient of the gated delta rule (the default rule above: scalar decay
- * alpha, scalar beta, exact inverse) with respect to q, k, v, alpha, beta and
+ * alpha, scalar beta; exact inverse, or the truncated series of the forward's
+ * Neumann modes) with respect to q, k, v, alpha, beta and
  * S0, given dL/do and dL/dS_T.  The pages use chunkwise forms to make
  * training parallel ("Quando o 'Bom o Suficiente' e Otimo ...", sections
  * "Resumo" and "Declaracao do Problema") but print no backward pass; this is
  * the reverse-mode derivative of the chunked WY/UT form, fp32 on CUDA cores,
- * in four launches:
+ * in four launches (five with the truncated series, below):
  *   1. per chunk-head: g, L, T = (I + L)^-1, the causal scores M, W, U, and the
  *      state-independent M^T dO and (diag(e^g) Q)^T dO;
  *   2. per 32-column value slice, chunks in order: the state at every chunk
