@@ -14,7 +14,7 @@ bool bwd_supports(const BwdParams &p, const char **why);
 size_t bwd_workspace_bytes(const BwdParams &p);
 // Points the ws_* fields of p into `workspace`.
 void bwd_carve_workspace(BwdParams &p, void *workspace);
-// Enqueues the four launches (five with the masked series) on `stream`.
+// Enqueues the four launches (five with either truncated series) on `stream`.
 cudaError_t launch_bwd(const BwdParams &p, cudaStream_t stream);
 
 }  // namespace gdn
