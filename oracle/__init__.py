@@ -16,8 +16,9 @@ Contents
                 forward that takes the inverse as a parameter, written with
                 numpy.
 ``chunk_grad``  the gradient of the chunked form with the masked truncated
-                Neumann inverse: the chunk model written in plain fp64
-                PyTorch ops, differentiated by autograd.
+                Neumann inverse, and with its residual correction: the chunk
+                model written in plain fp64 PyTorch ops, differentiated by
+                autograd.
 """
 from . import chunk_forms, chunk_grad, recurrent  # noqa: F401
 from .recurrent import gated_delta_bwd, gated_delta_fwd, precond_two_gate_fwd  # noqa: F401

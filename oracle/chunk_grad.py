@@ -1,13 +1,15 @@
 """Gradient of the chunked gated delta rule with the masked truncated Neumann
-inverse, fp64 PyTorch on the CPU -- TEST INFRASTRUCTURE only.
+inverse, and with that series' residual correction, fp64 PyTorch on the CPU --
+TEST INFRASTRUCTURE only.
 
 The pages ("Quando o 'Bom o Suficiente' e Otimo: Aproximacao de Inversao de
 Matriz Baseada Apenas em Multiplicacao para Gated DeltaNet Quantizado",
 sections "Resumo" and "Declaracao do Problema") use the chunkwise form to make
 training parallel, and replace the chunk inverse T = (I - A)^-1 by the masked
-series M^(N) (.) sum_{n<=N} A^n ("Metodologia", items 1 and 2).  With that
-replacement the model is no longer the token recurrence, so its gradient is
-the gradient of the chunk model itself.  This module writes the chunk model
+series M^(N) (.) sum_{n<=N} A^n ("Metodologia", items 1 and 2), optionally
+followed by S terms of the parallel residual correction ("Metodologia", item 3).
+With that replacement the model is no longer the token recurrence, so its
+gradient is the gradient of the chunk model itself.  This module writes the chunk model
 out once more, step by step in the same order as
 ``oracle.chunk_forms.chunked_gated_delta_fwd`` (whose fp64 numpy forward the
 tests hold it to), in plain differentiable PyTorch ops, and takes the
