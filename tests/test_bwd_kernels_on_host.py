@@ -59,6 +59,7 @@ NEUMANN_CASES = [  # ..., N: the masked truncated series of order N as the chunk
     (1, 77, 1, 128, 128, 64, True, True, True, 4),
     (2, 130, 1, 64, 32, 64, False, False, False, 1),
     (1, 64, 1, 32, 32, 64, True, True, False, 63),
+    (1, 9, 1, 16, 32, 16, True, True, False, 2),        # one partial chunk: T < C
 ]
 
 RESIDUAL_CASES = [  # ..., N, S: the masked series of order N with S correction terms
@@ -66,6 +67,8 @@ RESIDUAL_CASES = [  # ..., N, S: the masked series of order N with S correction 
     (1, 77, 1, 128, 128, 64, True, True, True, 3, 8),
     (1, 100, 1, 32, 64, 32, True, False, False, 2, 1),
     (1, 64, 1, 32, 32, 64, True, True, False, 1, 31),
+    (1, 5, 1, 16, 32, 32, True, True, False, 1, 1),     # one partial chunk: T < C
+    (1, 64, 1, 16, 32, 16, True, True, False, 0, 3),    # N = 0: T0 = I, E = I + L
 ]
 
 
